@@ -1,0 +1,162 @@
+/*
+ * CPU fp64 oracle for the gated delta rule -- TEST INFRASTRUCTURE ONLY.
+ *
+ * Only tests/, the package smoke check and the CPU-baseline leg of bench.py
+ * may load this library. The CUDA product path never calls it and shares no
+ * code, header or helper with it.
+ *
+ * Source of the arithmetic ("Gated Delta Networks: Improving Mamba2 with
+ * Delta Rule", as described on the pages collected for this project):
+ *   - recurrence   S_t = S_{t-1} (alpha_t (I - beta_t k_t k_t^T)) + beta_t v_t k_t^T
+ *                  (phantomic12 "gated-deltanet" page, mechanism paragraph;
+ *                   dmarx anthology LIT-137, "Standing in the anthology")
+ *   - readout      o_t = S_t q_t, read from the state AFTER the gated write
+ *                  (portpowered "Gated DeltaNet" page, "How It Works" and
+ *                   "Math Or Compute Schema")
+ *   - state shape  fixed per head (head_k_dim x head_v_dim), constant in T
+ *                  (phantomic12 page, mechanism paragraph)
+ *
+ * S is d_v x d_k in the formula (S k is a d_v vector). Expanding the product
+ * gives S_t = alpha S_{t-1} + beta (v - alpha S_{t-1} k) k^T, which is what the
+ * loop below evaluates (one matrix-vector product, one rank-1 update). Every
+ * value is fp64; inputs are upcast exactly by the caller; nothing is rounded
+ * on the way out.
+ *
+ * Memory layouts (row-major, same as the library's C ABI):
+ *   q, k [B, T, H, d_k]; v, o [B, T, H, d_v]; g, beta [B, T, H];
+ *   states [N, H, d_k, d_v] with state[n][h][j][i] = S_{i j}.
+ * g is log(alpha); alpha = exp(g). With cu_seqlens (B == 1) sequence n covers
+ * tokens [cu[n], cu[n+1]) and starts from its own initial state.
+ *
+ * Parity: pinned by tests/test_oracle_pins.py (closed forms, special cases,
+ * exact rational arithmetic, the dense chunked WY/UT form).
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+typedef struct {
+    const double *q, *k, *v, *g, *beta, *s0;
+    const int32_t *cu;
+    double *o, *s_out;
+    int B, T, H, dk, dv, N;
+    int next;              /* next (seq, head) unit to hand out */
+    pthread_mutex_t lock;
+} job_t;
+
+/* One (sequence, head) recurrence over tokens [t_begin, t_end) of row block
+ * `b` (b = batch index, or 0 for packed sequences). */
+static void run_unit(job_t *J, int n, int h)
+{
+    const int H = J->H, dk = J->dk, dv = J->dv;
+    int b, t0, t1;
+    if (J->cu) { b = 0; t0 = J->cu[n]; t1 = J->cu[n + 1]; }
+    else       { b = n; t0 = 0;        t1 = J->T; }
+
+    double *S = (double *)calloc((size_t)dv * dk, sizeof(double)); /* S[i*dk + j] */
+    double *x = (double *)malloc(sizeof(double) * dv);
+    if (J->s0) {
+        const double *st = J->s0 + ((size_t)n * H + h) * dk * dv;
+        for (int j = 0; j < dk; ++j)
+            for (int i = 0; i < dv; ++i) S[(size_t)i * dk + j] = st[(size_t)j * dv + i];
+    }
+    for (int t = t0; t < t1; ++t) {
+        const size_t row = ((size_t)b * J->T + t) * H + h;
+        const double *kt = J->k + row * dk, *qt = J->q + row * dk, *vt = J->v + row * dv;
+        const double alpha = exp(J->g[row]);
+        const double beta = J->beta[row];
+        /* x = S_{t-1} k_t */
+        for (int i = 0; i < dv; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < dk; ++j) acc += S[(size_t)i * dk + j] * kt[j];
+            x[i] = acc;
+        }
+        /* S_t = alpha S_{t-1} + beta (v_t - alpha x) k_t^T */
+        for (int i = 0; i < dv; ++i) {
+            const double u = beta * (vt[i] - alpha * x[i]);
+            for (int j = 0; j < dk; ++j)
+                S[(size_t)i * dk + j] = alpha * S[(size_t)i * dk + j] + u * kt[j];
+        }
+        /* o_t = S_t q_t (after the write) */
+        double *ot = J->o + row * dv;
+        for (int i = 0; i < dv; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < dk; ++j) acc += S[(size_t)i * dk + j] * qt[j];
+            ot[i] = acc;
+        }
+    }
+    if (J->s_out) {
+        double *st = J->s_out + ((size_t)n * H + h) * dk * dv;
+        for (int j = 0; j < dk; ++j)
+            for (int i = 0; i < dv; ++i) st[(size_t)j * dv + i] = S[(size_t)i * dk + j];
+    }
+    free(S);
+    free(x);
+}
+
+static void *worker(void *arg)
+{
+    job_t *J = (job_t *)arg;
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        int u = J->next++;
+        pthread_mutex_unlock(&J->lock);
+        if (u >= J->N * J->H) break;
+        run_unit(J, u / J->H, u % J->H);
+    }
+    return NULL;
+}
+
+/* Returns 0 on success, -1 on bad arguments. `o` must hold B*T*H*d_v values;
+ * `final_state` (nullable) N*H*d_k*d_v; `initial_state` nullable (zeros). */
+int gdn_oracle_chunk_fwd(const double *q, const double *k, const double *v,
+                         const double *g, const double *beta,
+                         const double *initial_state, const int32_t *cu_seqlens,
+                         int B, int T, int H, int d_k, int d_v, int num_seqs,
+                         double *o, double *final_state, int nthreads)
+{
+    if (!q || !k || !v || !g || !beta || !o) return -1;
+    if (B < 1 || T < 0 || H < 1 || d_k < 1 || d_v < 1) return -1;
+    int N = B;
+    if (cu_seqlens) {
+        if (B != 1 || num_seqs < 1 || cu_seqlens[0] != 0 || cu_seqlens[num_seqs] != T) return -1;
+        for (int n = 0; n < num_seqs; ++n)
+            if (cu_seqlens[n + 1] < cu_seqlens[n]) return -1;
+        N = num_seqs;
+    }
+    job_t J = {q, k, v, g, beta, initial_state, cu_seqlens, o, final_state,
+               B, T, H, d_k, d_v, N, 0};
+    pthread_mutex_init(&J.lock, NULL);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > N * H) nthreads = N * H;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * nthreads);
+    for (int i = 0; i < nthreads; ++i) pthread_create(&th[i], NULL, worker, &J);
+    for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+    free(th);
+    pthread_mutex_destroy(&J.lock);
+    return 0;
+}
+
+/* One recurrent step for N*H independent states, in place:
+ * state [N,H,d_k,d_v] (S^T storage), q/k [N,H,d_k], v/o [N,H,d_v], g/beta [N,H].
+ * Same arithmetic as one iteration of the loop above. */
+int gdn_oracle_decode_step(const double *q, const double *k, const double *v,
+                           const double *g, const double *beta, double *state,
+                           double *o, int N, int H, int d_k, int d_v, int nthreads)
+{
+    if (!q || !k || !v || !g || !beta || !state || !o) return -1;
+    if (N < 1 || H < 1 || d_k < 1 || d_v < 1) return -1;
+    /* A decode step is a length-1 sequence per (n, h) with its own state. */
+    int32_t *cu = (int32_t *)malloc(sizeof(int32_t) * (N + 1));
+    for (int n = 0; n <= N; ++n) cu[n] = n;
+    double *s_out = (double *)malloc(sizeof(double) * (size_t)N * H * d_k * d_v);
+    /* Tokens laid out as [1, N, H, d]: token index = n. */
+    int rc = gdn_oracle_chunk_fwd(q, k, v, g, beta, state, cu, 1, N, H, d_k, d_v, N,
+                                  o, s_out, nthreads);
+    if (rc == 0) memcpy(state, s_out, sizeof(double) * (size_t)N * H * d_k * d_v);
+    free(s_out);
+    free(cu);
+    return rc;
+}
