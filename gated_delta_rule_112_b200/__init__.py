@@ -1,1 +1,158 @@
-"""Gated delta rule forward pass and decode step for B200 (sm_100a)."""
+"""Gated delta rule forward pass and decode step on B200 (sm_100a).
+
+A thin ctypes binding over ``libgdn.so`` (C ABI in ``include/gdn.h``). This
+module only marshals arguments: it allocates outputs and workspace with
+PyTorch, passes device pointers and the current CUDA stream, and checks the
+returned status. Every step of the computation runs in the library's CUDA
+kernels; there is no CPU fallback -- if the library or a GPU is missing, the
+calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["chunk_fwd", "decode_step", "workspace_size", "chunk_path", "get_status",
+           "lib", "GdnError", "BF16", "F32", "PATH_TCGEN05", "PATH_SIMT"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdn.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOUT = range(6)
+BF16, F32 = 0, 1
+PATH_TCGEN05, PATH_SIMT = 1, 2
+
+_lib = None
+
+
+class GdnError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {_status_string(code)} ({code})")
+
+
+def _status_string(code: int) -> str:
+    try:
+        return lib().gdn_status_string(code).decode()
+    except Exception:  # library missing
+        return str(code)
+
+
+def lib() -> ctypes.CDLL:
+    """Load libgdn.so (built in-tree by ``gated_delta_rule_112_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libgdn.so not built ({LIB_PATH}); run "
+                               "python -m gated_delta_rule_112_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, fp, ip = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p
+        ci, sz = ctypes.c_int, ctypes.c_size_t
+        chunk_args = [vp, vp, vp, fp, fp, fp, ip, ci, ci, ci, ci, ci, ci, ci, ci, vp, fp, vp,
+                      sz, vp]
+        L.gdn_chunk_fwd.argtypes = chunk_args
+        L.gdn_chunk_fwd.restype = ci
+        L.gdn_chunk_fwd_simt.argtypes = chunk_args
+        L.gdn_chunk_fwd_simt.restype = ci
+        L.gdn_chunk_fwd_workspace_size.argtypes = [ci] * 8
+        L.gdn_chunk_fwd_workspace_size.restype = sz
+        L.gdn_chunk_fwd_path.argtypes = [ci] * 4
+        L.gdn_chunk_fwd_path.restype = ci
+        L.gdn_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, ci, ci, ci, ci, ci, vp]
+        L.gdn_decode_step.restype = ci
+        L.gdn_get_status.argtypes = [vp, vp]
+        L.gdn_get_status.restype = ci
+        L.gdn_status_string.argtypes = [ci]
+        L.gdn_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.bfloat16:
+        return BF16
+    if t == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t}; use bfloat16 or float32")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(code: int, what: str):
+    if code != OK:
+        raise GdnError(code, what)
+
+
+def workspace_size(B, T, H, d_k, d_v, num_seqs=0, chunk=64, dtype=torch.bfloat16) -> int:
+    return int(lib().gdn_chunk_fwd_workspace_size(B, T, H, d_k, d_v, num_seqs, chunk,
+                                                  _dtype_code(dtype)))
+
+
+def chunk_path(d_k, d_v, chunk=64, dtype=torch.bfloat16) -> int:
+    return int(lib().gdn_chunk_fwd_path(d_k, d_v, chunk, _dtype_code(dtype)))
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("all tensors must be contiguous CUDA tensors")
+
+
+def chunk_fwd(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk=64,
+              output_final_state=True, workspace=None, out=None, force_simt=False,
+              stream=None):
+    """Chunkwise forward pass. Returns ``(o, final_state or None)``.
+
+    q, k: [B,T,H,d_k]; v: [B,T,H,d_v] (bf16 or fp32, same dtype); g (= log
+    alpha), beta: [B,T,H] fp32; initial_state: [N,H,d_k,d_v] fp32 or None;
+    cu_seqlens: int32 [N+1] CUDA tensor (packed sequences, B == 1) or None.
+    """
+    _require_cuda(q, k, v, g, beta, initial_state, cu_seqlens)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    N = num_seqs if cu_seqlens is not None else B
+    dt = _dtype_code(q.dtype)
+    o = torch.empty(B, T, H, dv, dtype=q.dtype, device=q.device) if out is None else out
+    fs = (torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device)
+          if output_final_state else None)
+    need = workspace_size(B, T, H, dk, dv, num_seqs, chunk, q.dtype)
+    if need == 0:
+        raise GdnError(ERR_INVALID_ARG, "gdn_chunk_fwd_workspace_size")
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    fn = lib().gdn_chunk_fwd_simt if force_simt else lib().gdn_chunk_fwd
+    rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
+            _ptr(cu_seqlens), B, T, H, dk, dv, num_seqs, chunk, dt, _ptr(o), _ptr(fs),
+            _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    _check(rc, "gdn_chunk_fwd")
+    return o, fs
+
+
+def get_status(workspace=None, stream=None) -> int:
+    """Synchronise the stream and return the first recorded error code."""
+    return int(lib().gdn_get_status(_ptr(workspace), _stream_ptr(stream)))
+
+
+def decode_step(q, k, v, g, beta, state, out=None, stream=None):
+    """One recurrent step, updating ``state`` [N,H,d_k,d_v] fp32 in place.
+
+    q, k: [N,H,d_k]; v: [N,H,d_v]; g, beta: [N,H] fp32. Returns o [N,H,d_v].
+    """
+    _require_cuda(q, k, v, g, beta, state)
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    o = torch.empty(N, H, dv, dtype=q.dtype, device=q.device) if out is None else out
+    rc = lib().gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state),
+                               _ptr(o), N, H, dk, dv, _dtype_code(q.dtype), _stream_ptr(stream))
+    _check(rc, "gdn_decode_step")
+    return o

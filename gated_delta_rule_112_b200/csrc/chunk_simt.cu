@@ -1,0 +1,319 @@
+// Chunk bookkeeping shared by both chunked-forward paths, and the fp32
+// CUDA-core implementation of the chunkwise WY / UT-transform forward pass
+// ("Gated Delta Networks", phantomic12 page, mechanism paragraph; LIT-137,
+// "Standing in the anthology": the WY-based chunkwise algorithm extended to
+// carry the gate). This path serves fp32 inputs (where fp32 accuracy is
+// required end to end) and head sizes the tensor-core path does not cover.
+//
+// Per chunk (rows r, s < C; Gamma = inclusive cumsum of g inside the chunk):
+//   A_rs = beta_r exp(Gamma_r - Gamma_s) k_r.k_s  (s < r)     T = (I + A)^-1
+//   W = T diag(beta exp(Gamma)) K        U = T diag(beta) V     V_new = U - W S^T
+//   O = diag(exp(Gamma)) Q S^T + (Q K^T .* M) V_new,  M_rs = exp(Gamma_r - Gamma_s), s <= r
+//   S <- exp(Gamma_last) S + V_new^T diag(exp(Gamma_last - Gamma)) K
+// Rows past a sequence's end are treated as k = q = v = 0, beta = g = 0,
+// which leaves S unchanged; their outputs are not written.
+#include "gdn_internal.cuh"
+#include "sm100_ptx.cuh"
+
+namespace gdn {
+namespace {
+
+// ---------------------------------------------------------------------------
+// Chunk map: validates cu_seqlens and lists every (sequence, chunk).
+// One CTA of 1024 threads; thread t owns a contiguous range of sequences.
+__global__ void __launch_bounds__(1024) gdn_chunk_map_kernel(
+    const int32_t *__restrict__ cu, int B, int T, int num_seqs, int chunk,
+    uint32_t *__restrict__ ctrl, ChunkInfo *__restrict__ table,
+    int32_t *__restrict__ seq_first, int max_chunks) {
+  __shared__ int32_t scan[1024];
+  __shared__ int bad;
+  const int N = num_seqs > 0 ? num_seqs : B;
+  const int tid = threadIdx.x;
+  if (tid == 0) bad = 0;
+  __syncthreads();
+  const int per = (N + 1023) / 1024;
+  const int n0 = min(N, tid * per), n1 = min(N, n0 + per);
+  int32_t local = 0;
+  for (int n = n0; n < n1; ++n) {
+    int len;
+    if (cu) {
+      const int a = cu[n], b = cu[n + 1];
+      if ((n == 0 && a != 0) || b < a || (n == N - 1 && b != T)) bad = 1;
+      len = b - a;
+    } else {
+      len = T;
+    }
+    if (len > 0) local += (len + chunk - 1) / chunk;
+  }
+  scan[tid] = local;
+  __syncthreads();
+  for (int off = 1; off < 1024; off <<= 1) {
+    const int32_t add = tid >= off ? scan[tid - off] : 0;
+    __syncthreads();
+    scan[tid] += add;
+    __syncthreads();
+  }
+  const int32_t total = scan[1023];
+  if (bad || total > max_chunks) {
+    if (tid == 0) {
+      atomicOr(ctrl, kErrBadSeqlens);
+      ctrl[1] = 0;
+    }
+    return;
+  }
+  int32_t first = scan[tid] - local;
+  for (int n = n0; n < n1; ++n) {
+    const int row0 = cu ? cu[n] : n * T;
+    const int len = cu ? cu[n + 1] - cu[n] : T;
+    seq_first[n] = first;
+    for (int c = 0; c * chunk < len; ++c) {
+      ChunkInfo ci;
+      ci.seq = n;
+      ci.cidx = c;
+      ci.row0 = row0 + c * chunk;
+      ci.len = min(chunk, len - c * chunk);
+      table[first + c] = ci;
+    }
+    if (len > 0) first += (len + chunk - 1) / chunk;
+  }
+  if (tid == 1023) seq_first[N] = total;
+  if (tid == 0) ctrl[1] = uint32_t(total);
+}
+
+template <typename T>
+__device__ __forceinline__ float ld_f32(const T *p);
+template <>
+__device__ __forceinline__ float ld_f32<float>(const float *p) { return *p; }
+template <>
+__device__ __forceinline__ float ld_f32<__nv_bfloat16>(const __nv_bfloat16 *p) {
+  return __bfloat162float(*p);
+}
+template <typename T>
+__device__ __forceinline__ void st_from_f32(T *p, float x);
+template <>
+__device__ __forceinline__ void st_from_f32<float>(float *p, float x) { *p = x; }
+template <>
+__device__ __forceinline__ void st_from_f32<__nv_bfloat16>(__nv_bfloat16 *p, float x) {
+  *p = __float2bfloat16_rn(x);
+}
+
+constexpr int kSimtThreads = 256;
+constexpr int kDvt = 32;  // d_v columns per CTA
+
+// ---------------------------------------------------------------------------
+// fp32 chunked forward. Grid (N, H, ceil(d_v / 32)); one CTA walks all chunks
+// of one sequence for one head and one 32-column slice of d_v, carrying its
+// slice of the state in shared memory.
+template <int C, typename T>
+__global__ void __launch_bounds__(kSimtThreads) gdn_chunk_simt_kernel(
+    const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+    const float *__restrict__ g, const float *__restrict__ beta, const float *__restrict__ s0,
+    int H, int dk, int dv, T *__restrict__ o, float *__restrict__ sN,
+    const uint32_t *__restrict__ ctrl, const ChunkInfo *__restrict__ table,
+    const int32_t *__restrict__ seq_first) {
+  extern __shared__ float sm[];
+  if (ctrl[0] & kErrBadSeqlens) return;
+  const int n = blockIdx.x, h = blockIdx.y, i0 = blockIdx.z * kDvt;
+  const int tid = threadIdx.x;
+  const int dkp = dk + 1;
+  float *Ks = sm;                        // [C][dkp]
+  float *Qs = Ks + C * dkp;              // [C][dkp]
+  float *Ws = Qs + C * dkp;              // [C][dkp]
+  float *Vs = Ws + C * dkp;              // [C][kDvt]
+  float *Us = Vs + C * kDvt;             // [C][kDvt]
+  float *Vn = Us + C * kDvt;             // [C][kDvt]
+  float *Ss = Vn + C * kDvt;             // [dk][kDvt]  S^T slice: Ss[j][i'] = S[i0+i'][j]
+  float *As = Ss + dk * kDvt;            // [C][C+1]
+  float *Ts = As + C * (C + 1);          // [C][C+1]
+  float *Ps = Ts + C * (C + 1);          // [C][C+1]
+  float *Gm = Ps + C * (C + 1);          // [C] Gamma
+  float *Bt = Gm + C;                    // [C] beta
+  float *Ga = Bt + C;                    // [C] exp(Gamma)
+  float *Dd = Ga + C;                    // [C] exp(Gamma_last - Gamma)
+
+  // Initial state slice.
+  for (int e = tid; e < dk * kDvt; e += kSimtThreads) {
+    const int j = e / kDvt, ii = e % kDvt;
+    float x = 0.f;
+    if (s0 && i0 + ii < dv) x = s0[((size_t(n) * H + h) * dk + j) * dv + i0 + ii];
+    Ss[e] = x;
+  }
+  const int c_begin = seq_first[n], c_end = seq_first[n + 1];
+  for (int cg = c_begin; cg < c_end; ++cg) {
+    const ChunkInfo ci = table[cg];
+    const int L = ci.len;
+    __syncthreads();
+    // 1. load the chunk (rows >= L as zeros)
+    for (int e = tid; e < C * dk; e += kSimtThreads) {
+      const int r = e / dk, j = e % dk;
+      float kv = 0.f, qv = 0.f;
+      if (r < L) {
+        const size_t off = (size_t(ci.row0 + r) * H + h) * dk + j;
+        kv = ld_f32(k + off);
+        qv = ld_f32(q + off);
+      }
+      Ks[r * dkp + j] = kv;
+      Qs[r * dkp + j] = qv;
+    }
+    for (int e = tid; e < C * kDvt; e += kSimtThreads) {
+      const int r = e / kDvt, ii = e % kDvt;
+      float vv = 0.f;
+      if (r < L && i0 + ii < dv) vv = ld_f32(v + (size_t(ci.row0 + r) * H + h) * dv + i0 + ii);
+      Vs[e] = vv;
+    }
+    if (tid < C) {
+      const bool ok = tid < L;
+      Gm[tid] = ok ? g[size_t(ci.row0 + tid) * H + h] : 0.f;
+      Bt[tid] = ok ? beta[size_t(ci.row0 + tid) * H + h] : 0.f;
+    }
+    __syncthreads();
+    // 2. cumulative log-gate and the decay factors
+    if (tid == 0) {
+      float acc = 0.f;
+      for (int r = 0; r < C; ++r) { acc += Gm[r]; Gm[r] = acc; }
+    }
+    __syncthreads();
+    if (tid < C) {
+      Ga[tid] = expf(Gm[tid]);
+      Dd[tid] = expf(Gm[C - 1] - Gm[tid]);
+    }
+    // 3. A (strictly lower) and P = (Q K^T) .* M (diagonal included)
+    for (int e = tid; e < C * C; e += kSimtThreads) {
+      const int r = e / C, s = e % C;
+      float a = 0.f, p = 0.f;
+      if (s <= r) {
+        float dkk = 0.f, dqk = 0.f;
+        for (int j = 0; j < dk; ++j) {
+          const float ksj = Ks[s * dkp + j];
+          dkk += Ks[r * dkp + j] * ksj;
+          dqk += Qs[r * dkp + j] * ksj;
+        }
+        const float decay = expf(Gm[r] - Gm[s]);
+        if (s < r) a = Bt[r] * decay * dkk;
+        p = decay * dqk;
+      }
+      As[r * (C + 1) + s] = a;
+      Ps[r * (C + 1) + s] = p;
+    }
+    __syncthreads();
+    // 4. T = (I + A)^-1 by forward substitution; thread s owns column s.
+    if (tid < C) {
+      const int s = tid;
+      for (int r = 0; r < C; ++r) Ts[r * (C + 1) + s] = (r == s) ? 1.f : 0.f;
+      for (int r = s + 1; r < C; ++r) {
+        float acc = 0.f;
+        for (int m = s; m < r; ++m) acc += As[r * (C + 1) + m] * Ts[m * (C + 1) + s];
+        Ts[r * (C + 1) + s] = -acc;
+      }
+    }
+    __syncthreads();
+    // 5. W = T diag(beta gamma) K, U = T diag(beta) V
+    for (int e = tid; e < C * dk; e += kSimtThreads) {
+      const int r = e / dk, j = e % dk;
+      float acc = 0.f;
+      for (int s = 0; s <= r; ++s) acc += Ts[r * (C + 1) + s] * (Bt[s] * Ga[s]) * Ks[s * dkp + j];
+      Ws[r * dkp + j] = acc;
+    }
+    for (int e = tid; e < C * kDvt; e += kSimtThreads) {
+      const int r = e / kDvt, ii = e % kDvt;
+      float acc = 0.f;
+      for (int s = 0; s <= r; ++s) acc += Ts[r * (C + 1) + s] * Bt[s] * Vs[s * kDvt + ii];
+      Us[e] = acc;
+    }
+    __syncthreads();
+    // 6. V_new = U - W S^T
+    for (int e = tid; e < C * kDvt; e += kSimtThreads) {
+      const int r = e / kDvt, ii = e % kDvt;
+      float acc = 0.f;
+      for (int j = 0; j < dk; ++j) acc += Ws[r * dkp + j] * Ss[j * kDvt + ii];
+      Vn[e] = Us[e] - acc;
+    }
+    __syncthreads();
+    // 7. O = diag(gamma) Q S^T + P V_new   (old S)
+    for (int e = tid; e < C * kDvt; e += kSimtThreads) {
+      const int r = e / kDvt, ii = e % kDvt;
+      if (r < L && i0 + ii < dv) {
+        float acc = 0.f;
+        for (int j = 0; j < dk; ++j) acc += Qs[r * dkp + j] * Ss[j * kDvt + ii];
+        float acc2 = 0.f;
+        for (int s = 0; s <= r; ++s) acc2 += Ps[r * (C + 1) + s] * Vn[s * kDvt + ii];
+        st_from_f32(o + (size_t(ci.row0 + r) * H + h) * dv + i0 + ii, Ga[r] * acc + acc2);
+      }
+    }
+    __syncthreads();
+    // 8. S <- gamma_last S + V_new^T diag(D) K
+    const float glast = Ga[C - 1];
+    for (int e = tid; e < dk * kDvt; e += kSimtThreads) {
+      const int j = e / kDvt, ii = e % kDvt;
+      float acc = 0.f;
+      for (int s = 0; s < C; ++s) acc += Dd[s] * Ks[s * dkp + j] * Vn[s * kDvt + ii];
+      Ss[e] = glast * Ss[e] + acc;
+    }
+  }
+  __syncthreads();
+  if (sN) {
+    for (int e = tid; e < dk * kDvt; e += kSimtThreads) {
+      const int j = e / kDvt, ii = e % kDvt;
+      if (i0 + ii < dv) sN[((size_t(n) * H + h) * dk + j) * dv + i0 + ii] = Ss[e];
+    }
+  }
+}
+
+template <int C, typename T>
+cudaError_t launch_simt_t(const void *q, const void *k, const void *v, const float *g,
+                          const float *beta, const float *s0, int H, int dk, int dv, int N,
+                          void *o, float *sN, uint32_t *ctrl, const ChunkInfo *table,
+                          const int32_t *seq_first, cudaStream_t s) {
+  const size_t floats = size_t(3) * C * (dk + 1) + size_t(3) * C * kDvt + size_t(dk) * kDvt +
+                        size_t(3) * C * (C + 1) + 4 * C;
+  const size_t bytes = floats * sizeof(float);
+  auto kern = gdn_chunk_simt_kernel<C, T>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(bytes));
+  if (e != cudaSuccess) return e;
+  dim3 grid(N, H, (dv + kDvt - 1) / kDvt);
+  kern<<<grid, kSimtThreads, bytes, s>>>(
+      static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), g, beta,
+      s0, H, dk, dv, static_cast<T *>(o), sN, ctrl, table, seq_first);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_chunk_map(const int32_t *cu_seqlens, int B, int T, int num_seqs, int chunk,
+                             void *ws, const WsLayout &L, cudaStream_t s) {
+  char *base = static_cast<char *>(ws);
+  cudaError_t e = cudaMemsetAsync(base, 0, 256, s);
+  if (e != cudaSuccess) return e;
+  gdn_chunk_map_kernel<<<1, 1024, 0, s>>>(
+      cu_seqlens, B, T, num_seqs, chunk, reinterpret_cast<uint32_t *>(base),
+      reinterpret_cast<ChunkInfo *>(base + L.chunk_table),
+      reinterpret_cast<int32_t *>(base + L.seq_first), L.max_chunks);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const float *g,
+                              const float *beta, const float *s0, const int32_t *cu, int B,
+                              int T, int H, int dk, int dv, int N, int chunk, int dtype, void *o,
+                              float *sN, uint32_t *ws_ctrl, cudaStream_t s) {
+  (void)cu; (void)B; (void)T;
+  char *base = reinterpret_cast<char *>(ws_ctrl);
+  // The layout of the chunk table is the same for both paths.
+  const WsLayout L = ws_layout(B, T, H, cu ? N : 0, chunk, false);
+  const ChunkInfo *table = reinterpret_cast<const ChunkInfo *>(base + L.chunk_table);
+  const int32_t *seq_first = reinterpret_cast<const int32_t *>(base + L.seq_first);
+#define GDN_SIMT_CASE(CC)                                                                       \
+  if (chunk == CC)                                                                               \
+    return dtype == GDN_BF16                                                                     \
+               ? launch_simt_t<CC, __nv_bfloat16>(q, k, v, g, beta, s0, H, dk, dv, N, o, sN,   \
+                                                  ws_ctrl, table, seq_first, s)                 \
+               : launch_simt_t<CC, float>(q, k, v, g, beta, s0, H, dk, dv, N, o, sN, ws_ctrl,  \
+                                          table, seq_first, s);
+  GDN_SIMT_CASE(16)
+  GDN_SIMT_CASE(32)
+  GDN_SIMT_CASE(64)
+#undef GDN_SIMT_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace gdn

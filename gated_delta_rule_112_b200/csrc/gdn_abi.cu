@@ -1,0 +1,144 @@
+// Host side of the C ABI declared in include/gdn.h: argument validation,
+// workspace sizing, dispatch to the kernels and status reporting. Nothing
+// here allocates device memory.
+#include <cstdio>
+
+#include "gdn_internal.cuh"
+
+using namespace gdn;
+
+namespace {
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool tc_path(int dk, int dv, int chunk, int dtype) {
+  return dtype == GDN_BF16 && dk == 128 && dv == 128 && chunk == 64;
+}
+
+// Shared checks of gdn_chunk_fwd / gdn_chunk_fwd_simt.
+int check_chunk_args(const void *q, const void *k, const void *v, const float *g,
+                     const float *beta, const float *s0, const int32_t *cu, int B, int T, int H,
+                     int dk, int dv, int num_seqs, int chunk, int dtype, const void *o,
+                     const float *sN, const void *ws) {
+  if (dtype != GDN_BF16 && dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
+  if (B < 1 || T < 0 || H < 1 || dk < 1 || dv < 1) return GDN_ERR_INVALID_ARG;
+  if (cu && (B != 1 || num_seqs < 1)) return GDN_ERR_INVALID_ARG;
+  if (!cu && num_seqs != 0) return GDN_ERR_INVALID_ARG;
+  if (int64_t(B) * T * H * (dk > dv ? dk : dv) >= (int64_t(1) << 31)) return GDN_ERR_UNSUPPORTED;
+  if (dk > 128 || dv > 128) return GDN_ERR_UNSUPPORTED;
+  if (chunk != 16 && chunk != 32 && chunk != 64) return GDN_ERR_UNSUPPORTED;
+  if (T > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_ERR_INVALID_ARG;
+  if (!ws) return GDN_ERR_WORKSPACE;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(g, 4) || !aligned(beta, 4) || !aligned(s0, 16) || !aligned(sN, 16) ||
+      !aligned(cu, 4))
+    return GDN_ERR_INVALID_ARG;
+  if (!aligned(ws, 256)) return GDN_ERR_WORKSPACE;
+  return GDN_OK;
+}
+
+int run_chunk(bool force_simt, const void *q, const void *k, const void *v, const float *g,
+              const float *beta, const float *s0, const int32_t *cu, int B, int T, int H,
+              int dk, int dv, int num_seqs, int chunk, int dtype, void *o, float *sN, void *ws,
+              size_t ws_bytes, void *stream) {
+  int rc = check_chunk_args(q, k, v, g, beta, s0, cu, B, T, H, dk, dv, num_seqs, chunk, dtype,
+                            o, sN, ws);
+  if (rc != GDN_OK) return rc;
+  const bool tc = !force_simt && tc_path(dk, dv, chunk, dtype);
+  const WsLayout L = ws_layout(B, T, H, cu ? num_seqs : 0, chunk, tc);
+  if (ws_bytes < L.total) return GDN_ERR_WORKSPACE;
+  const int N = cu ? num_seqs : B;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_chunk_map(cu, B, T, cu ? num_seqs : 0, chunk, ws, L, s);
+  if (e != cudaSuccess) return GDN_ERR_CUDA;
+  if (tc)
+    e = launch_chunk_tc(q, k, v, g, beta, s0, B, T, H, N, o, sN, ws, L, s);
+  else
+    e = launch_chunk_simt(q, k, v, g, beta, s0, cu, B, T, H, dk, dv, N, chunk, dtype, o, sN,
+                          static_cast<uint32_t *>(ws), s);
+  return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t gdn_chunk_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int num_seqs,
+                                    int chunk, int dtype) {
+  if (B < 1 || T < 0 || H < 1 || d_k < 1 || d_v < 1 || num_seqs < 0) return 0;
+  if (chunk != 16 && chunk != 32 && chunk != 64) return 0;
+  return ws_layout(B, T, H, num_seqs, chunk, tc_path(d_k, d_v, chunk, dtype)).total;
+}
+
+int gdn_chunk_fwd_path(int d_k, int d_v, int chunk, int dtype) {
+  if (d_k < 1 || d_v < 1 || d_k > 128 || d_v > 128) return -1;
+  if (chunk != 16 && chunk != 32 && chunk != 64) return -1;
+  if (dtype != GDN_BF16 && dtype != GDN_F32) return -1;
+  return tc_path(d_k, d_v, chunk, dtype) ? GDN_PATH_TCGEN05 : GDN_PATH_SIMT;
+}
+
+int gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
+                  const float *beta, const float *initial_state, const int32_t *cu_seqlens,
+                  int B, int T, int H, int d_k, int d_v, int num_seqs, int chunk, int dtype,
+                  void *o, float *final_state, void *workspace, size_t workspace_bytes,
+                  void *stream) {
+  return run_chunk(false, q, k, v, g, beta, initial_state, cu_seqlens, B, T, H, d_k, d_v,
+                   num_seqs, chunk, dtype, o, final_state, workspace, workspace_bytes, stream);
+}
+
+int gdn_chunk_fwd_simt(const void *q, const void *k, const void *v, const float *g,
+                       const float *beta, const float *initial_state, const int32_t *cu_seqlens,
+                       int B, int T, int H, int d_k, int d_v, int num_seqs, int chunk, int dtype,
+                       void *o, float *final_state, void *workspace, size_t workspace_bytes,
+                       void *stream) {
+  return run_chunk(true, q, k, v, g, beta, initial_state, cu_seqlens, B, T, H, d_k, d_v,
+                   num_seqs, chunk, dtype, o, final_state, workspace, workspace_bytes, stream);
+}
+
+int gdn_decode_step(const void *q, const void *k, const void *v, const float *g,
+                    const float *beta, float *state, void *o, int N, int H, int d_k, int d_v,
+                    int dtype, void *stream) {
+  if (dtype != GDN_BF16 && dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
+  if (N < 1 || H < 1 || d_k < 1 || d_v < 1) return GDN_ERR_INVALID_ARG;
+  if (d_k > 128 || d_v > 128 || (d_v % 4) != 0) return GDN_ERR_UNSUPPORTED;
+  if (int64_t(N) * H >= (int64_t(1) << 31)) return GDN_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !g || !beta || !state || !o) return GDN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(state, 16) || !aligned(g, 4) || !aligned(beta, 4))
+    return GDN_ERR_INVALID_ARG;
+  cudaError_t e = launch_decode(q, k, v, g, beta, state, o, N, H, d_k, d_v, dtype,
+                                static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+int gdn_get_status(void *workspace, void *stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return GDN_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+  if (!workspace) return GDN_OK;
+  uint32_t err = 0;
+  if (cudaMemcpy(&err, workspace, sizeof(err), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  if (err) {
+    const uint32_t zero = 0;
+    if (cudaMemcpy(workspace, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+      return GDN_ERR_CUDA;
+  }
+  if (err & kErrTimeout) return GDN_ERR_DEVICE_TIMEOUT;
+  if (err & kErrBadSeqlens) return GDN_ERR_INVALID_ARG;
+  return GDN_OK;
+}
+
+const char *gdn_status_string(int status) {
+  switch (status) {
+    case GDN_OK: return "GDN_OK";
+    case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG";
+    case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
+    case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE";
+    case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
+    case GDN_ERR_DEVICE_TIMEOUT: return "GDN_ERR_DEVICE_TIMEOUT";
+    default: return "GDN_ERR_UNKNOWN";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,158 @@
+/*
+ * gdn.h -- C ABI of libgdn: the gated delta rule forward pass and decode step
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The operation ("Gated Delta Networks: Improving Mamba2 with Delta Rule";
+ * recurrence on the phantomic12 "gated-deltanet" page, mechanism paragraph,
+ * and the dmarx anthology LIT-137, "Standing in the anthology"; readout on the
+ * portpowered "Gated DeltaNet" page, "How It Works"):
+ *
+ *     S_t = S_{t-1} (alpha_t (I - beta_t k_t k_t^T)) + beta_t v_t k_t^T
+ *     o_t = S_t q_t                      (read after the write at t)
+ *
+ * with S_t a d_v x d_k matrix per (sequence, head), alpha_t = exp(g_t).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller. The library
+ *     allocates no memory and frees none.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream) and return once work is enqueued.
+ *   - Inputs are never modified, except `state` in gdn_decode_step.
+ *   - Outputs are undefined when a call returns an error.
+ *   - Row-major layouts:
+ *       q, k   [B, T, H, d_k]      v, o   [B, T, H, d_v]
+ *       g, beta [B, T, H] fp32      (g = log alpha; any finite value; beta is
+ *                                    not clamped, so beta in (0, 2) -- the
+ *                                    negative-eigenvalue extension -- works)
+ *       states [N, H, d_k, d_v] fp32 with state[n][h][j][i] = S_{i j}
+ *       (the memory holds S^T, d_v contiguous).
+ *   - dtype selects the type of q, k, v and o: GDN_BF16 or GDN_F32.
+ *   - No C++ exceptions cross the ABI. Host-side checks return an error code
+ *     and launch nothing.
+ */
+#ifndef GDN_H
+#define GDN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+#define GDN_OK                 0
+#define GDN_ERR_INVALID_ARG    1  /* null required pointer, bad size, misaligned pointer, bad cu_seqlens */
+#define GDN_ERR_UNSUPPORTED    2  /* valid but not implemented: d_k or d_v > 128, chunk not in {16,32,64} */
+#define GDN_ERR_WORKSPACE      3  /* workspace missing or smaller than gdn_chunk_fwd_workspace_size() */
+#define GDN_ERR_CUDA           4  /* a CUDA runtime/driver call or kernel launch failed */
+#define GDN_ERR_DEVICE_TIMEOUT 5  /* a bounded device-side wait expired (reported by gdn_get_status) */
+
+/* Element types of q, k, v, o. */
+#define GDN_BF16 0
+#define GDN_F32  1
+
+/* Chunked-forward implementations (gdn_chunk_fwd_path). */
+#define GDN_PATH_TCGEN05 1   /* bf16, d_k = d_v = 128, chunk = 64: tensor-core kernels */
+#define GDN_PATH_SIMT    2   /* everything else with d <= 128: fp32 CUDA-core kernel */
+
+/*
+ * gdn_chunk_fwd_workspace_size -- bytes of device workspace gdn_chunk_fwd needs.
+ *
+ * An upper bound that does not depend on the contents of cu_seqlens: for
+ * packed sequences (num_seqs > 0) it assumes the worst case of
+ * (T + num_seqs * (chunk - 1)) / chunk chunks. Returns 0 for invalid sizes.
+ * The workspace must be 256-byte aligned; its contents need no initialisation.
+ */
+size_t gdn_chunk_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int num_seqs,
+                                    int chunk, int dtype);
+
+/*
+ * gdn_chunk_fwd -- the whole-sequence forward pass, computed chunkwise.
+ *
+ * Algorithm: the chunkwise-parallel WY representation / UT transform extended
+ * to carry the decay gate (phantomic12 page, mechanism paragraph; LIT-137,
+ * "Standing in the anthology"; SOTA-135, "Source"). Per chunk of `chunk`
+ * tokens: Gamma = cumsum(g); A = strictly-lower beta (K K^T .* exp(Gamma_r -
+ * Gamma_s)); T = (I + A)^-1; W = T diag(beta exp(Gamma)) K; U = T diag(beta) V;
+ * V_new = U - W S^T; O = diag(exp(Gamma)) Q S^T + (Q K^T .* M) V_new with the
+ * diagonal included in M; S <- exp(Gamma_last) S + V_new^T diag(exp(Gamma_last
+ * - Gamma)) K. The result equals the token recurrence up to rounding.
+ *
+ *   q, k, v, o      see layouts above; 16-byte aligned.
+ *   g, beta         [B, T, H] fp32, 4-byte aligned.
+ *   initial_state   [N, H, d_k, d_v] fp32 or NULL (zero state); 16-byte aligned.
+ *   cu_seqlens      NULL, or int32 [num_seqs + 1] device array of packed
+ *                   sequence boundaries: cu[0] = 0, non-decreasing,
+ *                   cu[num_seqs] = T; requires B == 1. Sequence n covers
+ *                   tokens [cu[n], cu[n+1]), starts from initial_state[n] and
+ *                   ends in final_state[n]; no state flows between sequences.
+ *                   Its contents are checked on the device; a violation is
+ *                   reported as GDN_ERR_INVALID_ARG by gdn_get_status and no
+ *                   output is written.
+ *   N               num_seqs with cu_seqlens, otherwise B.
+ *   chunk           tokens per chunk: 64 for the tensor-core path; 16, 32 or
+ *                   64 for the CUDA-core path. Chunks start at each
+ *                   sequence's first token; the last one may be partial.
+ *   final_state     [N, H, d_k, d_v] fp32 or NULL (not written).
+ *   workspace       device scratch of at least gdn_chunk_fwd_workspace_size()
+ *                   bytes, 256-byte aligned, not used by any concurrent call.
+ *   stream          cudaStream_t as void*.
+ *
+ * Returns GDN_OK once all kernels are enqueued. Path: GDN_PATH_TCGEN05 for
+ * dtype GDN_BF16 with d_k = d_v = 128 and chunk = 64, GDN_PATH_SIMT otherwise.
+ */
+int gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
+                  const float *beta, const float *initial_state, const int32_t *cu_seqlens,
+                  int B, int T, int H, int d_k, int d_v, int num_seqs, int chunk, int dtype,
+                  void *o, float *final_state, void *workspace, size_t workspace_bytes,
+                  void *stream);
+
+/*
+ * gdn_chunk_fwd_simt -- same contract as gdn_chunk_fwd, but always runs the
+ * fp32 CUDA-core kernel (the path fp32 inputs and general head sizes take).
+ * Useful to cross-check the tensor-core path on the same bf16 inputs.
+ */
+int gdn_chunk_fwd_simt(const void *q, const void *k, const void *v, const float *g,
+                       const float *beta, const float *initial_state, const int32_t *cu_seqlens,
+                       int B, int T, int H, int d_k, int d_v, int num_seqs, int chunk, int dtype,
+                       void *o, float *final_state, void *workspace, size_t workspace_bytes,
+                       void *stream);
+
+/* Which implementation gdn_chunk_fwd would run for these sizes
+ * (GDN_PATH_TCGEN05 or GDN_PATH_SIMT), or a negative value if unsupported. */
+int gdn_chunk_fwd_path(int d_k, int d_v, int chunk, int dtype);
+
+/*
+ * gdn_decode_step -- one recurrent token for N*H independent states, in place.
+ *
+ * Per (n, h) (one step of the recurrence above; constant-size state, no KV
+ * cache: phantomic12 page, mechanism paragraph):
+ *     alpha = exp(g); x = S k; y = S q; u = beta (v - alpha x)
+ *     S <- alpha S + u k^T;  o = S q = alpha y + (k . q) u
+ *
+ *   q, k   [N, H, d_k]   v, o  [N, H, d_v]   (dtype), 16-byte aligned
+ *   g, beta [N, H] fp32
+ *   state  [N, H, d_k, d_v] fp32, read and overwritten; 16-byte aligned.
+ * Supports d_k <= 128, d_v <= 128 with d_v a multiple of 4.
+ */
+int gdn_decode_step(const void *q, const void *k, const void *v, const float *g,
+                    const float *beta, float *state, void *o, int N, int H, int d_k,
+                    int d_v, int dtype, void *stream);
+
+/*
+ * gdn_get_status -- synchronises `stream`, then reports the first error seen:
+ * GDN_ERR_CUDA for a failed kernel, or the code a gdn_chunk_fwd kernel left in
+ * `workspace` (GDN_ERR_DEVICE_TIMEOUT, GDN_ERR_INVALID_ARG for bad
+ * cu_seqlens). Clears the device error word. `workspace` may be NULL.
+ */
+int gdn_get_status(void *workspace, void *stream);
+
+/* Human-readable name of a status code (static string). */
+const char *gdn_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H */

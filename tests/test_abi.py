@@ -1,0 +1,111 @@
+"""The C ABI library: it loads, exports every symbol include/gdn.h declares,
+and rejects bad arguments on the host before touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_112_b200 as gdn
+from gated_delta_rule_112_b200 import build as gbuild
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "gdn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    gbuild.build()
+    return gdn.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for must in ("gdn_chunk_fwd", "gdn_chunk_fwd_workspace_size", "gdn_decode_step",
+                 "gdn_get_status", "gdn_status_string"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), f"libgdn.so does not export {name}"
+
+
+def test_status_strings(L):
+    assert L.gdn_status_string(0) == b"GDN_OK"
+    assert L.gdn_status_string(5) == b"GDN_ERR_DEVICE_TIMEOUT"
+    assert L.gdn_status_string(99) == b"GDN_ERR_UNKNOWN"
+
+
+def test_path_selection(L):
+    assert L.gdn_chunk_fwd_path(128, 128, 64, gdn.BF16) == gdn.PATH_TCGEN05
+    assert L.gdn_chunk_fwd_path(128, 128, 64, gdn.F32) == gdn.PATH_SIMT
+    assert L.gdn_chunk_fwd_path(64, 64, 64, gdn.BF16) == gdn.PATH_SIMT
+    assert L.gdn_chunk_fwd_path(128, 128, 32, gdn.BF16) == gdn.PATH_SIMT
+    assert L.gdn_chunk_fwd_path(256, 128, 64, gdn.BF16) < 0
+    assert L.gdn_chunk_fwd_path(128, 128, 48, gdn.BF16) < 0
+
+
+def test_workspace_size(L):
+    ws = L.gdn_chunk_fwd_workspace_size
+    tc = ws(4, 4096, 16, 128, 128, 0, 64, gdn.BF16)
+    # 4096 (chunk, head) units x (16 + 16 + 8 KB + 256 B) plus bookkeeping
+    assert tc >= 4096 * (16384 * 2 + 8192 + 256)
+    assert tc < 4096 * (16384 * 2 + 8192 + 256) + (1 << 20)
+    simt = ws(1, 256, 2, 64, 64, 0, 64, gdn.F32)
+    assert 0 < simt < (1 << 16)
+    # varlen bound: (T + N (C-1)) / C chunks
+    v = ws(1, 1000, 1, 128, 128, 10, 64, gdn.BF16)
+    assert v >= ((1000 + 10 * 63) // 64) * (16384 * 2 + 8192 + 256)
+    assert ws(0, 10, 1, 128, 128, 0, 64, gdn.BF16) == 0
+    assert ws(1, 10, 1, 128, 128, 0, 48, gdn.BF16) == 0
+
+
+def _chunk_call(L, **kw):
+    a = dict(q=1 << 20, k=1 << 20, v=1 << 20, g=1 << 20, beta=1 << 20, s0=None, cu=None, B=1,
+             T=64, H=1, dk=128, dv=128, ns=0, chunk=64, dtype=gdn.BF16, o=1 << 20, sN=None,
+             ws=1 << 20, wsb=1 << 30, stream=None)
+    a.update(kw)
+    vp = ctypes.c_void_p
+    return L.gdn_chunk_fwd(vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["g"]), vp(a["beta"]),
+                           vp(a["s0"]), vp(a["cu"]), a["B"], a["T"], a["H"], a["dk"], a["dv"],
+                           a["ns"], a["chunk"], a["dtype"], vp(a["o"]), vp(a["sN"]),
+                           vp(a["ws"]), a["wsb"], vp(a["stream"]))
+
+
+def test_host_argument_checks_launch_nothing(L):
+    # Each of these is rejected before any CUDA call is made.
+    assert _chunk_call(L, q=None) == gdn.ERR_INVALID_ARG
+    assert _chunk_call(L, o=None) == gdn.ERR_INVALID_ARG
+    assert _chunk_call(L, B=0) == gdn.ERR_INVALID_ARG
+    assert _chunk_call(L, T=-1) == gdn.ERR_INVALID_ARG
+    assert _chunk_call(L, dtype=7) == gdn.ERR_INVALID_ARG
+    assert _chunk_call(L, dk=256) == gdn.ERR_UNSUPPORTED
+    assert _chunk_call(L, chunk=48) == gdn.ERR_UNSUPPORTED
+    assert _chunk_call(L, q=(1 << 20) + 2) == gdn.ERR_INVALID_ARG      # misaligned
+    assert _chunk_call(L, ws=None) == gdn.ERR_WORKSPACE
+    assert _chunk_call(L, ws=(1 << 20) + 16) == gdn.ERR_WORKSPACE      # not 256-aligned
+    assert _chunk_call(L, wsb=100) == gdn.ERR_WORKSPACE
+    assert _chunk_call(L, cu=1 << 20, ns=2, B=2) == gdn.ERR_INVALID_ARG  # varlen needs B == 1
+    assert _chunk_call(L, ns=3) == gdn.ERR_INVALID_ARG                  # num_seqs without cu
+
+
+def test_decode_host_checks(L):
+    vp = ctypes.c_void_p
+    p = vp(1 << 20)
+
+    def call(**kw):
+        a = dict(N=2, H=2, dk=128, dv=128, dtype=gdn.BF16, state=p, q=p)
+        a.update(kw)
+        return L.gdn_decode_step(a["q"], p, p, p, p, a["state"], p, a["N"], a["H"], a["dk"],
+                                 a["dv"], a["dtype"], None)
+    assert call(state=None) == gdn.ERR_INVALID_ARG
+    assert call(q=vp((1 << 20) + 4)) == gdn.ERR_INVALID_ARG
+    assert call(N=0) == gdn.ERR_INVALID_ARG
+    assert call(dv=130) == gdn.ERR_UNSUPPORTED
+    assert call(dv=126) == gdn.ERR_UNSUPPORTED
