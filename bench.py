@@ -1,0 +1,394 @@
+#!/usr/bin/env python
+"""Benchmark of the gated delta rule hot path on B200.
+
+One step = one chunked forward pass (gdn_chunk_fwd: chunk map, prep and scan
+kernels) over the B=4, H=16, T=4096, d_k=d_v=128 bf16 workload, inputs
+already resident in HBM. The decode step (N=256, H=32, d=128, fp32 state,
+64 consecutive steps) is measured in the same run and reported under
+"decode". Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (launched by torchrun, one rank per GPU) every rank runs its own
+independent copy of the workload (weak scaling, no collective on the data
+path); times are the max over ranks. ``--impl reference`` times the CPU fp64
+oracle (the slow, obviously-correct program the GPU path is checked
+against) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "b4h16t4096"
+METRIC = "chunk-fwd Mtokens/s at B4·H16·T4096·d128 bf16; decode GB/s; % roofline"
+UNIT = "Mtokens/s"
+BYTES_PER_TOKEN_HEAD = 3 * 128 * 2 + 128 * 2 + 2 * 4    # q,k,v,o bf16 + g,beta fp32
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--no-decode", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+def kernel_source_hash() -> str:
+    """Hash of the CUDA sources: ncu traffic figures are only reported for the
+    exact kernels they were measured on."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for path in sorted(glob.glob(os.path.join(ROOT, "gated_delta_rule_112_b200", "csrc", "*"))):
+        h.update(open(path, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(key):
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    rec = json.load(open(path)).get(key)
+    if not rec or rec.get("src_hash") != kernel_source_hash():
+        return None
+    return rec["dram_bytes_per_launch"]
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.uuid}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, parts[3:7]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    """Time the CPU fp64 oracle on a bounded sample of the workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+    from gated_delta_rule_112_b200.inputs import make_chunk_inputs
+    inp = make_chunk_inputs(WORKLOAD)
+    heads = [0, 1]                              # sample: 2 of 16 heads, all B*T tokens
+    arr = {k: inp[k][:, :, heads].float().double().numpy() for k in ("q", "k", "v", "g", "beta")}
+    cores = oracle.default_threads()
+    tok_equiv = inp["B"] * inp["T"] * len(heads) / inp["H"]
+
+    def one():
+        oracle.chunk_fwd(arr["q"], arr["k"], arr["v"], arr["g"], arr["beta"], None, None,
+                         nthreads=cores)
+    for _ in range(args.warmup):
+        one()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one()
+    dt = (time.perf_counter() - t0) / max(args.steps, 1)
+    value = tok_equiv / dt / 1e6
+    sample = (f"oracle on {len(heads)} of {inp['H']} heads x B{inp['B']} x T{inp['T']} "
+              f"per step ({int(tok_equiv)} full-width tokens)")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "B": inp["B"], "T": inp["T"], "H": inp["H"],
+                       "d_k": 128, "d_v": 128, "chunk": 64},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- our arm
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+
+    import gated_delta_rule_112_b200 as gdn
+    from gated_delta_rule_112_b200.inputs import make_chunk_inputs, make_decode_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus > 1 and world != args.gpus:
+        raise SystemExit("--gpus N > 1 must be launched with torchrun --nproc-per-node N")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    pk = peaks()
+    stream = torch.cuda.current_stream()
+    L = gdn.lib()
+
+    # --------------------------------------------------------------- chunked forward
+    inp = make_chunk_inputs(WORKLOAD, seed=1 + rank)
+    B, T, H = inp["B"], inp["T"], inp["H"]
+    q, k, v, g, beta = (inp[x].to(dev) for x in ("q", "k", "v", "g", "beta"))
+    o = torch.empty(B, T, H, 128, dtype=torch.bfloat16, device=dev)
+    fs = torch.empty(B, H, 128, 128, dtype=torch.float32, device=dev)
+    ws = torch.empty(gdn.workspace_size(B, T, H, 128, 128), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        gdn.chunk_fwd(q, k, v, g, beta, None, None, out=o, workspace=ws)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    assert gdn.get_status(ws) == gdn.OK
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    for e in evs:                      # torch creates the CUDA event on first record
+        for x in e:
+            x.record(stream)
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    sampler.start()
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.fill_(i & 0xFF)                       # evict L2 between timed steps
+        e = evs[i]
+        L.gdn_set_profile_events(e[0].cuda_event, e[1].cuda_event, e[2].cuda_event,
+                                 e[3].cuda_event)
+        step()
+    L.gdn_set_profile_events(None, None, None, None)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    status = gdn.get_status(ws)
+    if status != gdn.OK:
+        raise SystemExit(f"device status {status}")
+    t_map = [e[0].elapsed_time(e[1]) for e in evs]
+    t_prep = [e[1].elapsed_time(e[2]) for e in evs]
+    t_scan = [e[2].elapsed_time(e[3]) for e in evs]
+    t_step = [e[0].elapsed_time(e[3]) for e in evs]
+    ms_local = sum(t_step) / K
+    ms = max_over_ranks(ms_local)
+    tokens = B * T
+    value = world * tokens / (ms * 1e-3) / 1e6
+
+    alg_bytes = tokens * H * BYTES_PER_TOKEN_HEAD + B * H * 128 * 128 * 4   # + final state
+    flops = tokens * H * 2 * (3 * 64 * 128 + 2 * 64 * 128 + 3 * 128 * 128)
+    ach_gbs = alg_bytes / (ms_local * 1e-3) / 1e9
+    kernels = {
+        "gdn_chunk_map_kernel": statistics.mean(t_map),
+        "gdn_prep_kernel": statistics.mean(t_prep),
+        "gdn_scan_kernel": statistics.mean(t_scan),
+    }
+    tot = sum(kernels.values())
+    traffic = recorded_traffic("chunk_fwd_step/" + WORKLOAD)
+
+    # --------------------------------------------------------------- end to end (host buffers)
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv, hg, hb = (inp[x].pin_memory() for x in ("q", "k", "v", "g", "beta"))
+        ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        hfs = torch.empty(fs.shape, dtype=fs.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hg, hb))
+        d2h = ho.numel() * ho.element_size() + hfs.numel() * hfs.element_size()
+
+        def e2e_step_with_state():
+            for dst, src in ((q, hq), (k, hk), (v, hv), (g, hg), (beta, hb)):
+                dst.copy_(src, non_blocking=True)
+            _, f = gdn.chunk_fwd(q, k, v, g, beta, None, None, out=o, workspace=ws)
+            ho.copy_(o, non_blocking=True)
+            hfs.copy_(f, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step_with_state()
+        torch.cuda.synchronize()
+        ke = max(3, min(K, 10))
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(ke)]
+        barrier()
+        torch.cuda.synchronize()
+        for i in range(ke):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            e2e_step_with_state()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms_e2e = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / ke)
+        e2e = {"value": world * tokens / (ms_e2e * 1e-3) / 1e6, "unit": UNIT,
+               "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "steps": ke, "api": "gated_delta_rule_112_b200.chunk_fwd (C ABI gdn_chunk_fwd)"}
+        del hq, hk, hv, hg, hb, ho, hfs
+
+    del q, k, v, g, beta, o, ws
+    torch.cuda.empty_cache()
+
+    # --------------------------------------------------------------- decode step
+    decode = None
+    if not args.no_decode:
+        d = make_decode_inputs("decode", seed=4 + rank)
+        N, Hd, S = d["N"], d["H"], d["steps"]
+        dq, dk, dvv, dg, db = (d[x].to(dev) for x in ("q", "k", "v", "g", "beta"))
+        st = d["state"].to(dev)
+        do = torch.empty(N, Hd, 128, dtype=torch.bfloat16, device=dev)
+        for t in range(3):
+            gdn.decode_step(dq[t], dk[t], dvv[t], dg[t], db[t], st, out=do)
+        st.copy_(d["state"].to(dev))
+        torch.cuda.synchronize()
+        reps = 3
+        times = []
+        barrier()
+        for r in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            a.record(stream)
+            for t in range(S):
+                gdn.decode_step(dq[t], dk[t], dvv[t], dg[t], db[t], st, out=do)
+            b.record(stream)
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b) / S)
+        barrier()
+        us = max_over_ranks(statistics.median(times)) * 1e3
+        bytes_step = (2 * N * Hd * 128 * 128 * 4 + 3 * N * Hd * 128 * 2 + N * Hd * 128 * 2
+                      + 2 * N * Hd * 4)
+        gbs = bytes_step / (us * 1e-6) / 1e9
+        decode = {"workload": "decode N256 H32 d128 fp32 state, 64 steps", "us_per_step": us,
+                  "value": world * gbs, "unit": "GB/s", "bytes_per_step": bytes_step,
+                  "gpu_launches": reps * S,
+                  "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"],
+                               "unit": "GB/s", "frac": gbs / pk["hbm"],
+                               "traffic": recorded_traffic("decode/n256h32"),
+                               "kernel": "gdn_decode_kernel", "peak_source": pk["source"]}}
+        del dq, dk, dvv, dg, db, st, do
+
+    # --------------------------------------------------------------- CPU baseline (oracle)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        arr = {x: inp[x].float().double().numpy() for x in ("q", "k", "v", "g", "beta")}
+        cores = oracle.default_threads()
+        t0 = time.perf_counter()
+        oracle.chunk_fwd(arr["q"], arr["k"], arr["v"], arr["g"], arr["beta"], None, None,
+                         nthreads=cores)
+        dt = time.perf_counter() - t0
+        cpu = {"value": tokens / dt / 1e6, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"the whole workload once (B{B} T{T} H{H}, {dt:.2f} s)"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": B, "T": T, "H": H, "d_k": 128, "d_v": 128,
+                   "chunk": 64, "initial_state": "zeros", "final_state": True,
+                   "l2": "flushed before every timed step (256 MiB device write)",
+                   "parallelism": f"{world} independent replica(s), no collective"},
+        "roofline": {"bound": "hbm", "achieved": ach_gbs, "peak": pk["hbm"], "unit": "GB/s",
+                     "frac": ach_gbs / pk["hbm"], "traffic": traffic,
+                     "kernel": "gdn_chunk_fwd step (chunk_map + prep + scan)",
+                     "algorithmic_bytes": alg_bytes, "flops": flops,
+                     "tensor_frac": flops / (ms_local * 1e-3) / (pk["bf16"] * 1e12),
+                     "peak_source": pk["source"]},
+        "kernels_ms": kernels,
+        "kernel_share": {k2: v2 / tot for k2, v2 in kernels.items()},
+        "gpu_launches": 3 * K,
+        "clocks": clocks,
+        "e2e": e2e,
+        "decode": decode,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -64,6 +64,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_decode_step.restype = ci
         L.gdn_get_status.argtypes = [vp, vp]
         L.gdn_get_status.restype = ci
+        L.gdn_set_profile_events.argtypes = [vp, vp, vp, vp]
+        L.gdn_set_profile_events.restype = ci
         L.gdn_status_string.argtypes = [ci]
         L.gdn_status_string.restype = ctypes.c_char_p
         _lib = L

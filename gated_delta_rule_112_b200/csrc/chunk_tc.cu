@@ -673,6 +673,7 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     cudaError_t e = cudaFuncSetAttribute(gdn_prep_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kPrepSmem);
     if (e != cudaSuccess) return e;
+    prof_record(g_profile.prep, s);
     gdn_prep_kernel<<<dim3(L.max_chunks, H), kPrepThreads, kPrepSmem, s>>>(
         mq, mk, mv, mwt, mut, mpm, g, beta, reinterpret_cast<float *>(base + L.gam), H, ctrl,
         table);
@@ -681,15 +682,15 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     e = cudaFuncSetAttribute(gdn_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kScanSmem);
     if (e != cudaSuccess) return e;
+    prof_record(g_profile.scan, s);
     gdn_scan_kernel<<<dim3(N, H), kScanThreads, kScanSmem, s>>>(
         mq, mk, mwt, mut, mpm, mgm, s0, sN, static_cast<__nv_bfloat16 *>(o), H, ctrl, table,
         seq_first);
     return cudaGetLastError();
   }
   // No tokens: the final state is the initial state.
-  CUtensorMap dummy;
-  memset(&dummy, 0, sizeof(dummy));
-  (void)dummy;
+  prof_record(g_profile.prep, s);
+  prof_record(g_profile.scan, s);
   if (sN) {
     const size_t bytes = size_t(N) * H * kD * kD * sizeof(float);
     return s0 ? cudaMemcpyAsync(sN, s0, bytes, cudaMemcpyDeviceToDevice, s)

@@ -7,6 +7,10 @@
 
 using namespace gdn;
 
+namespace gdn {
+ProfileEvents g_profile = {nullptr, nullptr, nullptr, nullptr};
+}
+
 namespace {
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -49,13 +53,18 @@ int run_chunk(bool force_simt, const void *q, const void *k, const void *v, cons
   if (ws_bytes < L.total) return GDN_ERR_WORKSPACE;
   const int N = cu ? num_seqs : B;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  prof_record(g_profile.start, s);
   cudaError_t e = launch_chunk_map(cu, B, T, cu ? num_seqs : 0, chunk, ws, L, s);
   if (e != cudaSuccess) return GDN_ERR_CUDA;
-  if (tc)
+  if (tc) {
     e = launch_chunk_tc(q, k, v, g, beta, s0, B, T, H, N, o, sN, ws, L, s);
-  else
+  } else {
+    prof_record(g_profile.prep, s);
+    prof_record(g_profile.scan, s);
     e = launch_chunk_simt(q, k, v, g, beta, s0, cu, B, T, H, dk, dv, N, chunk, dtype, o, sN,
                           static_cast<uint32_t *>(ws), s);
+  }
+  prof_record(g_profile.end, s);
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -126,6 +135,16 @@ int gdn_get_status(void *workspace, void *stream) {
   }
   if (err & kErrTimeout) return GDN_ERR_DEVICE_TIMEOUT;
   if (err & kErrBadSeqlens) return GDN_ERR_INVALID_ARG;
+  return GDN_OK;
+}
+
+int gdn_set_profile_events(void *ev_start, void *ev_prep, void *ev_scan, void *ev_end) {
+  const int nulls = !ev_start + !ev_prep + !ev_scan + !ev_end;
+  if (nulls != 0 && nulls != 4) return GDN_ERR_INVALID_ARG;
+  g_profile.start = static_cast<cudaEvent_t>(ev_start);
+  g_profile.prep = static_cast<cudaEvent_t>(ev_prep);
+  g_profile.scan = static_cast<cudaEvent_t>(ev_scan);
+  g_profile.end = static_cast<cudaEvent_t>(ev_end);
   return GDN_OK;
 }
 

@@ -61,6 +61,16 @@ inline WsLayout ws_layout(int B, int T, int H, int num_seqs, int chunk, bool tc)
   return L;
 }
 
+// Optional events recorded around the chunked-forward kernels (see
+// gdn_set_profile_events). All null when profiling is off.
+struct ProfileEvents {
+  cudaEvent_t start, prep, scan, end;
+};
+extern ProfileEvents g_profile;
+inline void prof_record(cudaEvent_t e, cudaStream_t s) {
+  if (e) cudaEventRecord(e, s);
+}
+
 // Kernel launchers (defined in the .cu files; return a cudaError_t).
 cudaError_t launch_chunk_map(const int32_t *cu_seqlens, int B, int T, int num_seqs, int chunk,
                              void *ws, const WsLayout &L, cudaStream_t s);

@@ -148,6 +148,23 @@ int gdn_decode_step(const void *q, const void *k, const void *v, const float *g,
  */
 int gdn_get_status(void *workspace, void *stream);
 
+/*
+ * gdn_set_profile_events -- optional timing hook for benchmarks and profilers.
+ *
+ * When set (non-NULL cudaEvent_t handles passed as void*), every later
+ * gdn_chunk_fwd / gdn_chunk_fwd_simt call records them on its stream:
+ *   ev_start   before the chunk-map kernel,
+ *   ev_prep    before the per-chunk preparation kernel (tensor-core path;
+ *              the CUDA-core path records it right before its one kernel),
+ *   ev_scan    before the sequential scan/output kernel (CUDA-core path: same
+ *              point as ev_prep),
+ *   ev_end     after the last kernel.
+ * Pass four NULLs to stop. Process-wide setting, not thread-safe; the caller
+ * owns the events. Returns GDN_OK, or GDN_ERR_INVALID_ARG if only some of the
+ * four are NULL.
+ */
+int gdn_set_profile_events(void *ev_start, void *ev_prep, void *ev_scan, void *ev_end);
+
 /* Human-readable name of a status code (static string). */
 const char *gdn_status_string(int status);
 
