@@ -14,19 +14,21 @@
 //   S <- gamma_last S + V_new^T diag(exp(Gamma_last - Gamma)) K
 //
 // Two kernels:
-//   gdn_prep_kernel  one CTA per (chunk, head), fully parallel. Everything that
-//                    does not depend on the state: Gamma, A, P = (QK^T).*M,
-//                    T by blocked forward substitution, W^T and U^T on tcgen05.
-//                    Writes W^T, U^T, P (bf16) and Gamma (fp32) to the workspace.
+//   gdn_prep_kernel  one CTA per (chunk, head), fully parallel: everything that
+//                    depends only on the chunk's own K, Q, g, beta -- Gamma, A,
+//                    P = (Q K^T) .* M, T by blocked forward substitution, and
+//                    W^T = K^T (T diag(beta gamma))^T on tcgen05. Writes W^T,
+//                    T diag(beta), P (bf16) and the decay factors (fp32).
 //   gdn_scan_kernel  one CTA per (sequence, head), sequential over chunks:
-//                    the state-dependent products on tcgen05 with the fp32
-//                    master state in registers of the epilogue warps, and O.
+//                    U^T = V^T (T diag(beta))^T and the state-dependent
+//                    products on tcgen05, the fp32 state in registers of the
+//                    epilogue warps, and O.
 //
-// All matrices below are worked in the "transposed frame" where the 128-wide
-// head dimension is the MMA M dimension, so every tcgen05.mma is M = 128 and
-// each thread of the epilogue warpgroup owns one TMEM lane = one row of d_v
-// (or d_k). Shared-memory operand tiles use the 128-byte swizzle with 64
-// bf16 (128 bytes) per row; TMA loads have no cluster broadcast.
+// All products are worked in the "transposed frame" where the 128-wide head
+// dimension is the MMA M dimension, so every tcgen05.mma is M = 128 and each
+// epilogue thread owns one TMEM lane = one row of d_v (or d_k). Shared-memory
+// operand tiles use the 128-byte swizzle with 64 bf16 (128 bytes) per row;
+// TMA loads have no cluster broadcast.
 #include <cstdio>
 #include <cstring>
 
@@ -34,6 +36,11 @@
 #include "sm100_ptx.cuh"
 
 namespace gdn {
+
+#ifdef GDN_TRACE
+__device__ unsigned long long g_gdn_trace[2][kTraceSlots][kTraceEvents];
+#endif
+
 namespace {
 
 constexpr int kC = 64;    // chunk
@@ -43,82 +50,129 @@ constexpr uint32_t kTile128x64 = 128 * 128;   // 128 rows x 128 B = 16 KB
 
 // ===================================================================== prep
 // Shared memory of the prep kernel (offsets from a 1024-aligned base).
-constexpr uint32_t kP_KQ = 0;                       // 2 blocks x [K rows 0-63 | Q rows 64-127] = 32 KB
-constexpr uint32_t kP_V = kP_KQ + 2 * kTile128x64;  // 2 blocks x 64 rows = 16 KB
-constexpr uint32_t kP_TB = kP_V + 2 * kTile64x64;   // T diag(beta), bf16, K-major 64x64
-constexpr uint32_t kP_TBG = kP_TB + kTile64x64;     // T diag(beta gamma)
-constexpr uint32_t kP_PST = kP_TBG + kTile64x64;    // P staging for the TMA store
-constexpr uint32_t kP_AS = kP_PST + kTile64x64;     // A, fp32 [64][65]
-constexpr uint32_t kP_TS = kP_AS + 64 * 65 * 4;     // T, fp32 [64][65]
-constexpr uint32_t kP_XS = kP_TS + 64 * 65 * 4;     // scratch, fp32 3 x 16 x 16
-constexpr uint32_t kP_VEC = kP_XS + 3 * 256 * 4;    // Gamma, beta, gamma: 3 x 64 fp32
-constexpr uint32_t kP_BAR = kP_VEC + 3 * 64 * 4;    // 2 mbarriers + tmem address
+constexpr int kLd = 68;                              // fp32 row stride of A and T (16-byte rows)
+constexpr uint32_t kP_KQ = 0;                        // 2 blocks x [K rows 0-63 | Q rows 64-127] = 32 KB
+constexpr uint32_t kP_PST = kP_KQ + kTile64x64;      // P staging, over Q of block 0 (dead after G)
+constexpr uint32_t kP_WST = kP_KQ + kTile128x64;     // W^T staging, over block 1 (dead after W)
+constexpr uint32_t kP_AS = kP_KQ + 2 * kTile128x64;  // A, fp32 [64][68]; after the solve it
+constexpr uint32_t kP_TB = kP_AS;                    //   holds T diag(beta)       (bf16 64x64)
+constexpr uint32_t kP_TBG = kP_AS + kTile64x64;      //   and   T diag(beta gamma) (bf16 64x64)
+constexpr uint32_t kP_TS = kP_AS + 64 * kLd * 4;     // T, fp32 [64][68]
+constexpr uint32_t kP_XS = kP_TS + 64 * kLd * 4;     // solve scratch, fp32 [32][32]
+constexpr uint32_t kP_VEC = kP_XS + 1024 * 4;        // Gamma, beta, gamma: 3 x 64 fp32
+constexpr uint32_t kP_BAR = kP_VEC + 3 * 64 * 4;     // 2 mbarriers + tmem address
 constexpr uint32_t kP_END = kP_BAR + 64;
-constexpr uint32_t kPrepSmem = kP_END + 1024;       // + alignment slack
-constexpr int kPrepThreads = 128;
+constexpr uint32_t kPrepSmem = kP_END + 1024;        // + alignment slack
+constexpr int kPrepThreads = 256;
+static_assert(2 * kTile64x64 <= 64 * kLd * 4, "T tiles must fit in the A area");
+static_assert(kP_AS % 1024 == 0 && kP_PST % 1024 == 0 && kP_WST % 1024 == 0,
+              "swizzled tiles need 1024-byte alignment");
 
-// T = (I + A)^-1 for the strictly lower-triangular 64 x 64 A, in fp32 shared
-// memory, with 16 x 16 blocks: the four diagonal blocks are inverted by
-// column-wise forward substitution in registers, then each off-diagonal block
-// follows from T_ij = -T_ii (sum_{m=j}^{i-1} A_im T_mj), one block diagonal
-// at a time (every T_mj it needs lies on an earlier block diagonal).
+// T = (I + A)^-1 for the strictly lower-triangular 64 x 64 A (fp32 shared
+// memory, row stride kLd), by recursive 2 x 2 blocking: for a lower block
+// triangular [[L11, 0], [L21, L22]], the inverse is [[T11, 0], [-T22 L21 T11, T22]].
+//   step 0  the four 16 x 16 diagonal blocks, by column-wise forward
+//           substitution in registers (thread = one column of one block)
+//   step 1  the two 16 x 16 blocks T(1,0), T(3,2)        (two half-steps)
+//   step 2  the 32 x 32 block T([2,3],[0,1])             (two half-steps)
+// Every half-step is an independent small product over all 256 threads.
+// Entries above the diagonal of T are left unwritten and never read.
 __device__ void solve_unit_lower_64(const float *__restrict__ As, float *__restrict__ Ts,
                                     float *__restrict__ Xs, int tid) {
-  constexpr int P = 65;
   if (tid < 64) {
-    const int bb = tid >> 4, jj = tid & 15, base = bb * 16;
+    const int base = (tid >> 4) * 16, jj = tid & 15;
     float x[16];
 #pragma unroll
     for (int r = 0; r < 16; ++r) x[r] = (r == jj) ? 1.f : 0.f;
 #pragma unroll
     for (int r = 1; r < 16; ++r) {
-      float acc = 0.f;
+      const float *arow = As + (base + r) * kLd + base;
+      float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-      for (int m = 0; m < r; ++m) acc += As[(base + r) * P + base + m] * x[m];
-      if (r > jj) x[r] = -acc;
+      for (int m = 0; m < r; m += 2) {
+        a0 = fmaf(arow[m], x[m], a0);
+        if (m + 1 < r) a1 = fmaf(arow[m + 1], x[m + 1], a1);
+      }
+      if (r > jj) x[r] = -(a0 + a1);
     }
 #pragma unroll
-    for (int r = 0; r < 16; ++r) Ts[(base + r) * P + base + jj] = x[r];
-  } else {
-    // zero the blocks above the diagonal
-    for (int e = tid - 64; e < 64 * 64; e += 64) {
-      const int r = e >> 6, c = e & 63;
-      if ((c >> 4) > (r >> 4)) Ts[r * P + c] = 0.f;
-    }
+    for (int r = 0; r < 16; ++r) Ts[(base + r) * kLd + base + jj] = x[r];
   }
   __syncthreads();
-  for (int d = 1; d < 4; ++d) {
-    const int nblk = 4 - d;
-    // X_ij = sum_{m=16j}^{16i-1} A[16i+r][m] T[m][16j+c]
-    for (int o = tid; o < nblk * 256; o += kPrepThreads) {
-      const int b = o >> 8, r = (o >> 4) & 15, c = o & 15;
-      const int i = b + d, j = b;
-      float acc = 0.f;
-      for (int m = 16 * j; m < 16 * i; ++m) acc += As[(16 * i + r) * P + m] * Ts[m * P + 16 * j + c];
-      Xs[o] = acc;
+  {  // step 1a: Y_b = A(i, i-1) T(i-1, i-1) for i = 1, 3; thread: row r, 2 columns
+    const int b = tid >> 7, r = (tid >> 3) & 15, c = (tid & 7) * 2;
+    const int i0 = 16 * (2 * b + 1), j0 = i0 - 16;
+    const float *arow = As + (i0 + r) * kLd + j0;
+    float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+      const float2 t = *reinterpret_cast<const float2 *>(Ts + (j0 + m) * kLd + j0 + c);
+      const float tx = (m >= c) ? t.x : 0.f, ty = (m >= c + 1) ? t.y : 0.f;
+      y0 = fmaf(arow[m], tx, y0);
+      y1 = fmaf(arow[m], ty, y1);
     }
-    __syncthreads();
-    // T_ij = -T_ii X_ij
-    for (int o = tid; o < nblk * 256; o += kPrepThreads) {
-      const int b = o >> 8, r = (o >> 4) & 15, c = o & 15;
-      const int i = b + d, j = b;
-      float acc = 0.f;
-      for (int m = 0; m <= r; ++m) acc += Ts[(16 * i + r) * P + 16 * i + m] * Xs[(b << 8) + (m << 4) + c];
-      Ts[(16 * i + r) * P + 16 * j + c] = -acc;
-    }
-    __syncthreads();
+    *reinterpret_cast<float2 *>(Xs + b * 256 + r * 16 + c) = make_float2(y0, y1);
   }
+  __syncthreads();
+  {  // step 1b: T(i, i-1) = -T(i, i) Y_b
+    const int b = tid >> 7, r = (tid >> 3) & 15, c = (tid & 7) * 2;
+    const int i0 = 16 * (2 * b + 1), j0 = i0 - 16;
+    const float *trow = Ts + (i0 + r) * kLd + i0;
+    float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+      const float t = (m <= r) ? trow[m] : 0.f;
+      const float2 x = *reinterpret_cast<const float2 *>(Xs + b * 256 + m * 16 + c);
+      y0 = fmaf(t, x.x, y0);
+      y1 = fmaf(t, x.y, y1);
+    }
+    *reinterpret_cast<float2 *>(Ts + (i0 + r) * kLd + j0 + c) = make_float2(-y0, -y1);
+  }
+  __syncthreads();
+  {  // step 2a: Y = A([32,64), [0,32)) T([0,32), [0,32)); thread: row r, 4 columns
+    const int r = tid >> 3, c = (tid & 7) * 4;
+    const float *arow = As + (32 + r) * kLd;
+    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int m = 0; m < 32; ++m) {
+      const float a = arow[m];
+      const float4 t = *reinterpret_cast<const float4 *>(Ts + m * kLd + c);
+      // T([0,32),[0,32)) is lower triangular; entries with column > row are garbage.
+      y.x = fmaf(a, (m >= c + 0) ? t.x : 0.f, y.x);
+      y.y = fmaf(a, (m >= c + 1) ? t.y : 0.f, y.y);
+      y.z = fmaf(a, (m >= c + 2) ? t.z : 0.f, y.z);
+      y.w = fmaf(a, (m >= c + 3) ? t.w : 0.f, y.w);
+    }
+    *reinterpret_cast<float4 *>(Xs + r * 32 + c) = y;
+  }
+  __syncthreads();
+  {  // step 2b: T([32,64), [0,32)) = -T([32,64), [32,64)) Y
+    const int r = tid >> 3, c = (tid & 7) * 4;
+    const float *trow = Ts + (32 + r) * kLd + 32;
+    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int m = 0; m < 32; ++m) {
+      const float t = (m <= r) ? trow[m] : 0.f;
+      const float4 x = *reinterpret_cast<const float4 *>(Xs + m * 32 + c);
+      y.x = fmaf(t, x.x, y.x); y.y = fmaf(t, x.y, y.y);
+      y.z = fmaf(t, x.z, y.z); y.w = fmaf(t, x.w, y.w);
+    }
+    *reinterpret_cast<float4 *>(Ts + (32 + r) * kLd + c) = make_float4(-y.x, -y.y, -y.z, -y.w);
+  }
+  __syncthreads();
 }
 
-__global__ void __launch_bounds__(kPrepThreads, 2) gdn_prep_kernel(
+// Warp roles: all 8 warps share the epilogues. TMEM lane quarter = warp % 4,
+// column half = warp / 4.
+__global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_wt,
-    const __grid_constant__ CUtensorMap tm_ut, const __grid_constant__ CUtensorMap tm_pm,
-    const float *__restrict__ g, const float *__restrict__ beta, float *__restrict__ gam_out,
-    int H, uint32_t *__restrict__ ctrl, const ChunkInfo *__restrict__ table) {
+    const __grid_constant__ CUtensorMap tm_wt, const __grid_constant__ CUtensorMap tm_tb,
+    const __grid_constant__ CUtensorMap tm_pm, const float *__restrict__ g,
+    const float *__restrict__ beta, float *__restrict__ gam_out, int H,
+    uint32_t *__restrict__ ctrl, const ChunkInfo *__restrict__ table) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                            ~uintptr_t(1023));
+  // Pointer arithmetic (not integer casts) keeps the shared address space.
+  uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   __shared__ int abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int chunk = blockIdx.x, h = blockIdx.y;
@@ -127,6 +181,9 @@ __global__ void __launch_bounds__(kPrepThreads, 2) gdn_prep_kernel(
   const ChunkInfo ci = table[chunk];
   const int L = ci.len;
   const int unit = chunk * H + h;
+  const bool tr = (h == 0 && tid == 0);   // traced thread (GDN_TRACE builds only)
+  (void)tr;
+  GDN_TRACE_POINT(tr, 1, chunk, 0);
 
   float *As = reinterpret_cast<float *>(sm + kP_AS);
   float *Ts = reinterpret_cast<float *>(sm + kP_TS);
@@ -142,13 +199,12 @@ __global__ void __launch_bounds__(kPrepThreads, 2) gdn_prep_kernel(
     abort_flag = 0;
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
     mbar_init(bar_load, 1);
     mbar_init(bar_mma, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(tmem_slot, 256);
+    tmem_alloc(tmem_slot, 128);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -157,13 +213,11 @@ __global__ void __launch_bounds__(kPrepThreads, 2) gdn_prep_kernel(
   const uint32_t tmem = *tmem_slot;
 
   if (tid == 0) {
-    mbar_arrive_expect_tx(bar_load, 2 * kTile128x64 + 2 * kTile64x64);
+    mbar_arrive_expect_tx(bar_load, 2 * kTile128x64);
     tma_load_3d(sm + kP_KQ, &tm_k, bar_load, 0, h, ci.row0);
     tma_load_3d(sm + kP_KQ + kTile64x64, &tm_q, bar_load, 0, h, ci.row0);
     tma_load_3d(sm + kP_KQ + kTile128x64, &tm_k, bar_load, 64, h, ci.row0);
     tma_load_3d(sm + kP_KQ + kTile128x64 + kTile64x64, &tm_q, bar_load, 64, h, ci.row0);
-    tma_load_3d(sm + kP_V, &tm_v, bar_load, 0, h, ci.row0);
-    tma_load_3d(sm + kP_V + kTile64x64, &tm_v, bar_load, 64, h, ci.row0);
   }
   if (tid < kC) {
     const bool ok = tid < L;
@@ -172,7 +226,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) gdn_prep_kernel(
   }
   __syncthreads();
   if (warp == 0) {  // inclusive cumsum of the 64 log-gates
-    float a0 = Gm[2 * lane], a1 = Gm[2 * lane + 1];
+    const float a0 = Gm[2 * lane], a1 = Gm[2 * lane + 1];
     float s = a0 + a1;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -184,8 +238,9 @@ __global__ void __launch_bounds__(kPrepThreads, 2) gdn_prep_kernel(
     Gm[2 * lane + 1] = s;
   }
   const bool loaded = mbar_wait(bar_load, 0, ctrl, &abort_flag);
+  GDN_TRACE_POINT(tr, 1, chunk, 1);
   if (loaded && L < kC) {
-    // Rows past the sequence end act as k = q = v = 0.
+    // Rows past the sequence end act as k = q = 0 (beta = g = 0 above).
     for (int e = tid; e < (kC - L) * 8; e += kPrepThreads) {
       const int r = L + e / 8, ch = e % 8;
       const uint4 z = make_uint4(0, 0, 0, 0);
@@ -193,8 +248,6 @@ __global__ void __launch_bounds__(kPrepThreads, 2) gdn_prep_kernel(
       *reinterpret_cast<uint4 *>(sm + kP_KQ + kTile64x64 + r * 128 + ch * 16) = z;
       *reinterpret_cast<uint4 *>(sm + kP_KQ + kTile128x64 + r * 128 + ch * 16) = z;
       *reinterpret_cast<uint4 *>(sm + kP_KQ + kTile128x64 + kTile64x64 + r * 128 + ch * 16) = z;
-      *reinterpret_cast<uint4 *>(sm + kP_V + r * 128 + ch * 16) = z;
-      *reinterpret_cast<uint4 *>(sm + kP_V + kTile64x64 + r * 128 + ch * 16) = z;
     }
     fence_proxy_async_smem();
   }
@@ -212,62 +265,73 @@ __global__ void __launch_bounds__(kPrepThreads, 2) gdn_prep_kernel(
     }
     tc_commit(bar_mma);
   }
-  if (tid < kC) Ga[tid] = expf(Gm[tid]);
+  if (tid < kC) {
+    Ga[tid] = __expf(Gm[tid]);
+    gam_out[size_t(unit) * 128 + tid] = expf(Gm[tid]);                   // gamma_c
+    gam_out[size_t(unit) * 128 + 64 + tid] = expf(Gm[kC - 1] - Gm[tid]);  // D_s
+  }
   mbar_wait(bar_mma, 0, ctrl, &abort_flag);
+  GDN_TRACE_POINT(tr, 1, chunk, 2);
   tc_fence_after();
-  const int m = warp * 32 + lane;  // TMEM lane = row of G
+  const int m = (warp & 3) * 32 + lane;   // TMEM lane = row of G
+  const int hc = warp >> 2;               // column half
+  const uint32_t lane_base = tmem + (uint32_t((warp & 3) * 32) << 16);
   if (!abort_flag) {
-    uint32_t r0[32], r1[32];
-    const uint32_t taddr = tmem + (uint32_t(warp * 32) << 16);
-    tmem_ld32(taddr, r0);
-    tmem_ld32(taddr + 32, r1);
+    uint32_t r0[32];
+    tmem_ld32(lane_base + 32 * hc, r0);
     tmem_ld_wait();
     if (m < kC) {
       const int r = m;
       const float br = Bt[r], gr = Gm[r];
 #pragma unroll
-      for (int s = 0; s < 32; ++s)
-        As[r * 65 + s] = (s < r) ? br * expf(gr - Gm[s]) * __uint_as_float(r0[s]) : 0.f;
-#pragma unroll
-      for (int s = 0; s < 32; ++s)
-        As[r * 65 + 32 + s] = (32 + s < r) ? br * expf(gr - Gm[32 + s]) * __uint_as_float(r1[s]) : 0.f;
+      for (int t = 0; t < 32; t += 4) {
+        float4 a;
+        const int s = 32 * hc + t;
+        a.x = (s + 0 < r) ? br * __expf(gr - Gm[s + 0]) * __uint_as_float(r0[t + 0]) : 0.f;
+        a.y = (s + 1 < r) ? br * __expf(gr - Gm[s + 1]) * __uint_as_float(r0[t + 1]) : 0.f;
+        a.z = (s + 2 < r) ? br * __expf(gr - Gm[s + 2]) * __uint_as_float(r0[t + 2]) : 0.f;
+        a.w = (s + 3 < r) ? br * __expf(gr - Gm[s + 3]) * __uint_as_float(r0[t + 3]) : 0.f;
+        *reinterpret_cast<float4 *>(As + r * kLd + s) = a;
+      }
     } else {
       const int c = m - kC;
       const float gc = Gm[c];
-      uint8_t *prow = sm + kP_PST;
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
+      for (int cc = 0; cc < 4; ++cc) {
+        const int ch = 4 * hc + cc;
         float f[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int s = ch * 8 + e;
-          const float gv = __uint_as_float(ch < 4 ? r0[s & 31] : r1[s & 31]);
-          f[e] = (s <= c) ? expf(gc - Gm[s]) * gv : 0.f;
+          f[e] = (s <= c) ? __expf(gc - Gm[s]) * __uint_as_float(r0[8 * cc + e]) : 0.f;
         }
-        uint4 pk = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
-                              pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
-        *reinterpret_cast<uint4 *>(prow + sw128_offset(c, ch)) = pk;
+        *reinterpret_cast<uint4 *>(sm + kP_PST + sw128_offset(c, ch)) =
+            make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                       pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
       }
     }
   }
   fence_proxy_async_smem();
+  tc_fence_before();
   __syncthreads();
   if (!abort_flag && tid == 0) {
     tma_store_2d(&tm_pm, sm + kP_PST, 0, unit * kC);
     tma_store_commit();
   }
+  GDN_TRACE_POINT(tr, 1, chunk, 3);
   if (!abort_flag) solve_unit_lower_64(As, Ts, Xs, tid);
-  // T diag(beta) and T diag(beta gamma) as bf16 K-major operand tiles
+  GDN_TRACE_POINT(tr, 1, chunk, 4);
+  // T diag(beta) and T diag(beta gamma) as bf16 K-major operand tiles (A is dead now)
   {
-    const int r = tid >> 1, half = tid & 1;
+    const int r = tid >> 2, q4 = tid & 3;
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-      const int ch = half * 4 + cc;
+    for (int cc = 0; cc < 2; ++cc) {
+      const int ch = q4 * 2 + cc;
       float fb[8], fg[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const int s = ch * 8 + e;
-        const float t = Ts[r * 65 + s] * Bt[s];
+        const float t = (s <= r) ? Ts[r * kLd + s] * Bt[s] : 0.f;
         fb[e] = t;
         fg[e] = t * Ga[s];
       }
@@ -281,48 +345,37 @@ __global__ void __launch_bounds__(kPrepThreads, 2) gdn_prep_kernel(
   }
   fence_proxy_async_smem();
   __syncthreads();
+  GDN_TRACE_POINT(tr, 1, chunk, 5);
   if (!abort_flag && tid == 0) {
+    tma_store_2d(&tm_tb, sm + kP_TB, 0, unit * kC);
+    tma_store_commit();
     tc_fence_after();
-    // W^T = K^T (T diag(beta gamma))^T : M = 128 (d_k), N = 64, K = 64 (tokens)
-    // U^T = V^T (T diag(beta))^T       : M = 128 (d_v), N = 64, K = 64
+    // W^T = K^T (T diag(beta gamma))^T : M = 128 (d_k), N = 64, K = 64 (tokens) -> cols [64, 128)
     const uint32_t idesc = make_idesc_bf16(128, 64, 1, 0);
-    const uint32_t kq = smem_u32(sm + kP_KQ), vv = smem_u32(sm + kP_V);
-    const uint32_t tbg = smem_u32(sm + kP_TBG), tb = smem_u32(sm + kP_TB);
+    const uint32_t kq = smem_u32(sm + kP_KQ), tbg = smem_u32(sm + kP_TBG);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
       tc_mma_bf16(tmem + 64, make_sdesc(kq + kk * 2048, kTile128x64, 1024),
                   make_sdesc(tbg + kk * 32, 16, 1024), idesc, kk > 0);
     }
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      tc_mma_bf16(tmem + 128, make_sdesc(vv + kk * 2048, kTile64x64, 1024),
-                  make_sdesc(tb + kk * 32, 16, 1024), idesc, kk > 0);
-    }
     tc_commit(bar_mma);
   }
-  if (tid < kC) gam_out[size_t(unit) * kC + tid] = Gm[tid];
   mbar_wait(bar_mma, 1, ctrl, &abort_flag);
+  GDN_TRACE_POINT(tr, 1, chunk, 6);
   tc_fence_after();
   if (!abort_flag) {
-    // Row m of W^T / U^T -> bf16 staging tiles (reusing the K/Q and V areas).
-    const uint32_t taddr = tmem + (uint32_t(warp * 32) << 16);
+    // Row m of W^T, columns [32 hc, 32 hc + 32) -> bf16 staging over K/Q block 1.
+    uint32_t r0[32];
+    tmem_ld32(lane_base + 64 + 32 * hc, r0);
+    tmem_ld_wait();
 #pragma unroll
-    for (int which = 0; which < 2; ++which) {
-      uint32_t r0[32], r1[32];
-      tmem_ld32(taddr + 64 + which * 64, r0);
-      tmem_ld32(taddr + 96 + which * 64, r1);
-      tmem_ld_wait();
-      uint8_t *dst = sm + (which == 0 ? kP_KQ : kP_V);
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        const uint32_t *src = ch < 4 ? r0 : r1;
-        const int b = (ch & 3) * 8;
-        *reinterpret_cast<uint4 *>(dst + sw128_offset(m, ch)) = make_uint4(
-            pack_bf16x2(__uint_as_float(src[b + 0]), __uint_as_float(src[b + 1])),
-            pack_bf16x2(__uint_as_float(src[b + 2]), __uint_as_float(src[b + 3])),
-            pack_bf16x2(__uint_as_float(src[b + 4]), __uint_as_float(src[b + 5])),
-            pack_bf16x2(__uint_as_float(src[b + 6]), __uint_as_float(src[b + 7])));
-      }
+    for (int cc = 0; cc < 4; ++cc) {
+      const int b = cc * 8;
+      *reinterpret_cast<uint4 *>(sm + kP_WST + sw128_offset(m, 4 * hc + cc)) = make_uint4(
+          pack_bf16x2(__uint_as_float(r0[b + 0]), __uint_as_float(r0[b + 1])),
+          pack_bf16x2(__uint_as_float(r0[b + 2]), __uint_as_float(r0[b + 3])),
+          pack_bf16x2(__uint_as_float(r0[b + 4]), __uint_as_float(r0[b + 5])),
+          pack_bf16x2(__uint_as_float(r0[b + 6]), __uint_as_float(r0[b + 7])));
     }
   }
   fence_proxy_async_smem();
@@ -330,78 +383,112 @@ __global__ void __launch_bounds__(kPrepThreads, 2) gdn_prep_kernel(
   __syncthreads();
   if (tid == 0) {
     if (!abort_flag) {
-      tma_store_2d(&tm_wt, sm + kP_KQ, 0, unit * kD);
-      tma_store_2d(&tm_ut, sm + kP_V, 0, unit * kD);
+      tma_store_2d(&tm_wt, sm + kP_WST, 0, unit * kD);
       tma_store_commit();
     }
+    GDN_TRACE_POINT(tr, 1, chunk, 7);
     tma_store_wait_all();
+    GDN_TRACE_POINT(tr, 1, chunk, 8);
   }
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 128);
   }
 }
 
 // ===================================================================== scan
-// Per stage (one chunk of one head): W^T, U^T, Q, K, P, Gamma.
-constexpr uint32_t kS_WT = 0;                       // [128 d_k][64 c]   MN-major B of S W^T
-constexpr uint32_t kS_UT = kS_WT + kTile128x64;     // [128 d_v][64 s]
-constexpr uint32_t kS_Q = kS_UT + kTile128x64;      // 2 x [64 c][64 d]  K-major B of S Q^T
-constexpr uint32_t kS_K = kS_Q + 2 * kTile64x64;    // 2 x [64 s][64 d]  MN-major B of dS
-constexpr uint32_t kS_P = kS_K + 2 * kTile64x64;    // [64 c][64 s]      K-major B of Y
-constexpr uint32_t kS_G = kS_P + kTile64x64;        // 64 fp32
-constexpr uint32_t kStageBytes = kS_G + 1024;       // keep stages 1024-aligned
-constexpr uint32_t kStageTx = 4 * kTile128x64 + kTile64x64 + 256;
-constexpr int kStages = 2;
-constexpr uint32_t kS_STATE = kStages * kStageBytes;          // S, bf16 [128 d_v][128 d_k]: 2 blocks
-constexpr uint32_t kS_A1 = kS_STATE + 2 * kTile128x64;        // V_new^T           [128][64]
-constexpr uint32_t kS_A2 = kS_A1 + kTile128x64;               // V_new^T diag(D)   [128][64]
-constexpr uint32_t kS_BAR = kS_A2 + kTile128x64;
-constexpr uint32_t kS_END = kS_BAR + 128;
-constexpr uint32_t kScanSmem = kS_END + 1024;
-constexpr int kScanThreads = 256;
-// TMEM columns
-constexpr uint32_t kT_X = 0, kT_Z = 64, kT_Y = 192, kT_DS = 320;
+// One stage (one chunk of one head): W^T, Q, K, V, T diag(beta), P. The
+// per-chunk decay factors (gamma[64], D[64]) travel in a separate 4-slot ring
+// so the output warps, which need only gamma, never hold a stage.
+constexpr uint32_t kS_WT = 0;                        // [128 d_k][64 c]   MN-major B of S W^T
+constexpr uint32_t kS_Q = kS_WT + kTile128x64;       // 2 x [64 c][64 d]  K-major B of S Q^T
+constexpr uint32_t kS_K = kS_Q + 2 * kTile64x64;     // 2 x [64 s][64 d]  MN-major B of dS
+constexpr uint32_t kS_V = kS_K + 2 * kTile64x64;     // 2 x [64 s][64 d]  MN-major A of U^T
+constexpr uint32_t kS_TB = kS_V + 2 * kTile64x64;    // [64 r][64 s]      K-major B of U^T
+constexpr uint32_t kS_P = kS_TB + kTile64x64;        // [64 c][64 s]      K-major B of Y
+constexpr uint32_t kStageBytes = kS_P + kTile64x64;  // 80 KB, multiple of 1024
+constexpr int kStages = 2, kGamSlots = 4;
+constexpr uint32_t kS_OST = kStages * kStageBytes;            // O staging, 2 x [64 c][64 d]
+constexpr uint32_t kS_GAM = kS_OST + 2 * kTile64x64;          // kGamSlots x 128 fp32
+constexpr uint32_t kS_BAR = kS_GAM + kGamSlots * 512;         // mbarriers, tmem slot, flags
+constexpr uint32_t kS_END = kS_BAR + 256;
+constexpr uint32_t kScanSmem = kS_END;   // the dynamic window starts 1024-aligned (checked)
+constexpr uint32_t kStageTx = kStageBytes;
+constexpr int kScanThreads = 512;
+// TMEM columns: fp32 accumulators, then the bf16 A operands of the MMAs.
+constexpr uint32_t kT_X = 0;      // U^T - S W^T = V_new^T   fp32 [128][64]
+constexpr uint32_t kT_Z = 64;     // S Q^T, two buffers      fp32 2 x [128][64]
+constexpr uint32_t kT_Y = 192;    // V_new^T P^T             fp32 [128][64]
+constexpr uint32_t kT_DS = 256;   // V_new^T D K             fp32 [128][128]
+constexpr uint32_t kT_S = 384;    // S                       bf16 [128][128] (64 columns)
+constexpr uint32_t kT_A1 = 448;   // V_new^T                 bf16 [128][64]  (32 columns)
+constexpr uint32_t kT_A2 = 480;   // V_new^T diag(D)         bf16 [128][64]  (32 columns)
+// Named barriers (0 is __syncthreads)
+constexpr uint32_t kBarChain = 1, kBarOut = 2;
+// Barrier slots in the kS_BAR area
+constexpr int kB_FULL = 0, kB_EMPTY = 2, kB_GFULL = 4, kB_GEMPTY = 8, kB_XFULL = 12,
+              kB_SFULL = 13, kB_YFULL = 14, kB_ZFREE = 15, kB_YFREE = 17, kB_DRAIN = 18,
+              kB_COUNT = 19;
 
+// Warp roles (16 warps):
+//   warp 0        TMA producer (one elected lane)
+//   warp 1        TMEM allocation
+//   warps 4-11    state chain: two warpgroups, warpgroup h owns columns
+//                 [32h, 32h+32) of V_new and [64h, 64h+64) of S; thread =
+//                 TMEM lane = row i of d_v; the fp32 S lives in its registers,
+//                 its bf16 copy (an MMA operand) in tensor memory.
+//                 Lane 0 of warp 4 also issues every tcgen05.mma.
+//   warps 12-15   output: O = diag(gamma) Q S^T + P V_new, staged for TMA stores
+// Chain per chunk: X = U^T - S W^T -> V_new -> dS = V_new^T diag(D) K ->
+// S = gamma_last S + dS. U^T = V^T (T diag(beta))^T is computed into X ahead
+// of time; Z = S Q^T and Y = V_new^T P^T run beside the chain. The A operands
+// of the state products live in tensor memory, so the tensor core reads only
+// the B tiles (and V) from shared memory.
 __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-    const __grid_constant__ CUtensorMap tm_wt, const __grid_constant__ CUtensorMap tm_ut,
-    const __grid_constant__ CUtensorMap tm_pm, const __grid_constant__ CUtensorMap tm_gam,
+    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_wt,
+    const __grid_constant__ CUtensorMap tm_tb, const __grid_constant__ CUtensorMap tm_pm,
+    const __grid_constant__ CUtensorMap tm_gam, const __grid_constant__ CUtensorMap tm_o,
     const float *__restrict__ s0, float *__restrict__ sN, __nv_bfloat16 *__restrict__ o, int H,
     uint32_t *__restrict__ ctrl, const ChunkInfo *__restrict__ table,
     const int32_t *__restrict__ seq_first) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                            ~uintptr_t(1023));
-  __shared__ int abort_flag;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *sm = smem_raw;                 // pointer arithmetic keeps the shared space
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n = blockIdx.x, h = blockIdx.y;
   if (ctrl[0] & kErrBadSeqlens) return;
+  if (smem_u32(sm) & 1023) {              // swizzled tiles need a 1024-aligned base
+    if (tid == 0) atomicOr(ctrl, kErrLayout);
+    return;
+  }
   const int c0 = seq_first[n], nch = seq_first[n + 1] - c0;
+  const bool tr = (n == 0 && h == 0);     // traced CTA (GDN_TRACE builds only)
+  (void)tr;
 
-  uint64_t *full = reinterpret_cast<uint64_t *>(sm + kS_BAR);  // [2]
-  uint64_t *empty = full + 2;                                   // [2]
-  uint64_t *s_ready = full + 4;
-  uint64_t *x_full = full + 5;
-  uint64_t *vnew_ready = full + 6;
-  uint64_t *s_full = full + 7;
-  uint64_t *y_full = full + 8;
-  uint64_t *drain = full + 9;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(full + 10);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kS_BAR);
+  uint64_t *full = bars + kB_FULL, *empty = bars + kB_EMPTY;
+  uint64_t *gfull = bars + kB_GFULL, *gempty = bars + kB_GEMPTY;
+  uint64_t *x_full = bars + kB_XFULL, *s_full = bars + kB_SFULL, *y_full = bars + kB_YFULL;
+  uint64_t *z_free = bars + kB_ZFREE, *y_free = bars + kB_YFREE, *drain = bars + kB_DRAIN;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kB_COUNT);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   if (tid == 0) {
-    abort_flag = 0;
+    *abort_flag = 0;
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_wt);
-    tma_prefetch_desc(&tm_ut);
+    tma_prefetch_desc(&tm_tb);
     tma_prefetch_desc(&tm_pm);
     tma_prefetch_desc(&tm_gam);
-    for (int i = 0; i < 10; ++i) mbar_init(full + i, 1);
+    tma_prefetch_desc(&tm_o);
+    for (int b = 0; b < kB_COUNT; ++b)
+      mbar_init(bars + b, (b >= kB_GEMPTY && b < kB_GEMPTY + 4) ? 2 : 1);
     fence_mbar_init();
   }
-  if (warp == 2) {
+  if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -409,191 +496,274 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Waits used by the warpgroups that keep named barriers in step: after an
+  // abort they return at once instead of leaving the loop.
+  auto wait = [&](uint64_t *bar, uint32_t parity) {
+    if (!*abort_flag) mbar_wait(bar, parity, ctrl, abort_flag);
+  };
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ TMA producer
     for (int c = 0; c < nch; ++c) {
-      const int st = c & 1;
-      if (c >= 2 && !mbar_wait(empty + st, ((c >> 1) - 1) & 1, ctrl, &abort_flag)) break;
+      const int st = c & 1, gs = c & 3;
+      if (c >= 2 && !mbar_wait(empty + st, ((c >> 1) - 1) & 1, ctrl, abort_flag)) break;
       const ChunkInfo ci = table[c0 + c];
       const int unit = (c0 + c) * H + h;
       uint8_t *sb = sm + st * kStageBytes;
+      GDN_TRACE_POINT(tr, 0, c, 0);
       mbar_arrive_expect_tx(full + st, kStageTx);
       tma_load_2d(sb + kS_WT, &tm_wt, full + st, 0, unit * kD);
-      tma_load_2d(sb + kS_UT, &tm_ut, full + st, 0, unit * kD);
+      tma_load_3d(sb + kS_V, &tm_v, full + st, 0, h, ci.row0);
+      tma_load_3d(sb + kS_V + kTile64x64, &tm_v, full + st, 64, h, ci.row0);
+      tma_load_2d(sb + kS_TB, &tm_tb, full + st, 0, unit * kC);
       tma_load_3d(sb + kS_Q, &tm_q, full + st, 0, h, ci.row0);
       tma_load_3d(sb + kS_Q + kTile64x64, &tm_q, full + st, 64, h, ci.row0);
       tma_load_3d(sb + kS_K, &tm_k, full + st, 0, h, ci.row0);
       tma_load_3d(sb + kS_K + kTile64x64, &tm_k, full + st, 64, h, ci.row0);
       tma_load_2d(sb + kS_P, &tm_pm, full + st, 0, unit * kC);
-      tma_load_2d(sb + kS_G, &tm_gam, full + st, 0, unit);
+      if (c >= 4 && !mbar_wait(gempty + gs, ((c >> 2) - 1) & 1, ctrl, abort_flag)) break;
+      mbar_arrive_expect_tx(gfull + gs, 512);
+      tma_load_2d(sm + kS_GAM + gs * 512, &tm_gam, gfull + gs, 0, unit);
     }
-  } else if (warp == 1 && lane == 0) {
-    // ------------------------------------------------------------ MMA issuer
-    const uint32_t id_x = make_idesc_bf16(128, 64, 0, 1);    // S W^T : B MN-major
-    const uint32_t id_z = make_idesc_bf16(128, 64, 0, 0);    // S Q^T : B K-major
-    const uint32_t id_s = make_idesc_bf16(128, 128, 0, 1);   // A2 K  : B MN-major
-    const uint32_t id_y = make_idesc_bf16(128, 64, 0, 0);    // A1 P^T: B K-major
-    const uint32_t sS = smem_u32(sm + kS_STATE);
-    const uint32_t sA1 = smem_u32(sm + kS_A1), sA2 = smem_u32(sm + kS_A2);
-    for (int c = 0; c < nch; ++c) {
+  } else if (warp >= 4 && warp < 12) {
+    // ------------------------------------------------------------ state chain
+    const int hh = (warp - 4) >> 2;                     // column half
+    const int i = ((warp & 3) << 5) + lane;             // TMEM lane = row of d_v
+    const uint32_t lane_base = tmem + (uint32_t((warp & 3) * 32) << 16);
+    const bool leader = (warp == 4 && lane == 0);
+    const uint32_t id_u = make_idesc_bf16(128, 64, 1, 0);       // V^T Tb^T : A MN-major
+    const uint32_t id_x = make_idesc_bf16(128, 64, 0, 1, 1);    // -S W^T   : B MN-major, negated
+    const uint32_t id_z = make_idesc_bf16(128, 64, 0, 0);       // S Q^T    : B K-major
+    const uint32_t id_s = make_idesc_bf16(128, 128, 0, 1);      // A2 K     : B MN-major
+    const uint32_t id_y = make_idesc_bf16(128, 64, 0, 0);       // A1 P^T   : B K-major
+    // Leader only. U(c): X = V^T (T diag(beta))^T, once chunk c is loaded and
+    // the chain has read X of chunk c - 1.
+    auto issue_u = [&](int c) {
       const int st = c & 1;
       const uint32_t sb = smem_u32(sm + st * kStageBytes);
-      if (!mbar_wait(full + st, (c >> 1) & 1, ctrl, &abort_flag)) break;
-      if (!mbar_wait(s_ready, c & 1, ctrl, &abort_flag)) break;
+      if (!mbar_wait(full + st, (c >> 1) & 1, ctrl, abort_flag)) return;
       tc_fence_after();
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint64_t a = make_sdesc(sS + (kk >> 2) * kTile128x64 + (kk & 3) * 32, 16, 1024);
-        tc_mma_bf16(tmem + kT_X, a, make_sdesc(sb + kS_WT + kk * 2048, kTile64x64, 1024), id_x,
-                    kk > 0);
-      }
+      for (int kk = 0; kk < 4; ++kk)
+        tc_mma_bf16(tmem + kT_X, make_sdesc(sb + kS_V + kk * 2048, kTile64x64, 1024),
+                    make_sdesc(sb + kS_TB + kk * 32, 16, 1024), id_u, kk > 0);
+    };
+    // Leader only. X(c) -= S_c W_c^T and Z(c) = S_c Q_c^T, both reading the
+    // bf16 copy of S_c.
+    auto issue_xz = [&](int c) {
+      const int st = c & 1;
+      const uint32_t sb = smem_u32(sm + st * kStageBytes);
+      GDN_TRACE_POINT(tr, 0, c, 1);
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        tc_mma_bf16_ts(tmem + kT_X, tmem + kT_S + 8 * kk,
+                       make_sdesc(sb + kS_WT + kk * 2048, kTile64x64, 1024), id_x, 1);
       tc_commit(x_full);
-      const uint32_t zcol = kT_Z + (c & 1) * 64;
+      // Z of chunk c uses buffer c & 1, last read by the output warps for
+      // chunk c - 2. One barrier per buffer, so no wait falls two phases behind.
+      if (c >= 2 && !mbar_wait(z_free + (c & 1), ((c >> 1) - 1) & 1, ctrl, abort_flag)) return;
+      GDN_TRACE_POINT(tr, 0, c, 2);
+      const uint32_t zcol = kT_Z + 64 * (c & 1);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
-        const uint64_t a = make_sdesc(sS + (kk >> 2) * kTile128x64 + (kk & 3) * 32, 16, 1024);
         const uint64_t b =
             make_sdesc(sb + kS_Q + (kk >> 2) * kTile64x64 + (kk & 3) * 32, 16, 1024);
-        tc_mma_bf16(tmem + zcol, a, b, id_z, kk > 0);
+        tc_mma_bf16_ts(tmem + zcol, tmem + kT_S + 8 * kk, b, id_z, kk > 0);
       }
-      if (!mbar_wait(vnew_ready, c & 1, ctrl, &abort_flag)) break;
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        tc_mma_bf16(tmem + kT_DS, make_sdesc(sA2 + kk * 32, 16, 1024),
-                    make_sdesc(sb + kS_K + kk * 2048, kTile64x64, 1024), id_s, kk > 0);
-      }
-      tc_commit(s_full);
-      const uint32_t ycol = kT_Y + (c & 1) * 64;
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        tc_mma_bf16(tmem + ycol, make_sdesc(sA1 + kk * 32, 16, 1024),
-                    make_sdesc(sb + kS_P + kk * 32, 16, 1024), id_y, kk > 0);
-      }
-      tc_commit(y_full);
-    }
-    // Every MMA issued above has completed once this fires.
-    tc_commit(drain);
-    mbar_wait(drain, 0, ctrl, &abort_flag);
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ epilogue
-    const int i = tid - 128;                      // TMEM lane = row of d_v
-    const uint32_t lane_base = tmem + (uint32_t((warp - 4) * 32) << 16);
-    float S[kD];                                  // S[i][j], fp32 master
+    };
+    float S[64];                                        // S[i][64 hh + t], fp32 master
     {
       const float *src = s0 ? s0 + (size_t(n) * H + h) * kD * kD : nullptr;
 #pragma unroll
-      for (int j = 0; j < kD; ++j) S[j] = src ? src[size_t(j) * kD + i] : 0.f;
+      for (int t = 0; t < 64; ++t) S[t] = src ? src[size_t(64 * hh + t) * kD + i] : 0.f;
     }
-    auto store_state_bf16 = [&]() {
+    // bf16 copy of S (row i, columns [64 hh, 64 hh + 64)) into tensor memory.
+    auto store_state = [&]() {
 #pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        const int j = ch * 8;
-        *reinterpret_cast<uint4 *>(sm + kS_STATE + (ch >> 3) * kTile128x64 +
-                                   sw128_offset(i, ch & 7)) =
-            make_uint4(pack_bf16x2(S[j], S[j + 1]), pack_bf16x2(S[j + 2], S[j + 3]),
-                       pack_bf16x2(S[j + 4], S[j + 5]), pack_bf16x2(S[j + 6], S[j + 7]));
+      for (int q = 0; q < 2; ++q) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) pk[t] = pack_bf16x2(S[32 * q + 2 * t], S[32 * q + 2 * t + 1]);
+        tmem_st16(lane_base + kT_S + 32 * hh + 16 * q, pk);
       }
-      fence_proxy_async_smem();
-      named_bar_sync(1, 128);
-      if (i == 0) mbar_arrive(s_ready);
+      tmem_st_wait();
     };
-    store_state_bf16();
-    // Every epilogue thread runs every iteration and every named barrier, even
-    // after an abort (waits then return at once), so no thread is stranded.
-    auto wait = [&](uint64_t *bar, uint32_t parity) {
-      if (!abort_flag) mbar_wait(bar, parity, ctrl, &abort_flag);
-    };
+    store_state();
+    tc_fence_before();
+    named_bar_sync(kBarChain, 256);
+    if (leader && nch > 0 && !*abort_flag) {
+      issue_u(0);
+      issue_xz(0);
+    }
     for (int c = 0; c < nch; ++c) {
-      const int st = c & 1;
-      uint8_t *sb = sm + st * kStageBytes;
-      wait(full + st, (c >> 1) & 1);
-      const ChunkInfo ci = table[c0 + c];
-      const float *G = reinterpret_cast<const float *>(sb + kS_G);
-      const float glast = G[kC - 1];
+      const int gs = c & 3;
+      const float *D = reinterpret_cast<const float *>(sm + kS_GAM + gs * 512) + 64;
+      GDN_TRACE_POINT(tr && leader, 0, c, 3);
+      wait(gfull + gs, (c >> 2) & 1);
+      GDN_TRACE_POINT(tr && leader, 0, c, 4);
       wait(x_full, c & 1);
+      GDN_TRACE_POINT(tr && leader, 0, c, 5);
       tc_fence_after();
-      // V_new^T row i = U^T row i - (S W^T) row i
-      {
-        uint32_t x0[32], x1[32];
-        tmem_ld32(lane_base + kT_X, x0);
-        tmem_ld32(lane_base + kT_X + 32, x1);
+      // V_new^T[i][s] = X[i][s] for s in [32 hh, 32 hh + 32): bf16 V_new^T and
+      // V_new^T diag(D) go back to TMEM as the A operands of dS and Y.
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        uint32_t x[16], a1[8], a2[8];
+        tmem_ld16(lane_base + kT_X + 32 * hh + 16 * q, x);
+        tmem_ld_wait();
+        const float *Dq = D + 32 * hh + 16 * q;
+#pragma unroll
+        for (int e = 0; e < 16; e += 4) {
+          const float4 d4 = *reinterpret_cast<const float4 *>(Dq + e);
+          const float v0 = __uint_as_float(x[e]), v1 = __uint_as_float(x[e + 1]);
+          const float v2 = __uint_as_float(x[e + 2]), v3 = __uint_as_float(x[e + 3]);
+          a1[e >> 1] = pack_bf16x2(v0, v1);
+          a1[(e >> 1) + 1] = pack_bf16x2(v2, v3);
+          a2[e >> 1] = pack_bf16x2(v0 * d4.x, v1 * d4.y);
+          a2[(e >> 1) + 1] = pack_bf16x2(v2 * d4.z, v3 * d4.w);
+        }
+        tmem_st8(lane_base + kT_A1 + 16 * hh + 8 * q, a1);
+        tmem_st8(lane_base + kT_A2 + 16 * hh + 8 * q, a2);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      named_bar_sync(kBarChain, 256);
+      GDN_TRACE_POINT(tr && leader, 0, c, 6);
+      if (leader && !*abort_flag) {
+        const int st = c & 1;
+        const uint32_t sb32 = smem_u32(sm + st * kStageBytes);
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma_bf16_ts(tmem + kT_DS, tmem + kT_A2 + 8 * kk,
+                         make_sdesc(sb32 + kS_K + kk * 2048, kTile64x64, 1024), id_s, kk > 0);
+        tc_commit(s_full);
+        // Y is single-buffered: the output warps must have read Y of chunk c - 1.
+        if (c == 0 || mbar_wait(y_free, (c - 1) & 1, ctrl, abort_flag)) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tc_mma_bf16_ts(tmem + kT_Y, tmem + kT_A1 + 8 * kk,
+                           make_sdesc(sb32 + kS_P + kk * 32, 16, 1024), id_y, kk > 0);
+          tc_commit(y_full);
+          tc_commit(empty + st);          // stage free once every MMA reading it is done
+          if (c + 1 < nch) issue_u(c + 1);
+        }
+      }
+      // S <- gamma_last S + dS on columns [64 hh, 64 hh + 64)
+      const float gl = reinterpret_cast<const float *>(sm + kS_GAM + gs * 512)[kC - 1];
+      wait(s_full, c & 1);
+      GDN_TRACE_POINT(tr && leader, 0, c, 7);
+      tc_fence_after();
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+        uint32_t d[32];
+        tmem_ld32(lane_base + kT_DS + 64 * hh + 32 * b, d);
         tmem_ld_wait();
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const uint4 u4 = *reinterpret_cast<const uint4 *>(sb + kS_UT + sw128_offset(i, ch));
-          const __nv_bfloat162 *u2 = reinterpret_cast<const __nv_bfloat162 *>(&u4);
-          float vn[8], vd[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int s = ch * 8 + e;
-            const float u = (e & 1) ? __high2float(u2[e >> 1]) : __low2float(u2[e >> 1]);
-            const float xv = __uint_as_float(ch < 4 ? x0[s & 31] : x1[s & 31]);
-            vn[e] = u - xv;
-            vd[e] = vn[e] * expf(glast - G[s]);
-          }
-          *reinterpret_cast<uint4 *>(sm + kS_A1 + sw128_offset(i, ch)) =
-              make_uint4(pack_bf16x2(vn[0], vn[1]), pack_bf16x2(vn[2], vn[3]),
-                         pack_bf16x2(vn[4], vn[5]), pack_bf16x2(vn[6], vn[7]));
-          *reinterpret_cast<uint4 *>(sm + kS_A2 + sw128_offset(i, ch)) =
-              make_uint4(pack_bf16x2(vd[0], vd[1]), pack_bf16x2(vd[2], vd[3]),
-                         pack_bf16x2(vd[4], vd[5]), pack_bf16x2(vd[6], vd[7]));
-        }
+        for (int t = 0; t < 32; ++t) S[32 * b + t] = fmaf(gl, S[32 * b + t], __uint_as_float(d[t]));
       }
-      fence_proxy_async_smem();
+      store_state();
       tc_fence_before();
-      named_bar_sync(1, 128);
-      if (i == 0) mbar_arrive(vnew_ready);
-      // S <- gamma_last S + dS
-      wait(s_full, c & 1);
-      tc_fence_after();
-      {
-        const float gl = expf(glast);
-#pragma unroll
-        for (int jb = 0; jb < 4; ++jb) {
-          uint32_t d[32];
-          tmem_ld32(lane_base + kT_DS + jb * 32, d);
-          tmem_ld_wait();
-#pragma unroll
-          for (int t = 0; t < 32; ++t) S[jb * 32 + t] = gl * S[jb * 32 + t] + __uint_as_float(d[t]);
-        }
+      named_bar_sync(kBarChain, 256);
+      GDN_TRACE_POINT(tr && leader, 0, c, 8);
+      if (leader) {
+        mbar_arrive(gempty + gs);
+        if (c + 1 < nch && !*abort_flag) issue_xz(c + 1);
       }
-      tc_fence_before();
-      store_state_bf16();
-      // O rows of this chunk: o[c'][i] = gamma_c' (S Q^T)[i][c'] + Y[i][c']
-      wait(y_full, c & 1);
-      tc_fence_after();
-      {
-        uint32_t z[32], y[32];
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          tmem_ld32(lane_base + kT_Z + (c & 1) * 64 + half * 32, z);
-          tmem_ld32(lane_base + kT_Y + (c & 1) * 64 + half * 32, y);
-          tmem_ld_wait();
-#pragma unroll
-          for (int t = 0; t < 32; ++t) {
-            const int cc = half * 32 + t;
-            if (cc < ci.len) {
-              const float val = expf(G[cc]) * __uint_as_float(z[t]) + __uint_as_float(y[t]);
-              o[(size_t(ci.row0 + cc) * H + h) * kD + i] = __float2bfloat16_rn(val);
-            }
-          }
-        }
-      }
-      tc_fence_before();
-      named_bar_sync(1, 128);
-      if (i == 0) mbar_arrive(empty + st);
     }
-    if (sN && !abort_flag) {
+    if (leader) {
+      // Every MMA issued above has completed once this fires.
+      tc_commit(drain);
+      mbar_wait(drain, 0, ctrl, abort_flag);
+    }
+    if (sN && !*abort_flag) {
       float *dst = sN + (size_t(n) * H + h) * kD * kD;
 #pragma unroll
-      for (int j = 0; j < kD; ++j) dst[size_t(j) * kD + i] = S[j];
+      for (int t = 0; t < 64; ++t) dst[size_t(64 * hh + t) * kD + i] = S[t];
     }
+  } else if (warp >= 12) {
+    // ------------------------------------------------------------ output
+    // O[c'][i] = gamma_c' Z[i][c'] + Y[i][c'] (Z, Y are O^T in TMEM). Each warp
+    // reads its 32 lanes in 16-lane x 16-column fragments (the mma accumulator
+    // layout) and writes them transposed into the swizzled staging tile with
+    // stmatrix, 16 bytes per row; a TMA store (whole chunks) or a 16-byte copy
+    // loop (a sequence's last, partial chunk) moves the tile to o.
+    const int q = warp & 3, ot = tid - 384;           // output thread 0..127
+    const uint32_t lane_q = tmem + (uint32_t(q * 32) << 16);
+    const bool leader = (warp == 12 && lane == 0);
+    const uint32_t ost = smem_u32(sm + kS_OST);
+    const int fc = 2 * (lane & 3);                     // fragment column pair
+    const int mj = lane & 7, mm = lane >> 3;           // stmatrix: row j of matrix m
+    for (int c = 0; c < nch; ++c) {
+      const int gs = c & 3;
+      const float *gam = reinterpret_cast<const float *>(sm + kS_GAM + gs * 512);
+      const ChunkInfo ci = table[c0 + c];
+      const bool whole = ci.len == kC;
+      wait(gfull + gs, (c >> 2) & 1);
+      if (leader) tma_store_wait_read();     // staging free again
+      named_bar_sync(kBarOut, 128);
+      wait(y_full, c & 1);
+      GDN_TRACE_POINT(tr && leader, 0, c, 9);
+      tc_fence_after();
+      const uint32_t zcol = kT_Z + 64 * (c & 1);
+#pragma unroll
+      for (int lb = 0; lb < 32; lb += 16) {
+#pragma unroll
+        for (int cb = 0; cb < 64; cb += 16) {
+          uint32_t z[8], y[8];
+          tmem_ld16x256_x2(lane_q + (uint32_t(lb) << 16) + zcol + cb, z);
+          tmem_ld16x256_x2(lane_q + (uint32_t(lb) << 16) + kT_Y + cb, y);
+          tmem_ld_wait();
+          const float2 g0 = *reinterpret_cast<const float2 *>(gam + cb + fc);
+          const float2 g1 = *reinterpret_cast<const float2 *>(gam + cb + 8 + fc);
+          uint32_t w[4];
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const float2 gg = (m < 2) ? g0 : g1;
+            const int k = 2 * m;
+            w[m] = pack_bf16x2(fmaf(gg.x, __uint_as_float(z[k]), __uint_as_float(y[k])),
+                               fmaf(gg.y, __uint_as_float(z[k + 1]), __uint_as_float(y[k + 1])));
+          }
+          // matrices: 0 = (lanes +0..7, cols +0..7), 1 = (lanes +8..15, cols +0..7),
+          //           2 = (lanes +0..7, cols +8..15), 3 = (lanes +8..15, cols +8..15)
+          const int i0 = q * 32 + lb + 8 * (mm & 1);    // first d_v index of my matrix
+          const int crow = cb + 8 * (mm >> 1) + mj;     // token row this thread addresses
+          const uint32_t addr =
+              ost + (i0 >> 6) * kTile64x64 + sw128_offset(crow, (i0 & 63) >> 3);
+          stmatrix_x4_trans(addr, w[0], w[1], w[2], w[3]);
+        }
+      }
+      tc_fence_before();
+      fence_proxy_async_smem();
+      named_bar_sync(kBarOut, 128);
+      GDN_TRACE_POINT(tr && leader, 0, c, 11);
+      if (leader) {
+        mbar_arrive(z_free + (c & 1));
+        mbar_arrive(y_free);
+        mbar_arrive(gempty + gs);
+        if (whole && !*abort_flag) {
+          tma_store_3d(&tm_o, sm + kS_OST, 0, h, ci.row0);
+          tma_store_3d(&tm_o, sm + kS_OST + kTile64x64, 64, h, ci.row0);
+          tma_store_commit();
+        }
+        GDN_TRACE_POINT(tr, 0, c, 10);
+      }
+      if (!whole && !*abort_flag) {
+        // rows [0, len) of the tile, 16 bytes at a time
+        for (int e = ot; e < ci.len * 16; e += 128) {
+          const int row = e >> 4, k = e & 15;
+          const uint4 v = *reinterpret_cast<const uint4 *>(
+              sm + kS_OST + (k >> 3) * kTile64x64 + sw128_offset(row, k & 7));
+          *reinterpret_cast<uint4 *>(o + (size_t(ci.row0 + row) * H + h) * kD + 8 * k) = v;
+        }
+      }
+    }
+    if (leader) tma_store_wait_all();
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 2) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -658,16 +828,16 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
   const long long rows = (long long)B * T;
   const long long units = (long long)L.max_chunks * H;
   if (T > 0 && L.max_chunks > 0) {
-    CUtensorMap mq, mk, mv, mwt, mut, mpm, mgm;
+    CUtensorMap mq, mk, mv, mo, mwt, mtb, mpm, mgm;
     if (!map_tokens(&mq, q, rows, H) || !map_tokens(&mk, k, rows, H) ||
-        !map_tokens(&mv, v, rows, H) ||
+        !map_tokens(&mv, v, rows, H) || !map_tokens(&mo, o, rows, H) ||
         !map_2d(&mwt, base + L.wt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, units * kD, 64, kD,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !map_2d(&mut, base + L.ut, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, units * kD, 64, kD,
+        !map_2d(&mtb, base + L.tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, units * kC, 64, kC,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
         !map_2d(&mpm, base + L.pm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, units * kC, 64, kC,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !map_2d(&mgm, base + L.gam, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, units, 64, 1,
+        !map_2d(&mgm, base + L.gam, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, units, 128, 1,
                 CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(gdn_prep_kernel,
@@ -675,8 +845,7 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     if (e != cudaSuccess) return e;
     prof_record(g_profile.prep, s);
     gdn_prep_kernel<<<dim3(L.max_chunks, H), kPrepThreads, kPrepSmem, s>>>(
-        mq, mk, mv, mwt, mut, mpm, g, beta, reinterpret_cast<float *>(base + L.gam), H, ctrl,
-        table);
+        mq, mk, mwt, mtb, mpm, g, beta, reinterpret_cast<float *>(base + L.gam), H, ctrl, table);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(gdn_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -684,8 +853,8 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     if (e != cudaSuccess) return e;
     prof_record(g_profile.scan, s);
     gdn_scan_kernel<<<dim3(N, H), kScanThreads, kScanSmem, s>>>(
-        mq, mk, mwt, mut, mpm, mgm, s0, sN, static_cast<__nv_bfloat16 *>(o), H, ctrl, table,
-        seq_first);
+        mq, mk, mv, mwt, mtb, mpm, mgm, mo, s0, sN, static_cast<__nv_bfloat16 *>(o), H, ctrl,
+        table, seq_first);
     return cudaGetLastError();
   }
   // No tokens: the final state is the initial state.
@@ -700,3 +869,12 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
 }
 
 }  // namespace gdn
+
+#ifdef GDN_TRACE
+// Trace builds only: copy the phase timestamps to `host` (2*64*16 u64).
+extern "C" int gdn_trace_fetch(unsigned long long *host) {
+  return cudaMemcpyFromSymbol(host, gdn::g_gdn_trace, sizeof(gdn::g_gdn_trace)) == cudaSuccess
+             ? 0
+             : -1;
+}
+#endif

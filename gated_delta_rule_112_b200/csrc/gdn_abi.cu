@@ -134,6 +134,7 @@ int gdn_get_status(void *workspace, void *stream) {
       return GDN_ERR_CUDA;
   }
   if (err & kErrTimeout) return GDN_ERR_DEVICE_TIMEOUT;
+  if (err & kErrLayout) return GDN_ERR_CUDA;
   if (err & kErrBadSeqlens) return GDN_ERR_INVALID_ARG;
   return GDN_OK;
 }

@@ -4,13 +4,14 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
-#include "../../include/gdn.h"
+#include "gdn.h"  // public C ABI (include/, on the -I path)
 
 namespace gdn {
 
 // Device error bits (stored in the first word of the workspace).
 constexpr uint32_t kErrBadSeqlens = 1u;
 constexpr uint32_t kErrTimeout = 2u;
+constexpr uint32_t kErrLayout = 4u;   // shared-memory window not 1024-byte aligned
 
 // One chunk of one sequence (shared by all heads).
 struct ChunkInfo {
@@ -26,11 +27,11 @@ struct ChunkInfo {
 //   seq_first      int32[N + 1]  global index of each sequence's first chunk
 //   tensor-core path only, per (chunk, head) unit u = chunk * H + h:
 //   wt             bf16 [units][d_k = 128][64]   W^T of the chunk
-//   ut             bf16 [units][d_v = 128][64]   U^T of the chunk
+//   tb             bf16 [units][64][64]          T diag(beta) of the chunk (UT transform)
 //   pm             bf16 [units][64][64]          (Q K^T) .* decay mask, diagonal included
-//   gam            fp32 [units][64]              cumulative log-gate Gamma
+//   gam            fp32 [units][128]             exp(Gamma_c) (64), then exp(Gamma_last - Gamma_s) (64)
 struct WsLayout {
-  size_t chunk_table, seq_first, wt, ut, pm, gam, total;
+  size_t chunk_table, seq_first, wt, tb, pm, gam, total;
   int max_chunks;
 };
 
@@ -53,9 +54,9 @@ inline WsLayout ws_layout(int B, int T, int H, int num_seqs, int chunk, bool tc)
   if (tc) {
     const size_t units = size_t(L.max_chunks) * H;
     L.wt = off;  off = align_up(off + units * 128 * 64 * 2, 1024);
-    L.ut = off;  off = align_up(off + units * 128 * 64 * 2, 1024);
+    L.tb = off;  off = align_up(off + units * 64 * 64 * 2, 1024);
     L.pm = off;  off = align_up(off + units * 64 * 64 * 2, 1024);
-    L.gam = off; off = align_up(off + units * 64 * 4, 1024);
+    L.gam = off; off = align_up(off + units * 128 * 4, 1024);
   }
   L.total = off;
   return L;
