@@ -119,6 +119,37 @@ int gdn_chunk_fwd_simt(const void *q, const void *k, const void *v, const float 
                        void *o, float *final_state, void *workspace, size_t workspace_bytes,
                        void *stream);
 
+/*
+ * gdn_chunk_fwd_noalloc -- gdn_chunk_fwd without a caller-supplied workspace.
+ *
+ * The paper has no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory: code running while a CUDA graph is
+ * being captured, plugins inside engines that own all device memory and
+ * offer no allocation hook, and latency-critical paths that cannot afford
+ * cudaMalloc's implicit synchronisation. It allocates nothing: its scratch is
+ * a fixed 64 MiB array built into the library, which every GPU that loads
+ * the library keeps reserved until the process exits.
+ *
+ *   Arguments, layouts and results are those of gdn_chunk_fwd, minus
+ *   workspace / workspace_bytes.
+ *   Returns GDN_ERR_WORKSPACE (and launches nothing) when these sizes need
+ *   more than 64 MiB of scratch, i.e. gdn_chunk_fwd_workspace_size(...) >
+ *   64 MiB -- roughly 2,000 (chunk, head) pairs on the tensor-core path.
+ *   The first call on a device looks up the array's device address (once per
+ *   device, thread-safe); make that first call before any stream capture.
+ *   All calls on a device share the array and it keeps the last call's
+ *   contents, so calls that overlap on the GPU (different streams, no
+ *   ordering between them) race and produce undefined results; serialise
+ *   them. Device-side errors (bad cu_seqlens contents, an expired bounded
+ *   wait) are recorded only in that internal scratch and are not reported by
+ *   gdn_get_status; check cu_seqlens on the host when using this variant.
+ */
+int gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const float *g,
+                          const float *beta, const float *initial_state,
+                          const int32_t *cu_seqlens, int B, int T, int H, int d_k, int d_v,
+                          int num_seqs, int chunk, int dtype, void *o, float *final_state,
+                          void *stream);
+
 /* Which implementation gdn_chunk_fwd would run for these sizes
  * (GDN_PATH_TCGEN05 or GDN_PATH_SIMT), or a negative value if unsupported. */
 int gdn_chunk_fwd_path(int d_k, int d_v, int chunk, int dtype);
