@@ -16,13 +16,17 @@
 // Two kernels:
 //   gdn_prep_kernel  one CTA per (chunk, head), fully parallel: everything that
 //                    depends only on the chunk's own K, Q, g, beta -- Gamma, A,
-//                    P = (Q K^T) .* M, T by blocked forward substitution, and
-//                    W^T = K^T (T diag(beta gamma))^T on tcgen05. Writes W^T,
+//                    P = (Q K^T) .* M, T by blocked forward substitution, and on
+//                    tcgen05 W = T diag(beta gamma) K and (D K)^T with
+//                    D = diag(exp(Gamma_last - Gamma)). Writes -W, (D K)^T,
 //                    T diag(beta), P (bf16) and the decay factors (fp32).
 //   gdn_scan_kernel  one CTA per (sequence, head), sequential over chunks:
 //                    U^T = V^T (T diag(beta))^T and the state-dependent
 //                    products on tcgen05, the fp32 state in registers of the
-//                    epilogue warps, and O.
+//                    epilogue warps, and O. Products that share an A operand
+//                    are issued as one wide MMA (N = 128 or 192): a tcgen05.mma
+//                    costs about the same whatever its N, so fewer, wider
+//                    instructions shorten the sequential chain.
 //
 // All products are worked in the "transposed frame" where the 128-wide head
 // dimension is the MMA M dimension, so every tcgen05.mma is M = 128 and each
@@ -53,11 +57,13 @@ constexpr uint32_t kTile128x64 = 128 * 128;   // 128 rows x 128 B = 16 KB
 constexpr int kLd = 68;                              // fp32 row stride of A and T (16-byte rows)
 constexpr uint32_t kP_KQ = 0;                        // 2 blocks x [K rows 0-63 | Q rows 64-127] = 32 KB
 constexpr uint32_t kP_PST = kP_KQ + kTile64x64;      // P staging, over Q of block 0 (dead after G)
-constexpr uint32_t kP_WST = kP_KQ + kTile128x64;     // W^T staging, over block 1 (dead after W)
+constexpr uint32_t kP_WST = kP_KQ;                   // -W staging [64 c][128 d] (2 blocks), over K/Q
+constexpr uint32_t kP_KST = kP_KQ + kTile128x64;     // (D K)^T staging [128 d][64 s], over K/Q
 constexpr uint32_t kP_AS = kP_KQ + 2 * kTile128x64;  // A, fp32 [64][68]; after the solve it
 constexpr uint32_t kP_TB = kP_AS;                    //   holds T diag(beta)       (bf16 64x64)
 constexpr uint32_t kP_TBG = kP_AS + kTile64x64;      //   and   T diag(beta gamma) (bf16 64x64)
-constexpr uint32_t kP_TS = kP_AS + 64 * kLd * 4;     // T, fp32 [64][68]
+constexpr uint32_t kP_TS = kP_AS + 64 * kLd * 4;     // T, fp32 [64][68]; then diag(D) (bf16 64x64)
+constexpr uint32_t kP_DIAG = kP_TS;
 constexpr uint32_t kP_XS = kP_TS + 64 * kLd * 4;     // solve scratch, fp32 [32][32]
 constexpr uint32_t kP_VEC = kP_XS + 1024 * 4;        // Gamma, beta, gamma: 3 x 64 fp32
 constexpr uint32_t kP_BAR = kP_VEC + 3 * 64 * 4;     // 2 mbarriers + tmem address
@@ -65,7 +71,8 @@ constexpr uint32_t kP_END = kP_BAR + 64;
 constexpr uint32_t kPrepSmem = kP_END + 1024;        // + alignment slack
 constexpr int kPrepThreads = 256;
 static_assert(2 * kTile64x64 <= 64 * kLd * 4, "T tiles must fit in the A area");
-static_assert(kP_AS % 1024 == 0 && kP_PST % 1024 == 0 && kP_WST % 1024 == 0,
+static_assert(kP_AS % 1024 == 0 && kP_PST % 1024 == 0 && kP_KST % 1024 == 0 &&
+                  kP_DIAG % 1024 == 0,
               "swizzled tiles need 1024-byte alignment");
 
 // T = (I + A)^-1 for the strictly lower-triangular 64 x 64 A (fp32 shared
@@ -166,8 +173,9 @@ __device__ void solve_unit_lower_64(const float *__restrict__ As, float *__restr
 // column half = warp / 4.
 __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-    const __grid_constant__ CUtensorMap tm_wt, const __grid_constant__ CUtensorMap tm_tb,
-    const __grid_constant__ CUtensorMap tm_pm, const float *__restrict__ g,
+    const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_kt,
+    const __grid_constant__ CUtensorMap tm_tb, const __grid_constant__ CUtensorMap tm_pm,
+    const float *__restrict__ g,
     const float *__restrict__ beta, float *__restrict__ gam_out, int H,
     uint32_t *__restrict__ ctrl, const ChunkInfo *__restrict__ table) {
   extern __shared__ uint8_t smem_raw[];
@@ -343,6 +351,23 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
                      pack_bf16x2(fg[4], fg[5]), pack_bf16x2(fg[6], fg[7]));
     }
   }
+  __syncthreads();
+  // T is dead: its area now holds diag(D), D_s = exp(Gamma_last - Gamma_s), as a
+  // bf16 K-major tile, the B operand that turns K^T into (D K)^T.
+  {
+    const int r = tid >> 2, q4 = tid & 3;
+    const float dr = expf(Gm[kC - 1] - Gm[r]);
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      const int ch = q4 * 2 + cc;
+      float f[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) f[e] = (ch * 8 + e == r) ? dr : 0.f;
+      *reinterpret_cast<uint4 *>(sm + kP_DIAG + sw128_offset(r, ch)) =
+          make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                     pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+    }
+  }
   fence_proxy_async_smem();
   __syncthreads();
   GDN_TRACE_POINT(tr, 1, chunk, 5);
@@ -350,32 +375,65 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
     tma_store_2d(&tm_tb, sm + kP_TB, 0, unit * kC);
     tma_store_commit();
     tc_fence_after();
-    // W^T = K^T (T diag(beta gamma))^T : M = 128 (d_k), N = 64, K = 64 (tokens) -> cols [64, 128)
+    // W^T    = K^T (T diag(beta gamma))^T : M = 128 (d_k), N = 64, K = 64 -> cols [64, 128)
+    // (DK)^T = K^T diag(D)                : M = 128 (d_k), N = 64, K = 64 -> cols [0, 64)
     const uint32_t idesc = make_idesc_bf16(128, 64, 1, 0);
     const uint32_t kq = smem_u32(sm + kP_KQ), tbg = smem_u32(sm + kP_TBG);
+    const uint32_t dg = smem_u32(sm + kP_DIAG);
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
+    for (int kk = 0; kk < 4; ++kk)
       tc_mma_bf16(tmem + 64, make_sdesc(kq + kk * 2048, kTile128x64, 1024),
                   make_sdesc(tbg + kk * 32, 16, 1024), idesc, kk > 0);
-    }
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      tc_mma_bf16(tmem, make_sdesc(kq + kk * 2048, kTile128x64, 1024),
+                  make_sdesc(dg + kk * 32, 16, 1024), idesc, kk > 0);
     tc_commit(bar_mma);
   }
   mbar_wait(bar_mma, 1, ctrl, &abort_flag);
   GDN_TRACE_POINT(tr, 1, chunk, 6);
+  if (tid == 0) tma_store_wait_read();   // the P staging lies under the W staging
   tc_fence_after();
+  __syncthreads();
   if (!abort_flag) {
-    // Row m of W^T, columns [32 hc, 32 hc + 32) -> bf16 staging over K/Q block 1.
-    uint32_t r0[32];
-    tmem_ld32(lane_base + 64 + 32 * hc, r0);
-    tmem_ld_wait();
+    if (hc == 0) {
+      // -W, K-major [64 c][128 d]: read W^T (lanes = d, columns = c) as
+      // mma-accumulator fragments and store them transposed with stmatrix.
+      const int q = warp & 3, mj = lane & 7, mm = lane >> 3;
+      const uint32_t wst = smem_u32(sm + kP_WST);
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-      const int b = cc * 8;
-      *reinterpret_cast<uint4 *>(sm + kP_WST + sw128_offset(m, 4 * hc + cc)) = make_uint4(
-          pack_bf16x2(__uint_as_float(r0[b + 0]), __uint_as_float(r0[b + 1])),
-          pack_bf16x2(__uint_as_float(r0[b + 2]), __uint_as_float(r0[b + 3])),
-          pack_bf16x2(__uint_as_float(r0[b + 4]), __uint_as_float(r0[b + 5])),
-          pack_bf16x2(__uint_as_float(r0[b + 6]), __uint_as_float(r0[b + 7])));
+      for (int lb = 0; lb < 32; lb += 16) {
+#pragma unroll
+        for (int cb = 0; cb < 64; cb += 16) {
+          uint32_t w8[8];
+          tmem_ld16x256_x2(lane_base + (uint32_t(lb) << 16) + 64 + cb, w8);
+          tmem_ld_wait();
+          uint32_t w[4];
+#pragma unroll
+          for (int mq = 0; mq < 4; ++mq)
+            w[mq] = pack_bf16x2(-__uint_as_float(w8[2 * mq]), -__uint_as_float(w8[2 * mq + 1]));
+          const int d0 = q * 32 + lb + 8 * (mm & 1);   // first d index of my matrix
+          const int crow = cb + 8 * (mm >> 1) + mj;     // chunk row this thread addresses
+          stmatrix_x4_trans(wst + (d0 >> 6) * kTile64x64 + sw128_offset(crow, (d0 & 63) >> 3),
+                            w[0], w[1], w[2], w[3]);
+        }
+      }
+    } else {
+      // (D K)^T row m (= d) -> [128 d][64 s] staging.
+      uint32_t r0[32], r1[32];
+      tmem_ld32(lane_base, r0);
+      tmem_ld32(lane_base + 32, r1);
+      tmem_ld_wait();
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        const uint32_t *src = ch < 4 ? r0 : r1;
+        const int b = (ch & 3) * 8;
+        *reinterpret_cast<uint4 *>(sm + kP_KST + sw128_offset(m, ch)) = make_uint4(
+            pack_bf16x2(__uint_as_float(src[b + 0]), __uint_as_float(src[b + 1])),
+            pack_bf16x2(__uint_as_float(src[b + 2]), __uint_as_float(src[b + 3])),
+            pack_bf16x2(__uint_as_float(src[b + 4]), __uint_as_float(src[b + 5])),
+            pack_bf16x2(__uint_as_float(src[b + 6]), __uint_as_float(src[b + 7])));
+      }
     }
   }
   fence_proxy_async_smem();
@@ -383,7 +441,9 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
   __syncthreads();
   if (tid == 0) {
     if (!abort_flag) {
-      tma_store_2d(&tm_wt, sm + kP_WST, 0, unit * kD);
+      tma_store_2d(&tm_w, sm + kP_WST, 0, unit * kC);
+      tma_store_2d(&tm_w, sm + kP_WST + kTile64x64, 64, unit * kC);
+      tma_store_2d(&tm_kt, sm + kP_KST, 0, unit * kD);
       tma_store_commit();
     }
     GDN_TRACE_POINT(tr, 1, chunk, 7);
@@ -398,38 +458,37 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
 }
 
 // ===================================================================== scan
-// One stage (one chunk of one head): W^T, Q, K, V, T diag(beta), P. The
-// per-chunk decay factors (gamma[64], D[64]) travel in a separate 4-slot ring
-// so the output warps, which need only gamma, never hold a stage.
-constexpr uint32_t kS_WT = 0;                        // [128 d_k][64 c]   MN-major B of S W^T
-constexpr uint32_t kS_Q = kS_WT + kTile128x64;       // 2 x [64 c][64 d]  K-major B of S Q^T
-constexpr uint32_t kS_K = kS_Q + 2 * kTile64x64;     // 2 x [64 s][64 d]  MN-major B of dS
-constexpr uint32_t kS_V = kS_K + 2 * kTile64x64;     // 2 x [64 s][64 d]  MN-major A of U^T
-constexpr uint32_t kS_TB = kS_V + 2 * kTile64x64;    // [64 r][64 s]      K-major B of U^T
-constexpr uint32_t kS_P = kS_TB + kTile64x64;        // [64 c][64 s]      K-major B of Y
-constexpr uint32_t kStageBytes = kS_P + kTile64x64;  // 80 KB, multiple of 1024
+// One stage (one chunk of one head), as the B operands of three wide MMAs:
+//   BXZ  2 x [ -W rows 0-63 | Q rows 64-127 ]  (128 rows, K = d_k in two blocks)
+//   BU   [ T diag(beta) rows 0-63 | zeros ]    (128 rows, K = 64 tokens)
+//   BSY  [ (D K)^T rows 0-127 | P rows 128-191 ] (192 rows, K = 64 tokens)
+// plus V (the MN-major A operand of U^T). The zero half of BU is written
+// once; TMA never touches it. The per-chunk decay factors (gamma[64], D[64])
+// travel in a separate 4-slot ring so the output warps never hold a stage.
+constexpr uint32_t kS_BXZ = 0;                        // 32 KB
+constexpr uint32_t kS_V = kS_BXZ + 2 * kTile128x64;   // 16 KB, 2 x [64 s][64 d]
+constexpr uint32_t kS_BU = kS_V + 2 * kTile64x64;     // 16 KB
+constexpr uint32_t kS_BSY = kS_BU + kTile128x64;      // 24 KB
+constexpr uint32_t kStageBytes = kS_BSY + kTile128x64 + kTile64x64;   // 88 KB
 constexpr int kStages = 2, kGamSlots = 4;
 constexpr uint32_t kS_OST = kStages * kStageBytes;            // O staging, 2 x [64 c][64 d]
 constexpr uint32_t kS_GAM = kS_OST + 2 * kTile64x64;          // kGamSlots x 128 fp32
 constexpr uint32_t kS_BAR = kS_GAM + kGamSlots * 512;         // mbarriers, tmem slot, flags
 constexpr uint32_t kS_END = kS_BAR + 256;
 constexpr uint32_t kScanSmem = kS_END;   // the dynamic window starts 1024-aligned (checked)
-constexpr uint32_t kStageTx = kStageBytes;
+constexpr uint32_t kStageTx = kStageBytes - kTile64x64;       // everything but the zero tile
 constexpr int kScanThreads = 512;
-// TMEM columns: fp32 accumulators, then the bf16 A operands of the MMAs.
-constexpr uint32_t kT_X = 0;      // U^T - S W^T = V_new^T   fp32 [128][64]
-constexpr uint32_t kT_Z = 64;     // S Q^T, two buffers      fp32 2 x [128][64]
-constexpr uint32_t kT_Y = 192;    // V_new^T P^T             fp32 [128][64]
-constexpr uint32_t kT_DS = 256;   // V_new^T D K             fp32 [128][128]
-constexpr uint32_t kT_S = 384;    // S                       bf16 [128][128] (64 columns)
-constexpr uint32_t kT_A1 = 448;   // V_new^T                 bf16 [128][64]  (32 columns)
-constexpr uint32_t kT_A2 = 480;   // V_new^T diag(D)         bf16 [128][64]  (32 columns)
+// TMEM columns (fp32 accumulators, then the bf16 A operands held in TMEM)
+constexpr uint32_t kT_XZ = 0;     // [X | Z]  = [U^T - S W^T | S Q^T]        fp32 [128][128]
+constexpr uint32_t kT_SY = 128;   // [dS | Y] = [V_new^T (DK) | V_new^T P^T] fp32 [128][192]
+constexpr uint32_t kT_S = 320;    // S        bf16 [128][128] (64 columns)
+constexpr uint32_t kT_A1 = 384;   // V_new^T  bf16 [128][64]  (32 columns)
 // Named barriers (0 is __syncthreads)
 constexpr uint32_t kBarChain = 1, kBarOut = 2;
 // Barrier slots in the kS_BAR area
 constexpr int kB_FULL = 0, kB_EMPTY = 2, kB_GFULL = 4, kB_GEMPTY = 8, kB_XFULL = 12,
-              kB_SFULL = 13, kB_YFULL = 14, kB_ZFREE = 15, kB_YFREE = 17, kB_DRAIN = 18,
-              kB_COUNT = 19;
+              kB_SFULL = 13, kB_YFULL = 14, kB_ZFREE = 15, kB_YFREE = 16, kB_DRAIN = 17,
+              kB_COUNT = 18;
 
 // Warp roles (16 warps):
 //   warp 0        TMA producer (one elected lane)
@@ -439,15 +498,16 @@ constexpr int kB_FULL = 0, kB_EMPTY = 2, kB_GFULL = 4, kB_GEMPTY = 8, kB_XFULL =
 //                 TMEM lane = row i of d_v; the fp32 S lives in its registers,
 //                 its bf16 copy (an MMA operand) in tensor memory.
 //                 Lane 0 of warp 4 also issues every tcgen05.mma.
-//   warps 12-15   output: O = diag(gamma) Q S^T + P V_new, staged for TMA stores
-// Chain per chunk: X = U^T - S W^T -> V_new -> dS = V_new^T diag(D) K ->
-// S = gamma_last S + dS. U^T = V^T (T diag(beta))^T is computed into X ahead
-// of time; Z = S Q^T and Y = V_new^T P^T run beside the chain. The A operands
-// of the state products live in tensor memory, so the tensor core reads only
-// the B tiles (and V) from shared memory.
+//   warps 12-15   output: O = diag(gamma) Z + Y, staged for TMA stores
+// Per chunk c the tensor core runs three wide products:
+//   U(c)   [X|Z]  = V^T [Tb | 0]^T            (4 MMAs, N = 128)  -- before S_c is known
+//   XZ(c)  [X|Z] += S [-W | Q]^T              (8 MMAs, N = 128)  -> X = V_new^T, Z = S Q^T
+//   SY(c)  [dS|Y] = V_new^T [(DK)^T | P]^T    (4 MMAs, N = 192)
+// and the chain is XZ -> V_new epilogue -> SY -> S epilogue -> XZ(c+1), with
+// U(c+1) running during the S epilogue.
 __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
-    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_wt,
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_v,
+    const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_kt,
     const __grid_constant__ CUtensorMap tm_tb, const __grid_constant__ CUtensorMap tm_pm,
     const __grid_constant__ CUtensorMap tm_gam, const __grid_constant__ CUtensorMap tm_o,
     const float *__restrict__ s0, float *__restrict__ sN, __nv_bfloat16 *__restrict__ o, int H,
@@ -477,9 +537,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
   if (tid == 0) {
     *abort_flag = 0;
     tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
-    tma_prefetch_desc(&tm_wt);
+    tma_prefetch_desc(&tm_w);
+    tma_prefetch_desc(&tm_kt);
     tma_prefetch_desc(&tm_tb);
     tma_prefetch_desc(&tm_pm);
     tma_prefetch_desc(&tm_gam);
@@ -488,6 +548,13 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
       mbar_init(bars + b, (b >= kB_GEMPTY && b < kB_GEMPTY + 4) ? 2 : 1);
     fence_mbar_init();
   }
+  // The zero half of BU in both stages.
+  for (int e = tid; e < kStages * (kTile64x64 / 16); e += kScanThreads) {
+    const int st = e / (kTile64x64 / 16), off = e % (kTile64x64 / 16);
+    *reinterpret_cast<uint4 *>(sm + st * kStageBytes + kS_BU + kTile64x64 + off * 16) =
+        make_uint4(0, 0, 0, 0);
+  }
+  fence_proxy_async_smem();
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
@@ -512,15 +579,15 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
       uint8_t *sb = sm + st * kStageBytes;
       GDN_TRACE_POINT(tr, 0, c, 0);
       mbar_arrive_expect_tx(full + st, kStageTx);
-      tma_load_2d(sb + kS_WT, &tm_wt, full + st, 0, unit * kD);
+      tma_load_2d(sb + kS_BXZ, &tm_w, full + st, 0, unit * kC);
+      tma_load_3d(sb + kS_BXZ + kTile64x64, &tm_q, full + st, 0, h, ci.row0);
+      tma_load_2d(sb + kS_BXZ + kTile128x64, &tm_w, full + st, 64, unit * kC);
+      tma_load_3d(sb + kS_BXZ + kTile128x64 + kTile64x64, &tm_q, full + st, 64, h, ci.row0);
       tma_load_3d(sb + kS_V, &tm_v, full + st, 0, h, ci.row0);
       tma_load_3d(sb + kS_V + kTile64x64, &tm_v, full + st, 64, h, ci.row0);
-      tma_load_2d(sb + kS_TB, &tm_tb, full + st, 0, unit * kC);
-      tma_load_3d(sb + kS_Q, &tm_q, full + st, 0, h, ci.row0);
-      tma_load_3d(sb + kS_Q + kTile64x64, &tm_q, full + st, 64, h, ci.row0);
-      tma_load_3d(sb + kS_K, &tm_k, full + st, 0, h, ci.row0);
-      tma_load_3d(sb + kS_K + kTile64x64, &tm_k, full + st, 64, h, ci.row0);
-      tma_load_2d(sb + kS_P, &tm_pm, full + st, 0, unit * kC);
+      tma_load_2d(sb + kS_BU, &tm_tb, full + st, 0, unit * kC);
+      tma_load_2d(sb + kS_BSY, &tm_kt, full + st, 0, unit * kD);
+      tma_load_2d(sb + kS_BSY + kTile128x64, &tm_pm, full + st, 0, unit * kC);
       if (c >= 4 && !mbar_wait(gempty + gs, ((c >> 2) - 1) & 1, ctrl, abort_flag)) break;
       mbar_arrive_expect_tx(gfull + gs, 512);
       tma_load_2d(sm + kS_GAM + gs * 512, &tm_gam, gfull + gs, 0, unit);
@@ -531,25 +598,23 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     const int i = ((warp & 3) << 5) + lane;             // TMEM lane = row of d_v
     const uint32_t lane_base = tmem + (uint32_t((warp & 3) * 32) << 16);
     const bool leader = (warp == 4 && lane == 0);
-    const uint32_t id_u = make_idesc_bf16(128, 64, 1, 0);       // V^T Tb^T : A MN-major
-    const uint32_t id_x = make_idesc_bf16(128, 64, 0, 1, 1);    // -S W^T   : B MN-major, negated
-    const uint32_t id_z = make_idesc_bf16(128, 64, 0, 0);       // S Q^T    : B K-major
-    const uint32_t id_s = make_idesc_bf16(128, 128, 0, 1);      // A2 K     : B MN-major
-    const uint32_t id_y = make_idesc_bf16(128, 64, 0, 0);       // A1 P^T   : B K-major
-    // Leader only. U(c): X = V^T (T diag(beta))^T, once chunk c is loaded and
-    // the chain has read X of chunk c - 1.
+    const uint32_t id_u = make_idesc_bf16(128, 128, 1, 0);     // V^T [Tb|0]^T : A MN-major
+    const uint32_t id_xz = make_idesc_bf16(128, 128, 0, 0);    // S [-W|Q]^T
+    const uint32_t id_sy = make_idesc_bf16(128, 192, 0, 0);    // A1 [(DK)^T|P]^T
+    // Leader only. U(c) into [X|Z]: needs chunk c loaded and the output warps
+    // done reading Z of chunk c - 1 (one barrier phase per chunk).
     auto issue_u = [&](int c) {
       const int st = c & 1;
       const uint32_t sb = smem_u32(sm + st * kStageBytes);
+      if (c >= 1 && !mbar_wait(z_free, (c - 1) & 1, ctrl, abort_flag)) return;
       if (!mbar_wait(full + st, (c >> 1) & 1, ctrl, abort_flag)) return;
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        tc_mma_bf16(tmem + kT_X, make_sdesc(sb + kS_V + kk * 2048, kTile64x64, 1024),
-                    make_sdesc(sb + kS_TB + kk * 32, 16, 1024), id_u, kk > 0);
+        tc_mma_bf16(tmem + kT_XZ, make_sdesc(sb + kS_V + kk * 2048, kTile64x64, 1024),
+                    make_sdesc(sb + kS_BU + kk * 32, 16, 1024), id_u, kk > 0);
     };
-    // Leader only. X(c) -= S_c W_c^T and Z(c) = S_c Q_c^T, both reading the
-    // bf16 copy of S_c.
+    // Leader only. XZ(c) += S_c [-W|Q]^T, reading the bf16 copy of S_c.
     auto issue_xz = [&](int c) {
       const int st = c & 1;
       const uint32_t sb = smem_u32(sm + st * kStageBytes);
@@ -557,20 +622,11 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        tc_mma_bf16_ts(tmem + kT_X, tmem + kT_S + 8 * kk,
-                       make_sdesc(sb + kS_WT + kk * 2048, kTile64x64, 1024), id_x, 1);
+        tc_mma_bf16_ts(tmem + kT_XZ, tmem + kT_S + 8 * kk,
+                       make_sdesc(sb + kS_BXZ + (kk >> 2) * kTile128x64 + (kk & 3) * 32, 16,
+                                  1024),
+                       id_xz, 1);
       tc_commit(x_full);
-      // Z of chunk c uses buffer c & 1, last read by the output warps for
-      // chunk c - 2. One barrier per buffer, so no wait falls two phases behind.
-      if (c >= 2 && !mbar_wait(z_free + (c & 1), ((c >> 1) - 1) & 1, ctrl, abort_flag)) return;
-      GDN_TRACE_POINT(tr, 0, c, 2);
-      const uint32_t zcol = kT_Z + 64 * (c & 1);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint64_t b =
-            make_sdesc(sb + kS_Q + (kk >> 2) * kTile64x64 + (kk & 3) * 32, 16, 1024);
-        tc_mma_bf16_ts(tmem + zcol, tmem + kT_S + 8 * kk, b, id_z, kk > 0);
-      }
     };
     float S[64];                                        // S[i][64 hh + t], fp32 master
     {
@@ -598,33 +654,23 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     }
     for (int c = 0; c < nch; ++c) {
       const int gs = c & 3;
-      const float *D = reinterpret_cast<const float *>(sm + kS_GAM + gs * 512) + 64;
       GDN_TRACE_POINT(tr && leader, 0, c, 3);
       wait(gfull + gs, (c >> 2) & 1);
       GDN_TRACE_POINT(tr && leader, 0, c, 4);
       wait(x_full, c & 1);
       GDN_TRACE_POINT(tr && leader, 0, c, 5);
       tc_fence_after();
-      // V_new^T[i][s] = X[i][s] for s in [32 hh, 32 hh + 32): bf16 V_new^T and
-      // V_new^T diag(D) go back to TMEM as the A operands of dS and Y.
+      // V_new^T[i][s] = X[i][s] for s in [32 hh, 32 hh + 32): bf16 back to TMEM
+      // as the A operand of SY.
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
-        uint32_t x[16], a1[8], a2[8];
-        tmem_ld16(lane_base + kT_X + 32 * hh + 16 * q, x);
+        uint32_t x[16], a1[8];
+        tmem_ld16(lane_base + kT_XZ + 32 * hh + 16 * q, x);
         tmem_ld_wait();
-        const float *Dq = D + 32 * hh + 16 * q;
 #pragma unroll
-        for (int e = 0; e < 16; e += 4) {
-          const float4 d4 = *reinterpret_cast<const float4 *>(Dq + e);
-          const float v0 = __uint_as_float(x[e]), v1 = __uint_as_float(x[e + 1]);
-          const float v2 = __uint_as_float(x[e + 2]), v3 = __uint_as_float(x[e + 3]);
-          a1[e >> 1] = pack_bf16x2(v0, v1);
-          a1[(e >> 1) + 1] = pack_bf16x2(v2, v3);
-          a2[e >> 1] = pack_bf16x2(v0 * d4.x, v1 * d4.y);
-          a2[(e >> 1) + 1] = pack_bf16x2(v2 * d4.z, v3 * d4.w);
-        }
+        for (int e = 0; e < 8; ++e)
+          a1[e] = pack_bf16x2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1]));
         tmem_st8(lane_base + kT_A1 + 16 * hh + 8 * q, a1);
-        tmem_st8(lane_base + kT_A2 + 16 * hh + 8 * q, a2);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -633,18 +679,14 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
       if (leader && !*abort_flag) {
         const int st = c & 1;
         const uint32_t sb32 = smem_u32(sm + st * kStageBytes);
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          tc_mma_bf16_ts(tmem + kT_DS, tmem + kT_A2 + 8 * kk,
-                         make_sdesc(sb32 + kS_K + kk * 2048, kTile64x64, 1024), id_s, kk > 0);
-        tc_commit(s_full);
         // Y is single-buffered: the output warps must have read Y of chunk c - 1.
         if (c == 0 || mbar_wait(y_free, (c - 1) & 1, ctrl, abort_flag)) {
+          tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            tc_mma_bf16_ts(tmem + kT_Y, tmem + kT_A1 + 8 * kk,
-                           make_sdesc(sb32 + kS_P + kk * 32, 16, 1024), id_y, kk > 0);
+            tc_mma_bf16_ts(tmem + kT_SY, tmem + kT_A1 + 8 * kk,
+                           make_sdesc(sb32 + kS_BSY + kk * 32, 16, 1024), id_sy, kk > 0);
+          tc_commit(s_full);
           tc_commit(y_full);
           tc_commit(empty + st);          // stage free once every MMA reading it is done
           if (c + 1 < nch) issue_u(c + 1);
@@ -658,7 +700,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
 #pragma unroll
       for (int b = 0; b < 2; ++b) {
         uint32_t d[32];
-        tmem_ld32(lane_base + kT_DS + 64 * hh + 32 * b, d);
+        tmem_ld32(lane_base + kT_SY + 64 * hh + 32 * b, d);
         tmem_ld_wait();
 #pragma unroll
         for (int t = 0; t < 32; ++t) S[32 * b + t] = fmaf(gl, S[32 * b + t], __uint_as_float(d[t]));
@@ -685,8 +727,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
   } else if (warp >= 12) {
     // ------------------------------------------------------------ output
     // O[c'][i] = gamma_c' Z[i][c'] + Y[i][c'] (Z, Y are O^T in TMEM). Each warp
-    // reads its 32 lanes in 16-lane x 16-column fragments (the mma accumulator
-    // layout) and writes them transposed into the swizzled staging tile with
+    // reads its 32 lanes as mma-accumulator fragments (16 lanes x 8 columns),
+    // Z as soon as XZ is done (so U of the next chunk may overwrite it), Y
+    // after SY, and writes O transposed into the swizzled staging tile with
     // stmatrix, 16 bytes per row; a TMA store (whole chunks) or a 16-byte copy
     // loop (a sequence's last, partial chunk) moves the tile to o.
     const int q = warp & 3, ot = tid - 384;           // output thread 0..127
@@ -700,20 +743,28 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
       const float *gam = reinterpret_cast<const float *>(sm + kS_GAM + gs * 512);
       const ChunkInfo ci = table[c0 + c];
       const bool whole = ci.len == kC;
+      uint32_t z[2][32];
+      wait(x_full, c & 1);
+      tc_fence_after();
+      tmem_ld16x256_x8(lane_q + kT_XZ + 64, z[0]);
+      tmem_ld16x256_x8(lane_q + (16u << 16) + kT_XZ + 64, z[1]);
+      tmem_ld_wait();
+      tc_fence_before();
+      named_bar_sync(kBarOut, 128);
+      if (leader) mbar_arrive(z_free);
       wait(gfull + gs, (c >> 2) & 1);
       if (leader) tma_store_wait_read();     // staging free again
       named_bar_sync(kBarOut, 128);
       wait(y_full, c & 1);
       GDN_TRACE_POINT(tr && leader, 0, c, 9);
       tc_fence_after();
-      const uint32_t zcol = kT_Z + 64 * (c & 1);
 #pragma unroll
-      for (int lb = 0; lb < 32; lb += 16) {
+      for (int lb = 0; lb < 2; ++lb) {
 #pragma unroll
-        for (int cb = 0; cb < 64; cb += 16) {
-          uint32_t z[8], y[8];
-          tmem_ld16x256_x2(lane_q + (uint32_t(lb) << 16) + zcol + cb, z);
-          tmem_ld16x256_x2(lane_q + (uint32_t(lb) << 16) + kT_Y + cb, y);
+        for (int cbi = 0; cbi < 4; ++cbi) {
+          const int cb = 16 * cbi;
+          uint32_t y[8];
+          tmem_ld16x256_x2(lane_q + (uint32_t(16 * lb) << 16) + kT_SY + 128 + cb, y);
           tmem_ld_wait();
           const float2 g0 = *reinterpret_cast<const float2 *>(gam + cb + fc);
           const float2 g1 = *reinterpret_cast<const float2 *>(gam + cb + 8 + fc);
@@ -722,13 +773,14 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
           for (int m = 0; m < 4; ++m) {
             const float2 gg = (m < 2) ? g0 : g1;
             const int k = 2 * m;
-            w[m] = pack_bf16x2(fmaf(gg.x, __uint_as_float(z[k]), __uint_as_float(y[k])),
-                               fmaf(gg.y, __uint_as_float(z[k + 1]), __uint_as_float(y[k + 1])));
+            w[m] = pack_bf16x2(
+                fmaf(gg.x, __uint_as_float(z[lb][8 * cbi + k]), __uint_as_float(y[k])),
+                fmaf(gg.y, __uint_as_float(z[lb][8 * cbi + k + 1]), __uint_as_float(y[k + 1])));
           }
           // matrices: 0 = (lanes +0..7, cols +0..7), 1 = (lanes +8..15, cols +0..7),
           //           2 = (lanes +0..7, cols +8..15), 3 = (lanes +8..15, cols +8..15)
-          const int i0 = q * 32 + lb + 8 * (mm & 1);    // first d_v index of my matrix
-          const int crow = cb + 8 * (mm >> 1) + mj;     // token row this thread addresses
+          const int i0 = q * 32 + 16 * lb + 8 * (mm & 1);  // first d_v index of my matrix
+          const int crow = cb + 8 * (mm >> 1) + mj;        // token row this thread addresses
           const uint32_t addr =
               ost + (i0 >> 6) * kTile64x64 + sw128_offset(crow, (i0 & 63) >> 3);
           stmatrix_x4_trans(addr, w[0], w[1], w[2], w[3]);
@@ -739,7 +791,6 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
       named_bar_sync(kBarOut, 128);
       GDN_TRACE_POINT(tr && leader, 0, c, 11);
       if (leader) {
-        mbar_arrive(z_free + (c & 1));
         mbar_arrive(y_free);
         mbar_arrive(gempty + gs);
         if (whole && !*abort_flag) {
@@ -802,14 +853,14 @@ bool map_tokens(CUtensorMap *m, const void *base, long long rows, int H) {
          CUDA_SUCCESS;
 }
 
-// [rows, inner] 2-D map with box (inner, box_rows).
+// [rows, inner] 2-D map with box (box_inner, box_rows).
 bool map_2d(CUtensorMap *m, const void *base, CUtensorMapDataType t, int esize, long long rows,
-            int inner, int box_rows, CUtensorMapSwizzle sw) {
+            int inner, int box_inner, int box_rows, CUtensorMapSwizzle sw) {
   EncodeTiledFn enc = get_encoder();
   if (!enc) return false;
   cuuint64_t dims[2] = {cuuint64_t(inner), cuuint64_t(rows)};
   cuuint64_t strides[1] = {cuuint64_t(inner) * esize};
-  cuuint32_t box[2] = {cuuint32_t(inner), cuuint32_t(box_rows)};
+  cuuint32_t box[2] = {cuuint32_t(box_inner), cuuint32_t(box_rows)};
   cuuint32_t es[2] = {1, 1};
   return enc(m, t, 2, const_cast<void *>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -828,16 +879,18 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
   const long long rows = (long long)B * T;
   const long long units = (long long)L.max_chunks * H;
   if (T > 0 && L.max_chunks > 0) {
-    CUtensorMap mq, mk, mv, mo, mwt, mtb, mpm, mgm;
+    CUtensorMap mq, mk, mv, mo, mw, mkt, mtb, mpm, mgm;
     if (!map_tokens(&mq, q, rows, H) || !map_tokens(&mk, k, rows, H) ||
         !map_tokens(&mv, v, rows, H) || !map_tokens(&mo, o, rows, H) ||
-        !map_2d(&mwt, base + L.wt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, units * kD, 64, kD,
+        !map_2d(&mw, base + L.w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, units * kC, kD, 64, kC,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !map_2d(&mtb, base + L.tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, units * kC, 64, kC,
+        !map_2d(&mkt, base + L.kt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, units * kD, 64, 64, kD,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !map_2d(&mpm, base + L.pm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, units * kC, 64, kC,
+        !map_2d(&mtb, base + L.tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, units * kC, 64, 64, kC,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !map_2d(&mgm, base + L.gam, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, units, 128, 1,
+        !map_2d(&mpm, base + L.pm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, units * kC, 64, 64, kC,
+                CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map_2d(&mgm, base + L.gam, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, units, 128, 128, 1,
                 CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(gdn_prep_kernel,
@@ -845,7 +898,8 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     if (e != cudaSuccess) return e;
     prof_record(g_profile.prep, s);
     gdn_prep_kernel<<<dim3(L.max_chunks, H), kPrepThreads, kPrepSmem, s>>>(
-        mq, mk, mwt, mtb, mpm, g, beta, reinterpret_cast<float *>(base + L.gam), H, ctrl, table);
+        mq, mk, mw, mkt, mtb, mpm, g, beta, reinterpret_cast<float *>(base + L.gam), H, ctrl,
+        table);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(gdn_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -853,7 +907,7 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     if (e != cudaSuccess) return e;
     prof_record(g_profile.scan, s);
     gdn_scan_kernel<<<dim3(N, H), kScanThreads, kScanSmem, s>>>(
-        mq, mk, mv, mwt, mtb, mpm, mgm, mo, s0, sN, static_cast<__nv_bfloat16 *>(o), H, ctrl,
+        mq, mv, mw, mkt, mtb, mpm, mgm, mo, s0, sN, static_cast<__nv_bfloat16 *>(o), H, ctrl,
         table, seq_first);
     return cudaGetLastError();
   }

@@ -26,12 +26,13 @@ struct ChunkInfo {
 //   chunk table    ChunkInfo[max_chunks]
 //   seq_first      int32[N + 1]  global index of each sequence's first chunk
 //   tensor-core path only, per (chunk, head) unit u = chunk * H + h:
-//   wt             bf16 [units][d_k = 128][64]   W^T of the chunk
+//   w              bf16 [units][64][d_k = 128]   -W of the chunk (rows = tokens)
+//   kt             bf16 [units][d_k = 128][64]   (D K)^T, D = diag(exp(Gamma_last - Gamma))
 //   tb             bf16 [units][64][64]          T diag(beta) of the chunk (UT transform)
 //   pm             bf16 [units][64][64]          (Q K^T) .* decay mask, diagonal included
 //   gam            fp32 [units][128]             exp(Gamma_c) (64), then exp(Gamma_last - Gamma_s) (64)
 struct WsLayout {
-  size_t chunk_table, seq_first, wt, tb, pm, gam, total;
+  size_t chunk_table, seq_first, w, kt, tb, pm, gam, total;
   int max_chunks;
 };
 
@@ -53,7 +54,8 @@ inline WsLayout ws_layout(int B, int T, int H, int num_seqs, int chunk, bool tc)
   off = align_up(off + sizeof(int32_t) * size_t(N + 1), 1024);
   if (tc) {
     const size_t units = size_t(L.max_chunks) * H;
-    L.wt = off;  off = align_up(off + units * 128 * 64 * 2, 1024);
+    L.w = off;   off = align_up(off + units * 64 * 128 * 2, 1024);
+    L.kt = off;  off = align_up(off + units * 128 * 64 * 2, 1024);
     L.tb = off;  off = align_up(off + units * 64 * 64 * 2, 1024);
     L.pm = off;  off = align_up(off + units * 64 * 64 * 2, 1024);
     L.gam = off; off = align_up(off + units * 128 * 4, 1024);

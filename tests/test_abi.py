@@ -54,16 +54,16 @@ def test_path_selection(L):
 def test_workspace_size(L):
     ws = L.gdn_chunk_fwd_workspace_size
     tc = ws(4, 4096, 16, 128, 128, 0, 64, gdn.BF16)
-    # 4096 (chunk, head) units x (W^T 16 KB + T diag(beta) 8 KB + P 8 KB + 512 B
-    # of decay factors) plus bookkeeping
-    per_unit = 16384 + 8192 + 8192 + 512
+    # 4096 (chunk, head) units x (-W 16 KB + (D K)^T 16 KB + T diag(beta) 8 KB +
+    # P 8 KB + 512 B of decay factors) plus bookkeeping
+    per_unit = 16384 + 16384 + 8192 + 8192 + 512
     assert tc >= 4096 * per_unit
     assert tc < 4096 * per_unit + (1 << 20)
     simt = ws(1, 256, 2, 64, 64, 0, 64, gdn.F32)
     assert 0 < simt < (1 << 16)
     # varlen bound: (T + N (C-1)) / C chunks
     v = ws(1, 1000, 1, 128, 128, 10, 64, gdn.BF16)
-    assert v >= ((1000 + 10 * 63) // 64) * (16384 + 8192 + 8192 + 512)
+    assert v >= ((1000 + 10 * 63) // 64) * (16384 + 16384 + 8192 + 8192 + 512)
     assert ws(0, 10, 1, 128, 128, 0, 64, gdn.BF16) == 0
     assert ws(1, 10, 1, 128, 128, 0, 48, gdn.BF16) == 0
 
