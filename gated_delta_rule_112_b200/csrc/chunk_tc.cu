@@ -64,9 +64,10 @@ constexpr uint32_t kP_TB = kP_AS;                    //   holds T diag(beta)    
 constexpr uint32_t kP_TBG = kP_AS + kTile64x64;      //   and   T diag(beta gamma) (bf16 64x64)
 constexpr uint32_t kP_TS = kP_AS + 64 * kLd * 4;     // T, fp32 [64][68]; then diag(D) (bf16 64x64)
 constexpr uint32_t kP_DIAG = kP_TS;
-constexpr uint32_t kP_XS = kP_TS + 64 * kLd * 4;     // solve scratch, fp32 [32][32]
-constexpr uint32_t kP_VEC = kP_XS + 1024 * 4;        // Gamma, beta, gamma: 3 x 64 fp32
-constexpr uint32_t kP_BAR = kP_VEC + 3 * 64 * 4;     // 2 mbarriers + tmem address
+constexpr int kLy = 36;                              // fp32 row stride of the solve scratch
+constexpr uint32_t kP_XS = kP_TS + 64 * kLd * 4;     // solve scratch, fp32 [32][36]
+constexpr uint32_t kP_VEC = kP_XS + 32 * kLy * 4;    // Gamma, beta, gamma, Gamma log2(e): 4 x 64 fp32
+constexpr uint32_t kP_BAR = kP_VEC + 4 * 64 * 4;     // 2 mbarriers + tmem address
 constexpr uint32_t kP_END = kP_BAR + 64;
 constexpr uint32_t kPrepSmem = kP_END + 1024;        // + alignment slack
 constexpr int kPrepThreads = 256;
@@ -75,17 +76,31 @@ static_assert(kP_AS % 1024 == 0 && kP_PST % 1024 == 0 && kP_KST % 1024 == 0 &&
                   kP_DIAG % 1024 == 0,
               "swizzled tiles need 1024-byte alignment");
 
+// 2^x on the special-function unit (PTX ex2.approx, flush-to-zero).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float4 lds4(const float *p) {
+  return *reinterpret_cast<const float4 *>(p);
+}
+
 // T = (I + A)^-1 for the strictly lower-triangular 64 x 64 A (fp32 shared
 // memory, row stride kLd), by recursive 2 x 2 blocking: for a lower block
 // triangular [[L11, 0], [L21, L22]], the inverse is [[T11, 0], [-T22 L21 T11, T22]].
 //   step 0  the four 16 x 16 diagonal blocks, by column-wise forward
-//           substitution in registers (thread = one column of one block)
+//           substitution in registers (thread = one column of one block);
+//           their upper triangles are written as zeros
 //   step 1  the two 16 x 16 blocks T(1,0), T(3,2)        (two half-steps)
 //   step 2  the 32 x 32 block T([2,3],[0,1])             (two half-steps)
-// Every half-step is an independent small product over all 256 threads.
-// Entries above the diagonal of T are left unwritten and never read.
+// Each half-step is a small product over all 256 threads with float4 operand
+// loads; loop bounds skip the blocks of T above the diagonal, which are never
+// written, and are uniform within a warp.
 __device__ void solve_unit_lower_64(const float *__restrict__ As, float *__restrict__ Ts,
                                     float *__restrict__ Xs, int tid) {
+  const int warp = tid >> 5, lane = tid & 31;
   if (tid < 64) {
     const int base = (tid >> 4) * 16, jj = tid & 15;
     float x[16];
@@ -94,77 +109,97 @@ __device__ void solve_unit_lower_64(const float *__restrict__ As, float *__restr
 #pragma unroll
     for (int r = 1; r < 16; ++r) {
       const float *arow = As + (base + r) * kLd + base;
-      float a0 = 0.f, a1 = 0.f;
+      float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-      for (int m = 0; m < r; m += 2) {
-        a0 = fmaf(arow[m], x[m], a0);
-        if (m + 1 < r) a1 = fmaf(arow[m + 1], x[m + 1], a1);
+      for (int m4 = 0; m4 < r; m4 += 4) {
+        const float4 a = lds4(arow + m4);
+        acc0 = fmaf(a.x, x[m4], acc0);
+        if (m4 + 1 < r) acc1 = fmaf(a.y, x[m4 + 1], acc1);
+        if (m4 + 2 < r) acc0 = fmaf(a.z, x[m4 + 2], acc0);
+        if (m4 + 3 < r) acc1 = fmaf(a.w, x[m4 + 3], acc1);
       }
-      if (r > jj) x[r] = -(a0 + a1);
+      if (r > jj) x[r] = -(acc0 + acc1);
     }
 #pragma unroll
     for (int r = 0; r < 16; ++r) Ts[(base + r) * kLd + base + jj] = x[r];
   }
   __syncthreads();
-  {  // step 1a: Y_b = A(i, i-1) T(i-1, i-1) for i = 1, 3; thread: row r, 2 columns
-    const int b = tid >> 7, r = (tid >> 3) & 15, c = (tid & 7) * 2;
-    const int i0 = 16 * (2 * b + 1), j0 = i0 - 16;
-    const float *arow = As + (i0 + r) * kLd + j0;
+  // step 1: block b in {0, 1} is T(2b+1, 2b); thread = row r, columns c, c+1
+  const int b1 = tid >> 7, r1 = (tid >> 3) & 15, c1 = (tid & 7) * 2;
+  const int i1 = 16 * (2 * b1 + 1), j1 = i1 - 16;
+  {  // Y_b = A(i, i-1) T(i-1, i-1)
+    const float *arow = As + (i1 + r1) * kLd + j1;
     float y0 = 0.f, y1 = 0.f;
 #pragma unroll
-    for (int m = 0; m < 16; ++m) {
-      const float2 t = *reinterpret_cast<const float2 *>(Ts + (j0 + m) * kLd + j0 + c);
-      const float tx = (m >= c) ? t.x : 0.f, ty = (m >= c + 1) ? t.y : 0.f;
-      y0 = fmaf(arow[m], tx, y0);
-      y1 = fmaf(arow[m], ty, y1);
+    for (int m4 = 0; m4 < 16; m4 += 4) {
+      const float4 a = lds4(arow + m4);
+      const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 t = *reinterpret_cast<const float2 *>(Ts + (j1 + m4 + e) * kLd + j1 + c1);
+        y0 = fmaf(av[e], t.x, y0);
+        y1 = fmaf(av[e], t.y, y1);
+      }
     }
-    *reinterpret_cast<float2 *>(Xs + b * 256 + r * 16 + c) = make_float2(y0, y1);
+    *reinterpret_cast<float2 *>(Xs + b1 * 16 * kLy + r1 * kLy + c1) = make_float2(y0, y1);
   }
   __syncthreads();
-  {  // step 1b: T(i, i-1) = -T(i, i) Y_b
-    const int b = tid >> 7, r = (tid >> 3) & 15, c = (tid & 7) * 2;
-    const int i0 = 16 * (2 * b + 1), j0 = i0 - 16;
-    const float *trow = Ts + (i0 + r) * kLd + i0;
+  {  // T(i, i-1) = -T(i, i) Y_b
+    const float *trow = Ts + (i1 + r1) * kLd + i1;
     float y0 = 0.f, y1 = 0.f;
 #pragma unroll
-    for (int m = 0; m < 16; ++m) {
-      const float t = (m <= r) ? trow[m] : 0.f;
-      const float2 x = *reinterpret_cast<const float2 *>(Xs + b * 256 + m * 16 + c);
-      y0 = fmaf(t, x.x, y0);
-      y1 = fmaf(t, x.y, y1);
+    for (int m4 = 0; m4 < 16; m4 += 4) {
+      const float4 t = lds4(trow + m4);
+      const float tv[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 y = *reinterpret_cast<const float2 *>(Xs + b1 * 16 * kLy + (m4 + e) * kLy + c1);
+        y0 = fmaf(tv[e], y.x, y0);
+        y1 = fmaf(tv[e], y.y, y1);
+      }
     }
-    *reinterpret_cast<float2 *>(Ts + (i0 + r) * kLd + j0 + c) = make_float2(-y0, -y1);
+    *reinterpret_cast<float2 *>(Ts + (i1 + r1) * kLd + j1 + c1) = make_float2(-y0, -y1);
   }
   __syncthreads();
-  {  // step 2a: Y = A([32,64), [0,32)) T([0,32), [0,32)); thread: row r, 4 columns
-    const int r = tid >> 3, c = (tid & 7) * 4;
-    const float *arow = As + (32 + r) * kLd;
+  // step 2: thread = row 16 (warp & 1) + (lane & 15), columns c2 .. c2 + 3 with
+  // c2 = 8 (warp >> 1) + 4 (lane >> 4)
+  const int r2 = 16 * (warp & 1) + (lane & 15), c2 = 8 * (warp >> 1) + 4 * (lane >> 4);
+  {  // Y = A([32,64), [0,32)) T([0,32), [0,32)); T(0,1) is unwritten: columns
+     // c >= 16 take rows m >= 16 only
+    const int m0 = (warp >> 2) * 16;
+    const float *arow = As + (32 + r2) * kLd;
     float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+    for (int m4 = m0; m4 < 32; m4 += 4) {
+      const float4 a = lds4(arow + m4);
+      const float av[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-    for (int m = 0; m < 32; ++m) {
-      const float a = arow[m];
-      const float4 t = *reinterpret_cast<const float4 *>(Ts + m * kLd + c);
-      // T([0,32),[0,32)) is lower triangular; entries with column > row are garbage.
-      y.x = fmaf(a, (m >= c + 0) ? t.x : 0.f, y.x);
-      y.y = fmaf(a, (m >= c + 1) ? t.y : 0.f, y.y);
-      y.z = fmaf(a, (m >= c + 2) ? t.z : 0.f, y.z);
-      y.w = fmaf(a, (m >= c + 3) ? t.w : 0.f, y.w);
+      for (int e = 0; e < 4; ++e) {
+        const float4 t = lds4(Ts + (m4 + e) * kLd + c2);
+        y.x = fmaf(av[e], t.x, y.x); y.y = fmaf(av[e], t.y, y.y);
+        y.z = fmaf(av[e], t.z, y.z); y.w = fmaf(av[e], t.w, y.w);
+      }
     }
-    *reinterpret_cast<float4 *>(Xs + r * 32 + c) = y;
+    *reinterpret_cast<float4 *>(Xs + r2 * kLy + c2) = y;
   }
   __syncthreads();
-  {  // step 2b: T([32,64), [0,32)) = -T([32,64), [32,64)) Y
-    const int r = tid >> 3, c = (tid & 7) * 4;
-    const float *trow = Ts + (32 + r) * kLd + 32;
+  {  // T([32,64), [0,32)) = -T([32,64), [32,64)) Y; T(2,3) is unwritten: rows
+     // r < 16 take m < 16 only
+    const int m1 = (warp & 1) ? 32 : 16;
+    const float *trow = Ts + (32 + r2) * kLd + 32;
     float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+    for (int m4 = 0; m4 < m1; m4 += 4) {
+      const float4 t = lds4(trow + m4);
+      const float tv[4] = {t.x, t.y, t.z, t.w};
 #pragma unroll
-    for (int m = 0; m < 32; ++m) {
-      const float t = (m <= r) ? trow[m] : 0.f;
-      const float4 x = *reinterpret_cast<const float4 *>(Xs + m * 32 + c);
-      y.x = fmaf(t, x.x, y.x); y.y = fmaf(t, x.y, y.y);
-      y.z = fmaf(t, x.z, y.z); y.w = fmaf(t, x.w, y.w);
+      for (int e = 0; e < 4; ++e) {
+        const float4 x = lds4(Xs + (m4 + e) * kLy + c2);
+        y.x = fmaf(tv[e], x.x, y.x); y.y = fmaf(tv[e], x.y, y.y);
+        y.z = fmaf(tv[e], x.z, y.z); y.w = fmaf(tv[e], x.w, y.w);
+      }
     }
-    *reinterpret_cast<float4 *>(Ts + (32 + r) * kLd + c) = make_float4(-y.x, -y.y, -y.z, -y.w);
+    *reinterpret_cast<float4 *>(Ts + (32 + r2) * kLd + c2) = make_float4(-y.x, -y.y, -y.z, -y.w);
   }
   __syncthreads();
 }
@@ -199,6 +234,7 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
   float *Gm = reinterpret_cast<float *>(sm + kP_VEC);
   float *Bt = Gm + 64;
   float *Ga = Bt + 64;
+  float *Gl = Ga + 64;                     // Gamma log2(e)
   uint64_t *bar_load = reinterpret_cast<uint64_t *>(sm + kP_BAR);
   uint64_t *bar_mma = bar_load + 1;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_load + 2);
@@ -244,6 +280,9 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
     const float excl = s - (a0 + a1);
     Gm[2 * lane] = excl + a0;
     Gm[2 * lane + 1] = s;
+    constexpr float kLog2e = 1.4426950408889634f;
+    Gl[2 * lane] = (excl + a0) * kLog2e;
+    Gl[2 * lane + 1] = s * kLog2e;
   }
   const bool loaded = mbar_wait(bar_load, 0, ctrl, &abort_flag);
   GDN_TRACE_POINT(tr, 1, chunk, 1);
@@ -284,34 +323,54 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
   const int m = (warp & 3) * 32 + lane;   // TMEM lane = row of G
   const int hc = warp >> 2;               // column half
   const uint32_t lane_base = tmem + (uint32_t((warp & 3) * 32) << 16);
+  // A[r][s] = beta_r 2^(Gl_r - Gl_s) G[r][s] for s < r (fp32, for the solve);
+  // P[c][s] = 2^(Gl_c - Gl_s) G[c][s] for s <= c (bf16 operand tile). Warps 4
+  // (A rows 0-31) and 6 (P rows 0-31) hold columns 32-63, all above the
+  // diagonal: they write zeros without touching tensor memory.
+  const bool zero_warp = (hc == 1) && ((warp & 1) == 0);
   if (!abort_flag) {
     uint32_t r0[32];
-    tmem_ld32(lane_base + 32 * hc, r0);
-    tmem_ld_wait();
+    if (!zero_warp) {
+      tmem_ld32(lane_base + 32 * hc, r0);
+      tmem_ld_wait();
+    } else {
+#pragma unroll
+      for (int t = 0; t < 32; ++t) r0[t] = 0u;
+    }
     if (m < kC) {
       const int r = m;
-      const float br = Bt[r], gr = Gm[r];
+      const float br = Bt[r], glr = Gl[r];
 #pragma unroll
       for (int t = 0; t < 32; t += 4) {
-        float4 a;
         const int s = 32 * hc + t;
-        a.x = (s + 0 < r) ? br * __expf(gr - Gm[s + 0]) * __uint_as_float(r0[t + 0]) : 0.f;
-        a.y = (s + 1 < r) ? br * __expf(gr - Gm[s + 1]) * __uint_as_float(r0[t + 1]) : 0.f;
-        a.z = (s + 2 < r) ? br * __expf(gr - Gm[s + 2]) * __uint_as_float(r0[t + 2]) : 0.f;
-        a.w = (s + 3 < r) ? br * __expf(gr - Gm[s + 3]) * __uint_as_float(r0[t + 3]) : 0.f;
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (!zero_warp) {
+          const float4 gs = lds4(Gl + s);
+          a.x = (s + 0 < r) ? br * ex2_approx(glr - gs.x) * __uint_as_float(r0[t + 0]) : 0.f;
+          a.y = (s + 1 < r) ? br * ex2_approx(glr - gs.y) * __uint_as_float(r0[t + 1]) : 0.f;
+          a.z = (s + 2 < r) ? br * ex2_approx(glr - gs.z) * __uint_as_float(r0[t + 2]) : 0.f;
+          a.w = (s + 3 < r) ? br * ex2_approx(glr - gs.w) * __uint_as_float(r0[t + 3]) : 0.f;
+        }
         *reinterpret_cast<float4 *>(As + r * kLd + s) = a;
       }
     } else {
       const int c = m - kC;
-      const float gc = Gm[c];
+      const float glc = Gl[c];
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         const int ch = 4 * hc + cc;
         float f[8];
+        if (!zero_warp) {
+          const float4 g0 = lds4(Gl + ch * 8), g1 = lds4(Gl + ch * 8 + 4);
+          const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int s = ch * 8 + e;
-          f[e] = (s <= c) ? __expf(gc - Gm[s]) * __uint_as_float(r0[8 * cc + e]) : 0.f;
+          for (int e = 0; e < 8; ++e) {
+            const int s = ch * 8 + e;
+            f[e] = (s <= c) ? ex2_approx(glc - gv[e]) * __uint_as_float(r0[8 * cc + e]) : 0.f;
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] = 0.f;
         }
         *reinterpret_cast<uint4 *>(sm + kP_PST + sw128_offset(c, ch)) =
             make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
@@ -329,26 +388,41 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
   GDN_TRACE_POINT(tr, 1, chunk, 3);
   if (!abort_flag) solve_unit_lower_64(As, Ts, Xs, tid);
   GDN_TRACE_POINT(tr, 1, chunk, 4);
-  // T diag(beta) and T diag(beta gamma) as bf16 K-major operand tiles (A is dead now)
+  // T diag(beta) and T diag(beta gamma) as bf16 K-major operand tiles (A is
+  // dead now). Thread: row r, columns [16 q4, 16 q4 + 16); T is lower
+  // triangular and its upper blocks are unwritten, so s > r reads as zero.
   {
     const int r = tid >> 2, q4 = tid & 3;
+    float fb[16], fg[16];
+    if (16 * q4 <= r) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int s0 = 16 * q4 + 4 * i;
+        const float4 t = lds4(Ts + r * kLd + s0);
+        const float4 bt = lds4(Bt + s0), ga = lds4(Ga + s0);
+        const float tv[4] = {t.x, t.y, t.z, t.w}, bv[4] = {bt.x, bt.y, bt.z, bt.w},
+                    gv[4] = {ga.x, ga.y, ga.z, ga.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float v = (s0 + e <= r) ? tv[e] * bv[e] : 0.f;
+          fb[4 * i + e] = v;
+          fg[4 * i + e] = v * gv[e];
+        }
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) fb[e] = fg[e] = 0.f;
+    }
 #pragma unroll
     for (int cc = 0; cc < 2; ++cc) {
       const int ch = q4 * 2 + cc;
-      float fb[8], fg[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int s = ch * 8 + e;
-        const float t = (s <= r) ? Ts[r * kLd + s] * Bt[s] : 0.f;
-        fb[e] = t;
-        fg[e] = t * Ga[s];
-      }
+      const float *xb = fb + 8 * cc, *xg = fg + 8 * cc;
       *reinterpret_cast<uint4 *>(sm + kP_TB + sw128_offset(r, ch)) =
-          make_uint4(pack_bf16x2(fb[0], fb[1]), pack_bf16x2(fb[2], fb[3]),
-                     pack_bf16x2(fb[4], fb[5]), pack_bf16x2(fb[6], fb[7]));
+          make_uint4(pack_bf16x2(xb[0], xb[1]), pack_bf16x2(xb[2], xb[3]),
+                     pack_bf16x2(xb[4], xb[5]), pack_bf16x2(xb[6], xb[7]));
       *reinterpret_cast<uint4 *>(sm + kP_TBG + sw128_offset(r, ch)) =
-          make_uint4(pack_bf16x2(fg[0], fg[1]), pack_bf16x2(fg[2], fg[3]),
-                     pack_bf16x2(fg[4], fg[5]), pack_bf16x2(fg[6], fg[7]));
+          make_uint4(pack_bf16x2(xg[0], xg[1]), pack_bf16x2(xg[2], xg[3]),
+                     pack_bf16x2(xg[4], xg[5]), pack_bf16x2(xg[6], xg[7]));
     }
   }
   __syncthreads();
@@ -461,50 +535,69 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
 // One stage (one chunk of one head), as the B operands of three wide MMAs:
 //   BXZ  2 x [ -W rows 0-63 | Q rows 64-127 ]  (128 rows, K = d_k in two blocks)
 //   BU   [ T diag(beta) rows 0-63 | zeros ]    (128 rows, K = 64 tokens)
-//   BSY  [ (D K)^T rows 0-127 | P rows 128-191 ] (192 rows, K = 64 tokens)
+//   BSY  stage 0: [ (D K)^T rows 0-127 | P rows 128-191 ]  (192 rows, K = 64 tokens)
+//        stage 1: [ P rows 0-63 | (D K)^T rows 64-191 ]
 // plus V (the MN-major A operand of U^T). The zero half of BU is written
-// once; TMA never touches it. The per-chunk decay factors (gamma[64], D[64])
-// travel in a separate 4-slot ring so the output warps never hold a stage.
+// once; TMA never touches it. The two BSY orders put dS in the same tensor
+// memory columns for every chunk and Y in one of two buffers (Y0 after dS,
+// Y1 before it), so SY(c+1) never waits for the output warps to finish Y(c).
+// The per-chunk decay factors (gamma[64], D[64]) travel in a separate 4-slot
+// ring so the output warps never hold a stage.
 constexpr uint32_t kS_BXZ = 0;                        // 32 KB
 constexpr uint32_t kS_V = kS_BXZ + 2 * kTile128x64;   // 16 KB, 2 x [64 s][64 d]
 constexpr uint32_t kS_BU = kS_V + 2 * kTile64x64;     // 16 KB
 constexpr uint32_t kS_BSY = kS_BU + kTile128x64;      // 24 KB
 constexpr uint32_t kStageBytes = kS_BSY + kTile128x64 + kTile64x64;   // 88 KB
 constexpr int kStages = 2, kGamSlots = 4;
+constexpr int kPrefetchAhead = 2;     // chunks prefetched into L2 ahead of the stage loads
 constexpr uint32_t kS_OST = kStages * kStageBytes;            // O staging, 2 x [64 c][64 d]
 constexpr uint32_t kS_GAM = kS_OST + 2 * kTile64x64;          // kGamSlots x 128 fp32
 constexpr uint32_t kS_BAR = kS_GAM + kGamSlots * 512;         // mbarriers, tmem slot, flags
 constexpr uint32_t kS_END = kS_BAR + 256;
 constexpr uint32_t kScanSmem = kS_END;   // the dynamic window starts 1024-aligned (checked)
-constexpr uint32_t kStageTx = kStageBytes - kTile64x64;       // everything but the zero tile
+constexpr uint32_t kStageTxA = kS_BSY - kTile64x64;   // BXZ, V and Tb (not the zero tile)
+constexpr uint32_t kStageTxB = kTile128x64 + kTile64x64;   // (D K)^T and P
 constexpr int kScanThreads = 512;
 // TMEM columns (fp32 accumulators, then the bf16 A operands held in TMEM)
-constexpr uint32_t kT_XZ = 0;     // [X | Z]  = [U^T - S W^T | S Q^T]        fp32 [128][128]
-constexpr uint32_t kT_SY = 128;   // [dS | Y] = [V_new^T (DK) | V_new^T P^T] fp32 [128][192]
-constexpr uint32_t kT_S = 320;    // S        bf16 [128][128] (64 columns)
-constexpr uint32_t kT_A1 = 384;   // V_new^T  bf16 [128][64]  (32 columns)
+constexpr uint32_t kT_XZ = 0;     // [X | Z] = [U^T - S W^T | S Q^T]      fp32 [128][128]
+constexpr uint32_t kT_Y1 = 128;   // Y of odd chunks  = V_new^T P^T       fp32 [128][64]
+constexpr uint32_t kT_DS = 192;   // dS = V_new^T (D K)                    fp32 [128][128]
+constexpr uint32_t kT_Y0 = 320;   // Y of even chunks                      fp32 [128][64]
+constexpr uint32_t kT_S = 384;    // S        bf16 [128][128] (64 columns)
+constexpr uint32_t kT_A1 = 448;   // V_new^T  bf16 [128][64]  (32 columns)
 // Named barriers (0 is __syncthreads)
-constexpr uint32_t kBarChain = 1, kBarOut = 2;
+constexpr uint32_t kBarOut = 2;
 // Barrier slots in the kS_BAR area
-constexpr int kB_FULL = 0, kB_EMPTY = 2, kB_GFULL = 4, kB_GEMPTY = 8, kB_XFULL = 12,
-              kB_SFULL = 13, kB_YFULL = 14, kB_ZFREE = 15, kB_YFREE = 16, kB_DRAIN = 17,
-              kB_COUNT = 18;
+// y_full[b] completes when Y buffer b holds a new chunk; the output warps wait
+// on it, the chain on s_full. (One barrier for both would let a slow output
+// warp miss a phase: it reports Z consumed before it waits for Y.)
+// Each stage has two parts with their own full/empty pairs: part A (BXZ, V,
+// BU) is last read by XZ(c) and part B (BSY) by SY(c), so the next loads of
+// part A start while SY(c) and the S epilogue still run.
+constexpr int kB_FULLA = 0, kB_EMPTYA = 2, kB_FULLB = 4, kB_EMPTYB = 6, kB_GFULL = 8,
+              kB_GEMPTY = 12, kB_XFULL = 16, kB_SFULL = 17, kB_YFULL = 18, kB_ZFREE = 20,
+              kB_A1RDY = 21, kB_SRDY = 22, kB_DRAIN = 23, kB_COUNT = 24;
+constexpr int kChainWarps = 8;
 
-// Warp roles (16 warps):
-//   warp 0        TMA producer (one elected lane)
-//   warp 1        TMEM allocation
+// Warp roles (16 warps). Every role runs its loop with all 32 lanes, so the
+// lanes of a warp wait on barriers together; one lane issues TMA copies,
+// MMAs and arrivals.
+//   warp 0        TMA producer
+//   warp 1        TMEM allocation and every tcgen05.mma
 //   warps 4-11    state chain: two warpgroups, warpgroup h owns columns
 //                 [32h, 32h+32) of V_new and [64h, 64h+64) of S; thread =
 //                 TMEM lane = row i of d_v; the fp32 S lives in its registers,
-//                 its bf16 copy (an MMA operand) in tensor memory.
-//                 Lane 0 of warp 4 also issues every tcgen05.mma.
+//                 its bf16 copy (an MMA operand) in tensor memory. Each warp
+//                 reports a finished epilogue with one mbarrier arrival.
 //   warps 12-15   output: O = diag(gamma) Z + Y, staged for TMA stores
 // Per chunk c the tensor core runs three wide products:
 //   U(c)   [X|Z]  = V^T [Tb | 0]^T            (4 MMAs, N = 128)  -- before S_c is known
 //   XZ(c)  [X|Z] += S [-W | Q]^T              (8 MMAs, N = 128)  -> X = V_new^T, Z = S Q^T
 //   SY(c)  [dS|Y] = V_new^T [(DK)^T | P]^T    (4 MMAs, N = 192)
 // and the chain is XZ -> V_new epilogue -> SY -> S epilogue -> XZ(c+1), with
-// U(c+1) running during the S epilogue.
+// U(c+1) running during the S epilogue. The MMA warp does its other waits
+// (output done with Z, next stage loaded) while the V_new epilogue runs, so
+// only the two epilogue handshakes sit on the chain.
 __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_v,
     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_kt,
@@ -527,10 +620,12 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
   (void)tr;
 
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kS_BAR);
-  uint64_t *full = bars + kB_FULL, *empty = bars + kB_EMPTY;
+  uint64_t *full_a = bars + kB_FULLA, *empty_a = bars + kB_EMPTYA;
+  uint64_t *full_b = bars + kB_FULLB, *empty_b = bars + kB_EMPTYB;
   uint64_t *gfull = bars + kB_GFULL, *gempty = bars + kB_GEMPTY;
   uint64_t *x_full = bars + kB_XFULL, *s_full = bars + kB_SFULL, *y_full = bars + kB_YFULL;
-  uint64_t *z_free = bars + kB_ZFREE, *y_free = bars + kB_YFREE, *drain = bars + kB_DRAIN;
+  uint64_t *z_free = bars + kB_ZFREE, *drain = bars + kB_DRAIN;
+  uint64_t *a1_rdy = bars + kB_A1RDY, *s_rdy = bars + kB_SRDY;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kB_COUNT);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -544,8 +639,12 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     tma_prefetch_desc(&tm_pm);
     tma_prefetch_desc(&tm_gam);
     tma_prefetch_desc(&tm_o);
-    for (int b = 0; b < kB_COUNT; ++b)
-      mbar_init(bars + b, (b >= kB_GEMPTY && b < kB_GEMPTY + 4) ? 2 : 1);
+    for (int b = 0; b < kB_COUNT; ++b) {
+      uint32_t count = 1;
+      if (b >= kB_GEMPTY && b < kB_GEMPTY + 4) count = 2;        // MMA warp + output
+      if (b == kB_A1RDY || b == kB_SRDY) count = kChainWarps;
+      mbar_init(bars + b, count);
+    }
     fence_mbar_init();
   }
   // The zero half of BU in both stages.
@@ -563,78 +662,160 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // Waits used by the warpgroups that keep named barriers in step: after an
-  // abort they return at once instead of leaving the loop.
-  auto wait = [&](uint64_t *bar, uint32_t parity) {
-    if (!*abort_flag) mbar_wait(bar, parity, ctrl, abort_flag);
-  };
+  // Waits inside the role loops: after an abort they return at once, so every
+  // loop runs to its end and named barriers stay in step.
+  auto wait = [&](uint64_t *bar, uint32_t parity) { mbar_wait(bar, parity, ctrl, abort_flag); };
 
-  if (warp == 0 && lane == 0) {
+  if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    for (int c = 0; c < nch; ++c) {
+    for (int c = 0; c < nch && !*abort_flag; ++c) {
       const int st = c & 1, gs = c & 3;
-      if (c >= 2 && !mbar_wait(empty + st, ((c >> 1) - 1) & 1, ctrl, abort_flag)) break;
       const ChunkInfo ci = table[c0 + c];
       const int unit = (c0 + c) * H + h;
       uint8_t *sb = sm + st * kStageBytes;
-      GDN_TRACE_POINT(tr, 0, c, 0);
-      mbar_arrive_expect_tx(full + st, kStageTx);
-      tma_load_2d(sb + kS_BXZ, &tm_w, full + st, 0, unit * kC);
-      tma_load_3d(sb + kS_BXZ + kTile64x64, &tm_q, full + st, 0, h, ci.row0);
-      tma_load_2d(sb + kS_BXZ + kTile128x64, &tm_w, full + st, 64, unit * kC);
-      tma_load_3d(sb + kS_BXZ + kTile128x64 + kTile64x64, &tm_q, full + st, 64, h, ci.row0);
-      tma_load_3d(sb + kS_V, &tm_v, full + st, 0, h, ci.row0);
-      tma_load_3d(sb + kS_V + kTile64x64, &tm_v, full + st, 64, h, ci.row0);
-      tma_load_2d(sb + kS_BU, &tm_tb, full + st, 0, unit * kC);
-      tma_load_2d(sb + kS_BSY, &tm_kt, full + st, 0, unit * kD);
-      tma_load_2d(sb + kS_BSY + kTile128x64, &tm_pm, full + st, 0, unit * kC);
-      if (c >= 4 && !mbar_wait(gempty + gs, ((c >> 2) - 1) & 1, ctrl, abort_flag)) break;
-      mbar_arrive_expect_tx(gfull + gs, 512);
-      tma_load_2d(sm + kS_GAM + gs * 512, &tm_gam, gfull + gs, 0, unit);
+      if (c >= 2) wait(empty_a + st, ((c >> 1) - 1) & 1);
+      if (lane == 0) {
+        GDN_TRACE_POINT(tr, 0, c, 0);
+        mbar_arrive_expect_tx(full_a + st, kStageTxA);
+        tma_load_2d(sb + kS_BXZ, &tm_w, full_a + st, 0, unit * kC);
+        tma_load_3d(sb + kS_BXZ + kTile64x64, &tm_q, full_a + st, 0, h, ci.row0);
+        tma_load_2d(sb + kS_BXZ + kTile128x64, &tm_w, full_a + st, 64, unit * kC);
+        tma_load_3d(sb + kS_BXZ + kTile128x64 + kTile64x64, &tm_q, full_a + st, 64, h, ci.row0);
+        tma_load_3d(sb + kS_V, &tm_v, full_a + st, 0, h, ci.row0);
+        tma_load_3d(sb + kS_V + kTile64x64, &tm_v, full_a + st, 64, h, ci.row0);
+        tma_load_2d(sb + kS_BU, &tm_tb, full_a + st, 0, unit * kC);
+      }
+      __syncwarp();
+      if (c >= 2) wait(empty_b + st, ((c >> 1) - 1) & 1);
+      if (lane == 0) {
+        mbar_arrive_expect_tx(full_b + st, kStageTxB);
+        tma_load_2d(sb + kS_BSY + (st ? kTile64x64 : 0u), &tm_kt, full_b + st, 0, unit * kD);
+        tma_load_2d(sb + kS_BSY + (st ? 0u : kTile128x64), &tm_pm, full_b + st, 0, unit * kC);
+        // The loads above take about one chunk period to land from HBM; the
+        // chunk after next goes to L2 now, so its own loads come from L2.
+        if (c + kPrefetchAhead < nch) {
+          const ChunkInfo cp = table[c0 + c + kPrefetchAhead];
+          const int up = (c0 + c + kPrefetchAhead) * H + h;
+          tma_prefetch_l2_2d(&tm_w, 0, up * kC);
+          tma_prefetch_l2_2d(&tm_w, 64, up * kC);
+          tma_prefetch_l2_3d(&tm_q, 0, h, cp.row0);
+          tma_prefetch_l2_3d(&tm_q, 64, h, cp.row0);
+          tma_prefetch_l2_3d(&tm_v, 0, h, cp.row0);
+          tma_prefetch_l2_3d(&tm_v, 64, h, cp.row0);
+          tma_prefetch_l2_2d(&tm_tb, 0, up * kC);
+          tma_prefetch_l2_2d(&tm_kt, 0, up * kD);
+          tma_prefetch_l2_2d(&tm_pm, 0, up * kC);
+        }
+      }
+      __syncwarp();
+      if (c >= 4) wait(gempty + gs, ((c >> 2) - 1) & 1);
+      if (lane == 0) {
+        mbar_arrive_expect_tx(gfull + gs, 512);
+        tma_load_2d(sm + kS_GAM + gs * 512, &tm_gam, gfull + gs, 0, unit);
+      }
+      __syncwarp();
     }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t id_u = make_idesc_bf16(128, 128, 1, 0);     // V^T [Tb|0]^T : A MN-major
+    const uint32_t id_xz = make_idesc_bf16(128, 128, 0, 0);    // S [-W|Q]^T
+    const uint32_t id_sy = make_idesc_bf16(128, 192, 0, 0);    // A1 [(DK)^T|P]^T
+    const bool issuer = lane == 0;
+    // U(c) into [X|Z]. The caller has seen chunk c loaded and the output
+    // warps done reading Z of chunk c - 1.
+    auto issue_u = [&](int c) {
+      const uint32_t sb = smem_u32(sm + (c & 1) * kStageBytes);
+      if (issuer) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma_bf16(tmem + kT_XZ, make_sdesc(sb + kS_V + kk * 2048, kTile64x64, 1024),
+                      make_sdesc(sb + kS_BU + kk * 32, 16, 1024), id_u, kk > 0);
+      }
+      __syncwarp();
+    };
+    // XZ(c) += S_c [-W|Q]^T, reading the bf16 copy of S_c.
+    auto issue_xz = [&](int c) {
+      const uint32_t sb = smem_u32(sm + (c & 1) * kStageBytes);
+      if (issuer) {
+        GDN_TRACE_POINT(tr, 0, c, 1);
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc_mma_bf16_ts(tmem + kT_XZ, tmem + kT_S + 8 * kk,
+                         make_sdesc(sb + kS_BXZ + (kk >> 2) * kTile128x64 + (kk & 3) * 32, 16,
+                                    1024),
+                         id_xz, 1);
+        tc_commit(x_full);
+        tc_commit(empty_a + (c & 1));     // U(c) and XZ(c) were the last readers of part A
+      }
+      __syncwarp();
+    };
+    if (nch > 0) {
+      wait(full_a, 0);
+      issue_u(0);
+      wait(s_rdy, 0);                     // S_0 stored
+      issue_xz(0);
+    }
+    for (int c = 0; c < nch; ++c) {
+      const int st = c & 1, gs = c & 3;
+      const bool more = c + 1 < nch;
+      wait(full_b + st, (c >> 1) & 1);    // (D K)^T and P of chunk c (while XZ(c) runs)
+      wait(a1_rdy, c & 1);                // V_new^T of chunk c in tensor memory
+      GDN_TRACE_POINT(tr && issuer, 0, c, 6);
+      if (issuer) {
+        const uint32_t sb = smem_u32(sm + st * kStageBytes);
+        tc_fence_after();
+        // even chunks: D = [dS | Y0] at kT_DS; odd: D = [Y1 | dS] at kT_Y1
+        const uint32_t d = tmem + (st ? kT_Y1 : kT_DS);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma_bf16_ts(d, tmem + kT_A1 + 8 * kk, make_sdesc(sb + kS_BSY + kk * 32, 16, 1024),
+                         id_sy, kk > 0);
+        tc_commit(s_full);
+        GDN_TRACE_POINT(tr, 0, c, 12);
+      }
+      __syncwarp();
+      // Off the chain (SY(c) and the S epilogue are running): U(c+1) needs the
+      // output warps done with Z(c) and part A of chunk c + 1.
+      if (more) {
+        wait(z_free, c & 1);
+        GDN_TRACE_POINT(tr && issuer, 0, c, 13);
+        wait(full_a + (st ^ 1), ((c + 1) >> 1) & 1);
+        GDN_TRACE_POINT(tr && issuer, 0, c, 14);
+        issue_u(c + 1);
+      }
+      if (issuer) {
+        tc_commit(y_full + st);           // also covers U(c+1): the output has slack
+        tc_commit(empty_b + st);          // SY(c) was the last reader of part B
+      }
+      __syncwarp();
+      wait(s_rdy, (c + 1) & 1);           // S_{c+1} stored, decay factors of c read
+      GDN_TRACE_POINT(tr && issuer, 0, c, 8);
+      if (more) issue_xz(c + 1);
+      if (issuer) mbar_arrive(gempty + gs);
+      __syncwarp();
+    }
+    if (issuer) tc_commit(drain);         // fires once every MMA above has completed
+    __syncwarp();
+    // Waited for even after an abort (bounded): tensor memory is freed below.
+    volatile int keep_waiting = 0;
+    mbar_wait(drain, 0, ctrl, &keep_waiting);
   } else if (warp >= 4 && warp < 12) {
     // ------------------------------------------------------------ state chain
     const int hh = (warp - 4) >> 2;                     // column half
     const int i = ((warp & 3) << 5) + lane;             // TMEM lane = row of d_v
     const uint32_t lane_base = tmem + (uint32_t((warp & 3) * 32) << 16);
-    const bool leader = (warp == 4 && lane == 0);
-    const uint32_t id_u = make_idesc_bf16(128, 128, 1, 0);     // V^T [Tb|0]^T : A MN-major
-    const uint32_t id_xz = make_idesc_bf16(128, 128, 0, 0);    // S [-W|Q]^T
-    const uint32_t id_sy = make_idesc_bf16(128, 192, 0, 0);    // A1 [(DK)^T|P]^T
-    // Leader only. U(c) into [X|Z]: needs chunk c loaded and the output warps
-    // done reading Z of chunk c - 1 (one barrier phase per chunk).
-    auto issue_u = [&](int c) {
-      const int st = c & 1;
-      const uint32_t sb = smem_u32(sm + st * kStageBytes);
-      if (c >= 1 && !mbar_wait(z_free, (c - 1) & 1, ctrl, abort_flag)) return;
-      if (!mbar_wait(full + st, (c >> 1) & 1, ctrl, abort_flag)) return;
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        tc_mma_bf16(tmem + kT_XZ, make_sdesc(sb + kS_V + kk * 2048, kTile64x64, 1024),
-                    make_sdesc(sb + kS_BU + kk * 32, 16, 1024), id_u, kk > 0);
-    };
-    // Leader only. XZ(c) += S_c [-W|Q]^T, reading the bf16 copy of S_c.
-    auto issue_xz = [&](int c) {
-      const int st = c & 1;
-      const uint32_t sb = smem_u32(sm + st * kStageBytes);
-      GDN_TRACE_POINT(tr, 0, c, 1);
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        tc_mma_bf16_ts(tmem + kT_XZ, tmem + kT_S + 8 * kk,
-                       make_sdesc(sb + kS_BXZ + (kk >> 2) * kTile128x64 + (kk & 3) * 32, 16,
-                                  1024),
-                       id_xz, 1);
-      tc_commit(x_full);
-    };
+    const bool tl = tr && warp == 4 && lane == 0;       // traced lane
+    (void)tl;
     float S[64];                                        // S[i][64 hh + t], fp32 master
     {
       const float *src = s0 ? s0 + (size_t(n) * H + h) * kD * kD : nullptr;
 #pragma unroll
       for (int t = 0; t < 64; ++t) S[t] = src ? src[size_t(64 * hh + t) * kD + i] : 0.f;
     }
-    // bf16 copy of S (row i, columns [64 hh, 64 hh + 64)) into tensor memory.
+    // bf16 copy of S (row i, columns [64 hh, 64 hh + 64)) into tensor memory,
+    // then one arrival per warp on s_rdy.
     auto store_state = [&]() {
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
@@ -644,80 +825,54 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
         tmem_st16(lane_base + kT_S + 32 * hh + 16 * q, pk);
       }
       tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_rdy);
     };
     store_state();
-    tc_fence_before();
-    named_bar_sync(kBarChain, 256);
-    if (leader && nch > 0 && !*abort_flag) {
-      issue_u(0);
-      issue_xz(0);
-    }
     for (int c = 0; c < nch; ++c) {
       const int gs = c & 3;
-      GDN_TRACE_POINT(tr && leader, 0, c, 3);
-      wait(gfull + gs, (c >> 2) & 1);
-      GDN_TRACE_POINT(tr && leader, 0, c, 4);
       wait(x_full, c & 1);
-      GDN_TRACE_POINT(tr && leader, 0, c, 5);
+      GDN_TRACE_POINT(tl, 0, c, 5);
       tc_fence_after();
       // V_new^T[i][s] = X[i][s] for s in [32 hh, 32 hh + 32): bf16 back to TMEM
       // as the A operand of SY.
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        uint32_t x[16], a1[8];
-        tmem_ld16(lane_base + kT_XZ + 32 * hh + 16 * q, x);
+      {
+        uint32_t x[32], a1[16];
+        tmem_ld32(lane_base + kT_XZ + 32 * hh, x);
         tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
+        for (int e = 0; e < 16; ++e)
           a1[e] = pack_bf16x2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1]));
-        tmem_st8(lane_base + kT_A1 + 16 * hh + 8 * q, a1);
+        tmem_st16(lane_base + kT_A1 + 16 * hh, a1);
       }
       tmem_st_wait();
       tc_fence_before();
-      named_bar_sync(kBarChain, 256);
-      GDN_TRACE_POINT(tr && leader, 0, c, 6);
-      if (leader && !*abort_flag) {
-        const int st = c & 1;
-        const uint32_t sb32 = smem_u32(sm + st * kStageBytes);
-        // Y is single-buffered: the output warps must have read Y of chunk c - 1.
-        if (c == 0 || mbar_wait(y_free, (c - 1) & 1, ctrl, abort_flag)) {
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            tc_mma_bf16_ts(tmem + kT_SY, tmem + kT_A1 + 8 * kk,
-                           make_sdesc(sb32 + kS_BSY + kk * 32, 16, 1024), id_sy, kk > 0);
-          tc_commit(s_full);
-          tc_commit(y_full);
-          tc_commit(empty + st);          // stage free once every MMA reading it is done
-          if (c + 1 < nch) issue_u(c + 1);
-        }
-      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(a1_rdy);
       // S <- gamma_last S + dS on columns [64 hh, 64 hh + 64)
+      wait(gfull + gs, (c >> 2) & 1);
       const float gl = reinterpret_cast<const float *>(sm + kS_GAM + gs * 512)[kC - 1];
       wait(s_full, c & 1);
-      GDN_TRACE_POINT(tr && leader, 0, c, 7);
+      GDN_TRACE_POINT(tl, 0, c, 7);
       tc_fence_after();
 #pragma unroll
       for (int b = 0; b < 2; ++b) {
         uint32_t d[32];
-        tmem_ld32(lane_base + kT_SY + 64 * hh + 32 * b, d);
+        tmem_ld32(lane_base + kT_DS + 64 * hh + 32 * b, d);
         tmem_ld_wait();
+        GDN_TRACE_POINT(tl && b == 0, 0, c, 3);
 #pragma unroll
-        for (int t = 0; t < 32; ++t) S[32 * b + t] = fmaf(gl, S[32 * b + t], __uint_as_float(d[t]));
+        for (int t = 0; t < 32; t += 2) {
+          const float2 r = ffma2(make_float2(gl, gl), make_float2(S[32 * b + t], S[32 * b + t + 1]),
+                                 make_float2(__uint_as_float(d[t]), __uint_as_float(d[t + 1])));
+          S[32 * b + t] = r.x;
+          S[32 * b + t + 1] = r.y;
+        }
       }
       store_state();
-      tc_fence_before();
-      named_bar_sync(kBarChain, 256);
-      GDN_TRACE_POINT(tr && leader, 0, c, 8);
-      if (leader) {
-        mbar_arrive(gempty + gs);
-        if (c + 1 < nch && !*abort_flag) issue_xz(c + 1);
-      }
-    }
-    if (leader) {
-      // Every MMA issued above has completed once this fires.
-      tc_commit(drain);
-      mbar_wait(drain, 0, ctrl, abort_flag);
+      GDN_TRACE_POINT(tl, 0, c, 4);
+      GDN_TRACE_POINT(tr && warp == 11 && lane == 0, 0, c, 15);
     }
     if (sN && !*abort_flag) {
       float *dst = sN + (size_t(n) * H + h) * kD * kD;
@@ -743,7 +898,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
       const float *gam = reinterpret_cast<const float *>(sm + kS_GAM + gs * 512);
       const ChunkInfo ci = table[c0 + c];
       const bool whole = ci.len == kC;
-      uint32_t z[2][32];
+      uint32_t z[2][32], ynext[8];
       wait(x_full, c & 1);
       tc_fence_after();
       tmem_ld16x256_x8(lane_q + kT_XZ + 64, z[0]);
@@ -755,8 +910,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
       wait(gfull + gs, (c >> 2) & 1);
       if (leader) tma_store_wait_read();     // staging free again
       named_bar_sync(kBarOut, 128);
-      wait(y_full, c & 1);
+      wait(y_full + (c & 1), (c >> 1) & 1);
       GDN_TRACE_POINT(tr && leader, 0, c, 9);
+      const uint32_t ycol = (c & 1) ? kT_Y1 : kT_Y0;
       tc_fence_after();
 #pragma unroll
       for (int lb = 0; lb < 2; ++lb) {
@@ -764,8 +920,14 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
         for (int cbi = 0; cbi < 4; ++cbi) {
           const int cb = 16 * cbi;
           uint32_t y[8];
-          tmem_ld16x256_x2(lane_q + (uint32_t(16 * lb) << 16) + kT_SY + 128 + cb, y);
-          tmem_ld_wait();
+          if ((cbi & 1) == 0) {              // two loads in flight per wait
+            tmem_ld16x256_x2(lane_q + (uint32_t(16 * lb) << 16) + ycol + cb, y);
+            tmem_ld16x256_x2(lane_q + (uint32_t(16 * lb) << 16) + ycol + cb + 16, ynext);
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) y[e] = ynext[e];
+          }
           const float2 g0 = *reinterpret_cast<const float2 *>(gam + cb + fc);
           const float2 g1 = *reinterpret_cast<const float2 *>(gam + cb + 8 + fc);
           uint32_t w[4];
@@ -791,7 +953,6 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
       named_bar_sync(kBarOut, 128);
       GDN_TRACE_POINT(tr && leader, 0, c, 11);
       if (leader) {
-        mbar_arrive(y_free);
         mbar_arrive(gempty + gs);
         if (whole && !*abort_flag) {
           tma_store_3d(&tm_o, sm + kS_OST, 0, h, ci.row0);
@@ -800,6 +961,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
         }
         GDN_TRACE_POINT(tr, 0, c, 10);
       }
+      __syncwarp();
       if (!whole && !*abort_flag) {
         // rows [0, len) of the tile, 16 bytes at a time
         for (int e = ot; e < ci.len * 16; e += 128) {
@@ -811,6 +973,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
       }
     }
     if (leader) tma_store_wait_all();
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();

@@ -84,10 +84,12 @@ constexpr uint32_t kSuspendNs = 1000000;   // 1 ms per sleep; wakes early on com
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t *err,
                                           volatile int *abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
+  // Slow path only: the abort flag is shared memory, and reading it on every
+  // call would put a shared-memory round trip on every wait.
   const long long t0 = clock64();
   while (true) {
-    if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
     if (*abort_flag) return false;
+    if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
     if (clock64() - t0 > kWaitLimitCycles) {
       atomicOr(err, kErrTimeout);
       *abort_flag = 1;
@@ -123,6 +125,32 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *m, uin
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
       : "memory");
+}
+// Two fp32 fused multiply-adds in one instruction (fma.rn.f32x2, sm_100):
+// returns {a.x * b.x + c.x, a.y * b.y + c.y}, each rounded once.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t ra, rb, rc, rd;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a.x), "f"(a.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(rb) : "f"(b.x), "f"(b.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(rc) : "f"(c.x), "f"(c.y));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(rd) : "l"(ra), "l"(rb), "l"(rc));
+  float2 d;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(rd));
+  return d;
+}
+// Prefetch a tile into L2 only (no shared memory, no barrier): a later TMA
+// load of the same tile then waits for L2 instead of HBM.
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *m, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap *m, int x, int y, int z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y), "r"(z)
+               : "memory");
 }
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap *m, const void *src, int x,
                                              int y) {
