@@ -229,7 +229,10 @@ def main():
     assert gdn.get_status(ws) == gdn.OK
 
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    # Timed region: one event pair around each step. The prep and scan kernels
+    # start with programmatic dependent launch; an event between them would
+    # serialise them, so the per-kernel split comes from a separate pass below.
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     for e in evs:                      # torch creates the CUDA event on first record
         for x in e:
             x.record(stream)
@@ -240,23 +243,37 @@ def main():
     torch.cuda.synchronize()
     for i in range(K):
         flush.fill_(i & 0xFF)                       # evict L2 between timed steps
-        e = evs[i]
-        L.gdn_set_profile_events(e[0].cuda_event, e[1].cuda_event, e[2].cuda_event,
-                                 e[3].cuda_event)
+        evs[i][0].record(stream)
         step()
-    L.gdn_set_profile_events(None, None, None, None)
+        evs[i][1].record(stream)
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
     status = gdn.get_status(ws)
     if status != gdn.OK:
         raise SystemExit(f"device status {status}")
-    t_map = [e[0].elapsed_time(e[1]) for e in evs]
-    t_prep = [e[1].elapsed_time(e[2]) for e in evs]
-    t_scan = [e[2].elapsed_time(e[3]) for e in evs]
-    t_step = [e[0].elapsed_time(e[3]) for e in evs]
+    t_step = [a.elapsed_time(b) for a, b in evs]
     ms_local = sum(t_step) / K
     ms = max_over_ranks(ms_local)
+
+    # Per-kernel split (untimed pass): events recorded between the launches.
+    kp = min(K, 10)
+    pev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(kp)]
+    for e in pev:
+        for x in e:
+            x.record(stream)
+    torch.cuda.synchronize()
+    for i in range(kp):
+        flush.fill_(i & 0xFF)
+        e = pev[i]
+        L.gdn_set_profile_events(e[0].cuda_event, e[1].cuda_event, e[2].cuda_event,
+                                 e[3].cuda_event)
+        step()
+    L.gdn_set_profile_events(None, None, None, None)
+    torch.cuda.synchronize()
+    t_map = [e[0].elapsed_time(e[1]) for e in pev]
+    t_prep = [e[1].elapsed_time(e[2]) for e in pev]
+    t_scan = [e[2].elapsed_time(e[3]) for e in pev]
     tokens = B * T
     value = world * tokens / (ms * 1e-3) / 1e6
 
@@ -378,6 +395,8 @@ def main():
                      "peak_source": pk["source"]},
         "kernels_ms": kernels,
         "kernel_share": {k2: v2 / tot for k2, v2 in kernels.items()},
+        "kernels_note": "per-kernel times from an untimed pass with events between the "
+                        "launches (no launch overlap); ms_per_step is the timed region",
         "gpu_launches": 3 * K,
         "clocks": clocks,
         "e2e": e2e,

@@ -25,24 +25,42 @@ __global__ void __launch_bounds__(1024) gdn_chunk_map_kernel(
     const int32_t *__restrict__ cu, int B, int T, int num_seqs, int chunk,
     uint32_t *__restrict__ ctrl, ChunkInfo *__restrict__ table,
     int32_t *__restrict__ seq_first, int max_chunks) {
-  __shared__ int32_t scan[1024];
-  __shared__ int bad;
+  // The kernels launched after this one may start their prologues now; they
+  // wait for this grid before reading what it writes.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int N = num_seqs > 0 ? num_seqs : B;
   const int tid = threadIdx.x;
+  if (!cu) {
+    // B sequences of T tokens: every entry has a closed form.
+    const int cps = (T + chunk - 1) / chunk;
+    const int total = B * cps;
+    for (int idx = tid; idx < total; idx += blockDim.x) {
+      const int n = idx / cps, c = idx - n * cps;
+      ChunkInfo ci;
+      ci.seq = n;
+      ci.cidx = c;
+      ci.row0 = n * T + c * chunk;
+      ci.len = min(chunk, T - c * chunk);
+      table[idx] = ci;
+    }
+    for (int n = tid; n <= N; n += blockDim.x) seq_first[n] = n * cps;
+    if (tid == 0) {
+      ctrl[0] = 0;
+      ctrl[1] = uint32_t(total);
+    }
+    return;
+  }
+  __shared__ int32_t scan[1024];
+  __shared__ int bad;
   if (tid == 0) bad = 0;
   __syncthreads();
   const int per = (N + 1023) / 1024;
   const int n0 = min(N, tid * per), n1 = min(N, n0 + per);
   int32_t local = 0;
   for (int n = n0; n < n1; ++n) {
-    int len;
-    if (cu) {
-      const int a = cu[n], b = cu[n + 1];
-      if ((n == 0 && a != 0) || b < a || (n == N - 1 && b != T)) bad = 1;
-      len = b - a;
-    } else {
-      len = T;
-    }
+    const int a = cu[n], b = cu[n + 1];
+    if ((n == 0 && a != 0) || b < a || (n == N - 1 && b != T)) bad = 1;
+    const int len = b - a;
     if (len > 0) local += (len + chunk - 1) / chunk;
   }
   scan[tid] = local;
@@ -56,15 +74,15 @@ __global__ void __launch_bounds__(1024) gdn_chunk_map_kernel(
   const int32_t total = scan[1023];
   if (bad || total > max_chunks) {
     if (tid == 0) {
-      atomicOr(ctrl, kErrBadSeqlens);
+      ctrl[0] = kErrBadSeqlens;
       ctrl[1] = 0;
     }
     return;
   }
   int32_t first = scan[tid] - local;
   for (int n = n0; n < n1; ++n) {
-    const int row0 = cu ? cu[n] : n * T;
-    const int len = cu ? cu[n + 1] - cu[n] : T;
+    const int row0 = cu[n];
+    const int len = cu[n + 1] - row0;
     seq_first[n] = first;
     for (int c = 0; c * chunk < len; ++c) {
       ChunkInfo ci;
@@ -77,7 +95,10 @@ __global__ void __launch_bounds__(1024) gdn_chunk_map_kernel(
     if (len > 0) first += (len + chunk - 1) / chunk;
   }
   if (tid == 1023) seq_first[N] = total;
-  if (tid == 0) ctrl[1] = uint32_t(total);
+  if (tid == 0) {
+    ctrl[0] = 0;
+    ctrl[1] = uint32_t(total);
+  }
 }
 
 template <typename T>
@@ -283,8 +304,7 @@ cudaError_t launch_simt_t(const void *q, const void *k, const void *v, const flo
 cudaError_t launch_chunk_map(const int32_t *cu_seqlens, int B, int T, int num_seqs, int chunk,
                              void *ws, const WsLayout &L, cudaStream_t s) {
   char *base = static_cast<char *>(ws);
-  cudaError_t e = cudaMemsetAsync(base, 0, 256, s);
-  if (e != cudaSuccess) return e;
+  // The kernel writes the control block itself (error word, chunk count).
   gdn_chunk_map_kernel<<<1, 1024, 0, s>>>(
       cu_seqlens, B, T, num_seqs, chunk, reinterpret_cast<uint32_t *>(base),
       reinterpret_cast<ChunkInfo *>(base + L.chunk_table),

@@ -33,6 +33,7 @@
 // epilogue thread owns one TMEM lane = one row of d_v (or d_k). Shared-memory
 // operand tiles use the 128-byte swizzle with 64 bf16 (128 bytes) per row;
 // TMA loads have no cluster broadcast.
+#include <algorithm>
 #include <cstdio>
 #include <cstring>
 
@@ -204,6 +205,12 @@ __device__ void solve_unit_lower_64(const float *__restrict__ As, float *__restr
   __syncthreads();
 }
 
+// Persistent: each CTA loops over (chunk, head) units u = blockIdx.x + i *
+// gridDim.x (u = chunk * H + h). The tensor memory, barriers and tensor-map
+// prefetches are set up once; while a unit runs, the next unit's K and Q
+// tiles are prefetched into L2 and its g and beta into registers, and the
+// unit's TMA stores drain while the next unit starts (a store only has to
+// finish reading shared memory before that memory is written again).
 // Warp roles: all 8 warps share the epilogues. TMEM lane quarter = warp % 4,
 // column half = warp / 4.
 __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
@@ -218,15 +225,7 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
   uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   __shared__ int abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int chunk = blockIdx.x, h = blockIdx.y;
-  if (ctrl[0] & kErrBadSeqlens) return;
-  if (chunk >= int(ctrl[1])) return;
-  const ChunkInfo ci = table[chunk];
-  const int L = ci.len;
-  const int unit = chunk * H + h;
-  const bool tr = (h == 0 && tid == 0);   // traced thread (GDN_TRACE builds only)
-  (void)tr;
-  GDN_TRACE_POINT(tr, 1, chunk, 0);
+  grid_launch_dependents();   // the scan may start its prologue on freed SMs
 
   float *As = reinterpret_cast<float *>(sm + kP_AS);
   float *Ts = reinterpret_cast<float *>(sm + kP_TS);
@@ -255,19 +254,61 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Everything above overlaps the chunk-map kernel; the chunk table, the
+  // chunk count and the error word are read only after it completes.
+  grid_dependency_wait();
+  const int nunits = (ctrl[0] & kErrBadSeqlens) ? 0 : int(ctrl[1]) * H;
+  const int m = (warp & 3) * 32 + lane;   // TMEM lane = row of G
+  const int hc = warp >> 2;               // column half
+  const uint32_t lane_base = tmem + (uint32_t((warp & 3) * 32) << 16);
 
+  // g and beta of unit u (rows past the sequence end read as 0), one row per
+  // thread of the first two warps.
+  float g_reg = 0.f, b_reg = 0.f;
+  auto fetch_gb = [&](int u) {
+    if (tid < kC && u < nunits) {
+      const int cu = u / H, hu = u - cu * H;
+      const ChunkInfo cf = table[cu];
+      const bool ok = tid < cf.len;
+      g_reg = ok ? g[size_t(cf.row0 + tid) * H + hu] : 0.f;
+      b_reg = ok ? beta[size_t(cf.row0 + tid) * H + hu] : 0.f;
+    }
+  };
+  fetch_gb(blockIdx.x);
+  int it = 0;
+  for (int unit = blockIdx.x; unit < nunits; unit += gridDim.x, ++it) {
+  const int chunk = unit / H, h = unit - chunk * H;
+  const ChunkInfo ci = table[chunk];
+  const int L = ci.len;
+  const bool tr = (h == 0 && tid == 0);   // traced thread (GDN_TRACE builds only)
+  (void)tr;
+  GDN_TRACE_POINT(tr && chunk < 64, 1, chunk, 0);
   if (tid == 0) {
-    mbar_arrive_expect_tx(bar_load, 2 * kTile128x64);
-    tma_load_3d(sm + kP_KQ, &tm_k, bar_load, 0, h, ci.row0);
-    tma_load_3d(sm + kP_KQ + kTile64x64, &tm_q, bar_load, 0, h, ci.row0);
-    tma_load_3d(sm + kP_KQ + kTile128x64, &tm_k, bar_load, 64, h, ci.row0);
-    tma_load_3d(sm + kP_KQ + kTile128x64 + kTile64x64, &tm_q, bar_load, 64, h, ci.row0);
+    // The previous unit's TMA stores read the K/Q and A areas: wait until
+    // they have (they need not have reached global memory).
+    tma_store_wait_read();
+    if (!abort_flag) {
+      mbar_arrive_expect_tx(bar_load, 2 * kTile128x64);
+      tma_load_3d(sm + kP_KQ, &tm_k, bar_load, 0, h, ci.row0);
+      tma_load_3d(sm + kP_KQ + kTile64x64, &tm_q, bar_load, 0, h, ci.row0);
+      tma_load_3d(sm + kP_KQ + kTile128x64, &tm_k, bar_load, 64, h, ci.row0);
+      tma_load_3d(sm + kP_KQ + kTile128x64 + kTile64x64, &tm_q, bar_load, 64, h, ci.row0);
+    }
+    const int nu = unit + int(gridDim.x);
+    if (nu < nunits) {
+      const int cn = nu / H, hn = nu - cn * H;
+      const int rn = table[cn].row0;
+      tma_prefetch_l2_3d(&tm_k, 0, hn, rn);
+      tma_prefetch_l2_3d(&tm_k, 64, hn, rn);
+      tma_prefetch_l2_3d(&tm_q, 0, hn, rn);
+      tma_prefetch_l2_3d(&tm_q, 64, hn, rn);
+    }
   }
   if (tid < kC) {
-    const bool ok = tid < L;
-    Gm[tid] = ok ? g[size_t(ci.row0 + tid) * H + h] : 0.f;
-    Bt[tid] = ok ? beta[size_t(ci.row0 + tid) * H + h] : 0.f;
+    Gm[tid] = g_reg;
+    Bt[tid] = b_reg;
   }
+  fetch_gb(unit + int(gridDim.x));
   __syncthreads();
   if (warp == 0) {  // inclusive cumsum of the 64 log-gates
     const float a0 = Gm[2 * lane], a1 = Gm[2 * lane + 1];
@@ -284,8 +325,8 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
     Gl[2 * lane] = (excl + a0) * kLog2e;
     Gl[2 * lane + 1] = s * kLog2e;
   }
-  const bool loaded = mbar_wait(bar_load, 0, ctrl, &abort_flag);
-  GDN_TRACE_POINT(tr, 1, chunk, 1);
+  const bool loaded = mbar_wait(bar_load, it & 1, ctrl, &abort_flag);
+  GDN_TRACE_POINT(tr && chunk < 64, 1, chunk, 1);
   if (loaded && L < kC) {
     // Rows past the sequence end act as k = q = 0 (beta = g = 0 above).
     for (int e = tid; e < (kC - L) * 8; e += kPrepThreads) {
@@ -318,11 +359,9 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
     gam_out[size_t(unit) * 128 + 64 + tid] = expf(Gm[kC - 1] - Gm[tid]);  // D_s
   }
   mbar_wait(bar_mma, 0, ctrl, &abort_flag);
-  GDN_TRACE_POINT(tr, 1, chunk, 2);
+  GDN_TRACE_POINT(tr && chunk < 64, 1, chunk, 2);
   tc_fence_after();
-  const int m = (warp & 3) * 32 + lane;   // TMEM lane = row of G
-  const int hc = warp >> 2;               // column half
-  const uint32_t lane_base = tmem + (uint32_t((warp & 3) * 32) << 16);
+
   // A[r][s] = beta_r 2^(Gl_r - Gl_s) G[r][s] for s < r (fp32, for the solve);
   // P[c][s] = 2^(Gl_c - Gl_s) G[c][s] for s <= c (bf16 operand tile). Warps 4
   // (A rows 0-31) and 6 (P rows 0-31) hold columns 32-63, all above the
@@ -385,9 +424,9 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
     tma_store_2d(&tm_pm, sm + kP_PST, 0, unit * kC);
     tma_store_commit();
   }
-  GDN_TRACE_POINT(tr, 1, chunk, 3);
+  GDN_TRACE_POINT(tr && chunk < 64, 1, chunk, 3);
   if (!abort_flag) solve_unit_lower_64(As, Ts, Xs, tid);
-  GDN_TRACE_POINT(tr, 1, chunk, 4);
+  GDN_TRACE_POINT(tr && chunk < 64, 1, chunk, 4);
   // T diag(beta) and T diag(beta gamma) as bf16 K-major operand tiles (A is
   // dead now). Thread: row r, columns [16 q4, 16 q4 + 16); T is lower
   // triangular and its upper blocks are unwritten, so s > r reads as zero.
@@ -444,7 +483,7 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
   }
   fence_proxy_async_smem();
   __syncthreads();
-  GDN_TRACE_POINT(tr, 1, chunk, 5);
+  GDN_TRACE_POINT(tr && chunk < 64, 1, chunk, 5);
   if (!abort_flag && tid == 0) {
     tma_store_2d(&tm_tb, sm + kP_TB, 0, unit * kC);
     tma_store_commit();
@@ -465,7 +504,7 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
     tc_commit(bar_mma);
   }
   mbar_wait(bar_mma, 1, ctrl, &abort_flag);
-  GDN_TRACE_POINT(tr, 1, chunk, 6);
+  GDN_TRACE_POINT(tr && chunk < 64, 1, chunk, 6);
   if (tid == 0) tma_store_wait_read();   // the P staging lies under the W staging
   tc_fence_after();
   __syncthreads();
@@ -520,10 +559,11 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
       tma_store_2d(&tm_kt, sm + kP_KST, 0, unit * kD);
       tma_store_commit();
     }
-    GDN_TRACE_POINT(tr, 1, chunk, 7);
-    tma_store_wait_all();
-    GDN_TRACE_POINT(tr, 1, chunk, 8);
+    GDN_TRACE_POINT(tr && chunk < 64, 1, chunk, 7);
   }
+  __syncthreads();   // shared memory and tensor memory free for the next unit
+  }
+  if (tid == 0) tma_store_wait_all();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
@@ -610,12 +650,11 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
   uint8_t *sm = smem_raw;                 // pointer arithmetic keeps the shared space
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n = blockIdx.x, h = blockIdx.y;
-  if (ctrl[0] & kErrBadSeqlens) return;
   if (smem_u32(sm) & 1023) {              // swizzled tiles need a 1024-aligned base
+    grid_dependency_wait();               // the error word is the map kernel's until then
     if (tid == 0) atomicOr(ctrl, kErrLayout);
     return;
   }
-  const int c0 = seq_first[n], nch = seq_first[n + 1] - c0;
   const bool tr = (n == 0 && h == 0);     // traced CTA (GDN_TRACE builds only)
   (void)tr;
 
@@ -665,6 +704,18 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
   // Waits inside the role loops: after an abort they return at once, so every
   // loop runs to its end and named barriers stay in step.
   auto wait = [&](uint64_t *bar, uint32_t parity) { mbar_wait(bar, parity, ctrl, abort_flag); };
+  // The chunk table and the prep kernel's outputs are read only after the
+  // kernels that write them have completed (the chain warps first load the
+  // initial state, which no earlier kernel of this call writes).
+  int c0 = 0, nch = 0;
+  auto read_chunks = [&]() {
+    grid_dependency_wait();
+    if (!(ctrl[0] & kErrBadSeqlens)) {
+      c0 = seq_first[n];
+      nch = seq_first[n + 1] - c0;
+    }
+  };
+  if (warp < 4 || warp >= 12) read_chunks();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -814,6 +865,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
 #pragma unroll
       for (int t = 0; t < 64; ++t) S[t] = src ? src[size_t(64 * hh + t) * kD + i] : 0.f;
     }
+    read_chunks();
     // bf16 copy of S (row i, columns [64 hh, 64 hh + 64)) into tensor memory,
     // then one arrival per warp on s_rdy.
     auto store_state = [&]() {
@@ -1060,19 +1112,37 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kPrepSmem);
     if (e != cudaSuccess) return e;
     prof_record(g_profile.prep, s);
-    gdn_prep_kernel<<<dim3(L.max_chunks, H), kPrepThreads, kPrepSmem, s>>>(
-        mq, mk, mw, mkt, mtb, mpm, g, beta, reinterpret_cast<float *>(base + L.gam), H, ctrl,
-        table);
-    e = cudaGetLastError();
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const long long prep_ctas = std::min<long long>(units, 3LL * sms);
+    // Both kernels start with programmatic dependent launch: their prologues
+    // overlap the tail of the kernel before them.
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(prep_ctas));
+    cfg.blockDim = dim3(kPrepThreads);
+    cfg.dynamicSmemBytes = kPrepSmem;
+    cfg.stream = s;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, gdn_prep_kernel, mq, mk, mw, mkt, mtb, mpm, g, beta,
+                           reinterpret_cast<float *>(base + L.gam), H, ctrl, table);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(gdn_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kScanSmem);
     if (e != cudaSuccess) return e;
     prof_record(g_profile.scan, s);
-    gdn_scan_kernel<<<dim3(N, H), kScanThreads, kScanSmem, s>>>(
-        mq, mv, mw, mkt, mtb, mpm, mgm, mo, s0, sN, static_cast<__nv_bfloat16 *>(o), H, ctrl,
-        table, seq_first);
-    return cudaGetLastError();
+    cfg.gridDim = dim3(N, H);
+    cfg.blockDim = dim3(kScanThreads);
+    cfg.dynamicSmemBytes = kScanSmem;
+    return cudaLaunchKernelEx(&cfg, gdn_scan_kernel, mq, mv, mw, mkt, mtb, mpm, mgm, mo, s0, sN,
+                              static_cast<__nv_bfloat16 *>(o), H, ctrl,
+                              static_cast<const ChunkInfo *>(table), seq_first);
   }
   // No tokens: the final state is the initial state.
   prof_record(g_profile.prep, s);

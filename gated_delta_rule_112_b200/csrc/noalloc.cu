@@ -54,10 +54,10 @@ extern "C" int gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v
     }
     scratch = g_scratch_addr[dev];
   }
-  // gdn_chunk_fwd validates every argument, and it clears the part of the
-  // scratch that must start at zero (the control block holding the device
-  // error word and the chunk count) on the stream before its kernels run; all
-  // other scratch contents are written before they are read.
+  // gdn_chunk_fwd validates every argument, and its first kernel writes the
+  // control block (the device error word and the chunk count) before the
+  // kernels that read it run; all other scratch contents are written before
+  // they are read.
   return gdn_chunk_fwd(q, k, v, g, beta, initial_state, cu_seqlens, B, T, H, d_k, d_v,
                        num_seqs, chunk, dtype, o, final_state, scratch, kNoAllocScratchBytes,
                        stream);
