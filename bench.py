@@ -196,23 +196,19 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
+    from gated_delta_rule_112_b200 import replicas
+
+    barrier = replicas.barrier
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return replicas.max_over_ranks(x, dev)
 
     pk = peaks()
     stream = torch.cuda.current_stream()
     L = gdn.lib()
 
     # --------------------------------------------------------------- chunked forward
-    inp = make_chunk_inputs(WORKLOAD, seed=1 + rank)
+    inp = make_chunk_inputs(WORKLOAD, seed=replicas.shard_seed(1, rank))
     B, T, H = inp["B"], inp["T"], inp["H"]
     q, k, v, g, beta = (inp[x].to(dev) for x in ("q", "k", "v", "g", "beta"))
     o = torch.empty(B, T, H, 128, dtype=torch.bfloat16, device=dev)
@@ -275,7 +271,7 @@ def main():
     t_prep = [e[1].elapsed_time(e[2]) for e in pev]
     t_scan = [e[2].elapsed_time(e[3]) for e in pev]
     tokens = B * T
-    value = world * tokens / (ms * 1e-3) / 1e6
+    value = replicas.job_rate(tokens, ms, world) / 1e6
 
     alg_bytes = tokens * H * BYTES_PER_TOKEN_HEAD + B * H * 128 * 128 * 4   # + final state
     flops = tokens * H * 2 * (3 * 64 * 128 + 2 * 64 * 128 + 3 * 128 * 128)
@@ -320,7 +316,7 @@ def main():
         torch.cuda.synchronize()
         barrier()
         ms_e2e = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / ke)
-        e2e = {"value": world * tokens / (ms_e2e * 1e-3) / 1e6, "unit": UNIT,
+        e2e = {"value": replicas.job_rate(tokens, ms_e2e, world) / 1e6, "unit": UNIT,
                "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "steps": ke, "api": "gated_delta_rule_112_b200.chunk_fwd (C ABI gdn_chunk_fwd)"}
         del hq, hk, hv, hg, hb, ho, hfs
@@ -331,7 +327,7 @@ def main():
     # --------------------------------------------------------------- decode step
     decode = None
     if not args.no_decode:
-        d = make_decode_inputs("decode", seed=4 + rank)
+        d = make_decode_inputs("decode", seed=replicas.shard_seed(4, rank))
         N, Hd, S = d["N"], d["H"], d["steps"]
         dq, dk, dvv, dg, db = (d[x].to(dev) for x in ("q", "k", "v", "g", "beta"))
         st = d["state"].to(dev)
