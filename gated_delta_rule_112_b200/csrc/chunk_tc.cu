@@ -607,6 +607,13 @@ constexpr uint32_t kT_S = 384;    // S        bf16 [128][128] (64 columns)
 constexpr uint32_t kT_A1 = 448;   // V_new^T  bf16 [128][64]  (32 columns)
 // Named barriers (0 is __syncthreads)
 constexpr uint32_t kBarOut = 2;
+// The chain warps hand each finished epilogue to the MMA warp through a
+// hardware named barrier (chain warps bar.arrive, the MMA warp bar.sync):
+// kBarA1 after V_new^T is in tensor memory, kBarS after S_{c+1} is. A chain
+// warp cannot arrive twice before the MMA warp syncs once: its next arrival
+// needs an MMA result that the MMA warp only issues after that sync.
+constexpr uint32_t kBarA1 = 3, kBarS = 4;
+constexpr uint32_t kChainHandoff = 8 * 32 + 32;   // 8 chain warps + the MMA warp
 // Barrier slots in the kS_BAR area
 // y_full[b] completes when Y buffer b holds a new chunk; the output warps wait
 // on it, the chain on s_full. (One barrier for both would let a slow output
@@ -616,8 +623,7 @@ constexpr uint32_t kBarOut = 2;
 // part A start while SY(c) and the S epilogue still run.
 constexpr int kB_FULLA = 0, kB_EMPTYA = 2, kB_FULLB = 4, kB_EMPTYB = 6, kB_GFULL = 8,
               kB_GEMPTY = 12, kB_XFULL = 16, kB_SFULL = 17, kB_YFULL = 18, kB_ZFREE = 20,
-              kB_A1RDY = 21, kB_SRDY = 22, kB_DRAIN = 23, kB_COUNT = 24;
-constexpr int kChainWarps = 8;
+              kB_DRAIN = 21, kB_COUNT = 22;
 
 // Warp roles (16 warps). Every role runs its loop with all 32 lanes, so the
 // lanes of a warp wait on barriers together; one lane issues TMA copies,
@@ -627,8 +633,8 @@ constexpr int kChainWarps = 8;
 //   warps 4-11    state chain: two warpgroups, warpgroup h owns columns
 //                 [32h, 32h+32) of V_new and [64h, 64h+64) of S; thread =
 //                 TMEM lane = row i of d_v; the fp32 S lives in its registers,
-//                 its bf16 copy (an MMA operand) in tensor memory. Each warp
-//                 reports a finished epilogue with one mbarrier arrival.
+//                 its bf16 copy (an MMA operand) in tensor memory. Each finished
+//                 epilogue is handed to the MMA warp through a named barrier.
 //   warps 12-15   output: O = diag(gamma) Z + Y, staged for TMA stores
 // Per chunk c the tensor core runs three wide products:
 //   U(c)   [X|Z]  = V^T [Tb | 0]^T            (4 MMAs, N = 128)  -- before S_c is known
@@ -664,7 +670,6 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
   uint64_t *gfull = bars + kB_GFULL, *gempty = bars + kB_GEMPTY;
   uint64_t *x_full = bars + kB_XFULL, *s_full = bars + kB_SFULL, *y_full = bars + kB_YFULL;
   uint64_t *z_free = bars + kB_ZFREE, *drain = bars + kB_DRAIN;
-  uint64_t *a1_rdy = bars + kB_A1RDY, *s_rdy = bars + kB_SRDY;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kB_COUNT);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -681,7 +686,6 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     for (int b = 0; b < kB_COUNT; ++b) {
       uint32_t count = 1;
       if (b >= kB_GEMPTY && b < kB_GEMPTY + 4) count = 2;        // MMA warp + output
-      if (b == kB_A1RDY || b == kB_SRDY) count = kChainWarps;
       mbar_init(bars + b, count);
     }
     fence_mbar_init();
@@ -805,14 +809,14 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     if (nch > 0) {
       wait(full_a, 0);
       issue_u(0);
-      wait(s_rdy, 0);                     // S_0 stored
-      issue_xz(0);
     }
+    named_bar_sync(kBarS, kChainHandoff);     // S_0 stored (the chain hands it over even if nch = 0)
+    if (nch > 0) issue_xz(0);
     for (int c = 0; c < nch; ++c) {
       const int st = c & 1, gs = c & 3;
       const bool more = c + 1 < nch;
       wait(full_b + st, (c >> 1) & 1);    // (D K)^T and P of chunk c (while XZ(c) runs)
-      wait(a1_rdy, c & 1);                // V_new^T of chunk c in tensor memory
+      named_bar_sync(kBarA1, kChainHandoff);  // V_new^T of chunk c in tensor memory
       GDN_TRACE_POINT(tr && issuer, 0, c, 6);
       if (issuer) {
         const uint32_t sb = smem_u32(sm + st * kStageBytes);
@@ -824,6 +828,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
           tc_mma_bf16_ts(d, tmem + kT_A1 + 8 * kk, make_sdesc(sb + kS_BSY + kk * 32, 16, 1024),
                          id_sy, kk > 0);
         tc_commit(s_full);
+        tc_commit(y_full + st);
+        tc_commit(empty_b + st);          // SY(c) was the last reader of part B
         GDN_TRACE_POINT(tr, 0, c, 12);
       }
       __syncwarp();
@@ -836,12 +842,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
         GDN_TRACE_POINT(tr && issuer, 0, c, 14);
         issue_u(c + 1);
       }
-      if (issuer) {
-        tc_commit(y_full + st);           // also covers U(c+1): the output has slack
-        tc_commit(empty_b + st);          // SY(c) was the last reader of part B
-      }
-      __syncwarp();
-      wait(s_rdy, (c + 1) & 1);           // S_{c+1} stored, decay factors of c read
+      named_bar_sync(kBarS, kChainHandoff);   // S_{c+1} stored, decay factors of c read
       GDN_TRACE_POINT(tr && issuer, 0, c, 8);
       if (more) issue_xz(c + 1);
       if (issuer) mbar_arrive(gempty + gs);
@@ -867,7 +868,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     }
     read_chunks();
     // bf16 copy of S (row i, columns [64 hh, 64 hh + 64)) into tensor memory,
-    // then one arrival per warp on s_rdy.
+    // then hand it to the MMA warp.
     auto store_state = [&]() {
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
@@ -878,8 +879,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
       }
       tmem_st_wait();
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_rdy);
+      named_bar_arrive(kBarS, kChainHandoff);
     };
     store_state();
     for (int c = 0; c < nch; ++c) {
@@ -900,8 +900,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
       }
       tmem_st_wait();
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(a1_rdy);
+      named_bar_arrive(kBarA1, kChainHandoff);
       // S <- gamma_last S + dS on columns [64 hh, 64 hh + 64)
       wait(gfull + gs, (c >> 2) & 1);
       const float gl = reinterpret_cast<const float *>(sm + kS_GAM + gs * 512)[kC - 1];
