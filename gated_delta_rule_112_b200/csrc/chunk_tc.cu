@@ -344,12 +344,13 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
     // G = [K; Q] K^T : M = 128 (K rows then Q rows), N = 64, K = 128 (d_k)
     tc_fence_after();
     const uint32_t idesc = make_idesc_bf16(128, 64, 0, 0);
-    const uint32_t kq = smem_u32(sm + kP_KQ);
+    // One descriptor, k steps added to its start-address field (see the scan's
+    // MMA warp): no dependent integer chain between the MMAs.
+    const uint64_t dkq = make_sdesc(smem_u32(sm + kP_KQ), 16, 1024);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
-      const uint32_t off = (kk >> 2) * kTile128x64 + (kk & 3) * 32;
-      tc_mma_bf16(tmem, make_sdesc(kq + off, 16, 1024), make_sdesc(kq + off, 16, 1024), idesc,
-                  kk > 0);
+      const uint64_t d = dkq + uint64_t(((kk >> 2) * kTile128x64 + (kk & 3) * 32) >> 4);
+      tc_mma_bf16(tmem, d, d, idesc, kk > 0);
     }
     tc_commit(bar_mma);
   }
@@ -491,16 +492,17 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
     // W^T    = K^T (T diag(beta gamma))^T : M = 128 (d_k), N = 64, K = 64 -> cols [64, 128)
     // (DK)^T = K^T diag(D)                : M = 128 (d_k), N = 64, K = 64 -> cols [0, 64)
     const uint32_t idesc = make_idesc_bf16(128, 64, 1, 0);
-    const uint32_t kq = smem_u32(sm + kP_KQ), tbg = smem_u32(sm + kP_TBG);
-    const uint32_t dg = smem_u32(sm + kP_DIAG);
+    const uint64_t dkt = make_sdesc(smem_u32(sm + kP_KQ), kTile128x64, 1024);
+    const uint64_t dtbg = make_sdesc(smem_u32(sm + kP_TBG), 16, 1024);
+    const uint64_t ddg = make_sdesc(smem_u32(sm + kP_DIAG), 16, 1024);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      tc_mma_bf16(tmem + 64, make_sdesc(kq + kk * 2048, kTile128x64, 1024),
-                  make_sdesc(tbg + kk * 32, 16, 1024), idesc, kk > 0);
+      tc_mma_bf16(tmem + 64, dkt + uint64_t(kk * 2048 >> 4), dtbg + uint64_t(kk * 32 >> 4), idesc,
+                  kk > 0);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      tc_mma_bf16(tmem, make_sdesc(kq + kk * 2048, kTile128x64, 1024),
-                  make_sdesc(dg + kk * 32, 16, 1024), idesc, kk > 0);
+      tc_mma_bf16(tmem, dkt + uint64_t(kk * 2048 >> 4), ddg + uint64_t(kk * 32 >> 4), idesc,
+                  kk > 0);
     tc_commit(bar_mma);
   }
   mbar_wait(bar_mma, 1, ctrl, &abort_flag);
@@ -776,31 +778,43 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     const uint32_t id_xz = make_idesc_bf16(128, 128, 0, 0);    // S [-W|Q]^T
     const uint32_t id_sy = make_idesc_bf16(128, 192, 0, 0);    // A1 [(DK)^T|P]^T
     const bool issuer = lane == 0;
+    // Shared-memory descriptors of the operand tiles of both stages, built
+    // once: a single issuing thread pays the latency of every dependent
+    // integer op, so rebuilding descriptors between MMAs doubles the issue
+    // time. A k step is added to the start-address field (smem offsets >> 4
+    // stay below 2^14, so the field never carries into the next one).
+    uint64_t dV[kStages], dBU[kStages], dBXZ[kStages], dBSY[kStages];
+#pragma unroll
+    for (int st = 0; st < kStages; ++st) {
+      const uint32_t sb = smem_u32(sm + st * kStageBytes);
+      dV[st] = make_sdesc(sb + kS_V, kTile64x64, 1024);
+      dBU[st] = make_sdesc(sb + kS_BU, 16, 1024);
+      dBXZ[st] = make_sdesc(sb + kS_BXZ, 16, 1024);
+      dBSY[st] = make_sdesc(sb + kS_BSY, 16, 1024);
+    }
     // U(c) into [X|Z]. The caller has seen chunk c loaded and the output
     // warps done reading Z of chunk c - 1.
     auto issue_u = [&](int c) {
-      const uint32_t sb = smem_u32(sm + (c & 1) * kStageBytes);
       if (issuer) {
+        const uint64_t da = (c & 1) ? dV[1] : dV[0], db = (c & 1) ? dBU[1] : dBU[0];
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          tc_mma_bf16(tmem + kT_XZ, make_sdesc(sb + kS_V + kk * 2048, kTile64x64, 1024),
-                      make_sdesc(sb + kS_BU + kk * 32, 16, 1024), id_u, kk > 0);
+          tc_mma_bf16(tmem + kT_XZ, da + uint64_t(kk * 2048 >> 4), db + uint64_t(kk * 32 >> 4),
+                      id_u, kk > 0);
       }
       __syncwarp();
     };
     // XZ(c) += S_c [-W|Q]^T, reading the bf16 copy of S_c.
     auto issue_xz = [&](int c) {
-      const uint32_t sb = smem_u32(sm + (c & 1) * kStageBytes);
       if (issuer) {
         GDN_TRACE_POINT(tr, 0, c, 1);
+        const uint64_t db = (c & 1) ? dBXZ[1] : dBXZ[0];
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           tc_mma_bf16_ts(tmem + kT_XZ, tmem + kT_S + 8 * kk,
-                         make_sdesc(sb + kS_BXZ + (kk >> 2) * kTile128x64 + (kk & 3) * 32, 16,
-                                    1024),
-                         id_xz, 1);
+                         db + uint64_t(((kk >> 2) * kTile128x64 + (kk & 3) * 32) >> 4), id_xz, 1);
         tc_commit(x_full);
         tc_commit(empty_a + (c & 1));     // U(c) and XZ(c) were the last readers of part A
       }
@@ -819,14 +833,13 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
       named_bar_sync(kBarA1, kChainHandoff);  // V_new^T of chunk c in tensor memory
       GDN_TRACE_POINT(tr && issuer, 0, c, 6);
       if (issuer) {
-        const uint32_t sb = smem_u32(sm + st * kStageBytes);
+        const uint64_t db = st ? dBSY[1] : dBSY[0];
         tc_fence_after();
         // even chunks: D = [dS | Y0] at kT_DS; odd: D = [Y1 | dS] at kT_Y1
         const uint32_t d = tmem + (st ? kT_Y1 : kT_DS);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          tc_mma_bf16_ts(d, tmem + kT_A1 + 8 * kk, make_sdesc(sb + kS_BSY + kk * 32, 16, 1024),
-                         id_sy, kk > 0);
+          tc_mma_bf16_ts(d, tmem + kT_A1 + 8 * kk, db + uint64_t(kk * 32 >> 4), id_sy, kk > 0);
         tc_commit(s_full);
         tc_commit(y_full + st);
         tc_commit(empty_b + st);          // SY(c) was the last reader of part B
