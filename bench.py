@@ -45,6 +45,9 @@ def parse_args():
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--workload", default=WORKLOAD,
+                   help="chunked-forward workload (inputs.WORKLOADS); the default is the "
+                        "headline configuration, the others are for extra measurements")
     return p.parse_args()
 
 
@@ -141,14 +144,18 @@ def run_reference(args):
     import numpy as np
     import oracle
     from gated_delta_rule_112_b200.inputs import make_chunk_inputs
-    inp = make_chunk_inputs(WORKLOAD)
+    inp = make_chunk_inputs(args.workload)
     heads = [0, 1]                              # sample: 2 of 16 heads, all B*T tokens
     arr = {k: inp[k][:, :, heads].float().double().numpy() for k in ("q", "k", "v", "g", "beta")}
     cores = oracle.default_threads()
     tok_equiv = inp["B"] * inp["T"] * len(heads) / inp["H"]
 
+    s0 = (inp["initial_state"][:, heads].double().numpy()
+          if inp["initial_state"] is not None else None)
+    cu = inp["cu_seqlens"].numpy() if inp["cu_seqlens"] is not None else None
+
     def one():
-        oracle.chunk_fwd(arr["q"], arr["k"], arr["v"], arr["g"], arr["beta"], None, None,
+        oracle.chunk_fwd(arr["q"], arr["k"], arr["v"], arr["g"], arr["beta"], s0, cu,
                          nthreads=cores)
     for _ in range(args.warmup):
         one()
@@ -163,7 +170,7 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "B": inp["B"], "T": inp["T"], "H": inp["H"],
+            "config": {"workload": args.workload, "B": inp["B"], "T": inp["T"], "H": inp["H"],
                        "d_k": 128, "d_v": 128, "chunk": 64},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": sample},
@@ -208,16 +215,23 @@ def main():
     L = gdn.lib()
 
     # --------------------------------------------------------------- chunked forward
-    inp = make_chunk_inputs(WORKLOAD, seed=replicas.shard_seed(1, rank))
+    from gated_delta_rule_112_b200.inputs import WORKLOADS
+    wl = args.workload
+    seed = replicas.shard_seed(WORKLOADS[wl].seed, rank)
+    inp = make_chunk_inputs(wl, seed=seed)
     B, T, H = inp["B"], inp["T"], inp["H"]
     q, k, v, g, beta = (inp[x].to(dev) for x in ("q", "k", "v", "g", "beta"))
+    s0 = inp["initial_state"].to(dev) if inp["initial_state"] is not None else None
+    cu = inp["cu_seqlens"].to(dev) if inp["cu_seqlens"] is not None else None
+    nseq = B if cu is None else cu.numel() - 1
     o = torch.empty(B, T, H, 128, dtype=torch.bfloat16, device=dev)
-    fs = torch.empty(B, H, 128, 128, dtype=torch.float32, device=dev)
-    ws = torch.empty(gdn.workspace_size(B, T, H, 128, 128), dtype=torch.uint8, device=dev)
+    fs = torch.empty(nseq, H, 128, 128, dtype=torch.float32, device=dev)
+    ws = torch.empty(gdn.workspace_size(B, T, H, 128, 128, 0 if cu is None else nseq),
+                     dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def step():
-        gdn.chunk_fwd(q, k, v, g, beta, None, None, out=o, workspace=ws)
+        gdn.chunk_fwd(q, k, v, g, beta, s0, cu, out=o, workspace=ws)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -273,7 +287,8 @@ def main():
     tokens = B * T
     value = replicas.job_rate(tokens, ms, world) / 1e6
 
-    alg_bytes = tokens * H * BYTES_PER_TOKEN_HEAD + B * H * 128 * 128 * 4   # + final state
+    state_io = (2 if s0 is not None else 1) * nseq * H * 128 * 128 * 4   # final (+ initial) state
+    alg_bytes = tokens * H * BYTES_PER_TOKEN_HEAD + state_io
     flops = tokens * H * 2 * (3 * 64 * 128 + 2 * 64 * 128 + 3 * 128 * 128)
     ach_gbs = alg_bytes / (ms_local * 1e-3) / 1e9
     kernels = {
@@ -282,7 +297,7 @@ def main():
         "gdn_scan_kernel": statistics.mean(t_scan),
     }
     tot = sum(kernels.values())
-    traffic = recorded_traffic("chunk_fwd_step/" + WORKLOAD)
+    traffic = recorded_traffic("chunk_fwd_step/" + wl)
 
     # --------------------------------------------------------------- end to end (host buffers)
     e2e = None
@@ -296,7 +311,7 @@ def main():
         def e2e_step_with_state():
             for dst, src in ((q, hq), (k, hk), (v, hv), (g, hg), (beta, hb)):
                 dst.copy_(src, non_blocking=True)
-            _, f = gdn.chunk_fwd(q, k, v, g, beta, None, None, out=o, workspace=ws)
+            _, f = gdn.chunk_fwd(q, k, v, g, beta, s0, cu, out=o, workspace=ws)
             ho.copy_(o, non_blocking=True)
             hfs.copy_(f, non_blocking=True)
 
@@ -379,8 +394,10 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "B": B, "T": T, "H": H, "d_k": 128, "d_v": 128,
-                   "chunk": 64, "initial_state": "zeros", "final_state": True,
+        "config": {"workload": wl, "B": B, "T": T, "H": H, "d_k": 128, "d_v": 128,
+                   "chunk": 64, "sequences": nseq,
+                   "initial_state": "zeros" if s0 is None else "random",
+                   "final_state": True,
                    "l2": "flushed before every timed step (256 MiB device write)",
                    "parallelism": f"{world} independent replica(s), no collective"},
         "roofline": {"bound": "hbm", "achieved": ach_gbs, "peak": pk["hbm"], "unit": "GB/s",

@@ -24,7 +24,7 @@ namespace {
 __global__ void __launch_bounds__(1024) gdn_chunk_map_kernel(
     const int32_t *__restrict__ cu, int B, int T, int num_seqs, int chunk,
     uint32_t *__restrict__ ctrl, ChunkInfo *__restrict__ table,
-    int32_t *__restrict__ seq_first, int max_chunks) {
+    int32_t *__restrict__ seq_first, int max_chunks, int segs, int32_t *__restrict__ seg_first) {
   // The kernels launched after this one may start their prologues now; they
   // wait for this grid before reading what it writes.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -44,6 +44,14 @@ __global__ void __launch_bounds__(1024) gdn_chunk_map_kernel(
       table[idx] = ci;
     }
     for (int n = tid; n <= N; n += blockDim.x) seq_first[n] = n * cps;
+    if (segs > 1) {
+      // segment g of sequence n: chunks [n cps + g len, min(n cps + (g + 1) len, (n + 1) cps))
+      const int len = (cps + segs - 1) / segs;
+      for (int e = tid; e <= N * segs; e += blockDim.x) {
+        const int n = e / segs, gi = e - n * segs;
+        seg_first[e] = (n >= N) ? N * cps : n * cps + min(gi * len, cps);
+      }
+    }
     if (tid == 0) {
       ctrl[0] = 0;
       ctrl[1] = uint32_t(total);
@@ -308,7 +316,8 @@ cudaError_t launch_chunk_map(const int32_t *cu_seqlens, int B, int T, int num_se
   gdn_chunk_map_kernel<<<1, 1024, 0, s>>>(
       cu_seqlens, B, T, num_seqs, chunk, reinterpret_cast<uint32_t *>(base),
       reinterpret_cast<ChunkInfo *>(base + L.chunk_table),
-      reinterpret_cast<int32_t *>(base + L.seq_first), L.max_chunks);
+      reinterpret_cast<int32_t *>(base + L.seq_first), L.max_chunks, L.segs,
+      L.segs > 1 ? reinterpret_cast<int32_t *>(base + L.seg_first) : nullptr);
   return cudaGetLastError();
 }
 

@@ -653,11 +653,19 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     const __grid_constant__ CUtensorMap tm_gam, const __grid_constant__ CUtensorMap tm_o,
     const float *__restrict__ s0, float *__restrict__ sN, __nv_bfloat16 *__restrict__ o, int H,
     uint32_t *__restrict__ ctrl, const ChunkInfo *__restrict__ table,
-    const int32_t *__restrict__ seq_first) {
+    const int32_t *__restrict__ seq_first, int split, float *__restrict__ sN_trans,
+    int sN_group) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *sm = smem_raw;                 // pointer arithmetic keeps the shared space
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n = blockIdx.x, h = blockIdx.y;
+  // Sequences (or segments of sequences) n = blockIdx.x. With split > 0, the
+  // CTAs from `split` on run segment n = blockIdx.x - split as a transition:
+  // V = 0 (no U product) from S = I, writing the resulting state to sN_trans.
+  // o == nullptr: no output is written. The final state of n goes to
+  // sN[n / sN_group] when n % sN_group == sN_group - 1 (sN_group = 1: every n).
+  const bool trans = split > 0 && int(blockIdx.x) >= split;
+  const int n = trans ? int(blockIdx.x) - split : int(blockIdx.x), h = blockIdx.y;
+  const bool write_o = o != nullptr;
   if (smem_u32(sm) & 1023) {              // swizzled tiles need a 1024-aligned base
     grid_dependency_wait();               // the error word is the map kernel's until then
     if (tid == 0) atomicOr(ctrl, kErrLayout);
@@ -733,21 +741,32 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
       if (c >= 2) wait(empty_a + st, ((c >> 1) - 1) & 1);
       if (lane == 0) {
         GDN_TRACE_POINT(tr, 0, c, 0);
-        mbar_arrive_expect_tx(full_a + st, kStageTxA);
+        // Only what this CTA's products read: a run without output needs
+        // neither Q nor P, a transition run neither V nor T diag(beta).
+        mbar_arrive_expect_tx(full_a + st, (write_o ? kStageTxA : kStageTxA - kTile128x64) -
+                                               (trans ? 2 * kTile64x64 + kTile64x64 : 0u));
         tma_load_2d(sb + kS_BXZ, &tm_w, full_a + st, 0, unit * kC);
-        tma_load_3d(sb + kS_BXZ + kTile64x64, &tm_q, full_a + st, 0, h, ci.row0);
         tma_load_2d(sb + kS_BXZ + kTile128x64, &tm_w, full_a + st, 64, unit * kC);
-        tma_load_3d(sb + kS_BXZ + kTile128x64 + kTile64x64, &tm_q, full_a + st, 64, h, ci.row0);
-        tma_load_3d(sb + kS_V, &tm_v, full_a + st, 0, h, ci.row0);
-        tma_load_3d(sb + kS_V + kTile64x64, &tm_v, full_a + st, 64, h, ci.row0);
-        tma_load_2d(sb + kS_BU, &tm_tb, full_a + st, 0, unit * kC);
+        if (write_o) {
+          tma_load_3d(sb + kS_BXZ + kTile64x64, &tm_q, full_a + st, 0, h, ci.row0);
+          tma_load_3d(sb + kS_BXZ + kTile128x64 + kTile64x64, &tm_q, full_a + st, 64, h,
+                      ci.row0);
+        }
+        if (!trans) {
+          tma_load_3d(sb + kS_V, &tm_v, full_a + st, 0, h, ci.row0);
+          tma_load_3d(sb + kS_V + kTile64x64, &tm_v, full_a + st, 64, h, ci.row0);
+          tma_load_2d(sb + kS_BU, &tm_tb, full_a + st, 0, unit * kC);
+        }
       }
       __syncwarp();
       if (c >= 2) wait(empty_b + st, ((c >> 1) - 1) & 1);
       if (lane == 0) {
-        mbar_arrive_expect_tx(full_b + st, kStageTxB);
-        tma_load_2d(sb + kS_BSY + (st ? kTile64x64 : 0u), &tm_kt, full_b + st, 0, unit * kD);
-        tma_load_2d(sb + kS_BSY + (st ? 0u : kTile128x64), &tm_pm, full_b + st, 0, unit * kC);
+        // Without output, (D K)^T goes first in both stages and P is not loaded.
+        const bool swap = st && write_o;
+        mbar_arrive_expect_tx(full_b + st, write_o ? kStageTxB : kTile128x64);
+        tma_load_2d(sb + kS_BSY + (swap ? kTile64x64 : 0u), &tm_kt, full_b + st, 0, unit * kD);
+        if (write_o)
+          tma_load_2d(sb + kS_BSY + (st ? 0u : kTile128x64), &tm_pm, full_b + st, 0, unit * kC);
         // The loads above take about one chunk period to land from HBM; the
         // chunk after next goes to L2 now, so its own loads come from L2.
         if (c + kPrefetchAhead < nch) {
@@ -755,13 +774,17 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
           const int up = (c0 + c + kPrefetchAhead) * H + h;
           tma_prefetch_l2_2d(&tm_w, 0, up * kC);
           tma_prefetch_l2_2d(&tm_w, 64, up * kC);
-          tma_prefetch_l2_3d(&tm_q, 0, h, cp.row0);
-          tma_prefetch_l2_3d(&tm_q, 64, h, cp.row0);
-          tma_prefetch_l2_3d(&tm_v, 0, h, cp.row0);
-          tma_prefetch_l2_3d(&tm_v, 64, h, cp.row0);
-          tma_prefetch_l2_2d(&tm_tb, 0, up * kC);
           tma_prefetch_l2_2d(&tm_kt, 0, up * kD);
-          tma_prefetch_l2_2d(&tm_pm, 0, up * kC);
+          if (write_o) {
+            tma_prefetch_l2_3d(&tm_q, 0, h, cp.row0);
+            tma_prefetch_l2_3d(&tm_q, 64, h, cp.row0);
+            tma_prefetch_l2_2d(&tm_pm, 0, up * kC);
+          }
+          if (!trans) {
+            tma_prefetch_l2_3d(&tm_v, 0, h, cp.row0);
+            tma_prefetch_l2_3d(&tm_v, 64, h, cp.row0);
+            tma_prefetch_l2_2d(&tm_tb, 0, up * kC);
+          }
         }
       }
       __syncwarp();
@@ -774,9 +797,11 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    const uint32_t id_u = make_idesc_bf16(128, 128, 1, 0);     // V^T [Tb|0]^T : A MN-major
-    const uint32_t id_xz = make_idesc_bf16(128, 128, 0, 0);    // S [-W|Q]^T
-    const uint32_t id_sy = make_idesc_bf16(128, 192, 0, 0);    // A1 [(DK)^T|P]^T
+    // Without output, Z and Y are not needed: U and XZ shrink to X (N = 64),
+    // SY to dS (N = 128, (D K)^T then first in both stages).
+    const uint32_t id_u = make_idesc_bf16(128, write_o ? 128 : 64, 1, 0);   // V^T [Tb|0]^T
+    const uint32_t id_xz = make_idesc_bf16(128, write_o ? 128 : 64, 0, 0);  // S [-W|Q]^T
+    const uint32_t id_sy = make_idesc_bf16(128, write_o ? 192 : 128, 0, 0); // A1 [(DK)^T|P]^T
     const bool issuer = lane == 0;
     // Shared-memory descriptors of the operand tiles of both stages, built
     // once: a single issuing thread pays the latency of every dependent
@@ -812,9 +837,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
         const uint64_t db = (c & 1) ? dBXZ[1] : dBXZ[0];
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
+        for (int kk = 0; kk < 8; ++kk)   // a transition run has no U: XZ starts the sum
           tc_mma_bf16_ts(tmem + kT_XZ, tmem + kT_S + 8 * kk,
-                         db + uint64_t(((kk >> 2) * kTile128x64 + (kk & 3) * 32) >> 4), id_xz, 1);
+                         db + uint64_t(((kk >> 2) * kTile128x64 + (kk & 3) * 32) >> 4), id_xz,
+                         (kk > 0) || !trans);
         tc_commit(x_full);
         tc_commit(empty_a + (c & 1));     // U(c) and XZ(c) were the last readers of part A
       }
@@ -822,7 +848,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     };
     if (nch > 0) {
       wait(full_a, 0);
-      issue_u(0);
+      if (!trans) issue_u(0);
     }
     named_bar_sync(kBarS, kChainHandoff);     // S_0 stored (the chain hands it over even if nch = 0)
     if (nch > 0) issue_xz(0);
@@ -836,7 +862,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
         const uint64_t db = st ? dBSY[1] : dBSY[0];
         tc_fence_after();
         // even chunks: D = [dS | Y0] at kT_DS; odd: D = [Y1 | dS] at kT_Y1
-        const uint32_t d = tmem + (st ? kT_Y1 : kT_DS);
+        // (without output: D = dS at kT_DS for every chunk)
+        const uint32_t d = tmem + ((st && write_o) ? kT_Y1 : kT_DS);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           tc_mma_bf16_ts(d, tmem + kT_A1 + 8 * kk, db + uint64_t(kk * 32 >> 4), id_sy, kk > 0);
@@ -853,7 +880,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
         GDN_TRACE_POINT(tr && issuer, 0, c, 13);
         wait(full_a + (st ^ 1), ((c + 1) >> 1) & 1);
         GDN_TRACE_POINT(tr && issuer, 0, c, 14);
-        issue_u(c + 1);
+        if (!trans) issue_u(c + 1);
       }
       named_bar_sync(kBarS, kChainHandoff);   // S_{c+1} stored, decay factors of c read
       GDN_TRACE_POINT(tr && issuer, 0, c, 8);
@@ -875,9 +902,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     (void)tl;
     float S[64];                                        // S[i][64 hh + t], fp32 master
     {
-      const float *src = s0 ? s0 + (size_t(n) * H + h) * kD * kD : nullptr;
+      const float *src = (s0 && !trans) ? s0 + (size_t(n) * H + h) * kD * kD : nullptr;
 #pragma unroll
-      for (int t = 0; t < 64; ++t) S[t] = src ? src[size_t(64 * hh + t) * kD + i] : 0.f;
+      for (int t = 0; t < 64; ++t)
+        S[t] = trans ? (64 * hh + t == i ? 1.f : 0.f) : (src ? src[size_t(64 * hh + t) * kD + i] : 0.f);
     }
     read_chunks();
     // bf16 copy of S (row i, columns [64 hh, 64 hh + 64)) into tensor memory,
@@ -938,8 +966,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
       GDN_TRACE_POINT(tl, 0, c, 4);
       GDN_TRACE_POINT(tr && warp == 11 && lane == 0, 0, c, 15);
     }
-    if (sN && !*abort_flag) {
-      float *dst = sN + (size_t(n) * H + h) * kD * kD;
+    float *sNp = trans ? sN_trans : sN;
+    const int sN_idx = trans ? n : n / sN_group;
+    if (sNp && (trans || n % sN_group == sN_group - 1) && !*abort_flag) {
+      float *dst = sNp + (size_t(sN_idx) * H + h) * kD * kD;
 #pragma unroll
       for (int t = 0; t < 64; ++t) dst[size_t(64 * hh + t) * kD + i] = S[t];
     }
@@ -957,7 +987,16 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     const uint32_t ost = smem_u32(sm + kS_OST);
     const int fc = 2 * (lane & 3);                     // fragment column pair
     const int mj = lane & 7, mm = lane >> 3;           // stmatrix: row j of matrix m
-    for (int c = 0; c < nch; ++c) {
+    for (int c = 0; c < nch && !write_o; ++c) {
+      // No output: keep only this role's side of the barrier protocol.
+      const int gs = c & 3;
+      wait(x_full, c & 1);
+      if (leader) mbar_arrive(z_free);
+      wait(gfull + gs, (c >> 2) & 1);
+      if (leader) mbar_arrive(gempty + gs);
+      __syncwarp();
+    }
+    for (int c = 0; c < nch && write_o; ++c) {
       const int gs = c & 3;
       const float *gam = reinterpret_cast<const float *>(sm + kS_GAM + gs * 512);
       const ChunkInfo ci = table[c0 + c];
@@ -1044,6 +1083,61 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// ============================================================ segment composition
+// For a sequence whose state scan was split into `segs` segments: the first
+// pass gave each segment's state from S = 0 (H_g, in hbuf) and its transition
+// (the state from S = I with V = 0, P_g, in pbuf), so S_{g+1} = S_g P_g + H_g
+// (the chunk map S -> S (gamma_last I - W^T D K) + U^T D K is affine in S).
+// In the stored orientation X = S^T ([d_k][d_v]) that is X_{g+1} = P~_g X_g +
+// H~_g, where P~_g is pbuf's stored matrix. Every column of X evolves alone,
+// so one CTA owns 16 columns of one (sequence, head); fp32 throughout.
+// Writes X_g, the start state of segment g, to sstart.
+__global__ void __launch_bounds__(256) gdn_segment_combine_kernel(
+    const float *__restrict__ s0, const float *__restrict__ hbuf,
+    const float *__restrict__ pbuf, float *__restrict__ sstart, int H, int segs,
+    const uint32_t *__restrict__ ctrl) {
+  __shared__ __align__(16) float X[kD][16];
+  const int b = blockIdx.x / H, h = blockIdx.x - b * H, col0 = 16 * blockIdx.y;
+  const int tid = threadIdx.x;
+  if (ctrl[0] & kErrBadSeqlens) return;
+  for (int e = tid; e < kD * 16; e += blockDim.x) {
+    const int j = e >> 4, c = e & 15;
+    X[j][c] = s0 ? s0[((size_t(b) * H + h) * kD + j) * kD + col0 + c] : 0.f;
+  }
+  __syncthreads();
+  const int j = tid >> 1, c0 = (tid & 1) * 8;   // this thread's row and 8 columns
+  for (int gi = 0; gi < segs; ++gi) {
+    const size_t base = ((size_t(b) * segs + gi) * H + h) * kD * kD;
+    float4 *dst = reinterpret_cast<float4 *>(sstart + base + size_t(j) * kD + col0 + c0);
+    dst[0] = *reinterpret_cast<const float4 *>(&X[j][c0]);
+    dst[1] = *reinterpret_cast<const float4 *>(&X[j][c0 + 4]);
+    if (gi == segs - 1) break;
+    const float4 h0 = *reinterpret_cast<const float4 *>(hbuf + base + size_t(j) * kD + col0 + c0);
+    const float4 h1 =
+        *reinterpret_cast<const float4 *>(hbuf + base + size_t(j) * kD + col0 + c0 + 4);
+    float acc[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+    const float4 *prow = reinterpret_cast<const float4 *>(pbuf + base + size_t(j) * kD);
+#pragma unroll 4
+    for (int m4 = 0; m4 < kD / 4; ++m4) {
+      const float4 p = prow[m4];
+      const float pv[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float4 xa = *reinterpret_cast<const float4 *>(&X[4 * m4 + e][c0]);
+        const float4 xb = *reinterpret_cast<const float4 *>(&X[4 * m4 + e][c0 + 4]);
+        acc[0] = fmaf(pv[e], xa.x, acc[0]); acc[1] = fmaf(pv[e], xa.y, acc[1]);
+        acc[2] = fmaf(pv[e], xa.z, acc[2]); acc[3] = fmaf(pv[e], xa.w, acc[3]);
+        acc[4] = fmaf(pv[e], xb.x, acc[4]); acc[5] = fmaf(pv[e], xb.y, acc[5]);
+        acc[6] = fmaf(pv[e], xb.z, acc[6]); acc[7] = fmaf(pv[e], xb.w, acc[7]);
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < 8; ++e) X[j][c0 + e] = acc[e];
+    __syncthreads();
   }
 }
 
@@ -1149,12 +1243,42 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
                              kScanSmem);
     if (e != cudaSuccess) return e;
     prof_record(g_profile.scan, s);
-    cfg.gridDim = dim3(N, H);
     cfg.blockDim = dim3(kScanThreads);
     cfg.dynamicSmemBytes = kScanSmem;
-    return cudaLaunchKernelEx(&cfg, gdn_scan_kernel, mq, mv, mw, mkt, mtb, mpm, mgm, mo, s0, sN,
+    if (L.segs <= 1) {
+      cfg.gridDim = dim3(N, H);
+      return cudaLaunchKernelEx(&cfg, gdn_scan_kernel, mq, mv, mw, mkt, mtb, mpm, mgm, mo, s0,
+                                sN, static_cast<__nv_bfloat16 *>(o), H, ctrl,
+                                static_cast<const ChunkInfo *>(table), seq_first, 0,
+                                static_cast<float *>(nullptr), 1);
+    }
+    // Segmented state scan (few long sequences): three passes over B * segs
+    // segments. (1) every segment from S = 0 and as a transition, no output;
+    // (2) the segments' start states; (3) every segment from its start state,
+    // writing o and, for each sequence's last segment, the final state.
+    const int nseg = B * L.segs;
+    const int32_t *seg_first = reinterpret_cast<const int32_t *>(base + L.seg_first);
+    float *hbuf = reinterpret_cast<float *>(base + L.hbuf);
+    float *pbuf = reinterpret_cast<float *>(base + L.pbuf);
+    float *sstart = reinterpret_cast<float *>(base + L.sstart);
+    cfg.gridDim = dim3(2 * nseg, H);
+    e = cudaLaunchKernelEx(&cfg, gdn_scan_kernel, mq, mv, mw, mkt, mtb, mpm, mgm, mo,
+                           static_cast<const float *>(nullptr), hbuf,
+                           static_cast<__nv_bfloat16 *>(nullptr), H, ctrl,
+                           static_cast<const ChunkInfo *>(table), seg_first, nseg, pbuf, 1);
+    if (e != cudaSuccess) return e;
+    gdn_segment_combine_kernel<<<dim3(B * H, kD / 16), 256, 0, s>>>(s0, hbuf, pbuf, sstart, H,
+                                                                   L.segs, ctrl);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    // A plain launch: the start states come from the kernel just before it.
+    cfg.gridDim = dim3(nseg, H);
+    cfg.numAttrs = 0;
+    return cudaLaunchKernelEx(&cfg, gdn_scan_kernel, mq, mv, mw, mkt, mtb, mpm, mgm, mo,
+                              static_cast<const float *>(sstart), sN,
                               static_cast<__nv_bfloat16 *>(o), H, ctrl,
-                              static_cast<const ChunkInfo *>(table), seq_first);
+                              static_cast<const ChunkInfo *>(table), seg_first, 0,
+                              static_cast<float *>(nullptr), L.segs);
   }
   // No tokens: the final state is the initial state.
   prof_record(g_profile.prep, s);

@@ -8,6 +8,14 @@
 using namespace gdn;
 
 namespace gdn {
+
+int device_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return sms;
+}
+
 ProfileEvents g_profile = {nullptr, nullptr, nullptr, nullptr};
 }
 
@@ -49,7 +57,8 @@ int run_chunk(bool force_simt, const void *q, const void *k, const void *v, cons
                             o, sN, ws);
   if (rc != GDN_OK) return rc;
   const bool tc = !force_simt && tc_path(dk, dv, chunk, dtype);
-  const WsLayout L = ws_layout(B, T, H, cu ? num_seqs : 0, chunk, tc);
+  const int segs = scan_segments(B, T, H, cu ? num_seqs : 0, chunk, tc, device_sms());
+  const WsLayout L = ws_layout(B, T, H, cu ? num_seqs : 0, chunk, tc, segs);
   if (ws_bytes < L.total) return GDN_ERR_WORKSPACE;
   const int N = cu ? num_seqs : B;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -76,7 +85,16 @@ size_t gdn_chunk_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int n
                                     int chunk, int dtype) {
   if (B < 1 || T < 0 || H < 1 || d_k < 1 || d_v < 1 || num_seqs < 0) return 0;
   if (chunk != 16 && chunk != 32 && chunk != 64) return 0;
-  return ws_layout(B, T, H, num_seqs, chunk, tc_path(d_k, d_v, chunk, dtype)).total;
+  const bool tc = tc_path(d_k, d_v, chunk, dtype);
+  return ws_layout(B, T, H, num_seqs, chunk, tc,
+                   scan_segments(B, T, H, num_seqs, chunk, tc, device_sms()))
+      .total;
+}
+
+int gdn_chunk_fwd_scan_segments(int B, int T, int H, int d_k, int d_v, int num_seqs, int chunk,
+                                int dtype, int sms) {
+  if (B < 0 || T < 0 || H < 0 || num_seqs < 0 || sms < 0) return 1;
+  return scan_segments(B, T, H, num_seqs, chunk, tc_path(d_k, d_v, chunk, dtype), sms);
 }
 
 int gdn_chunk_fwd_path(int d_k, int d_v, int chunk, int dtype) {

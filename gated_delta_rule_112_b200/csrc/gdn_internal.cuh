@@ -31,9 +31,14 @@ struct ChunkInfo {
 //   tb             bf16 [units][64][64]          T diag(beta) of the chunk (UT transform)
 //   pm             bf16 [units][64][64]          (Q K^T) .* decay mask, diagonal included
 //   gam            fp32 [units][128]             exp(Gamma_c) (64), then exp(Gamma_last - Gamma_s) (64)
+//   tensor-core path with a segmented state scan (segs > 1, see scan_segments):
+//   seg_first      int32[B * segs + 1]  first chunk of each segment
+//   hbuf, pbuf     fp32 [B * segs][H][d_k][d_v]  each segment's state from S = 0,
+//                  and its transition (the state from S = I with V = 0)
+//   sstart         fp32 [B * segs][H][d_k][d_v]  each segment's true start state
 struct WsLayout {
-  size_t chunk_table, seq_first, w, kt, tb, pm, gam, total;
-  int max_chunks;
+  size_t chunk_table, seq_first, w, kt, tb, pm, gam, seg_first, hbuf, pbuf, sstart, total;
+  int max_chunks, segs;
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -43,10 +48,41 @@ inline int max_chunks_for(int B, int T, int num_seqs, int chunk) {
   return int(int64_t(B) * ((int64_t(T) + chunk - 1) / chunk));
 }
 
-inline WsLayout ws_layout(int B, int T, int H, int num_seqs, int chunk, bool tc) {
+// Segments per sequence for the tensor-core state scan. The scan is a chain
+// of dependent chunks per (sequence, head), one CTA each; with few chains and
+// many chunks most SMs idle. Split into G segments, the chain runs as three
+// passes of T / G chunks: every segment from S = 0 and, with V = 0, from
+// S = I (its affine map S -> S P_g + H_g), a short fp32 composition of the
+// segments' start states, and every segment again from its true start. G is
+// chosen by counting chunk periods on `sms` SMs (one CTA per SM); 1 means one
+// plain pass. Only for B sequences of equal length (no cu_seqlens).
+constexpr int kMaxScanSegments = 16;
+inline int scan_segments(int B, int T, int H, int num_seqs, int chunk, bool tc, int sms) {
+  if (!tc || num_seqs > 0 || B <= 0 || T <= 0 || H <= 0 || sms <= 0) return 1;
+  const long long cps = (int64_t(T) + chunk - 1) / chunk;
+  const long long chains = int64_t(B) * H;
+  auto waves = [&](long long ctas) { return (ctas + sms - 1) / sms; };
+  const long long plain = waves(chains) * cps;
+  int best = 1;
+  long long best_cost = plain;
+  for (int G = 2; G <= kMaxScanSegments && G <= cps; ++G) {
+    const long long len = (cps + G - 1) / G;
+    const long long g = (cps + len - 1) / len;            // non-empty segments
+    // + 8 chunk periods for the composition kernel and the extra launches
+    const long long cost = (waves(2 * chains * g) + waves(chains * g)) * len + 8;
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = int(g);
+    }
+  }
+  return (best > 1 && best_cost * 10 <= plain * 7) ? best : 1;   // at least 30 % faster
+}
+
+inline WsLayout ws_layout(int B, int T, int H, int num_seqs, int chunk, bool tc, int segs = 1) {
   WsLayout L{};
   const int N = num_seqs > 0 ? num_seqs : B;
   L.max_chunks = max_chunks_for(B, T, num_seqs, chunk);
+  L.segs = segs;
   size_t off = 256;
   L.chunk_table = off;
   off = align_up(off + sizeof(ChunkInfo) * size_t(L.max_chunks > 0 ? L.max_chunks : 1), 256);
@@ -59,6 +95,14 @@ inline WsLayout ws_layout(int B, int T, int H, int num_seqs, int chunk, bool tc)
     L.tb = off;  off = align_up(off + units * 64 * 64 * 2, 1024);
     L.pm = off;  off = align_up(off + units * 64 * 64 * 2, 1024);
     L.gam = off; off = align_up(off + units * 128 * 4, 1024);
+    if (segs > 1) {
+      const size_t nseg = size_t(B) * segs;
+      const size_t states = nseg * H * 128 * 128 * sizeof(float);
+      L.seg_first = off; off = align_up(off + sizeof(int32_t) * (nseg + 1), 1024);
+      L.hbuf = off;      off = align_up(off + states, 1024);
+      L.pbuf = off;      off = align_up(off + states, 1024);
+      L.sstart = off;    off = align_up(off + states, 1024);
+    }
   }
   L.total = off;
   return L;
@@ -77,6 +121,8 @@ inline void prof_record(cudaEvent_t e, cudaStream_t s) {
 // Kernel launchers (defined in the .cu files; return a cudaError_t).
 cudaError_t launch_chunk_map(const int32_t *cu_seqlens, int B, int T, int num_seqs, int chunk,
                              void *ws, const WsLayout &L, cudaStream_t s);
+// Streaming multiprocessors of the current device (0 if it cannot be read).
+int device_sms();
 cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const float *g,
                               const float *beta, const float *s0, const int32_t *cu, int B,
                               int T, int H, int dk, int dv, int N, int chunk, int dtype, void *o,

@@ -63,6 +63,9 @@ extern "C" {
  * packed sequences (num_seqs > 0) it assumes the worst case of
  * (T + num_seqs * (chunk - 1)) / chunk chunks. Returns 0 for invalid sizes.
  * The workspace must be 256-byte aligned; its contents need no initialisation.
+ * Sized for the current CUDA device: with few long sequences the tensor-core
+ * path splits the state scan into segments (gdn_chunk_fwd_scan_segments) and
+ * needs three fp32 states per segment and head more.
  */
 size_t gdn_chunk_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int num_seqs,
                                     int chunk, int dtype);
@@ -153,6 +156,23 @@ int gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const flo
 /* Which implementation gdn_chunk_fwd would run for these sizes
  * (GDN_PATH_TCGEN05 or GDN_PATH_SIMT), or a negative value if unsupported. */
 int gdn_chunk_fwd_path(int d_k, int d_v, int chunk, int dtype);
+
+/*
+ * gdn_chunk_fwd_scan_segments -- into how many segments per sequence the
+ * tensor-core path splits its sequential state scan, on a device with `sms`
+ * streaming multiprocessors (1 = no split). Pure host arithmetic.
+ *
+ * The chunk-to-chunk state map S -> S (gamma_last I - W^T D K) + U^T D K is
+ * affine in S, so a sequence's chain of chunks can run as segments: every
+ * segment from S = 0 and, with V = 0, from S = I (its map S -> S P + H), a
+ * short fp32 composition of the start states, and every segment again from
+ * its start state. This is a reading of the pages' parallel-over-chunks
+ * training algorithm (phantomic12 page, mechanism paragraph), not a step they
+ * print. Used only for equal-length sequences (no cu_seqlens) when the three
+ * passes take at most 70 % of the chunk periods of one plain pass.
+ */
+int gdn_chunk_fwd_scan_segments(int B, int T, int H, int d_k, int d_v, int num_seqs, int chunk,
+                                int dtype, int sms);
 
 /*
  * gdn_decode_step -- one recurrent token for N*H independent states, in place.

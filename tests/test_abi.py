@@ -111,3 +111,19 @@ def test_decode_host_checks(L):
     assert call(N=0) == gdn.ERR_INVALID_ARG
     assert call(dv=130) == gdn.ERR_UNSUPPORTED
     assert call(dv=126) == gdn.ERR_UNSUPPORTED
+
+
+def test_scan_segments_rule(L):
+    seg = L.gdn_chunk_fwd_scan_segments
+    BF, F = gdn.BF16, gdn.F32
+    # few long chains: split; one chain per SM-wave of short chains: no split
+    assert seg(1, 65536, 16, 128, 128, 0, 64, BF, 148) == 9     # long64k: 16 chains x 1024 chunks
+    assert seg(4, 4096, 16, 128, 128, 0, 64, BF, 148) == 1      # 64 chains x 64 chunks
+    assert seg(1, 64 * 40, 1, 128, 128, 0, 64, BF, 148) > 1
+    assert seg(1, 320, 2, 128, 128, 0, 64, BF, 148) == 1        # 5 chunks
+    assert seg(1, 65536, 16, 128, 128, 4, 64, BF, 148) == 1     # packed sequences: never
+    assert seg(1, 65536, 16, 128, 128, 0, 64, F, 148) == 1      # CUDA-core path: never
+    assert seg(1, 65536, 16, 128, 128, 0, 64, BF, 0) == 1       # unknown device
+    for sms in (1, 16, 148, 160):
+        g = seg(1, 64 * 1000, 3, 128, 128, 0, 64, BF, sms)
+        assert 1 <= g <= 16

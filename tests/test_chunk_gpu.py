@@ -141,6 +141,39 @@ def test_simt_chunk_size_independence():
         assert rel_l2(np64(fs), np64(outs[0][1])) < 1e-5
 
 
+# ---------------------------------------------------------------- segmented state scan
+def _segments(inp):
+    import gated_delta_rule_112_b200 as gdn
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    return gdn.lib().gdn_chunk_fwd_scan_segments(inp["B"], inp["T"], inp["H"], 128, 128, 0, 64,
+                                                 gdn.BF16, sms)
+
+
+def test_tc_segmented_scan_one_head_ragged_tail():
+    inp = make_chunk_inputs(SMALL, B=1, H=1, T=64 * 40 + 37, random_state=True)
+    assert _segments(inp) > 1
+    check(inp, TOL_BF16)
+
+
+def test_tc_segmented_scan_batch_heads_slow_decay():
+    inp = make_chunk_inputs(SMALL, B=2, H=2, T=64 * 47, random_state=True, gate_mu=-4.0)
+    assert _segments(inp) > 1
+    check(inp, TOL_BF16)
+
+
+def test_tc_segmented_scan_without_final_state_or_initial_state():
+    import gated_delta_rule_112_b200 as gdn
+    inp = make_chunk_inputs(SMALL, B=1, H=2, T=64 * 33)
+    assert _segments(inp) > 1
+    d = to_dev(inp)
+    o, fs = gdn.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], None, None,
+                          output_final_state=False)
+    torch.cuda.synchronize()
+    assert fs is None
+    ro, _ = oracle_chunk(inp)
+    assert_close("o", np64(o), ro, TOL_BF16)
+
+
 # ---------------------------------------------------------------- the workloads
 def test_workload_tiny_fp32():
     check(make_chunk_inputs("tiny_fp32"), TOL_F32)
