@@ -60,6 +60,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_chunk_fwd_workspace_size.restype = sz
         L.gdn_chunk_fwd_scan_segments.argtypes = [ci] * 9
         L.gdn_chunk_fwd_scan_segments.restype = ci
+        L.gdn_selftest_wait_timeout.argtypes = [vp, vp]
+        L.gdn_selftest_wait_timeout.restype = ci
         L.gdn_chunk_fwd_path.argtypes = [ci] * 4
         L.gdn_chunk_fwd_path.restype = ci
         L.gdn_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, ci, ci, ci, ci, ci, vp]

@@ -192,6 +192,21 @@ int gdn_decode_step(const void *q, const void *k, const void *v, const float *g,
                     int d_v, int dtype, void *stream);
 
 /*
+ * gdn_selftest_wait_timeout -- device self-test of the bounded waits (the
+ * pages have no counterpart; it tests this library's failure handling).
+ *
+ * Launches, on `stream`, one small kernel that waits on a barrier nothing
+ * ever completes, with the same bounded wait (about 1 s of SM clock) that the
+ * chunked-forward kernels use. The wait must give up: afterwards
+ * gdn_get_status(workspace, stream) returns GDN_ERR_DEVICE_TIMEOUT (and clears
+ * the error word), and the context stays usable. `workspace`: caller-owned
+ * device memory of at least 256 bytes, 256-byte aligned; its first 256 bytes
+ * are overwritten. Returns GDN_OK once launched, GDN_ERR_WORKSPACE or
+ * GDN_ERR_CUDA otherwise.
+ */
+int gdn_selftest_wait_timeout(void *workspace, void *stream);
+
+/*
  * gdn_get_status -- synchronises `stream`, then reports the first error seen:
  * GDN_ERR_CUDA for a failed kernel, or the code a gdn_chunk_fwd kernel left in
  * `workspace` (GDN_ERR_DEVICE_TIMEOUT, GDN_ERR_INVALID_ARG for bad
