@@ -12,6 +12,8 @@ library is measured on:
 * ``long64k``    B=1 H=16 T=65536 d=128, bf16, slow decay, random state, seed 2
 * ``varlen64``   64 packed sequences, lengths log-uniform in [128, 2048], H=32
 * ``decode``     N=256 H=32 d=128 fp32 state, 64 consecutive single-token steps
+* ``b4h16t4096_beta2`` the b4h16t4096 shape with beta = 2 sigmoid(N(0, 1)) in
+  (0, 2): the negative-eigenvalue range of I - beta k k^T, seed 5
 
 Distributions (all drawn in fp32 with ``torch.Generator('cpu')``):
 q, k ~ N(0, 1) then L2-normalised per (token, head) over d_k; v ~ N(0, 1);
@@ -46,6 +48,7 @@ class Workload:
     num_seqs: int = 0          # >0: packed variable-length batch (B must be 1)
     len_range: tuple = field(default=(128, 2048))
     steps: int = 1             # decode workloads: consecutive steps
+    beta_scale: float = 1.0    # beta = beta_scale * sigmoid(N(0, 1))
 
 
 WORKLOADS = {
@@ -58,6 +61,8 @@ WORKLOADS = {
                          num_seqs=64),
     "decode": Workload("decode", B=256, T=1, H=32, d_k=128, d_v=128,
                        random_state=True, seed=4, steps=64),
+    "b4h16t4096_beta2": Workload("b4h16t4096_beta2", B=4, T=4096, H=16, d_k=128, d_v=128,
+                                 seed=5, beta_scale=2.0),
 }
 
 
@@ -74,8 +79,8 @@ def _unit_rows(x: torch.Tensor) -> torch.Tensor:
     return x / x.norm(dim=-1, keepdim=True).clamp_min(1e-12)
 
 
-def _gates(gen, shape, mu):
-    beta = torch.sigmoid(torch.randn(shape, generator=gen, dtype=torch.float32))
+def _gates(gen, shape, mu, beta_scale=1.0):
+    beta = beta_scale * torch.sigmoid(torch.randn(shape, generator=gen, dtype=torch.float32))
     g = -torch.nn.functional.softplus(
         torch.randn(shape, generator=gen, dtype=torch.float32) + mu)
     return g.contiguous(), beta.contiguous()
@@ -115,7 +120,7 @@ def make_chunk_inputs(w: Workload | str, *, seed: int | None = None, T: int | No
     q = _unit_rows(torch.randn(Bn, Tn, H, w.d_k, generator=gen, dtype=torch.float32))
     k = _unit_rows(torch.randn(Bn, Tn, H, w.d_k, generator=gen, dtype=torch.float32))
     v = torch.randn(Bn, Tn, H, w.d_v, generator=gen, dtype=torch.float32)
-    g, beta = _gates(gen, (Bn, Tn, H), gate_mu)
+    g, beta = _gates(gen, (Bn, Tn, H), gate_mu, w.beta_scale)
     s0 = None
     if random_state:
         s0 = 0.02 * torch.randn(N, H, w.d_k, w.d_v, generator=gen, dtype=torch.float32)

@@ -188,6 +188,14 @@ def test_workload_long64k_sampled_heads():
     check(make_chunk_inputs("long64k"), TOL_BF16, heads=[3, 12])
 
 
+def test_workload_beta_up_to_two_sampled_heads():
+    """b4h16t4096 with beta in (0, 2) (I - beta k k^T has a negative eigenvalue
+    for beta > 1); oracle on 2 of the 16 heads."""
+    inp = make_chunk_inputs("b4h16t4096_beta2")
+    assert float(inp["beta"].max()) > 1.9
+    check(inp, TOL_BF16, heads=[0, 9])
+
+
 def test_workload_varlen64_sampled_heads():
     """64 packed sequences (~44K tokens), H=32, on the GPU; oracle on 3 heads."""
     check(make_chunk_inputs("varlen64"), TOL_BF16, heads=[0, 17, 31])

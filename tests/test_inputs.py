@@ -45,3 +45,12 @@ def test_decode_inputs():
     d = make_decode_inputs(N=4, H=2, steps=3)
     assert d["state"].shape == (4, 2, 128, 128) and d["q"].shape == (3, 4, 2, 128)
     assert abs(float(d["state"].std()) - 0.02) < 2e-3
+
+
+def test_beta_up_to_two_workload_draws_the_same_bytes_scaled():
+    a = make_chunk_inputs("b4h16t4096", T=128, seed=5)
+    b = make_chunk_inputs("b4h16t4096_beta2", T=128)
+    assert torch.equal(a["q"], b["q"]) and torch.equal(a["g"], b["g"])
+    assert torch.allclose(b["beta"], 2.0 * a["beta"])
+    assert float(b["beta"].min()) > 0.0 and float(b["beta"].max()) < 2.0
+    assert float(b["beta"].max()) > 1.0
