@@ -60,6 +60,7 @@ constexpr uint32_t kP_KQ = 0;                        // 2 blocks x [K rows 0-63 
 constexpr uint32_t kP_PST = kP_KQ + kTile64x64;      // P staging, over Q of block 0 (dead after G)
 constexpr uint32_t kP_WST = kP_KQ;                   // -W staging [64 c][128 d] (2 blocks), over K/Q
 constexpr uint32_t kP_KST = kP_KQ + kTile128x64;     // (D K)^T staging [128 d][64 s], over K/Q
+constexpr uint32_t kP_TT = kP_KST + kTile64x64;      // solve: T transposed, fp32 [48][36], over Q of block 1
 constexpr uint32_t kP_AS = kP_KQ + 2 * kTile128x64;  // A, fp32 [64][68]; after the solve it
 constexpr uint32_t kP_TB = kP_AS;                    //   holds T diag(beta)       (bf16 64x64)
 constexpr uint32_t kP_TBG = kP_AS + kTile64x64;      //   and   T diag(beta gamma) (bf16 64x64)
@@ -67,6 +68,8 @@ constexpr uint32_t kP_TS = kP_AS + 64 * kLd * 4;     // T, fp32 [64][68]; then d
 constexpr uint32_t kP_DIAG = kP_TS;
 constexpr int kLy = 36;                              // fp32 row stride of the solve scratch
 constexpr uint32_t kP_XS = kP_TS + 64 * kLd * 4;     // solve scratch, fp32 [32][36]
+static_assert(kLy % 32 == 4 && kLd % 32 == 4 && 48 * kLy * 4 <= kTile64x64,
+              "solve strides and the transposed-T area");
 constexpr uint32_t kP_VEC = kP_XS + 32 * kLy * 4;    // Gamma, beta, gamma, Gamma log2(e): 4 x 64 fp32
 constexpr uint32_t kP_BAR = kP_VEC + 4 * 64 * 4;     // 2 mbarriers + tmem address
 constexpr uint32_t kP_END = kP_BAR + 64;
@@ -88,20 +91,62 @@ __device__ __forceinline__ float4 lds4(const float *p) {
   return *reinterpret_cast<const float4 *>(p);
 }
 
+// Shared address of this lane's row for an ldmatrix.x4 A fragment (16 x 8,
+// rows r0.., columns c0..) of a row-major fp32 matrix with row stride ld.
+__device__ __forceinline__ uint32_t frag_a(const float *m, int ld, int r0, int c0, int lane) {
+  return smem_u32(m + (r0 + (lane & 7) + 8 * ((lane >> 3) & 1)) * ld + c0 + 4 * (lane >> 4));
+}
+// ... and for a B fragment (8 x 8, k x n) read from the transposed copy
+// (row n, word k): x2 gives k0.. k0 + 7, x4 also k0 + 8 .. k0 + 15.
+__device__ __forceinline__ uint32_t frag_bt(const float *mt, int ld, int n0, int k0, int lane) {
+  return smem_u32(mt + (n0 + (lane & 7)) * ld + k0 + 4 * (lane >> 3));
+}
+
+// d += a b for fp32 fragments on the tf32 tensor-core path, each operand split
+// into tf32 parts x = hi + lo (|lo| <= 2^-11 |x|, the rest <= 2^-22 |x|) and
+// the three products that matter: lo hi + hi lo + hi hi. The dropped lo lo
+// term and the tails keep each product term within about 2^-21 of fp32.
+__device__ __forceinline__ void mma_3xtf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                           uint32_t b1) {
+  uint32_t ah[4], al[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    ah[i] = cvt_tf32(__uint_as_float(a[i]));
+    al[i] = cvt_tf32(__uint_as_float(a[i]) - __uint_as_float(ah[i]));
+  }
+  const uint32_t bh0 = cvt_tf32(__uint_as_float(b0)), bh1 = cvt_tf32(__uint_as_float(b1));
+  const uint32_t bl0 = cvt_tf32(__uint_as_float(b0) - __uint_as_float(bh0));
+  const uint32_t bl1 = cvt_tf32(__uint_as_float(b1) - __uint_as_float(bh1));
+  mma_tf32_m16n8k8(d, al, bh0, bh1);
+  mma_tf32_m16n8k8(d, ah, bl0, bl1);
+  mma_tf32_m16n8k8(d, ah, bh0, bh1);
+}
+
 // T = (I + A)^-1 for the strictly lower-triangular 64 x 64 A (fp32 shared
 // memory, row stride kLd), by recursive 2 x 2 blocking: for a lower block
 // triangular [[L11, 0], [L21, L22]], the inverse is [[T11, 0], [-T22 L21 T11, T22]].
 //   step 0  the four 16 x 16 diagonal blocks, by column-wise forward
 //           substitution in registers (thread = one column of one block);
-//           their upper triangles are written as zeros
-//   step 1  the two 16 x 16 blocks T(1,0), T(3,2)        (two half-steps)
-//   step 2  the 32 x 32 block T([2,3],[0,1])             (two half-steps)
-// Each half-step is a small product over all 256 threads with float4 operand
-// loads; loop bounds skip the blocks of T above the diagonal, which are never
-// written, and are uniform within a warp.
+//           their upper triangles are written as zeros. Blocks 0-2 are also
+//           written transposed into Tt (row stride kLy): T(0,0), T(1,1) at
+//           [0, 32) x [0, 32), T(2,2) at rows [32, 48)
+//   step 1  T(1,0) and T(3,2): Y_b = A(i,j) T(j,j), then T(i,j) = -T(i,i) Y_b
+//           (i = 2b + 1, j = 2b); warp (b, column half) computes both
+//           products for its 8 columns, so only a warp sync lies between them
+//   step 2  T([2,3],[0,1]): Y = A(..) T([0,1],[0,1]), then -T([2,3],[2,3]) Y;
+//           warp = one 16 x 8 tile of each product, the two warps that share
+//           a column tile meet on a named barrier
+// The products are warp-level tensor-core tiles (m16n8k8, split tf32, fp32
+// accumulation) whose operands are read with ldmatrix: A operands from the
+// row-major A and T, B operands from transposed copies (Tt, and Y stored
+// transposed in Xs), all with row strides = 4 (mod 32) words, so that an
+// 8-row ldmatrix and the transposed fragment stores are free of bank
+// conflicts. Loop bounds skip the blocks of T above the diagonal, which are
+// never written, and are uniform within a warp.
 __device__ void solve_unit_lower_64(const float *__restrict__ As, float *__restrict__ Ts,
-                                    float *__restrict__ Xs, int tid) {
+                                    float *__restrict__ Tt, float *__restrict__ Xs, int tid) {
   const int warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;
   if (tid < 64) {
     const int base = (tid >> 4) * 16, jj = tid & 15;
     float x[16];
@@ -123,84 +168,82 @@ __device__ void solve_unit_lower_64(const float *__restrict__ As, float *__restr
     }
 #pragma unroll
     for (int r = 0; r < 16; ++r) Ts[(base + r) * kLd + base + jj] = x[r];
+    if (base < 48) {   // transposed: row = column of T, word = row of T
+      float *dst = Tt + (base + jj) * kLy + (base < 32 ? base : 0);
+#pragma unroll
+      for (int r = 0; r < 16; r += 4)
+        *reinterpret_cast<float4 *>(dst + r) = make_float4(x[r], x[r + 1], x[r + 2], x[r + 3]);
+    }
   }
   __syncthreads();
-  // step 1: block b in {0, 1} is T(2b+1, 2b); thread = row r, columns c, c+1
-  const int b1 = tid >> 7, r1 = (tid >> 3) & 15, c1 = (tid & 7) * 2;
-  const int i1 = 16 * (2 * b1 + 1), j1 = i1 - 16;
-  {  // Y_b = A(i, i-1) T(i-1, i-1)
-    const float *arow = As + (i1 + r1) * kLd + j1;
-    float y0 = 0.f, y1 = 0.f;
-#pragma unroll
-    for (int m4 = 0; m4 < 16; m4 += 4) {
-      const float4 a = lds4(arow + m4);
-      const float av[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 t = *reinterpret_cast<const float2 *>(Ts + (j1 + m4 + e) * kLd + j1 + c1);
-        y0 = fmaf(av[e], t.x, y0);
-        y1 = fmaf(av[e], t.y, y1);
-      }
+  if (warp < 4) {  // step 1
+    const int b = warp >> 1, n0 = 8 * (warp & 1);
+    const int i = 16 * (2 * b + 1), j = i - 16;
+    const float *tjt = Tt + (b ? 32 * kLy : 0);   // T(j,j) transposed, block-local indices
+    float *yt = Xs + b * 16 * kLy;                // Y_b transposed
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+    // columns n >= 8 of T(j,j) are zero in rows k < 8
+    for (int k0 = n0; k0 < 16; k0 += 8) {
+      uint32_t a[4], bb[2];
+      ldsm_x4(frag_a(As, kLd, i, j + k0, lane), a);
+      ldsm_x2(frag_bt(tjt, kLy, n0, k0, lane), bb);
+      mma_3xtf32(c, a, bb[0], bb[1]);
     }
-    *reinterpret_cast<float2 *>(Xs + b1 * 16 * kLy + r1 * kLy + c1) = make_float2(y0, y1);
+    const int n = n0 + 2 * t;
+    yt[n * kLy + g] = c[0];
+    yt[(n + 1) * kLy + g] = c[1];
+    yt[n * kLy + g + 8] = c[2];
+    yt[(n + 1) * kLy + g + 8] = c[3];
+    __syncwarp();
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+    uint32_t bb[4];
+    ldsm_x4(frag_bt(yt, kLy, n0, 0, lane), bb);
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk) {
+      uint32_t a[4];
+      ldsm_x4(frag_a(Ts, kLd, i, i + 8 * kk, lane), a);
+      mma_3xtf32(d, a, bb[2 * kk], bb[2 * kk + 1]);
+    }
+    *reinterpret_cast<float2 *>(Ts + (i + g) * kLd + j + n) = make_float2(-d[0], -d[1]);
+    *reinterpret_cast<float2 *>(Ts + (i + g + 8) * kLd + j + n) = make_float2(-d[2], -d[3]);
+    if (b == 0) {   // T(1,0) is also a B operand of step 2
+      Tt[n * kLy + i + g] = -d[0];
+      Tt[(n + 1) * kLy + i + g] = -d[1];
+      Tt[n * kLy + i + g + 8] = -d[2];
+      Tt[(n + 1) * kLy + i + g + 8] = -d[3];
+    }
   }
   __syncthreads();
-  {  // T(i, i-1) = -T(i, i) Y_b
-    const float *trow = Ts + (i1 + r1) * kLd + i1;
-    float y0 = 0.f, y1 = 0.f;
+  {  // step 2: output tile rows 32 + m0 .. + 15, columns n0 .. n0 + 7
+    const int mi = warp >> 2, m0 = 16 * mi, n0 = 8 * (warp & 3);
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+    // columns n of T([0,1],[0,1]) are zero in rows k < n: start at k = n0
+    for (int k0 = n0; k0 < 32; k0 += 8) {
+      uint32_t a[4], bb[2];
+      ldsm_x4(frag_a(As, kLd, 32 + m0, k0, lane), a);
+      ldsm_x2(frag_bt(Tt, kLy, n0, k0, lane), bb);
+      mma_3xtf32(c, a, bb[0], bb[1]);
+    }
+    const int n = n0 + 2 * t;
+    Xs[n * kLy + m0 + g] = c[0];
+    Xs[(n + 1) * kLy + m0 + g] = c[1];
+    Xs[n * kLy + m0 + g + 8] = c[2];
+    Xs[(n + 1) * kLy + m0 + g + 8] = c[3];
+    named_bar_sync(1 + (warp & 3), 64);   // Y rows [0, 32) of columns n0.. are in Xs
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+    // rows [32, 48) of T([2,3],[2,3]) have columns [32, 48) only
+    for (int k0 = 0; k0 < m0 + 16; k0 += 16) {
+      uint32_t bb[4];
+      ldsm_x4(frag_bt(Xs, kLy, n0, k0, lane), bb);
 #pragma unroll
-    for (int m4 = 0; m4 < 16; m4 += 4) {
-      const float4 t = lds4(trow + m4);
-      const float tv[4] = {t.x, t.y, t.z, t.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 y = *reinterpret_cast<const float2 *>(Xs + b1 * 16 * kLy + (m4 + e) * kLy + c1);
-        y0 = fmaf(tv[e], y.x, y0);
-        y1 = fmaf(tv[e], y.y, y1);
+      for (int kk = 0; kk < 2; ++kk) {
+        uint32_t a[4];
+        ldsm_x4(frag_a(Ts, kLd, 32 + m0, 32 + k0 + 8 * kk, lane), a);
+        mma_3xtf32(d, a, bb[2 * kk], bb[2 * kk + 1]);
       }
     }
-    *reinterpret_cast<float2 *>(Ts + (i1 + r1) * kLd + j1 + c1) = make_float2(-y0, -y1);
-  }
-  __syncthreads();
-  // step 2: thread = row 16 (warp & 1) + (lane & 15), columns c2 .. c2 + 3 with
-  // c2 = 8 (warp >> 1) + 4 (lane >> 4)
-  const int r2 = 16 * (warp & 1) + (lane & 15), c2 = 8 * (warp >> 1) + 4 * (lane >> 4);
-  {  // Y = A([32,64), [0,32)) T([0,32), [0,32)); T(0,1) is unwritten: columns
-     // c >= 16 take rows m >= 16 only
-    const int m0 = (warp >> 2) * 16;
-    const float *arow = As + (32 + r2) * kLd;
-    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 2
-    for (int m4 = m0; m4 < 32; m4 += 4) {
-      const float4 a = lds4(arow + m4);
-      const float av[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float4 t = lds4(Ts + (m4 + e) * kLd + c2);
-        y.x = fmaf(av[e], t.x, y.x); y.y = fmaf(av[e], t.y, y.y);
-        y.z = fmaf(av[e], t.z, y.z); y.w = fmaf(av[e], t.w, y.w);
-      }
-    }
-    *reinterpret_cast<float4 *>(Xs + r2 * kLy + c2) = y;
-  }
-  __syncthreads();
-  {  // T([32,64), [0,32)) = -T([32,64), [32,64)) Y; T(2,3) is unwritten: rows
-     // r < 16 take m < 16 only
-    const int m1 = (warp & 1) ? 32 : 16;
-    const float *trow = Ts + (32 + r2) * kLd + 32;
-    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 2
-    for (int m4 = 0; m4 < m1; m4 += 4) {
-      const float4 t = lds4(trow + m4);
-      const float tv[4] = {t.x, t.y, t.z, t.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float4 x = lds4(Xs + (m4 + e) * kLy + c2);
-        y.x = fmaf(tv[e], x.x, y.x); y.y = fmaf(tv[e], x.y, y.y);
-        y.z = fmaf(tv[e], x.z, y.z); y.w = fmaf(tv[e], x.w, y.w);
-      }
-    }
-    *reinterpret_cast<float4 *>(Ts + (32 + r2) * kLd + c2) = make_float4(-y.x, -y.y, -y.z, -y.w);
+    *reinterpret_cast<float2 *>(Ts + (32 + m0 + g) * kLd + n) = make_float2(-d[0], -d[1]);
+    *reinterpret_cast<float2 *>(Ts + (32 + m0 + g + 8) * kLd + n) = make_float2(-d[2], -d[3]);
   }
   __syncthreads();
 }
@@ -230,6 +273,7 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
   float *As = reinterpret_cast<float *>(sm + kP_AS);
   float *Ts = reinterpret_cast<float *>(sm + kP_TS);
   float *Xs = reinterpret_cast<float *>(sm + kP_XS);
+  float *Tt = reinterpret_cast<float *>(sm + kP_TT);
   float *Gm = reinterpret_cast<float *>(sm + kP_VEC);
   float *Bt = Gm + 64;
   float *Ga = Bt + 64;
@@ -426,7 +470,7 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
     tma_store_commit();
   }
   GDN_TRACE_POINT(tr && chunk < 64, 1, chunk, 3);
-  if (!abort_flag) solve_unit_lower_64(As, Ts, Xs, tid);
+  if (!abort_flag) solve_unit_lower_64(As, Ts, Tt, Xs, tid);
   GDN_TRACE_POINT(tr && chunk < 64, 1, chunk, 4);
   // T diag(beta) and T diag(beta gamma) as bf16 K-major operand tiles (A is
   // dead now). Thread: row r, columns [16 q4, 16 q4 + 16); T is lower

@@ -366,6 +366,42 @@ __device__ __forceinline__ void stmatrix_x4_trans(uint32_t saddr, uint32_t r0, u
                : "memory");
 }
 
+// Four (two) 8x8 b16 matrices from shared memory: thread 8m+j supplies the
+// address of row j of matrix m (16 bytes), and register r[m] of thread t
+// receives 32-bit word t%4 of row t/4 of matrix m. Words move intact, so the
+// same instruction loads fp32 tiles of 8 rows x 4 words.
+__device__ __forceinline__ void ldsm_x4(uint32_t saddr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(saddr)
+               : "memory");
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t saddr, uint32_t (&r)[2]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(saddr)
+               : "memory");
+}
+
+// fp32 -> tf32 (round to nearest, ties away), as a 32-bit pattern.
+__device__ __forceinline__ uint32_t cvt_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+
+// d += a b on the warp-level tensor-core path, m16n8k8 with tf32 operands and
+// fp32 accumulators. With g = lane/4, t = lane%4: a = A(g, t), A(g+8, t),
+// A(g, t+4), A(g+8, t+4); b = B(t, g), B(t+4, g); d = D(g, 2t), D(g, 2t+1),
+// D(g+8, 2t), D(g+8, 2t+1).
+__device__ __forceinline__ void mma_tf32_m16n8k8(float (&d)[4], const uint32_t (&a)[4],
+                                                 uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 // Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a tile that
 // uses the 128-byte swizzle (rows of 128 bytes, 8-row / 1024-byte atoms).
 __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {
