@@ -13,8 +13,12 @@ Two independent formulations live here:
 * ``chunked.chunk_fwd_dense``: the chunkwise WY / UT-transform form in numpy
   (dense inversion of I + A per chunk). It is used to pin the recurrence and
   to give per-chunk intermediates (T, W, U, P) for debugging kernels.
+* ``kda_chunk_fwd`` / ``kda_decode_step`` and ``chunked.kda_chunk_fwd_dense``:
+  the same two formulations for the channel-wise gate (the Kimi Delta
+  Attention variant: g = log alpha has one value per d_k channel).
 
-Every function is pinned by ``tests/test_oracle_pins.py``.
+Every function is pinned by ``tests/test_oracle_pins.py`` and
+``tests/test_oracle_kda_pins.py``.
 """
 from __future__ import annotations
 
@@ -54,6 +58,10 @@ def _load():
         lib.gdn_oracle_chunk_fwd.restype = ci
         lib.gdn_oracle_decode_step.argtypes = [d, d, d, d, d, d, d, ci, ci, ci, ci, ci]
         lib.gdn_oracle_decode_step.restype = ci
+        lib.gdn_oracle_kda_chunk_fwd.argtypes = lib.gdn_oracle_chunk_fwd.argtypes
+        lib.gdn_oracle_kda_chunk_fwd.restype = ci
+        lib.gdn_oracle_kda_decode_step.argtypes = lib.gdn_oracle_decode_step.argtypes
+        lib.gdn_oracle_kda_decode_step.restype = ci
         _lib = lib
     return _lib
 
@@ -79,9 +87,26 @@ def chunk_fwd(q, k, v, g, beta, initial_state=None, cu_seqlens=None, nthreads=No
     initial_state: [N,H,d_k,d_v] or None (zeros); cu_seqlens: int [N+1] or None.
     Returns (o [B,T,H,d_v], final_state [N,H,d_k,d_v]) as float64 arrays.
     """
+    return _run_chunk("gdn_oracle_chunk_fwd", q, k, v, g, beta, initial_state, cu_seqlens,
+                      nthreads, channel=False)
+
+
+def kda_chunk_fwd(q, k, v, g, beta, initial_state=None, cu_seqlens=None, nthreads=None):
+    """The fp64 token recurrence with the channel-wise gate:
+    S_t = S_{t-1} diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T, o_t = S_t q_t.
+
+    Same layouts as ``chunk_fwd`` except g (= log alpha): [B,T,H,d_k].
+    """
+    return _run_chunk("gdn_oracle_kda_chunk_fwd", q, k, v, g, beta, initial_state, cu_seqlens,
+                      nthreads, channel=True)
+
+
+def _run_chunk(fn, q, k, v, g, beta, initial_state, cu_seqlens, nthreads, channel):
     q, k, v, g, beta = (_f64(a) for a in (q, k, v, g, beta))
     B, T, H, dk = q.shape
     dv = v.shape[-1]
+    if g.shape != ((B, T, H, dk) if channel else (B, T, H)):
+        raise ValueError(f"g has shape {g.shape}")
     cu = None
     N = B
     if cu_seqlens is not None:
@@ -90,7 +115,7 @@ def chunk_fwd(q, k, v, g, beta, initial_state=None, cu_seqlens=None, nthreads=No
     s0 = None if initial_state is None else _f64(initial_state)
     o = np.zeros((B, T, H, dv), dtype=np.float64)
     fs = np.zeros((N, H, dk, dv), dtype=np.float64)
-    rc = _load().gdn_oracle_chunk_fwd(
+    rc = getattr(_load(), fn)(
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(s0),
         None if cu is None else cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
         B, T, H, dk, dv, N, _ptr(o), _ptr(fs), nthreads or default_threads())
@@ -101,14 +126,23 @@ def chunk_fwd(q, k, v, g, beta, initial_state=None, cu_seqlens=None, nthreads=No
 
 def decode_step(q, k, v, g, beta, state, nthreads=None):
     """One recurrent step for every (n, h). Returns (o [N,H,d_v], new_state)."""
+    return _run_decode("gdn_oracle_decode_step", q, k, v, g, beta, state, nthreads)
+
+
+def kda_decode_step(q, k, v, g, beta, state, nthreads=None):
+    """One channel-wise-gated step for every (n, h); g: [N,H,d_k]."""
+    return _run_decode("gdn_oracle_kda_decode_step", q, k, v, g, beta, state, nthreads)
+
+
+def _run_decode(fn, q, k, v, g, beta, state, nthreads):
     q, k, v, g, beta = (_f64(a) for a in (q, k, v, g, beta))
     st = _f64(state).copy()
     N, H, dk = q.shape
     dv = v.shape[-1]
     o = np.zeros((N, H, dv), dtype=np.float64)
-    rc = _load().gdn_oracle_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
-                                        _ptr(st), _ptr(o), N, H, dk, dv,
-                                        nthreads or default_threads())
+    rc = getattr(_load(), fn)(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                              _ptr(st), _ptr(o), N, H, dk, dv,
+                              nthreads or default_threads())
     if rc != 0:
         raise ValueError("oracle rejected the arguments")
     return o, st

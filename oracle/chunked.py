@@ -60,11 +60,58 @@ def chunk_dense(Kc, Vc, Qc, gc, bc, S0):
     return dict(Gamma=Gam, A=A, T=T, W=W, U=U, V_new=Vnew, P=P, O=O, S_next=S_next)
 
 
+def kda_chunk_dense(Kc, Vc, Qc, Gc, bc, S0):
+    """The chunk equations for the channel-wise gate (g = log alpha per d_k
+    channel; the Kimi Delta Attention variant, named on the dmarx anthology
+    LIT-137 page, "Standing in the anthology", and SOTA-135, "Sequence").
+
+    With S_t = S_{t-1} diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+    unrolling one chunk from S_0 gives, per channel j, Gamma_rj = sum_{s<=r} g_sj
+    and
+
+        S_r = S_0 diag(exp(Gamma_r)) + sum_{s<=r} u_s (k_s (.) exp(Gamma_r - Gamma_s))^T
+        u_r = beta_r (v_r - S_{r-1} diag(alpha_r) k_r)
+
+    so the decay moves inside the dot products:
+
+        A_rs = beta_r sum_j k_rj k_sj exp(Gamma_rj - Gamma_sj)   (s < r)
+        T = (I + A)^-1,  W = T diag(beta) (K (.) exp(Gamma)),  U = T diag(beta) V
+        V_new = U - W S_0^T
+        P_rs = sum_j q_rj k_sj exp(Gamma_rj - Gamma_sj)          (s <= r)
+        O = (Q (.) exp(Gamma)) S_0^T + P V_new
+        S_C = S_0 diag(exp(Gamma_last)) + V_new^T (K (.) exp(Gamma_last - Gamma))
+
+    Gc: [L, d_k]; other arguments as in ``chunk_dense``. Every exponent above
+    is a difference of cumulative sums taken over the tokens in between, as
+    written (no rescaling).
+    """
+    L = Kc.shape[0]
+    Gam = np.cumsum(Gc, axis=0)                            # [L, d_k]
+    incl = np.tril(np.ones((L, L), dtype=bool), 0)
+    lower = np.tril(np.ones((L, L), dtype=bool), -1)
+    diff = Gam[:, None, :] - Gam[None, :, :]               # [r, s, j]
+    E = np.where(incl[:, :, None], np.exp(np.where(incl[:, :, None], diff, 0.0)), 0.0)
+    KK = np.einsum("rj,sj,rsj->rs", Kc, Kc, E)
+    A = np.where(lower, bc[:, None] * KK, 0.0)
+    T = np.linalg.solve(np.eye(L) + A, np.eye(L))
+    W = T @ (bc[:, None] * (Kc * np.exp(Gam)))
+    U = T @ (bc[:, None] * Vc)
+    Vnew = U - W @ S0.T
+    P = np.einsum("rj,sj,rsj->rs", Qc, Kc, E)
+    O = (Qc * np.exp(Gam)) @ S0.T + P @ Vnew
+    if L:
+        S_next = S0 * np.exp(Gam[-1])[None, :] + Vnew.T @ (Kc * np.exp(Gam[-1][None, :] - Gam))
+    else:
+        S_next = S0.copy()
+    return dict(Gamma=Gam, A=A, T=T, W=W, U=U, V_new=Vnew, P=P, O=O, S_next=S_next)
+
+
 def chunk_fwd_dense(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk=64,
-                    keep=False):
+                    keep=False, channel_gate=False):
     """Whole-sequence forward by chunks of ``chunk`` tokens (fp64).
 
-    Same argument layout as ``oracle.chunk_fwd``. Chunks start at each
+    Same argument layout as ``oracle.chunk_fwd`` (``oracle.kda_chunk_fwd``
+    with ``channel_gate=True``: g is [B,T,H,d_k]). Chunks start at each
     sequence's first token; the last chunk of a sequence may be partial.
     With ``keep=True`` also returns the per-chunk intermediates as a list of
     dicts keyed by (seq, head, chunk index).
@@ -87,8 +134,9 @@ def chunk_fwd_dense(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk
                  else np.asarray(initial_state, dtype=np.float64)[n, h].T.copy())
             for ci, c0 in enumerate(range(t0, t1, chunk)):
                 c1 = min(c0 + chunk, t1)
-                r = chunk_dense(k[b, c0:c1, h], v[b, c0:c1, h], q[b, c0:c1, h],
-                                g[b, c0:c1, h], beta[b, c0:c1, h], S)
+                step = kda_chunk_dense if channel_gate else chunk_dense
+                r = step(k[b, c0:c1, h], v[b, c0:c1, h], q[b, c0:c1, h],
+                         g[b, c0:c1, h], beta[b, c0:c1, h], S)
                 o[b, c0:c1, h] = r["O"]
                 if keep:
                     r["S0"] = S
@@ -98,3 +146,10 @@ def chunk_fwd_dense(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk
     if keep:
         return o, fs, inter
     return o, fs
+
+
+def kda_chunk_fwd_dense(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk=64,
+                        keep=False):
+    """``chunk_fwd_dense`` for the channel-wise gate (g: [B,T,H,d_k])."""
+    return chunk_fwd_dense(q, k, v, g, beta, initial_state, cu_seqlens, chunk, keep,
+                           channel_gate=True)

@@ -28,8 +28,19 @@
  * g is log(alpha); alpha = exp(g). With cu_seqlens (B == 1) sequence n covers
  * tokens [cu[n], cu[n+1]) and starts from its own initial state.
  *
- * Parity: pinned by tests/test_oracle_pins.py (closed forms, special cases,
- * exact rational arithmetic, the dense chunked WY/UT form).
+ * Channel-wise gate (the Kimi Delta Attention variant, named as this
+ * recurrence's successor on the dmarx anthology LIT-137 page, "Standing in the
+ * anthology", and on SOTA-135, "Sequence": the scalar decay becomes one decay
+ * per d_k channel). alpha_t is then a d_k vector and diag(alpha_t) stands
+ * where the scalar stood:
+ *     S_t = S_{t-1} diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ * so, with R = S_{t-1} diag(alpha_t) (column j of S scaled by alpha_tj),
+ * S_t = R + beta_t (v_t - R k_t) k_t^T and o_t = S_t q_t. The gate input is
+ * g = log(alpha) of shape [B, T, H, d_k] (gdn_oracle_kda_*).
+ *
+ * Parity: pinned by tests/test_oracle_pins.py and tests/test_oracle_kda_pins.py
+ * (closed forms, special cases, exact rational arithmetic, hand-worked
+ * tokens, the dense chunked WY/UT forms).
  */
 #include <math.h>
 #include <pthread.h>
@@ -42,26 +53,50 @@ typedef struct {
     const int32_t *cu;
     double *o, *s_out;
     int B, T, H, dk, dv, N;
+    int channel_gate;      /* 0: g [B,T,H] scalar gate; 1: g [B,T,H,d_k] per channel */
     int next;              /* next (seq, head) unit to hand out */
     pthread_mutex_t lock;
 } job_t;
 
-/* One (sequence, head) recurrence over tokens [t_begin, t_end) of row block
- * `b` (b = batch index, or 0 for packed sequences). */
+/* Tokens [t0, t1) of row block b (b = batch index, or 0 for packed sequences)
+ * that sequence n covers. */
+static void seq_span(const job_t *J, int n, int *b, int *t0, int *t1)
+{
+    if (J->cu) { *b = 0; *t0 = J->cu[n]; *t1 = J->cu[n + 1]; }
+    else       { *b = n; *t0 = 0;        *t1 = J->T; }
+}
+
+/* S (formula orientation, S[i*dk + j] = S_ij) from the S^T memory layout. */
+static void load_state(const job_t *J, int n, int h, double *S)
+{
+    const int dk = J->dk, dv = J->dv;
+    if (J->s0) {
+        const double *st = J->s0 + ((size_t)n * J->H + h) * dk * dv;
+        for (int j = 0; j < dk; ++j)
+            for (int i = 0; i < dv; ++i) S[(size_t)i * dk + j] = st[(size_t)j * dv + i];
+    }
+}
+
+static void store_state(const job_t *J, int n, int h, const double *S)
+{
+    const int dk = J->dk, dv = J->dv;
+    if (J->s_out) {
+        double *st = J->s_out + ((size_t)n * J->H + h) * dk * dv;
+        for (int j = 0; j < dk; ++j)
+            for (int i = 0; i < dv; ++i) st[(size_t)j * dv + i] = S[(size_t)i * dk + j];
+    }
+}
+
+/* One (sequence, head) recurrence with the scalar gate. */
 static void run_unit(job_t *J, int n, int h)
 {
     const int H = J->H, dk = J->dk, dv = J->dv;
     int b, t0, t1;
-    if (J->cu) { b = 0; t0 = J->cu[n]; t1 = J->cu[n + 1]; }
-    else       { b = n; t0 = 0;        t1 = J->T; }
+    seq_span(J, n, &b, &t0, &t1);
 
     double *S = (double *)calloc((size_t)dv * dk, sizeof(double)); /* S[i*dk + j] */
     double *x = (double *)malloc(sizeof(double) * dv);
-    if (J->s0) {
-        const double *st = J->s0 + ((size_t)n * H + h) * dk * dv;
-        for (int j = 0; j < dk; ++j)
-            for (int i = 0; i < dv; ++i) S[(size_t)i * dk + j] = st[(size_t)j * dv + i];
-    }
+    load_state(J, n, h, S);
     for (int t = t0; t < t1; ++t) {
         const size_t row = ((size_t)b * J->T + t) * H + h;
         const double *kt = J->k + row * dk, *qt = J->q + row * dk, *vt = J->v + row * dv;
@@ -87,13 +122,53 @@ static void run_unit(job_t *J, int n, int h)
             ot[i] = acc;
         }
     }
-    if (J->s_out) {
-        double *st = J->s_out + ((size_t)n * H + h) * dk * dv;
-        for (int j = 0; j < dk; ++j)
-            for (int i = 0; i < dv; ++i) st[(size_t)j * dv + i] = S[(size_t)i * dk + j];
-    }
+    store_state(J, n, h, S);
     free(S);
     free(x);
+}
+
+/* One (sequence, head) recurrence with the channel-wise gate (see the header):
+ * R = S_{t-1} diag(alpha_t); S_t = R + beta_t (v_t - R k_t) k_t^T; o_t = S_t q_t. */
+static void run_unit_kda(job_t *J, int n, int h)
+{
+    const int H = J->H, dk = J->dk, dv = J->dv;
+    int b, t0, t1;
+    seq_span(J, n, &b, &t0, &t1);
+
+    double *S = (double *)calloc((size_t)dv * dk, sizeof(double)); /* S[i*dk + j] */
+    double *x = (double *)malloc(sizeof(double) * dv);
+    double *a = (double *)malloc(sizeof(double) * dk);
+    load_state(J, n, h, S);
+    for (int t = t0; t < t1; ++t) {
+        const size_t row = ((size_t)b * J->T + t) * H + h;
+        const double *kt = J->k + row * dk, *qt = J->q + row * dk, *vt = J->v + row * dv;
+        const double *gt = J->g + row * dk;
+        const double beta = J->beta[row];
+        for (int j = 0; j < dk; ++j) a[j] = exp(gt[j]);
+        /* x = R k_t = S_{t-1} diag(alpha_t) k_t */
+        for (int i = 0; i < dv; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < dk; ++j) acc += S[(size_t)i * dk + j] * a[j] * kt[j];
+            x[i] = acc;
+        }
+        /* S_t = R + beta (v_t - x) k_t^T */
+        for (int i = 0; i < dv; ++i) {
+            const double ui = beta * (vt[i] - x[i]);
+            for (int j = 0; j < dk; ++j)
+                S[(size_t)i * dk + j] = a[j] * S[(size_t)i * dk + j] + ui * kt[j];
+        }
+        /* o_t = S_t q_t (after the write) */
+        double *ot = J->o + row * dv;
+        for (int i = 0; i < dv; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < dk; ++j) acc += S[(size_t)i * dk + j] * qt[j];
+            ot[i] = acc;
+        }
+    }
+    store_state(J, n, h, S);
+    free(S);
+    free(x);
+    free(a);
 }
 
 static void *worker(void *arg)
@@ -104,18 +179,17 @@ static void *worker(void *arg)
         int u = J->next++;
         pthread_mutex_unlock(&J->lock);
         if (u >= J->N * J->H) break;
-        run_unit(J, u / J->H, u % J->H);
+        if (J->channel_gate) run_unit_kda(J, u / J->H, u % J->H);
+        else                 run_unit(J, u / J->H, u % J->H);
     }
     return NULL;
 }
 
-/* Returns 0 on success, -1 on bad arguments. `o` must hold B*T*H*d_v values;
- * `final_state` (nullable) N*H*d_k*d_v; `initial_state` nullable (zeros). */
-int gdn_oracle_chunk_fwd(const double *q, const double *k, const double *v,
-                         const double *g, const double *beta,
-                         const double *initial_state, const int32_t *cu_seqlens,
-                         int B, int T, int H, int d_k, int d_v, int num_seqs,
-                         double *o, double *final_state, int nthreads)
+static int run_all(const double *q, const double *k, const double *v,
+                   const double *g, const double *beta,
+                   const double *initial_state, const int32_t *cu_seqlens,
+                   int B, int T, int H, int d_k, int d_v, int num_seqs,
+                   double *o, double *final_state, int nthreads, int channel_gate)
 {
     if (!q || !k || !v || !g || !beta || !o) return -1;
     if (B < 1 || T < 0 || H < 1 || d_k < 1 || d_v < 1) return -1;
@@ -127,7 +201,7 @@ int gdn_oracle_chunk_fwd(const double *q, const double *k, const double *v,
         N = num_seqs;
     }
     job_t J = {q, k, v, g, beta, initial_state, cu_seqlens, o, final_state,
-               B, T, H, d_k, d_v, N, 0};
+               B, T, H, d_k, d_v, N, channel_gate, 0};
     pthread_mutex_init(&J.lock, NULL);
     if (nthreads < 1) nthreads = 1;
     if (nthreads > N * H) nthreads = N * H;
@@ -139,12 +213,33 @@ int gdn_oracle_chunk_fwd(const double *q, const double *k, const double *v,
     return 0;
 }
 
-/* One recurrent step for N*H independent states, in place:
- * state [N,H,d_k,d_v] (S^T storage), q/k [N,H,d_k], v/o [N,H,d_v], g/beta [N,H].
- * Same arithmetic as one iteration of the loop above. */
-int gdn_oracle_decode_step(const double *q, const double *k, const double *v,
-                           const double *g, const double *beta, double *state,
-                           double *o, int N, int H, int d_k, int d_v, int nthreads)
+/* Returns 0 on success, -1 on bad arguments. `o` must hold B*T*H*d_v values;
+ * `final_state` (nullable) N*H*d_k*d_v; `initial_state` nullable (zeros). */
+int gdn_oracle_chunk_fwd(const double *q, const double *k, const double *v,
+                         const double *g, const double *beta,
+                         const double *initial_state, const int32_t *cu_seqlens,
+                         int B, int T, int H, int d_k, int d_v, int num_seqs,
+                         double *o, double *final_state, int nthreads)
+{
+    return run_all(q, k, v, g, beta, initial_state, cu_seqlens, B, T, H, d_k, d_v,
+                   num_seqs, o, final_state, nthreads, 0);
+}
+
+/* Channel-wise gate: same contract, g = log(alpha) is [B, T, H, d_k]. */
+int gdn_oracle_kda_chunk_fwd(const double *q, const double *k, const double *v,
+                             const double *g, const double *beta,
+                             const double *initial_state, const int32_t *cu_seqlens,
+                             int B, int T, int H, int d_k, int d_v, int num_seqs,
+                             double *o, double *final_state, int nthreads)
+{
+    return run_all(q, k, v, g, beta, initial_state, cu_seqlens, B, T, H, d_k, d_v,
+                   num_seqs, o, final_state, nthreads, 1);
+}
+
+static int decode_all(const double *q, const double *k, const double *v,
+                      const double *g, const double *beta, double *state,
+                      double *o, int N, int H, int d_k, int d_v, int nthreads,
+                      int channel_gate)
 {
     if (!q || !k || !v || !g || !beta || !state || !o) return -1;
     if (N < 1 || H < 1 || d_k < 1 || d_v < 1) return -1;
@@ -153,10 +248,28 @@ int gdn_oracle_decode_step(const double *q, const double *k, const double *v,
     for (int n = 0; n <= N; ++n) cu[n] = n;
     double *s_out = (double *)malloc(sizeof(double) * (size_t)N * H * d_k * d_v);
     /* Tokens laid out as [1, N, H, d]: token index = n. */
-    int rc = gdn_oracle_chunk_fwd(q, k, v, g, beta, state, cu, 1, N, H, d_k, d_v, N,
-                                  o, s_out, nthreads);
+    int rc = run_all(q, k, v, g, beta, state, cu, 1, N, H, d_k, d_v, N,
+                     o, s_out, nthreads, channel_gate);
     if (rc == 0) memcpy(state, s_out, sizeof(double) * (size_t)N * H * d_k * d_v);
     free(s_out);
     free(cu);
     return rc;
+}
+
+/* One recurrent step for N*H independent states, in place:
+ * state [N,H,d_k,d_v] (S^T storage), q/k [N,H,d_k], v/o [N,H,d_v], g/beta [N,H].
+ * Same arithmetic as one iteration of the scalar-gate loop. */
+int gdn_oracle_decode_step(const double *q, const double *k, const double *v,
+                           const double *g, const double *beta, double *state,
+                           double *o, int N, int H, int d_k, int d_v, int nthreads)
+{
+    return decode_all(q, k, v, g, beta, state, o, N, H, d_k, d_v, nthreads, 0);
+}
+
+/* Channel-wise gate: g is [N, H, d_k]. */
+int gdn_oracle_kda_decode_step(const double *q, const double *k, const double *v,
+                               const double *g, const double *beta, double *state,
+                               double *o, int N, int H, int d_k, int d_v, int nthreads)
+{
+    return decode_all(q, k, v, g, beta, state, o, N, H, d_k, d_v, nthreads, 1);
 }

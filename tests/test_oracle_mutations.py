@@ -12,6 +12,7 @@ import subprocess
 import pytest
 
 import oracle
+import tests.test_oracle_kda_pins as kda_pins
 import tests.test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "gdn_oracle.c")
@@ -28,6 +29,32 @@ MUTATIONS = {
                            "S[(size_t)i * dk + j] = S[(size_t)i * dk + j] + u * kt[j];"),
 }
 
+# Mistakes in the channel-wise-gate loop, caught by its own pins.
+KDA_MUTATIONS = {
+    "kda_gate_ignored": ("for (int j = 0; j < dk; ++j) a[j] = exp(gt[j]);",
+                         "for (int j = 0; j < dk; ++j) a[j] = 1.0;"),
+    "kda_residual_from_undecayed_state": (
+        "acc += S[(size_t)i * dk + j] * a[j] * kt[j];",
+        "acc += S[(size_t)i * dk + j] * kt[j];"),
+    "kda_decay_after_write": (
+        "S[(size_t)i * dk + j] = a[j] * S[(size_t)i * dk + j] + ui * kt[j];",
+        "S[(size_t)i * dk + j] = a[j] * (S[(size_t)i * dk + j] + ui * kt[j]);"),
+    "kda_decay_on_value_axis": (
+        "S[(size_t)i * dk + j] = a[j] * S[(size_t)i * dk + j] + ui * kt[j];",
+        "S[(size_t)i * dk + j] = a[i % dk] * S[(size_t)i * dk + j] + ui * kt[j];"),
+    "kda_gate_of_previous_token": (
+        "const double *gt = J->g + row * dk;",
+        "const double *gt = J->g + (row >= (size_t)H ? row - H : row) * dk;"),
+}
+
+KDA_PIN_CASES = [
+    kda_pins.test_kda_hand_worked_two_tokens,
+    kda_pins.test_kda_equal_channels_is_scalar_gate,
+    kda_pins.test_kda_beta_zero_is_channel_decay,
+    lambda: kda_pins.test_kda_unit_key_beta_one_overwrites(3),
+    lambda: kda_pins.test_kda_dense_chunked_matches_token_loop(4, 7),
+]
+
 PIN_CASES = [
     pins.test_hand_worked_two_tokens,
     pins.test_beta_zero_is_pure_decay,
@@ -39,9 +66,10 @@ PIN_CASES = [
 ]
 
 
-@pytest.mark.parametrize("name", sorted(MUTATIONS))
+@pytest.mark.parametrize("name", sorted(MUTATIONS) + sorted(KDA_MUTATIONS))
 def test_planted_mistake_is_caught(name, tmp_path, monkeypatch):
-    before, after = MUTATIONS[name]
+    before, after = MUTATIONS[name] if name in MUTATIONS else KDA_MUTATIONS[name]
+    cases = PIN_CASES if name in MUTATIONS else KDA_PIN_CASES
     src = open(SRC).read()
     assert src.count(before) == 1, f"mutation anchor for {name} not unique"
     mutated = tmp_path / "mut.c"
@@ -51,12 +79,13 @@ def test_planted_mistake_is_caught(name, tmp_path, monkeypatch):
                            str(mutated), "-o", str(so), "-lm"])
     real = oracle._load()
     lib = ctypes.CDLL(str(so))
-    for fn in ("gdn_oracle_chunk_fwd", "gdn_oracle_decode_step"):
+    for fn in ("gdn_oracle_chunk_fwd", "gdn_oracle_decode_step", "gdn_oracle_kda_chunk_fwd",
+               "gdn_oracle_kda_decode_step"):
         getattr(lib, fn).argtypes = getattr(real, fn).argtypes
         getattr(lib, fn).restype = getattr(real, fn).restype
     monkeypatch.setattr(oracle, "_lib", lib)
     failures = 0
-    for case in PIN_CASES:
+    for case in cases:
         try:
             case()
         except AssertionError:
