@@ -14,6 +14,10 @@ independent copy of the workload (weak scaling, no collective on the data
 path); times are the max over ranks. ``--impl reference`` times the CPU fp64
 oracle (the slow, obviously-correct program the GPU path is checked
 against) on a bounded sample of the same workload.
+
+``--workload kda_b4h16t4096`` measures the channel-wise-gate variant instead
+(gdn_kda_chunk_fwd on the fp32 CUDA-core kernel, and gdn_kda_decode_step on
+the kda_decode workload); its roofline is the CUDA cores' fp32 FMA rate.
 """
 from __future__ import annotations
 
@@ -32,8 +36,13 @@ sys.path.insert(0, ROOT)
 WORKLOAD = "b4h16t4096"
 METRIC = "chunk-fwd Mtokens/s at B4·H16·T4096·d128 bf16; decode GB/s; % roofline"
 UNIT = "Mtokens/s"
+METRIC_KDA = ("chunk-fwd Mtokens/s at B4·H16·T4096·d128 bf16, channel-wise gate; "
+              "decode GB/s; % roofline")
 BYTES_PER_TOKEN_HEAD = 3 * 128 * 2 + 128 * 2 + 2 * 4    # q,k,v,o bf16 + g,beta fp32
+BYTES_PER_TOKEN_HEAD_KDA = 3 * 128 * 2 + 128 * 2 + 128 * 4 + 4   # g is one fp32 per channel
 L2_FLUSH_BYTES = 256 << 20
+# fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 flop x 1965 MHz (max SM clock)
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def parse_args():
@@ -51,23 +60,33 @@ def parse_args():
     return p.parse_args()
 
 
-def kernel_source_hash() -> str:
-    """Hash of the CUDA sources: ncu traffic figures are only reported for the
-    exact kernels they were measured on."""
-    import glob
+# The sources each measured kernel set is built from (under csrc/).
+KERNEL_SOURCES = {
+    "chunk_fwd_step": ["chunk_map.cu", "chunk_tc.cu", "gdn_internal.cuh", "sm100_ptx.cuh"],
+    "kda_chunk_fwd_step": ["chunk_map.cu", "chunk_simt.cu", "gdn_internal.cuh",
+                           "sm100_ptx.cuh"],
+    "decode": ["decode.cu", "gdn_internal.cuh", "sm100_ptx.cuh"],
+}
+
+
+def kernel_source_hash(kind: str) -> str:
+    """Hash of the sources of one kernel set: ncu traffic figures are only
+    reported for the exact kernels they were measured on."""
     import hashlib
     h = hashlib.sha256()
-    for path in sorted(glob.glob(os.path.join(ROOT, "gated_delta_rule_112_b200", "csrc", "*"))):
-        h.update(open(path, "rb").read())
+    for name in KERNEL_SOURCES[kind]:
+        h.update(open(os.path.join(ROOT, "gated_delta_rule_112_b200", "csrc", name), "rb").read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(key):
+    """DRAM bytes per launch recorded for `key` ("<kind>/<workload>"), or None
+    when there is no record or the kernels changed since it was taken."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     rec = json.load(open(path)).get(key)
-    if not rec or rec.get("src_hash") != kernel_source_hash():
+    if not rec or rec.get("src_hash") != kernel_source_hash(key.split("/")[0]):
         return None
     return rec["dram_bytes_per_launch"]
 
@@ -145,6 +164,8 @@ def run_reference(args):
     import oracle
     from gated_delta_rule_112_b200.inputs import make_chunk_inputs
     inp = make_chunk_inputs(args.workload)
+    kda = inp["gate"] == "channel"
+    run = oracle.kda_chunk_fwd if kda else oracle.chunk_fwd
     heads = [0, 1]                              # sample: 2 of 16 heads, all B*T tokens
     arr = {k: inp[k][:, :, heads].float().double().numpy() for k in ("q", "k", "v", "g", "beta")}
     cores = oracle.default_threads()
@@ -155,8 +176,7 @@ def run_reference(args):
     cu = inp["cu_seqlens"].numpy() if inp["cu_seqlens"] is not None else None
 
     def one():
-        oracle.chunk_fwd(arr["q"], arr["k"], arr["v"], arr["g"], arr["beta"], s0, cu,
-                         nthreads=cores)
+        run(arr["q"], arr["k"], arr["v"], arr["g"], arr["beta"], s0, cu, nthreads=cores)
     for _ in range(args.warmup):
         one()
     t0 = time.perf_counter()
@@ -166,7 +186,8 @@ def run_reference(args):
     value = tok_equiv / dt / 1e6
     sample = (f"oracle on {len(heads)} of {inp['H']} heads x B{inp['B']} x T{inp['T']} "
               f"per step ({int(tok_equiv)} full-width tokens)")
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+    line = {"impl": "reference", "metric": METRIC_KDA if kda else METRIC, "value": value,
+            "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -219,6 +240,9 @@ def main():
     wl = args.workload
     seed = replicas.shard_seed(WORKLOADS[wl].seed, rank)
     inp = make_chunk_inputs(wl, seed=seed)
+    kda = inp["gate"] == "channel"
+    fwd = gdn.kda_chunk_fwd if kda else gdn.chunk_fwd
+    ws_size = gdn.kda_workspace_size if kda else gdn.workspace_size
     B, T, H = inp["B"], inp["T"], inp["H"]
     q, k, v, g, beta = (inp[x].to(dev) for x in ("q", "k", "v", "g", "beta"))
     s0 = inp["initial_state"].to(dev) if inp["initial_state"] is not None else None
@@ -226,12 +250,12 @@ def main():
     nseq = B if cu is None else cu.numel() - 1
     o = torch.empty(B, T, H, 128, dtype=torch.bfloat16, device=dev)
     fs = torch.empty(nseq, H, 128, 128, dtype=torch.float32, device=dev)
-    ws = torch.empty(gdn.workspace_size(B, T, H, 128, 128, 0 if cu is None else nseq),
+    ws = torch.empty(ws_size(B, T, H, 128, 128, 0 if cu is None else nseq),
                      dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def step():
-        gdn.chunk_fwd(q, k, v, g, beta, s0, cu, out=o, workspace=ws)
+        fwd(q, k, v, g, beta, s0, cu, out=o, workspace=ws)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -288,16 +312,21 @@ def main():
     value = replicas.job_rate(tokens, ms, world) / 1e6
 
     state_io = (2 if s0 is not None else 1) * nseq * H * 128 * 128 * 4   # final (+ initial) state
-    alg_bytes = tokens * H * BYTES_PER_TOKEN_HEAD + state_io
+    alg_bytes = tokens * H * (BYTES_PER_TOKEN_HEAD_KDA if kda else BYTES_PER_TOKEN_HEAD) \
+        + state_io
     flops = tokens * H * 2 * (3 * 64 * 128 + 2 * 64 * 128 + 3 * 128 * 128)
     ach_gbs = alg_bytes / (ms_local * 1e-3) / 1e9
-    kernels = {
-        "gdn_chunk_map_kernel": statistics.mean(t_map),
-        "gdn_prep_kernel": statistics.mean(t_prep),
-        "gdn_scan_kernel": statistics.mean(t_scan),
-    }
+    if kda:   # one CUDA-core kernel after the chunk map (prep/scan events coincide)
+        kernels = {"gdn_chunk_map_kernel": statistics.mean(t_map),
+                   "gdn_chunk_simt_kernel": statistics.mean(t_scan)}
+    else:
+        kernels = {
+            "gdn_chunk_map_kernel": statistics.mean(t_map),
+            "gdn_prep_kernel": statistics.mean(t_prep),
+            "gdn_scan_kernel": statistics.mean(t_scan),
+        }
     tot = sum(kernels.values())
-    traffic = recorded_traffic("chunk_fwd_step/" + wl)
+    traffic = recorded_traffic(("kda_chunk_fwd_step/" if kda else "chunk_fwd_step/") + wl)
 
     # --------------------------------------------------------------- end to end (host buffers)
     e2e = None
@@ -311,7 +340,7 @@ def main():
         def e2e_step_with_state():
             for dst, src in ((q, hq), (k, hk), (v, hv), (g, hg), (beta, hb)):
                 dst.copy_(src, non_blocking=True)
-            _, f = gdn.chunk_fwd(q, k, v, g, beta, s0, cu, out=o, workspace=ws)
+            _, f = fwd(q, k, v, g, beta, s0, cu, out=o, workspace=ws)
             ho.copy_(o, non_blocking=True)
             hfs.copy_(f, non_blocking=True)
 
@@ -333,7 +362,9 @@ def main():
         ms_e2e = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / ke)
         e2e = {"value": replicas.job_rate(tokens, ms_e2e, world) / 1e6, "unit": UNIT,
                "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "steps": ke, "api": "gated_delta_rule_112_b200.chunk_fwd (C ABI gdn_chunk_fwd)"}
+               "steps": ke,
+               "api": ("gated_delta_rule_112_b200.kda_chunk_fwd (C ABI gdn_kda_chunk_fwd)" if kda
+                       else "gated_delta_rule_112_b200.chunk_fwd (C ABI gdn_chunk_fwd)")}
         del hq, hk, hv, hg, hb, ho, hfs
 
     del q, k, v, g, beta, o, ws
@@ -342,13 +373,15 @@ def main():
     # --------------------------------------------------------------- decode step
     decode = None
     if not args.no_decode:
-        d = make_decode_inputs("decode", seed=replicas.shard_seed(4, rank))
+        dwl = "kda_decode" if kda else "decode"
+        d = make_decode_inputs(dwl, seed=replicas.shard_seed(WORKLOADS[dwl].seed, rank))
+        dstep = gdn.kda_decode_step if kda else gdn.decode_step
         N, Hd, S = d["N"], d["H"], d["steps"]
         dq, dk, dvv, dg, db = (d[x].to(dev) for x in ("q", "k", "v", "g", "beta"))
         st = d["state"].to(dev)
         do = torch.empty(N, Hd, 128, dtype=torch.bfloat16, device=dev)
         for t in range(3):
-            gdn.decode_step(dq[t], dk[t], dvv[t], dg[t], db[t], st, out=do)
+            dstep(dq[t], dk[t], dvv[t], dg[t], db[t], st, out=do)
         st.copy_(d["state"].to(dev))
         torch.cuda.synchronize()
         reps = 3
@@ -359,21 +392,21 @@ def main():
             torch.cuda.synchronize()
             a.record(stream)
             for t in range(S):
-                gdn.decode_step(dq[t], dk[t], dvv[t], dg[t], db[t], st, out=do)
+                dstep(dq[t], dk[t], dvv[t], dg[t], db[t], st, out=do)
             b.record(stream)
             torch.cuda.synchronize()
             times.append(a.elapsed_time(b) / S)
         barrier()
         us = max_over_ranks(statistics.median(times)) * 1e3
         bytes_step = (2 * N * Hd * 128 * 128 * 4 + 3 * N * Hd * 128 * 2 + N * Hd * 128 * 2
-                      + 2 * N * Hd * 4)
+                      + N * Hd * 4 + N * Hd * (128 if kda else 1) * 4)
         gbs = bytes_step / (us * 1e-6) / 1e9
-        decode = {"workload": "decode N256 H32 d128 fp32 state, 64 steps", "us_per_step": us,
+        decode = {"workload": f"{dwl} N256 H32 d128 fp32 state, 64 steps", "us_per_step": us,
                   "value": world * gbs, "unit": "GB/s", "bytes_per_step": bytes_step,
                   "gpu_launches": reps * S,
                   "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"],
                                "unit": "GB/s", "frac": gbs / pk["hbm"],
-                               "traffic": recorded_traffic("decode/n256h32"),
+                               "traffic": recorded_traffic(f"decode/{dwl}_n256h32"),
                                "kernel": "gdn_decode_kernel", "peak_source": pk["source"]}}
         del dq, dk, dvv, dg, db, st, do
 
@@ -384,33 +417,46 @@ def main():
         arr = {x: inp[x].float().double().numpy() for x in ("q", "k", "v", "g", "beta")}
         cores = oracle.default_threads()
         t0 = time.perf_counter()
-        oracle.chunk_fwd(arr["q"], arr["k"], arr["v"], arr["g"], arr["beta"], None, None,
-                         nthreads=cores)
+        (oracle.kda_chunk_fwd if kda else oracle.chunk_fwd)(
+            arr["q"], arr["k"], arr["v"], arr["g"], arr["beta"], None, None, nthreads=cores)
         dt = time.perf_counter() - t0
         cpu = {"value": tokens / dt / 1e6, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"the whole workload once (B{B} T{T} H{H}, {dt:.2f} s)"}
 
+    if kda:
+        tflops = flops / (ms_local * 1e-3) / 1e12
+        roof = {"bound": "alu", "achieved": tflops, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
+                "frac": tflops / FP32_ALU_TFLOPS, "traffic": traffic,
+                "kernel": "gdn_chunk_simt_kernel (channel-wise gate, fp32 CUDA cores)",
+                "algorithmic_bytes": alg_bytes, "flops": flops,
+                "hbm_frac": ach_gbs / pk["hbm"],
+                "peak_source": "fp32 FMA rate from unit counts: 148 SMs x 128 lanes x 2 flop "
+                               "x 1965 MHz"}
+    else:
+        roof = {"bound": "hbm", "achieved": ach_gbs, "peak": pk["hbm"], "unit": "GB/s",
+                "frac": ach_gbs / pk["hbm"], "traffic": traffic,
+                "kernel": "gdn_chunk_fwd step (chunk_map + prep + scan)",
+                "algorithmic_bytes": alg_bytes, "flops": flops,
+                "tensor_frac": flops / (ms_local * 1e-3) / (pk["bf16"] * 1e12),
+                "peak_source": pk["source"]}
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "metric": METRIC_KDA if kda else METRIC, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl, "B": B, "T": T, "H": H, "d_k": 128, "d_v": 128,
                    "chunk": 64, "sequences": nseq,
+                   "gate": "channel-wise [B,T,H,d_k]" if kda else "scalar [B,T,H]",
                    "initial_state": "zeros" if s0 is None else "random",
                    "final_state": True,
                    "l2": "flushed before every timed step (256 MiB device write)",
                    "parallelism": f"{world} independent replica(s), no collective"},
-        "roofline": {"bound": "hbm", "achieved": ach_gbs, "peak": pk["hbm"], "unit": "GB/s",
-                     "frac": ach_gbs / pk["hbm"], "traffic": traffic,
-                     "kernel": "gdn_chunk_fwd step (chunk_map + prep + scan)",
-                     "algorithmic_bytes": alg_bytes, "flops": flops,
-                     "tensor_frac": flops / (ms_local * 1e-3) / (pk["bf16"] * 1e12),
-                     "peak_source": pk["source"]},
+        "roofline": roof,
         "kernels_ms": kernels,
         "kernel_share": {k2: v2 / tot for k2, v2 in kernels.items()},
         "kernels_note": "per-kernel times from an untimed pass with events between the "
                         "launches (no launch overlap); ms_per_step is the timed region",
-        "gpu_launches": 3 * K,
+        "gpu_launches": (2 if kda else 3) * K,
         "clocks": clocks,
         "e2e": e2e,
         "decode": decode,
@@ -423,4 +469,7 @@ def main():
 
 
 if __name__ == "__main__":
-    main()
+    if len(sys.argv) == 2 and sys.argv[1] == "--source-hashes":
+        print(json.dumps({kind: kernel_source_hash(kind) for kind in KERNEL_SOURCES}))
+    else:
+        main()

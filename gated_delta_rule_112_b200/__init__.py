@@ -66,6 +66,12 @@ def lib() -> ctypes.CDLL:
         L.gdn_chunk_fwd_path.restype = ci
         L.gdn_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, ci, ci, ci, ci, ci, vp]
         L.gdn_decode_step.restype = ci
+        L.gdn_kda_chunk_fwd.argtypes = chunk_args
+        L.gdn_kda_chunk_fwd.restype = ci
+        L.gdn_kda_chunk_fwd_workspace_size.argtypes = [ci] * 8
+        L.gdn_kda_chunk_fwd_workspace_size.restype = sz
+        L.gdn_kda_decode_step.argtypes = L.gdn_decode_step.argtypes
+        L.gdn_kda_decode_step.restype = ci
         L.gdn_get_status.argtypes = [vp, vp]
         L.gdn_get_status.restype = ci
         L.gdn_set_profile_events.argtypes = [vp, vp, vp, vp]
@@ -122,25 +128,49 @@ def chunk_fwd(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk=64,
     alpha), beta: [B,T,H] fp32; initial_state: [N,H,d_k,d_v] fp32 or None;
     cu_seqlens: int32 [N+1] CUDA tensor (packed sequences, B == 1) or None.
     """
+    fn = lib().gdn_chunk_fwd_simt if force_simt else lib().gdn_chunk_fwd
+    return _chunk_call(fn, "gdn_chunk_fwd", lib().gdn_chunk_fwd_workspace_size, q, k, v, g,
+                       beta, initial_state, cu_seqlens, chunk, output_final_state, workspace,
+                       out, stream, channel_gate=False)
+
+
+def kda_workspace_size(B, T, H, d_k, d_v, num_seqs=0, chunk=64, dtype=torch.bfloat16) -> int:
+    return int(lib().gdn_kda_chunk_fwd_workspace_size(B, T, H, d_k, d_v, num_seqs, chunk,
+                                                      _dtype_code(dtype)))
+
+
+def kda_chunk_fwd(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk=64,
+                  output_final_state=True, workspace=None, out=None, stream=None):
+    """Chunkwise forward pass with the channel-wise gate: as ``chunk_fwd`` but
+    g (= log alpha) is [B,T,H,d_k] fp32. Returns ``(o, final_state or None)``."""
+    return _chunk_call(lib().gdn_kda_chunk_fwd, "gdn_kda_chunk_fwd",
+                       lib().gdn_kda_chunk_fwd_workspace_size, q, k, v, g, beta, initial_state,
+                       cu_seqlens, chunk, output_final_state, workspace, out, stream,
+                       channel_gate=True)
+
+
+def _chunk_call(fn, name, ws_fn, q, k, v, g, beta, initial_state, cu_seqlens, chunk,
+                output_final_state, workspace, out, stream, channel_gate):
     _require_cuda(q, k, v, g, beta, initial_state, cu_seqlens)
     B, T, H, dk = q.shape
     dv = v.shape[-1]
+    if tuple(g.shape) != ((B, T, H, dk) if channel_gate else (B, T, H)):
+        raise ValueError(f"{name}: g has shape {tuple(g.shape)}")
     num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
     N = num_seqs if cu_seqlens is not None else B
     dt = _dtype_code(q.dtype)
     o = torch.empty(B, T, H, dv, dtype=q.dtype, device=q.device) if out is None else out
     fs = (torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device)
           if output_final_state else None)
-    need = workspace_size(B, T, H, dk, dv, num_seqs, chunk, q.dtype)
+    need = int(ws_fn(B, T, H, dk, dv, num_seqs, chunk, dt))
     if need == 0:
-        raise GdnError(ERR_INVALID_ARG, "gdn_chunk_fwd_workspace_size")
+        raise GdnError(ERR_INVALID_ARG, name + "_workspace_size")
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    fn = lib().gdn_chunk_fwd_simt if force_simt else lib().gdn_chunk_fwd
     rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
             _ptr(cu_seqlens), B, T, H, dk, dv, num_seqs, chunk, dt, _ptr(o), _ptr(fs),
             _ptr(workspace), workspace.numel(), _stream_ptr(stream))
-    _check(rc, "gdn_chunk_fwd")
+    _check(rc, name)
     return o, fs
 
 
@@ -154,11 +184,24 @@ def decode_step(q, k, v, g, beta, state, out=None, stream=None):
 
     q, k: [N,H,d_k]; v: [N,H,d_v]; g, beta: [N,H] fp32. Returns o [N,H,d_v].
     """
+    return _decode_call(lib().gdn_decode_step, "gdn_decode_step", q, k, v, g, beta, state,
+                        out, stream, channel_gate=False)
+
+
+def kda_decode_step(q, k, v, g, beta, state, out=None, stream=None):
+    """One channel-wise-gated step (g: [N,H,d_k] fp32), ``state`` updated in place."""
+    return _decode_call(lib().gdn_kda_decode_step, "gdn_kda_decode_step", q, k, v, g, beta,
+                        state, out, stream, channel_gate=True)
+
+
+def _decode_call(fn, name, q, k, v, g, beta, state, out, stream, channel_gate):
     _require_cuda(q, k, v, g, beta, state)
     N, H, dk = q.shape
     dv = v.shape[-1]
+    if tuple(g.shape) != ((N, H, dk) if channel_gate else (N, H)):
+        raise ValueError(f"{name}: g has shape {tuple(g.shape)}")
     o = torch.empty(N, H, dv, dtype=q.dtype, device=q.device) if out is None else out
-    rc = lib().gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state),
-                               _ptr(o), N, H, dk, dv, _dtype_code(q.dtype), _stream_ptr(stream))
-    _check(rc, "gdn_decode_step")
+    rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), _ptr(o), N, H, dk, dv,
+            _dtype_code(q.dtype), _stream_ptr(stream))
+    _check(rc, name)
     return o

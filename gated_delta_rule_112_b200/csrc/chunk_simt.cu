@@ -1,5 +1,4 @@
-// Chunk bookkeeping shared by both chunked-forward paths, and the fp32
-// CUDA-core implementation of the chunkwise WY / UT-transform forward pass
+// The fp32 CUDA-core implementation of the chunkwise WY / UT-transform forward pass
 // ("Gated Delta Networks", phantomic12 page, mechanism paragraph; LIT-137,
 // "Standing in the anthology": the WY-based chunkwise algorithm extended to
 // carry the gate). This path serves fp32 inputs (where fp32 accuracy is
@@ -12,102 +11,23 @@
 //   S <- exp(Gamma_last) S + V_new^T diag(exp(Gamma_last - Gamma)) K
 // Rows past a sequence's end are treated as k = q = v = 0, beta = g = 0,
 // which leaves S unchanged; their outputs are not written.
+//
+// Channel-wise gate (the Kimi Delta Attention variant: dmarx anthology
+// LIT-137, "Standing in the anthology"; SOTA-135, "Sequence"), g = log alpha
+// per (token, head, d_k channel), S_t = S_{t-1} diag(alpha_t)(I - beta_t k_t
+// k_t^T) + beta_t v_t k_t^T. Gamma is then a cumsum per channel and the decay
+// moves inside the dot products:
+//   A_rs = beta_r sum_j k_rj k_sj exp(Gamma_rj - Gamma_sj)  (s < r)
+//   P_rs = sum_j q_rj k_sj exp(Gamma_rj - Gamma_sj)         (s <= r)
+//   W = T diag(beta) (K .* exp(Gamma)),  O = (Q .* exp(Gamma)) S^T + P V_new
+//   S <- S diag(exp(Gamma_last)) + V_new^T (K .* exp(Gamma_last - Gamma))
+// Every exponent is a difference of cumulative sums over the tokens in
+// between, so with alpha <= 1 no factor exceeds 1.
 #include "gdn_internal.cuh"
 #include "sm100_ptx.cuh"
 
 namespace gdn {
 namespace {
-
-// ---------------------------------------------------------------------------
-// Chunk map: validates cu_seqlens and lists every (sequence, chunk).
-// One CTA of 1024 threads; thread t owns a contiguous range of sequences.
-__global__ void __launch_bounds__(1024) gdn_chunk_map_kernel(
-    const int32_t *__restrict__ cu, int B, int T, int num_seqs, int chunk,
-    uint32_t *__restrict__ ctrl, ChunkInfo *__restrict__ table,
-    int32_t *__restrict__ seq_first, int max_chunks, int segs, int32_t *__restrict__ seg_first) {
-  // The kernels launched after this one may start their prologues now; they
-  // wait for this grid before reading what it writes.
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int N = num_seqs > 0 ? num_seqs : B;
-  const int tid = threadIdx.x;
-  if (!cu) {
-    // B sequences of T tokens: every entry has a closed form.
-    const int cps = (T + chunk - 1) / chunk;
-    const int total = B * cps;
-    for (int idx = tid; idx < total; idx += blockDim.x) {
-      const int n = idx / cps, c = idx - n * cps;
-      ChunkInfo ci;
-      ci.seq = n;
-      ci.cidx = c;
-      ci.row0 = n * T + c * chunk;
-      ci.len = min(chunk, T - c * chunk);
-      table[idx] = ci;
-    }
-    for (int n = tid; n <= N; n += blockDim.x) seq_first[n] = n * cps;
-    if (segs > 1) {
-      // segment g of sequence n: chunks [n cps + g len, min(n cps + (g + 1) len, (n + 1) cps))
-      const int len = (cps + segs - 1) / segs;
-      for (int e = tid; e <= N * segs; e += blockDim.x) {
-        const int n = e / segs, gi = e - n * segs;
-        seg_first[e] = (n >= N) ? N * cps : n * cps + min(gi * len, cps);
-      }
-    }
-    if (tid == 0) {
-      ctrl[0] = 0;
-      ctrl[1] = uint32_t(total);
-    }
-    return;
-  }
-  __shared__ int32_t scan[1024];
-  __shared__ int bad;
-  if (tid == 0) bad = 0;
-  __syncthreads();
-  const int per = (N + 1023) / 1024;
-  const int n0 = min(N, tid * per), n1 = min(N, n0 + per);
-  int32_t local = 0;
-  for (int n = n0; n < n1; ++n) {
-    const int a = cu[n], b = cu[n + 1];
-    if ((n == 0 && a != 0) || b < a || (n == N - 1 && b != T)) bad = 1;
-    const int len = b - a;
-    if (len > 0) local += (len + chunk - 1) / chunk;
-  }
-  scan[tid] = local;
-  __syncthreads();
-  for (int off = 1; off < 1024; off <<= 1) {
-    const int32_t add = tid >= off ? scan[tid - off] : 0;
-    __syncthreads();
-    scan[tid] += add;
-    __syncthreads();
-  }
-  const int32_t total = scan[1023];
-  if (bad || total > max_chunks) {
-    if (tid == 0) {
-      ctrl[0] = kErrBadSeqlens;
-      ctrl[1] = 0;
-    }
-    return;
-  }
-  int32_t first = scan[tid] - local;
-  for (int n = n0; n < n1; ++n) {
-    const int row0 = cu[n];
-    const int len = cu[n + 1] - row0;
-    seq_first[n] = first;
-    for (int c = 0; c * chunk < len; ++c) {
-      ChunkInfo ci;
-      ci.seq = n;
-      ci.cidx = c;
-      ci.row0 = row0 + c * chunk;
-      ci.len = min(chunk, len - c * chunk);
-      table[first + c] = ci;
-    }
-    if (len > 0) first += (len + chunk - 1) / chunk;
-  }
-  if (tid == 1023) seq_first[N] = total;
-  if (tid == 0) {
-    ctrl[0] = 0;
-    ctrl[1] = uint32_t(total);
-  }
-}
 
 template <typename T>
 __device__ __forceinline__ float ld_f32(const T *p);
@@ -132,8 +52,8 @@ constexpr int kDvt = 32;  // d_v columns per CTA
 // ---------------------------------------------------------------------------
 // fp32 chunked forward. Grid (N, H, ceil(d_v / 32)); one CTA walks all chunks
 // of one sequence for one head and one 32-column slice of d_v, carrying its
-// slice of the state in shared memory.
-template <int C, typename T>
+// slice of the state in shared memory. KDA: channel-wise gate (g [rows, H, d_k]).
+template <int C, typename T, bool KDA>
 __global__ void __launch_bounds__(kSimtThreads) gdn_chunk_simt_kernel(
     const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
     const float *__restrict__ g, const float *__restrict__ beta, const float *__restrict__ s0,
@@ -159,6 +79,9 @@ __global__ void __launch_bounds__(kSimtThreads) gdn_chunk_simt_kernel(
   float *Bt = Gm + C;                    // [C] beta
   float *Ga = Bt + C;                    // [C] exp(Gamma)
   float *Dd = Ga + C;                    // [C] exp(Gamma_last - Gamma)
+  // KDA only: per-channel Gamma, then K .* exp(Gamma); and Gamma_last per channel
+  float *Gk = Dd + C;                    // [C][dkp]
+  float *Gl = Gk + C * dkp;              // [dk]
 
   // Initial state slice.
   for (int e = tid; e < dk * kDvt; e += kSimtThreads) {
@@ -192,17 +115,28 @@ __global__ void __launch_bounds__(kSimtThreads) gdn_chunk_simt_kernel(
     }
     if (tid < C) {
       const bool ok = tid < L;
-      Gm[tid] = ok ? g[size_t(ci.row0 + tid) * H + h] : 0.f;
+      if (!KDA) Gm[tid] = ok ? g[size_t(ci.row0 + tid) * H + h] : 0.f;
       Bt[tid] = ok ? beta[size_t(ci.row0 + tid) * H + h] : 0.f;
+    }
+    if (KDA) {
+      for (int e = tid; e < C * dk; e += kSimtThreads) {
+        const int r = e / dk, j = e % dk;
+        Gk[r * dkp + j] = r < L ? g[(size_t(ci.row0 + r) * H + h) * dk + j] : 0.f;
+      }
     }
     __syncthreads();
     // 2. cumulative log-gate and the decay factors
-    if (tid == 0) {
+    if (!KDA && tid == 0) {
       float acc = 0.f;
       for (int r = 0; r < C; ++r) { acc += Gm[r]; Gm[r] = acc; }
     }
+    if (KDA && tid < dk) {   // one channel per thread
+      float acc = 0.f;
+      for (int r = 0; r < C; ++r) { acc += Gk[r * dkp + tid]; Gk[r * dkp + tid] = acc; }
+      Gl[tid] = acc;
+    }
     __syncthreads();
-    if (tid < C) {
+    if (!KDA && tid < C) {
       Ga[tid] = expf(Gm[tid]);
       Dd[tid] = expf(Gm[C - 1] - Gm[tid]);
     }
@@ -212,19 +146,40 @@ __global__ void __launch_bounds__(kSimtThreads) gdn_chunk_simt_kernel(
       float a = 0.f, p = 0.f;
       if (s <= r) {
         float dkk = 0.f, dqk = 0.f;
-        for (int j = 0; j < dk; ++j) {
-          const float ksj = Ks[s * dkp + j];
-          dkk += Ks[r * dkp + j] * ksj;
-          dqk += Qs[r * dkp + j] * ksj;
+        if (KDA) {
+          for (int j = 0; j < dk; ++j) {
+            const float ksj = Ks[s * dkp + j] * expf(Gk[r * dkp + j] - Gk[s * dkp + j]);
+            dkk += Ks[r * dkp + j] * ksj;
+            dqk += Qs[r * dkp + j] * ksj;
+          }
+          if (s < r) a = Bt[r] * dkk;
+          p = dqk;
+        } else {
+          for (int j = 0; j < dk; ++j) {
+            const float ksj = Ks[s * dkp + j];
+            dkk += Ks[r * dkp + j] * ksj;
+            dqk += Qs[r * dkp + j] * ksj;
+          }
+          const float decay = expf(Gm[r] - Gm[s]);
+          if (s < r) a = Bt[r] * decay * dkk;
+          p = decay * dqk;
         }
-        const float decay = expf(Gm[r] - Gm[s]);
-        if (s < r) a = Bt[r] * decay * dkk;
-        p = decay * dqk;
       }
       As[r * (C + 1) + s] = a;
       Ps[r * (C + 1) + s] = p;
     }
     __syncthreads();
+    if (KDA) {
+      // K and Q now enter only with their decays: Gk <- K .* exp(Gamma) (for W),
+      // Ks <- K .* exp(Gamma_last - Gamma) (state update), Qs <- Q .* exp(Gamma).
+      for (int e = tid; e < C * dk; e += kSimtThreads) {
+        const int r = e / dk, j = e % dk;
+        const float gam = Gk[r * dkp + j], kv = Ks[r * dkp + j];
+        Gk[r * dkp + j] = kv * expf(gam);
+        Ks[r * dkp + j] = kv * expf(Gl[j] - gam);
+        Qs[r * dkp + j] *= expf(gam);
+      }
+    }
     // 4. T = (I + A)^-1 by forward substitution; thread s owns column s.
     if (tid < C) {
       const int s = tid;
@@ -240,7 +195,11 @@ __global__ void __launch_bounds__(kSimtThreads) gdn_chunk_simt_kernel(
     for (int e = tid; e < C * dk; e += kSimtThreads) {
       const int r = e / dk, j = e % dk;
       float acc = 0.f;
-      for (int s = 0; s <= r; ++s) acc += Ts[r * (C + 1) + s] * (Bt[s] * Ga[s]) * Ks[s * dkp + j];
+      if (KDA)
+        for (int s = 0; s <= r; ++s) acc += Ts[r * (C + 1) + s] * Bt[s] * Gk[s * dkp + j];
+      else
+        for (int s = 0; s <= r; ++s)
+          acc += Ts[r * (C + 1) + s] * (Bt[s] * Ga[s]) * Ks[s * dkp + j];
       Ws[r * dkp + j] = acc;
     }
     for (int e = tid; e < C * kDvt; e += kSimtThreads) {
@@ -266,17 +225,22 @@ __global__ void __launch_bounds__(kSimtThreads) gdn_chunk_simt_kernel(
         for (int j = 0; j < dk; ++j) acc += Qs[r * dkp + j] * Ss[j * kDvt + ii];
         float acc2 = 0.f;
         for (int s = 0; s <= r; ++s) acc2 += Ps[r * (C + 1) + s] * Vn[s * kDvt + ii];
-        st_from_f32(o + (size_t(ci.row0 + r) * H + h) * dv + i0 + ii, Ga[r] * acc + acc2);
+        st_from_f32(o + (size_t(ci.row0 + r) * H + h) * dv + i0 + ii,
+                    (KDA ? acc : Ga[r] * acc) + acc2);
       }
     }
     __syncthreads();
     // 8. S <- gamma_last S + V_new^T diag(D) K
-    const float glast = Ga[C - 1];
     for (int e = tid; e < dk * kDvt; e += kSimtThreads) {
       const int j = e / kDvt, ii = e % kDvt;
       float acc = 0.f;
-      for (int s = 0; s < C; ++s) acc += Dd[s] * Ks[s * dkp + j] * Vn[s * kDvt + ii];
-      Ss[e] = glast * Ss[e] + acc;
+      if (KDA) {
+        for (int s = 0; s < C; ++s) acc += Ks[s * dkp + j] * Vn[s * kDvt + ii];
+        Ss[e] = expf(Gl[j]) * Ss[e] + acc;
+      } else {
+        for (int s = 0; s < C; ++s) acc += Dd[s] * Ks[s * dkp + j] * Vn[s * kDvt + ii];
+        Ss[e] = Ga[C - 1] * Ss[e] + acc;
+      }
     }
   }
   __syncthreads();
@@ -288,15 +252,16 @@ __global__ void __launch_bounds__(kSimtThreads) gdn_chunk_simt_kernel(
   }
 }
 
-template <int C, typename T>
+template <int C, typename T, bool KDA>
 cudaError_t launch_simt_t(const void *q, const void *k, const void *v, const float *g,
                           const float *beta, const float *s0, int H, int dk, int dv, int N,
                           void *o, float *sN, uint32_t *ctrl, const ChunkInfo *table,
                           const int32_t *seq_first, cudaStream_t s) {
   const size_t floats = size_t(3) * C * (dk + 1) + size_t(3) * C * kDvt + size_t(dk) * kDvt +
-                        size_t(3) * C * (C + 1) + 4 * C;
+                        size_t(3) * C * (C + 1) + 4 * C +
+                        (KDA ? size_t(C) * (dk + 1) + dk : 0);
   const size_t bytes = floats * sizeof(float);
-  auto kern = gdn_chunk_simt_kernel<C, T>;
+  auto kern = gdn_chunk_simt_kernel<C, T, KDA>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(bytes));
   if (e != cudaSuccess) return e;
@@ -309,38 +274,29 @@ cudaError_t launch_simt_t(const void *q, const void *k, const void *v, const flo
 
 }  // namespace
 
-cudaError_t launch_chunk_map(const int32_t *cu_seqlens, int B, int T, int num_seqs, int chunk,
-                             void *ws, const WsLayout &L, cudaStream_t s) {
-  char *base = static_cast<char *>(ws);
-  // The kernel writes the control block itself (error word, chunk count).
-  gdn_chunk_map_kernel<<<1, 1024, 0, s>>>(
-      cu_seqlens, B, T, num_seqs, chunk, reinterpret_cast<uint32_t *>(base),
-      reinterpret_cast<ChunkInfo *>(base + L.chunk_table),
-      reinterpret_cast<int32_t *>(base + L.seq_first), L.max_chunks, L.segs,
-      L.segs > 1 ? reinterpret_cast<int32_t *>(base + L.seg_first) : nullptr);
-  return cudaGetLastError();
-}
-
 cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const float *g,
                               const float *beta, const float *s0, const int32_t *cu, int B,
                               int T, int H, int dk, int dv, int N, int chunk, int dtype, void *o,
-                              float *sN, uint32_t *ws_ctrl, cudaStream_t s) {
+                              float *sN, uint32_t *ws_ctrl, cudaStream_t s, bool channel_gate) {
   (void)cu; (void)B; (void)T;
   char *base = reinterpret_cast<char *>(ws_ctrl);
   // The layout of the chunk table is the same for both paths.
   const WsLayout L = ws_layout(B, T, H, cu ? N : 0, chunk, false);
   const ChunkInfo *table = reinterpret_cast<const ChunkInfo *>(base + L.chunk_table);
   const int32_t *seq_first = reinterpret_cast<const int32_t *>(base + L.seq_first);
-#define GDN_SIMT_CASE(CC)                                                                       \
-  if (chunk == CC)                                                                               \
+#define GDN_SIMT_CASE(CC, KK)                                                                   \
+  if (chunk == CC && channel_gate == KK)                                                         \
     return dtype == GDN_BF16                                                                     \
-               ? launch_simt_t<CC, __nv_bfloat16>(q, k, v, g, beta, s0, H, dk, dv, N, o, sN,   \
-                                                  ws_ctrl, table, seq_first, s)                 \
-               : launch_simt_t<CC, float>(q, k, v, g, beta, s0, H, dk, dv, N, o, sN, ws_ctrl,  \
-                                          table, seq_first, s);
-  GDN_SIMT_CASE(16)
-  GDN_SIMT_CASE(32)
-  GDN_SIMT_CASE(64)
+               ? launch_simt_t<CC, __nv_bfloat16, KK>(q, k, v, g, beta, s0, H, dk, dv, N, o, \
+                                                      sN, ws_ctrl, table, seq_first, s)         \
+               : launch_simt_t<CC, float, KK>(q, k, v, g, beta, s0, H, dk, dv, N, o, sN,       \
+                                              ws_ctrl, table, seq_first, s);
+  GDN_SIMT_CASE(16, false)
+  GDN_SIMT_CASE(32, false)
+  GDN_SIMT_CASE(64, false)
+  GDN_SIMT_CASE(16, true)
+  GDN_SIMT_CASE(32, true)
+  GDN_SIMT_CASE(64, true)
 #undef GDN_SIMT_CASE
   return cudaErrorInvalidValue;
 }

@@ -9,6 +9,13 @@
 //   st[j][i] <- alpha st[j][i] + u_i k_j
 //   o_i = alpha y_i + (k . q) u_i     (= S_t q, read after the write)
 //
+// Channel-wise gate (the Kimi Delta Attention variant: dmarx anthology
+// LIT-137, "Standing in the anthology"; SOTA-135, "Sequence"): alpha_j per d_k
+// channel j, S_t = S_{t-1} diag(alpha)(I - beta k k^T) + beta v k^T, so
+//   x_i = sum_j st[j][i] alpha_j k_j    y_i = sum_j st[j][i] alpha_j q_j
+//   u_i = beta (v_i - x_i)    st[j][i] <- alpha_j st[j][i] + u_i k_j
+//   o_i = y_i + (k . q) u_i
+//
 // One CTA per state (256 threads = 8 warps). Lane t owns columns 4t..4t+3
 // (one 16-byte vector per row, so a warp reads a 512-byte row contiguously),
 // warp w owns rows w, w+8, w+16, ... The whole 64 KB state sits in registers
@@ -42,13 +49,13 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
 }
 
-template <typename T>
+template <typename T, bool KDA>
 __global__ void __launch_bounds__(kDecThreads, 2)
     gdn_decode_kernel(const T *__restrict__ q, const T *__restrict__ k,
                       const T *__restrict__ v, const float *__restrict__ g,
                       const float *__restrict__ beta, float *__restrict__ state,
                       T *__restrict__ o, int dk, int dv) {
-  __shared__ float ks[128], qs[128], us[128];
+  __shared__ float ks[128], qs[128], us[128], as[128];
   __shared__ float xpart[kDecWarps][128], ypart[kDecWarps][128];
   __shared__ float kq_s;
 
@@ -71,6 +78,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   if (tid < dk) {
     ks[tid] = to_f32(k[size_t(unit) * dk + tid]);
     qs[tid] = to_f32(q[size_t(unit) * dk + tid]);
+    if (KDA) as[tid] = expf(g[size_t(unit) * dk + tid]);
   }
   __syncthreads();
   if (warp == 0) {  // k . q
@@ -85,7 +93,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
 #pragma unroll
   for (int r = 0; r < kMaxRowsPerWarp; ++r) {
     const int j = warp + r * kDecWarps;
-    const float kj = j < dk ? ks[j] : 0.f, qj = j < dk ? qs[j] : 0.f;
+    const float aj = KDA && j < dk ? as[j] : 1.f;
+    const float kj = j < dk ? aj * ks[j] : 0.f, qj = j < dk ? aj * qs[j] : 0.f;
     xp.x += S[r].x * kj; xp.y += S[r].y * kj; xp.z += S[r].z * kj; xp.w += S[r].w * kj;
     yp.x += S[r].x * qj; yp.y += S[r].y * qj; yp.z += S[r].z * qj; yp.w += S[r].w * qj;
   }
@@ -94,7 +103,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     *reinterpret_cast<float4 *>(&ypart[warp][col]) = yp;
   }
   __syncthreads();
-  const float alpha = expf(g[unit]);
+  // scalar gate: alpha multiplies x and y here; channel gate: already inside them
+  const float alpha = KDA ? 1.f : expf(g[unit]);
   const float b = beta[unit];
   if (tid < dv) {
     float x = 0.f, y = 0.f;
@@ -111,33 +121,43 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     for (int r = 0; r < kMaxRowsPerWarp; ++r) {
       const int j = warp + r * kDecWarps;
       if (j < dk) {
-        const float kj = ks[j];
+        const float kj = ks[j], aj = KDA ? as[j] : alpha;
         float4 n;
-        n.x = alpha * S[r].x + u4.x * kj;
-        n.y = alpha * S[r].y + u4.y * kj;
-        n.z = alpha * S[r].z + u4.z * kj;
-        n.w = alpha * S[r].w + u4.w * kj;
+        n.x = aj * S[r].x + u4.x * kj;
+        n.y = aj * S[r].y + u4.y * kj;
+        n.z = aj * S[r].z + u4.z * kj;
+        n.w = aj * S[r].w + u4.w * kj;
         __stcs(reinterpret_cast<float4 *>(st + size_t(j) * dv + col), n);
       }
     }
   }
 }
 
-}  // namespace
-
-cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *g,
-                          const float *beta, float *state, void *o, int N, int H, int dk, int dv,
-                          int dtype, cudaStream_t s) {
-  const unsigned units = unsigned(N) * unsigned(H);
+template <bool KDA>
+void launch_decode_t(const void *q, const void *k, const void *v, const float *g,
+                     const float *beta, float *state, void *o, unsigned units, int dk, int dv,
+                     int dtype, cudaStream_t s) {
   if (dtype == GDN_BF16)
-    gdn_decode_kernel<__nv_bfloat16><<<units, kDecThreads, 0, s>>>(
+    gdn_decode_kernel<__nv_bfloat16, KDA><<<units, kDecThreads, 0, s>>>(
         static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
         static_cast<const __nv_bfloat16 *>(v), g, beta, state,
         static_cast<__nv_bfloat16 *>(o), dk, dv);
   else
-    gdn_decode_kernel<float><<<units, kDecThreads, 0, s>>>(
+    gdn_decode_kernel<float, KDA><<<units, kDecThreads, 0, s>>>(
         static_cast<const float *>(q), static_cast<const float *>(k),
         static_cast<const float *>(v), g, beta, state, static_cast<float *>(o), dk, dv);
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *g,
+                          const float *beta, float *state, void *o, int N, int H, int dk, int dv,
+                          int dtype, cudaStream_t s, bool channel_gate) {
+  const unsigned units = unsigned(N) * unsigned(H);
+  if (channel_gate)
+    launch_decode_t<true>(q, k, v, g, beta, state, o, units, dk, dv, dtype, s);
+  else
+    launch_decode_t<false>(q, k, v, g, beta, state, o, units, dk, dv, dtype, s);
   return cudaGetLastError();
 }
 

@@ -49,14 +49,17 @@ int check_chunk_args(const void *q, const void *k, const void *v, const float *g
   return GDN_OK;
 }
 
-int run_chunk(bool force_simt, const void *q, const void *k, const void *v, const float *g,
-              const float *beta, const float *s0, const int32_t *cu, int B, int T, int H,
-              int dk, int dv, int num_seqs, int chunk, int dtype, void *o, float *sN, void *ws,
-              size_t ws_bytes, void *stream) {
+// force_simt: the CUDA-core kernel even where the tensor-core path applies.
+// channel_gate: g is [B, T, H, d_k] (one log-decay per d_k channel); the
+// CUDA-core kernel is the only path for it.
+int run_chunk(bool force_simt, bool channel_gate, const void *q, const void *k, const void *v,
+              const float *g, const float *beta, const float *s0, const int32_t *cu, int B,
+              int T, int H, int dk, int dv, int num_seqs, int chunk, int dtype, void *o,
+              float *sN, void *ws, size_t ws_bytes, void *stream) {
   int rc = check_chunk_args(q, k, v, g, beta, s0, cu, B, T, H, dk, dv, num_seqs, chunk, dtype,
                             o, sN, ws);
   if (rc != GDN_OK) return rc;
-  const bool tc = !force_simt && tc_path(dk, dv, chunk, dtype);
+  const bool tc = !force_simt && !channel_gate && tc_path(dk, dv, chunk, dtype);
   const int segs = scan_segments(B, T, H, cu ? num_seqs : 0, chunk, tc, device_sms());
   const WsLayout L = ws_layout(B, T, H, cu ? num_seqs : 0, chunk, tc, segs);
   if (ws_bytes < L.total) return GDN_ERR_WORKSPACE;
@@ -71,7 +74,7 @@ int run_chunk(bool force_simt, const void *q, const void *k, const void *v, cons
     prof_record(g_profile.prep, s);
     prof_record(g_profile.scan, s);
     e = launch_chunk_simt(q, k, v, g, beta, s0, cu, B, T, H, dk, dv, N, chunk, dtype, o, sN,
-                          static_cast<uint32_t *>(ws), s);
+                          static_cast<uint32_t *>(ws), s, channel_gate);
   }
   prof_record(g_profile.end, s);
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
@@ -109,8 +112,9 @@ int gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
                   int B, int T, int H, int d_k, int d_v, int num_seqs, int chunk, int dtype,
                   void *o, float *final_state, void *workspace, size_t workspace_bytes,
                   void *stream) {
-  return run_chunk(false, q, k, v, g, beta, initial_state, cu_seqlens, B, T, H, d_k, d_v,
-                   num_seqs, chunk, dtype, o, final_state, workspace, workspace_bytes, stream);
+  return run_chunk(false, false, q, k, v, g, beta, initial_state, cu_seqlens, B, T, H, d_k,
+                   d_v, num_seqs, chunk, dtype, o, final_state, workspace, workspace_bytes,
+                   stream);
 }
 
 int gdn_chunk_fwd_simt(const void *q, const void *k, const void *v, const float *g,
@@ -118,13 +122,32 @@ int gdn_chunk_fwd_simt(const void *q, const void *k, const void *v, const float 
                        int B, int T, int H, int d_k, int d_v, int num_seqs, int chunk, int dtype,
                        void *o, float *final_state, void *workspace, size_t workspace_bytes,
                        void *stream) {
-  return run_chunk(true, q, k, v, g, beta, initial_state, cu_seqlens, B, T, H, d_k, d_v,
+  return run_chunk(true, false, q, k, v, g, beta, initial_state, cu_seqlens, B, T, H, d_k,
+                   d_v, num_seqs, chunk, dtype, o, final_state, workspace, workspace_bytes,
+                   stream);
+}
+
+size_t gdn_kda_chunk_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int num_seqs,
+                                        int chunk, int dtype) {
+  (void)dtype;
+  if (B < 1 || T < 0 || H < 1 || d_k < 1 || d_v < 1 || num_seqs < 0) return 0;
+  if (chunk != 16 && chunk != 32 && chunk != 64) return 0;
+  return ws_layout(B, T, H, num_seqs, chunk, false).total;
+}
+
+int gdn_kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
+                      const float *beta, const float *initial_state, const int32_t *cu_seqlens,
+                      int B, int T, int H, int d_k, int d_v, int num_seqs, int chunk, int dtype,
+                      void *o, float *final_state, void *workspace, size_t workspace_bytes,
+                      void *stream) {
+  return run_chunk(true, true, q, k, v, g, beta, initial_state, cu_seqlens, B, T, H, d_k, d_v,
                    num_seqs, chunk, dtype, o, final_state, workspace, workspace_bytes, stream);
 }
 
-int gdn_decode_step(const void *q, const void *k, const void *v, const float *g,
-                    const float *beta, float *state, void *o, int N, int H, int d_k, int d_v,
-                    int dtype, void *stream) {
+namespace {
+int run_decode(bool channel_gate, const void *q, const void *k, const void *v, const float *g,
+               const float *beta, float *state, void *o, int N, int H, int d_k, int d_v,
+               int dtype, void *stream) {
   if (dtype != GDN_BF16 && dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
   if (N < 1 || H < 1 || d_k < 1 || d_v < 1) return GDN_ERR_INVALID_ARG;
   if (d_k > 128 || d_v > 128 || (d_v % 4) != 0) return GDN_ERR_UNSUPPORTED;
@@ -134,8 +157,21 @@ int gdn_decode_step(const void *q, const void *k, const void *v, const float *g,
       !aligned(state, 16) || !aligned(g, 4) || !aligned(beta, 4))
     return GDN_ERR_INVALID_ARG;
   cudaError_t e = launch_decode(q, k, v, g, beta, state, o, N, H, d_k, d_v, dtype,
-                                static_cast<cudaStream_t>(stream));
+                                static_cast<cudaStream_t>(stream), channel_gate);
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+}  // namespace
+
+int gdn_decode_step(const void *q, const void *k, const void *v, const float *g,
+                    const float *beta, float *state, void *o, int N, int H, int d_k, int d_v,
+                    int dtype, void *stream) {
+  return run_decode(false, q, k, v, g, beta, state, o, N, H, d_k, d_v, dtype, stream);
+}
+
+int gdn_kda_decode_step(const void *q, const void *k, const void *v, const float *g,
+                        const float *beta, float *state, void *o, int N, int H, int d_k,
+                        int d_v, int dtype, void *stream) {
+  return run_decode(true, q, k, v, g, beta, state, o, N, H, d_k, d_v, dtype, stream);
 }
 
 int gdn_get_status(void *workspace, void *stream) {

@@ -126,12 +126,13 @@ int device_sms();
 cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const float *g,
                               const float *beta, const float *s0, const int32_t *cu, int B,
                               int T, int H, int dk, int dv, int N, int chunk, int dtype, void *o,
-                              float *sN, uint32_t *err, cudaStream_t s);
+                              float *sN, uint32_t *err, cudaStream_t s, bool channel_gate);
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const float *g,
                             const float *beta, const float *s0, int B, int T, int H, int N,
                             void *o, float *sN, void *ws, const WsLayout &L, cudaStream_t s);
+// channel_gate: g is [N, H, d_k] (one log-decay per d_k channel), else [N, H].
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *g,
                           const float *beta, float *state, void *o, int N, int H, int dk, int dv,
-                          int dtype, cudaStream_t s);
+                          int dtype, cudaStream_t s, bool channel_gate);
 
 }  // namespace gdn

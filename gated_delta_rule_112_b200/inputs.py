@@ -14,12 +14,17 @@ library is measured on:
 * ``decode``     N=256 H=32 d=128 fp32 state, 64 consecutive single-token steps
 * ``b4h16t4096_beta2`` the b4h16t4096 shape with beta = 2 sigmoid(N(0, 1)) in
   (0, 2): the negative-eigenvalue range of I - beta k k^T, seed 5
+* ``kda_b4h16t4096`` the b4h16t4096 shape with the channel-wise gate (one
+  log-decay per d_k channel, g [B,T,H,d_k]), seed 6
+* ``kda_decode``  the decode shape with the channel-wise gate, seed 7
 
 Distributions (all drawn in fp32 with ``torch.Generator('cpu')``):
 q, k ~ N(0, 1) then L2-normalised per (token, head) over d_k; v ~ N(0, 1);
 beta = sigmoid(N(0, 1)); g = log(alpha) = -softplus(N(mu, 1)) with mu = -2
-(mu = -4 for the long-context workload); random states ~ N(0, 0.02) (std).
-Draw order: lengths (varlen only), q, k, v, beta-logits, g-normal, state.
+(mu = -4 for the long-context workload), drawn per token and head, or per
+token, head and d_k channel for the channel-wise gate; random states
+~ N(0, 0.02) (std). Draw order: lengths (varlen only), q, k, v, beta-logits,
+g-normal, state.
 """
 from __future__ import annotations
 
@@ -49,6 +54,7 @@ class Workload:
     len_range: tuple = field(default=(128, 2048))
     steps: int = 1             # decode workloads: consecutive steps
     beta_scale: float = 1.0    # beta = beta_scale * sigmoid(N(0, 1))
+    gate: str = "scalar"       # "scalar": g [..., H]; "channel": g [..., H, d_k]
 
 
 WORKLOADS = {
@@ -63,6 +69,10 @@ WORKLOADS = {
                        random_state=True, seed=4, steps=64),
     "b4h16t4096_beta2": Workload("b4h16t4096_beta2", B=4, T=4096, H=16, d_k=128, d_v=128,
                                  seed=5, beta_scale=2.0),
+    "kda_b4h16t4096": Workload("kda_b4h16t4096", B=4, T=4096, H=16, d_k=128, d_v=128,
+                               seed=6, gate="channel"),
+    "kda_decode": Workload("kda_decode", B=256, T=1, H=32, d_k=128, d_v=128,
+                           random_state=True, seed=7, steps=64, gate="channel"),
 }
 
 
@@ -79,11 +89,16 @@ def _unit_rows(x: torch.Tensor) -> torch.Tensor:
     return x / x.norm(dim=-1, keepdim=True).clamp_min(1e-12)
 
 
-def _gates(gen, shape, mu, beta_scale=1.0):
+def _gates(gen, shape, mu, beta_scale=1.0, g_shape=None):
     beta = beta_scale * torch.sigmoid(torch.randn(shape, generator=gen, dtype=torch.float32))
     g = -torch.nn.functional.softplus(
-        torch.randn(shape, generator=gen, dtype=torch.float32) + mu)
+        torch.randn(shape if g_shape is None else g_shape, generator=gen,
+                    dtype=torch.float32) + mu)
     return g.contiguous(), beta.contiguous()
+
+
+def _g_shape(w, shape):
+    return tuple(shape) + (w.d_k,) if w.gate == "channel" else None
 
 
 def make_chunk_inputs(w: Workload | str, *, seed: int | None = None, T: int | None = None,
@@ -93,7 +108,8 @@ def make_chunk_inputs(w: Workload | str, *, seed: int | None = None, T: int | No
     """Draw one batch for the chunked forward pass (CPU tensors).
 
     Returns a dict with q, k ``[B,T,H,d_k]``, v ``[B,T,H,d_v]`` in the workload
-    dtype, g and beta ``[B,T,H]`` fp32, ``initial_state`` ``[N,H,d_k,d_v]`` fp32
+    dtype, g and beta ``[B,T,H]`` fp32 (g ``[B,T,H,d_k]`` for the channel-wise
+    gate), ``initial_state`` ``[N,H,d_k,d_v]`` fp32
     or None, ``cu_seqlens`` int32 ``[N+1]`` or None, and the workload fields.
     Keyword overrides shrink a workload for tests (same distributions).
     """
@@ -120,14 +136,14 @@ def make_chunk_inputs(w: Workload | str, *, seed: int | None = None, T: int | No
     q = _unit_rows(torch.randn(Bn, Tn, H, w.d_k, generator=gen, dtype=torch.float32))
     k = _unit_rows(torch.randn(Bn, Tn, H, w.d_k, generator=gen, dtype=torch.float32))
     v = torch.randn(Bn, Tn, H, w.d_v, generator=gen, dtype=torch.float32)
-    g, beta = _gates(gen, (Bn, Tn, H), gate_mu, w.beta_scale)
+    g, beta = _gates(gen, (Bn, Tn, H), gate_mu, w.beta_scale, _g_shape(w, (Bn, Tn, H)))
     s0 = None
     if random_state:
         s0 = 0.02 * torch.randn(N, H, w.d_k, w.d_v, generator=gen, dtype=torch.float32)
     return dict(q=q.to(dtype).contiguous(), k=k.to(dtype).contiguous(),
                 v=v.to(dtype).contiguous(), g=g, beta=beta, initial_state=s0,
                 cu_seqlens=cu, chunk=w.chunk, B=Bn, T=Tn, H=H, d_k=w.d_k, d_v=w.d_v,
-                num_seqs=N, dtype=dtype)
+                num_seqs=N, dtype=dtype, gate=w.gate)
 
 
 def make_decode_inputs(w: Workload | str = "decode", *, seed: int | None = None,
@@ -136,7 +152,8 @@ def make_decode_inputs(w: Workload | str = "decode", *, seed: int | None = None,
     """Draw the initial state and ``steps`` single-token inputs (CPU tensors).
 
     Returns dict(state ``[N,H,d_k,d_v]`` fp32, q/k ``[steps,N,H,d_k]``,
-    v ``[steps,N,H,d_v]``, g/beta ``[steps,N,H]`` fp32). The state is drawn
+    v ``[steps,N,H,d_v]``, g/beta ``[steps,N,H]`` fp32, g ``[steps,N,H,d_k]``
+    for the channel-wise gate). The state is drawn
     first, then each step's q, k, v, beta-logits, g-normal in step order.
     """
     if isinstance(w, str):
@@ -153,7 +170,7 @@ def make_decode_inputs(w: Workload | str = "decode", *, seed: int | None = None,
         qs.append(_unit_rows(torch.randn(N, H, w.d_k, generator=gen, dtype=torch.float32)))
         ks.append(_unit_rows(torch.randn(N, H, w.d_k, generator=gen, dtype=torch.float32)))
         vs.append(torch.randn(N, H, w.d_v, generator=gen, dtype=torch.float32))
-        g, b = _gates(gen, (N, H), w.gate_mu)
+        g, b = _gates(gen, (N, H), w.gate_mu, 1.0, _g_shape(w, (N, H)))
         gs.append(g)
         bs.append(b)
     return dict(state=state.contiguous(),
@@ -161,4 +178,4 @@ def make_decode_inputs(w: Workload | str = "decode", *, seed: int | None = None,
                 k=torch.stack(ks).to(dtype).contiguous(),
                 v=torch.stack(vs).to(dtype).contiguous(),
                 g=torch.stack(gs).contiguous(), beta=torch.stack(bs).contiguous(),
-                N=N, H=H, d_k=w.d_k, d_v=w.d_v, steps=steps, dtype=dtype)
+                N=N, H=H, d_k=w.d_k, d_v=w.d_v, steps=steps, dtype=dtype, gate=w.gate)

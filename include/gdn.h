@@ -192,6 +192,56 @@ int gdn_decode_step(const void *q, const void *k, const void *v, const float *g,
                     int d_v, int dtype, void *stream);
 
 /*
+ * Channel-wise gate (the Kimi Delta Attention variant, named as the
+ * recurrence's successor on the dmarx anthology LIT-137 page, "Standing in the
+ * anthology", and on SOTA-135, "Sequence": the scalar decay becomes one decay
+ * per d_k channel). With alpha_t a d_k vector, diag(alpha_t) stands where the
+ * scalar stood:
+ *
+ *     S_t = S_{t-1} diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *     o_t = S_t q_t
+ *
+ * g = log alpha is then fp32 [B, T, H, d_k] (chunked) or [N, H, d_k] (decode),
+ * 4-byte aligned; everything else is as for the scalar gate. The pages give no
+ * equations for the variant; this reading is the plain substitution.
+ */
+
+/* Bytes of workspace gdn_kda_chunk_fwd needs (same rules as
+ * gdn_chunk_fwd_workspace_size); 0 for invalid sizes. */
+size_t gdn_kda_chunk_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int num_seqs,
+                                        int chunk, int dtype);
+
+/*
+ * gdn_kda_chunk_fwd -- the whole-sequence forward pass with the channel-wise
+ * gate, chunkwise. Per chunk, Gamma = cumsum(g) per channel and the decay
+ * moves inside the dot products:
+ *   A_rs = beta_r sum_j k_rj k_sj exp(Gamma_rj - Gamma_sj) (s < r); T = (I + A)^-1
+ *   W = T diag(beta) (K .* exp(Gamma)); U = T diag(beta) V; V_new = U - W S^T
+ *   P_rs = sum_j q_rj k_sj exp(Gamma_rj - Gamma_sj) (s <= r)
+ *   O = (Q .* exp(Gamma)) S^T + P V_new
+ *   S <- S diag(exp(Gamma_last)) + V_new^T (K .* exp(Gamma_last - Gamma))
+ * Runs on the fp32 CUDA-core kernel for every dtype. Arguments, layouts,
+ * ownership and errors as gdn_chunk_fwd, except g: [B, T, H, d_k] fp32.
+ * Supports d_k, d_v <= 128 and chunk 16, 32 or 64.
+ */
+int gdn_kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
+                      const float *beta, const float *initial_state, const int32_t *cu_seqlens,
+                      int B, int T, int H, int d_k, int d_v, int num_seqs, int chunk, int dtype,
+                      void *o, float *final_state, void *workspace, size_t workspace_bytes,
+                      void *stream);
+
+/*
+ * gdn_kda_decode_step -- one token with the channel-wise gate for N*H states,
+ * in place. Per (n, h), with a = exp(g) [d_k]:
+ *     x = S diag(a) k; y = S diag(a) q; u = beta (v - x)
+ *     S <- S diag(a) + u k^T;  o = S q = y + (k . q) u
+ * Arguments as gdn_decode_step, except g: [N, H, d_k] fp32.
+ */
+int gdn_kda_decode_step(const void *q, const void *k, const void *v, const float *g,
+                        const float *beta, float *state, void *o, int N, int H, int d_k,
+                        int d_v, int dtype, void *stream);
+
+/*
  * gdn_selftest_wait_timeout -- device self-test of the bounded waits (the
  * pages have no counterpart; it tests this library's failure handling).
  *

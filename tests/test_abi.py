@@ -68,13 +68,13 @@ def test_workspace_size(L):
     assert ws(1, 10, 1, 128, 128, 0, 48, gdn.BF16) == 0
 
 
-def _chunk_call(L, **kw):
+def _chunk_call(L, fn="gdn_chunk_fwd", **kw):
     a = dict(q=1 << 20, k=1 << 20, v=1 << 20, g=1 << 20, beta=1 << 20, s0=None, cu=None, B=1,
              T=64, H=1, dk=128, dv=128, ns=0, chunk=64, dtype=gdn.BF16, o=1 << 20, sN=None,
              ws=1 << 20, wsb=1 << 30, stream=None)
     a.update(kw)
     vp = ctypes.c_void_p
-    return L.gdn_chunk_fwd(vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["g"]), vp(a["beta"]),
+    return getattr(L, fn)(vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["g"]), vp(a["beta"]),
                            vp(a["s0"]), vp(a["cu"]), a["B"], a["T"], a["H"], a["dk"], a["dv"],
                            a["ns"], a["chunk"], a["dtype"], vp(a["o"]), vp(a["sN"]),
                            vp(a["ws"]), a["wsb"], vp(a["stream"]))
@@ -127,3 +127,25 @@ def test_scan_segments_rule(L):
     for sms in (1, 16, 148, 160):
         g = seg(1, 64 * 1000, 3, 128, 128, 0, 64, BF, sms)
         assert 1 <= g <= 16
+
+
+def test_kda_entry_points_host_checks(L):
+    kda = "gdn_kda_chunk_fwd"
+    assert _chunk_call(L, fn=kda, q=None) == gdn.ERR_INVALID_ARG
+    assert _chunk_call(L, fn=kda, g=(1 << 20) + 2) == gdn.ERR_INVALID_ARG   # misaligned gate
+    assert _chunk_call(L, fn=kda, dk=256) == gdn.ERR_UNSUPPORTED
+    assert _chunk_call(L, fn=kda, chunk=48) == gdn.ERR_UNSUPPORTED
+    assert _chunk_call(L, fn=kda, ws=None) == gdn.ERR_WORKSPACE
+    assert _chunk_call(L, fn=kda, wsb=100) == gdn.ERR_WORKSPACE
+    # the channel-wise gate runs on the CUDA-core kernel: its workspace is the
+    # chunk table alone, no per-(chunk, head) intermediates
+    kws = L.gdn_kda_chunk_fwd_workspace_size(4, 4096, 16, 128, 128, 0, 64, gdn.BF16)
+    assert kws == L.gdn_chunk_fwd_workspace_size(4, 4096, 16, 128, 128, 0, 64, gdn.F32)
+    assert 0 < kws < (1 << 20)
+    assert L.gdn_kda_chunk_fwd_workspace_size(1, 10, 1, 128, 128, 0, 48, gdn.BF16) == 0
+    vp = ctypes.c_void_p
+    p = vp(1 << 20)
+    assert L.gdn_kda_decode_step(p, p, p, p, p, None, p, 2, 2, 128, 128, gdn.BF16,
+                                 None) == gdn.ERR_INVALID_ARG
+    assert L.gdn_kda_decode_step(p, p, p, p, p, p, p, 2, 2, 128, 126, gdn.BF16,
+                                 None) == gdn.ERR_UNSUPPORTED
