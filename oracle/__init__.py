@@ -16,9 +16,11 @@ Two independent formulations live here:
 * ``kda_chunk_fwd`` / ``kda_decode_step`` and ``chunked.kda_chunk_fwd_dense``:
   the same two formulations for the channel-wise gate (the Kimi Delta
   Attention variant: g = log alpha has one value per d_k channel).
+* ``chunk_bwd``: the gradients of ``chunk_fwd`` by reverse-mode
+  differentiation of the token recurrence (C, fp64).
 
-Every function is pinned by ``tests/test_oracle_pins.py`` and
-``tests/test_oracle_kda_pins.py``.
+Every function is pinned by ``tests/test_oracle_pins.py``,
+``tests/test_oracle_kda_pins.py`` and ``tests/test_oracle_bwd_pins.py``.
 """
 from __future__ import annotations
 
@@ -62,6 +64,9 @@ def _load():
         lib.gdn_oracle_kda_chunk_fwd.restype = ci
         lib.gdn_oracle_kda_decode_step.argtypes = lib.gdn_oracle_decode_step.argtypes
         lib.gdn_oracle_kda_decode_step.restype = ci
+        lib.gdn_oracle_chunk_bwd.argtypes = [d, d, d, d, d, d, i32, ci, ci, ci, ci, ci, ci,
+                                             d, d, d, d, d, d, d, d, ci]
+        lib.gdn_oracle_chunk_bwd.restype = ci
         _lib = lib
     return _lib
 
@@ -122,6 +127,41 @@ def _run_chunk(fn, q, k, v, g, beta, initial_state, cu_seqlens, nthreads, channe
     if rc != 0:
         raise ValueError("oracle rejected the arguments")
     return o, fs
+
+
+def chunk_bwd(q, k, v, g, beta, d_o, initial_state=None, cu_seqlens=None,
+              d_final_state=None, nthreads=None):
+    """Gradients of ``chunk_fwd`` (scalar gate) for the loss
+    L = sum(d_o * o) + sum(d_final_state * final_state), by reverse-mode
+    differentiation of the token recurrence in fp64.
+
+    Returns a dict of float64 arrays: dq, dk [B,T,H,d_k], dv [B,T,H,d_v],
+    dg, dbeta [B,T,H], d_initial_state [N,H,d_k,d_v].
+    """
+    q, k, v, g, beta, d_o = (_f64(a) for a in (q, k, v, g, beta, d_o))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if g.shape != (B, T, H) or d_o.shape != (B, T, H, dv):
+        raise ValueError("g or d_o has the wrong shape")
+    cu = None
+    N = B
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+        N = cu.shape[0] - 1
+    s0 = None if initial_state is None else _f64(initial_state)
+    dsN = None if d_final_state is None else _f64(d_final_state)
+    out = dict(dq=np.zeros((B, T, H, dk)), dk=np.zeros((B, T, H, dk)),
+               dv=np.zeros((B, T, H, dv)), dg=np.zeros((B, T, H)), dbeta=np.zeros((B, T, H)),
+               d_initial_state=np.zeros((N, H, dk, dv)))
+    rc = _load().gdn_oracle_chunk_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(s0),
+        None if cu is None else cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+        B, T, H, dk, dv, N, _ptr(d_o), _ptr(dsN), _ptr(out["dq"]), _ptr(out["dk"]),
+        _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dbeta"]), _ptr(out["d_initial_state"]),
+        nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return out
 
 
 def decode_step(q, k, v, g, beta, state, nthreads=None):

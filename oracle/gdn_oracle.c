@@ -38,7 +38,23 @@
  * S_t = R + beta_t (v_t - R k_t) k_t^T and o_t = S_t q_t. The gate input is
  * g = log(alpha) of shape [B, T, H, d_k] (gdn_oracle_kda_*).
  *
- * Parity: pinned by tests/test_oracle_pins.py and tests/test_oracle_kda_pins.py
+ * Gradients (gdn_oracle_chunk_bwd). The pages call the chunkwise algorithm a
+ * training algorithm (phantomic12 page, mechanism paragraph) but give no
+ * gradients. For a loss with dL/do_t = do_t and dL/dS_final = dS_N they
+ * follow by reverse-mode differentiation of the scalar-gate recurrence above.
+ * With G = dL/dS_t (all later tokens' contributions already in),
+ * x = S_{t-1} k, u = beta (v - alpha x), going backwards over t:
+ *     G += do_t q_t^T                         (o_t = S_t q_t)
+ *     dq_t = S_t^T do_t
+ *     Gk = G k;   dv_t = beta Gk;   dbeta_t = Gk . (v - alpha x)
+ *     dalpha_t = <G, S_{t-1}> - beta (Gk . x);   dg_t = alpha dalpha_t
+ *     dk_t = G^T u - alpha beta S_{t-1}^T Gk
+ *     G <- alpha (G - beta Gk k^T)            (= dL/dS_{t-1})
+ * and dS_0 = G at the sequence start. S_{t-1} is recomputed forward from
+ * states kept every 64 tokens.
+ *
+ * Parity: pinned by tests/test_oracle_pins.py, tests/test_oracle_kda_pins.py
+ * and tests/test_oracle_bwd_pins.py
  * (closed forms, special cases, exact rational arithmetic, hand-worked
  * tokens, the dense chunked WY/UT forms).
  */
@@ -54,6 +70,9 @@ typedef struct {
     double *o, *s_out;
     int B, T, H, dk, dv, N;
     int channel_gate;      /* 0: g [B,T,H] scalar gate; 1: g [B,T,H,d_k] per channel */
+    /* backward only (o, s_out unused): upstream gradients and the outputs */
+    const double *d_o, *d_sN;
+    double *dq, *dk_, *dv_, *dg, *dbeta, *ds0;
     int next;              /* next (seq, head) unit to hand out */
     pthread_mutex_t lock;
 } job_t;
@@ -171,6 +190,123 @@ static void run_unit_kda(job_t *J, int n, int h)
     free(a);
 }
 
+/* One scalar-gate step in place: S <- alpha S + beta (v - alpha S k) k^T;
+ * x (d_v) receives S_{t-1} k. */
+static void step_forward(int dk, int dv, double *S, double *x, const double *kt,
+                         const double *vt, double alpha, double beta)
+{
+    for (int i = 0; i < dv; ++i) {
+        double acc = 0.0;
+        for (int j = 0; j < dk; ++j) acc += S[(size_t)i * dk + j] * kt[j];
+        x[i] = acc;
+    }
+    for (int i = 0; i < dv; ++i) {
+        const double ui = beta * (vt[i] - alpha * x[i]);
+        for (int j = 0; j < dk; ++j)
+            S[(size_t)i * dk + j] = alpha * S[(size_t)i * dk + j] + ui * kt[j];
+    }
+}
+
+#define BWD_CKPT 64   /* tokens between kept states in the backward pass */
+
+/* Gradients of one (sequence, head) recurrence (see the header). */
+static void run_unit_bwd(job_t *J, int n, int h)
+{
+    const int H = J->H, dk = J->dk, dv = J->dv;
+    const size_t SS = (size_t)dv * dk;
+    int b, t0, t1;
+    seq_span(J, n, &b, &t0, &t1);
+    const int L = t1 - t0;
+    const int nck = (L + BWD_CKPT - 1) / BWD_CKPT;
+
+    /* states at the start of every BWD_CKPT-token block */
+    double *ck = (double *)calloc((size_t)(nck > 0 ? nck : 1) * SS, sizeof(double));
+    double *S = (double *)calloc(SS, sizeof(double));
+    double *blk = (double *)malloc(sizeof(double) * BWD_CKPT * SS);  /* S_{t-1} of one block */
+    double *G = (double *)calloc(SS, sizeof(double));
+    double *x = (double *)malloc(sizeof(double) * dv);
+    double *u = (double *)malloc(sizeof(double) * dv);
+    double *Gk = (double *)malloc(sizeof(double) * dv);
+    load_state(J, n, h, S);
+    for (int c = 0; c < nck; ++c) {
+        memcpy(ck + (size_t)c * SS, S, sizeof(double) * SS);
+        const int ta = t0 + c * BWD_CKPT, tb = ta + BWD_CKPT < t1 ? ta + BWD_CKPT : t1;
+        for (int t = ta; t < tb; ++t) {
+            const size_t row = ((size_t)b * J->T + t) * H + h;
+            step_forward(dk, dv, S, x, J->k + row * dk, J->v + row * dv, exp(J->g[row]),
+                         J->beta[row]);
+        }
+    }
+    /* G = dL/dS_final, formula orientation */
+    if (J->d_sN) {
+        const double *st = J->d_sN + ((size_t)n * H + h) * SS;
+        for (int j = 0; j < dk; ++j)
+            for (int i = 0; i < dv; ++i) G[(size_t)i * dk + j] = st[(size_t)j * dv + i];
+    }
+    for (int c = nck - 1; c >= 0; --c) {
+        const int ta = t0 + c * BWD_CKPT, tb = ta + BWD_CKPT < t1 ? ta + BWD_CKPT : t1;
+        /* recompute S_{t-1} for every token of the block */
+        memcpy(S, ck + (size_t)c * SS, sizeof(double) * SS);
+        for (int t = ta; t < tb; ++t) {
+            const size_t row = ((size_t)b * J->T + t) * H + h;
+            memcpy(blk + (size_t)(t - ta) * SS, S, sizeof(double) * SS);
+            step_forward(dk, dv, S, x, J->k + row * dk, J->v + row * dv, exp(J->g[row]),
+                         J->beta[row]);
+        }
+        for (int t = tb - 1; t >= ta; --t) {
+            const size_t row = ((size_t)b * J->T + t) * H + h;
+            const double *kt = J->k + row * dk, *qt = J->q + row * dk, *vt = J->v + row * dv;
+            const double *dot = J->d_o + row * dv;
+            const double alpha = exp(J->g[row]), beta = J->beta[row];
+            const double *Sp = blk + (size_t)(t - ta) * SS;      /* S_{t-1} */
+            for (int i = 0; i < dv; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < dk; ++j) acc += Sp[(size_t)i * dk + j] * kt[j];
+                x[i] = acc;
+                u[i] = beta * (vt[i] - alpha * acc);
+            }
+            /* G += do_t q_t^T */
+            for (int i = 0; i < dv; ++i)
+                for (int j = 0; j < dk; ++j) G[(size_t)i * dk + j] += dot[i] * qt[j];
+            /* dq_t = S_t^T do_t with S_t = alpha S_{t-1} + u k^T */
+            for (int j = 0; j < dk; ++j) {
+                double acc = 0.0;
+                for (int i = 0; i < dv; ++i)
+                    acc += (alpha * Sp[(size_t)i * dk + j] + u[i] * kt[j]) * dot[i];
+                J->dq[row * dk + j] = acc;
+            }
+            double gx = 0.0, db = 0.0, gs = 0.0;
+            for (int i = 0; i < dv; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < dk; ++j) acc += G[(size_t)i * dk + j] * kt[j];
+                Gk[i] = acc;
+                J->dv_[row * dv + i] = beta * acc;
+                db += acc * (vt[i] - alpha * x[i]);
+                gx += acc * x[i];
+            }
+            for (size_t e = 0; e < SS; ++e) gs += G[e] * Sp[e];
+            J->dbeta[row] = db;
+            J->dg[row] = alpha * (gs - beta * gx);
+            for (int j = 0; j < dk; ++j) {
+                double acc = 0.0;
+                for (int i = 0; i < dv; ++i)
+                    acc += G[(size_t)i * dk + j] * u[i] - alpha * beta * Sp[(size_t)i * dk + j] * Gk[i];
+                J->dk_[row * dk + j] = acc;
+            }
+            /* G <- dL/dS_{t-1} */
+            for (int i = 0; i < dv; ++i)
+                for (int j = 0; j < dk; ++j)
+                    G[(size_t)i * dk + j] = alpha * (G[(size_t)i * dk + j] - beta * Gk[i] * kt[j]);
+        }
+    }
+    {
+        double *st = J->ds0 + ((size_t)n * H + h) * SS;
+        for (int j = 0; j < dk; ++j)
+            for (int i = 0; i < dv; ++i) st[(size_t)j * dv + i] = G[(size_t)i * dk + j];
+    }
+    free(ck); free(S); free(blk); free(G); free(x); free(u); free(Gk);
+}
+
 static void *worker(void *arg)
 {
     job_t *J = (job_t *)arg;
@@ -179,10 +315,24 @@ static void *worker(void *arg)
         int u = J->next++;
         pthread_mutex_unlock(&J->lock);
         if (u >= J->N * J->H) break;
-        if (J->channel_gate) run_unit_kda(J, u / J->H, u % J->H);
-        else                 run_unit(J, u / J->H, u % J->H);
+        if (J->d_o)               run_unit_bwd(J, u / J->H, u % J->H);
+        else if (J->channel_gate) run_unit_kda(J, u / J->H, u % J->H);
+        else                      run_unit(J, u / J->H, u % J->H);
     }
     return NULL;
+}
+
+static int run_jobs(job_t *J, int nthreads)
+{
+    pthread_mutex_init(&J->lock, NULL);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > J->N * J->H) nthreads = J->N * J->H;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * nthreads);
+    for (int i = 0; i < nthreads; ++i) pthread_create(&th[i], NULL, worker, J);
+    for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+    free(th);
+    pthread_mutex_destroy(&J->lock);
+    return 0;
 }
 
 static int run_all(const double *q, const double *k, const double *v,
@@ -201,16 +351,38 @@ static int run_all(const double *q, const double *k, const double *v,
         N = num_seqs;
     }
     job_t J = {q, k, v, g, beta, initial_state, cu_seqlens, o, final_state,
-               B, T, H, d_k, d_v, N, channel_gate, 0};
-    pthread_mutex_init(&J.lock, NULL);
-    if (nthreads < 1) nthreads = 1;
-    if (nthreads > N * H) nthreads = N * H;
-    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * nthreads);
-    for (int i = 0; i < nthreads; ++i) pthread_create(&th[i], NULL, worker, &J);
-    for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
-    free(th);
-    pthread_mutex_destroy(&J.lock);
-    return 0;
+               B, T, H, d_k, d_v, N, channel_gate, NULL, NULL,
+               NULL, NULL, NULL, NULL, NULL, NULL, 0};
+    return run_jobs(&J, nthreads);
+}
+
+/* Gradients of gdn_oracle_chunk_fwd (scalar gate) for the loss
+ * L = sum(d_o * o) + sum(d_final_state * final_state). d_o [B,T,H,d_v];
+ * d_final_state [N,H,d_k,d_v] or NULL (zero). Outputs: dq, dk [B,T,H,d_k],
+ * dv [B,T,H,d_v], dg, dbeta [B,T,H], d_initial_state [N,H,d_k,d_v] (all
+ * required). Returns 0, or -1 on bad arguments. */
+int gdn_oracle_chunk_bwd(const double *q, const double *k, const double *v,
+                         const double *g, const double *beta,
+                         const double *initial_state, const int32_t *cu_seqlens,
+                         int B, int T, int H, int d_k, int d_v, int num_seqs,
+                         const double *d_o, const double *d_final_state,
+                         double *dq, double *dk, double *dv, double *dg, double *dbeta,
+                         double *d_initial_state, int nthreads)
+{
+    if (!q || !k || !v || !g || !beta || !d_o) return -1;
+    if (!dq || !dk || !dv || !dg || !dbeta || !d_initial_state) return -1;
+    if (B < 1 || T < 0 || H < 1 || d_k < 1 || d_v < 1) return -1;
+    int N = B;
+    if (cu_seqlens) {
+        if (B != 1 || num_seqs < 1 || cu_seqlens[0] != 0 || cu_seqlens[num_seqs] != T) return -1;
+        for (int n = 0; n < num_seqs; ++n)
+            if (cu_seqlens[n + 1] < cu_seqlens[n]) return -1;
+        N = num_seqs;
+    }
+    job_t J = {q, k, v, g, beta, initial_state, cu_seqlens, NULL, NULL,
+               B, T, H, d_k, d_v, N, 0, d_o, d_final_state,
+               dq, dk, dv, dg, dbeta, d_initial_state, 0};
+    return run_jobs(&J, nthreads);
 }
 
 /* Returns 0 on success, -1 on bad arguments. `o` must hold B*T*H*d_v values;

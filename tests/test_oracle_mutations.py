@@ -12,13 +12,15 @@ import subprocess
 import pytest
 
 import oracle
+import tests.test_oracle_bwd_pins as bwd_pins
 import tests.test_oracle_kda_pins as kda_pins
 import tests.test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "gdn_oracle.c")
 
 MUTATIONS = {
-    "residual_without_alpha": ("(vt[i] - alpha * x[i])", "(vt[i] - x[i])"),
+    "residual_without_alpha": ("const double u = beta * (vt[i] - alpha * x[i]);",
+                               "const double u = beta * (vt[i] - x[i]);"),
     "write_without_beta": ("const double u = beta * (", "const double u = ("),
     "state_not_transposed": ("S[(size_t)i * dk + j] = st[(size_t)j * dv + i];",
                              "S[(size_t)i * dk + j] = st[(size_t)i * dk + j];"),
@@ -55,6 +57,29 @@ KDA_PIN_CASES = [
     lambda: kda_pins.test_kda_dense_chunked_matches_token_loop(4, 7),
 ]
 
+# Mistakes in the gradient loop, caught by the gradient pins.
+BWD_MUTATIONS = {
+    "bwd_dk_without_state_term": (
+        "acc += G[(size_t)i * dk + j] * u[i] - alpha * beta * Sp[(size_t)i * dk + j] * Gk[i];",
+        "acc += G[(size_t)i * dk + j] * u[i];"),
+    "bwd_carry_without_beta": (
+        "G[(size_t)i * dk + j] = alpha * (G[(size_t)i * dk + j] - beta * Gk[i] * kt[j]);",
+        "G[(size_t)i * dk + j] = alpha * (G[(size_t)i * dk + j] - Gk[i] * kt[j]);"),
+    "bwd_dg_without_alpha": ("J->dg[row] = alpha * (gs - beta * gx);",
+                             "J->dg[row] = gs - beta * gx;"),
+    "bwd_dq_from_previous_state": (
+        "acc += (alpha * Sp[(size_t)i * dk + j] + u[i] * kt[j]) * dot[i];",
+        "acc += Sp[(size_t)i * dk + j] * dot[i];"),
+    "bwd_output_grad_not_added": ("for (int j = 0; j < dk; ++j) G[(size_t)i * dk + j] += dot[i] * qt[j];",
+                                  "for (int j = 0; j < dk; ++j) G[(size_t)i * dk + j] += 0.0 * qt[j];"),
+}
+
+BWD_PIN_CASES = [
+    lambda: bwd_pins.test_bwd_matches_central_differences("plain"),
+    bwd_pins.test_bwd_homogeneity_identities,
+    bwd_pins.test_bwd_beta_zero_closed_form,
+]
+
 PIN_CASES = [
     pins.test_hand_worked_two_tokens,
     pins.test_beta_zero_is_pure_decay,
@@ -66,10 +91,14 @@ PIN_CASES = [
 ]
 
 
-@pytest.mark.parametrize("name", sorted(MUTATIONS) + sorted(KDA_MUTATIONS))
+ALL = {**{n: (m, PIN_CASES) for n, m in MUTATIONS.items()},
+       **{n: (m, KDA_PIN_CASES) for n, m in KDA_MUTATIONS.items()},
+       **{n: (m, BWD_PIN_CASES) for n, m in BWD_MUTATIONS.items()}}
+
+
+@pytest.mark.parametrize("name", sorted(ALL))
 def test_planted_mistake_is_caught(name, tmp_path, monkeypatch):
-    before, after = MUTATIONS[name] if name in MUTATIONS else KDA_MUTATIONS[name]
-    cases = PIN_CASES if name in MUTATIONS else KDA_PIN_CASES
+    (before, after), cases = ALL[name]
     src = open(SRC).read()
     assert src.count(before) == 1, f"mutation anchor for {name} not unique"
     mutated = tmp_path / "mut.c"
@@ -80,7 +109,7 @@ def test_planted_mistake_is_caught(name, tmp_path, monkeypatch):
     real = oracle._load()
     lib = ctypes.CDLL(str(so))
     for fn in ("gdn_oracle_chunk_fwd", "gdn_oracle_decode_step", "gdn_oracle_kda_chunk_fwd",
-               "gdn_oracle_kda_decode_step"):
+               "gdn_oracle_kda_decode_step", "gdn_oracle_chunk_bwd"):
         getattr(lib, fn).argtypes = getattr(real, fn).argtypes
         getattr(lib, fn).restype = getattr(real, fn).restype
     monkeypatch.setattr(oracle, "_lib", lib)
