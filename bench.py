@@ -54,6 +54,8 @@ def parse_args():
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--bwd", action="store_true",
+                   help="also time the backward pass (gdn_chunk_bwd) on the workload")
     p.add_argument("--workload", default=WORKLOAD,
                    help="chunked-forward workload (inputs.WORKLOADS); the default is the "
                         "headline configuration, the others are for extra measurements")
@@ -66,6 +68,7 @@ KERNEL_SOURCES = {
     "kda_chunk_fwd_step": ["chunk_map.cu", "chunk_simt.cu", "gdn_internal.cuh",
                            "sm100_ptx.cuh"],
     "decode": ["decode.cu", "gdn_internal.cuh", "sm100_ptx.cuh"],
+    "bwd_step": ["backward.cu", "bwd_internal.cuh", "gdn_internal.cuh", "sm100_ptx.cuh"],
 }
 
 
@@ -367,6 +370,59 @@ def main():
                        else "gated_delta_rule_112_b200.chunk_fwd (C ABI gdn_chunk_fwd)")}
         del hq, hk, hv, hg, hb, ho, hfs
 
+    # --------------------------------------------------------------- backward pass
+    backward = None
+    if args.bwd and not kda:
+        del ws
+        torch.cuda.empty_cache()
+        gen = torch.Generator("cpu").manual_seed(1000 + rank)
+        d_o = torch.randn(B, T, H, 128, generator=gen).to(torch.bfloat16).to(dev)
+        dsN = (0.1 * torch.randn(nseq, H, 128, 128, generator=gen)).to(dev)
+        bws = torch.empty(gdn.bwd_workspace_size(B, T, H, 128, 128, 0 if cu is None else nseq),
+                          dtype=torch.uint8, device=dev)
+
+        def bstep():
+            return gdn.chunk_bwd(q, k, v, g, beta, d_o, s0, cu, dsN, workspace=bws)
+
+        for _ in range(3):
+            bstep()
+        torch.cuda.synchronize()
+        assert gdn.get_status(bws) == gdn.OK
+        kb = max(1, min(K, 5))
+        bev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(kb)]
+        barrier()
+        torch.cuda.synchronize()
+        for i in range(kb):
+            flush.fill_(i & 0xFF)
+            bev[i][0].record(stream)
+            bstep()
+            bev[i][1].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms_b = max_over_ranks(sum(a.elapsed_time(b) for a, b in bev) / kb)
+        # the operation's own bytes: q, k, v, d_o bf16 and g, beta in; dq, dk, dv fp32 and
+        # dg, dbeta out; the final-state gradient in and the initial-state gradient out
+        bw_bytes = tokens * H * (4 * 128 * 2 + 2 * 4 + 3 * 128 * 4 + 2 * 4) + \
+            (2 + (1 if s0 is not None else 0)) * nseq * H * 128 * 128 * 4
+        # every token's S_{t-1} written by the replay and read back by the reverse sweep
+        scratch = 2 * tokens * H * 128 * 128 * 4
+        gbs_b = bw_bytes / (ms_b * 1e-3) / 1e9
+        backward = {"workload": wl, "ms_per_step": ms_b, "steps": kb, "warmup": 3,
+                    "value": replicas.job_rate(tokens, ms_b, world) / 1e6, "unit": UNIT,
+                    "gpu_launches": 2 * kb,
+                    "api": "gated_delta_rule_112_b200.chunk_bwd (C ABI gdn_chunk_bwd)",
+                    "roofline": {"bound": "hbm", "achieved": gbs_b, "peak": pk["hbm"],
+                                 "unit": "GB/s", "frac": gbs_b / pk["hbm"],
+                                 "algorithmic_bytes": bw_bytes,
+                                 "scratch_bytes": scratch,
+                                 "traffic": recorded_traffic("bwd_step/" + wl),
+                                 "scratch_frac": scratch / (ms_b * 1e-3) / 1e9 / pk["hbm"],
+                                 "kernel": "gdn_bwd_replay_kernel + gdn_bwd_kernel",
+                                 "peak_source": pk["source"]}}
+        del d_o, dsN, bws
+        ws = None
+
     del q, k, v, g, beta, o, ws
     torch.cuda.empty_cache()
 
@@ -460,6 +516,7 @@ def main():
         "clocks": clocks,
         "e2e": e2e,
         "decode": decode,
+        "backward": backward,
         "cpu_baseline": cpu,
     }
     if rank == 0:

@@ -1,0 +1,28 @@
+// Internal declarations of the backward pass (host ABI layer and kernels).
+#pragma once
+#include "gdn_internal.cuh"
+
+namespace gdn {
+
+// Workspace of the backward pass: the 256 B control block, then S_{t-1}
+// before every token (fp32 [B*T][H][d_k][d_v], the S^T storage) and
+// x_t = S_{t-1} k_t (fp32 [B*T][H][d_v]).
+struct BwdLayout {
+  size_t s_prev, x, total;
+};
+inline BwdLayout bwd_layout(int B, int T, int H, int dk, int dv) {
+  BwdLayout L{};
+  const size_t rows = size_t(B) * size_t(T) * size_t(H);
+  L.s_prev = 256;
+  L.x = align_up(L.s_prev + rows * size_t(dk) * dv * sizeof(float), 256);
+  L.total = align_up(L.x + rows * size_t(dv) * sizeof(float), 256);
+  return L;
+}
+
+cudaError_t launch_bwd(const void *q, const void *k, const void *v, const float *g,
+                       const float *beta, const float *s0, const int32_t *cu, const void *d_o,
+                       const float *d_sN, int N, int B, int T, int H, int dk, int dv, int dtype,
+                       float *dq, float *dkk, float *dvv, float *dg, float *dbeta, float *ds0,
+                       void *ws, const BwdLayout &L, cudaStream_t s);
+
+}  // namespace gdn

@@ -3,6 +3,7 @@
 // here allocates device memory.
 #include <cstdio>
 
+#include "bwd_internal.cuh"
 #include "gdn_internal.cuh"
 
 using namespace gdn;
@@ -172,6 +173,42 @@ int gdn_kda_decode_step(const void *q, const void *k, const void *v, const float
                         const float *beta, float *state, void *o, int N, int H, int d_k,
                         int d_v, int dtype, void *stream) {
   return run_decode(true, q, k, v, g, beta, state, o, N, H, d_k, d_v, dtype, stream);
+}
+
+size_t gdn_chunk_bwd_workspace_size(int B, int T, int H, int d_k, int d_v, int num_seqs) {
+  if (B < 1 || T < 0 || H < 1 || d_k < 1 || d_v < 1 || num_seqs < 0) return 0;
+  return bwd_layout(B, T, H, d_k, d_v).total;
+}
+
+int gdn_chunk_bwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                  const float *initial_state, const int32_t *cu_seqlens, const void *d_o,
+                  const float *d_final_state, int B, int T, int H, int d_k, int d_v,
+                  int num_seqs, int dtype, float *dq, float *dk, float *dv, float *dg,
+                  float *dbeta, float *d_initial_state, void *workspace,
+                  size_t workspace_bytes, void *stream) {
+  if (dtype != GDN_BF16 && dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
+  if (B < 1 || T < 0 || H < 1 || d_k < 1 || d_v < 1) return GDN_ERR_INVALID_ARG;
+  if (cu_seqlens && (B != 1 || num_seqs < 1)) return GDN_ERR_INVALID_ARG;
+  if (!cu_seqlens && num_seqs != 0) return GDN_ERR_INVALID_ARG;
+  if (d_k > 128 || d_v > 128 || (d_v % 4) != 0) return GDN_ERR_UNSUPPORTED;
+  if (int64_t(B) * T * H * (d_k > d_v ? d_k : d_v) >= (int64_t(1) << 31)) return GDN_ERR_UNSUPPORTED;
+  if (!d_initial_state) return GDN_ERR_INVALID_ARG;
+  if (T > 0 && (!q || !k || !v || !g || !beta || !d_o || !dq || !dk || !dv || !dg || !dbeta))
+    return GDN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(d_o, 16) ||
+      !aligned(g, 4) || !aligned(beta, 4) || !aligned(initial_state, 16) ||
+      !aligned(d_final_state, 16) || !aligned(d_initial_state, 16) || !aligned(dq, 4) ||
+      !aligned(dk, 4) || !aligned(dv, 4) || !aligned(dg, 4) || !aligned(dbeta, 4) ||
+      !aligned(cu_seqlens, 4))
+    return GDN_ERR_INVALID_ARG;
+  if (!workspace || !aligned(workspace, 256)) return GDN_ERR_WORKSPACE;
+  const BwdLayout L = bwd_layout(B, T, H, d_k, d_v);
+  if (workspace_bytes < L.total) return GDN_ERR_WORKSPACE;
+  const int N = cu_seqlens ? num_seqs : B;
+  cudaError_t e = launch_bwd(q, k, v, g, beta, initial_state, cu_seqlens, d_o, d_final_state, N,
+                             B, T, H, d_k, d_v, dtype, dq, dk, dv, dg, dbeta, d_initial_state,
+                             workspace, L, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 int gdn_get_status(void *workspace, void *stream) {

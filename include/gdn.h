@@ -242,6 +242,52 @@ int gdn_kda_decode_step(const void *q, const void *k, const void *v, const float
                         int d_v, int dtype, void *stream);
 
 /*
+ * Backward pass (gradients of gdn_chunk_fwd, scalar gate). The pages call the
+ * chunkwise algorithm a training algorithm (phantomic12 page, mechanism
+ * paragraph) but give no gradients; they follow by reverse-mode
+ * differentiation of the recurrence. For the loss
+ *     L = sum(d_o * o) + sum(d_final_state * final_state)
+ * with G = dL/dS_t, x_t = S_{t-1} k_t, u_t = beta_t (v_t - alpha_t x_t), going
+ * backwards over t:
+ *     G += d_o_t q_t^T;  dq_t = S_t^T d_o_t
+ *     Gk = G k_t;  dv_t = beta_t Gk;  dbeta_t = Gk . (v_t - alpha_t x_t)
+ *     dg_t = alpha_t (<G, S_{t-1}> - beta_t Gk . x_t)
+ *     dk_t = G^T u_t - alpha_t beta_t S_{t-1}^T Gk
+ *     G <- alpha_t (G - beta_t Gk k_t^T)
+ * and d_initial_state = G at each sequence's start.
+ */
+
+/* Bytes of workspace gdn_chunk_bwd needs: 256 + B*T*H*(d_k*d_v + d_v)*4
+ * (every token's S_{t-1} and S_{t-1} k_t, fp32), rounded up; 0 for invalid sizes. */
+size_t gdn_chunk_bwd_workspace_size(int B, int T, int H, int d_k, int d_v, int num_seqs);
+
+/*
+ * gdn_chunk_bwd -- gradients of the forward pass for the loss above.
+ *
+ *   q, k, v, g, beta, initial_state, cu_seqlens, B, T, H, d_k, d_v, num_seqs,
+ *   dtype              as for gdn_chunk_fwd (the forward inputs).
+ *   d_o                [B, T, H, d_v] (dtype), 16-byte aligned: dL/do.
+ *   d_final_state      [N, H, d_k, d_v] fp32 (S^T storage) or NULL (zero).
+ *   dq, dk             [B, T, H, d_k] fp32 outputs.
+ *   dv                 [B, T, H, d_v] fp32 output.
+ *   dg, dbeta          [B, T, H] fp32 outputs (dg = dL/d(log alpha)).
+ *   d_initial_state    [N, H, d_k, d_v] fp32 output (also when
+ *                      initial_state is NULL: the gradient at a zero state).
+ *   workspace          >= gdn_chunk_bwd_workspace_size() bytes, 256-byte
+ *                      aligned, not shared with a concurrent call.
+ * Supports d_k <= 128 and d_v <= 128 with d_v a multiple of 4. Runs two
+ * kernels: a forward replay that stores every S_{t-1}, then the reverse
+ * sweep. Bad cu_seqlens contents are reported by gdn_get_status
+ * (GDN_ERR_INVALID_ARG); the affected sequences are not computed.
+ */
+int gdn_chunk_bwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                  const float *initial_state, const int32_t *cu_seqlens, const void *d_o,
+                  const float *d_final_state, int B, int T, int H, int d_k, int d_v,
+                  int num_seqs, int dtype, float *dq, float *dk, float *dv, float *dg,
+                  float *dbeta, float *d_initial_state, void *workspace,
+                  size_t workspace_bytes, void *stream);
+
+/*
  * gdn_selftest_wait_timeout -- device self-test of the bounded waits (the
  * pages have no counterpart; it tests this library's failure handling).
  *

@@ -149,3 +149,29 @@ def test_kda_entry_points_host_checks(L):
                                  None) == gdn.ERR_INVALID_ARG
     assert L.gdn_kda_decode_step(p, p, p, p, p, p, p, 2, 2, 128, 126, gdn.BF16,
                                  None) == gdn.ERR_UNSUPPORTED
+
+
+def test_bwd_host_checks(L):
+    vp = ctypes.c_void_p
+    p = vp(1 << 20)
+
+    def call(**kw):
+        a = dict(B=1, T=64, H=1, dk=128, dv=128, ns=0, dtype=gdn.BF16, q=p, ds0=p, ws=p,
+                 wsb=1 << 40, cu=None)
+        a.update(kw)
+        return L.gdn_chunk_bwd(a["q"], p, p, p, p, None, a["cu"], p, None, a["B"], a["T"],
+                               a["H"], a["dk"], a["dv"], a["ns"], a["dtype"], p, p, p, p, p,
+                               a["ds0"], a["ws"], a["wsb"], None)
+    assert call(q=None) == gdn.ERR_INVALID_ARG
+    assert call(ds0=None) == gdn.ERR_INVALID_ARG
+    assert call(dtype=9) == gdn.ERR_INVALID_ARG
+    assert call(dv=126) == gdn.ERR_UNSUPPORTED
+    assert call(dk=256) == gdn.ERR_UNSUPPORTED
+    assert call(ns=2) == gdn.ERR_INVALID_ARG                  # num_seqs without cu_seqlens
+    assert call(ws=None) == gdn.ERR_WORKSPACE
+    assert call(wsb=1000) == gdn.ERR_WORKSPACE
+    # every token's S_{t-1} and S_{t-1} k_t in fp32, plus the control block
+    need = L.gdn_chunk_bwd_workspace_size(4, 4096, 16, 128, 128, 0)
+    assert need >= 4 * 4096 * 16 * (128 * 128 + 128) * 4
+    assert need < 4 * 4096 * 16 * (128 * 128 + 128) * 4 + 4096
+    assert L.gdn_chunk_bwd_workspace_size(0, 1, 1, 128, 128, 0) == 0

@@ -1,0 +1,110 @@
+"""GPU parity of gdn_chunk_bwd (the gradients of the forward pass) against the
+fp64 oracle ``oracle.chunk_bwd`` on the same seeded inputs, through the C ABI.
+
+The CUDA backward computes in fp32 from the given inputs (bf16 inputs are
+upcast exactly, as the oracle sees them); a CPU emulation of its arithmetic in
+fp32 stays within 3e-7 of the fp64 gradients, so the fp32 tolerance applies to
+both input types."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_delta_rule_112_b200.inputs import Workload, make_chunk_inputs
+from tests.parity import TOL_F32, assert_close, np64, to_dev
+
+pytestmark = pytest.mark.gpu
+
+SMALL = Workload("bwd_small", B=2, T=64, H=2, d_k=128, d_v=128, seed=31, dtype=torch.float32)
+KEYS = ("dq", "dk", "dv", "dg", "dbeta", "d_initial_state")
+
+
+def upstream(inp, seed=0, with_dsN=True):
+    gen = torch.Generator("cpu").manual_seed(seed)
+    B, T, H, dv = inp["B"], inp["T"], inp["H"], inp["d_v"]
+    d_o = torch.randn(B, T, H, dv, generator=gen).to(inp["dtype"])
+    N = inp["num_seqs"]
+    dsN = 0.1 * torch.randn(N, H, inp["d_k"], dv, generator=gen) if with_dsN else None
+    return d_o, dsN
+
+
+def check(inp, d_o, dsN, tol=TOL_F32, heads=None):
+    import gated_delta_rule_112_b200 as gdn
+    d = to_dev(inp)
+    got = gdn.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d_o.cuda(),
+                        d["initial_state"], d["cu_seqlens"],
+                        None if dsN is None else dsN.cuda())
+    torch.cuda.synchronize()
+    assert gdn.get_status() == gdn.OK
+    sl = slice(None) if heads is None else heads
+    s0, cu = inp["initial_state"], inp["cu_seqlens"]
+    ref = oracle.chunk_bwd(np64(inp["q"][:, :, sl]), np64(inp["k"][:, :, sl]),
+                           np64(inp["v"][:, :, sl]), np64(inp["g"][:, :, sl]),
+                           np64(inp["beta"][:, :, sl]), np64(d_o[:, :, sl]),
+                           None if s0 is None else np64(s0[:, sl]),
+                           None if cu is None else cu.numpy(),
+                           None if dsN is None else np64(dsN[:, sl]))
+    for key in KEYS:
+        g = got[key]
+        g = g[:, sl] if key == "d_initial_state" else g[:, :, sl]
+        assert_close(key, np64(g), ref[key], tol)
+    return got
+
+
+@pytest.mark.parametrize("T", [1, 7, 130])
+@pytest.mark.parametrize("with_state", [False, True])
+def test_bwd_fp32_lengths(T, with_state):
+    inp = make_chunk_inputs(SMALL, T=T, random_state=with_state)
+    d_o, dsN = upstream(inp, seed=T, with_dsN=with_state)
+    check(inp, d_o, dsN)
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 32), (96, 128), (128, 64)])
+def test_bwd_fp32_head_sizes(dk, dv):
+    w = Workload("bwd_sizes", B=2, T=90, H=2, d_k=dk, d_v=dv, seed=32, dtype=torch.float32,
+                 random_state=True)
+    inp = make_chunk_inputs(w)
+    d_o, dsN = upstream(inp, seed=1)
+    check(inp, d_o, dsN)
+
+
+def test_bwd_bf16_varlen_with_empty_sequences():
+    inp = make_chunk_inputs(SMALL, lengths=[50, 0, 131, 1], random_state=True,
+                            dtype=torch.bfloat16)
+    d_o, dsN = upstream(inp, seed=2)
+    got = check(inp, d_o, dsN)
+    # an empty sequence passes the final-state gradient straight through
+    np.testing.assert_array_equal(np64(got["d_initial_state"][1]), np64(dsN[1]))
+
+
+def test_bwd_zero_tokens():
+    import gated_delta_rule_112_b200 as gdn
+    inp = make_chunk_inputs(SMALL, T=0, random_state=True)
+    d_o, dsN = upstream(inp, seed=3)
+    d = to_dev(inp)
+    got = gdn.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d_o.cuda(),
+                        d["initial_state"], None, dsN.cuda())
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(np64(got["d_initial_state"]), np64(dsN))
+
+
+def test_bwd_bad_cu_seqlens_reported():
+    import gated_delta_rule_112_b200 as gdn
+    inp = make_chunk_inputs(SMALL, lengths=[5, 5, 5], random_state=True)
+    d_o, dsN = upstream(inp, seed=4)
+    d = to_dev(inp)
+    bad = torch.tensor([0, 9, 4, 15], dtype=torch.int32, device="cuda")   # decreasing
+    ws = torch.empty(gdn.bwd_workspace_size(1, 15, 2, 128, 128, 3), dtype=torch.uint8,
+                     device="cuda")
+    gdn.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d_o.cuda(), d["initial_state"],
+                  bad, dsN.cuda(), workspace=ws)
+    assert gdn.get_status(ws) == gdn.ERR_INVALID_ARG
+    assert gdn.get_status(ws) == gdn.OK          # the word is cleared
+
+
+def test_bwd_full_size_workload_sampled_heads():
+    """The b4h16t4096 workload (bf16, B=4, T=4096, H=16, d=128) in one call;
+    the oracle differentiates two heads of every sequence."""
+    inp = make_chunk_inputs("b4h16t4096")
+    d_o, dsN = upstream(inp, seed=5)
+    check(inp, d_o, dsN, heads=[2, 9])
