@@ -50,6 +50,37 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
+// Sums v[r] over the 32 lanes for 16 rows at once: at each butterfly step a
+// lane keeps half of its rows and adds the partner's copy of them, so after
+// 8 + 4 + 2 + 1 exchanges and a last one with lane ^ 1, lane L holds the sum
+// for row L >> 1 (16 shuffles instead of 16 separate five-shuffle sums).
+__device__ __forceinline__ float warp_rows16_sum(float (&v)[16], int lane) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const bool hi = lane & 16;
+    const float keep = hi ? v[i + 8] : v[i], send = hi ? v[i] : v[i + 8];
+    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const bool hi = lane & 8;
+    const float keep = hi ? v[i + 4] : v[i], send = hi ? v[i] : v[i + 4];
+    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const bool hi = lane & 4;
+    const float keep = hi ? v[i + 2] : v[i], send = hi ? v[i] : v[i + 2];
+    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+  }
+  {
+    const bool hi = lane & 2;
+    const float keep = hi ? v[1] : v[0], send = hi ? v[0] : v[1];
+    v[0] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+  }
+  return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
+}
+
 __device__ __forceinline__ float dot4(float4 a, float4 b) {
   return a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w;
 }
@@ -234,6 +265,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) gdn_bwd_kernel(
     const float udo = warp_sum(dot4(u4, do4));                 // u . do (a warp spans all columns)
     float4 gk = make_float4(0.f, 0.f, 0.f, 0.f);
     float gs = 0.f;
+    float part[kRows];
 #pragma unroll
     for (int r = 0; r < kRows; ++r) {
       const int j = warp + r * kBwdWarps;
@@ -242,9 +274,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) gdn_bwd_kernel(
       G[r].x += do4.x * qj; G[r].y += do4.y * qj; G[r].z += do4.z * qj; G[r].w += do4.w * qj;
       gk.x += G[r].x * kj; gk.y += G[r].y * kj; gk.z += G[r].z * kj; gk.w += G[r].w * kj;
       gs += dot4(G[r], S[r]);
-      // dq_j = alpha (S_{t-1}^T do)_j + k_j (u . do)
-      const float sdo = warp_sum(dot4(S[r], do4));
-      if (lane == r && j < dk) dq[row * dk + j] = alpha * sdo + kj * udo;
+      part[r] = dot4(S[r], do4);                               // (S_{t-1}^T do)_j, this lane's columns
+    }
+    {  // dq_j = alpha (S_{t-1}^T do)_j + k_j (u . do); lanes 2m, 2m+1 hold row j = warp + 8m
+      const float sdo = warp_rows16_sum(part, lane);
+      const int j = warp + kBwdWarps * (lane >> 1);
+      if ((lane & 1) == 0 && j < dk) dq[row * dk + j] = alpha * sdo + ks[j] * udo;
     }
     if (col_ok) *reinterpret_cast<float4 *>(&gkpart[warp * 128 + col]) = gk;
     gs = warp_sum(gs);
@@ -286,14 +321,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) gdn_bwd_kernel(
     for (int r = 0; r < kRows; ++r) {
       const int j = warp + r * kBwdWarps;
       const float kj = j < dk ? ks[j] : 0.f;
-      // dk_j = (G^T u)_j - alpha beta (S_{t-1}^T Gk)_j
-      const float d = warp_sum(dot4(G[r], u4) - ab * dot4(S[r], gk4));
-      if (lane == r && j < dk) dkk[row * dk + j] = d;
+      // dk_j = (G^T u)_j - alpha beta (S_{t-1}^T Gk)_j, this lane's columns
+      part[r] = dot4(G[r], u4) - ab * dot4(S[r], gk4);
       // G <- alpha (G - beta Gk k^T)
       G[r].x = alpha * (G[r].x - b * gk4.x * kj);
       G[r].y = alpha * (G[r].y - b * gk4.y * kj);
       G[r].z = alpha * (G[r].z - b * gk4.z * kj);
       G[r].w = alpha * (G[r].w - b * gk4.w * kj);
+    }
+    {
+      const float d = warp_rows16_sum(part, lane);
+      const int j = warp + kBwdWarps * (lane >> 1);
+      if ((lane & 1) == 0 && j < dk) dkk[row * dk + j] = d;
     }
     __syncthreads();                                           // (D) vectors free for t - 1
   }

@@ -48,19 +48,32 @@ __device__ __forceinline__ void st_from_f32<__nv_bfloat16>(__nv_bfloat16 *p, flo
 
 constexpr int kSimtThreads = 256;
 constexpr int kDvt = 32;  // d_v columns per CTA
+// The channel-wise gate runs with 16 warps: its CTA (219 KB of shared
+// memory) is alone on its SM, and the extra warps hide the latency of the
+// per-channel exponentials.
+template <bool KDA>
+constexpr int simt_threads() { return KDA ? 512 : kSimtThreads; }
+
+// 2^x on the special-function unit (PTX ex2.approx, flush-to-zero).
+__device__ __forceinline__ float ex2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 // ---------------------------------------------------------------------------
 // fp32 chunked forward. Grid (N, H, ceil(d_v / 32)); one CTA walks all chunks
 // of one sequence for one head and one 32-column slice of d_v, carrying its
 // slice of the state in shared memory. KDA: channel-wise gate (g [rows, H, d_k]).
 template <int C, typename T, bool KDA>
-__global__ void __launch_bounds__(kSimtThreads) gdn_chunk_simt_kernel(
+__global__ void __launch_bounds__(simt_threads<KDA>()) gdn_chunk_simt_kernel(
     const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
     const float *__restrict__ g, const float *__restrict__ beta, const float *__restrict__ s0,
     int H, int dk, int dv, T *__restrict__ o, float *__restrict__ sN,
     const uint32_t *__restrict__ ctrl, const ChunkInfo *__restrict__ table,
     const int32_t *__restrict__ seq_first) {
   extern __shared__ float sm[];
+  constexpr int kThr = simt_threads<KDA>();
   if (ctrl[0] & kErrBadSeqlens) return;
   const int n = blockIdx.x, h = blockIdx.y, i0 = blockIdx.z * kDvt;
   const int tid = threadIdx.x;
@@ -79,12 +92,13 @@ __global__ void __launch_bounds__(kSimtThreads) gdn_chunk_simt_kernel(
   float *Bt = Gm + C;                    // [C] beta
   float *Ga = Bt + C;                    // [C] exp(Gamma)
   float *Dd = Ga + C;                    // [C] exp(Gamma_last - Gamma)
-  // KDA only: per-channel Gamma, then K .* exp(Gamma); and Gamma_last per channel
+  // KDA only: per-channel Gamma log2(e), then K .* exp(Gamma); and Gamma_last
+  // log2(e) per channel (exponentials as 2^x on the special-function unit)
   float *Gk = Dd + C;                    // [C][dkp]
   float *Gl = Gk + C * dkp;              // [dk]
 
   // Initial state slice.
-  for (int e = tid; e < dk * kDvt; e += kSimtThreads) {
+  for (int e = tid; e < dk * kDvt; e += kThr) {
     const int j = e / kDvt, ii = e % kDvt;
     float x = 0.f;
     if (s0 && i0 + ii < dv) x = s0[((size_t(n) * H + h) * dk + j) * dv + i0 + ii];
@@ -96,7 +110,7 @@ __global__ void __launch_bounds__(kSimtThreads) gdn_chunk_simt_kernel(
     const int L = ci.len;
     __syncthreads();
     // 1. load the chunk (rows >= L as zeros)
-    for (int e = tid; e < C * dk; e += kSimtThreads) {
+    for (int e = tid; e < C * dk; e += kThr) {
       const int r = e / dk, j = e % dk;
       float kv = 0.f, qv = 0.f;
       if (r < L) {
@@ -107,7 +121,7 @@ __global__ void __launch_bounds__(kSimtThreads) gdn_chunk_simt_kernel(
       Ks[r * dkp + j] = kv;
       Qs[r * dkp + j] = qv;
     }
-    for (int e = tid; e < C * kDvt; e += kSimtThreads) {
+    for (int e = tid; e < C * kDvt; e += kThr) {
       const int r = e / kDvt, ii = e % kDvt;
       float vv = 0.f;
       if (r < L && i0 + ii < dv) vv = ld_f32(v + (size_t(ci.row0 + r) * H + h) * dv + i0 + ii);
@@ -119,7 +133,7 @@ __global__ void __launch_bounds__(kSimtThreads) gdn_chunk_simt_kernel(
       Bt[tid] = ok ? beta[size_t(ci.row0 + tid) * H + h] : 0.f;
     }
     if (KDA) {
-      for (int e = tid; e < C * dk; e += kSimtThreads) {
+      for (int e = tid; e < C * dk; e += kThr) {
         const int r = e / dk, j = e % dk;
         Gk[r * dkp + j] = r < L ? g[(size_t(ci.row0 + r) * H + h) * dk + j] : 0.f;
       }
@@ -131,9 +145,10 @@ __global__ void __launch_bounds__(kSimtThreads) gdn_chunk_simt_kernel(
       for (int r = 0; r < C; ++r) { acc += Gm[r]; Gm[r] = acc; }
     }
     if (KDA && tid < dk) {   // one channel per thread
+      constexpr float kLog2e = 1.4426950408889634f;
       float acc = 0.f;
-      for (int r = 0; r < C; ++r) { acc += Gk[r * dkp + tid]; Gk[r * dkp + tid] = acc; }
-      Gl[tid] = acc;
+      for (int r = 0; r < C; ++r) { acc += Gk[r * dkp + tid]; Gk[r * dkp + tid] = acc * kLog2e; }
+      Gl[tid] = acc * kLog2e;
     }
     __syncthreads();
     if (!KDA && tid < C) {
@@ -141,14 +156,14 @@ __global__ void __launch_bounds__(kSimtThreads) gdn_chunk_simt_kernel(
       Dd[tid] = expf(Gm[C - 1] - Gm[tid]);
     }
     // 3. A (strictly lower) and P = (Q K^T) .* M (diagonal included)
-    for (int e = tid; e < C * C; e += kSimtThreads) {
+    for (int e = tid; e < C * C; e += kThr) {
       const int r = e / C, s = e % C;
       float a = 0.f, p = 0.f;
       if (s <= r) {
         float dkk = 0.f, dqk = 0.f;
         if (KDA) {
           for (int j = 0; j < dk; ++j) {
-            const float ksj = Ks[s * dkp + j] * expf(Gk[r * dkp + j] - Gk[s * dkp + j]);
+            const float ksj = Ks[s * dkp + j] * ex2_fast(Gk[r * dkp + j] - Gk[s * dkp + j]);
             dkk += Ks[r * dkp + j] * ksj;
             dqk += Qs[r * dkp + j] * ksj;
           }
@@ -172,12 +187,12 @@ __global__ void __launch_bounds__(kSimtThreads) gdn_chunk_simt_kernel(
     if (KDA) {
       // K and Q now enter only with their decays: Gk <- K .* exp(Gamma) (for W),
       // Ks <- K .* exp(Gamma_last - Gamma) (state update), Qs <- Q .* exp(Gamma).
-      for (int e = tid; e < C * dk; e += kSimtThreads) {
+      for (int e = tid; e < C * dk; e += kThr) {
         const int r = e / dk, j = e % dk;
-        const float gam = Gk[r * dkp + j], kv = Ks[r * dkp + j];
-        Gk[r * dkp + j] = kv * expf(gam);
-        Ks[r * dkp + j] = kv * expf(Gl[j] - gam);
-        Qs[r * dkp + j] *= expf(gam);
+        const float gam = Gk[r * dkp + j], kv = Ks[r * dkp + j], eg = ex2_fast(gam);
+        Gk[r * dkp + j] = kv * eg;
+        Ks[r * dkp + j] = kv * ex2_fast(Gl[j] - gam);
+        Qs[r * dkp + j] *= eg;
       }
     }
     // 4. T = (I + A)^-1 by forward substitution; thread s owns column s.
@@ -192,7 +207,7 @@ __global__ void __launch_bounds__(kSimtThreads) gdn_chunk_simt_kernel(
     }
     __syncthreads();
     // 5. W = T diag(beta gamma) K, U = T diag(beta) V
-    for (int e = tid; e < C * dk; e += kSimtThreads) {
+    for (int e = tid; e < C * dk; e += kThr) {
       const int r = e / dk, j = e % dk;
       float acc = 0.f;
       if (KDA)
@@ -202,7 +217,7 @@ __global__ void __launch_bounds__(kSimtThreads) gdn_chunk_simt_kernel(
           acc += Ts[r * (C + 1) + s] * (Bt[s] * Ga[s]) * Ks[s * dkp + j];
       Ws[r * dkp + j] = acc;
     }
-    for (int e = tid; e < C * kDvt; e += kSimtThreads) {
+    for (int e = tid; e < C * kDvt; e += kThr) {
       const int r = e / kDvt, ii = e % kDvt;
       float acc = 0.f;
       for (int s = 0; s <= r; ++s) acc += Ts[r * (C + 1) + s] * Bt[s] * Vs[s * kDvt + ii];
@@ -210,7 +225,7 @@ __global__ void __launch_bounds__(kSimtThreads) gdn_chunk_simt_kernel(
     }
     __syncthreads();
     // 6. V_new = U - W S^T
-    for (int e = tid; e < C * kDvt; e += kSimtThreads) {
+    for (int e = tid; e < C * kDvt; e += kThr) {
       const int r = e / kDvt, ii = e % kDvt;
       float acc = 0.f;
       for (int j = 0; j < dk; ++j) acc += Ws[r * dkp + j] * Ss[j * kDvt + ii];
@@ -218,7 +233,7 @@ __global__ void __launch_bounds__(kSimtThreads) gdn_chunk_simt_kernel(
     }
     __syncthreads();
     // 7. O = diag(gamma) Q S^T + P V_new   (old S)
-    for (int e = tid; e < C * kDvt; e += kSimtThreads) {
+    for (int e = tid; e < C * kDvt; e += kThr) {
       const int r = e / kDvt, ii = e % kDvt;
       if (r < L && i0 + ii < dv) {
         float acc = 0.f;
@@ -231,12 +246,12 @@ __global__ void __launch_bounds__(kSimtThreads) gdn_chunk_simt_kernel(
     }
     __syncthreads();
     // 8. S <- gamma_last S + V_new^T diag(D) K
-    for (int e = tid; e < dk * kDvt; e += kSimtThreads) {
+    for (int e = tid; e < dk * kDvt; e += kThr) {
       const int j = e / kDvt, ii = e % kDvt;
       float acc = 0.f;
       if (KDA) {
         for (int s = 0; s < C; ++s) acc += Ks[s * dkp + j] * Vn[s * kDvt + ii];
-        Ss[e] = expf(Gl[j]) * Ss[e] + acc;
+        Ss[e] = ex2_fast(Gl[j]) * Ss[e] + acc;
       } else {
         for (int s = 0; s < C; ++s) acc += Dd[s] * Ks[s * dkp + j] * Vn[s * kDvt + ii];
         Ss[e] = Ga[C - 1] * Ss[e] + acc;
@@ -245,7 +260,7 @@ __global__ void __launch_bounds__(kSimtThreads) gdn_chunk_simt_kernel(
   }
   __syncthreads();
   if (sN) {
-    for (int e = tid; e < dk * kDvt; e += kSimtThreads) {
+    for (int e = tid; e < dk * kDvt; e += kThr) {
       const int j = e / kDvt, ii = e % kDvt;
       if (i0 + ii < dv) sN[((size_t(n) * H + h) * dk + j) * dv + i0 + ii] = Ss[e];
     }
@@ -266,7 +281,7 @@ cudaError_t launch_simt_t(const void *q, const void *k, const void *v, const flo
                                        int(bytes));
   if (e != cudaSuccess) return e;
   dim3 grid(N, H, (dv + kDvt - 1) / kDvt);
-  kern<<<grid, kSimtThreads, bytes, s>>>(
+  kern<<<grid, simt_threads<KDA>(), bytes, s>>>(
       static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), g, beta,
       s0, H, dk, dv, static_cast<T *>(o), sN, ctrl, table, seq_first);
   return cudaGetLastError();
