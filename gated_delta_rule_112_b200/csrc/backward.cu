@@ -21,8 +21,9 @@
 // (S^T storage st[j][i]: lane l owns rows 4l..4l+3, 64 fp32 registers), so
 // every reduction over d_k stays inside a warp:
 //   gdn_bwd_replay_kernel  runs the recurrence forward and streams every
-//                          S_{t-1} (64 KB) and x_t to the workspace; no
-//                          barrier at all, the warps never wait on each other;
+//                          S_{t-1} (64 KB, in the warps' own slot order) and
+//                          x_t to the workspace; no barrier at all, the warps
+//                          never wait on each other;
 //   gdn_bwd_kernel         walks the tokens backwards with G in registers,
 //                          S_{t-1} of the next token prefetched into shared
 //                          memory with cp.async and the next token's vectors
@@ -120,6 +121,15 @@ __device__ __forceinline__ void load_block(float (&X)[4][kCols], const float *sr
     }
 }
 
+// Position of a lane's float4 (column group w, row a of the lane, float4 m of
+// the warp's 16 columns) inside one token's 128 x 128 block of the workspace.
+// Consecutive lanes hold consecutive 16-byte slots, so every warp-wide store
+// or load of S_{t-1} moves 512 contiguous bytes.
+__device__ __forceinline__ int slot(int w, int a, int m, int lane) {
+  return (((w * 4 + a) * 4 + m) * 32 + lane) * 4;
+}
+constexpr int kBlockWords = 128 * 128;   // one token's S_{t-1} in the workspace
+
 template <bool kStreaming>
 __device__ __forceinline__ void store_block(const float (&X)[4][kCols], float *dst, int j0, int c0,
                                             int dk, int dv) {
@@ -177,7 +187,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1) gdn_bwd_replay_kernel(
     for (int a = 0; a < 4; ++a) kt[a] = kn[a];
     const float vt = vn, alpha = expf(an), b = bn;
     if (t + 1 < t1) fetch(t + 1);   // the next token's loads overlap this one
-    store_block<true>(S, s_prev + row * SS, j0, c0, dk, dv);
+    {
+      float *dst = s_prev + row * kBlockWords;
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+          if (j0 + a < dk && c0 + 4 * m < dv)
+            __stcs(reinterpret_cast<float4 *>(dst + slot(warp, a, m, lane)),
+                   make_float4(S[a][4 * m], S[a][4 * m + 1], S[a][4 * m + 2], S[a][4 * m + 3]));
+    }
     float xp[kCols];
 #pragma unroll
     for (int c = 0; c < kCols; ++c)
@@ -246,15 +265,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1) gdn_bwd_kernel(
       for (int c = 0; c < kCols; ++c) G[a][c] = 0.f;
 
   auto prefetch_state = [&](int t, int buf) {
-    const float *src = s_prev + (size_t(t) * H + h) * SS;
+    const float *src = s_prev + (size_t(t) * H + h) * kBlockWords;
     float *dst = stage + buf * kStageWords;
 #pragma unroll
     for (int a = 0; a < 4; ++a)
 #pragma unroll
       for (int m = 0; m < 4; ++m)
-        if (j0 + a < dk && c0 + 4 * m < dv)
-          cp_async16(smem_u32(dst + (j0 + a) * 128 + c0 + 4 * m),
-                     src + size_t(j0 + a) * dv + c0 + 4 * m);
+        if (j0 + a < dk && c0 + 4 * m < dv) {
+          const int o = slot(warp, a, m, lane);
+          cp_async16(smem_u32(dst + o), src + o);
+        }
     cp_async_commit();
   };
   // Staging of one token's vectors: thread tid < 128 owns index tid of k and q,
@@ -315,7 +335,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) gdn_bwd_kernel(
         for (int m = 0; m < 4; ++m) {
           float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
           if (j0 + a < dk && c0 + 4 * m < dv)
-            x = *reinterpret_cast<const float4 *>(cur + (j0 + a) * 128 + c0 + 4 * m);
+            x = *reinterpret_cast<const float4 *>(cur + slot(warp, a, m, lane));
           S[a][4 * m] = x.x; S[a][4 * m + 1] = x.y; S[a][4 * m + 2] = x.z; S[a][4 * m + 3] = x.w;
         }
     }

@@ -5,16 +5,18 @@
 namespace gdn {
 
 // Workspace of the backward pass: the 256 B control block, then S_{t-1}
-// before every token (fp32 [B*T][H][d_k][d_v], the S^T storage) and
-// x_t = S_{t-1} k_t (fp32 [B*T][H][d_v]).
+// before every token (fp32, one 128 x 128 block per (token, head) in the
+// kernels' own slot order, whatever d_k, d_v <= 128) and x_t = S_{t-1} k_t
+// (fp32 [B*T][H][d_v]).
 struct BwdLayout {
   size_t s_prev, x, total;
 };
 inline BwdLayout bwd_layout(int B, int T, int H, int dk, int dv) {
+  (void)dk;
   BwdLayout L{};
   const size_t rows = size_t(B) * size_t(T) * size_t(H);
   L.s_prev = 256;
-  L.x = align_up(L.s_prev + rows * size_t(dk) * dv * sizeof(float), 256);
+  L.x = align_up(L.s_prev + rows * size_t(128 * 128) * sizeof(float), 256);
   L.total = align_up(L.x + rows * size_t(dv) * sizeof(float), 256);
   return L;
 }

@@ -257,8 +257,9 @@ int gdn_kda_decode_step(const void *q, const void *k, const void *v, const float
  * and d_initial_state = G at each sequence's start.
  */
 
-/* Bytes of workspace gdn_chunk_bwd needs: 256 + B*T*H*(d_k*d_v + d_v)*4
- * (every token's S_{t-1} and S_{t-1} k_t, fp32), rounded up; 0 for invalid sizes. */
+/* Bytes of workspace gdn_chunk_bwd needs: 256 + B*T*H*(128*128 + d_v)*4
+ * (every token's S_{t-1} in a 128 x 128 fp32 block, and S_{t-1} k_t), rounded
+ * up; 0 for invalid sizes. */
 size_t gdn_chunk_bwd_workspace_size(int B, int T, int H, int d_k, int d_v, int num_seqs);
 
 /*
