@@ -128,3 +128,16 @@ def test_bwd_varlen_equals_separate_sequences():
             np.testing.assert_allclose(gr[key][:, s:e], gn[key], rtol=0, atol=1e-14)
         np.testing.assert_allclose(gr["d_initial_state"][n], gn["d_initial_state"][0], rtol=0,
                                    atol=1e-14)
+
+
+def test_bwd_is_causal():
+    # a loss on the outputs of tokens < t_cut only: no gradient reaches the
+    # inputs of later tokens (exact zeros, not small numbers)
+    a = make(8, T=12, H=2, dk=3, dv=4)
+    t_cut = 7
+    a["d_o"][:, t_cut:] = 0.0
+    a["dsN"][:] = 0.0
+    gr = grads(a)
+    for key in ("dk", "dv", "dg", "dbeta", "dq"):
+        assert np.max(np.abs(gr[key][:, t_cut:])) == 0.0, key
+    assert np.max(np.abs(gr["dv"][:, :t_cut])) > 0.0

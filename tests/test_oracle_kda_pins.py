@@ -141,3 +141,33 @@ def test_kda_rejects_scalar_shaped_gate():
     q, k, v, g, beta, S0 = make(7)
     with pytest.raises(ValueError):
         oracle.kda_chunk_fwd(q, k, v, g[..., 0], beta, S0)
+
+
+def test_kda_linear_in_values_and_state():
+    # S_t and o_t are jointly linear in (V, S_0) for fixed keys, queries and gates
+    q, k, v, g, beta, S0 = make(8, T=15, dk=4, dv=3)
+    o1, f1 = oracle.kda_chunk_fwd(q, k, v, g, beta, S0)
+    o2, f2 = oracle.kda_chunk_fwd(q, k, -2.5 * v, g, beta, -2.5 * S0)
+    np.testing.assert_allclose(o2, -2.5 * o1, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(f2, -2.5 * f1, rtol=1e-13, atol=1e-14)
+
+
+def test_kda_cycling_unit_keys_closed_form():
+    # k_t = e_{t mod d_k}, beta = 1: each token first decays every column of S by
+    # its own channel's alpha, then overwrites column t mod d_k with v_t. So
+    # column m of S_T is v_tau times the decays of channel m after tau (tau = the
+    # last token that wrote it), or S_0's column times all its decays.
+    dk, dv, T = 4, 3, 10
+    q, k, v, g, beta, S0 = make(9, T=T, H=1, dk=dk, dv=dv)
+    k[:] = 0.0
+    for t in range(T):
+        k[0, t, 0, t % dk] = 1.0
+    beta[:] = 1.0
+    _, fs = oracle.kda_chunk_fwd(q, k, v, g, beta, S0)
+    alpha = np.exp(g[0, :, 0])                   # [T, dk]
+    want = np.zeros((dk, dv))                    # S^T storage: row m = column m of S
+    for m in range(dk):
+        writers = [t for t in range(T) if t % dk == m]
+        tau = writers[-1]
+        want[m] = v[0, tau, 0] * np.prod(alpha[tau + 1:, m])
+    np.testing.assert_allclose(fs[0, 0], want, rtol=1e-13, atol=1e-15)

@@ -55,6 +55,7 @@ KDA_PIN_CASES = [
     kda_pins.test_kda_beta_zero_is_channel_decay,
     lambda: kda_pins.test_kda_unit_key_beta_one_overwrites(3),
     lambda: kda_pins.test_kda_dense_chunked_matches_token_loop(4, 7),
+    kda_pins.test_kda_cycling_unit_keys_closed_form,
 ]
 
 # Mistakes in the gradient loop, caught by the gradient pins.
@@ -78,6 +79,7 @@ BWD_PIN_CASES = [
     lambda: bwd_pins.test_bwd_matches_central_differences("plain"),
     bwd_pins.test_bwd_homogeneity_identities,
     bwd_pins.test_bwd_beta_zero_closed_form,
+    bwd_pins.test_bwd_is_causal,
 ]
 
 PIN_CASES = [
