@@ -156,20 +156,50 @@ __global__ void __launch_bounds__(simt_threads<KDA>()) gdn_chunk_simt_kernel(
       Dd[tid] = expf(Gm[C - 1] - Gm[tid]);
     }
     // 3. A (strictly lower) and P = (Q K^T) .* M (diagonal included)
-    for (int e = tid; e < C * C; e += kThr) {
+    if (KDA) {
+      // One thread per 2 x 2 block of (r, s) pairs: every loaded row element is
+      // used twice. Pair (r0, s1) of a diagonal block lies above the diagonal
+      // and is skipped before its exponent is formed (it could overflow).
+      constexpr int Cb = C / 2;
+      for (int e = tid; e < Cb * Cb; e += kThr) {
+        const int R = e / Cb, Sb = e % Cb;
+        const int r0 = 2 * R, r1 = r0 + 1, s0 = 2 * Sb, s1 = s0 + 1;
+        float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
+        float p00 = 0.f, p01 = 0.f, p10 = 0.f, p11 = 0.f;
+        if (Sb <= R) {
+          const bool v01 = s1 <= r0;
+          for (int j = 0; j < dk; ++j) {
+            const float gr0 = Gk[r0 * dkp + j], gr1 = Gk[r1 * dkp + j];
+            const float gs0 = Gk[s0 * dkp + j], gs1 = Gk[s1 * dkp + j];
+            const float ks0 = Ks[s0 * dkp + j], ks1 = Ks[s1 * dkp + j];
+            const float kr0 = Ks[r0 * dkp + j], kr1 = Ks[r1 * dkp + j];
+            const float qr0 = Qs[r0 * dkp + j], qr1 = Qs[r1 * dkp + j];
+            const float e00 = ks0 * ex2_fast(gr0 - gs0);
+            const float e01 = v01 ? ks1 * ex2_fast(gr0 - gs1) : 0.f;
+            const float e10 = ks0 * ex2_fast(gr1 - gs0);
+            const float e11 = ks1 * ex2_fast(gr1 - gs1);
+            a00 += kr0 * e00; p00 += qr0 * e00;
+            a01 += kr0 * e01; p01 += qr0 * e01;
+            a10 += kr1 * e10; p10 += qr1 * e10;
+            a11 += kr1 * e11; p11 += qr1 * e11;
+          }
+        }
+        As[r0 * (C + 1) + s0] = s0 < r0 ? Bt[r0] * a00 : 0.f;
+        As[r0 * (C + 1) + s1] = s1 < r0 ? Bt[r0] * a01 : 0.f;
+        As[r1 * (C + 1) + s0] = s0 < r1 ? Bt[r1] * a10 : 0.f;
+        As[r1 * (C + 1) + s1] = s1 < r1 ? Bt[r1] * a11 : 0.f;
+        Ps[r0 * (C + 1) + s0] = s0 <= r0 ? p00 : 0.f;
+        Ps[r0 * (C + 1) + s1] = s1 <= r0 ? p01 : 0.f;
+        Ps[r1 * (C + 1) + s0] = s0 <= r1 ? p10 : 0.f;
+        Ps[r1 * (C + 1) + s1] = s1 <= r1 ? p11 : 0.f;
+      }
+    }
+    for (int e = tid; !KDA && e < C * C; e += kThr) {
       const int r = e / C, s = e % C;
       float a = 0.f, p = 0.f;
       if (s <= r) {
         float dkk = 0.f, dqk = 0.f;
-        if (KDA) {
-          for (int j = 0; j < dk; ++j) {
-            const float ksj = Ks[s * dkp + j] * ex2_fast(Gk[r * dkp + j] - Gk[s * dkp + j]);
-            dkk += Ks[r * dkp + j] * ksj;
-            dqk += Qs[r * dkp + j] * ksj;
-          }
-          if (s < r) a = Bt[r] * dkk;
-          p = dqk;
-        } else {
+        {
           for (int j = 0; j < dk; ++j) {
             const float ksj = Ks[s * dkp + j];
             dkk += Ks[r * dkp + j] * ksj;
