@@ -23,7 +23,8 @@
 //   gdn_bwd_replay_kernel  runs the recurrence forward and streams every
 //                          S_{t-1} (64 KB, in the warps' own slot order) and
 //                          x_t to the workspace; no barrier at all, the warps
-//                          never wait on each other;
+//                          never wait on each other, so a (sequence, head)
+//                          runs as two CTAs of 4 warps;
 //   gdn_bwd_kernel         walks the tokens backwards with G in registers,
 //                          S_{t-1} of the next token prefetched into shared
 //                          memory with cp.async and the next token's vectors
@@ -41,6 +42,9 @@ namespace {
 constexpr int kBwdThreads = 256;
 constexpr int kBwdWarps = kBwdThreads / 32;
 constexpr int kCols = 16;   // d_v columns per warp (8 warps x 16 = 128)
+// The replay's warps never wait on each other, so each (sequence, head) runs
+// as two CTAs of 4 warps (64 columns each): twice the SMs streaming states.
+constexpr int kReplayWarps = 4;
 
 template <typename Elt>
 __device__ __forceinline__ float ldf(const Elt *p);
@@ -147,13 +151,14 @@ __device__ __forceinline__ void store_block(const float (&X)[4][kCols], float *d
 }
 
 template <typename Elt>
-__global__ void __launch_bounds__(kBwdThreads, 1) gdn_bwd_replay_kernel(
+__global__ void __launch_bounds__(kReplayWarps * 32) gdn_bwd_replay_kernel(
     const Elt *__restrict__ k, const Elt *__restrict__ v, const float *__restrict__ g,
     const float *__restrict__ beta, const float *__restrict__ s0, const int32_t *__restrict__ cu,
     int N, int B, int T, int H, int dk, int dv, float *__restrict__ s_prev,
     float *__restrict__ x_out, uint32_t *__restrict__ ctrl) {
   const int n = blockIdx.x / H, h = blockIdx.x - n * H;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int warp = blockIdx.y * kReplayWarps + (threadIdx.x >> 5);   // column group 0..7
   int t0, t1;
   if (!seq_range(cu, n, N, B, T, t0, t1, ctrl)) return;
   const int c0 = warp * kCols, j0 = 4 * lane, cc = lane >> 1;
@@ -439,7 +444,8 @@ cudaError_t launch_bwd_t(const void *q, const void *k, const void *v, const floa
   float *sp = reinterpret_cast<float *>(base + L.s_prev);
   float *xo = reinterpret_cast<float *>(base + L.x);
   const unsigned units = unsigned(N) * unsigned(H);
-  gdn_bwd_replay_kernel<Elt><<<units, kBwdThreads, 0, s>>>(
+  const dim3 rgrid(units, (dv + kReplayWarps * kCols - 1) / (kReplayWarps * kCols));
+  gdn_bwd_replay_kernel<Elt><<<rgrid, kReplayWarps * 32, 0, s>>>(
       static_cast<const Elt *>(k), static_cast<const Elt *>(v), g, beta, s0, cu, N, B, T, H, dk,
       dv, sp, xo, ctrl);
   cudaError_t e = cudaGetLastError();
