@@ -9,9 +9,16 @@ already resident in HBM. The decode step (N=256, H=32, d=128, fp32 state,
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-With N > 1 (launched by torchrun, one rank per GPU) every rank runs its own
-independent copy of the workload (weak scaling, no collective on the data
-path); times are the max over ranks. ``--impl reference`` times the CPU fp64
+With N > 1 (launched by torchrun, one rank per GPU) the job is partitioned
+with no collective on the data path (every (sequence, head) recurrence is
+independent): by default every rank owns its own batch of B sequences of a
+job of N*B sequences (weak scaling); ``--scaling strong`` splits the one
+workload's heads across the ranks (gated_delta_rule_112_b200.partition).
+Times are the max over ranks.
+
+The long-context (long64k) and packed-varlen (varlen64) configurations are
+measured in the same run and reported under their names, each against its
+own algorithmic bytes. ``--impl reference`` times the CPU fp64
 oracle (the slow, obviously-correct program the GPU path is checked
 against) on a bounded sample of the same workload.
 
@@ -41,6 +48,8 @@ METRIC_KDA = ("chunk-fwd Mtokens/s at B4·H16·T4096·d128 bf16, channel-wise ga
 BYTES_PER_TOKEN_HEAD = 3 * 128 * 2 + 128 * 2 + 2 * 4    # q,k,v,o bf16 + g,beta fp32
 BYTES_PER_TOKEN_HEAD_KDA = 3 * 128 * 2 + 128 * 2 + 128 * 4 + 4   # g is one fp32 per channel
 L2_FLUSH_BYTES = 256 << 20
+# Chunked-forward configurations measured beside the headline one.
+EXTRA_WORKLOADS = ("long64k", "varlen64")
 # fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 flop x 1965 MHz (max SM clock)
 FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
@@ -54,6 +63,11 @@ def parse_args():
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--scaling", choices=["weak", "strong"], default="weak",
+                   help="N > 1: weak = every rank owns B sequences of a job of N*B "
+                        "sequences; strong = one workload split by heads across the ranks")
+    p.add_argument("--no-extra-workloads", action="store_true",
+                   help="skip the long64k and varlen64 sub-measurements")
     p.add_argument("--bwd", action="store_true",
                    help="also time the backward pass (gdn_chunk_bwd) on the workload")
     p.add_argument("--workload", default=WORKLOAD,
@@ -213,7 +227,7 @@ def main():
     import torch.distributed as dist
 
     import gated_delta_rule_112_b200 as gdn
-    from gated_delta_rule_112_b200.inputs import make_chunk_inputs, make_decode_inputs
+    from gated_delta_rule_112_b200.inputs import WORKLOADS, make_chunk_inputs, make_decode_inputs
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -227,7 +241,14 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
-    from gated_delta_rule_112_b200 import replicas
+    from gated_delta_rule_112_b200 import partition, replicas
+    strong = args.scaling == "strong" and world > 1
+    if strong and world > WORKLOADS[args.workload].H:
+        raise SystemExit("--scaling strong needs at least one head per rank")
+    # Whole-job rate: weak scaling counts every rank's tokens, strong scaling
+    # the one workload's tokens (each rank did a part of every token).
+    def job_value(tokens, ms):
+        return tokens / (ms * 1e-3) if strong else replicas.job_rate(tokens, ms, world)
 
     barrier = replicas.barrier
 
@@ -239,97 +260,141 @@ def main():
     L = gdn.lib()
 
     # --------------------------------------------------------------- chunked forward
-    from gated_delta_rule_112_b200.inputs import WORKLOADS
     wl = args.workload
-    seed = replicas.shard_seed(WORKLOADS[wl].seed, rank)
-    inp = make_chunk_inputs(wl, seed=seed)
-    kda = inp["gate"] == "channel"
-    fwd = gdn.kda_chunk_fwd if kda else gdn.chunk_fwd
-    ws_size = gdn.kda_workspace_size if kda else gdn.workspace_size
-    B, T, H = inp["B"], inp["T"], inp["H"]
-    q, k, v, g, beta = (inp[x].to(dev) for x in ("q", "k", "v", "g", "beta"))
-    s0 = inp["initial_state"].to(dev) if inp["initial_state"] is not None else None
-    cu = inp["cu_seqlens"].to(dev) if inp["cu_seqlens"] is not None else None
-    nseq = B if cu is None else cu.numel() - 1
-    o = torch.empty(B, T, H, 128, dtype=torch.bfloat16, device=dev)
-    fs = torch.empty(nseq, H, 128, 128, dtype=torch.float32, device=dev)
-    ws = torch.empty(ws_size(B, T, H, 128, 128, 0 if cu is None else nseq),
-                     dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-
-    def step():
-        fwd(q, k, v, g, beta, s0, cu, out=o, workspace=ws)
-
-    for _ in range(max(args.warmup, 3)):
-        step()
-    torch.cuda.synchronize()
-    assert gdn.get_status(ws) == gdn.OK
-
     K = args.steps
-    # Timed region: one event pair around each step. The prep and scan kernels
-    # start with programmatic dependent launch; an event between them would
-    # serialise them, so the per-kernel split comes from a separate pass below.
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
-    for e in evs:                      # torch creates the CUDA event on first record
-        for x in e:
-            x.record(stream)
+
+    def measure_chunk(wname, steps, warmup, sampler=None):
+        """Time `steps` chunked forward passes of workload `wname` (inputs
+        resident in HBM, L2 flushed before each step) and, in a separate untimed
+        pass, the per-kernel split. Returns the tensors and the figures."""
+        if strong:
+            # one workload (one seed) split by heads; this rank runs its range
+            inp = make_chunk_inputs(wname)
+            inp = partition.shard(inp, partition.plan(inp, world, "heads")[rank])
+        else:
+            # weak scaling: the job is `world` batches of sequences, rank r owning
+            # the r-th (drawn with its own seed); no data crosses ranks
+            inp = make_chunk_inputs(wname, seed=replicas.shard_seed(WORKLOADS[wname].seed, rank))
+        kda = inp["gate"] == "channel"
+        fwd = gdn.kda_chunk_fwd if kda else gdn.chunk_fwd
+        ws_size = gdn.kda_workspace_size if kda else gdn.workspace_size
+        B, T, H = inp["B"], inp["T"], inp["H"]
+        t = {x: inp[x].to(dev) for x in ("q", "k", "v", "g", "beta")}
+        s0 = inp["initial_state"].to(dev) if inp["initial_state"] is not None else None
+        cu = inp["cu_seqlens"].to(dev) if inp["cu_seqlens"] is not None else None
+        nseq = B if cu is None else cu.numel() - 1
+        o = torch.empty(B, T, H, 128, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(ws_size(B, T, H, 128, 128, 0 if cu is None else nseq),
+                         dtype=torch.uint8, device=dev)
+
+        def step():
+            return fwd(t["q"], t["k"], t["v"], t["g"], t["beta"], s0, cu, out=o, workspace=ws)
+
+        for _ in range(max(warmup, 3)):
+            step()
+        torch.cuda.synchronize()
+        assert gdn.get_status(ws) == gdn.OK
+        # Timed region: one event pair around each step. The kernels of a step
+        # start with programmatic dependent launch; an event between them would
+        # serialise them, so the per-kernel split comes from a separate pass.
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+        for e in evs:                  # torch creates the CUDA event on first record
+            for x in e:
+                x.record(stream)
+        if sampler is not None:
+            sampler.start()
+        barrier()
+        torch.cuda.synchronize()
+        for i in range(steps):
+            flush.fill_(i & 0xFF)                       # evict L2 between timed steps
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        clocks = sampler.stop() if sampler is not None else None
+        status = gdn.get_status(ws)
+        if status != gdn.OK:
+            raise SystemExit(f"device status {status}")
+        ms_local = sum(a.elapsed_time(b) for a, b in evs) / steps
+        ms = max_over_ranks(ms_local)
+        # Per-kernel split (untimed pass): events recorded between the launches.
+        kp = min(steps, 10)
+        pev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(kp)]
+        for e in pev:
+            for x in e:
+                x.record(stream)
+        torch.cuda.synchronize()
+        for i in range(kp):
+            flush.fill_(i & 0xFF)
+            e = pev[i]
+            L.gdn_set_profile_events(e[0].cuda_event, e[1].cuda_event, e[2].cuda_event,
+                                     e[3].cuda_event)
+            step()
+        L.gdn_set_profile_events(None, None, None, None)
+        torch.cuda.synchronize()
+        t_map = statistics.mean(e[0].elapsed_time(e[1]) for e in pev)
+        t_prep = statistics.mean(e[1].elapsed_time(e[2]) for e in pev)
+        t_scan = statistics.mean(e[2].elapsed_time(e[3]) for e in pev)
+        tokens = B * T if cu is None else int(inp["cu_seqlens"][-1])
+        state_io = (2 if s0 is not None else 1) * nseq * H * 128 * 128 * 4   # final (+ initial)
+        alg_bytes = tokens * H * (BYTES_PER_TOKEN_HEAD_KDA if kda else BYTES_PER_TOKEN_HEAD) \
+            + state_io
+        flops = tokens * H * 2 * (3 * 64 * 128 + 2 * 64 * 128 + 3 * 128 * 128)
+        if kda:   # one CUDA-core kernel after the chunk map (prep/scan events coincide)
+            kernels = {"gdn_chunk_map_kernel": t_map, "gdn_chunk_simt_kernel": t_scan}
+        else:
+            kernels = {"gdn_chunk_map_kernel": t_map, "gdn_prep_kernel": t_prep,
+                       "gdn_scan_kernel": t_scan}
+        segs = 1 if kda else int(L.gdn_chunk_fwd_scan_segments(
+            B, T, H, 128, 128, 0 if cu is None else nseq, 64, gdn.BF16,
+            torch.cuda.get_device_properties(dev).multi_processor_count))
+        launches = 2 if kda else (3 if segs <= 1 else 5)
+        return dict(inp=inp, kda=kda, fwd=fwd, t=t, s0=s0, cu=cu, o=o, ws=ws, B=B, T=T, H=H,
+                    nseq=nseq, tokens=tokens, ms=ms, ms_local=ms_local, alg_bytes=alg_bytes,
+                    flops=flops, kernels=kernels, clocks=clocks, launches=launches, segs=segs)
+
+    def workload_summary(r, steps):
+        gbs = r["alg_bytes"] / (r["ms_local"] * 1e-3) / 1e9
+        tot = sum(r["kernels"].values())
+        return {"workload": r["wname"], "tokens": r["tokens"], "heads": r["H"],
+                "sequences": r["nseq"], "ms_per_step": r["ms"], "steps": steps,
+                "value": job_value(r["tokens"], r["ms"]) / 1e6, "unit": UNIT,
+                "gpu_launches": r["launches"] * steps, "scan_segments": r["segs"],
+                "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
+                             "frac": gbs / pk["hbm"], "algorithmic_bytes": r["alg_bytes"],
+                             "traffic": recorded_traffic("chunk_fwd_step/" + r["wname"]),
+                             "peak_source": pk["source"]},
+                "kernels_ms": r["kernels"],
+                "kernel_share": {k2: v2 / tot for k2, v2 in r["kernels"].items()}}
+
     uuid = str(torch.cuda.get_device_properties(dev).uuid)
     sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
-    sampler.start()
-    barrier()
-    torch.cuda.synchronize()
-    for i in range(K):
-        flush.fill_(i & 0xFF)                       # evict L2 between timed steps
-        evs[i][0].record(stream)
-        step()
-        evs[i][1].record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    clocks = sampler.stop()
-    status = gdn.get_status(ws)
-    if status != gdn.OK:
-        raise SystemExit(f"device status {status}")
-    t_step = [a.elapsed_time(b) for a, b in evs]
-    ms_local = sum(t_step) / K
-    ms = max_over_ranks(ms_local)
-
-    # Per-kernel split (untimed pass): events recorded between the launches.
-    kp = min(K, 10)
-    pev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(kp)]
-    for e in pev:
-        for x in e:
-            x.record(stream)
-    torch.cuda.synchronize()
-    for i in range(kp):
-        flush.fill_(i & 0xFF)
-        e = pev[i]
-        L.gdn_set_profile_events(e[0].cuda_event, e[1].cuda_event, e[2].cuda_event,
-                                 e[3].cuda_event)
-        step()
-    L.gdn_set_profile_events(None, None, None, None)
-    torch.cuda.synchronize()
-    t_map = [e[0].elapsed_time(e[1]) for e in pev]
-    t_prep = [e[1].elapsed_time(e[2]) for e in pev]
-    t_scan = [e[2].elapsed_time(e[3]) for e in pev]
-    tokens = B * T
-    value = replicas.job_rate(tokens, ms, world) / 1e6
-
-    state_io = (2 if s0 is not None else 1) * nseq * H * 128 * 128 * 4   # final (+ initial) state
-    alg_bytes = tokens * H * (BYTES_PER_TOKEN_HEAD_KDA if kda else BYTES_PER_TOKEN_HEAD) \
-        + state_io
-    flops = tokens * H * 2 * (3 * 64 * 128 + 2 * 64 * 128 + 3 * 128 * 128)
+    main_r = measure_chunk(wl, K, args.warmup, sampler)
+    main_r["wname"] = wl
+    inp, kda, fwd = main_r["inp"], main_r["kda"], main_r["fwd"]
+    q, k, v, g, beta = (main_r["t"][x] for x in ("q", "k", "v", "g", "beta"))
+    s0, cu, o, ws = main_r["s0"], main_r["cu"], main_r["o"], main_r["ws"]
+    B, T, H, nseq, tokens = main_r["B"], main_r["T"], main_r["H"], main_r["nseq"], main_r["tokens"]
+    ms, ms_local, clocks = main_r["ms"], main_r["ms_local"], main_r["clocks"]
+    alg_bytes, flops, kernels = main_r["alg_bytes"], main_r["flops"], main_r["kernels"]
+    fs = torch.empty(nseq, H, 128, 128, dtype=torch.float32, device=dev)
+    value = job_value(tokens, ms) / 1e6
     ach_gbs = alg_bytes / (ms_local * 1e-3) / 1e9
-    if kda:   # one CUDA-core kernel after the chunk map (prep/scan events coincide)
-        kernels = {"gdn_chunk_map_kernel": statistics.mean(t_map),
-                   "gdn_chunk_simt_kernel": statistics.mean(t_scan)}
-    else:
-        kernels = {
-            "gdn_chunk_map_kernel": statistics.mean(t_map),
-            "gdn_prep_kernel": statistics.mean(t_prep),
-            "gdn_scan_kernel": statistics.mean(t_scan),
-        }
     tot = sum(kernels.values())
     traffic = recorded_traffic(("kda_chunk_fwd_step/" if kda else "chunk_fwd_step/") + wl)
+
+    # The other chunked-forward configurations (long context; packed varlen),
+    # each with its own roofline against its own algorithmic bytes.
+    others = {}
+    if wl == WORKLOAD and not args.no_extra_workloads:
+        for extra in EXTRA_WORKLOADS:
+            r = measure_chunk(extra, min(K, 10), 3)
+            r["wname"] = extra
+            others[extra] = workload_summary(r, min(K, 10))
+            del r
+            torch.cuda.empty_cache()
 
     # --------------------------------------------------------------- end to end (host buffers)
     e2e = None
@@ -363,7 +428,7 @@ def main():
         torch.cuda.synchronize()
         barrier()
         ms_e2e = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / ke)
-        e2e = {"value": replicas.job_rate(tokens, ms_e2e, world) / 1e6, "unit": UNIT,
+        e2e = {"value": job_value(tokens, ms_e2e) / 1e6, "unit": UNIT,
                "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "steps": ke,
                "api": ("gated_delta_rule_112_b200.kda_chunk_fwd (C ABI gdn_kda_chunk_fwd)" if kda
@@ -498,7 +563,8 @@ def main():
     line = {
         "metric": METRIC_KDA if kda else METRIC, "value": value, "unit": UNIT,
         "n_gpus": world, "steps": K,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "strong" if strong else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl, "B": B, "T": T, "H": H, "d_k": 128, "d_v": 128,
                    "chunk": 64, "sequences": nseq,
@@ -506,7 +572,9 @@ def main():
                    "initial_state": "zeros" if s0 is None else "random",
                    "final_state": True,
                    "l2": "flushed before every timed step (256 MiB device write)",
-                   "parallelism": f"{world} independent replica(s), no collective"},
+                   "parallelism": (f"{world} ranks, heads split across ranks, no collective"
+                                   if strong else f"{world} rank(s), each owning its own "
+                                   f"batch of sequences, no collective")},
         "roofline": roof,
         "kernels_ms": kernels,
         "kernel_share": {k2: v2 / tot for k2, v2 in kernels.items()},
@@ -519,6 +587,7 @@ def main():
         "backward": backward,
         "cpu_baseline": cpu,
     }
+    line.update(others)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

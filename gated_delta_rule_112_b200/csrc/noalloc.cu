@@ -12,8 +12,10 @@
 // library keeps kNoAllocScratchBytes of device memory reserved for it until
 // the process exits. Its device address is looked up once per device (under a
 // mutex) with cudaGetSymbolAddress; in host code the array's name is only a
-// host-side stand-in and must never be handed to a kernel. All calls on a
-// device share the one array, and it keeps whatever the last call left there.
+// host-side stand-in and must never be handed to a kernel. The looked-up
+// address is cached for the life of the process: after cudaDeviceReset it is
+// stale and this entry point must not be called again. All calls on a device
+// share the one array, and it keeps whatever the last call left there.
 #include <mutex>
 
 #include "gdn_internal.cuh"
@@ -36,7 +38,8 @@ extern "C" int gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v
                                      int B, int T, int H, int d_k, int d_v, int num_seqs,
                                      int chunk, int dtype, void *o, float *final_state,
                                      void *stream) {
-  // Size check first: it needs no CUDA call.
+  // Size check first. It launches nothing, but the size depends on the current
+  // device's SM count (the segmented scan's layout does), which it queries.
   const size_t need =
       gdn_chunk_fwd_workspace_size(B, T, H, d_k, d_v, num_seqs, chunk, dtype);
   if (need > kNoAllocScratchBytes) return GDN_ERR_WORKSPACE;

@@ -138,8 +138,12 @@ int gdn_chunk_fwd_simt(const void *q, const void *k, const void *v, const float 
  *   Returns GDN_ERR_WORKSPACE (and launches nothing) when these sizes need
  *   more than 64 MiB of scratch, i.e. gdn_chunk_fwd_workspace_size(...) >
  *   64 MiB -- roughly 2,000 (chunk, head) pairs on the tensor-core path.
+ *   That size is evaluated against the current device's SM count (the
+ *   segmented scan's layout depends on it); the check launches nothing.
  *   The first call on a device looks up the array's device address (once per
  *   device, thread-safe); make that first call before any stream capture.
+ *   The address stays cached for the process: after cudaDeviceReset it is
+ *   stale, and this entry point must not be called again.
  *   All calls on a device share the array and it keeps the last call's
  *   contents, so calls that overlap on the GPU (different streams, no
  *   ordering between them) race and produce undefined results; serialise

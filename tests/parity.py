@@ -10,6 +10,13 @@ import oracle
 TOL_BF16 = 5e-3
 TOL_F32 = 1e-5
 
+# Every comparison made through assert_close, in order: the test that made it,
+# the tensor's name, relative L2, max-abs and the tolerance. conftest.py prints
+# them at the end of the session and writes them as JSON when the environment
+# variable GDN_PARITY_MARGINS names a file.
+RECORDS = []
+CURRENT_TEST = {"id": None}
+
 
 def np64(t):
     return None if t is None else t.detach().float().cpu().double().numpy()
@@ -59,6 +66,9 @@ def gpu_chunk(inp, force_simt=False, chunk=None):
 def assert_close(name, got, ref, tol):
     r = rel_l2(got, ref)
     m = max_abs(got, ref)
+    RECORDS.append({"test": CURRENT_TEST["id"], "tensor": name, "rel_l2": r, "max_abs": m,
+                    "ref_max_abs": float(np.max(np.abs(ref))) if np.size(ref) else 0.0,
+                    "tol": tol, "passed": bool(np.all(np.isfinite(got)) and r <= tol)})
     assert np.all(np.isfinite(got)), f"{name}: non-finite values"
     assert r <= tol, f"{name}: rel-L2 {r:.3e} > {tol:.1e} (max-abs {m:.3e})"
     return r, m

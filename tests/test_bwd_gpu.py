@@ -59,7 +59,7 @@ def test_bwd_fp32_lengths(T, with_state):
     check(inp, d_o, dsN)
 
 
-@pytest.mark.parametrize("dk,dv", [(64, 32), (96, 128), (128, 64)])
+@pytest.mark.parametrize("dk,dv", [(64, 32), (96, 128), (128, 64), (128, 96), (64, 80)])
 def test_bwd_fp32_head_sizes(dk, dv):
     w = Workload("bwd_sizes", B=2, T=90, H=2, d_k=dk, d_v=dv, seed=32, dtype=torch.float32,
                  random_state=True)

@@ -12,7 +12,7 @@ import torch
 
 import gated_delta_rule_112_b200 as gdn
 from gated_delta_rule_112_b200.inputs import Workload, make_chunk_inputs
-from tests.parity import TOL_BF16, TOL_F32, np64, rel_l2, to_dev
+from tests.parity import TOL_BF16, TOL_F32, assert_close, np64, oracle_chunk, rel_l2, to_dev
 
 SCRATCH_BYTES = 64 << 20
 
@@ -38,7 +38,8 @@ def _call(L, d, B, T, H, dk, dv, num_seqs, chunk, dtype, o, fs):
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
-    # Checked on the host before any CUDA call: B4 H16 T8192 needs far more than 64 MiB.
+    # Checked on the host before any launch (the size query reads the current
+    # device's SM count, nothing more): B4 H16 T8192 needs far more than 64 MiB.
     L = _lib()
     need = L.gdn_chunk_fwd_workspace_size(4, 8192, 16, 128, 128, 0, 64, gdn.BF16)
     assert need > SCRATCH_BYTES
@@ -79,3 +80,7 @@ def test_noalloc_matches_chunk_fwd_on_consecutive_calls(case):
         torch.cuda.synchronize()
         assert rel_l2(np64(o), np64(o_ref)) <= tol
         assert rel_l2(np64(fs), np64(fs_ref)) <= tol
+        # and directly against the fp64 oracle on the same inputs
+        ro, rfs = oracle_chunk(inp)
+        assert_close(f"o (call {rep})", np64(o), ro, tol)
+        assert_close(f"final_state (call {rep})", np64(fs), rfs, tol)
