@@ -23,8 +23,9 @@ oracle (the slow, obviously-correct program the GPU path is checked
 against) on a bounded sample of the same workload.
 
 ``--workload kda_b4h16t4096`` measures the channel-wise-gate variant instead
-(gdn_kda_chunk_fwd on the fp32 CUDA-core kernel, and gdn_kda_decode_step on
-the kda_decode workload); its roofline is the CUDA cores' fp32 FMA rate.
+(gdn_kda_chunk_fwd on the tensor-core kernels, and gdn_kda_decode_step on the
+kda_decode workload), against its own algorithmic bytes (g is one fp32 per
+channel).
 """
 from __future__ import annotations
 
@@ -50,8 +51,6 @@ BYTES_PER_TOKEN_HEAD_KDA = 3 * 128 * 2 + 128 * 2 + 128 * 4 + 4   # g is one fp32
 L2_FLUSH_BYTES = 256 << 20
 # Chunked-forward configurations measured beside the headline one.
 EXTRA_WORKLOADS = ("long64k", "varlen64")
-# fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 flop x 1965 MHz (max SM clock)
-FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def parse_args():
@@ -79,8 +78,7 @@ def parse_args():
 # The sources each measured kernel set is built from (under csrc/).
 KERNEL_SOURCES = {
     "chunk_fwd_step": ["chunk_map.cu", "chunk_tc.cu", "gdn_internal.cuh", "sm100_ptx.cuh"],
-    "kda_chunk_fwd_step": ["chunk_map.cu", "chunk_simt.cu", "gdn_internal.cuh",
-                           "sm100_ptx.cuh"],
+    "kda_chunk_fwd_step": ["chunk_map.cu", "chunk_tc.cu", "gdn_internal.cuh", "sm100_ptx.cuh"],
     "decode": ["decode.cu", "gdn_internal.cuh", "sm100_ptx.cuh"],
     "bwd_step": ["backward.cu", "bwd_internal.cuh", "gdn_internal.cuh", "sm100_ptx.cuh"],
 }
@@ -342,15 +340,13 @@ def main():
         alg_bytes = tokens * H * (BYTES_PER_TOKEN_HEAD_KDA if kda else BYTES_PER_TOKEN_HEAD) \
             + state_io
         flops = tokens * H * 2 * (3 * 64 * 128 + 2 * 64 * 128 + 3 * 128 * 128)
-        if kda:   # one CUDA-core kernel after the chunk map (prep/scan events coincide)
-            kernels = {"gdn_chunk_map_kernel": t_map, "gdn_chunk_simt_kernel": t_scan}
-        else:
-            kernels = {"gdn_chunk_map_kernel": t_map, "gdn_prep_kernel": t_prep,
-                       "gdn_scan_kernel": t_scan}
-        segs = 1 if kda else int(L.gdn_chunk_fwd_scan_segments(
+        kernels = {"gdn_chunk_map_kernel": t_map,
+                   ("gdn_kda_prep_kernel" if kda else "gdn_prep_kernel"): t_prep,
+                   "gdn_scan_kernel": t_scan}
+        segs = int(L.gdn_chunk_fwd_scan_segments(
             B, T, H, 128, 128, 0 if cu is None else nseq, 64, gdn.BF16,
             torch.cuda.get_device_properties(dev).multi_processor_count))
-        launches = 2 if kda else (3 if segs <= 1 else 5)
+        launches = 3 if segs <= 1 else 5
         return dict(inp=inp, kda=kda, fwd=fwd, t=t, s0=s0, cu=cu, o=o, ws=ws, B=B, T=T, H=H,
                     nseq=nseq, tokens=tokens, ms=ms, ms_local=ms_local, alg_bytes=alg_bytes,
                     flops=flops, kernels=kernels, clocks=clocks, launches=launches, segs=segs)
@@ -544,22 +540,13 @@ def main():
         cpu = {"value": tokens / dt / 1e6, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"the whole workload once (B{B} T{T} H{H}, {dt:.2f} s)"}
 
-    if kda:
-        tflops = flops / (ms_local * 1e-3) / 1e12
-        roof = {"bound": "alu", "achieved": tflops, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
-                "frac": tflops / FP32_ALU_TFLOPS, "traffic": traffic,
-                "kernel": "gdn_chunk_simt_kernel (channel-wise gate, fp32 CUDA cores)",
-                "algorithmic_bytes": alg_bytes, "flops": flops,
-                "hbm_frac": ach_gbs / pk["hbm"],
-                "peak_source": "fp32 FMA rate from unit counts: 148 SMs x 128 lanes x 2 flop "
-                               "x 1965 MHz"}
-    else:
-        roof = {"bound": "hbm", "achieved": ach_gbs, "peak": pk["hbm"], "unit": "GB/s",
-                "frac": ach_gbs / pk["hbm"], "traffic": traffic,
-                "kernel": "gdn_chunk_fwd step (chunk_map + prep + scan)",
-                "algorithmic_bytes": alg_bytes, "flops": flops,
-                "tensor_frac": flops / (ms_local * 1e-3) / (pk["bf16"] * 1e12),
-                "peak_source": pk["source"]}
+    roof = {"bound": "hbm", "achieved": ach_gbs, "peak": pk["hbm"], "unit": "GB/s",
+            "frac": ach_gbs / pk["hbm"], "traffic": traffic,
+            "kernel": ("gdn_kda_chunk_fwd step (chunk_map + kda prep + scan)" if kda
+                       else "gdn_chunk_fwd step (chunk_map + prep + scan)"),
+            "algorithmic_bytes": alg_bytes, "flops": flops,
+            "tensor_frac": flops / (ms_local * 1e-3) / (pk["bf16"] * 1e12),
+            "peak_source": pk["source"]}
     line = {
         "metric": METRIC_KDA if kda else METRIC, "value": value, "unit": UNIT,
         "n_gpus": world, "steps": K,
@@ -580,7 +567,7 @@ def main():
         "kernel_share": {k2: v2 / tot for k2, v2 in kernels.items()},
         "kernels_note": "per-kernel times from an untimed pass with events between the "
                         "launches (no launch overlap); ms_per_step is the timed region",
-        "gpu_launches": (2 if kda else 3) * K,
+        "gpu_launches": main_r["launches"] * K,
         "clocks": clocks,
         "e2e": e2e,
         "decode": decode,

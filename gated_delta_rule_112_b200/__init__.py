@@ -18,9 +18,12 @@ __all__ = ["chunk_fwd", "decode_step", "workspace_size", "chunk_path", "get_stat
            "lib", "GdnError", "BF16", "F32", "PATH_TCGEN05", "PATH_SIMT"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libgdn.so")
+# GDN_LIBRARY selects another build of the same library (e.g. the bounds-checked
+# libgdn_checked.so); the default is the in-tree libgdn.so.
+LIB_PATH = os.environ.get("GDN_LIBRARY") or os.path.join(_HERE, "libgdn.so")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOUT = range(6)
+(OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOUT,
+ ERR_DEVICE_BOUNDS) = range(7)
 BF16, F32 = 0, 1
 PATH_TCGEN05, PATH_SIMT = 1, 2
 
@@ -81,6 +84,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_get_status.restype = ci
         L.gdn_set_profile_events.argtypes = [vp, vp, vp, vp]
         L.gdn_set_profile_events.restype = ci
+        L.gdn_checked_build.argtypes = []
+        L.gdn_checked_build.restype = ci
         L.gdn_status_string.argtypes = [ci]
         L.gdn_status_string.restype = ctypes.c_char_p
         _lib = L

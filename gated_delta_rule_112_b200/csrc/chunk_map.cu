@@ -31,15 +31,17 @@ __global__ void __launch_bounds__(1024) gdn_chunk_map_kernel(
       ci.cidx = c;
       ci.row0 = n * T + c * chunk;
       ci.len = min(chunk, T - c * chunk);
-      table[idx] = ci;
+      if (GDN_IN_BOUNDS(ctrl, idx, max_chunks)) table[idx] = ci;
     }
-    for (int n = tid; n <= N; n += blockDim.x) seq_first[n] = n * cps;
+    for (int n = tid; n <= N; n += blockDim.x)
+      if (GDN_IN_BOUNDS(ctrl, n, N + 1)) seq_first[n] = n * cps;
     if (segs > 1) {
       // segment g of sequence n: chunks [n cps + g len, min(n cps + (g + 1) len, (n + 1) cps))
       const int len = (cps + segs - 1) / segs;
       for (int e = tid; e <= N * segs; e += blockDim.x) {
         const int n = e / segs, gi = e - n * segs;
-        seg_first[e] = (n >= N) ? N * cps : n * cps + min(gi * len, cps);
+        if (GDN_IN_BOUNDS(ctrl, e, N * segs + 1))
+          seg_first[e] = (n >= N) ? N * cps : n * cps + min(gi * len, cps);
       }
     }
     if (tid == 0) {
@@ -56,7 +58,8 @@ __global__ void __launch_bounds__(1024) gdn_chunk_map_kernel(
   const int n0 = min(N, tid * per), n1 = min(N, n0 + per);
   int32_t local = 0;
   for (int n = n0; n < n1; ++n) {
-    const int a = cu[n], b = cu[n + 1];
+    const int a = GDN_IN_BOUNDS(ctrl, n + 1, N + 1) ? cu[n] : 0;
+    const int b = GDN_IN_BOUNDS(ctrl, n + 1, N + 1) ? cu[n + 1] : 0;
     if ((n == 0 && a != 0) || b < a || (n == N - 1 && b != T)) bad = 1;
     const int len = b - a;
     if (len > 0) local += (len + chunk - 1) / chunk;
@@ -79,16 +82,17 @@ __global__ void __launch_bounds__(1024) gdn_chunk_map_kernel(
   }
   int32_t first = scan[tid] - local;
   for (int n = n0; n < n1; ++n) {
-    const int row0 = cu[n];
-    const int len = cu[n + 1] - row0;
-    seq_first[n] = first;
+    const bool ok = GDN_IN_BOUNDS(ctrl, n + 1, N + 1);
+    const int row0 = ok ? cu[n] : 0;
+    const int len = ok ? cu[n + 1] - row0 : 0;
+    if (ok) seq_first[n] = first;
     for (int c = 0; c * chunk < len; ++c) {
       ChunkInfo ci;
       ci.seq = n;
       ci.cidx = c;
       ci.row0 = row0 + c * chunk;
       ci.len = min(chunk, len - c * chunk);
-      table[first + c] = ci;
+      if (GDN_IN_BOUNDS(ctrl, first + c, max_chunks)) table[first + c] = ci;
     }
     if (len > 0) first += (len + chunk - 1) / chunk;
   }

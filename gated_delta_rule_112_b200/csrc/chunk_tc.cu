@@ -44,6 +44,13 @@ namespace gdn {
 
 #ifdef GDN_TRACE
 __device__ unsigned long long g_gdn_trace[2][kTraceSlots][kTraceEvents];
+__device__ unsigned long long g_gdn_cta_ns[1024][4];   // per scan CTA: start, XZ(0), last XZ, end
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
 #endif
 
 namespace {
@@ -59,25 +66,24 @@ constexpr int kLd = 68;                              // fp32 row stride of A and
 constexpr uint32_t kP_KQ = 0;                        // 2 blocks x [K rows 0-63 | Q rows 64-127] = 32 KB
 constexpr uint32_t kP_PST = kP_KQ + kTile64x64;      // P staging, over Q of block 0 (dead after G)
 constexpr uint32_t kP_WST = kP_KQ;                   // -W staging [64 c][128 d] (2 blocks), over K/Q
-constexpr uint32_t kP_KST = kP_KQ + kTile128x64;     // (D K)^T staging [128 d][64 s], over K/Q
-constexpr uint32_t kP_TT = kP_KST + kTile64x64;      // solve: T transposed, fp32 [48][36], over Q of block 1
+constexpr uint32_t kP_TT = kP_KQ + kTile128x64 + kTile64x64;   // solve: T transposed, fp32 [48][36], over Q of block 1
 constexpr uint32_t kP_AS = kP_KQ + 2 * kTile128x64;  // A, fp32 [64][68]; after the solve it
 constexpr uint32_t kP_TB = kP_AS;                    //   holds T diag(beta)       (bf16 64x64)
 constexpr uint32_t kP_TBG = kP_AS + kTile64x64;      //   and   T diag(beta gamma) (bf16 64x64)
-constexpr uint32_t kP_TS = kP_AS + 64 * kLd * 4;     // T, fp32 [64][68]; then diag(D) (bf16 64x64)
-constexpr uint32_t kP_DIAG = kP_TS;
+constexpr uint32_t kP_TS = kP_AS + 64 * kLd * 4;     // T, fp32 [64][68]; then the (D K)^T
+constexpr uint32_t kP_KST = kP_TS;                   //   staging [128 d][64 s] (bf16, 16 KB)
 constexpr int kLy = 36;                              // fp32 row stride of the solve scratch
 constexpr uint32_t kP_XS = kP_TS + 64 * kLd * 4;     // solve scratch, fp32 [32][36]
 static_assert(kLy % 32 == 4 && kLd % 32 == 4 && 48 * kLy * 4 <= kTile64x64,
               "solve strides and the transposed-T area");
-constexpr uint32_t kP_VEC = kP_XS + 32 * kLy * 4;    // Gamma, beta, gamma, Gamma log2(e): 4 x 64 fp32
-constexpr uint32_t kP_BAR = kP_VEC + 4 * 64 * 4;     // 2 mbarriers + tmem address
+constexpr uint32_t kP_VEC = kP_XS + 32 * kLy * 4;    // Gamma, beta, gamma, Gamma log2(e), D: 5 x 64 fp32
+constexpr uint32_t kP_BAR = kP_VEC + 5 * 64 * 4;     // 2 mbarriers + tmem address
 constexpr uint32_t kP_END = kP_BAR + 64;
 constexpr uint32_t kPrepSmem = kP_END + 1024;        // + alignment slack
 constexpr int kPrepThreads = 256;
 static_assert(2 * kTile64x64 <= 64 * kLd * 4, "T tiles must fit in the A area");
-static_assert(kP_AS % 1024 == 0 && kP_PST % 1024 == 0 && kP_KST % 1024 == 0 &&
-                  kP_DIAG % 1024 == 0,
+static_assert(kTile128x64 <= 64 * kLd * 4, "the (D K)^T staging must fit in the T area");
+static_assert(kP_AS % 1024 == 0 && kP_PST % 1024 == 0 && kP_KST % 1024 == 0,
               "swizzled tiles need 1024-byte alignment");
 
 // 2^x on the special-function unit (PTX ex2.approx, flush-to-zero).
@@ -102,24 +108,16 @@ __device__ __forceinline__ uint32_t frag_bt(const float *mt, int ld, int n0, int
   return smem_u32(mt + (n0 + (lane & 7)) * ld + k0 + 4 * (lane >> 3));
 }
 
-// d += a b for fp32 fragments on the tf32 tensor-core path, each operand split
-// into tf32 parts x = hi + lo (|lo| <= 2^-11 |x|, the rest <= 2^-22 |x|) and
-// the three products that matter: lo hi + hi lo + hi hi. The dropped lo lo
-// term and the tails keep each product term within about 2^-21 of fp32.
-__device__ __forceinline__ void mma_3xtf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                           uint32_t b1) {
-  uint32_t ah[4], al[4];
+// d += a b for fp32 fragments on the warp-level tf32 tensor-core path, each
+// operand rounded once to tf32 (10-bit mantissa, round to nearest). T is
+// rounded to bf16 (8-bit mantissa) before any product uses it, and the block
+// products' tf32 error stays about ten times below that rounding.
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  uint32_t ar[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    ah[i] = cvt_tf32(__uint_as_float(a[i]));
-    al[i] = cvt_tf32(__uint_as_float(a[i]) - __uint_as_float(ah[i]));
-  }
-  const uint32_t bh0 = cvt_tf32(__uint_as_float(b0)), bh1 = cvt_tf32(__uint_as_float(b1));
-  const uint32_t bl0 = cvt_tf32(__uint_as_float(b0) - __uint_as_float(bh0));
-  const uint32_t bl1 = cvt_tf32(__uint_as_float(b1) - __uint_as_float(bh1));
-  mma_tf32_m16n8k8(d, al, bh0, bh1);
-  mma_tf32_m16n8k8(d, ah, bl0, bl1);
-  mma_tf32_m16n8k8(d, ah, bh0, bh1);
+  for (int i = 0; i < 4; ++i) ar[i] = cvt_tf32(__uint_as_float(a[i]));
+  mma_tf32_m16n8k8(d, ar, cvt_tf32(__uint_as_float(b0)), cvt_tf32(__uint_as_float(b1)));
 }
 
 // T = (I + A)^-1 for the strictly lower-triangular 64 x 64 A (fp32 shared
@@ -136,7 +134,7 @@ __device__ __forceinline__ void mma_3xtf32(float (&d)[4], const uint32_t (&a)[4]
 //   step 2  T([2,3],[0,1]): Y = A(..) T([0,1],[0,1]), then -T([2,3],[2,3]) Y;
 //           warp = one 16 x 8 tile of each product, the two warps that share
 //           a column tile meet on a named barrier
-// The products are warp-level tensor-core tiles (m16n8k8, split tf32, fp32
+// The products are warp-level tensor-core tiles (m16n8k8, tf32, fp32
 // accumulation) whose operands are read with ldmatrix: A operands from the
 // row-major A and T, B operands from transposed copies (Tt, and Y stored
 // transposed in Xs), all with row strides = 4 (mod 32) words, so that an
@@ -187,7 +185,7 @@ __device__ void solve_unit_lower_64(const float *__restrict__ As, float *__restr
       uint32_t a[4], bb[2];
       ldsm_x4(frag_a(As, kLd, i, j + k0, lane), a);
       ldsm_x2(frag_bt(tjt, kLy, n0, k0, lane), bb);
-      mma_3xtf32(c, a, bb[0], bb[1]);
+      mma_tf32(c, a, bb[0], bb[1]);
     }
     const int n = n0 + 2 * t;
     yt[n * kLy + g] = c[0];
@@ -202,7 +200,7 @@ __device__ void solve_unit_lower_64(const float *__restrict__ As, float *__restr
     for (int kk = 0; kk < 2; ++kk) {
       uint32_t a[4];
       ldsm_x4(frag_a(Ts, kLd, i, i + 8 * kk, lane), a);
-      mma_3xtf32(d, a, bb[2 * kk], bb[2 * kk + 1]);
+      mma_tf32(d, a, bb[2 * kk], bb[2 * kk + 1]);
     }
     *reinterpret_cast<float2 *>(Ts + (i + g) * kLd + j + n) = make_float2(-d[0], -d[1]);
     *reinterpret_cast<float2 *>(Ts + (i + g + 8) * kLd + j + n) = make_float2(-d[2], -d[3]);
@@ -222,7 +220,7 @@ __device__ void solve_unit_lower_64(const float *__restrict__ As, float *__restr
       uint32_t a[4], bb[2];
       ldsm_x4(frag_a(As, kLd, 32 + m0, k0, lane), a);
       ldsm_x2(frag_bt(Tt, kLy, n0, k0, lane), bb);
-      mma_3xtf32(c, a, bb[0], bb[1]);
+      mma_tf32(c, a, bb[0], bb[1]);
     }
     const int n = n0 + 2 * t;
     Xs[n * kLy + m0 + g] = c[0];
@@ -239,7 +237,7 @@ __device__ void solve_unit_lower_64(const float *__restrict__ As, float *__restr
       for (int kk = 0; kk < 2; ++kk) {
         uint32_t a[4];
         ldsm_x4(frag_a(Ts, kLd, 32 + m0, 32 + k0 + 8 * kk, lane), a);
-        mma_3xtf32(d, a, bb[2 * kk], bb[2 * kk + 1]);
+        mma_tf32(d, a, bb[2 * kk], bb[2 * kk + 1]);
       }
     }
     *reinterpret_cast<float2 *>(Ts + (32 + m0 + g) * kLd + n) = make_float2(-d[0], -d[1]);
@@ -262,7 +260,10 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
     const __grid_constant__ CUtensorMap tm_tb, const __grid_constant__ CUtensorMap tm_pm,
     const float *__restrict__ g,
     const float *__restrict__ beta, float *__restrict__ gam_out, int H,
-    uint32_t *__restrict__ ctrl, const ChunkInfo *__restrict__ table) {
+    uint32_t *__restrict__ ctrl, const ChunkInfo *__restrict__ table, long long rows,
+    int max_chunks) {
+  (void)rows;
+  (void)max_chunks;   // extents of the bounds checks (GDN_CHECKS builds)
   extern __shared__ uint8_t smem_raw[];
   // Pointer arithmetic (not integer casts) keeps the shared address space.
   uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -278,6 +279,7 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
   float *Bt = Gm + 64;
   float *Ga = Bt + 64;
   float *Gl = Ga + 64;                     // Gamma log2(e)
+  float *Dv = Gl + 64;                     // D_s = exp(Gamma_last - Gamma_s)
   uint64_t *bar_load = reinterpret_cast<uint64_t *>(sm + kP_BAR);
   uint64_t *bar_mma = bar_load + 1;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_load + 2);
@@ -312,17 +314,19 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
   auto fetch_gb = [&](int u) {
     if (tid < kC && u < nunits) {
       const int cu = u / H, hu = u - cu * H;
-      const ChunkInfo cf = table[cu];
-      const bool ok = tid < cf.len;
-      g_reg = ok ? g[size_t(cf.row0 + tid) * H + hu] : 0.f;
-      b_reg = ok ? beta[size_t(cf.row0 + tid) * H + hu] : 0.f;
+      const ChunkInfo cf = GDN_IN_BOUNDS(ctrl, cu, max_chunks) ? table[cu] : ChunkInfo{0, 0, 0, 0};
+      const long long idx = (long long)(cf.row0 + tid) * H + hu;
+      const bool ok = tid < cf.len && GDN_IN_BOUNDS(ctrl, idx, rows * H);
+      g_reg = ok ? g[idx] : 0.f;
+      b_reg = ok ? beta[idx] : 0.f;
     }
   };
   fetch_gb(blockIdx.x);
   int it = 0;
   for (int unit = blockIdx.x; unit < nunits; unit += gridDim.x, ++it) {
   const int chunk = unit / H, h = unit - chunk * H;
-  const ChunkInfo ci = table[chunk];
+  const ChunkInfo ci =
+      GDN_IN_BOUNDS(ctrl, chunk, max_chunks) ? table[chunk] : ChunkInfo{0, 0, 0, 0};
   const int L = ci.len;
   const bool tr = (h == 0 && tid == 0);   // traced thread (GDN_TRACE builds only)
   (void)tr;
@@ -341,7 +345,7 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
     const int nu = unit + int(gridDim.x);
     if (nu < nunits) {
       const int cn = nu / H, hn = nu - cn * H;
-      const int rn = table[cn].row0;
+      const int rn = GDN_IN_BOUNDS(ctrl, cn, max_chunks) ? table[cn].row0 : 0;
       tma_prefetch_l2_3d(&tm_k, 0, hn, rn);
       tma_prefetch_l2_3d(&tm_k, 64, hn, rn);
       tma_prefetch_l2_3d(&tm_q, 0, hn, rn);
@@ -399,9 +403,13 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
     tc_commit(bar_mma);
   }
   if (tid < kC) {
-    Ga[tid] = __expf(Gm[tid]);
-    gam_out[size_t(unit) * 128 + tid] = expf(Gm[tid]);                   // gamma_c
-    gam_out[size_t(unit) * 128 + 64 + tid] = expf(Gm[kC - 1] - Gm[tid]);  // D_s
+    const float ga = expf(Gm[tid]), dv = expf(Gm[kC - 1] - Gm[tid]);
+    Ga[tid] = ga;
+    Dv[tid] = dv;
+    if (GDN_IN_BOUNDS(ctrl, (long long)unit * 128 + 64 + tid, (long long)max_chunks * H * 128)) {
+      gam_out[size_t(unit) * 128 + tid] = ga;        // gamma_c
+      gam_out[size_t(unit) * 128 + 64 + tid] = dv;   // D_s
+    }
   }
   mbar_wait(bar_mma, 0, ctrl, &abort_flag);
   GDN_TRACE_POINT(tr && chunk < 64, 1, chunk, 2);
@@ -509,23 +517,6 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
                      pack_bf16x2(xg[4], xg[5]), pack_bf16x2(xg[6], xg[7]));
     }
   }
-  __syncthreads();
-  // T is dead: its area now holds diag(D), D_s = exp(Gamma_last - Gamma_s), as a
-  // bf16 K-major tile, the B operand that turns K^T into (D K)^T.
-  {
-    const int r = tid >> 2, q4 = tid & 3;
-    const float dr = expf(Gm[kC - 1] - Gm[r]);
-#pragma unroll
-    for (int cc = 0; cc < 2; ++cc) {
-      const int ch = q4 * 2 + cc;
-      float f[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) f[e] = (ch * 8 + e == r) ? dr : 0.f;
-      *reinterpret_cast<uint4 *>(sm + kP_DIAG + sw128_offset(r, ch)) =
-          make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
-                     pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
-    }
-  }
   fence_proxy_async_smem();
   __syncthreads();
   GDN_TRACE_POINT(tr && chunk < 64, 1, chunk, 5);
@@ -533,21 +524,42 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
     tma_store_2d(&tm_tb, sm + kP_TB, 0, unit * kC);
     tma_store_commit();
     tc_fence_after();
-    // W^T    = K^T (T diag(beta gamma))^T : M = 128 (d_k), N = 64, K = 64 -> cols [64, 128)
-    // (DK)^T = K^T diag(D)                : M = 128 (d_k), N = 64, K = 64 -> cols [0, 64)
+    // W^T = K^T (T diag(beta gamma))^T : M = 128 (d_k), N = 64, K = 64 -> cols [64, 128)
     const uint32_t idesc = make_idesc_bf16(128, 64, 1, 0);
     const uint64_t dkt = make_sdesc(smem_u32(sm + kP_KQ), kTile128x64, 1024);
     const uint64_t dtbg = make_sdesc(smem_u32(sm + kP_TBG), 16, 1024);
-    const uint64_t ddg = make_sdesc(smem_u32(sm + kP_DIAG), 16, 1024);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
       tc_mma_bf16(tmem + 64, dkt + uint64_t(kk * 2048 >> 4), dtbg + uint64_t(kk * 32 >> 4), idesc,
                   kk > 0);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      tc_mma_bf16(tmem, dkt + uint64_t(kk * 2048 >> 4), ddg + uint64_t(kk * 32 >> 4), idesc,
-                  kk > 0);
     tc_commit(bar_mma);
+  }
+  // While the tensor core computes W^T (both read K), (D K)^T goes straight
+  // from the K tile into its staging tile (the dead T area): 8 x 8 blocks are
+  // read transposed with ldmatrix (thread t gets tokens 2(t%4), 2(t%4)+1 of
+  // d_k row t/4), scaled by (D_s, D_s+1) in bf16 with one rounding -- the
+  // bits the MMA against a bf16 diag(D) tile gave -- and stored with
+  // stmatrix. Warp w owns d_k rows [16 w, 16 w + 16).
+  if (!abort_flag) {
+    const int mj = lane & 7, mm = lane >> 3;
+    const int sp = 2 * (lane & 3);                  // first token of this thread's pair
+    const uint32_t kq = smem_u32(sm + kP_KQ), kst = smem_u32(sm + kP_KST);
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      // matrix mm: d_k block jb = 2 warp + (mm & 1), token block sb = 2 it + (mm >> 1)
+      const int jb = 2 * warp + (mm & 1), sb = 2 * it + (mm >> 1);
+      const int srow = 8 * sb + mj;                 // K row (token) this thread addresses
+      uint32_t x[4];
+      ldsm_x4_trans(kq + (jb >> 3) * kTile128x64 + sw128_offset(srow, jb & 7), x);
+      uint32_t y[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int s0 = 16 * it + 8 * (m >> 1) + sp;
+        y[m] = mul_bf16x2(x[m], pack_bf16x2(Dv[s0], Dv[s0 + 1]));
+      }
+      const int jrow = 8 * jb + mj;                 // (D K)^T row this thread addresses
+      stmatrix_x4(kst + sw128_offset(jrow, sb), y[0], y[1], y[2], y[3]);
+    }
   }
   mbar_wait(bar_mma, 1, ctrl, &abort_flag);
   GDN_TRACE_POINT(tr && chunk < 64, 1, chunk, 6);
@@ -555,43 +567,26 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
   tc_fence_after();
   __syncthreads();
   if (!abort_flag) {
-    if (hc == 0) {
-      // -W, K-major [64 c][128 d]: read W^T (lanes = d, columns = c) as
-      // mma-accumulator fragments and store them transposed with stmatrix.
-      const int q = warp & 3, mj = lane & 7, mm = lane >> 3;
-      const uint32_t wst = smem_u32(sm + kP_WST);
+    // -W, K-major [64 c][128 d]: read W^T (lanes = d, columns = c) as
+    // mma-accumulator fragments and store them transposed with stmatrix.
+    // Warp w: lane quarter w % 4, token columns [32 (w / 4), 32 (w / 4) + 32).
+    const int q = warp & 3, mj = lane & 7, mm = lane >> 3;
+    const uint32_t wst = smem_u32(sm + kP_WST);
 #pragma unroll
-      for (int lb = 0; lb < 32; lb += 16) {
+    for (int lb = 0; lb < 32; lb += 16) {
 #pragma unroll
-        for (int cb = 0; cb < 64; cb += 16) {
-          uint32_t w8[8];
-          tmem_ld16x256_x2(lane_base + (uint32_t(lb) << 16) + 64 + cb, w8);
-          tmem_ld_wait();
-          uint32_t w[4];
+      for (int cb = 32 * hc; cb < 32 * hc + 32; cb += 16) {
+        uint32_t w8[8];
+        tmem_ld16x256_x2(lane_base + (uint32_t(lb) << 16) + 64 + cb, w8);
+        tmem_ld_wait();
+        uint32_t w[4];
 #pragma unroll
-          for (int mq = 0; mq < 4; ++mq)
-            w[mq] = pack_bf16x2(-__uint_as_float(w8[2 * mq]), -__uint_as_float(w8[2 * mq + 1]));
-          const int d0 = q * 32 + lb + 8 * (mm & 1);   // first d index of my matrix
-          const int crow = cb + 8 * (mm >> 1) + mj;     // chunk row this thread addresses
-          stmatrix_x4_trans(wst + (d0 >> 6) * kTile64x64 + sw128_offset(crow, (d0 & 63) >> 3),
-                            w[0], w[1], w[2], w[3]);
-        }
-      }
-    } else {
-      // (D K)^T row m (= d) -> [128 d][64 s] staging.
-      uint32_t r0[32], r1[32];
-      tmem_ld32(lane_base, r0);
-      tmem_ld32(lane_base + 32, r1);
-      tmem_ld_wait();
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        const uint32_t *src = ch < 4 ? r0 : r1;
-        const int b = (ch & 3) * 8;
-        *reinterpret_cast<uint4 *>(sm + kP_KST + sw128_offset(m, ch)) = make_uint4(
-            pack_bf16x2(__uint_as_float(src[b + 0]), __uint_as_float(src[b + 1])),
-            pack_bf16x2(__uint_as_float(src[b + 2]), __uint_as_float(src[b + 3])),
-            pack_bf16x2(__uint_as_float(src[b + 4]), __uint_as_float(src[b + 5])),
-            pack_bf16x2(__uint_as_float(src[b + 6]), __uint_as_float(src[b + 7])));
+        for (int mq = 0; mq < 4; ++mq)
+          w[mq] = pack_bf16x2(-__uint_as_float(w8[2 * mq]), -__uint_as_float(w8[2 * mq + 1]));
+        const int d0 = q * 32 + lb + 8 * (mm & 1);   // first d index of my matrix
+        const int crow = cb + 8 * (mm >> 1) + mj;     // chunk row this thread addresses
+        stmatrix_x4_trans(wst + (d0 >> 6) * kTile64x64 + sw128_offset(crow, (d0 & 63) >> 3),
+                          w[0], w[1], w[2], w[3]);
       }
     }
   }
@@ -617,35 +612,445 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
   }
 }
 
+// ============================================================ channel-wise gate: prep
+// The channel-wise (Kimi Delta Attention) gate of dmarx anthology LIT-137,
+// "Standing in the anthology", and SOTA-135, "Sequence": alpha_t has one value
+// per d_k channel, S_t = S_{t-1} diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t
+// v_t k_t^T. Per chunk, with Gamma_rj = sum_{s <= r} log alpha_sj:
+//   A_rs = beta_r sum_j k_rj k_sj e^(Gamma_rj - Gamma_sj)   (s < r)
+//   P_rs = sum_j q_rj k_sj e^(Gamma_rj - Gamma_sj)          (s <= r)
+//   W = T diag(beta) (K .* e^Gamma),  U = T diag(beta) V,  T = (I + A)^-1
+//   O = (Q .* e^Gamma) S^T + P V_new
+//   S <- S diag(e^Gamma_last) + V_new^T (K .* e^(Gamma_last - Gamma))
+// The decay sits inside the dot products. For the 16-row block R of A and P
+// the factor splits through the block's first row b = 16 R:
+//   e^(Gamma_r - Gamma_s) = e^(Gamma_r - Gamma_b) e^(Gamma_b - Gamma_s),
+// so block row R is one product of a left operand (K or Q rows of the block
+// scaled by e^(Gamma_r - Gamma_b) <= 1) with a right operand (K rows 0 ..
+// 16 R + 15 scaled by e^(Gamma_b - Gamma_s): <= 1 below the block, within
+// e^(15 max |log alpha|) inside it), on the warp-level tensor-core path
+// (mma.sync m16n8k16, bf16 operands, fp32 accumulation). Everything after A
+// is the scalar gate's prep: the same blocked solve, T diag(beta) and W on
+// tcgen05. The state scan then consumes the same operand tiles, with
+// Q .* e^Gamma in place of Q (gamma = 1 in the decay record) and the
+// per-channel state decay e^Gamma_last.
+constexpr uint32_t kK_KQ = 0;                          // K, Q (bf16, 128-byte swizzle) as in prep
+constexpr uint32_t kK_GM = kK_KQ + 2 * kTile128x64;    // Gamma fp32 [64][128]
+constexpr uint32_t kK_LK = kK_GM + 64 * 128 * 4;       // left operands bf16 [64][128] (256-B rows)
+constexpr uint32_t kK_LQ = kK_LK + 64 * 256;
+constexpr uint32_t kK_RR = kK_LQ + 64 * 256;           // right operand of block row R
+constexpr uint32_t kK_DK = kK_RR + 64 * 256;           // (D K)^T staging [128][64]
+constexpr uint32_t kK_AS = kK_DK + kTile128x64;        // A fp32 [64][68]
+constexpr uint32_t kK_TS = kK_AS + 64 * kLd * 4;       // T fp32 [64][68]
+constexpr uint32_t kK_XS = kK_TS + 64 * kLd * 4;       // solve scratch fp32 [32][36]
+constexpr uint32_t kK_TT = kK_XS + 32 * kLy * 4;       // solve: T transposed fp32 [48][36]
+constexpr uint32_t kK_TB = (kK_TT + 48 * kLy * 4 + 1023) / 1024 * 1024;   // T diag(beta) bf16
+constexpr uint32_t kK_PST = kK_TB + kTile64x64;        // P staging bf16 [64][64]
+constexpr uint32_t kK_VEC = kK_PST + kTile64x64;       // beta[64], e^Gamma_last[128]
+constexpr uint32_t kK_BAR = kK_VEC + 192 * 4;
+constexpr uint32_t kKdaPrepSmem = kK_BAR + 64;         // the dynamic window starts 1024-aligned (checked)
+constexpr int kKdaPrepThreads = 256;
+static_assert(kK_LK % 1024 == 0 && kK_RR % 1024 == 0 && kK_DK % 1024 == 0 &&
+                  kK_TB % 1024 == 0 && kK_PST % 1024 == 0 && kKdaPrepSmem <= 232448,
+              "channel-wise prep layout");
+
+// Byte offset of 16-byte chunk c (0..15) of row r in a [rows][128 bf16] tile
+// with 256-byte rows, XOR-swizzled so that 8 consecutive rows at the same
+// chunk hit distinct banks (ldmatrix reads 8 rows x 16 bytes).
+__device__ __forceinline__ uint32_t sw256(uint32_t r, uint32_t c) {
+  return r * 256u + ((c ^ (r & 7u)) << 4);
+}
+
+// d += a b, m16n8k16, bf16 operands, fp32 accumulators (fragment layouts as
+// for m16n8k8 with each register holding two consecutive k).
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Eight bf16 (one 16-byte chunk) times eight fp32 factors, rounded once.
+__device__ __forceinline__ uint4 scale8(uint4 x, const float (&f)[8]) {
+  const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xffff0000u);
+    o[i] = pack_bf16x2(lo * f[2 * i], hi * f[2 * i + 1]);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__global__ void __launch_bounds__(kKdaPrepThreads, 1) gdn_kda_prep_kernel(
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+    const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_kt,
+    const __grid_constant__ CUtensorMap tm_tb, const __grid_constant__ CUtensorMap tm_pm,
+    const __grid_constant__ CUtensorMap tm_qt, const float *__restrict__ g,
+    const float *__restrict__ beta, float *__restrict__ gam_out, int H,
+    uint32_t *__restrict__ ctrl, const ChunkInfo *__restrict__ table, long long rows,
+    int max_chunks) {
+  (void)rows;
+  (void)max_chunks;   // extents of the bounds checks (GDN_CHECKS builds)
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *sm = smem_raw;
+  __shared__ int abort_flag;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  grid_launch_dependents();
+  if (smem_u32(sm) & 1023) {
+    grid_dependency_wait();
+    if (tid == 0) atomicOr(ctrl, kErrLayout);
+    return;
+  }
+  float *Gm = reinterpret_cast<float *>(sm + kK_GM);
+  float *As = reinterpret_cast<float *>(sm + kK_AS);
+  float *Ts = reinterpret_cast<float *>(sm + kK_TS);
+  float *Xs = reinterpret_cast<float *>(sm + kK_XS);
+  float *Tt = reinterpret_cast<float *>(sm + kK_TT);
+  float *Bt = reinterpret_cast<float *>(sm + kK_VEC);   // beta [64]
+  float *El = Bt + 64;                                  // e^Gamma_last [128]
+  uint64_t *bar_load = reinterpret_cast<uint64_t *>(sm + kK_BAR);
+  uint64_t *bar_mma = bar_load + 1;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_load + 2);
+  constexpr float kLog2e = 1.4426950408889634f;
+  if (tid == 0) {
+    abort_flag = 0;
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    mbar_init(bar_load, 1);
+    mbar_init(bar_mma, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 64);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  grid_dependency_wait();
+  const int nunits = (ctrl[0] & kErrBadSeqlens) ? 0 : int(ctrl[1]) * H;
+  int it = 0;
+  for (int unit = blockIdx.x; unit < nunits; unit += gridDim.x, ++it) {
+    const int chunk = unit / H, h = unit - chunk * H;
+    const ChunkInfo ci =
+        GDN_IN_BOUNDS(ctrl, chunk, max_chunks) ? table[chunk] : ChunkInfo{0, 0, 0, 0};
+    const int L = ci.len;
+    if (tid == 0) {
+      // The previous unit's stores must have read the areas reused below.
+      tma_store_wait_read();
+      if (!abort_flag) {
+        mbar_arrive_expect_tx(bar_load, 2 * kTile128x64);
+        tma_load_3d(sm + kK_KQ, &tm_k, bar_load, 0, h, ci.row0);
+        tma_load_3d(sm + kK_KQ + kTile64x64, &tm_q, bar_load, 0, h, ci.row0);
+        tma_load_3d(sm + kK_KQ + kTile128x64, &tm_k, bar_load, 64, h, ci.row0);
+        tma_load_3d(sm + kK_KQ + kTile128x64 + kTile64x64, &tm_q, bar_load, 64, h, ci.row0);
+      }
+    }
+    __syncthreads();   // every thread is past the previous unit's reads of Gm and PST
+    // g of the chunk (rows past the sequence end read as 0) and beta.
+    for (int e = tid; e < 64 * 32; e += kKdaPrepThreads) {
+      const int r = e >> 5, c4 = e & 31;
+      const long long idx = ((long long)(ci.row0 + r) * H + h) * 128 + 4 * c4;
+      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r < L && GDN_IN_BOUNDS(ctrl, idx + 3, rows * H * 128))
+        x = *reinterpret_cast<const float4 *>(g + idx);
+      *reinterpret_cast<float4 *>(Gm + r * 128 + 4 * c4) = x;
+    }
+    if (tid < 64) {
+      const long long idx = (long long)(ci.row0 + tid) * H + h;
+      Bt[tid] = (tid < L && GDN_IN_BOUNDS(ctrl, idx, rows * H)) ? beta[idx] : 0.f;
+    }
+    // P staging starts at zero: blocks above the diagonal are never written.
+    for (int e = tid; e < kTile64x64 / 16; e += kKdaPrepThreads)
+      *reinterpret_cast<uint4 *>(sm + kK_PST + 16 * e) = make_uint4(0, 0, 0, 0);
+    __syncthreads();
+    // Gamma: inclusive cumsum over the tokens, one thread per channel.
+    if (tid < 128) {
+      float acc = 0.f;
+#pragma unroll 8
+      for (int r = 0; r < 64; ++r) {
+        acc += Gm[r * 128 + tid];
+        Gm[r * 128 + tid] = acc;
+      }
+      El[tid] = expf(acc);
+    }
+    const bool loaded = mbar_wait(bar_load, it & 1, ctrl, &abort_flag);
+    if (loaded && L < kC) {
+      // Rows past the sequence end act as k = q = 0.
+      for (int e = tid; e < (kC - L) * 8; e += kKdaPrepThreads) {
+        const int r = L + e / 8, ch = e % 8;
+        const uint4 z = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4 *>(sm + kK_KQ + r * 128 + ch * 16) = z;
+        *reinterpret_cast<uint4 *>(sm + kK_KQ + kTile64x64 + r * 128 + ch * 16) = z;
+        *reinterpret_cast<uint4 *>(sm + kK_KQ + kTile128x64 + r * 128 + ch * 16) = z;
+        *reinterpret_cast<uint4 *>(sm + kK_KQ + kTile128x64 + kTile64x64 + r * 128 + ch * 16) = z;
+      }
+    }
+    __syncthreads();
+    // Left operands K and Q .* e^(Gamma_r - Gamma_b(r)) and Q .* e^Gamma (in
+    // place of Q). Pair (row r, 16-byte chunk c) = channels 8 c .. 8 c + 7.
+    for (int e = tid; e < 64 * 16; e += kKdaPrepThreads) {
+      const int r = e >> 4, c = e & 15, b = r & ~15;
+      const uint32_t kq = kK_KQ + (c >> 3) * kTile128x64 + sw128_offset(r, c & 7);
+      const float *gr = Gm + r * 128 + 8 * c, *gb = Gm + b * 128 + 8 * c;
+      const float4 r0 = lds4(gr), r1 = lds4(gr + 4), b0 = lds4(gb), b1 = lds4(gb + 4);
+      const float gv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      float f1[8], fg[8];
+#pragma unroll
+      for (int x = 0; x < 8; ++x) {
+        f1[x] = ex2_approx((gv[x] - bv[x]) * kLog2e);
+        fg[x] = ex2_approx(gv[x] * kLog2e);
+      }
+      const uint4 kx = *reinterpret_cast<const uint4 *>(sm + kq);
+      const uint4 qx = *reinterpret_cast<const uint4 *>(sm + kq + kTile64x64);
+      *reinterpret_cast<uint4 *>(sm + kK_LK + sw256(r, c)) = scale8(kx, f1);
+      *reinterpret_cast<uint4 *>(sm + kK_LQ + sw256(r, c)) = scale8(qx, f1);
+      *reinterpret_cast<uint4 *>(sm + kq + kTile64x64) = scale8(qx, fg);
+    }
+    // (D K)^T with D_sj = e^(Gamma_last,j - Gamma_sj), straight from the K tile
+    // (ldmatrix.trans gives thread t tokens s, s + 1 of d_k row t / 4); warp w
+    // owns d_k rows [16 w, 16 w + 16).
+    {
+      const int mj = lane & 7, mm = lane >> 3, sp = 2 * (lane & 3), jq = lane >> 2;
+      const uint32_t kq = smem_u32(sm + kK_KQ), kst = smem_u32(sm + kK_DK);
+#pragma unroll
+      for (int it2 = 0; it2 < 4; ++it2) {
+        const int jb = 2 * warp + (mm & 1), sb = 2 * it2 + (mm >> 1);
+        uint32_t x[4];
+        ldsm_x4_trans(kq + (jb >> 3) * kTile128x64 + sw128_offset(8 * sb + mj, jb & 7), x);
+        uint32_t y[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int j = 8 * (2 * warp + (m & 1)) + jq, s0 = 8 * (2 * it2 + (m >> 1)) + sp;
+          const float gl = Gm[63 * 128 + j];
+          const float d0 = ex2_approx((gl - Gm[s0 * 128 + j]) * kLog2e);
+          const float d1 = ex2_approx((gl - Gm[(s0 + 1) * 128 + j]) * kLog2e);
+          y[m] = pack_bf16x2(__uint_as_float(x[m] << 16) * d0,
+                             __uint_as_float(x[m] & 0xffff0000u) * d1);
+        }
+        stmatrix_x4(kst + sw128_offset(8 * jb + mj, sb), y[0], y[1], y[2], y[3]);
+      }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0 && !abort_flag) {
+      tma_store_2d(&tm_qt, sm + kK_KQ + kTile64x64, 0, unit * kC);
+      tma_store_2d(&tm_qt, sm + kK_KQ + kTile128x64 + kTile64x64, 64, unit * kC);
+      tma_store_2d(&tm_kt, sm + kK_DK, 0, unit * kD);
+      tma_store_commit();
+    }
+    // A and P, one 16-row block row at a time.
+    for (int R = 0; R < 4; ++R) {
+      const int nrow = 16 * R + 16;
+      // right operand: K rows s < 16 R + 16 scaled by e^(Gamma_16R - Gamma_s)
+      for (int e = tid; e < nrow * 16; e += kKdaPrepThreads) {
+        const int s = e >> 4, c = e & 15;
+        const uint32_t kq = kK_KQ + (c >> 3) * kTile128x64 + sw128_offset(s, c & 7);
+        const float *gs = Gm + s * 128 + 8 * c, *gb = Gm + 16 * R * 128 + 8 * c;
+        const float4 s0 = lds4(gs), s1 = lds4(gs + 4), b0 = lds4(gb), b1 = lds4(gb + 4);
+        const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+        const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        float f[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) f[x] = ex2_approx((bv[x] - sv[x]) * kLog2e);
+        *reinterpret_cast<uint4 *>(sm + kK_RR + sw256(s, c)) =
+            scale8(*reinterpret_cast<const uint4 *>(sm + kq), f);
+      }
+      __syncthreads();
+      // jobs: (n-tile of 8 columns, A or P); warp w takes jobs w and w + 8
+      const int njobs = 4 * (R + 1);
+      for (int job = warp; job < njobs; job += 8) {
+        const int nt = job >> 1, isP = job & 1;
+        const uint32_t left = smem_u32(sm + (isP ? kK_LQ : kK_LK));
+        const uint32_t right = smem_u32(sm + kK_RR);
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        const int ar = 16 * R + (lane & 7) + 8 * ((lane >> 3) & 1);   // A fragment row
+        const int brow = 8 * nt + (lane & 7);                          // B fragment row (= column s)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          uint32_t a[4], bb[2];
+          ldsm_x4(left + sw256(ar, 2 * kk + (lane >> 4)), a);
+          ldsm_x2(right + sw256(brow, 2 * kk + ((lane >> 3) & 1)), bb);
+          mma_bf16_16816(acc, a, bb[0], bb[1]);
+        }
+        const int gq = lane >> 2, tq = lane & 3;
+        const int r0 = 16 * R + gq, s0 = 8 * nt + 2 * tq;
+        if (!isP) {
+          const float b0 = Bt[r0], b1 = Bt[r0 + 8];
+          *reinterpret_cast<float2 *>(As + r0 * kLd + s0) = make_float2(b0 * acc[0], b0 * acc[1]);
+          *reinterpret_cast<float2 *>(As + (r0 + 8) * kLd + s0) =
+              make_float2(b1 * acc[2], b1 * acc[3]);
+        } else {
+          const uint32_t p0 = pack_bf16x2(s0 <= r0 ? acc[0] : 0.f, s0 + 1 <= r0 ? acc[1] : 0.f);
+          const uint32_t p1 =
+              pack_bf16x2(s0 <= r0 + 8 ? acc[2] : 0.f, s0 + 1 <= r0 + 8 ? acc[3] : 0.f);
+          *reinterpret_cast<uint32_t *>(sm + kK_PST + sw128_offset(r0, s0 >> 3) + 2 * (s0 & 7)) = p0;
+          *reinterpret_cast<uint32_t *>(sm + kK_PST + sw128_offset(r0 + 8, s0 >> 3) +
+                                        2 * (s0 & 7)) = p1;
+        }
+      }
+      fence_proxy_async_smem();   // P staging rows -> the TMA store below
+      __syncthreads();
+    }
+    // P is complete; K .* e^Gamma replaces K (the W operand).
+    if (tid == 0 && !abort_flag) {
+      tma_store_2d(&tm_pm, sm + kK_PST, 0, unit * kC);
+      tma_store_commit();
+    }
+    for (int e = tid; e < 64 * 16; e += kKdaPrepThreads) {
+      const int r = e >> 4, c = e & 15;
+      const uint32_t kq = kK_KQ + (c >> 3) * kTile128x64 + sw128_offset(r, c & 7);
+      const float *gr = Gm + r * 128 + 8 * c;
+      const float4 r0 = lds4(gr), r1 = lds4(gr + 4);
+      const float f[8] = {ex2_approx(r0.x * kLog2e), ex2_approx(r0.y * kLog2e),
+                          ex2_approx(r0.z * kLog2e), ex2_approx(r0.w * kLog2e),
+                          ex2_approx(r1.x * kLog2e), ex2_approx(r1.y * kLog2e),
+                          ex2_approx(r1.z * kLog2e), ex2_approx(r1.w * kLog2e)};
+      *reinterpret_cast<uint4 *>(sm + kq) = scale8(*reinterpret_cast<const uint4 *>(sm + kq), f);
+    }
+    solve_unit_lower_64(As, Ts, Tt, Xs, tid);   // ends with __syncthreads
+    // T diag(beta), bf16 K-major (T is lower triangular; its upper blocks are
+    // unwritten, so s > r reads as zero).
+    {
+      const int r = tid >> 2, q4 = tid & 3;
+      float fb[16];
+      if (16 * q4 <= r) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int s0 = 16 * q4 + 4 * i;
+          const float4 t4 = lds4(Ts + r * kLd + s0);
+          const float4 bt = lds4(Bt + s0);
+          const float tv[4] = {t4.x, t4.y, t4.z, t4.w}, bv[4] = {bt.x, bt.y, bt.z, bt.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) fb[4 * i + e] = (s0 + e <= r) ? tv[e] * bv[e] : 0.f;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) fb[e] = 0.f;
+      }
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        const int ch = q4 * 2 + cc;
+        const float *xb = fb + 8 * cc;
+        *reinterpret_cast<uint4 *>(sm + kK_TB + sw128_offset(r, ch)) =
+            make_uint4(pack_bf16x2(xb[0], xb[1]), pack_bf16x2(xb[2], xb[3]),
+                       pack_bf16x2(xb[4], xb[5]), pack_bf16x2(xb[6], xb[7]));
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (!abort_flag && tid == 0) {
+      tma_store_2d(&tm_tb, sm + kK_TB, 0, unit * kC);
+      tma_store_commit();
+      tc_fence_after();
+      // W^T = (K .* e^Gamma)^T (T diag(beta))^T : M = 128 (d_k), N = 64, K = 64
+      const uint32_t idesc = make_idesc_bf16(128, 64, 1, 0);
+      const uint64_t dkt = make_sdesc(smem_u32(sm + kK_KQ), kTile128x64, 1024);
+      const uint64_t dtb = make_sdesc(smem_u32(sm + kK_TB), 16, 1024);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        tc_mma_bf16(tmem, dkt + uint64_t(kk * 2048 >> 4), dtb + uint64_t(kk * 32 >> 4), idesc,
+                    kk > 0);
+      tc_commit(bar_mma);
+    }
+    // The decay record: gamma = 1 (the output uses Q .* e^Gamma directly),
+    // then the per-channel state decay e^Gamma_last.
+    {
+      const long long base = (long long)unit * 256;
+      if (GDN_IN_BOUNDS(ctrl, base + 255, (long long)max_chunks * H * 256)) {
+        // [0, 64): gamma = 1, [64, 128): unused, [128, 256): e^Gamma_last
+        gam_out[base + tid] = tid < 64 ? 1.f : (tid < 128 ? 0.f : El[tid - 128]);
+      }
+    }
+    mbar_wait(bar_mma, it & 1, ctrl, &abort_flag);
+    if (tid == 0) tma_store_wait_read();   // Q .* e^Gamma is staged where -W goes
+    tc_fence_after();
+    __syncthreads();
+    if (!abort_flag) {
+      // -W, K-major [64 c][128 d], from W^T (lanes = d, columns = c); warp w:
+      // lane quarter w % 4, token columns [32 (w / 4), 32 (w / 4) + 32).
+      const int q = warp & 3, hc = warp >> 2, mj = lane & 7, mm = lane >> 3;
+      const uint32_t lane_base = tmem + (uint32_t(32 * q) << 16);
+      const uint32_t wst = smem_u32(sm + kK_KQ);
+#pragma unroll
+      for (int lb = 0; lb < 32; lb += 16) {
+#pragma unroll
+        for (int cb = 32 * hc; cb < 32 * hc + 32; cb += 16) {
+          uint32_t w8[8];
+          tmem_ld16x256_x2(lane_base + (uint32_t(lb) << 16) + cb, w8);
+          tmem_ld_wait();
+          uint32_t w[4];
+#pragma unroll
+          for (int mq = 0; mq < 4; ++mq)
+            w[mq] = pack_bf16x2(-__uint_as_float(w8[2 * mq]), -__uint_as_float(w8[2 * mq + 1]));
+          const int d0 = q * 32 + lb + 8 * (mm & 1);
+          const int crow = cb + 8 * (mm >> 1) + mj;
+          stmatrix_x4_trans(wst + (d0 >> 6) * kTile64x64 + sw128_offset(crow, (d0 & 63) >> 3),
+                            w[0], w[1], w[2], w[3]);
+        }
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && !abort_flag) {
+      tma_store_2d(&tm_w, sm + kK_KQ, 0, unit * kC);
+      tma_store_2d(&tm_w, sm + kK_KQ + kTile64x64, 64, unit * kC);
+      tma_store_commit();
+    }
+  }
+  if (tid == 0) tma_store_wait_all();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 64);
+  }
+}
+
 // ===================================================================== scan
-// One stage (one chunk of one head), as the B operands of three wide MMAs:
-//   BXZ  2 x [ -W rows 0-63 | Q rows 64-127 ]  (128 rows, K = d_k in two blocks)
-//   BU   [ T diag(beta) rows 0-63 | zeros ]    (128 rows, K = 64 tokens)
-//   BSY  stage 0: [ (D K)^T rows 0-127 | P rows 128-191 ]  (192 rows, K = 64 tokens)
-//        stage 1: [ P rows 0-63 | (D K)^T rows 64-191 ]
-// plus V (the MN-major A operand of U^T). The zero half of BU is written
-// once; TMA never touches it. The two BSY orders put dS in the same tensor
+// One chunk of one head is loaded in three parts, each with its own ring so
+// that it can come in as soon as its last reader is done:
+//   X part  BXZ  2 x [ -W rows 0-63 | Q rows 64-127 ]  (128 rows, K = d_k in two
+//                blocks), the B operand of XZ; 3 stages, freed by XZ(c): a
+//                load from HBM takes about a chunk period here, so it is
+//                issued two chunks ahead
+//   U part  V (MN-major A operand of U^T, 2 x [64 s][64 d]) and
+//           BU = T diag(beta) (64 rows, K = 64 tokens); 2 slots, freed by U(c),
+//           which runs early in the previous chunk
+//   B part  BSY  stage 0: [ (D K)^T rows 0-127 | P rows 128-191 ]  (192 rows,
+//                K = 64 tokens), stage 1: [ P rows 0-63 | (D K)^T rows 64-191 ];
+//                2 stages, freed by SY(c)
+// The two BSY orders put dS in the same tensor
 // memory columns for every chunk and Y in one of two buffers (Y0 after dS,
 // Y1 before it), so SY(c+1) never waits for the output warps to finish Y(c).
 // The per-chunk decay factors (gamma[64], D[64]) travel in a separate 4-slot
 // ring so the output warps never hold a stage.
-constexpr uint32_t kS_BXZ = 0;                        // 32 KB
-constexpr uint32_t kS_V = kS_BXZ + 2 * kTile128x64;   // 16 KB, 2 x [64 s][64 d]
-constexpr uint32_t kS_BU = kS_V + 2 * kTile64x64;     // 16 KB
-constexpr uint32_t kS_BSY = kS_BU + kTile128x64;      // 24 KB
-constexpr uint32_t kStageBytes = kS_BSY + kTile128x64 + kTile64x64;   // 88 KB
-constexpr int kStages = 2, kGamSlots = 4;
-constexpr int kPrefetchAhead = 2;     // chunks prefetched into L2 ahead of the stage loads
-constexpr uint32_t kS_OST = kStages * kStageBytes;            // O staging, 2 x [64 c][64 d]
+constexpr int kStages = 2, kXStages = 3, kUSlots = 2, kGamSlots = 4;
+constexpr uint32_t kXStage = 2 * kTile128x64;                  // 32 KB
+constexpr uint32_t kUSlot = 2 * kTile64x64 + kTile64x64;       // 24 KB: V, then BU
+constexpr uint32_t kBStage = kTile128x64 + kTile64x64;         // 24 KB
+constexpr uint32_t kS_X = 0;
+constexpr uint32_t kS_U = kS_X + kXStages * kXStage;
+constexpr uint32_t kS_B = kS_U + kUSlots * kUSlot;
+constexpr int kPrefetchAhead = 0;     // chunks prefetched into L2 ahead of the stage loads (0: none)
+constexpr uint32_t kS_OST = kS_B + kStages * kBStage;          // O staging, 2 x [64 c][64 d]
 constexpr uint32_t kS_GAM = kS_OST + 2 * kTile64x64;          // kGamSlots x 128 fp32
-constexpr uint32_t kS_BAR = kS_GAM + kGamSlots * 512;         // mbarriers, tmem slot, flags
-constexpr uint32_t kS_END = kS_BAR + 256;
+constexpr uint32_t kGamRec = 1024;   // decay record slot: 128 fp32 (scalar) or 256 (channel-wise)
+constexpr uint32_t kS_BAR = kS_GAM + kGamSlots * kGamRec;      // mbarriers, tmem slot, flags
+constexpr uint32_t kS_END = kS_BAR + 512;
 constexpr uint32_t kScanSmem = kS_END;   // the dynamic window starts 1024-aligned (checked)
-constexpr uint32_t kStageTxA = kS_BSY - kTile64x64;   // BXZ, V and Tb (not the zero tile)
-constexpr uint32_t kStageTxB = kTile128x64 + kTile64x64;   // (D K)^T and P
+static_assert(kS_U % 1024 == 0 && kUSlot % 1024 == 0 && kS_B % 1024 == 0 &&
+                  kS_OST % 1024 == 0 && kScanSmem <= 232448,
+              "scan shared-memory layout");
 constexpr int kScanThreads = 512;
 // TMEM columns (fp32 accumulators, then the bf16 A operands held in TMEM)
 constexpr uint32_t kT_XZ = 0;     // [X | Z] = [U^T - S W^T | S Q^T]      fp32 [128][128]
+constexpr uint32_t kT_Z = 64;     //   (Z: zeroed by the output warps once they have read it)
 constexpr uint32_t kT_Y1 = 128;   // Y of odd chunks  = V_new^T P^T       fp32 [128][64]
 constexpr uint32_t kT_DS = 192;   // dS = V_new^T (D K)                    fp32 [128][128]
 constexpr uint32_t kT_Y0 = 320;   // Y of even chunks                      fp32 [128][64]
@@ -660,22 +1065,31 @@ constexpr uint32_t kBarOut = 2;
 // needs an MMA result that the MMA warp only issues after that sync.
 constexpr uint32_t kBarA1 = 3, kBarS = 4;
 constexpr uint32_t kChainHandoff = 8 * 32 + 32;   // 8 chain warps + the MMA warp
-// Barrier slots in the kS_BAR area
+// Barrier slots in the kS_BAR area (full_a / empty_a: the X part; full_u /
+// empty_u: the U part)
 // y_full[b] completes when Y buffer b holds a new chunk; the output warps wait
 // on it, the chain on s_full. (One barrier for both would let a slow output
 // warp miss a phase: it reports Z consumed before it waits for Y.)
 // Each stage has two parts with their own full/empty pairs: part A (BXZ, V,
 // BU) is last read by XZ(c) and part B (BSY) by SY(c), so the next loads of
 // part A start while SY(c) and the S epilogue still run.
-constexpr int kB_FULLA = 0, kB_EMPTYA = 2, kB_FULLB = 4, kB_EMPTYB = 6, kB_GFULL = 8,
-              kB_GEMPTY = 12, kB_XFULL = 16, kB_SFULL = 17, kB_YFULL = 18, kB_ZFREE = 20,
-              kB_DRAIN = 21, kB_COUNT = 22;
+// x_free / u_done hand U(c+1) to its own issuing warp and back: x_free(c)
+// completes once the V_new epilogue has read X(c), u_done(c+1) once U(c+1)
+// has run (XZ(c+1) accumulates on it).
+constexpr int kB_FULLA = 0, kB_EMPTYA = 3, kB_FULLB = 6, kB_EMPTYB = 8, kB_GFULL = 10,
+              kB_GEMPTY = 14, kB_XFULL = 18, kB_SFULL = 19, kB_YFULL = 20, kB_ZFREE = 22,
+              kB_DRAIN = 23, kB_XFREE = 24, kB_UDONE = 25, kB_DRAINU = 26, kB_FULLU = 27,
+              kB_EMPTYU = 29, kB_COUNT = 31;
+static_assert(kB_COUNT * 8 + 8 <= 512, "barrier area");
 
 // Warp roles (16 warps). Every role runs its loop with all 32 lanes, so the
 // lanes of a warp wait on barriers together; one lane issues TMA copies,
 // MMAs and arrivals.
 //   warp 0        TMA producer
-//   warp 1        TMEM allocation and every tcgen05.mma
+//   warp 1        TMEM allocation and the chain's tcgen05.mma (XZ, SY)
+//   warp 2        U = V^T Tb^T (tcgen05.mma): a thread issues MMAs only about
+//                 as fast as the tensor core runs them, so U has an issuer of
+//                 its own and the chain's issuer is free when S is ready
 //   warps 4-11    state chain: two warpgroups, warpgroup h owns columns
 //                 [32h, 32h+32) of V_new and [64h, 64h+64) of S; thread =
 //                 TMEM lane = row i of d_v; the fp32 S lives in its registers,
@@ -683,13 +1097,15 @@ constexpr int kB_FULLA = 0, kB_EMPTYA = 2, kB_FULLB = 4, kB_EMPTYB = 6, kB_GFULL
 //                 epilogue is handed to the MMA warp through a named barrier.
 //   warps 12-15   output: O = diag(gamma) Z + Y, staged for TMA stores
 // Per chunk c the tensor core runs three wide products:
-//   U(c)   [X|Z]  = V^T [Tb | 0]^T            (4 MMAs, N = 128)  -- before S_c is known
+//   U(c)   X      = V^T Tb^T                  (4 MMAs, N = 64)   -- before S_c is known
 //   XZ(c)  [X|Z] += S [-W | Q]^T              (8 MMAs, N = 128)  -> X = V_new^T, Z = S Q^T
 //   SY(c)  [dS|Y] = V_new^T [(DK)^T | P]^T    (4 MMAs, N = 192)
 // and the chain is XZ -> V_new epilogue -> SY -> S epilogue -> XZ(c+1), with
-// U(c+1) running during the S epilogue. The MMA warp does its other waits
-// (output done with Z, next stage loaded) while the V_new epilogue runs, so
-// only the two epilogue handshakes sit on the chain.
+// U(c+1) running during the S epilogue. XZ
+// accumulates Z on zeros: the output warps read Z(c), store zeros in its
+// place and then free it (z_free), which only XZ(c+1) waits for -- by then
+// the output warps are long done. So only the two epilogue handshakes sit on
+// the chain.
 __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_v,
     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_kt,
@@ -698,7 +1114,18 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     const float *__restrict__ s0, float *__restrict__ sN, __nv_bfloat16 *__restrict__ o, int H,
     uint32_t *__restrict__ ctrl, const ChunkInfo *__restrict__ table,
     const int32_t *__restrict__ seq_first, int split, float *__restrict__ sN_trans,
-    int sN_group) {
+    int sN_group, long long rows, int max_chunks, int n_first, int n_s0, int n_sN, int kda) {
+  // kda: the channel-wise gate. Q comes per unit from the prep (Q .* e^Gamma,
+  // 2-D map tm_q over [units * 64][128]), the decay records are 256 wide and
+  // S decays per d_k channel.
+  // rows, max_chunks: token rows of q/k/v/o and chunk-table entries; n_first:
+  // entries of seq_first; n_s0 / n_sN: states in s0 and in the array the final
+  // states go to (the extents of the bounds checks of GDN_CHECKS builds).
+  (void)rows;
+  (void)max_chunks;
+  (void)n_first;
+  (void)n_s0;
+  (void)n_sN;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *sm = smem_raw;                 // pointer arithmetic keeps the shared space
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -717,6 +1144,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
   }
   const bool tr = (n == 0 && h == 0);     // traced CTA (GDN_TRACE builds only)
   (void)tr;
+#ifdef GDN_TRACE
+  const int cta_id = int(blockIdx.y * gridDim.x + blockIdx.x);
+  if (tid == 0 && cta_id < 1024) g_gdn_cta_ns[cta_id][0] = global_ns();
+#endif
 
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kS_BAR);
   uint64_t *full_a = bars + kB_FULLA, *empty_a = bars + kB_EMPTYA;
@@ -724,6 +1155,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
   uint64_t *gfull = bars + kB_GFULL, *gempty = bars + kB_GEMPTY;
   uint64_t *x_full = bars + kB_XFULL, *s_full = bars + kB_SFULL, *y_full = bars + kB_YFULL;
   uint64_t *z_free = bars + kB_ZFREE, *drain = bars + kB_DRAIN;
+  uint64_t *x_free = bars + kB_XFREE, *u_done = bars + kB_UDONE;
+  uint64_t *full_u = bars + kB_FULLU, *empty_u = bars + kB_EMPTYU;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kB_COUNT);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -744,12 +1177,6 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     }
     fence_mbar_init();
   }
-  // The zero half of BU in both stages.
-  for (int e = tid; e < kStages * (kTile64x64 / 16); e += kScanThreads) {
-    const int st = e / (kTile64x64 / 16), off = e % (kTile64x64 / 16);
-    *reinterpret_cast<uint4 *>(sm + st * kStageBytes + kS_BU + kTile64x64 + off * 16) =
-        make_uint4(0, 0, 0, 0);
-  }
   fence_proxy_async_smem();
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -765,68 +1192,92 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
   // The chunk table and the prep kernel's outputs are read only after the
   // kernels that write them have completed (the chain warps first load the
   // initial state, which no earlier kernel of this call writes).
-  int c0 = 0, nch = 0;
+  // A sequence's (or segment's) chunks are consecutive 64-token blocks from
+  // its first row, only the last one possibly partial: chunk c starts at row
+  // row_first + 64 c and is last_len long if c == nch - 1, else 64. Read once
+  // here rather than a table entry per chunk (a dependent global load on the
+  // producer's path).
+  int c0 = 0, nch = 0, row_first = 0, last_len = kC;
   auto read_chunks = [&]() {
     grid_dependency_wait();
     if (!(ctrl[0] & kErrBadSeqlens)) {
-      c0 = seq_first[n];
-      nch = seq_first[n + 1] - c0;
+      if (GDN_IN_BOUNDS(ctrl, n + 1, n_first)) {
+        c0 = seq_first[n];
+        nch = seq_first[n + 1] - c0;
+      }
+      if (nch > 0 && GDN_IN_BOUNDS(ctrl, c0, max_chunks) &&
+          GDN_IN_BOUNDS(ctrl, c0 + nch - 1, max_chunks)) {
+        row_first = table[c0].row0;
+        last_len = table[c0 + nch - 1].len;
+      } else {
+        nch = 0;
+      }
     }
   };
-  if (warp < 4 || warp >= 12) read_chunks();
+  auto chunk_row0 = [&](int c) { return row_first + kC * c; };
+  auto chunk_len = [&](int c) { return c == nch - 1 ? last_len : kC; };
+  if (warp < 4 || warp >= 12) read_chunks();   // warps 0-2 issue, 3 idles
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     for (int c = 0; c < nch && !*abort_flag; ++c) {
-      const int st = c & 1, gs = c & 3;
-      const ChunkInfo ci = table[c0 + c];
+      const int st = c & 1, gs = c & 3, us = c % kUSlots;
+      const int row0 = chunk_row0(c);
       const int unit = (c0 + c) * H + h;
-      uint8_t *sb = sm + st * kStageBytes;
-      if (c >= 2) wait(empty_a + st, ((c >> 1) - 1) & 1);
-      if (lane == 0) {
-        GDN_TRACE_POINT(tr, 0, c, 0);
-        // Only what this CTA's products read: a run without output needs
-        // neither Q nor P, a transition run neither V nor T diag(beta).
-        mbar_arrive_expect_tx(full_a + st, (write_o ? kStageTxA : kStageTxA - kTile128x64) -
-                                               (trans ? 2 * kTile64x64 + kTile64x64 : 0u));
-        tma_load_2d(sb + kS_BXZ, &tm_w, full_a + st, 0, unit * kC);
-        tma_load_2d(sb + kS_BXZ + kTile128x64, &tm_w, full_a + st, 64, unit * kC);
-        if (write_o) {
-          tma_load_3d(sb + kS_BXZ + kTile64x64, &tm_q, full_a + st, 0, h, ci.row0);
-          tma_load_3d(sb + kS_BXZ + kTile128x64 + kTile64x64, &tm_q, full_a + st, 64, h,
-                      ci.row0);
+      GDN_TRACE_POINT(tr && lane == 0, 0, c, 0);
+      // Only what this CTA's products read: a run without output needs
+      // neither Q nor P, a transition run neither V nor T diag(beta).
+      if (!trans) {
+        if (c >= kUSlots) wait(empty_u + us, ((c / kUSlots) - 1) & 1);
+        if (lane == 0) {
+          uint8_t *ub = sm + kS_U + us * kUSlot;
+          mbar_arrive_expect_tx(full_u + us, kUSlot);
+          tma_load_3d(ub, &tm_v, full_u + us, 0, h, row0);
+          tma_load_3d(ub + kTile64x64, &tm_v, full_u + us, 64, h, row0);
+          tma_load_2d(ub + 2 * kTile64x64, &tm_tb, full_u + us, 0, unit * kC);
         }
-        if (!trans) {
-          tma_load_3d(sb + kS_V, &tm_v, full_a + st, 0, h, ci.row0);
-          tma_load_3d(sb + kS_V + kTile64x64, &tm_v, full_a + st, 64, h, ci.row0);
-          tma_load_2d(sb + kS_BU, &tm_tb, full_a + st, 0, unit * kC);
+        __syncwarp();
+      }
+      const int xs = c % kXStages;
+      uint8_t *xb = sm + kS_X + xs * kXStage;
+      if (c >= kXStages) wait(empty_a + xs, ((c / kXStages) - 1) & 1);
+      if (lane == 0) {
+        mbar_arrive_expect_tx(full_a + xs, write_o ? kXStage : kTile128x64);
+        tma_load_2d(xb, &tm_w, full_a + xs, 0, unit * kC);
+        tma_load_2d(xb + kTile128x64, &tm_w, full_a + xs, 64, unit * kC);
+        if (write_o && kda) {
+          tma_load_2d(xb + kTile64x64, &tm_q, full_a + xs, 0, unit * kC);
+          tma_load_2d(xb + kTile128x64 + kTile64x64, &tm_q, full_a + xs, 64, unit * kC);
+        } else if (write_o) {
+          tma_load_3d(xb + kTile64x64, &tm_q, full_a + xs, 0, h, row0);
+          tma_load_3d(xb + kTile128x64 + kTile64x64, &tm_q, full_a + xs, 64, h, row0);
         }
       }
       __syncwarp();
+      uint8_t *bb = sm + kS_B + st * kBStage;
       if (c >= 2) wait(empty_b + st, ((c >> 1) - 1) & 1);
       if (lane == 0) {
         // Without output, (D K)^T goes first in both stages and P is not loaded.
         const bool swap = st && write_o;
-        mbar_arrive_expect_tx(full_b + st, write_o ? kStageTxB : kTile128x64);
-        tma_load_2d(sb + kS_BSY + (swap ? kTile64x64 : 0u), &tm_kt, full_b + st, 0, unit * kD);
-        if (write_o)
-          tma_load_2d(sb + kS_BSY + (st ? 0u : kTile128x64), &tm_pm, full_b + st, 0, unit * kC);
-        // The loads above take about one chunk period to land from HBM; the
-        // chunk after next goes to L2 now, so its own loads come from L2.
-        if (c + kPrefetchAhead < nch) {
-          const ChunkInfo cp = table[c0 + c + kPrefetchAhead];
+        mbar_arrive_expect_tx(full_b + st, write_o ? kBStage : kTile128x64);
+        tma_load_2d(bb + (swap ? kTile64x64 : 0u), &tm_kt, full_b + st, 0, unit * kD);
+        if (write_o) tma_load_2d(bb + (st ? 0u : kTile128x64), &tm_pm, full_b + st, 0, unit * kC);
+        // Stage loads wait for their ring slot; the chunks ahead go to L2 now,
+        // so those loads come from L2.
+        if (kPrefetchAhead > 0 && c + kPrefetchAhead < nch) {
+          const int rp = chunk_row0(c + kPrefetchAhead);
           const int up = (c0 + c + kPrefetchAhead) * H + h;
           tma_prefetch_l2_2d(&tm_w, 0, up * kC);
           tma_prefetch_l2_2d(&tm_w, 64, up * kC);
           tma_prefetch_l2_2d(&tm_kt, 0, up * kD);
           if (write_o) {
-            tma_prefetch_l2_3d(&tm_q, 0, h, cp.row0);
-            tma_prefetch_l2_3d(&tm_q, 64, h, cp.row0);
+            tma_prefetch_l2_3d(&tm_q, 0, h, rp);
+            tma_prefetch_l2_3d(&tm_q, 64, h, rp);
             tma_prefetch_l2_2d(&tm_pm, 0, up * kC);
           }
           if (!trans) {
-            tma_prefetch_l2_3d(&tm_v, 0, h, cp.row0);
-            tma_prefetch_l2_3d(&tm_v, 64, h, cp.row0);
+            tma_prefetch_l2_3d(&tm_v, 0, h, rp);
+            tma_prefetch_l2_3d(&tm_v, 64, h, rp);
             tma_prefetch_l2_2d(&tm_tb, 0, up * kC);
           }
         }
@@ -834,8 +1285,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
       __syncwarp();
       if (c >= 4) wait(gempty + gs, ((c >> 2) - 1) & 1);
       if (lane == 0) {
-        mbar_arrive_expect_tx(gfull + gs, 512);
-        tma_load_2d(sm + kS_GAM + gs * 512, &tm_gam, gfull + gs, 0, unit);
+        mbar_arrive_expect_tx(gfull + gs, kda ? 1024 : 512);
+        tma_load_2d(sm + kS_GAM + gs * kGamRec, &tm_gam, gfull + gs, 0, unit);
       }
       __syncwarp();
     }
@@ -843,7 +1294,6 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     // ------------------------------------------------------------ MMA issuer
     // Without output, Z and Y are not needed: U and XZ shrink to X (N = 64),
     // SY to dS (N = 128, (D K)^T then first in both stages).
-    const uint32_t id_u = make_idesc_bf16(128, write_o ? 128 : 64, 1, 0);   // V^T [Tb|0]^T
     const uint32_t id_xz = make_idesc_bf16(128, write_o ? 128 : 64, 0, 0);  // S [-W|Q]^T
     const uint32_t id_sy = make_idesc_bf16(128, write_o ? 192 : 128, 0, 0); // A1 [(DK)^T|P]^T
     const bool issuer = lane == 0;
@@ -852,33 +1302,18 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     // integer op, so rebuilding descriptors between MMAs doubles the issue
     // time. A k step is added to the start-address field (smem offsets >> 4
     // stay below 2^14, so the field never carries into the next one).
-    uint64_t dV[kStages], dBU[kStages], dBXZ[kStages], dBSY[kStages];
+    uint64_t dBSY[kStages];
 #pragma unroll
-    for (int st = 0; st < kStages; ++st) {
-      const uint32_t sb = smem_u32(sm + st * kStageBytes);
-      dV[st] = make_sdesc(sb + kS_V, kTile64x64, 1024);
-      dBU[st] = make_sdesc(sb + kS_BU, 16, 1024);
-      dBXZ[st] = make_sdesc(sb + kS_BXZ, 16, 1024);
-      dBSY[st] = make_sdesc(sb + kS_BSY, 16, 1024);
-    }
-    // U(c) into [X|Z]. The caller has seen chunk c loaded and the output
-    // warps done reading Z of chunk c - 1.
-    auto issue_u = [&](int c) {
-      if (issuer) {
-        const uint64_t da = (c & 1) ? dV[1] : dV[0], db = (c & 1) ? dBU[1] : dBU[0];
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          tc_mma_bf16(tmem + kT_XZ, da + uint64_t(kk * 2048 >> 4), db + uint64_t(kk * 32 >> 4),
-                      id_u, kk > 0);
-      }
-      __syncwarp();
-    };
+    for (int st = 0; st < kStages; ++st)
+      dBSY[st] = make_sdesc(smem_u32(sm + kS_B + st * kBStage), 16, 1024);
     // XZ(c) += S_c [-W|Q]^T, reading the bf16 copy of S_c.
     auto issue_xz = [&](int c) {
       if (issuer) {
         GDN_TRACE_POINT(tr, 0, c, 1);
-        const uint64_t db = (c & 1) ? dBXZ[1] : dBXZ[0];
+#ifdef GDN_TRACE
+        if (cta_id < 1024) g_gdn_cta_ns[cta_id][c == 0 ? 1 : 2] = global_ns();
+#endif
+        const uint64_t db = make_sdesc(smem_u32(sm + kS_X + (c % kXStages) * kXStage), 16, 1024);
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)   // a transition run has no U: XZ starts the sum
@@ -886,13 +1321,14 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
                          db + uint64_t(((kk >> 2) * kTile128x64 + (kk & 3) * 32) >> 4), id_xz,
                          (kk > 0) || !trans);
         tc_commit(x_full);
-        tc_commit(empty_a + (c & 1));     // U(c) and XZ(c) were the last readers of part A
+        tc_commit(empty_a + (c % kXStages));   // XZ(c) was the last reader of the X part
       }
       __syncwarp();
     };
     if (nch > 0) {
-      wait(full_a, 0);
-      if (!trans) issue_u(0);
+      wait(full_a, 0);                        // -W and Q of chunk 0 (stage 0)
+      if (!trans) wait(u_done, 0);            // X = U(0)
+      wait(z_free, 0);                        // Z zeroed at the start
     }
     named_bar_sync(kBarS, kChainHandoff);     // S_0 stored (the chain hands it over even if nch = 0)
     if (nch > 0) issue_xz(0);
@@ -903,10 +1339,12 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
       named_bar_sync(kBarA1, kChainHandoff);  // V_new^T of chunk c in tensor memory
       GDN_TRACE_POINT(tr && issuer, 0, c, 6);
       if (issuer) {
+        mbar_arrive(x_free);              // X(c) read: U(c + 1) may overwrite it
         const uint64_t db = st ? dBSY[1] : dBSY[0];
         tc_fence_after();
         // even chunks: D = [dS | Y0] at kT_DS; odd: D = [Y1 | dS] at kT_Y1
-        // (without output: D = dS at kT_DS for every chunk)
+        // (without output: D = dS at kT_DS for every chunk). One N = 192
+        // group: a separate Y group would hold this issuer up as well.
         const uint32_t d = tmem + ((st && write_o) ? kT_Y1 : kT_DS);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
@@ -917,14 +1355,14 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
         GDN_TRACE_POINT(tr, 0, c, 12);
       }
       __syncwarp();
-      // Off the chain (SY(c) and the S epilogue are running): U(c+1) needs the
-      // output warps done with Z(c) and part A of chunk c + 1.
+      // While SY(c) and the S epilogue run: XZ(c + 1) needs U(c + 1) done,
+      // -W and Q of chunk c + 1, and Z(c) read and zeroed by the output warps.
       if (more) {
-        wait(z_free, c & 1);
-        GDN_TRACE_POINT(tr && issuer, 0, c, 13);
-        wait(full_a + (st ^ 1), ((c + 1) >> 1) & 1);
+        if (!trans) wait(u_done, (c + 1) & 1);
+        wait(full_a + (c + 1) % kXStages, ((c + 1) / kXStages) & 1);
         GDN_TRACE_POINT(tr && issuer, 0, c, 14);
-        if (!trans) issue_u(c + 1);
+        wait(z_free, (c + 1) & 1);
+        GDN_TRACE_POINT(tr && issuer, 0, c, 13);
       }
       named_bar_sync(kBarS, kChainHandoff);   // S_{c+1} stored, decay factors of c read
       GDN_TRACE_POINT(tr && issuer, 0, c, 8);
@@ -937,6 +1375,34 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     // Waited for even after an abort (bounded): tensor memory is freed below.
     volatile int keep_waiting = 0;
     mbar_wait(drain, 0, ctrl, &keep_waiting);
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ U issuer
+    // U(c) = V^T Tb^T into X (accumulate = 0). U(c) needs chunk c loaded and,
+    // for c > 0, X(c - 1) read by the V_new epilogue.
+    const bool issuer = lane == 0;
+    const uint32_t id_u = make_idesc_bf16(128, 64, 1, 0);
+    for (int c = 0; c < nch && !trans; ++c) {
+      const int us = c % kUSlots;
+      if (c > 0) wait(x_free, (c - 1) & 1);
+      wait(full_u + us, (c / kUSlots) & 1);
+      if (issuer) {
+        const uint32_t ub = smem_u32(sm + kS_U + us * kUSlot);
+        const uint64_t da = make_sdesc(ub, kTile64x64, 1024);
+        const uint64_t db = make_sdesc(ub + 2 * kTile64x64, 16, 1024);
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma_bf16(tmem + kT_XZ, da + uint64_t(kk * 2048 >> 4), db + uint64_t(kk * 32 >> 4),
+                      id_u, kk > 0);
+        tc_commit(u_done);
+        tc_commit(empty_u + us);
+      }
+      __syncwarp();
+    }
+    if (issuer) tc_commit(bars + kB_DRAINU);  // fires once every U above has completed
+    __syncwarp();
+    volatile int keep_waiting = 0;
+    mbar_wait(bars + kB_DRAINU, 0, ctrl, &keep_waiting);
   } else if (warp >= 4 && warp < 12) {
     // ------------------------------------------------------------ state chain
     const int hh = (warp - 4) >> 2;                     // column half
@@ -946,7 +1412,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     (void)tl;
     float S[64];                                        // S[i][64 hh + t], fp32 master
     {
-      const float *src = (s0 && !trans) ? s0 + (size_t(n) * H + h) * kD * kD : nullptr;
+      const float *src = (s0 && !trans && GDN_IN_BOUNDS(ctrl, (long long)n * H + h, (long long)n_s0 * H))
+                             ? s0 + (size_t(n) * H + h) * kD * kD
+                             : nullptr;
 #pragma unroll
       for (int t = 0; t < 64; ++t)
         S[t] = trans ? (64 * hh + t == i ? 1.f : 0.f) : (src ? src[size_t(64 * hh + t) * kD + i] : 0.f);
@@ -988,7 +1456,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
       named_bar_arrive(kBarA1, kChainHandoff);
       // S <- gamma_last S + dS on columns [64 hh, 64 hh + 64)
       wait(gfull + gs, (c >> 2) & 1);
-      const float gl = reinterpret_cast<const float *>(sm + kS_GAM + gs * 512)[kC - 1];
+      const float *rec = reinterpret_cast<const float *>(sm + kS_GAM + gs * kGamRec);
+      const float gl = rec[kC - 1];
       wait(s_full, c & 1);
       GDN_TRACE_POINT(tl, 0, c, 7);
       tc_fence_after();
@@ -998,12 +1467,25 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
         tmem_ld32(lane_base + kT_DS + 64 * hh + 32 * b, d);
         tmem_ld_wait();
         GDN_TRACE_POINT(tl && b == 0, 0, c, 3);
+        if (!kda) {
 #pragma unroll
-        for (int t = 0; t < 32; t += 2) {
-          const float2 r = ffma2(make_float2(gl, gl), make_float2(S[32 * b + t], S[32 * b + t + 1]),
-                                 make_float2(__uint_as_float(d[t]), __uint_as_float(d[t + 1])));
-          S[32 * b + t] = r.x;
-          S[32 * b + t + 1] = r.y;
+          for (int t = 0; t < 32; t += 2) {
+            const float2 r = ffma2(make_float2(gl, gl), make_float2(S[32 * b + t], S[32 * b + t + 1]),
+                                   make_float2(__uint_as_float(d[t]), __uint_as_float(d[t + 1])));
+            S[32 * b + t] = r.x;
+            S[32 * b + t + 1] = r.y;
+          }
+        } else {
+          // channel-wise gate: column j of S (d_k channel) decays by e^Gamma_last,j
+          const float *dec = rec + 128 + 64 * hh + 32 * b;
+#pragma unroll
+          for (int t = 0; t < 32; t += 2) {
+            const float2 r = ffma2(*reinterpret_cast<const float2 *>(dec + t),
+                                   make_float2(S[32 * b + t], S[32 * b + t + 1]),
+                                   make_float2(__uint_as_float(d[t]), __uint_as_float(d[t + 1])));
+            S[32 * b + t] = r.x;
+            S[32 * b + t + 1] = r.y;
+          }
         }
       }
       store_state();
@@ -1012,7 +1494,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     }
     float *sNp = trans ? sN_trans : sN;
     const int sN_idx = trans ? n : n / sN_group;
-    if (sNp && (trans || n % sN_group == sN_group - 1) && !*abort_flag) {
+    if (sNp && (trans || n % sN_group == sN_group - 1) && !*abort_flag &&
+        GDN_IN_BOUNDS(ctrl, (long long)sN_idx * H + h, (long long)n_sN * H)) {
       float *dst = sNp + (size_t(sN_idx) * H + h) * kD * kD;
 #pragma unroll
       for (int t = 0; t < 64; ++t) dst[size_t(64 * hh + t) * kD + i] = S[t];
@@ -1021,7 +1504,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     // ------------------------------------------------------------ output
     // O[c'][i] = gamma_c' Z[i][c'] + Y[i][c'] (Z, Y are O^T in TMEM). Each warp
     // reads its 32 lanes as mma-accumulator fragments (16 lanes x 8 columns),
-    // Z as soon as XZ is done (so U of the next chunk may overwrite it), Y
+    // Z as soon as XZ is done (then zeroes it for XZ of the next chunk), Y
     // after SY, and writes O transposed into the swizzled staging tile with
     // stmatrix, 16 bytes per row; a TMA store (whole chunks) or a 16-byte copy
     // loop (a sequence's last, partial chunk) moves the tile to o.
@@ -1031,6 +1514,20 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     const uint32_t ost = smem_u32(sm + kS_OST);
     const int fc = 2 * (lane & 3);                     // fragment column pair
     const int mj = lane & 7, mm = lane >> 3;           // stmatrix: row j of matrix m
+    // Zeros into this warp's 32 lanes of the Z columns (waited for here).
+    auto zero_z = [&]() {
+      uint32_t zr[32];
+#pragma unroll
+      for (int t = 0; t < 32; ++t) zr[t] = 0u;
+      tmem_st32(lane_q + kT_Z, zr);
+      tmem_st32(lane_q + kT_Z + 32, zr);
+      tmem_st_wait();
+    };
+    // z_free phase 0: Z starts at zero (XZ accumulates it on top).
+    if (write_o) zero_z();
+    tc_fence_before();
+    named_bar_sync(kBarOut, 128);
+    if (leader) mbar_arrive(z_free);
     for (int c = 0; c < nch && !write_o; ++c) {
       // No output: keep only this role's side of the barrier protocol.
       const int gs = c & 3;
@@ -1042,15 +1539,16 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     }
     for (int c = 0; c < nch && write_o; ++c) {
       const int gs = c & 3;
-      const float *gam = reinterpret_cast<const float *>(sm + kS_GAM + gs * 512);
-      const ChunkInfo ci = table[c0 + c];
-      const bool whole = ci.len == kC;
+      const float *gam = reinterpret_cast<const float *>(sm + kS_GAM + gs * kGamRec);
+      const int row0 = chunk_row0(c), len = chunk_len(c);
+      const bool whole = len == kC;
       uint32_t z[2][32], ynext[8];
       wait(x_full, c & 1);
       tc_fence_after();
       tmem_ld16x256_x8(lane_q + kT_XZ + 64, z[0]);
       tmem_ld16x256_x8(lane_q + (16u << 16) + kT_XZ + 64, z[1]);
       tmem_ld_wait();
+      zero_z();                                  // for XZ(c + 1)
       tc_fence_before();
       named_bar_sync(kBarOut, 128);
       if (leader) mbar_arrive(z_free);
@@ -1102,8 +1600,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
       if (leader) {
         mbar_arrive(gempty + gs);
         if (whole && !*abort_flag) {
-          tma_store_3d(&tm_o, sm + kS_OST, 0, h, ci.row0);
-          tma_store_3d(&tm_o, sm + kS_OST + kTile64x64, 64, h, ci.row0);
+          tma_store_3d(&tm_o, sm + kS_OST, 0, h, row0);
+          tma_store_3d(&tm_o, sm + kS_OST + kTile64x64, 64, h, row0);
           tma_store_commit();
         }
         GDN_TRACE_POINT(tr, 0, c, 10);
@@ -1111,11 +1609,13 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
       __syncwarp();
       if (!whole && !*abort_flag) {
         // rows [0, len) of the tile, 16 bytes at a time
-        for (int e = ot; e < ci.len * 16; e += 128) {
+        for (int e = ot; e < len * 16; e += 128) {
           const int row = e >> 4, k = e & 15;
           const uint4 v = *reinterpret_cast<const uint4 *>(
               sm + kS_OST + (k >> 3) * kTile64x64 + sw128_offset(row, k & 7));
-          *reinterpret_cast<uint4 *>(o + (size_t(ci.row0 + row) * H + h) * kD + 8 * k) = v;
+          const long long oi = ((long long)(row0 + row) * H + h) * kD + 8 * k;
+          if (GDN_IN_BOUNDS(ctrl, oi + 7, rows * H * kD))
+            *reinterpret_cast<uint4 *>(o + oi) = v;
         }
       }
     }
@@ -1124,6 +1624,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
   }
   tc_fence_before();
   __syncthreads();
+#ifdef GDN_TRACE
+  if (tid == 0 && cta_id < 1024) g_gdn_cta_ns[cta_id][3] = global_ns();
+#endif
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -1142,7 +1645,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
 __global__ void __launch_bounds__(256) gdn_segment_combine_kernel(
     const float *__restrict__ s0, const float *__restrict__ hbuf,
     const float *__restrict__ pbuf, float *__restrict__ sstart, int H, int segs,
-    const uint32_t *__restrict__ ctrl) {
+    uint32_t *__restrict__ ctrl) {
   __shared__ __align__(16) float X[kD][16];
   const int b = blockIdx.x / H, h = blockIdx.x - b * H, col0 = 16 * blockIdx.y;
   const int tid = threadIdx.x;
@@ -1154,6 +1657,10 @@ __global__ void __launch_bounds__(256) gdn_segment_combine_kernel(
   __syncthreads();
   const int j = tid >> 1, c0 = (tid & 1) * 8;   // this thread's row and 8 columns
   for (int gi = 0; gi < segs; ++gi) {
+    // (uniform across the CTA, so the barriers below stay matched)
+    if (!GDN_IN_BOUNDS(ctrl, (long long)(b * segs + gi) * H + h,
+                       (long long)(gridDim.x / H) * segs * H))
+      break;
     const size_t base = ((size_t(b) * segs + gi) * H + h) * kD * kD;
     float4 *dst = reinterpret_cast<float4 *>(sstart + base + size_t(j) * kD + col0 + c0);
     dst[0] = *reinterpret_cast<const float4 *>(&X[j][c0]);
@@ -1244,7 +1751,8 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
   const long long rows = (long long)B * T;
   const long long units = (long long)L.max_chunks * H;
   if (T > 0 && L.max_chunks > 0) {
-    CUtensorMap mq, mk, mv, mo, mw, mkt, mtb, mpm, mgm;
+    CUtensorMap mq, mk, mv, mo, mw, mkt, mtb, mpm, mgm, mqt;
+    const int rec = L.kda ? 256 : 128;   // decay record width
     if (!map_tokens(&mq, q, rows, H) || !map_tokens(&mk, k, rows, H) ||
         !map_tokens(&mv, v, rows, H) || !map_tokens(&mo, o, rows, H) ||
         !map_2d(&mw, base + L.w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, units * kC, kD, 64, kC,
@@ -1255,11 +1763,17 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
         !map_2d(&mpm, base + L.pm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, units * kC, 64, 64, kC,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !map_2d(&mgm, base + L.gam, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, units, 128, 128, 1,
-                CU_TENSOR_MAP_SWIZZLE_NONE))
+        !map_2d(&mgm, base + L.gam, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, units, rec, rec, 1,
+                CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        (L.kda && !map_2d(&mqt, base + L.qt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, units * kC, kD,
+                          64, kC, CU_TENSOR_MAP_SWIZZLE_128B)))
       return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(gdn_prep_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kPrepSmem);
+    cudaError_t e = L.kda ? cudaFuncSetAttribute(gdn_kda_prep_kernel,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 kKdaPrepSmem)
+                          : cudaFuncSetAttribute(gdn_prep_kernel,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 kPrepSmem);
     if (e != cudaSuccess) return e;
     prof_record(g_profile.prep, s);
     int dev = 0, sms = 0;
@@ -1267,7 +1781,7 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     if (e != cudaSuccess) return e;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    const long long prep_ctas = std::min<long long>(units, 3LL * sms);
+    const long long prep_ctas = std::min<long long>(units, (L.kda ? 1LL : 3LL) * sms);
     // Both kernels start with programmatic dependent launch: their prologues
     // overlap the tail of the kernel before them.
     cudaLaunchAttribute pdl[1];
@@ -1275,14 +1789,22 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     pdl[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(prep_ctas));
-    cfg.blockDim = dim3(kPrepThreads);
-    cfg.dynamicSmemBytes = kPrepSmem;
+    cfg.blockDim = dim3(L.kda ? kKdaPrepThreads : kPrepThreads);
+    cfg.dynamicSmemBytes = L.kda ? kKdaPrepSmem : kPrepSmem;
     cfg.stream = s;
     cfg.attrs = pdl;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, gdn_prep_kernel, mq, mk, mw, mkt, mtb, mpm, g, beta,
-                           reinterpret_cast<float *>(base + L.gam), H, ctrl, table);
+    if (L.kda)
+      e = cudaLaunchKernelEx(&cfg, gdn_kda_prep_kernel, mq, mk, mw, mkt, mtb, mpm, mqt, g, beta,
+                             reinterpret_cast<float *>(base + L.gam), H, ctrl, table, rows,
+                             L.max_chunks);
+    else
+      e = cudaLaunchKernelEx(&cfg, gdn_prep_kernel, mq, mk, mw, mkt, mtb, mpm, g, beta,
+                             reinterpret_cast<float *>(base + L.gam), H, ctrl, table, rows,
+                             L.max_chunks);
     if (e != cudaSuccess) return e;
+    // the scan reads Q from the prep's Q .* e^Gamma with the channel-wise gate
+    const CUtensorMap mqs = L.kda ? mqt : mq;
     e = cudaFuncSetAttribute(gdn_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kScanSmem);
     if (e != cudaSuccess) return e;
@@ -1291,10 +1813,11 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     cfg.dynamicSmemBytes = kScanSmem;
     if (L.segs <= 1) {
       cfg.gridDim = dim3(N, H);
-      return cudaLaunchKernelEx(&cfg, gdn_scan_kernel, mq, mv, mw, mkt, mtb, mpm, mgm, mo, s0,
+      return cudaLaunchKernelEx(&cfg, gdn_scan_kernel, mqs, mv, mw, mkt, mtb, mpm, mgm, mo, s0,
                                 sN, static_cast<__nv_bfloat16 *>(o), H, ctrl,
                                 static_cast<const ChunkInfo *>(table), seq_first, 0,
-                                static_cast<float *>(nullptr), 1);
+                                static_cast<float *>(nullptr), 1, rows, L.max_chunks, N + 1, N,
+                                N, int(L.kda));
     }
     // Segmented state scan (few long sequences): three passes over B * segs
     // segments. (1) every segment from S = 0 and as a transition, no output;
@@ -1306,10 +1829,11 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     float *pbuf = reinterpret_cast<float *>(base + L.pbuf);
     float *sstart = reinterpret_cast<float *>(base + L.sstart);
     cfg.gridDim = dim3(2 * nseg, H);
-    e = cudaLaunchKernelEx(&cfg, gdn_scan_kernel, mq, mv, mw, mkt, mtb, mpm, mgm, mo,
+    e = cudaLaunchKernelEx(&cfg, gdn_scan_kernel, mqs, mv, mw, mkt, mtb, mpm, mgm, mo,
                            static_cast<const float *>(nullptr), hbuf,
                            static_cast<__nv_bfloat16 *>(nullptr), H, ctrl,
-                           static_cast<const ChunkInfo *>(table), seg_first, nseg, pbuf, 1);
+                           static_cast<const ChunkInfo *>(table), seg_first, nseg, pbuf, 1, rows,
+                           L.max_chunks, nseg + 1, 0, nseg, int(L.kda));
     if (e != cudaSuccess) return e;
     gdn_segment_combine_kernel<<<dim3(B * H, kD / 16), 256, 0, s>>>(s0, hbuf, pbuf, sstart, H,
                                                                    L.segs, ctrl);
@@ -1318,11 +1842,12 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     // A plain launch: the start states come from the kernel just before it.
     cfg.gridDim = dim3(nseg, H);
     cfg.numAttrs = 0;
-    return cudaLaunchKernelEx(&cfg, gdn_scan_kernel, mq, mv, mw, mkt, mtb, mpm, mgm, mo,
+    return cudaLaunchKernelEx(&cfg, gdn_scan_kernel, mqs, mv, mw, mkt, mtb, mpm, mgm, mo,
                               static_cast<const float *>(sstart), sN,
                               static_cast<__nv_bfloat16 *>(o), H, ctrl,
                               static_cast<const ChunkInfo *>(table), seg_first, 0,
-                              static_cast<float *>(nullptr), L.segs);
+                              static_cast<float *>(nullptr), L.segs, rows, L.max_chunks, nseg + 1,
+                              nseg, B, int(L.kda));
   }
   // No tokens: the final state is the initial state.
   prof_record(g_profile.prep, s);
@@ -1339,6 +1864,11 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
 
 #ifdef GDN_TRACE
 // Trace builds only: copy the phase timestamps to `host` (2*64*16 u64).
+extern "C" int gdn_trace_fetch_cta(unsigned long long *host) {
+  return cudaMemcpyFromSymbol(host, gdn::g_gdn_cta_ns, sizeof(gdn::g_gdn_cta_ns)) == cudaSuccess
+             ? 0
+             : -1;
+}
 extern "C" int gdn_trace_fetch(unsigned long long *host) {
   return cudaMemcpyFromSymbol(host, gdn::g_gdn_trace, sizeof(gdn::g_gdn_trace)) == cudaSuccess
              ? 0

@@ -60,9 +60,11 @@ int run_chunk(bool force_simt, bool channel_gate, const void *q, const void *k, 
   int rc = check_chunk_args(q, k, v, g, beta, s0, cu, B, T, H, dk, dv, num_seqs, chunk, dtype,
                             o, sN, ws);
   if (rc != GDN_OK) return rc;
-  const bool tc = !force_simt && !channel_gate && tc_path(dk, dv, chunk, dtype);
+  // bf16 with d_k = d_v = 128 and 64-token chunks runs on the tensor-core
+  // kernels for both gates; everything else on the CUDA-core kernel.
+  const bool tc = !force_simt && tc_path(dk, dv, chunk, dtype);
   const int segs = scan_segments(B, T, H, cu ? num_seqs : 0, chunk, tc, device_sms());
-  const WsLayout L = ws_layout(B, T, H, cu ? num_seqs : 0, chunk, tc, segs);
+  const WsLayout L = ws_layout(B, T, H, cu ? num_seqs : 0, chunk, tc, segs, tc && channel_gate);
   if (ws_bytes < L.total) return GDN_ERR_WORKSPACE;
   const int N = cu ? num_seqs : B;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -130,10 +132,11 @@ int gdn_chunk_fwd_simt(const void *q, const void *k, const void *v, const float 
 
 size_t gdn_kda_chunk_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int num_seqs,
                                         int chunk, int dtype) {
-  (void)dtype;
   if (B < 1 || T < 0 || H < 1 || d_k < 1 || d_v < 1 || num_seqs < 0) return 0;
   if (chunk != 16 && chunk != 32 && chunk != 64) return 0;
-  return ws_layout(B, T, H, num_seqs, chunk, false).total;
+  const bool tc = tc_path(d_k, d_v, chunk, dtype);
+  const int segs = scan_segments(B, T, H, num_seqs, chunk, tc, device_sms());
+  return ws_layout(B, T, H, num_seqs, chunk, tc, segs, tc).total;
 }
 
 int gdn_kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
@@ -141,7 +144,7 @@ int gdn_kda_chunk_fwd(const void *q, const void *k, const void *v, const float *
                       int B, int T, int H, int d_k, int d_v, int num_seqs, int chunk, int dtype,
                       void *o, float *final_state, void *workspace, size_t workspace_bytes,
                       void *stream) {
-  return run_chunk(true, true, q, k, v, g, beta, initial_state, cu_seqlens, B, T, H, d_k, d_v,
+  return run_chunk(false, true, q, k, v, g, beta, initial_state, cu_seqlens, B, T, H, d_k, d_v,
                    num_seqs, chunk, dtype, o, final_state, workspace, workspace_bytes, stream);
 }
 
@@ -225,6 +228,7 @@ int gdn_get_status(void *workspace, void *stream) {
       return GDN_ERR_CUDA;
   }
   if (err & kErrTimeout) return GDN_ERR_DEVICE_TIMEOUT;
+  if (err & kErrBounds) return GDN_ERR_DEVICE_BOUNDS;
   if (err & kErrLayout) return GDN_ERR_CUDA;
   if (err & kErrBadSeqlens) return GDN_ERR_INVALID_ARG;
   return GDN_OK;
@@ -240,6 +244,8 @@ int gdn_set_profile_events(void *ev_start, void *ev_prep, void *ev_scan, void *e
   return GDN_OK;
 }
 
+int gdn_checked_build(void) { return GDN_CHECKS ? 1 : 0; }
+
 const char *gdn_status_string(int status) {
   switch (status) {
     case GDN_OK: return "GDN_OK";
@@ -248,6 +254,7 @@ const char *gdn_status_string(int status) {
     case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE";
     case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
     case GDN_ERR_DEVICE_TIMEOUT: return "GDN_ERR_DEVICE_TIMEOUT";
+    case GDN_ERR_DEVICE_BOUNDS: return "GDN_ERR_DEVICE_BOUNDS";
     default: return "GDN_ERR_UNKNOWN";
   }
 }

@@ -12,6 +12,34 @@ namespace gdn {
 constexpr uint32_t kErrBadSeqlens = 1u;
 constexpr uint32_t kErrTimeout = 2u;
 constexpr uint32_t kErrLayout = 4u;   // shared-memory window not 1024-byte aligned
+constexpr uint32_t kErrBounds = 8u;   // checked builds: an index outside its buffer (access skipped)
+
+// Bounds checks of plain global-memory accesses, compiled in with
+// -DGDN_CHECKS=1 (gdn_checked_build() == 1). GDN_IN_BOUNDS(err, idx, extent)
+// is true when 0 <= idx < extent; otherwise it records kErrBounds in *err
+// (and, the first time, the source line in err[2] and the index in err[3])
+// and is false, so the caller skips the access. Without GDN_CHECKS it is the
+// constant true and costs nothing.
+#ifndef GDN_CHECKS
+#define GDN_CHECKS 0
+#endif
+#ifdef __CUDACC__
+__device__ __forceinline__ bool gdn_bounds_fail(uint32_t *err, long long idx, int line) {
+  if (err && !(atomicOr(err, kErrBounds) & kErrBounds)) {
+    err[2] = uint32_t(line);
+    err[3] = uint32_t(idx);
+  }
+  return false;
+}
+#if GDN_CHECKS
+#define GDN_IN_BOUNDS(err, idx, extent)                                                   \
+  ((static_cast<long long>(idx) >= 0 && static_cast<long long>(idx) < static_cast<long long>(extent)) \
+       ? true                                                                            \
+       : ::gdn::gdn_bounds_fail((err), static_cast<long long>(idx), __LINE__))
+#else
+#define GDN_IN_BOUNDS(err, idx, extent) true
+#endif
+#endif
 
 // One chunk of one sequence (shared by all heads).
 struct ChunkInfo {
@@ -31,14 +59,18 @@ struct ChunkInfo {
 //   tb             bf16 [units][64][64]          T diag(beta) of the chunk (UT transform)
 //   pm             bf16 [units][64][64]          (Q K^T) .* decay mask, diagonal included
 //   gam            fp32 [units][128]             exp(Gamma_c) (64), then exp(Gamma_last - Gamma_s) (64)
+//                  channel-wise gate: fp32 [units][256]: 1 (64), unused (64), then the
+//                  per-channel state decay exp(Gamma_last,j) (128)
+//   qt             channel-wise gate only: bf16 [units][64][d_k]  Q .* exp(Gamma)
 //   tensor-core path with a segmented state scan (segs > 1, see scan_segments):
 //   seg_first      int32[B * segs + 1]  first chunk of each segment
 //   hbuf, pbuf     fp32 [B * segs][H][d_k][d_v]  each segment's state from S = 0,
 //                  and its transition (the state from S = I with V = 0)
 //   sstart         fp32 [B * segs][H][d_k][d_v]  each segment's true start state
 struct WsLayout {
-  size_t chunk_table, seq_first, w, kt, tb, pm, gam, seg_first, hbuf, pbuf, sstart, total;
+  size_t chunk_table, seq_first, w, kt, tb, pm, gam, qt, seg_first, hbuf, pbuf, sstart, total;
   int max_chunks, segs;
+  bool kda;
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -78,8 +110,10 @@ inline int scan_segments(int B, int T, int H, int num_seqs, int chunk, bool tc, 
   return (best > 1 && best_cost * 10 <= plain * 7) ? best : 1;   // at least 30 % faster
 }
 
-inline WsLayout ws_layout(int B, int T, int H, int num_seqs, int chunk, bool tc, int segs = 1) {
+inline WsLayout ws_layout(int B, int T, int H, int num_seqs, int chunk, bool tc, int segs = 1,
+                          bool kda = false) {
   WsLayout L{};
+  L.kda = kda;
   const int N = num_seqs > 0 ? num_seqs : B;
   L.max_chunks = max_chunks_for(B, T, num_seqs, chunk);
   L.segs = segs;
@@ -94,7 +128,10 @@ inline WsLayout ws_layout(int B, int T, int H, int num_seqs, int chunk, bool tc,
     L.kt = off;  off = align_up(off + units * 128 * 64 * 2, 1024);
     L.tb = off;  off = align_up(off + units * 64 * 64 * 2, 1024);
     L.pm = off;  off = align_up(off + units * 64 * 64 * 2, 1024);
-    L.gam = off; off = align_up(off + units * 128 * 4, 1024);
+    L.gam = off; off = align_up(off + units * (kda ? 256 : 128) * 4, 1024);
+    if (kda) {
+      L.qt = off;  off = align_up(off + units * 64 * 128 * 2, 1024);
+    }
     if (segs > 1) {
       const size_t nseg = size_t(B) * segs;
       const size_t states = nseg * H * 128 * 128 * sizeof(float);

@@ -366,6 +366,34 @@ __device__ __forceinline__ void stmatrix_x4_trans(uint32_t saddr, uint32_t r0, u
                : "memory");
 }
 
+// Four 8x8 b16 matrices stored as they are: register r[m] of thread t holds
+// row t/4, columns 2(t%4), 2(t%4)+1 of matrix m; memory row j of matrix m is
+// the 16 bytes at the address thread 8m+j supplies.
+__device__ __forceinline__ void stmatrix_x4(uint32_t saddr, uint32_t r0, uint32_t r1, uint32_t r2,
+                                            uint32_t r3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(saddr),
+               "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+               : "memory");
+}
+
+// Four 8x8 b16 matrices loaded transposed: thread 8m+j supplies the address of
+// memory row j of matrix m (16 bytes), and register r[m] of thread t receives
+// the elements (row 2(t%4), column t/4) and (row 2(t%4)+1, column t/4).
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t saddr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(saddr)
+               : "memory");
+}
+
+// Two bf16 products a * b, each rounded once to nearest even (a fused
+// multiply-add with -0 as the addend leaves the product unchanged).
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(0x80008000u));
+  return d;
+}
+
 // Four (two) 8x8 b16 matrices from shared memory: thread 8m+j supplies the
 // address of row j of matrix m (16 bytes), and register r[m] of thread t
 // receives 32-bit word t%4 of row t/4 of matrix m. Words move intact, so the

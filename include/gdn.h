@@ -47,6 +47,9 @@ extern "C" {
 #define GDN_ERR_WORKSPACE      3  /* workspace missing or smaller than gdn_chunk_fwd_workspace_size() */
 #define GDN_ERR_CUDA           4  /* a CUDA runtime/driver call or kernel launch failed */
 #define GDN_ERR_DEVICE_TIMEOUT 5  /* a bounded device-side wait expired (reported by gdn_get_status) */
+#define GDN_ERR_DEVICE_BOUNDS  6  /* bounds-checked builds only (-DGDN_CHECKS=1): a kernel computed a
+                                     global-memory index outside its buffer and skipped the access
+                                     (reported by gdn_get_status) */
 
 /* Element types of q, k, v, o. */
 #define GDN_BF16 0
@@ -157,8 +160,19 @@ int gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const flo
                           int num_seqs, int chunk, int dtype, void *o, float *final_state,
                           void *stream);
 
-/* Which implementation gdn_chunk_fwd would run for these sizes
- * (GDN_PATH_TCGEN05 or GDN_PATH_SIMT), or a negative value if unsupported. */
+/* 1 if this library was built with device-side bounds checks (-DGDN_CHECKS=1),
+ * else 0. In a checked build the tensor-core chunked forward pass (chunk map,
+ * prep, state scan, segment composition) compares every plain global-memory
+ * index with the extent of its buffer before the access; an index outside it
+ * skips the access and records GDN_ERR_DEVICE_BOUNDS for gdn_get_status. (TMA
+ * copies need no check: the hardware clips them to the tensor map.) It is
+ * the stand-in for a memory checker when none is available; it is slower and
+ * not meant for production. */
+int gdn_checked_build(void);
+
+/* Which implementation gdn_chunk_fwd and gdn_kda_chunk_fwd would run for
+ * these sizes (GDN_PATH_TCGEN05 or GDN_PATH_SIMT), or a negative value if
+ * unsupported. */
 int gdn_chunk_fwd_path(int d_k, int d_v, int chunk, int dtype);
 
 /*
@@ -224,9 +238,16 @@ size_t gdn_kda_chunk_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, i
  *   P_rs = sum_j q_rj k_sj exp(Gamma_rj - Gamma_sj) (s <= r)
  *   O = (Q .* exp(Gamma)) S^T + P V_new
  *   S <- S diag(exp(Gamma_last)) + V_new^T (K .* exp(Gamma_last - Gamma))
- * Runs on the fp32 CUDA-core kernel for every dtype. Arguments, layouts,
- * ownership and errors as gdn_chunk_fwd, except g: [B, T, H, d_k] fp32.
- * Supports d_k, d_v <= 128 and chunk 16, 32 or 64.
+ * bf16 with d_k = d_v = 128 and chunk = 64 runs on the tensor-core kernels:
+ * A and P come from warp-level bf16 tensor-core tiles of operands scaled
+ * against the first row b of each 16-row block, e^(Gamma_r - Gamma_b) and
+ * e^(Gamma_b - Gamma_s), which factor the decay exactly; the rest is the
+ * scalar gate's chunk pipeline with Q .* exp(Gamma) and a per-channel state
+ * decay. Those scalings need e^(15 max|g|) to fit fp32, i.e. |g| < 5.9 per
+ * token and channel (alpha > 0.0028); the fp32 CUDA-core kernel (every other
+ * size and dtype) has no such bound. Arguments, layouts, ownership and errors
+ * as gdn_chunk_fwd, except g: [B, T, H, d_k] fp32. Supports d_k, d_v <= 128
+ * and chunk 16, 32 or 64.
  */
 int gdn_kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
                       const float *beta, const float *initial_state, const int32_t *cu_seqlens,

@@ -36,9 +36,20 @@ def test_library_exports_every_declared_symbol(L):
         assert hasattr(L, name), f"libgdn.so does not export {name}"
 
 
+def test_checked_variant_exports_the_same_symbols():
+    lib = gbuild.build(checked=True)
+    C = ctypes.CDLL(lib)
+    for name in declared_functions():
+        assert hasattr(C, name), f"libgdn_checked.so does not export {name}"
+    C.gdn_checked_build.restype = ctypes.c_int
+    assert C.gdn_checked_build() == 1
+
+
 def test_status_strings(L):
     assert L.gdn_status_string(0) == b"GDN_OK"
     assert L.gdn_status_string(5) == b"GDN_ERR_DEVICE_TIMEOUT"
+    assert L.gdn_status_string(6) == b"GDN_ERR_DEVICE_BOUNDS"
+    assert L.gdn_checked_build() == 0
     assert L.gdn_status_string(99) == b"GDN_ERR_UNKNOWN"
 
 
@@ -137,11 +148,16 @@ def test_kda_entry_points_host_checks(L):
     assert _chunk_call(L, fn=kda, chunk=48) == gdn.ERR_UNSUPPORTED
     assert _chunk_call(L, fn=kda, ws=None) == gdn.ERR_WORKSPACE
     assert _chunk_call(L, fn=kda, wsb=100) == gdn.ERR_WORKSPACE
-    # the channel-wise gate runs on the CUDA-core kernel: its workspace is the
-    # chunk table alone, no per-(chunk, head) intermediates
+    # bf16, d = 128, chunk 64: the tensor-core path, whose workspace holds the
+    # scalar gate's per-(chunk, head) operand tiles plus Q .* exp(Gamma) (16 KB)
+    # and a 1 KB decay record (256 fp32) instead of 512 B
     kws = L.gdn_kda_chunk_fwd_workspace_size(4, 4096, 16, 128, 128, 0, 64, gdn.BF16)
-    assert kws == L.gdn_chunk_fwd_workspace_size(4, 4096, 16, 128, 128, 0, 64, gdn.F32)
-    assert 0 < kws < (1 << 20)
+    sws = L.gdn_chunk_fwd_workspace_size(4, 4096, 16, 128, 128, 0, 64, gdn.BF16)
+    assert kws == sws + 4096 * (16384 + 512)
+    # every other size and dtype: the CUDA-core kernel, chunk table alone
+    fws = L.gdn_kda_chunk_fwd_workspace_size(4, 4096, 16, 128, 128, 0, 64, gdn.F32)
+    assert fws == L.gdn_chunk_fwd_workspace_size(4, 4096, 16, 128, 128, 0, 64, gdn.F32)
+    assert 0 < fws < (1 << 20)
     assert L.gdn_kda_chunk_fwd_workspace_size(1, 10, 1, 128, 128, 0, 48, gdn.BF16) == 0
     vp = ctypes.c_void_p
     p = vp(1 << 20)

@@ -63,6 +63,63 @@ def test_kda_bf16_varlen_odd_lengths_with_states():
     check(inp, TOL_BF16)
 
 
+# ---------------------------------------------------------------- tensor-core path
+KDA_TC = Workload("kda_tc", B=1, T=64, H=1, d_k=128, d_v=128, seed=24, gate="channel")
+
+
+def test_kda_tc_path_is_selected():
+    import gated_delta_rule_112_b200 as gdn
+    assert gdn.chunk_path(128, 128, 64, torch.bfloat16) == gdn.PATH_TCGEN05
+    tc = gdn.lib().gdn_kda_chunk_fwd_workspace_size(1, 64, 1, 128, 128, 0, 64, gdn.BF16)
+    simt = gdn.lib().gdn_kda_chunk_fwd_workspace_size(1, 64, 1, 128, 128, 0, 64, gdn.F32)
+    assert tc > simt          # the tensor-core layout holds the per-chunk operand tiles
+    # The tensor-core kernels run the chunk on bf16 operand tiles, so the state
+    # carries their rounding; the fp32 CUDA-core kernel agrees with the fp64
+    # oracle to about 1e-6. Both stay within the bf16 tolerance.
+    inp = make_chunk_inputs(KDA_TC, T=200, H=2, random_state=True)
+    _, fs = gpu_kda(inp)
+    _, rfs = oracle_kda(inp)
+    assert 2e-5 < rel_l2(np64(fs), rfs) < TOL_BF16
+
+
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 200])
+def test_kda_tc_ragged_lengths(T):
+    check(make_chunk_inputs(KDA_TC, T=T, H=2, random_state=True), TOL_BF16)
+
+
+def test_kda_tc_batch_heads_with_initial_state():
+    check(make_chunk_inputs(KDA_TC, B=3, H=3, T=257, random_state=True), TOL_BF16)
+
+
+def test_kda_tc_strong_decay():
+    # log alpha ~ -softplus(N(3, 1)) per token and channel: within a chunk the
+    # decay reaches exp(-200); the block-scaled factors stay within fp32.
+    check(make_chunk_inputs(KDA_TC, B=2, H=2, T=192, random_state=True, gate_mu=3.0), TOL_BF16)
+
+
+def test_kda_tc_segmented_scan():
+    import gated_delta_rule_112_b200 as gdn
+    inp = make_chunk_inputs(KDA_TC, B=1, H=1, T=64 * 40 + 37, random_state=True)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert gdn.lib().gdn_chunk_fwd_scan_segments(1, inp["T"], 1, 128, 128, 0, 64, gdn.BF16,
+                                                 sms) > 1
+    check(inp, TOL_BF16)
+
+
+def test_kda_tc_equal_channels_match_the_scalar_gate():
+    import gated_delta_rule_112_b200 as gdn
+    inp = make_chunk_inputs(KDA_TC, B=2, H=2, T=160, random_state=True)
+    gs = inp["g"][..., 0].contiguous()
+    inp["g"] = gs[..., None].expand(-1, -1, -1, 128).contiguous()
+    o1, f1 = gpu_kda(inp)
+    d = to_dev(inp)
+    o2, f2 = gdn.chunk_fwd(d["q"], d["k"], d["v"], gs.cuda(), d["beta"], d["initial_state"])
+    torch.cuda.synchronize()
+    # both on bf16 tensor-core tiles, with different roundings of the decays
+    assert rel_l2(np64(o1), np64(o2)) < TOL_BF16
+    assert rel_l2(np64(f1), np64(f2)) < TOL_BF16
+
+
 def test_kda_empty_sequences_keep_their_state():
     inp = make_chunk_inputs(SMALL, H=2, lengths=[0, 40, 0, 3], random_state=True)
     o, fs = check(inp, TOL_F32)
