@@ -19,6 +19,7 @@ library is measured on:
 * ``kda_decode``  the decode shape with the channel-wise gate, seed 7
 * ``b1h16t1024``  one sequence of the b4h16t4096 kind, 1024 tokens, seed 8: a
   small case of the same kernels for full profiler captures
+* ``kda_b1h16t1024`` the same with the channel-wise gate, seed 9
 
 Distributions (all drawn in fp32 with ``torch.Generator('cpu')``):
 q, k ~ N(0, 1) then L2-normalised per (token, head) over d_k; v ~ N(0, 1);
@@ -76,6 +77,8 @@ WORKLOADS = {
     "b1h16t1024": Workload("b1h16t1024", B=1, T=1024, H=16, d_k=128, d_v=128, seed=8),
     "kda_decode": Workload("kda_decode", B=256, T=1, H=32, d_k=128, d_v=128,
                            random_state=True, seed=7, steps=64, gate="channel"),
+    "kda_b1h16t1024": Workload("kda_b1h16t1024", B=1, T=1024, H=16, d_k=128, d_v=128, seed=9,
+                               gate="channel"),
 }
 
 
