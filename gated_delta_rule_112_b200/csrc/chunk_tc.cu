@@ -634,25 +634,32 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
 // tcgen05. The state scan then consumes the same operand tiles, with
 // Q .* e^Gamma in place of Q (gamma = 1 in the decay record) and the
 // per-channel state decay e^Gamma_last.
-constexpr uint32_t kK_KQ = 0;                          // K, Q (bf16, 128-byte swizzle) as in prep
-constexpr uint32_t kK_GM = kK_KQ + 2 * kTile128x64;    // Gamma fp32 [64][128]
-constexpr uint32_t kK_LK = kK_GM + 64 * 128 * 4;       // left operands bf16 [64][128] (256-B rows)
-constexpr uint32_t kK_LQ = kK_LK + 64 * 256;
-constexpr uint32_t kK_RR = kK_LQ + 64 * 256;           // right operand of block row R
-constexpr uint32_t kK_DK = kK_RR + 64 * 256;           // (D K)^T staging [128][64]
-constexpr uint32_t kK_AS = kK_DK + kTile128x64;        // A fp32 [64][68]
-constexpr uint32_t kK_TS = kK_AS + 64 * kLd * 4;       // T fp32 [64][68]
-constexpr uint32_t kK_XS = kK_TS + 64 * kLd * 4;       // solve scratch fp32 [32][36]
-constexpr uint32_t kK_TT = kK_XS + 32 * kLy * 4;       // solve: T transposed fp32 [48][36]
-constexpr uint32_t kK_TB = (kK_TT + 48 * kLy * 4 + 1023) / 1024 * 1024;   // T diag(beta) bf16
-constexpr uint32_t kK_PST = kK_TB + kTile64x64;        // P staging bf16 [64][64]
-constexpr uint32_t kK_VEC = kK_PST + kTile64x64;       // beta[64], e^Gamma_last[128]
+// Shared memory holds one unit at a time, laid out for two CTAs per SM
+// (each CTA: this window, 1 KB of static shared memory and the 1 KB the
+// hardware reserves); areas are reused once their last reader is done. P
+// goes to global memory straight from the mma fragments.
+constexpr uint32_t kK_KQ = 0;                          // K, Q (bf16, 128-byte swizzle) as in prep;
+                                                       // later Q .* e^Gamma, K .* e^Gamma, -W
+constexpr uint32_t kK_GM = kK_KQ + 2 * kTile128x64;    // log2(e) Gamma fp32 [64][128]; then the
+                                                       // solve's T, T^T blocks and scratch
+constexpr uint32_t kK_AS = kK_GM + 64 * 128 * 4;       // A fp32 [64][68]
+constexpr uint32_t kK_RR = (kK_AS + 64 * kLd * 4 + 1023) / 1024 * 1024;   // right operand of
+                                                       // block row R [64][128] (256-B rows);
+                                                       // later the (D K)^T staging [128][64]
+constexpr uint32_t kK_LK = kK_RR + 64 * 256;           // left operands of block row R [16][128]
+constexpr uint32_t kK_LQ = kK_LK + 16 * 256;           // (LK, LQ: later T diag(beta) bf16)
+constexpr uint32_t kK_VEC = kK_LQ + 16 * 256;          // beta[64], e^Gamma_last[128]
 constexpr uint32_t kK_BAR = kK_VEC + 192 * 4;
 constexpr uint32_t kKdaPrepSmem = kK_BAR + 64;         // the dynamic window starts 1024-aligned (checked)
+constexpr uint32_t kK_TS = kK_GM;                      // solve: T fp32 [64][68]
+constexpr uint32_t kK_TT = kK_TS + 64 * kLd * 4;       // solve: T transposed fp32 [48][36]
+constexpr uint32_t kK_XS = kK_TT + 48 * kLy * 4;       // solve scratch fp32 [32][36]
+constexpr uint32_t kK_TB = kK_LK;
 constexpr int kKdaPrepThreads = 256;
-static_assert(kK_LK % 1024 == 0 && kK_RR % 1024 == 0 && kK_DK % 1024 == 0 &&
-                  kK_TB % 1024 == 0 && kK_PST % 1024 == 0 && kKdaPrepSmem <= 232448,
-              "channel-wise prep layout");
+static_assert(kK_GM % 1024 == 0 && kK_RR % 1024 == 0 && kK_LK % 1024 == 0 &&
+                  kK_XS + 32 * kLy * 4 <= kK_AS && 2 * 16 * 256 >= kTile64x64 &&
+                  kTile128x64 <= 64 * 256 && 2 * (kKdaPrepSmem + 2048) <= 233472,
+              "channel-wise prep layout: two CTAs per SM");
 
 // Byte offset of 16-byte chunk c (0..15) of row r in a [rows][128 bf16] tile
 // with 256-byte rows, XOR-swizzled so that 8 consecutive rows at the same
@@ -683,14 +690,26 @@ __device__ __forceinline__ uint4 scale8(uint4 x, const float (&f)[8]) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-__global__ void __launch_bounds__(kKdaPrepThreads, 1) gdn_kda_prep_kernel(
+// 2^(a_x - b_x) for the eight channels of two float4 pairs.
+__device__ __forceinline__ void ex2_diff8(float (&f)[8], float4 a0, float4 a1, float4 b0,
+                                          float4 b1) {
+  f[0] = ex2_approx(a0.x - b0.x);
+  f[1] = ex2_approx(a0.y - b0.y);
+  f[2] = ex2_approx(a0.z - b0.z);
+  f[3] = ex2_approx(a0.w - b0.w);
+  f[4] = ex2_approx(a1.x - b1.x);
+  f[5] = ex2_approx(a1.y - b1.y);
+  f[6] = ex2_approx(a1.z - b1.z);
+  f[7] = ex2_approx(a1.w - b1.w);
+}
+
+__global__ void __launch_bounds__(kKdaPrepThreads, 2) gdn_kda_prep_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_kt,
-    const __grid_constant__ CUtensorMap tm_tb, const __grid_constant__ CUtensorMap tm_pm,
-    const __grid_constant__ CUtensorMap tm_qt, const float *__restrict__ g,
-    const float *__restrict__ beta, float *__restrict__ gam_out, int H,
-    uint32_t *__restrict__ ctrl, const ChunkInfo *__restrict__ table, long long rows,
-    int max_chunks) {
+    const __grid_constant__ CUtensorMap tm_tb, const __grid_constant__ CUtensorMap tm_qt,
+    const float *__restrict__ g, const float *__restrict__ beta, float *__restrict__ gam_out,
+    uint32_t *__restrict__ pm_out, int H, uint32_t *__restrict__ ctrl,
+    const ChunkInfo *__restrict__ table, long long rows, int max_chunks) {
   (void)rows;
   (void)max_chunks;   // extents of the bounds checks (GDN_CHECKS builds)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -703,7 +722,7 @@ __global__ void __launch_bounds__(kKdaPrepThreads, 1) gdn_kda_prep_kernel(
     if (tid == 0) atomicOr(ctrl, kErrLayout);
     return;
   }
-  float *Gm = reinterpret_cast<float *>(sm + kK_GM);
+  float *Gm = reinterpret_cast<float *>(sm + kK_GM);   // log2(e) Gamma
   float *As = reinterpret_cast<float *>(sm + kK_AS);
   float *Ts = reinterpret_cast<float *>(sm + kK_TS);
   float *Xs = reinterpret_cast<float *>(sm + kK_XS);
@@ -732,12 +751,14 @@ __global__ void __launch_bounds__(kKdaPrepThreads, 1) gdn_kda_prep_kernel(
   const uint32_t tmem = *tmem_slot;
   grid_dependency_wait();
   const int nunits = (ctrl[0] & kErrBadSeqlens) ? 0 : int(ctrl[1]) * H;
+  const long long pm_words = (long long)max_chunks * H * (64 * 64 / 2);
   int it = 0;
   for (int unit = blockIdx.x; unit < nunits; unit += gridDim.x, ++it) {
     const int chunk = unit / H, h = unit - chunk * H;
     const ChunkInfo ci =
         GDN_IN_BOUNDS(ctrl, chunk, max_chunks) ? table[chunk] : ChunkInfo{0, 0, 0, 0};
     const int L = ci.len;
+    uint32_t *pm = pm_out + (long long)unit * (64 * 64 / 2);   // P of this unit, [64][64] bf16
     if (tid == 0) {
       // The previous unit's stores must have read the areas reused below.
       tma_store_wait_read();
@@ -749,7 +770,7 @@ __global__ void __launch_bounds__(kKdaPrepThreads, 1) gdn_kda_prep_kernel(
         tma_load_3d(sm + kK_KQ + kTile128x64 + kTile64x64, &tm_q, bar_load, 64, h, ci.row0);
       }
     }
-    __syncthreads();   // every thread is past the previous unit's reads of Gm and PST
+    __syncthreads();   // every thread is past the previous unit's reads of Gm, RR, LK, LQ
     // g of the chunk (rows past the sequence end read as 0) and beta.
     for (int e = tid; e < 64 * 32; e += kKdaPrepThreads) {
       const int r = e >> 5, c4 = e & 31;
@@ -763,19 +784,25 @@ __global__ void __launch_bounds__(kKdaPrepThreads, 1) gdn_kda_prep_kernel(
       const long long idx = (long long)(ci.row0 + tid) * H + h;
       Bt[tid] = (tid < L && GDN_IN_BOUNDS(ctrl, idx, rows * H)) ? beta[idx] : 0.f;
     }
-    // P staging starts at zero: blocks above the diagonal are never written.
-    for (int e = tid; e < kTile64x64 / 16; e += kKdaPrepThreads)
-      *reinterpret_cast<uint4 *>(sm + kK_PST + 16 * e) = make_uint4(0, 0, 0, 0);
+    // P is zero above its diagonal 16 x 16 blocks: blocks (R, S), S > R, are
+    // written here, the others by the block-row products below.
+    if (tid < 192) {
+      const int bi = tid >> 5, rr = (tid >> 1) & 15, half = tid & 1;
+      const int R = bi < 3 ? 0 : (bi < 5 ? 1 : 2), S = bi < 3 ? bi + 1 : (bi < 5 ? bi - 1 : 3);
+      const long long wi = (long long)(16 * R + rr) * 32 + 8 * S + 4 * half;
+      if (GDN_IN_BOUNDS(ctrl, (long long)unit * 2048 + wi + 3, pm_words))
+        *reinterpret_cast<uint4 *>(pm + wi) = make_uint4(0, 0, 0, 0);
+    }
     __syncthreads();
-    // Gamma: inclusive cumsum over the tokens, one thread per channel.
+    // log2(e) Gamma: inclusive cumsum over the tokens, one thread per channel.
     if (tid < 128) {
       float acc = 0.f;
 #pragma unroll 8
       for (int r = 0; r < 64; ++r) {
-        acc += Gm[r * 128 + tid];
+        acc = fmaf(Gm[r * 128 + tid], kLog2e, acc);
         Gm[r * 128 + tid] = acc;
       }
-      El[tid] = expf(acc);
+      El[tid] = ex2_approx(acc);
     }
     const bool loaded = mbar_wait(bar_load, it & 1, ctrl, &abort_flag);
     if (loaded && L < kC) {
@@ -790,73 +817,27 @@ __global__ void __launch_bounds__(kKdaPrepThreads, 1) gdn_kda_prep_kernel(
       }
     }
     __syncthreads();
-    // Left operands K and Q .* e^(Gamma_r - Gamma_b(r)) and Q .* e^Gamma (in
-    // place of Q). Pair (row r, 16-byte chunk c) = channels 8 c .. 8 c + 7.
-    for (int e = tid; e < 64 * 16; e += kKdaPrepThreads) {
-      const int r = e >> 4, c = e & 15, b = r & ~15;
-      const uint32_t kq = kK_KQ + (c >> 3) * kTile128x64 + sw128_offset(r, c & 7);
-      const float *gr = Gm + r * 128 + 8 * c, *gb = Gm + b * 128 + 8 * c;
-      const float4 r0 = lds4(gr), r1 = lds4(gr + 4), b0 = lds4(gb), b1 = lds4(gb + 4);
-      const float gv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-      float f1[8], fg[8];
-#pragma unroll
-      for (int x = 0; x < 8; ++x) {
-        f1[x] = ex2_approx((gv[x] - bv[x]) * kLog2e);
-        fg[x] = ex2_approx(gv[x] * kLog2e);
-      }
-      const uint4 kx = *reinterpret_cast<const uint4 *>(sm + kq);
-      const uint4 qx = *reinterpret_cast<const uint4 *>(sm + kq + kTile64x64);
-      *reinterpret_cast<uint4 *>(sm + kK_LK + sw256(r, c)) = scale8(kx, f1);
-      *reinterpret_cast<uint4 *>(sm + kK_LQ + sw256(r, c)) = scale8(qx, f1);
-      *reinterpret_cast<uint4 *>(sm + kq + kTile64x64) = scale8(qx, fg);
-    }
-    // (D K)^T with D_sj = e^(Gamma_last,j - Gamma_sj), straight from the K tile
-    // (ldmatrix.trans gives thread t tokens s, s + 1 of d_k row t / 4); warp w
-    // owns d_k rows [16 w, 16 w + 16).
-    {
-      const int mj = lane & 7, mm = lane >> 3, sp = 2 * (lane & 3), jq = lane >> 2;
-      const uint32_t kq = smem_u32(sm + kK_KQ), kst = smem_u32(sm + kK_DK);
-#pragma unroll
-      for (int it2 = 0; it2 < 4; ++it2) {
-        const int jb = 2 * warp + (mm & 1), sb = 2 * it2 + (mm >> 1);
-        uint32_t x[4];
-        ldsm_x4_trans(kq + (jb >> 3) * kTile128x64 + sw128_offset(8 * sb + mj, jb & 7), x);
-        uint32_t y[4];
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const int j = 8 * (2 * warp + (m & 1)) + jq, s0 = 8 * (2 * it2 + (m >> 1)) + sp;
-          const float gl = Gm[63 * 128 + j];
-          const float d0 = ex2_approx((gl - Gm[s0 * 128 + j]) * kLog2e);
-          const float d1 = ex2_approx((gl - Gm[(s0 + 1) * 128 + j]) * kLog2e);
-          y[m] = pack_bf16x2(__uint_as_float(x[m] << 16) * d0,
-                             __uint_as_float(x[m] & 0xffff0000u) * d1);
-        }
-        stmatrix_x4(kst + sw128_offset(8 * jb + mj, sb), y[0], y[1], y[2], y[3]);
-      }
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0 && !abort_flag) {
-      tma_store_2d(&tm_qt, sm + kK_KQ + kTile64x64, 0, unit * kC);
-      tma_store_2d(&tm_qt, sm + kK_KQ + kTile128x64 + kTile64x64, 64, unit * kC);
-      tma_store_2d(&tm_kt, sm + kK_DK, 0, unit * kD);
-      tma_store_commit();
-    }
-    // A and P, one 16-row block row at a time.
+    // A and P, one 16-row block row R at a time, b = 16 R.
     for (int R = 0; R < 4; ++R) {
-      const int nrow = 16 * R + 16;
-      // right operand: K rows s < 16 R + 16 scaled by e^(Gamma_16R - Gamma_s)
+      const int b = 16 * R, nrow = b + 16;
+      {  // left operands: rows of block R, K and Q .* e^(Gamma_r - Gamma_b); one pair per thread
+        const int r = b + (tid >> 4), c = tid & 15;
+        const uint32_t kq = kK_KQ + (c >> 3) * kTile128x64 + sw128_offset(r, c & 7);
+        const float *gr = Gm + r * 128 + 8 * c, *gb = Gm + b * 128 + 8 * c;
+        float f[8];
+        ex2_diff8(f, lds4(gr), lds4(gr + 4), lds4(gb), lds4(gb + 4));
+        *reinterpret_cast<uint4 *>(sm + kK_LK + sw256(r - b, c)) =
+            scale8(*reinterpret_cast<const uint4 *>(sm + kq), f);
+        *reinterpret_cast<uint4 *>(sm + kK_LQ + sw256(r - b, c)) =
+            scale8(*reinterpret_cast<const uint4 *>(sm + kq + kTile64x64), f);
+      }
+      // right operand: K rows s < b + 16 scaled by e^(Gamma_b - Gamma_s)
       for (int e = tid; e < nrow * 16; e += kKdaPrepThreads) {
         const int s = e >> 4, c = e & 15;
         const uint32_t kq = kK_KQ + (c >> 3) * kTile128x64 + sw128_offset(s, c & 7);
-        const float *gs = Gm + s * 128 + 8 * c, *gb = Gm + 16 * R * 128 + 8 * c;
-        const float4 s0 = lds4(gs), s1 = lds4(gs + 4), b0 = lds4(gb), b1 = lds4(gb + 4);
-        const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-        const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        const float *gs = Gm + s * 128 + 8 * c, *gb = Gm + b * 128 + 8 * c;
         float f[8];
-#pragma unroll
-        for (int x = 0; x < 8; ++x) f[x] = ex2_approx((bv[x] - sv[x]) * kLog2e);
+        ex2_diff8(f, lds4(gb), lds4(gb + 4), lds4(gs), lds4(gs + 4));
         *reinterpret_cast<uint4 *>(sm + kK_RR + sw256(s, c)) =
             scale8(*reinterpret_cast<const uint4 *>(sm + kq), f);
       }
@@ -868,8 +849,8 @@ __global__ void __launch_bounds__(kKdaPrepThreads, 1) gdn_kda_prep_kernel(
         const uint32_t left = smem_u32(sm + (isP ? kK_LQ : kK_LK));
         const uint32_t right = smem_u32(sm + kK_RR);
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        const int ar = 16 * R + (lane & 7) + 8 * ((lane >> 3) & 1);   // A fragment row
-        const int brow = 8 * nt + (lane & 7);                          // B fragment row (= column s)
+        const int ar = (lane & 7) + 8 * ((lane >> 3) & 1);   // A fragment row within the block
+        const int brow = 8 * nt + (lane & 7);                // B fragment row (= column s)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           uint32_t a[4], bb[2];
@@ -878,7 +859,7 @@ __global__ void __launch_bounds__(kKdaPrepThreads, 1) gdn_kda_prep_kernel(
           mma_bf16_16816(acc, a, bb[0], bb[1]);
         }
         const int gq = lane >> 2, tq = lane & 3;
-        const int r0 = 16 * R + gq, s0 = 8 * nt + 2 * tq;
+        const int r0 = b + gq, s0 = 8 * nt + 2 * tq;
         if (!isP) {
           const float b0 = Bt[r0], b1 = Bt[r0 + 8];
           *reinterpret_cast<float2 *>(As + r0 * kLd + s0) = make_float2(b0 * acc[0], b0 * acc[1]);
@@ -888,29 +869,60 @@ __global__ void __launch_bounds__(kKdaPrepThreads, 1) gdn_kda_prep_kernel(
           const uint32_t p0 = pack_bf16x2(s0 <= r0 ? acc[0] : 0.f, s0 + 1 <= r0 ? acc[1] : 0.f);
           const uint32_t p1 =
               pack_bf16x2(s0 <= r0 + 8 ? acc[2] : 0.f, s0 + 1 <= r0 + 8 ? acc[3] : 0.f);
-          *reinterpret_cast<uint32_t *>(sm + kK_PST + sw128_offset(r0, s0 >> 3) + 2 * (s0 & 7)) = p0;
-          *reinterpret_cast<uint32_t *>(sm + kK_PST + sw128_offset(r0 + 8, s0 >> 3) +
-                                        2 * (s0 & 7)) = p1;
+          const long long w0 = (long long)r0 * 32 + (s0 >> 1);
+          if (GDN_IN_BOUNDS(ctrl, (long long)unit * 2048 + w0 + 8 * 32, pm_words)) {
+            pm[w0] = p0;
+            pm[w0 + 8 * 32] = p1;
+          }
         }
       }
-      fence_proxy_async_smem();   // P staging rows -> the TMA store below
-      __syncthreads();
+      __syncthreads();   // LK, LQ and RR are rewritten by the next block row
     }
-    // P is complete; K .* e^Gamma replaces K (the W operand).
-    if (tid == 0 && !abort_flag) {
-      tma_store_2d(&tm_pm, sm + kK_PST, 0, unit * kC);
-      tma_store_commit();
+    // (D K)^T with D_sj = e^(Gamma_last,j - Gamma_sj), straight from the K tile
+    // (ldmatrix.trans gives thread t tokens s, s + 1 of d_k row t / 4), staged
+    // in the right-operand area; warp w owns d_k rows [16 w, 16 w + 16).
+    {
+      const int mj = lane & 7, mm = lane >> 3, sp = 2 * (lane & 3), jq = lane >> 2;
+      const uint32_t kq = smem_u32(sm + kK_KQ), kst = smem_u32(sm + kK_RR);
+#pragma unroll
+      for (int it2 = 0; it2 < 4; ++it2) {
+        const int jb = 2 * warp + (mm & 1), sb = 2 * it2 + (mm >> 1);
+        uint32_t x[4];
+        ldsm_x4_trans(kq + (jb >> 3) * kTile128x64 + sw128_offset(8 * sb + mj, jb & 7), x);
+        uint32_t y[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int j = 8 * (2 * warp + (m & 1)) + jq, s0 = 8 * (2 * it2 + (m >> 1)) + sp;
+          const float gl = Gm[63 * 128 + j];
+          const float d0 = ex2_approx(gl - Gm[s0 * 128 + j]);
+          const float d1 = ex2_approx(gl - Gm[(s0 + 1) * 128 + j]);
+          y[m] = pack_bf16x2(__uint_as_float(x[m] << 16) * d0,
+                             __uint_as_float(x[m] & 0xffff0000u) * d1);
+        }
+        stmatrix_x4(kst + sw128_offset(8 * jb + mj, sb), y[0], y[1], y[2], y[3]);
+      }
     }
+    __syncthreads();   // every read of the plain K tile is done
+    // Q .* e^Gamma (the scan's Q) and K .* e^Gamma (the W operand), in place.
     for (int e = tid; e < 64 * 16; e += kKdaPrepThreads) {
       const int r = e >> 4, c = e & 15;
       const uint32_t kq = kK_KQ + (c >> 3) * kTile128x64 + sw128_offset(r, c & 7);
       const float *gr = Gm + r * 128 + 8 * c;
       const float4 r0 = lds4(gr), r1 = lds4(gr + 4);
-      const float f[8] = {ex2_approx(r0.x * kLog2e), ex2_approx(r0.y * kLog2e),
-                          ex2_approx(r0.z * kLog2e), ex2_approx(r0.w * kLog2e),
-                          ex2_approx(r1.x * kLog2e), ex2_approx(r1.y * kLog2e),
-                          ex2_approx(r1.z * kLog2e), ex2_approx(r1.w * kLog2e)};
+      const float f[8] = {ex2_approx(r0.x), ex2_approx(r0.y), ex2_approx(r0.z),
+                          ex2_approx(r0.w), ex2_approx(r1.x), ex2_approx(r1.y),
+                          ex2_approx(r1.z), ex2_approx(r1.w)};
       *reinterpret_cast<uint4 *>(sm + kq) = scale8(*reinterpret_cast<const uint4 *>(sm + kq), f);
+      *reinterpret_cast<uint4 *>(sm + kq + kTile64x64) =
+          scale8(*reinterpret_cast<const uint4 *>(sm + kq + kTile64x64), f);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();   // Gamma is dead: the solve's scratch takes its place
+    if (tid == 0 && !abort_flag) {
+      tma_store_2d(&tm_qt, sm + kK_KQ + kTile64x64, 0, unit * kC);
+      tma_store_2d(&tm_qt, sm + kK_KQ + kTile128x64 + kTile64x64, 64, unit * kC);
+      tma_store_2d(&tm_kt, sm + kK_RR, 0, unit * kD);
+      tma_store_commit();
     }
     solve_unit_lower_64(As, Ts, Tt, Xs, tid);   // ends with __syncthreads
     // T diag(beta), bf16 K-major (T is lower triangular; its upper blocks are
@@ -1781,7 +1793,7 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     if (e != cudaSuccess) return e;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    const long long prep_ctas = std::min<long long>(units, (L.kda ? 1LL : 3LL) * sms);
+    const long long prep_ctas = std::min<long long>(units, (L.kda ? 2LL : 3LL) * sms);
     // Both kernels start with programmatic dependent launch: their prologues
     // overlap the tail of the kernel before them.
     cudaLaunchAttribute pdl[1];
@@ -1795,8 +1807,9 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     cfg.attrs = pdl;
     cfg.numAttrs = 1;
     if (L.kda)
-      e = cudaLaunchKernelEx(&cfg, gdn_kda_prep_kernel, mq, mk, mw, mkt, mtb, mpm, mqt, g, beta,
-                             reinterpret_cast<float *>(base + L.gam), H, ctrl, table, rows,
+      e = cudaLaunchKernelEx(&cfg, gdn_kda_prep_kernel, mq, mk, mw, mkt, mtb, mqt, g, beta,
+                             reinterpret_cast<float *>(base + L.gam),
+                             reinterpret_cast<uint32_t *>(base + L.pm), H, ctrl, table, rows,
                              L.max_chunks);
     else
       e = cudaLaunchKernelEx(&cfg, gdn_prep_kernel, mq, mk, mw, mkt, mtb, mpm, g, beta,

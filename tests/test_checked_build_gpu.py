@@ -45,6 +45,26 @@ def _cases():
             assert_close("final_state", np64(fs), rfs, TOL_BF16)
         else:
             assert np.array_equal(np64(fs), np64(inp["initial_state"]))
+    # the channel-wise gate's tensor-core path (its own prep kernel)
+    import oracle
+    wk = Workload("chk_kda", B=1, T=64, H=1, d_k=128, d_v=128, seed=72, gate="channel")
+    for inp in (make_chunk_inputs(wk, B=2, H=3, T=193, random_state=True),
+                make_chunk_inputs(wk, H=2, lengths=[70, 0, 1, 130, 64], random_state=True)):
+        d = to_dev(inp)
+        num_seqs = inp["num_seqs"] if inp["cu_seqlens"] is not None else 0
+        ws = torch.empty(gdn.kda_workspace_size(inp["B"], inp["T"], inp["H"], 128, 128, num_seqs),
+                         dtype=torch.uint8, device="cuda")
+        o, fs = gdn.kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"],
+                                  d["initial_state"], d["cu_seqlens"], workspace=ws)
+        status = gdn.get_status(ws)
+        assert status == gdn.OK, gdn.lib().gdn_status_string(status)
+        cu = inp["cu_seqlens"]
+        ro, rfs = oracle.kda_chunk_fwd(np64(inp["q"]), np64(inp["k"]), np64(inp["v"]),
+                                       np64(inp["g"]), np64(inp["beta"]),
+                                       np64(inp["initial_state"]),
+                                       None if cu is None else cu.numpy())
+        assert_close("o", np64(o), ro, TOL_BF16)
+        assert_close("final_state", np64(fs), rfs, TOL_BF16)
     print("checked build: all cases clean")
 
 
