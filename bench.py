@@ -346,12 +346,10 @@ def main():
         segs = int(L.gdn_chunk_fwd_scan_segments(
             B, T, H, 128, 128, 0 if cu is None else nseq, 64, gdn.BF16,
             torch.cuda.get_device_properties(dev).multi_processor_count))
-        pieces = gdn.chunk_pieces(B, T, H, 128, 128, 0 if cu is None else nseq)
-        launches = (1 + 2 * pieces) if segs <= 1 else 5
+        launches = 3 if segs <= 1 else 5
         return dict(inp=inp, kda=kda, fwd=fwd, t=t, s0=s0, cu=cu, o=o, ws=ws, B=B, T=T, H=H,
                     nseq=nseq, tokens=tokens, ms=ms, ms_local=ms_local, alg_bytes=alg_bytes,
-                    flops=flops, kernels=kernels, clocks=clocks, launches=launches, segs=segs,
-                    pieces=pieces)
+                    flops=flops, kernels=kernels, clocks=clocks, launches=launches, segs=segs)
 
     def workload_summary(r, steps):
         gbs = r["alg_bytes"] / (r["ms_local"] * 1e-3) / 1e9
@@ -360,7 +358,6 @@ def main():
                 "sequences": r["nseq"], "ms_per_step": r["ms"], "steps": steps,
                 "value": job_value(r["tokens"], r["ms"]) / 1e6, "unit": UNIT,
                 "gpu_launches": r["launches"] * steps, "scan_segments": r["segs"],
-                "pipeline_pieces": r["pieces"],
                 "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
                              "frac": gbs / pk["hbm"], "algorithmic_bytes": r["alg_bytes"],
                              "traffic": recorded_traffic("chunk_fwd_step/" + r["wname"]),
@@ -569,9 +566,7 @@ def main():
         "kernels_ms": kernels,
         "kernel_share": {k2: v2 / tot for k2, v2 in kernels.items()},
         "kernels_note": "per-kernel times from an untimed pass with events between the "
-                        "launches, run as one piece (no launch overlap); ms_per_step is the "
-                        "timed region, where prep and scan overlap in pipeline_pieces pieces",
-        "pipeline_pieces": main_r["pieces"],
+                        "launches (no launch overlap); ms_per_step is the timed region",
         "gpu_launches": main_r["launches"] * K,
         "clocks": clocks,
         "e2e": e2e,

@@ -14,8 +14,7 @@ import os
 
 import torch
 
-__all__ = ["chunk_fwd", "decode_step", "workspace_size", "chunk_path", "chunk_pieces",
-           "set_chunk_pipeline", "get_status",
+__all__ = ["chunk_fwd", "decode_step", "workspace_size", "chunk_path", "get_status",
            "lib", "GdnError", "BF16", "F32", "PATH_TCGEN05", "PATH_SIMT"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -64,10 +63,6 @@ def lib() -> ctypes.CDLL:
         L.gdn_chunk_fwd_workspace_size.restype = sz
         L.gdn_chunk_fwd_scan_segments.argtypes = [ci] * 9
         L.gdn_chunk_fwd_scan_segments.restype = ci
-        L.gdn_chunk_fwd_pieces.argtypes = [ci] * 9 + [vp]
-        L.gdn_chunk_fwd_pieces.restype = ci
-        L.gdn_set_chunk_pipeline.argtypes = [ci]
-        L.gdn_set_chunk_pipeline.restype = ci
         L.gdn_selftest_wait_timeout.argtypes = [vp, vp]
         L.gdn_selftest_wait_timeout.restype = ci
         L.gdn_chunk_fwd_path.argtypes = [ci] * 4
@@ -122,29 +117,6 @@ def _check(code: int, what: str):
 def workspace_size(B, T, H, d_k, d_v, num_seqs=0, chunk=64, dtype=torch.bfloat16) -> int:
     return int(lib().gdn_chunk_fwd_workspace_size(B, T, H, d_k, d_v, num_seqs, chunk,
                                                   _dtype_code(dtype)))
-
-
-def chunk_pieces(B, T, H, d_k, d_v, num_seqs=0, chunk=64, dtype=torch.bfloat16, sms=None,
-                 bounds=False):
-    """Pieces the tensor-core path pipelines a call of these sizes into (1 =
-    none) on a device with `sms` SMs (default: the current CUDA device, 0
-    without one); with bounds=True also the list of piece chunk offsets."""
-    if sms is None:
-        sms = (torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
-               if torch.cuda.is_available() else 0)
-    buf = (ctypes.c_int * 17)()
-    n = lib().gdn_chunk_fwd_pieces(B, T, H, d_k, d_v, num_seqs, chunk, _dtype_code(dtype), sms,
-                                   ctypes.cast(buf, ctypes.c_void_p))
-    return (n, list(buf[:n + 1])) if bounds else n
-
-
-def set_chunk_pipeline(pieces: int) -> int:
-    """Process-wide piece count: 0 automatic, 1 off, P > 1 fixed. Returns the
-    previous setting."""
-    prev = lib().gdn_set_chunk_pipeline(int(pieces))
-    if prev < 0:
-        raise ValueError(f"invalid piece count {pieces}")
-    return prev
 
 
 def chunk_path(d_k, d_v, chunk=64, dtype=torch.bfloat16) -> int:

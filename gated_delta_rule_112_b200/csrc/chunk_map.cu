@@ -14,8 +14,7 @@ namespace {
 __global__ void __launch_bounds__(1024) gdn_chunk_map_kernel(
     const int32_t *__restrict__ cu, int B, int T, int num_seqs, int chunk,
     uint32_t *__restrict__ ctrl, ChunkInfo *__restrict__ table,
-    int32_t *__restrict__ seq_first, int max_chunks, int segs, int32_t *__restrict__ seg_first,
-    PieceBounds pieces) {
+    int32_t *__restrict__ seq_first, int max_chunks, int segs, int32_t *__restrict__ seg_first) {
   // The kernels launched after this one may start their prologues now; they
   // wait for this grid before reading what it writes.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -43,14 +42,6 @@ __global__ void __launch_bounds__(1024) gdn_chunk_map_kernel(
         const int n = e / segs, gi = e - n * segs;
         if (GDN_IN_BOUNDS(ctrl, e, N * segs + 1))
           seg_first[e] = (n >= N) ? N * cps : n * cps + min(gi * len, cps);
-      }
-    } else if (pieces.n > 1) {
-      // piece p of sequence n: chunks [n cps + c[p], n cps + c[p + 1])
-      const int P = pieces.n;
-      for (int e = tid; e <= N * P; e += blockDim.x) {
-        const int n = e / P, p = e - n * P;
-        if (GDN_IN_BOUNDS(ctrl, e, N * P + 1) && GDN_IN_BOUNDS(ctrl, p, kMaxPieces + 1))
-          seg_first[e] = (n >= N) ? N * cps : n * cps + pieces.c[p];
       }
     }
     if (tid == 0) {
@@ -122,8 +113,7 @@ cudaError_t launch_chunk_map(const int32_t *cu_seqlens, int B, int T, int num_se
       cu_seqlens, B, T, num_seqs, chunk, reinterpret_cast<uint32_t *>(base),
       reinterpret_cast<ChunkInfo *>(base + L.chunk_table),
       reinterpret_cast<int32_t *>(base + L.seq_first), L.max_chunks, L.segs,
-      (L.segs > 1 || L.pieces > 1) ? reinterpret_cast<int32_t *>(base + L.seg_first) : nullptr,
-      L.pb);
+      L.segs > 1 ? reinterpret_cast<int32_t *>(base + L.seg_first) : nullptr);
   return cudaGetLastError();
 }
 

@@ -254,30 +254,6 @@ __device__ void solve_unit_lower_64(const float *__restrict__ As, float *__restr
 // finish reading shared memory before that memory is written again).
 // Warp roles: all 8 warps share the epilogues. TMEM lane quarter = warp % 4,
 // column half = warp / 4.
-// The units a prep launch covers. len == 0: every (chunk, head) unit of the
-// call, unit = chunk * H + h. Otherwise a piece of a pipelined call over nseq
-// sequences of cps chunks each: chunks [c0, c0 + len) of every sequence, the
-// launch's unit j being (sequence j / (len H), chunk c0 + (j / H) % len,
-// head j % H). after != 0: the launch follows a state scan of the same call
-// in the stream. It reads nothing that scan writes, so it does not wait for
-// it at the start (it runs beside it on the SMs the scan leaves idle); it
-// waits at the end instead, so that the scan after it, which waits for this
-// launch, also sees the state the scan before it wrote.
-struct PieceSpec {
-  int c0, len, cps, nseq, after;
-};
-
-__device__ __forceinline__ int piece_units(const PieceSpec &p, int all_units, int H) {
-  return p.len == 0 ? all_units : p.nseq * p.len * H;
-}
-
-__device__ __forceinline__ int piece_unit(const PieceSpec &p, int j, int H) {
-  if (p.len == 0) return j;
-  const int per_seq = p.len * H;
-  const int b = j / per_seq, r = j - b * per_seq;
-  return (b * p.cps + p.c0) * H + r;
-}
-
 __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_kt,
@@ -285,7 +261,7 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
     const float *__restrict__ g,
     const float *__restrict__ beta, float *__restrict__ gam_out, int H,
     uint32_t *__restrict__ ctrl, const ChunkInfo *__restrict__ table, long long rows,
-    int max_chunks, PieceSpec piece) {
+    int max_chunks) {
   (void)rows;
   (void)max_chunks;   // extents of the bounds checks (GDN_CHECKS builds)
   extern __shared__ uint8_t smem_raw[];
@@ -325,11 +301,9 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // Everything above overlaps the chunk-map kernel; the chunk table, the
-  // chunk count and the error word are read only after it completes (a later
-  // piece starts after it completed, see PieceSpec).
-  if (!piece.after) grid_dependency_wait();
-  const int nunits =
-      (ctrl[0] & kErrBadSeqlens) ? 0 : piece_units(piece, int(ctrl[1]) * H, H);
+  // chunk count and the error word are read only after it completes.
+  grid_dependency_wait();
+  const int nunits = (ctrl[0] & kErrBadSeqlens) ? 0 : int(ctrl[1]) * H;
   const int m = (warp & 3) * 32 + lane;   // TMEM lane = row of G
   const int hc = warp >> 2;               // column half
   const uint32_t lane_base = tmem + (uint32_t((warp & 3) * 32) << 16);
@@ -337,9 +311,8 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
   // g and beta of unit u (rows past the sequence end read as 0), one row per
   // thread of the first two warps.
   float g_reg = 0.f, b_reg = 0.f;
-  auto fetch_gb = [&](int j) {
-    if (tid < kC && j < nunits) {
-      const int u = piece_unit(piece, j, H);
+  auto fetch_gb = [&](int u) {
+    if (tid < kC && u < nunits) {
       const int cu = u / H, hu = u - cu * H;
       const ChunkInfo cf = GDN_IN_BOUNDS(ctrl, cu, max_chunks) ? table[cu] : ChunkInfo{0, 0, 0, 0};
       const long long idx = (long long)(cf.row0 + tid) * H + hu;
@@ -350,8 +323,7 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
   };
   fetch_gb(blockIdx.x);
   int it = 0;
-  for (int j = blockIdx.x; j < nunits; j += gridDim.x, ++it) {
-  const int unit = piece_unit(piece, j, H);
+  for (int unit = blockIdx.x; unit < nunits; unit += gridDim.x, ++it) {
   const int chunk = unit / H, h = unit - chunk * H;
   const ChunkInfo ci =
       GDN_IN_BOUNDS(ctrl, chunk, max_chunks) ? table[chunk] : ChunkInfo{0, 0, 0, 0};
@@ -370,9 +342,8 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
       tma_load_3d(sm + kP_KQ + kTile128x64, &tm_k, bar_load, 64, h, ci.row0);
       tma_load_3d(sm + kP_KQ + kTile128x64 + kTile64x64, &tm_q, bar_load, 64, h, ci.row0);
     }
-    const int nj = j + int(gridDim.x);
-    if (nj < nunits) {
-      const int nu = piece_unit(piece, nj, H);
+    const int nu = unit + int(gridDim.x);
+    if (nu < nunits) {
       const int cn = nu / H, hn = nu - cn * H;
       const int rn = GDN_IN_BOUNDS(ctrl, cn, max_chunks) ? table[cn].row0 : 0;
       tma_prefetch_l2_3d(&tm_k, 0, hn, rn);
@@ -385,7 +356,7 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
     Gm[tid] = g_reg;
     Bt[tid] = b_reg;
   }
-  fetch_gb(j + int(gridDim.x));
+  fetch_gb(unit + int(gridDim.x));
   __syncthreads();
   if (warp == 0) {  // inclusive cumsum of the 64 log-gates
     const float a0 = Gm[2 * lane], a1 = Gm[2 * lane + 1];
@@ -639,7 +610,6 @@ __global__ void __launch_bounds__(kPrepThreads, 3) gdn_prep_kernel(
     tc_fence_after();
     tmem_dealloc(tmem, 128);
   }
-  if (piece.after) grid_dependency_wait();
 }
 
 // ============================================================ channel-wise gate: prep
@@ -739,7 +709,7 @@ __global__ void __launch_bounds__(kKdaPrepThreads, 2) gdn_kda_prep_kernel(
     const __grid_constant__ CUtensorMap tm_tb, const __grid_constant__ CUtensorMap tm_qt,
     const float *__restrict__ g, const float *__restrict__ beta, float *__restrict__ gam_out,
     uint32_t *__restrict__ pm_out, int H, uint32_t *__restrict__ ctrl,
-    const ChunkInfo *__restrict__ table, long long rows, int max_chunks, PieceSpec piece) {
+    const ChunkInfo *__restrict__ table, long long rows, int max_chunks) {
   (void)rows;
   (void)max_chunks;   // extents of the bounds checks (GDN_CHECKS builds)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -779,14 +749,11 @@ __global__ void __launch_bounds__(kKdaPrepThreads, 2) gdn_kda_prep_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (!piece.after) grid_dependency_wait();   // see PieceSpec
-  const int nunits =
-      (ctrl[0] & kErrBadSeqlens) ? 0 : piece_units(piece, int(ctrl[1]) * H, H);
+  grid_dependency_wait();
+  const int nunits = (ctrl[0] & kErrBadSeqlens) ? 0 : int(ctrl[1]) * H;
   const long long pm_words = (long long)max_chunks * H * (64 * 64 / 2);
-  (void)pm_words;
   int it = 0;
-  for (int j = blockIdx.x; j < nunits; j += gridDim.x, ++it) {
-    const int unit = piece_unit(piece, j, H);
+  for (int unit = blockIdx.x; unit < nunits; unit += gridDim.x, ++it) {
     const int chunk = unit / H, h = unit - chunk * H;
     const ChunkInfo ci =
         GDN_IN_BOUNDS(ctrl, chunk, max_chunks) ? table[chunk] : ChunkInfo{0, 0, 0, 0};
@@ -1055,7 +1022,6 @@ __global__ void __launch_bounds__(kKdaPrepThreads, 2) gdn_kda_prep_kernel(
     tc_fence_after();
     tmem_dealloc(tmem, 64);
   }
-  if (piece.after) grid_dependency_wait();
 }
 
 // ===================================================================== scan
@@ -1160,13 +1126,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     const float *__restrict__ s0, float *__restrict__ sN, __nv_bfloat16 *__restrict__ o, int H,
     uint32_t *__restrict__ ctrl, const ChunkInfo *__restrict__ table,
     const int32_t *__restrict__ seq_first, int split, float *__restrict__ sN_trans,
-    int sN_group, long long rows, int max_chunks, int n_first, int n_s0, int n_sN, int kda,
-    int pstride, int poff, int state_dep) {
-  // pstride, poff: CTA n runs the chunk range seq_first[m] .. seq_first[m + 1]
-  // of entry m = n pstride + poff, with its states s0[n] and sN[n / sN_group]
-  // (1, 0: entry n; a piece of a pipelined call: pieces per sequence, piece).
-  // state_dep: s0 is written by an earlier kernel of the call (the scan of the
-  // piece before), so it is read only after the dependency wait.
+    int sN_group, long long rows, int max_chunks, int n_first, int n_s0, int n_sN, int kda) {
   // kda: the channel-wise gate. Q comes per unit from the prep (Q .* e^Gamma,
   // 2-D map tm_q over [units * 64][128]), the decay records are 256 wide and
   // S decays per d_k channel.
@@ -1252,14 +1212,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
   int c0 = 0, nch = 0, row_first = 0, last_len = kC;
   auto read_chunks = [&]() {
     grid_dependency_wait();
-    // The next kernel of the stream (the prep of the next piece of a
-    // pipelined call) may start on the SMs this grid leaves idle.
-    grid_launch_dependents();
     if (!(ctrl[0] & kErrBadSeqlens)) {
-      const int m = n * pstride + poff;
-      if (GDN_IN_BOUNDS(ctrl, m + 1, n_first)) {
-        c0 = seq_first[m];
-        nch = seq_first[m + 1] - c0;
+      if (GDN_IN_BOUNDS(ctrl, n + 1, n_first)) {
+        c0 = seq_first[n];
+        nch = seq_first[n + 1] - c0;
       }
       if (nch > 0 && GDN_IN_BOUNDS(ctrl, c0, max_chunks) &&
           GDN_IN_BOUNDS(ctrl, c0 + nch - 1, max_chunks)) {
@@ -1467,7 +1423,6 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     const bool tl = tr && warp == 4 && lane == 0;       // traced lane
     (void)tl;
     float S[64];                                        // S[i][64 hh + t], fp32 master
-    if (state_dep) grid_dependency_wait();
     {
       const float *src = (s0 && !trans && GDN_IN_BOUNDS(ctrl, (long long)n * H + h, (long long)n_s0 * H))
                              ? s0 + (size_t(n) * H + h) * kD * kD
@@ -1851,58 +1806,20 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     cfg.stream = s;
     cfg.attrs = pdl;
     cfg.numAttrs = 1;
-    auto launch_prep = [&](const PieceSpec &piece) {
-      if (L.kda)
-        return cudaLaunchKernelEx(&cfg, gdn_kda_prep_kernel, mq, mk, mw, mkt, mtb, mqt, g, beta,
-                                  reinterpret_cast<float *>(base + L.gam),
-                                  reinterpret_cast<uint32_t *>(base + L.pm), H, ctrl, table,
-                                  rows, L.max_chunks, piece);
-      return cudaLaunchKernelEx(&cfg, gdn_prep_kernel, mq, mk, mw, mkt, mtb, mpm, g, beta,
-                                reinterpret_cast<float *>(base + L.gam), H, ctrl, table, rows,
-                                L.max_chunks, piece);
-    };
+    if (L.kda)
+      e = cudaLaunchKernelEx(&cfg, gdn_kda_prep_kernel, mq, mk, mw, mkt, mtb, mqt, g, beta,
+                             reinterpret_cast<float *>(base + L.gam),
+                             reinterpret_cast<uint32_t *>(base + L.pm), H, ctrl, table, rows,
+                             L.max_chunks);
+    else
+      e = cudaLaunchKernelEx(&cfg, gdn_prep_kernel, mq, mk, mw, mkt, mtb, mpm, g, beta,
+                             reinterpret_cast<float *>(base + L.gam), H, ctrl, table, rows,
+                             L.max_chunks);
+    if (e != cudaSuccess) return e;
     // the scan reads Q from the prep's Q .* e^Gamma with the channel-wise gate
     const CUtensorMap mqs = L.kda ? mqt : mq;
     e = cudaFuncSetAttribute(gdn_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kScanSmem);
-    if (e != cudaSuccess) return e;
-    const int cps = int((T + kC - 1) / kC);
-    if (L.pieces > 1 && L.segs <= 1 && !g_profile.start) {
-      // Pipelined, in this stream: prep(0), scan(0), prep(1), scan(1), ...,
-      // all with programmatic dependent launch. scan(p) lets the next kernel
-      // launch once it has passed its dependency wait; prep(p + 1) then runs
-      // on the SMs the chains leave idle (its grid sized to them) and waits
-      // for scan(p) only at its end; scan(p + 1) waits for prep(p + 1) and so
-      // reads the state scan(p) left in the handoff buffer (in place: CTA n
-      // reads and writes only slot n).
-      const int chains = B * H;
-      float *handoff = reinterpret_cast<float *>(base + L.handoff);
-      const int32_t *piece_first = reinterpret_cast<const int32_t *>(base + L.seg_first);
-      for (int p = 0; p < L.pieces; ++p) {
-        const int c0 = L.pb.c[p], plen = L.pb.c[p + 1] - c0;
-        const PieceSpec piece{c0, plen, cps, B, p > 0 ? 1 : 0};
-        const long long punits = (long long)B * plen * H;
-        const long long fit = (L.kda ? 2LL : 3LL) * (p > 0 ? std::max(sms - chains, 1) : sms);
-        cfg.gridDim = dim3(unsigned(std::min<long long>(punits, fit)));
-        cfg.blockDim = dim3(L.kda ? kKdaPrepThreads : kPrepThreads);
-        cfg.dynamicSmemBytes = L.kda ? kKdaPrepSmem : kPrepSmem;
-        e = launch_prep(piece);
-        if (e != cudaSuccess) return e;
-        cfg.gridDim = dim3(B, H);
-        cfg.blockDim = dim3(kScanThreads);
-        cfg.dynamicSmemBytes = kScanSmem;
-        const float *sin = p == 0 ? s0 : handoff;
-        float *sout = p == L.pieces - 1 ? sN : handoff;
-        e = cudaLaunchKernelEx(&cfg, gdn_scan_kernel, mqs, mv, mw, mkt, mtb, mpm, mgm, mo, sin,
-                               sout, static_cast<__nv_bfloat16 *>(o), H, ctrl,
-                               static_cast<const ChunkInfo *>(table), piece_first, 0,
-                               static_cast<float *>(nullptr), 1, rows, L.max_chunks,
-                               B * L.pieces + 1, B, B, int(L.kda), L.pieces, p, p > 0 ? 1 : 0);
-        if (e != cudaSuccess) return e;
-      }
-      return cudaSuccess;
-    }
-    e = launch_prep(PieceSpec{0, 0, cps, N, 0});
     if (e != cudaSuccess) return e;
     prof_record(g_profile.scan, s);
     cfg.blockDim = dim3(kScanThreads);
@@ -1913,7 +1830,7 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
                                 sN, static_cast<__nv_bfloat16 *>(o), H, ctrl,
                                 static_cast<const ChunkInfo *>(table), seq_first, 0,
                                 static_cast<float *>(nullptr), 1, rows, L.max_chunks, N + 1, N,
-                                N, int(L.kda), 1, 0, 0);
+                                N, int(L.kda));
     }
     // Segmented state scan (few long sequences): three passes over B * segs
     // segments. (1) every segment from S = 0 and as a transition, no output;
@@ -1929,7 +1846,7 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
                            static_cast<const float *>(nullptr), hbuf,
                            static_cast<__nv_bfloat16 *>(nullptr), H, ctrl,
                            static_cast<const ChunkInfo *>(table), seg_first, nseg, pbuf, 1, rows,
-                           L.max_chunks, nseg + 1, 0, nseg, int(L.kda), 1, 0, 0);
+                           L.max_chunks, nseg + 1, 0, nseg, int(L.kda));
     if (e != cudaSuccess) return e;
     gdn_segment_combine_kernel<<<dim3(B * H, kD / 16), 256, 0, s>>>(s0, hbuf, pbuf, sstart, H,
                                                                    L.segs, ctrl);
@@ -1943,7 +1860,7 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
                               static_cast<__nv_bfloat16 *>(o), H, ctrl,
                               static_cast<const ChunkInfo *>(table), seg_first, 0,
                               static_cast<float *>(nullptr), L.segs, rows, L.max_chunks, nseg + 1,
-                              nseg, B, int(L.kda), 1, 0, 0);
+                              nseg, B, int(L.kda));
   }
   // No tokens: the final state is the initial state.
   prof_record(g_profile.prep, s);

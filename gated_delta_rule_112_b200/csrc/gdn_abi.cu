@@ -18,7 +18,6 @@ int device_sms() {
 }
 
 ProfileEvents g_profile = {nullptr, nullptr, nullptr, nullptr};
-int g_pipeline_pieces = 0;
 }
 
 namespace {
@@ -64,10 +63,8 @@ int run_chunk(bool force_simt, bool channel_gate, const void *q, const void *k, 
   // bf16 with d_k = d_v = 128 and 64-token chunks runs on the tensor-core
   // kernels for both gates; everything else on the CUDA-core kernel.
   const bool tc = !force_simt && tc_path(dk, dv, chunk, dtype);
-  const int sms = device_sms();
-  const int segs = scan_segments(B, T, H, cu ? num_seqs : 0, chunk, tc, sms);
-  const WsLayout L =
-      ws_layout(B, T, H, cu ? num_seqs : 0, chunk, tc, segs, tc && channel_gate, sms);
+  const int segs = scan_segments(B, T, H, cu ? num_seqs : 0, chunk, tc, device_sms());
+  const WsLayout L = ws_layout(B, T, H, cu ? num_seqs : 0, chunk, tc, segs, tc && channel_gate);
   if (ws_bytes < L.total) return GDN_ERR_WORKSPACE;
   const int N = cu ? num_seqs : B;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -95,9 +92,8 @@ size_t gdn_chunk_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int n
   if (B < 1 || T < 0 || H < 1 || d_k < 1 || d_v < 1 || num_seqs < 0) return 0;
   if (chunk != 16 && chunk != 32 && chunk != 64) return 0;
   const bool tc = tc_path(d_k, d_v, chunk, dtype);
-  const int sms = device_sms();
-  return ws_layout(B, T, H, num_seqs, chunk, tc, scan_segments(B, T, H, num_seqs, chunk, tc, sms),
-                   false, sms)
+  return ws_layout(B, T, H, num_seqs, chunk, tc,
+                   scan_segments(B, T, H, num_seqs, chunk, tc, device_sms()))
       .total;
 }
 
@@ -105,24 +101,6 @@ int gdn_chunk_fwd_scan_segments(int B, int T, int H, int d_k, int d_v, int num_s
                                 int dtype, int sms) {
   if (B < 0 || T < 0 || H < 0 || num_seqs < 0 || sms < 0) return 1;
   return scan_segments(B, T, H, num_seqs, chunk, tc_path(d_k, d_v, chunk, dtype), sms);
-}
-
-int gdn_chunk_fwd_pieces(int B, int T, int H, int d_k, int d_v, int num_seqs, int chunk,
-                         int dtype, int sms, int *bounds) {
-  if (B < 1 || T < 0 || H < 1 || num_seqs < 0 || sms < 0) return 1;
-  const bool tc = tc_path(d_k, d_v, chunk, dtype);
-  const int segs = scan_segments(B, T, H, num_seqs, chunk, tc, sms);
-  const PieceBounds pb = piece_bounds(B, T, H, num_seqs, chunk, tc, segs, sms);
-  if (bounds)
-    for (int i = 0; i <= pb.n; ++i) bounds[i] = pb.c[i];
-  return pb.n;
-}
-
-int gdn_set_chunk_pipeline(int pieces) {
-  if (pieces < 0) return GDN_ERR_INVALID_ARG;
-  const int prev = g_pipeline_pieces;
-  g_pipeline_pieces = pieces;
-  return prev;
 }
 
 int gdn_chunk_fwd_path(int d_k, int d_v, int chunk, int dtype) {
@@ -157,9 +135,8 @@ size_t gdn_kda_chunk_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, i
   if (B < 1 || T < 0 || H < 1 || d_k < 1 || d_v < 1 || num_seqs < 0) return 0;
   if (chunk != 16 && chunk != 32 && chunk != 64) return 0;
   const bool tc = tc_path(d_k, d_v, chunk, dtype);
-  const int sms = device_sms();
-  const int segs = scan_segments(B, T, H, num_seqs, chunk, tc, sms);
-  return ws_layout(B, T, H, num_seqs, chunk, tc, segs, tc, sms).total;
+  const int segs = scan_segments(B, T, H, num_seqs, chunk, tc, device_sms());
+  return ws_layout(B, T, H, num_seqs, chunk, tc, segs, tc).total;
 }
 
 int gdn_kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g,

@@ -49,6 +49,30 @@ struct ChunkInfo {
   int32_t len;    // valid tokens in this chunk (1..chunk)
 };
 
+// Workspace layout. Offsets are in bytes from the (256-byte aligned) base.
+//   [0, 256)       control block: word 0 = device error bits, word 1 = total chunks
+//   chunk table    ChunkInfo[max_chunks]
+//   seq_first      int32[N + 1]  global index of each sequence's first chunk
+//   tensor-core path only, per (chunk, head) unit u = chunk * H + h:
+//   w              bf16 [units][64][d_k = 128]   -W of the chunk (rows = tokens)
+//   kt             bf16 [units][d_k = 128][64]   (D K)^T, D = diag(exp(Gamma_last - Gamma))
+//   tb             bf16 [units][64][64]          T diag(beta) of the chunk (UT transform)
+//   pm             bf16 [units][64][64]          (Q K^T) .* decay mask, diagonal included
+//   gam            fp32 [units][128]             exp(Gamma_c) (64), then exp(Gamma_last - Gamma_s) (64)
+//                  channel-wise gate: fp32 [units][256]: 1 (64), unused (64), then the
+//                  per-channel state decay exp(Gamma_last,j) (128)
+//   qt             channel-wise gate only: bf16 [units][64][d_k]  Q .* exp(Gamma)
+//   tensor-core path with a segmented state scan (segs > 1, see scan_segments):
+//   seg_first      int32[B * segs + 1]  first chunk of each segment
+//   hbuf, pbuf     fp32 [B * segs][H][d_k][d_v]  each segment's state from S = 0,
+//                  and its transition (the state from S = I with V = 0)
+//   sstart         fp32 [B * segs][H][d_k][d_v]  each segment's true start state
+struct WsLayout {
+  size_t chunk_table, seq_first, w, kt, tb, pm, gam, qt, seg_first, hbuf, pbuf, sstart, total;
+  int max_chunks, segs;
+  bool kda;
+};
+
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 inline int max_chunks_for(int B, int T, int num_seqs, int chunk) {
@@ -86,105 +110,10 @@ inline int scan_segments(int B, int T, int H, int num_seqs, int chunk, bool tc, 
   return (best > 1 && best_cost * 10 <= plain * 7) ? best : 1;   // at least 30 % faster
 }
 
-// Pieces of a pipelined tensor-core call. The state scan runs one CTA per
-// (sequence, head) chain and leaves the other SMs idle, while the per-chunk
-// prep has no dependence between chunks. B equal-length sequences of cps
-// chunks are cut into pieces of consecutive chunks, launched in one stream
-// as prep(0), scan(0), prep(1), scan(1), ... with programmatic dependent
-// launch: prep(p + 1) starts once scan(p) runs and fills the idle SMs, and
-// scan(p + 1) starts from the state scan(p) ends with. The first piece is
-// prepped on the whole GPU while nothing else runs, so it is the longest; each
-// next piece is r times the one before, r = (chunks the scan does per unit
-// of time) / (chunks the prep does on the idle SMs), so that the prep of a
-// piece takes about as long as the scan of the piece before. r comes from
-// the measured rates of the two kernels on B200: a chunk period of about
-// 1.3 us and 2.93 SM-us of prep per (chunk, head) unit. Pieces shorter than
-// kMinPiece chunks join the last one. No pipeline (1 piece) for packed
-// sequences, a segmented scan, the CUDA-core path, fewer than 16 chunks per
-// sequence, or when the chains leave fewer than a quarter of the SMs idle.
-// g_pipeline_pieces overrides the choice: 0 automatic, 1 off, P > 1 P pieces
-// of equal length (at most one per chunk).
-constexpr int kMaxPieces = 16;
-constexpr int kMinPiece = 4;
-extern int g_pipeline_pieces;
-struct PieceBounds {
-  int n;                      // pieces
-  int c[kMaxPieces + 1];      // piece p covers chunks [c[p], c[p + 1]) of every sequence
-};
-inline PieceBounds piece_bounds(int B, int T, int H, int num_seqs, int chunk, bool tc, int segs,
-                                int sms) {
-  PieceBounds pb{};
-  pb.n = 1;
-  if (!tc || num_seqs > 0 || segs > 1 || chunk != 64 || B <= 0 || T <= 0 || H <= 0) return pb;
-  const int cps = int((int64_t(T) + chunk - 1) / chunk);
-  pb.c[1] = cps;
-  const int over = g_pipeline_pieces;
-  if (over == 1) return pb;
-  if (over > 1) {
-    const int p = over < kMaxPieces ? (over < cps ? over : cps) : (kMaxPieces < cps ? kMaxPieces : cps);
-    const int len = (cps + p - 1) / p;
-    pb.n = (cps + len - 1) / len;
-    for (int i = 0; i <= pb.n; ++i) pb.c[i] = i * len < cps ? i * len : cps;
-    return pb;
-  }
-  const long long chains = int64_t(B) * H;
-  const long long idle = int64_t(sms) - chains;
-  if (cps < 16 || sms <= 0 || idle * 4 < sms) return pb;
-  double r = 1.3 * double(idle) / (2.93 * double(chains));
-  if (r > 0.9) r = 0.9;
-  int s = int(double(cps) * (1.0 - r) + 0.999);
-  int done = 0, n = 0;
-  while (done < cps) {
-    int take = s > kMinPiece ? s : kMinPiece;
-    if (take > cps - done || cps - done - take < kMinPiece || n == kMaxPieces - 1) take = cps - done;
-    pb.c[n] = done;
-    done += take;
-    ++n;
-    s = int(double(s) * r + 0.5);
-  }
-  pb.c[n] = cps;
-  pb.n = n;
-  return pb;
-}
-inline int chunk_pieces(int B, int T, int H, int num_seqs, int chunk, bool tc, int segs, int sms) {
-  return piece_bounds(B, T, H, num_seqs, chunk, tc, segs, sms).n;
-}
-
-// Workspace layout. Offsets are in bytes from the (256-byte aligned) base.
-//   [0, 256)       control block: word 0 = device error bits, word 1 = total chunks
-//   chunk table    ChunkInfo[max_chunks]
-//   seq_first      int32[N + 1]  global index of each sequence's first chunk
-//   tensor-core path only, per (chunk, head) unit u = chunk * H + h:
-//   w              bf16 [units][64][d_k = 128]   -W of the chunk (rows = tokens)
-//   kt             bf16 [units][d_k = 128][64]   (D K)^T, D = diag(exp(Gamma_last - Gamma))
-//   tb             bf16 [units][64][64]          T diag(beta) of the chunk (UT transform)
-//   pm             bf16 [units][64][64]          (Q K^T) .* decay mask, diagonal included
-//   gam            fp32 [units][128]             exp(Gamma_c) (64), then exp(Gamma_last - Gamma_s) (64)
-//                  channel-wise gate: fp32 [units][256]: 1 (64), unused (64), then the
-//                  per-channel state decay exp(Gamma_last,j) (128)
-//   qt             channel-wise gate only: bf16 [units][64][d_k]  Q .* exp(Gamma)
-//   tensor-core path with a segmented state scan (segs > 1, see scan_segments):
-//   seg_first      int32[B * segs + 1]  first chunk of each segment
-//   hbuf, pbuf     fp32 [B * segs][H][d_k][d_v]  each segment's state from S = 0,
-//                  and its transition (the state from S = I with V = 0)
-//   sstart         fp32 [B * segs][H][d_k][d_v]  each segment's true start state
-//   tensor-core path run as a pipeline of pieces (pieces > 1, see chunk_pieces):
-//   seg_first      int32[B * pieces + 1]  first chunk of each piece of each sequence
-//   handoff        fp32 [B][H][d_k][d_v]  the state between consecutive pieces
-struct WsLayout {
-  size_t chunk_table, seq_first, w, kt, tb, pm, gam, qt, seg_first, hbuf, pbuf, sstart, handoff,
-      total;
-  int max_chunks, segs, pieces;
-  bool kda;
-  PieceBounds pb;
-};
-
 inline WsLayout ws_layout(int B, int T, int H, int num_seqs, int chunk, bool tc, int segs = 1,
-                          bool kda = false, int sms = 0) {
+                          bool kda = false) {
   WsLayout L{};
   L.kda = kda;
-  L.pb = piece_bounds(B, T, H, num_seqs, chunk, tc, segs, sms);
-  L.pieces = L.pb.n;
   const int N = num_seqs > 0 ? num_seqs : B;
   L.max_chunks = max_chunks_for(B, T, num_seqs, chunk);
   L.segs = segs;
@@ -210,9 +139,6 @@ inline WsLayout ws_layout(int B, int T, int H, int num_seqs, int chunk, bool tc,
       L.hbuf = off;      off = align_up(off + states, 1024);
       L.pbuf = off;      off = align_up(off + states, 1024);
       L.sstart = off;    off = align_up(off + states, 1024);
-    } else if (L.pieces > 1) {
-      L.seg_first = off; off = align_up(off + sizeof(int32_t) * (size_t(B) * L.pieces + 1), 1024);
-      L.handoff = off;   off = align_up(off + size_t(B) * H * 128 * 128 * sizeof(float), 1024);
     }
   }
   L.total = off;

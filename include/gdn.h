@@ -68,8 +68,7 @@ extern "C" {
  * The workspace must be 256-byte aligned; its contents need no initialisation.
  * Sized for the current CUDA device: with few long sequences the tensor-core
  * path splits the state scan into segments (gdn_chunk_fwd_scan_segments) and
- * needs three fp32 states per segment and head more; a pipelined call
- * (gdn_chunk_fwd_pieces > 1) needs one fp32 state per sequence and head more.
+ * needs three fp32 states per segment and head more.
  */
 size_t gdn_chunk_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int num_seqs,
                                     int chunk, int dtype);
@@ -192,37 +191,6 @@ int gdn_chunk_fwd_path(int d_k, int d_v, int chunk, int dtype);
  */
 int gdn_chunk_fwd_scan_segments(int B, int T, int H, int d_k, int d_v, int num_seqs, int chunk,
                                 int dtype, int sms);
-
-/*
- * gdn_chunk_fwd_pieces -- into how many pieces the tensor-core path cuts a
- * call of these sizes on a device with `sms` streaming multiprocessors to
- * overlap its two kernels (1 = no pipeline). Pure host arithmetic; depends
- * on gdn_set_chunk_pipeline. If `bounds` is not NULL it receives the pieces'
- * chunk offsets: piece p covers chunks [bounds[p], bounds[p + 1]) of every
- * sequence (pieces + 1 ints, at most 17).
- *
- * The state scan runs one CTA per (sequence, head) chain and leaves the other
- * SMs idle; the per-chunk prep has no dependence between chunks. For B
- * equal-length sequences of at least 16 chunks (no cu_seqlens, no segmented
- * scan) whose chains leave at least a quarter of the SMs idle, the call runs
- * in the caller's stream as prep(0), scan(0), prep(1), scan(1), ... with
- * programmatic dependent launch: prep(p + 1) starts once every CTA of
- * scan(p) runs and fills the idle SMs, and scan(p + 1) starts from the state
- * scan(p) ended with. Pieces shrink geometrically so that the prep of each
- * piece takes about as long as the scan of the one before. The result is the
- * same computation as one piece, to the bit.
- */
-int gdn_chunk_fwd_pieces(int B, int T, int H, int d_k, int d_v, int num_seqs, int chunk,
-                         int dtype, int sms, int *bounds);
-
-/*
- * gdn_set_chunk_pipeline -- process-wide choice of the piece count:
- * 0 automatic (geometric pieces, see gdn_chunk_fwd_pieces), 1 off, P > 1
- * that many pieces of equal length (at most 16, at most one per chunk). Returns the previous setting,
- * or GDN_ERR_INVALID_ARG for P < 0. Workspace sizes depend on it: query
- * gdn_chunk_fwd_workspace_size after changing it.
- */
-int gdn_set_chunk_pipeline(int pieces);
 
 /*
  * gdn_decode_step -- one recurrent token for N*H independent states, in place.

@@ -68,17 +68,8 @@ def test_workspace_size(L):
     # 4096 (chunk, head) units x (-W 16 KB + (D K)^T 16 KB + T diag(beta) 8 KB +
     # P 8 KB + 512 B of decay factors) plus bookkeeping
     per_unit = 16384 + 16384 + 8192 + 8192 + 512
-    # a pipelined call (a device with SMs to spare) also holds one fp32
-    # handoff state per (sequence, head); without a device there is no pipeline
-    handoff = 4 * 16 * 128 * 128 * 4
     assert tc >= 4096 * per_unit
-    assert tc < 4096 * per_unit + handoff + (1 << 20)
-    prev = L.gdn_set_chunk_pipeline(1)
-    try:
-        off = ws(4, 4096, 16, 128, 128, 0, 64, gdn.BF16)
-        assert 4096 * per_unit <= off < 4096 * per_unit + (1 << 20)
-    finally:
-        L.gdn_set_chunk_pipeline(prev)
+    assert tc < 4096 * per_unit + (1 << 20)
     simt = ws(1, 256, 2, 64, 64, 0, 64, gdn.F32)
     assert 0 < simt < (1 << 16)
     # varlen bound: (T + N (C-1)) / C chunks
@@ -131,41 +122,6 @@ def test_decode_host_checks(L):
     assert call(N=0) == gdn.ERR_INVALID_ARG
     assert call(dv=130) == gdn.ERR_UNSUPPORTED
     assert call(dv=126) == gdn.ERR_UNSUPPORTED
-
-
-def test_pipeline_pieces_rule(L):
-    import ctypes
-
-    def P(B, T, H, ns=0, dtype=gdn.BF16, sms=148):
-        buf = (ctypes.c_int * 17)()
-        n = L.gdn_chunk_fwd_pieces(B, T, H, 128, 128, ns, 64, dtype, sms,
-                                   ctypes.cast(buf, ctypes.c_void_p))
-        return n, list(buf[:n + 1])
-
-    # 64 chains on 148 SMs leave 84 idle: pieces shrink by r = 1.3 * 84 / (2.93 * 64)
-    assert P(4, 4096, 16) == (5, [0, 27, 43, 52, 57, 64])
-    n, b = P(2, 64 * 40, 24)                      # 48 chains, 40 chunks
-    assert n > 1 and b[0] == 0 and b[-1] == 40
-    sizes = [y - x for x, y in zip(b, b[1:])]
-    assert all(x >= 4 for x in sizes) and sizes[0] == max(sizes)
-    assert P(2, 64 * 15, 24)[0] == 1              # fewer than 16 chunks
-    assert P(4, 4096, 32)[0] == 1                 # 128 chains: under a quarter of the SMs idle
-    assert P(1, 4096, 16, ns=3)[0] == 1           # packed sequences
-    assert P(4, 4096, 16, dtype=gdn.F32)[0] == 1  # CUDA-core path
-    assert P(4, 4096, 16, sms=0)[0] == 1          # unknown device
-    assert P(1, 65536, 16)[0] == 1                # few long chains: the segmented scan instead
-    assert L.gdn_set_chunk_pipeline(-1) == gdn.ERR_INVALID_ARG
-    prev = L.gdn_set_chunk_pipeline(5)
-    try:
-        assert P(4, 4096, 16) == (5, [0, 13, 26, 39, 52, 64])   # equal pieces of 13
-        assert P(1, 64 * 3, 1)[0] == 3            # at most one per chunk
-        assert P(4, 4096, 16, sms=0)[0] == 5      # forced even without a device
-        assert L.gdn_set_chunk_pipeline(40) == 5
-        assert P(4, 4096, 16)[0] == 16            # at most 16
-        L.gdn_set_chunk_pipeline(7)
-        assert P(1, 64 * 10, 1)[0] == 5           # pieces of ceil(10 / 7) = 2 chunks
-    finally:
-        L.gdn_set_chunk_pipeline(prev)
 
 
 def test_scan_segments_rule(L):

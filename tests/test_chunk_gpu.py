@@ -174,82 +174,6 @@ def test_tc_segmented_scan_without_final_state_or_initial_state():
     assert_close("o", np64(o), ro, TOL_BF16)
 
 
-# ---------------------------------------------------------------- pipelined pieces
-def _pieces(inp):
-    import gated_delta_rule_112_b200 as gdn
-    return gdn.chunk_pieces(inp["B"], inp["T"], inp["H"], 128, 128, 0)
-
-
-class _pipeline:
-    """Sets the process-wide piece count for the duration of a with-block."""
-
-    def __init__(self, pieces):
-        self.pieces = pieces
-
-    def __enter__(self):
-        import gated_delta_rule_112_b200 as gdn
-        self.prev = gdn.set_chunk_pipeline(self.pieces)
-
-    def __exit__(self, *exc):
-        import gated_delta_rule_112_b200 as gdn
-        gdn.set_chunk_pipeline(self.prev)
-
-
-def test_tc_pipelined_call_against_the_oracle():
-    inp = make_chunk_inputs(SMALL, B=2, H=24, T=64 * 17 + 37, random_state=True)  # 18 chunks
-    assert _pieces(inp) > 1
-    check(inp, TOL_BF16)
-
-
-@pytest.mark.parametrize("pieces,expect", [(2, 2), (5, 5), (16, 9)])
-def test_tc_pipeline_is_bit_identical_to_one_piece(pieces, expect):
-    """The pieces run the same per-chunk arithmetic and hand the fp32 state
-    over exactly, so the result does not depend on the piece count."""
-    inp = make_chunk_inputs(SMALL, B=2, H=24, T=64 * 18 - 5, random_state=True)
-    with _pipeline(1):
-        assert _pieces(inp) == 1
-        o1, f1 = gpu_chunk(inp)
-    with _pipeline(pieces):
-        assert _pieces(inp) == expect
-        o2, f2 = gpu_chunk(inp)
-    assert torch.equal(o1, o2)
-    assert torch.equal(f1, f2)
-
-
-def test_tc_pipeline_without_initial_or_final_state():
-    import gated_delta_rule_112_b200 as gdn
-    inp = make_chunk_inputs(SMALL, B=2, H=24, T=64 * 20)
-    assert _pieces(inp) > 1
-    d = to_dev(inp)
-    o, fs = gdn.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], None, None,
-                          output_final_state=False)
-    torch.cuda.synchronize()
-    assert fs is None
-    ro, _ = oracle_chunk(inp)
-    assert_close("o", np64(o), ro, TOL_BF16)
-
-
-def test_tc_pipeline_inside_a_cuda_graph():
-    """The pieces are kernels of the caller's stream linked by programmatic
-    dependent launch, which a stream capture records: a captured call replays
-    to the same bits as a direct one."""
-    import gated_delta_rule_112_b200 as gdn
-    inp = make_chunk_inputs(SMALL, B=2, H=24, T=64 * 24, random_state=True)
-    assert _pieces(inp) > 1
-    d = to_dev(inp)
-    args = (d["q"], d["k"], d["v"], d["g"], d["beta"], d["initial_state"], None)
-    o_ref, f_ref = gdn.chunk_fwd(*args)
-    torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        o_g, f_g = gdn.chunk_fwd(*args)
-    graph.replay()
-    torch.cuda.synchronize()
-    assert torch.equal(o_g, o_ref)
-    assert torch.equal(f_g, f_ref)
-    del graph
-
-
 # ---------------------------------------------------------------- the workloads
 def test_workload_tiny_fp32():
     check(make_chunk_inputs("tiny_fp32"), TOL_F32)

@@ -106,22 +106,6 @@ def test_kda_tc_segmented_scan():
     check(inp, TOL_BF16)
 
 
-def test_kda_tc_pipeline_is_bit_identical_to_one_piece():
-    import gated_delta_rule_112_b200 as gdn
-    inp = make_chunk_inputs(KDA_TC, B=2, H=24, T=64 * 18 - 5, random_state=True)
-    prev = gdn.set_chunk_pipeline(1)
-    try:
-        o1, f1 = gpu_kda(inp)
-        gdn.set_chunk_pipeline(4)
-        assert gdn.chunk_pieces(2, 64 * 18 - 5, 24, 128, 128) == 4
-        o2, f2 = gpu_kda(inp)
-    finally:
-        gdn.set_chunk_pipeline(prev)
-    assert torch.equal(o1, o2)
-    assert torch.equal(f1, f2)
-    check(inp, TOL_BF16)
-
-
 def test_kda_tc_equal_channels_match_the_scalar_gate():
     import gated_delta_rule_112_b200 as gdn
     inp = make_chunk_inputs(KDA_TC, B=2, H=2, T=160, random_state=True)
