@@ -75,11 +75,16 @@ def lib() -> ctypes.CDLL:
         L.gdn_kda_chunk_fwd_workspace_size.restype = sz
         L.gdn_kda_decode_step.argtypes = L.gdn_decode_step.argtypes
         L.gdn_kda_decode_step.restype = ci
-        L.gdn_chunk_bwd_workspace_size.argtypes = [ci] * 6
+        L.gdn_chunk_bwd_workspace_size.argtypes = [ci] * 7
         L.gdn_chunk_bwd_workspace_size.restype = sz
+        L.gdn_chunk_bwd_exact_workspace_size.argtypes = [ci] * 6
+        L.gdn_chunk_bwd_exact_workspace_size.restype = sz
         L.gdn_chunk_bwd.argtypes = [vp, vp, vp, fp, fp, fp, ip, vp, fp, ci, ci, ci, ci, ci, ci,
                                     ci, fp, fp, fp, fp, fp, fp, vp, sz, vp]
         L.gdn_chunk_bwd.restype = ci
+        L.gdn_chunk_bwd_exact.argtypes = [vp, vp, vp, fp, fp, fp, ip, vp, fp, ci, ci, ci, ci, ci, ci,
+                                    ci, fp, fp, fp, fp, fp, fp, vp, sz, vp]
+        L.gdn_chunk_bwd_exact.restype = ci
         L.gdn_get_status.argtypes = [vp, vp]
         L.gdn_get_status.restype = ci
         L.gdn_set_profile_events.argtypes = [vp, vp, vp, vp]
@@ -184,19 +189,27 @@ def _chunk_call(fn, name, ws_fn, q, k, v, g, beta, initial_state, cu_seqlens, ch
     return o, fs
 
 
-def bwd_workspace_size(B, T, H, d_k, d_v, num_seqs=0) -> int:
-    return int(lib().gdn_chunk_bwd_workspace_size(B, T, H, d_k, d_v, num_seqs))
+def bwd_workspace_size(B, T, H, d_k, d_v, num_seqs=0, dtype=torch.bfloat16,
+                       exact=False) -> int:
+    """Workspace bytes of ``chunk_bwd`` (exact=False: the path gdn_chunk_bwd
+    picks for dtype; exact=True: the token-level fp32 path)."""
+    if exact:
+        return int(lib().gdn_chunk_bwd_exact_workspace_size(B, T, H, d_k, d_v, num_seqs))
+    return int(lib().gdn_chunk_bwd_workspace_size(B, T, H, d_k, d_v, num_seqs,
+                                                   _dtype_code(dtype)))
 
 
 def chunk_bwd(q, k, v, g, beta, d_o, initial_state=None, cu_seqlens=None, d_final_state=None,
-              workspace=None, stream=None):
+              workspace=None, stream=None, exact=False):
     """Gradients of ``chunk_fwd`` (scalar gate) for the loss
     sum(d_o * o) + sum(d_final_state * final_state).
 
     Inputs as for ``chunk_fwd``, plus d_o [B,T,H,d_v] (same dtype as v) and
     d_final_state [N,H,d_k,d_v] fp32 or None. Returns a dict of fp32 CUDA
     tensors: dq, dk [B,T,H,d_k], dv [B,T,H,d_v], dg, dbeta [B,T,H],
-    d_initial_state [N,H,d_k,d_v].
+    d_initial_state [N,H,d_k,d_v]. bf16 with d_k = d_v = 128 runs the chunkwise
+    tensor-core backward; exact=True (or any other size or dtype) the
+    token-level fp32 backward.
     """
     _require_cuda(q, k, v, g, beta, d_o, initial_state, cu_seqlens, d_final_state)
     B, T, H, dk = q.shape
@@ -209,18 +222,19 @@ def chunk_bwd(q, k, v, g, beta, d_o, initial_state=None, cu_seqlens=None, d_fina
                dv=torch.empty(B, T, H, dv, **f32), dg=torch.empty(B, T, H, **f32),
                dbeta=torch.empty(B, T, H, **f32),
                d_initial_state=torch.empty(N, H, dk, dv, **f32))
-    need = bwd_workspace_size(B, T, H, dk, dv, num_seqs)
+    need = bwd_workspace_size(B, T, H, dk, dv, num_seqs, q.dtype, exact)
     if need == 0:
         raise GdnError(ERR_INVALID_ARG, "gdn_chunk_bwd_workspace_size")
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
-    rc = lib().gdn_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
-                             _ptr(cu_seqlens), _ptr(d_o), _ptr(d_final_state), B, T, H, dk, dv,
-                             num_seqs, _dtype_code(q.dtype), _ptr(out["dq"]), _ptr(out["dk"]),
-                             _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dbeta"]),
-                             _ptr(out["d_initial_state"]), _ptr(workspace), workspace.numel(),
-                             _stream_ptr(stream))
-    _check(rc, "gdn_chunk_bwd")
+    fn = lib().gdn_chunk_bwd_exact if exact else lib().gdn_chunk_bwd
+    rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
+            _ptr(cu_seqlens), _ptr(d_o), _ptr(d_final_state), B, T, H, dk, dv,
+            num_seqs, _dtype_code(q.dtype), _ptr(out["dq"]), _ptr(out["dk"]),
+            _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dbeta"]),
+            _ptr(out["d_initial_state"]), _ptr(workspace), workspace.numel(),
+            _stream_ptr(stream))
+    _check(rc, "gdn_chunk_bwd_exact" if exact else "gdn_chunk_bwd")
     return out
 
 

@@ -21,6 +21,33 @@ inline BwdLayout bwd_layout(int B, int T, int H, int dk, int dv) {
   return L;
 }
 
+// Workspace of the chunkwise backward pass on the tensor cores (bf16,
+// d_k = d_v = 128, 64-token chunks): the forward pass's layout (one segment:
+// chunk table, prep tiles -W, (D K)^T, T diag(beta), P and the decay
+// factors), then per (chunk, head) unit the state entering the chunk and the
+// gradient with respect to the state leaving it, both bf16 [d_v][d_k]:
+// O(T / 64 d^2) in all.
+struct BwdTcLayout {
+  WsLayout fwd;
+  size_t s_chunks, gprime, total;
+};
+inline BwdTcLayout bwd_tc_layout(int B, int T, int H, int num_seqs) {
+  BwdTcLayout L{};
+  L.fwd = ws_layout(B, T, H, num_seqs, 64, true, 1, false);
+  const size_t units = size_t(L.fwd.max_chunks) * size_t(H);
+  L.s_chunks = L.fwd.total;
+  L.gprime = align_up(L.s_chunks + units * 128 * 128 * 2, 1024);
+  L.total = align_up(L.gprime + units * 128 * 128 * 2, 1024);
+  return L;
+}
+
+cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const float *g,
+                          const float *beta, const float *s0, const int32_t *cu,
+                          const void *d_o, const float *d_sN, int N, int B, int T, int H,
+                          int num_seqs, float *dq, float *dkk, float *dvv, float *dg,
+                          float *dbeta, float *ds0, void *ws, const BwdTcLayout &L,
+                          cudaStream_t s);
+
 cudaError_t launch_bwd(const void *q, const void *k, const void *v, const float *g,
                        const float *beta, const float *s0, const int32_t *cu, const void *d_o,
                        const float *d_sN, int N, int B, int T, int H, int dk, int dv, int dtype,

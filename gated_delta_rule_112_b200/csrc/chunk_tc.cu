@@ -752,6 +752,7 @@ __global__ void __launch_bounds__(kKdaPrepThreads, 2) gdn_kda_prep_kernel(
   grid_dependency_wait();
   const int nunits = (ctrl[0] & kErrBadSeqlens) ? 0 : int(ctrl[1]) * H;
   const long long pm_words = (long long)max_chunks * H * (64 * 64 / 2);
+  (void)pm_words;
   int it = 0;
   for (int unit = blockIdx.x; unit < nunits; unit += gridDim.x, ++it) {
     const int chunk = unit / H, h = unit - chunk * H;
@@ -1126,7 +1127,11 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     const float *__restrict__ s0, float *__restrict__ sN, __nv_bfloat16 *__restrict__ o, int H,
     uint32_t *__restrict__ ctrl, const ChunkInfo *__restrict__ table,
     const int32_t *__restrict__ seq_first, int split, float *__restrict__ sN_trans,
-    int sN_group, long long rows, int max_chunks, int n_first, int n_s0, int n_sN, int kda) {
+    int sN_group, long long rows, int max_chunks, int n_first, int n_s0, int n_sN, int kda,
+    __nv_bfloat16 *__restrict__ s_chunks) {
+  // s_chunks (may be null): the state entering every chunk, bf16 [unit][d_v][d_k]
+  // (unit = chunk * H + head, formula orientation: row i = d_v), for the
+  // backward pass.
   // kda: the channel-wise gate. Q comes per unit from the prep (Q .* e^Gamma,
   // 2-D map tm_q over [units * 64][128]), the decay records are 256 wide and
   // S decays per d_k channel.
@@ -1434,19 +1439,31 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     read_chunks();
     // bf16 copy of S (row i, columns [64 hh, 64 hh + 64)) into tensor memory,
     // then hand it to the MMA warp.
-    auto store_state = [&]() {
+    // cs: the chunk the state enters (its bf16 copy also goes to s_chunks).
+    auto store_state = [&](int cs) {
+      uint32_t pk[2][16];
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
-        uint32_t pk[16];
 #pragma unroll
-        for (int t = 0; t < 16; ++t) pk[t] = pack_bf16x2(S[32 * q + 2 * t], S[32 * q + 2 * t + 1]);
-        tmem_st16(lane_base + kT_S + 32 * hh + 16 * q, pk);
+        for (int t = 0; t < 16; ++t) pk[q][t] = pack_bf16x2(S[32 * q + 2 * t], S[32 * q + 2 * t + 1]);
+        tmem_st16(lane_base + kT_S + 32 * hh + 16 * q, pk[q]);
+      }
+      if (s_chunks && cs < nch) {
+        const long long u = (long long)(c0 + cs) * H + h;
+        if (GDN_IN_BOUNDS(ctrl, u, (long long)max_chunks * H)) {
+          uint4 *dst = reinterpret_cast<uint4 *>(s_chunks + (u * kD + i) * kD + 64 * hh);
+#pragma unroll
+          for (int q = 0; q < 2; ++q)
+#pragma unroll
+            for (int t = 0; t < 16; t += 4)
+              dst[4 * q + t / 4] = make_uint4(pk[q][t], pk[q][t + 1], pk[q][t + 2], pk[q][t + 3]);
+        }
       }
       tmem_st_wait();
       tc_fence_before();
       named_bar_arrive(kBarS, kChainHandoff);
     };
-    store_state();
+    store_state(0);
     for (int c = 0; c < nch; ++c) {
       const int gs = c & 3;
       wait(x_full, c & 1);
@@ -1500,7 +1517,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
           }
         }
       }
-      store_state();
+      store_state(c + 1);
       GDN_TRACE_POINT(tl, 0, c, 4);
       GDN_TRACE_POINT(tr && warp == 11 && lane == 0, 0, c, 15);
     }
@@ -1755,7 +1772,11 @@ bool map_2d(CUtensorMap *m, const void *base, CUtensorMapDataType t, int esize, 
 
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const float *g,
                             const float *beta, const float *s0, int B, int T, int H, int N,
-                            void *o, float *sN, void *ws, const WsLayout &L, cudaStream_t s) {
+                            void *o, float *sN, void *ws, const WsLayout &L, cudaStream_t s,
+                            __nv_bfloat16 *s_chunks) {
+  // s_chunks != null (the backward pass): the scan also stores every chunk's
+  // entering state; o may then be null (no output written; its tensor map
+  // is built over q and never stored through).
   char *base = static_cast<char *>(ws);
   uint32_t *ctrl = reinterpret_cast<uint32_t *>(base);
   const ChunkInfo *table = reinterpret_cast<const ChunkInfo *>(base + L.chunk_table);
@@ -1766,7 +1787,7 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
     CUtensorMap mq, mk, mv, mo, mw, mkt, mtb, mpm, mgm, mqt;
     const int rec = L.kda ? 256 : 128;   // decay record width
     if (!map_tokens(&mq, q, rows, H) || !map_tokens(&mk, k, rows, H) ||
-        !map_tokens(&mv, v, rows, H) || !map_tokens(&mo, o, rows, H) ||
+        !map_tokens(&mv, v, rows, H) || !map_tokens(&mo, o ? o : q, rows, H) ||
         !map_2d(&mw, base + L.w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, units * kC, kD, 64, kC,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
         !map_2d(&mkt, base + L.kt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, units * kD, 64, 64, kD,
@@ -1830,7 +1851,7 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
                                 sN, static_cast<__nv_bfloat16 *>(o), H, ctrl,
                                 static_cast<const ChunkInfo *>(table), seq_first, 0,
                                 static_cast<float *>(nullptr), 1, rows, L.max_chunks, N + 1, N,
-                                N, int(L.kda));
+                                N, int(L.kda), s_chunks);
     }
     // Segmented state scan (few long sequences): three passes over B * segs
     // segments. (1) every segment from S = 0 and as a transition, no output;
@@ -1846,7 +1867,8 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
                            static_cast<const float *>(nullptr), hbuf,
                            static_cast<__nv_bfloat16 *>(nullptr), H, ctrl,
                            static_cast<const ChunkInfo *>(table), seg_first, nseg, pbuf, 1, rows,
-                           L.max_chunks, nseg + 1, 0, nseg, int(L.kda));
+                           L.max_chunks, nseg + 1, 0, nseg, int(L.kda),
+                           static_cast<__nv_bfloat16 *>(nullptr));
     if (e != cudaSuccess) return e;
     gdn_segment_combine_kernel<<<dim3(B * H, kD / 16), 256, 0, s>>>(s0, hbuf, pbuf, sstart, H,
                                                                    L.segs, ctrl);
@@ -1860,7 +1882,7 @@ cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const f
                               static_cast<__nv_bfloat16 *>(o), H, ctrl,
                               static_cast<const ChunkInfo *>(table), seg_first, 0,
                               static_cast<float *>(nullptr), L.segs, rows, L.max_chunks, nseg + 1,
-                              nseg, B, int(L.kda));
+                              nseg, B, int(L.kda), static_cast<__nv_bfloat16 *>(nullptr));
   }
   // No tokens: the final state is the initial state.
   prof_record(g_profile.prep, s);

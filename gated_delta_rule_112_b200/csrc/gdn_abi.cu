@@ -178,17 +178,27 @@ int gdn_kda_decode_step(const void *q, const void *k, const void *v, const float
   return run_decode(true, q, k, v, g, beta, state, o, N, H, d_k, d_v, dtype, stream);
 }
 
-size_t gdn_chunk_bwd_workspace_size(int B, int T, int H, int d_k, int d_v, int num_seqs) {
+size_t gdn_chunk_bwd_exact_workspace_size(int B, int T, int H, int d_k, int d_v, int num_seqs) {
   if (B < 1 || T < 0 || H < 1 || d_k < 1 || d_v < 1 || num_seqs < 0) return 0;
   return bwd_layout(B, T, H, d_k, d_v).total;
 }
 
-int gdn_chunk_bwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
-                  const float *initial_state, const int32_t *cu_seqlens, const void *d_o,
-                  const float *d_final_state, int B, int T, int H, int d_k, int d_v,
-                  int num_seqs, int dtype, float *dq, float *dk, float *dv, float *dg,
-                  float *dbeta, float *d_initial_state, void *workspace,
-                  size_t workspace_bytes, void *stream) {
+size_t gdn_chunk_bwd_workspace_size(int B, int T, int H, int d_k, int d_v, int num_seqs,
+                                    int dtype) {
+  if (B < 1 || T < 0 || H < 1 || d_k < 1 || d_v < 1 || num_seqs < 0) return 0;
+  if (tc_path(d_k, d_v, 64, dtype)) return bwd_tc_layout(B, T, H, num_seqs).total;
+  return bwd_layout(B, T, H, d_k, d_v).total;
+}
+
+}  // extern "C"
+
+namespace {
+
+int run_bwd(bool exact, const void *q, const void *k, const void *v, const float *g,
+            const float *beta, const float *initial_state, const int32_t *cu_seqlens,
+            const void *d_o, const float *d_final_state, int B, int T, int H, int d_k, int d_v,
+            int num_seqs, int dtype, float *dq, float *dk, float *dv, float *dg, float *dbeta,
+            float *d_initial_state, void *workspace, size_t workspace_bytes, void *stream) {
   if (dtype != GDN_BF16 && dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
   if (B < 1 || T < 0 || H < 1 || d_k < 1 || d_v < 1) return GDN_ERR_INVALID_ARG;
   if (cu_seqlens && (B != 1 || num_seqs < 1)) return GDN_ERR_INVALID_ARG;
@@ -200,18 +210,63 @@ int gdn_chunk_bwd(const void *q, const void *k, const void *v, const float *g, c
     return GDN_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(d_o, 16) ||
       !aligned(g, 4) || !aligned(beta, 4) || !aligned(initial_state, 16) ||
-      !aligned(d_final_state, 16) || !aligned(d_initial_state, 16) || !aligned(dq, 4) ||
-      !aligned(dk, 4) || !aligned(dv, 4) || !aligned(dg, 4) || !aligned(dbeta, 4) ||
+      !aligned(d_final_state, 16) || !aligned(d_initial_state, 16) || !aligned(dq, 8) ||
+      !aligned(dk, 8) || !aligned(dv, 8) || !aligned(dg, 4) || !aligned(dbeta, 4) ||
       !aligned(cu_seqlens, 4))
     return GDN_ERR_INVALID_ARG;
   if (!workspace || !aligned(workspace, 256)) return GDN_ERR_WORKSPACE;
-  const BwdLayout L = bwd_layout(B, T, H, d_k, d_v);
-  if (workspace_bytes < L.total) return GDN_ERR_WORKSPACE;
   const int N = cu_seqlens ? num_seqs : B;
-  cudaError_t e = launch_bwd(q, k, v, g, beta, initial_state, cu_seqlens, d_o, d_final_state, N,
-                             B, T, H, d_k, d_v, dtype, dq, dk, dv, dg, dbeta, d_initial_state,
-                             workspace, L, static_cast<cudaStream_t>(stream));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (!exact && tc_path(d_k, d_v, 64, dtype)) {
+    const BwdTcLayout L = bwd_tc_layout(B, T, H, cu_seqlens ? num_seqs : 0);
+    if (workspace_bytes < L.total) return GDN_ERR_WORKSPACE;
+    if (T == 0) {
+      // no tokens: the initial-state gradient is the final-state gradient
+      const size_t bytes = size_t(N) * H * 128 * 128 * sizeof(float);
+      e = d_final_state ? cudaMemcpyAsync(d_initial_state, d_final_state, bytes,
+                                          cudaMemcpyDeviceToDevice, s)
+                        : cudaMemsetAsync(d_initial_state, 0, bytes, s);
+      if (e == cudaSuccess) e = cudaMemsetAsync(workspace, 0, 256, s);
+    } else {
+      e = launch_bwd_tc(q, k, v, g, beta, initial_state, cu_seqlens, d_o, d_final_state, N, B,
+                        T, H, cu_seqlens ? num_seqs : 0, dq, dk, dv, dg, dbeta,
+                        d_initial_state, workspace, L, s);
+    }
+  } else {
+    const BwdLayout L = bwd_layout(B, T, H, d_k, d_v);
+    if (workspace_bytes < L.total) return GDN_ERR_WORKSPACE;
+    e = launch_bwd(q, k, v, g, beta, initial_state, cu_seqlens, d_o, d_final_state, N, B, T, H,
+                   d_k, d_v, dtype, dq, dk, dv, dg, dbeta, d_initial_state, workspace, L, s);
+  }
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdn_chunk_bwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                  const float *initial_state, const int32_t *cu_seqlens, const void *d_o,
+                  const float *d_final_state, int B, int T, int H, int d_k, int d_v,
+                  int num_seqs, int dtype, float *dq, float *dk, float *dv, float *dg,
+                  float *dbeta, float *d_initial_state, void *workspace,
+                  size_t workspace_bytes, void *stream) {
+  return run_bwd(false, q, k, v, g, beta, initial_state, cu_seqlens, d_o, d_final_state, B, T, H,
+                 d_k, d_v, num_seqs, dtype, dq, dk, dv, dg, dbeta, d_initial_state, workspace,
+                 workspace_bytes, stream);
+}
+
+int gdn_chunk_bwd_exact(const void *q, const void *k, const void *v, const float *g,
+                        const float *beta, const float *initial_state,
+                        const int32_t *cu_seqlens, const void *d_o, const float *d_final_state,
+                        int B, int T, int H, int d_k, int d_v, int num_seqs, int dtype,
+                        float *dq, float *dk, float *dv, float *dg, float *dbeta,
+                        float *d_initial_state, void *workspace, size_t workspace_bytes,
+                        void *stream) {
+  return run_bwd(true, q, k, v, g, beta, initial_state, cu_seqlens, d_o, d_final_state, B, T, H,
+                 d_k, d_v, num_seqs, dtype, dq, dk, dv, dg, dbeta, d_initial_state, workspace,
+                 workspace_bytes, stream);
 }
 
 int gdn_get_status(void *workspace, void *stream) {

@@ -2,6 +2,7 @@
 #pragma once
 #include <cstddef>
 #include <cstdint>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "gdn.h"  // public C ABI (include/, on the -I path)
@@ -164,9 +165,11 @@ cudaError_t launch_chunk_simt(const void *q, const void *k, const void *v, const
                               const float *beta, const float *s0, const int32_t *cu, int B,
                               int T, int H, int dk, int dv, int N, int chunk, int dtype, void *o,
                               float *sN, uint32_t *err, cudaStream_t s, bool channel_gate);
+// s_chunks: see the state scan (backward pass only; requires L.segs == 1).
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const float *g,
                             const float *beta, const float *s0, int B, int T, int H, int N,
-                            void *o, float *sN, void *ws, const WsLayout &L, cudaStream_t s);
+                            void *o, float *sN, void *ws, const WsLayout &L, cudaStream_t s,
+                            __nv_bfloat16 *s_chunks = nullptr);
 // channel_gate: g is [N, H, d_k] (one log-decay per d_k channel), else [N, H].
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *g,
                           const float *beta, float *state, void *o, int N, int H, int dk, int dv,

@@ -282,10 +282,19 @@ int gdn_kda_decode_step(const void *q, const void *k, const void *v, const float
  * and d_initial_state = G at each sequence's start.
  */
 
-/* Bytes of workspace gdn_chunk_bwd needs: 256 + B*T*H*(128*128 + d_v)*4
+/* Bytes of workspace gdn_chunk_bwd needs for these sizes and dtype; 0 for
+ * invalid sizes. The chunkwise tensor-core backward (bf16, d_k = d_v = 128)
+ * needs the forward pass's gdn_chunk_fwd workspace (one scan segment) plus,
+ * per (chunk, head), two bf16 128 x 128 states (64 KB): O(T / 64 d^2). Every
+ * other size and dtype runs the token-level backward; see
+ * gdn_chunk_bwd_exact_workspace_size. */
+size_t gdn_chunk_bwd_workspace_size(int B, int T, int H, int d_k, int d_v, int num_seqs,
+                                    int dtype);
+
+/* Bytes of workspace gdn_chunk_bwd_exact needs: 256 + B*T*H*(128*128 + d_v)*4
  * (every token's S_{t-1} in a 128 x 128 fp32 block, and S_{t-1} k_t), rounded
  * up; 0 for invalid sizes. */
-size_t gdn_chunk_bwd_workspace_size(int B, int T, int H, int d_k, int d_v, int num_seqs);
+size_t gdn_chunk_bwd_exact_workspace_size(int B, int T, int H, int d_k, int d_v, int num_seqs);
 
 /*
  * gdn_chunk_bwd -- gradients of the forward pass for the loss above.
@@ -301,10 +310,18 @@ size_t gdn_chunk_bwd_workspace_size(int B, int T, int H, int d_k, int d_v, int n
  *                      initial_state is NULL: the gradient at a zero state).
  *   workspace          >= gdn_chunk_bwd_workspace_size() bytes, 256-byte
  *                      aligned, not shared with a concurrent call.
- * Supports d_k <= 128 and d_v <= 128 with d_v a multiple of 4. Runs two
- * kernels: a forward replay that stores every S_{t-1}, then the reverse
- * sweep. Bad cu_seqlens contents are reported by gdn_get_status
- * (GDN_ERR_INVALID_ARG); the affected sequences are not computed.
+ * Supports d_k <= 128 and d_v <= 128 with d_v a multiple of 4; dq, dk, dv
+ * 8-byte aligned. bf16 with d_k = d_v = 128 runs the chunkwise backward on
+ * the tensor cores (64-token chunks; the derivation is in the header of the
+ * kernels' source): the forward pass again, its scan also keeping every
+ * chunk's entering state S_c (bf16); a reverse scan over the chunks, one CTA
+ * per (sequence, head), of dS_c = gamma_last dS_{c+1} - dX^T W +
+ * (gamma dO)^T Q, keeping each chunk's dS_{c+1} (bf16); and one kernel over
+ * all (chunk, head) units for dq, dk, dv, dg, dbeta. bf16 operands, fp32
+ * accumulation: its parity bar is the bf16 tolerance. Every other size and
+ * dtype runs gdn_chunk_bwd_exact. Bad cu_seqlens contents are reported by
+ * gdn_get_status (GDN_ERR_INVALID_ARG); the affected sequences are not
+ * computed.
  */
 int gdn_chunk_bwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
                   const float *initial_state, const int32_t *cu_seqlens, const void *d_o,
@@ -312,6 +329,20 @@ int gdn_chunk_bwd(const void *q, const void *k, const void *v, const float *g, c
                   int num_seqs, int dtype, float *dq, float *dk, float *dv, float *dg,
                   float *dbeta, float *d_initial_state, void *workspace,
                   size_t workspace_bytes, void *stream);
+
+/*
+ * gdn_chunk_bwd_exact -- the same gradients by the token-level recurrence in
+ * fp32, for every supported size and dtype (bf16 inputs are upcast exactly):
+ * a forward replay that stores every S_{t-1} (gdn_chunk_bwd_exact_workspace_size
+ * bytes, O(T d^2)), then the reverse sweep. Arguments as gdn_chunk_bwd.
+ */
+int gdn_chunk_bwd_exact(const void *q, const void *k, const void *v, const float *g,
+                        const float *beta, const float *initial_state,
+                        const int32_t *cu_seqlens, const void *d_o, const float *d_final_state,
+                        int B, int T, int H, int d_k, int d_v, int num_seqs, int dtype,
+                        float *dq, float *dk, float *dv, float *dg, float *dbeta,
+                        float *d_initial_state, void *workspace, size_t workspace_bytes,
+                        void *stream);
 
 /*
  * gdn_selftest_wait_timeout -- device self-test of the bounded waits (the

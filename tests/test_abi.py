@@ -186,8 +186,16 @@ def test_bwd_host_checks(L):
     assert call(ns=2) == gdn.ERR_INVALID_ARG                  # num_seqs without cu_seqlens
     assert call(ws=None) == gdn.ERR_WORKSPACE
     assert call(wsb=1000) == gdn.ERR_WORKSPACE
-    # every token's S_{t-1} and S_{t-1} k_t in fp32, plus the control block
-    need = L.gdn_chunk_bwd_workspace_size(4, 4096, 16, 128, 128, 0)
+    # token-level path: every token's S_{t-1} and S_{t-1} k_t in fp32, plus the control block
+    need = L.gdn_chunk_bwd_exact_workspace_size(4, 4096, 16, 128, 128, 0)
     assert need >= 4 * 4096 * 16 * (128 * 128 + 128) * 4
     assert need < 4 * 4096 * 16 * (128 * 128 + 128) * 4 + 4096
-    assert L.gdn_chunk_bwd_workspace_size(0, 1, 1, 128, 128, 0) == 0
+    assert L.gdn_chunk_bwd_workspace_size(4, 4096, 16, 128, 128, 0, gdn.F32) == need
+    assert L.gdn_chunk_bwd_exact_workspace_size(0, 1, 1, 128, 128, 0) == 0
+    assert L.gdn_chunk_bwd_workspace_size(0, 1, 1, 128, 128, 0, gdn.BF16) == 0
+    # chunkwise path (bf16, d = 128): the forward's workspace plus two bf16
+    # 128 x 128 states per (chunk, head) unit
+    tc = L.gdn_chunk_bwd_workspace_size(4, 4096, 16, 128, 128, 0, gdn.BF16)
+    fwd = L.gdn_chunk_fwd_workspace_size(4, 4096, 16, 128, 128, 0, 64, gdn.BF16)
+    assert tc >= fwd + 4096 * 2 * 128 * 128 * 2
+    assert tc < fwd + 4096 * 2 * 128 * 128 * 2 + (1 << 20)

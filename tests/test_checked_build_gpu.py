@@ -65,6 +65,28 @@ def _cases():
                                        None if cu is None else cu.numpy())
         assert_close("o", np64(o), ro, TOL_BF16)
         assert_close("final_state", np64(fs), rfs, TOL_BF16)
+    # the chunkwise backward (forward replay with chunk states, reverse chain,
+    # per-unit gradients)
+    wb = Workload("chk_bwd", B=1, T=64, H=1, d_k=128, d_v=128, seed=73)
+    for inp in (make_chunk_inputs(wb, B=2, H=3, T=193, random_state=True),
+                make_chunk_inputs(wb, H=2, lengths=[70, 0, 1, 130, 64], random_state=True)):
+        d = to_dev(inp)
+        gen = torch.Generator("cpu").manual_seed(5)
+        d_o = torch.randn(inp["B"], inp["T"], inp["H"], 128, generator=gen).to(torch.bfloat16)
+        dsN = 0.1 * torch.randn(inp["num_seqs"], inp["H"], 128, 128, generator=gen)
+        num_seqs = inp["num_seqs"] if inp["cu_seqlens"] is not None else 0
+        ws = torch.empty(gdn.bwd_workspace_size(inp["B"], inp["T"], inp["H"], 128, 128, num_seqs),
+                         dtype=torch.uint8, device="cuda")
+        got = gdn.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d_o.cuda(),
+                            d["initial_state"], d["cu_seqlens"], dsN.cuda(), workspace=ws)
+        status = gdn.get_status(ws)
+        assert status == gdn.OK, gdn.lib().gdn_status_string(status)
+        cu = inp["cu_seqlens"]
+        ref = oracle.chunk_bwd(np64(inp["q"]), np64(inp["k"]), np64(inp["v"]), np64(inp["g"]),
+                               np64(inp["beta"]), np64(d_o), np64(inp["initial_state"]),
+                               None if cu is None else cu.numpy(), np64(dsN))
+        for key in ("dq", "dk", "dv", "dg", "dbeta", "d_initial_state"):
+            assert_close(key, np64(got[key]), ref[key], TOL_BF16)
     print("checked build: all cases clean")
 
 
