@@ -53,7 +53,7 @@ constexpr uint32_t kT64x128 = 64 * kLd128 * 2;    // [64][128] tile, 17,408 B
 constexpr uint32_t kT128x128 = 128 * kLd128 * 2;  // [128][128] tile, 34,816 B
 constexpr uint32_t kT64x64 = 64 * kLd64 * 2;      // [64][64] tile, 9,216 B
 constexpr uint32_t kT128x64 = 128 * kLd64 * 2;    // [128][64] tile, 18,432 B
-constexpr int kThreads = 256;
+constexpr int kThreads = 256, kWarps = kThreads / 32;   // the unit kernel's block
 constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
@@ -84,15 +84,15 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // One warp: acc[MT][NT] (16 x 8 tiles, rows m0 + 16 mt, columns n0 + 8 nt)
-// += op(A) op(B) over k in [0, K). A is stored [m][k] (AT = false) or [k][m]
+// += op(A) op(B) over k in [0, K) (fully unrolled). A is stored [m][k] (AT = false) or [k][m]
 // (AT = true) at shared address A with row stride lda elements; B is stored
 // [n][k] (BT = false) or [k][n] (BT = true). Fragment layout of acc[mt][nt]:
 // with g = lane / 4, t = lane % 4, elements (g, 2t), (g, 2t+1), (g+8, 2t),
 // (g+8, 2t+1) of the tile. NT is even (B is read two n-tiles at a time).
-template <int MT, int NT, bool AT, bool BT>
+template <int MT, int NT, bool AT, bool BT, int K>
 __device__ __forceinline__ void warp_mma(float (&acc)[MT][NT][4], uint32_t A, int lda, int m0,
-                                         uint32_t B, int ldb, int n0, int K, int lane) {
-#pragma unroll 2
+                                         uint32_t B, int ldb, int n0, int lane) {
+#pragma unroll
   for (int k0 = 0; k0 < K; k0 += 16) {
     uint32_t a[MT][4];
 #pragma unroll
@@ -119,6 +119,56 @@ __device__ __forceinline__ void warp_mma(float (&acc)[MT][NT][4], uint32_t A, in
       for (int mt = 0; mt < MT; ++mt) {
         mma16816(acc[mt][nt], a[mt], b[0], b[1]);
         mma16816(acc[mt][nt + 1], a[mt], b[2], b[3]);
+      }
+    }
+  }
+}
+
+// Two independent products of the same shape and depth in one loop (twice
+// the independent accumulators per step): acc1 += op(A1) op(B1), acc2 +=
+// op(A2) op(B2), operands as for warp_mma.
+template <int MT, int NT, bool AT1, bool BT1, bool AT2, bool BT2, int K>
+__device__ __forceinline__ void warp_mma2(float (&acc1)[MT][NT][4], uint32_t A1, int lda1,
+                                          uint32_t B1, int ldb1, float (&acc2)[MT][NT][4],
+                                          uint32_t A2, int lda2, uint32_t B2, int ldb2, int m0,
+                                          int n0, int lane) {
+#pragma unroll
+  for (int k0 = 0; k0 < K; k0 += 16) {
+    uint32_t a1[MT][4], a2[MT][4];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      if (!AT1)
+        ldsm_x4(A1 + 2u * uint32_t((m0 + 16 * mt + (lane & 15)) * lda1 + k0 + 8 * (lane >> 4)), a1[mt]);
+      else
+        ldsm_x4_trans(A1 + 2u * uint32_t((k0 + (lane & 7) + 8 * (lane >> 4)) * lda1 + m0 + 16 * mt +
+                                         8 * ((lane >> 3) & 1)), a1[mt]);
+      if (!AT2)
+        ldsm_x4(A2 + 2u * uint32_t((m0 + 16 * mt + (lane & 15)) * lda2 + k0 + 8 * (lane >> 4)), a2[mt]);
+      else
+        ldsm_x4_trans(A2 + 2u * uint32_t((k0 + (lane & 7) + 8 * (lane >> 4)) * lda2 + m0 + 16 * mt +
+                                         8 * ((lane >> 3) & 1)), a2[mt]);
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; nt += 2) {
+      uint32_t b1[4], b2[4];
+      if (!BT1)
+        ldsm_x4(B1 + 2u * uint32_t((n0 + 8 * nt + 8 * (lane >> 4) + (lane & 7)) * ldb1 + k0 +
+                                   8 * ((lane >> 3) & 1)), b1);
+      else
+        ldsm_x4_trans(B1 + 2u * uint32_t((k0 + (lane & 7) + 8 * ((lane >> 3) & 1)) * ldb1 + n0 +
+                                         8 * nt + 8 * (lane >> 4)), b1);
+      if (!BT2)
+        ldsm_x4(B2 + 2u * uint32_t((n0 + 8 * nt + 8 * (lane >> 4) + (lane & 7)) * ldb2 + k0 +
+                                   8 * ((lane >> 3) & 1)), b2);
+      else
+        ldsm_x4_trans(B2 + 2u * uint32_t((k0 + (lane & 7) + 8 * ((lane >> 3) & 1)) * ldb2 + n0 +
+                                         8 * nt + 8 * (lane >> 4)), b2);
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        mma16816(acc1[mt][nt], a1[mt], b1[0], b1[1]);
+        mma16816(acc2[mt][nt], a2[mt], b2[0], b2[1]);
+        mma16816(acc1[mt][nt + 1], a1[mt], b1[2], b1[3]);
+        mma16816(acc2[mt][nt + 1], a2[mt], b2[2], b2[3]);
       }
     }
   }
@@ -166,22 +216,27 @@ __device__ __forceinline__ void load_dense(uint32_t dst, const bf16 *src, int ro
 }
 
 // ------------------------------------------------------------------ chain
-// Shared memory of the chain kernel: G (bf16, [d_v][d_k]), dX (bf16,
-// [tokens][d_v]) and two stages of one chunk's inputs.
-constexpr uint32_t kCh_G = 0;
-constexpr uint32_t kCh_DX = kCh_G + kT128x128;
-constexpr uint32_t kCh_STAGE = kCh_DX + kT64x128;
-constexpr uint32_t kSt_KT = 0;                       // (D K)^T [d_k][tokens]
-constexpr uint32_t kSt_PM = kSt_KT + kT128x64;       // P [r][s]
-constexpr uint32_t kSt_DO = kSt_PM + kT64x64;        // dO [tokens][d_v], then gamma dO
-constexpr uint32_t kSt_WN = kSt_DO + kT64x128;       // -W [tokens][d_k]
-constexpr uint32_t kSt_Q = kSt_WN + kT64x128;        // Q [tokens][d_k]
-constexpr uint32_t kSt_GAM = kSt_Q + kT64x128;       // gamma [64], D [64]
-constexpr uint32_t kStage = kSt_GAM + 128 * 4;
-constexpr uint32_t kChainSmem = kCh_STAGE + 2 * kStage;
-static_assert(kChainSmem <= 232448, "chain kernel shared memory");
+// Row i of dS_c depends only on row i of dS_{c+1} (dX column i only on row i
+// of G'), so each (sequence, head) chain runs as kSlices CTAs of kSlice d_v
+// rows, two CTAs per SM. Shared memory: the G slice (bf16 [kSlice][d_k]), the
+// dX slice (bf16 [tokens][kSlice]), one chunk's (D K)^T, P, -W and Q, and two
+// stages of the dO slice and the decay factors. (D K)^T and P of the next
+// chunk load while the G update runs, -W and Q while the next dX runs.
+constexpr int kSlices = 4, kSlice = kD / kSlices, kLdS = kSlice + 8;
+constexpr int kChainThreads = 256, kChainWarps = kChainThreads / 32;
+constexpr uint32_t kTDoS = 64 * kLdS * 2;             // [64][kSlice] tile
+constexpr uint32_t kCh_G = 0;                          // [kSlice][kLd128]
+constexpr uint32_t kCh_DX = kCh_G + kSlice * kLd128 * 2;
+constexpr uint32_t kCh_KT = kCh_DX + kTDoS;            // (D K)^T [d_k][tokens]
+constexpr uint32_t kCh_PM = kCh_KT + kT128x64;         // P [r][s]
+constexpr uint32_t kCh_WN = kCh_PM + kT64x64;          // -W [tokens][d_k]
+constexpr uint32_t kCh_Q = kCh_WN + kT64x128;          // Q [tokens][d_k]
+constexpr uint32_t kCh_DO = kCh_Q + kT64x128;          // 2 x dO slice, then gamma dO
+constexpr uint32_t kCh_GAM = kCh_DO + 2 * kTDoS;       // 2 x (gamma [64], D [64])
+constexpr uint32_t kChainSmem = kCh_GAM + 2 * 128 * 4;
+static_assert(2 * (kChainSmem + 1024) <= 233472, "chain kernel: two CTAs per SM");
 
-__global__ void __launch_bounds__(kThreads, 1) gdn_bwd_chain_kernel(
+__global__ void __launch_bounds__(kChainThreads, 2) gdn_bwd_chain_kernel(
     const bf16 *__restrict__ q, const bf16 *__restrict__ d_o, const float *__restrict__ d_sN,
     float *__restrict__ ds0, const uint8_t *__restrict__ ws_w, const uint8_t *__restrict__ ws_kt,
     const uint8_t *__restrict__ ws_pm, const float *__restrict__ ws_gam,
@@ -192,8 +247,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_chain_kernel(
   extern __shared__ __align__(16) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
-  const int n = blockIdx.x, h = blockIdx.y;
-  const uint32_t sbase = smem_u32(smem);
+  const int n = blockIdx.x, h = blockIdx.y, i0 = kSlice * int(blockIdx.z);
+  const uint32_t sb = smem_u32(smem);
   bf16 *Gs = reinterpret_cast<bf16 *>(smem + kCh_G);
   bf16 *DXs = reinterpret_cast<bf16 *>(smem + kCh_DX);
   int c0 = 0, nch = 0;
@@ -201,106 +256,138 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_chain_kernel(
     c0 = seq_first[n];
     nch = seq_first[n + 1] - c0;
   }
-  // G = dL/dS (formula orientation [d_v i][d_k j]); warp w owns rows
-  // [16 w, 16 w + 16), all 128 columns: acc[0][nt] = rows 16 w + g (+8),
-  // columns 8 nt + 2 t (+1).
-  float G[1][16][4];
+  // G = dL/dS rows [i0, i0 + kSlice) (formula orientation [d_v i][d_k j]);
+  // warp w: local rows [gm0, gm0 + 16), columns [gn0, gn0 + 32).
+  constexpr int kGT = 4;
+  const int gm0 = 16 * (warp & 1), gn0 = 32 * (warp >> 1);
+  float G[1][kGT][4];
   {
     const float *src = d_sN ? d_sN + (size_t(n) * H + h) * kD * kD : nullptr;
 #pragma unroll
-    for (int nt = 0; nt < 16; ++nt)
+    for (int nt = 0; nt < kGT; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int i = 16 * warp + g + 8 * (e >> 1), j = 8 * nt + 2 * t + (e & 1);
+        const int i = i0 + gm0 + g + 8 * (e >> 1), j = gn0 + 8 * nt + 2 * t + (e & 1);
         G[0][nt][e] = src ? src[j * kD + i] : 0.f;   // stored [d_k][d_v]
       }
   }
-  auto stage_addr = [&](int st) { return sbase + kCh_STAGE + uint32_t(st) * kStage; };
-  auto issue_loads = [&](int c, int st) {   // chunk c of this sequence into stage st
+  auto unit_of = [&](int c) { return (long long)(c0 + c) * H + h; };
+  auto info_of = [&](int c) {
     const long long chunk = c0 + c;
-    const long long unit = chunk * H + h;
-    const ChunkInfo ci = GDN_IN_BOUNDS(ctrl, chunk, max_chunks) ? table[chunk] : ChunkInfo{0, 0, 0, 0};
-    const uint32_t sa = stage_addr(st);
-    load_dense<64>(sa + kSt_KT, reinterpret_cast<const bf16 *>(ws_kt) + unit * (kD * kC), 128, tid);
-    load_dense<64>(sa + kSt_PM, reinterpret_cast<const bf16 *>(ws_pm) + unit * (kC * kC), 64, tid);
-    load_dense<128>(sa + kSt_WN, reinterpret_cast<const bf16 *>(ws_w) + unit * (kC * kD), 64, tid);
-    load_tokens(sa + kSt_DO, d_o + size_t(h) * kD, ci.row0, (long long)H * kD, ci.len, tid);
-    load_tokens(sa + kSt_Q, q + size_t(h) * kD, ci.row0, (long long)H * kD, ci.len, tid);
-    if (tid < 32) cp_async16(sa + kSt_GAM + 16 * tid, ws_gam + unit * 128 + 4 * tid, 16u);
+    return GDN_IN_BOUNDS(ctrl, chunk, max_chunks) ? table[chunk] : ChunkInfo{0, 0, 0, 0};
+  };
+  // group A: (D K)^T, P, the dO slice and the decay factors of chunk c
+  auto load_a = [&](int c, int st) {
+    if (c >= 0) {
+      const long long unit = unit_of(c);
+      const ChunkInfo ci = info_of(c);
+      for (int e = tid; e < 128 * 8; e += kChainThreads) {
+        const int r = e >> 3, cc = e & 7;
+        cp_async16(sb + kCh_KT + uint32_t(r * kLd64 + 8 * cc) * 2u,
+                   reinterpret_cast<const bf16 *>(ws_kt) + unit * (kD * kC) + r * kC + 8 * cc, 16u);
+      }
+      for (int e = tid; e < 64 * 8; e += kChainThreads) {
+        const int r = e >> 3, cc = e & 7;
+        cp_async16(sb + kCh_PM + uint32_t(r * kLd64 + 8 * cc) * 2u,
+                   reinterpret_cast<const bf16 *>(ws_pm) + unit * (kC * kC) + r * kC + 8 * cc, 16u);
+      }
+      for (int e = tid; e < 64 * (kSlice / 8); e += kChainThreads) {
+        const int r = e / (kSlice / 8), cc = e - r * (kSlice / 8);
+        const bool ok = r < ci.len;
+        const bf16 *src = ok ? d_o + ((long long)ci.row0 + r) * H * kD + size_t(h) * kD + i0 + 8 * cc
+                             : d_o;
+        cp_async16(sb + kCh_DO + st * kTDoS + uint32_t(r * kLdS + 8 * cc) * 2u, src, ok ? 16u : 0u);
+      }
+      if (tid < 32)
+        cp_async16(sb + kCh_GAM + st * 512 + 16 * tid, ws_gam + unit * 128 + 4 * tid, 16u);
+    }
     cp_async_commit();
   };
-  if (nch > 0) issue_loads(nch - 1, 0);
+  // group B: -W and Q of chunk c
+  auto load_b = [&](int c) {
+    if (c >= 0) {
+      const long long unit = unit_of(c);
+      const ChunkInfo ci = info_of(c);
+      for (int e = tid; e < 64 * 16; e += kChainThreads) {
+        const int r = e >> 4, cc = e & 15;
+        cp_async16(sb + kCh_WN + uint32_t(r * kLd128 + 8 * cc) * 2u,
+                   reinterpret_cast<const bf16 *>(ws_w) + unit * (kC * kD) + r * kD + 8 * cc, 16u);
+        const bool ok = r < ci.len;
+        const bf16 *src = ok ? q + ((long long)ci.row0 + r) * H * kD + size_t(h) * kD + 8 * cc : q;
+        cp_async16(sb + kCh_Q + uint32_t(r * kLd128 + 8 * cc) * 2u, src, ok ? 16u : 0u);
+      }
+    }
+    cp_async_commit();
+  };
+  load_a(nch - 1, 0);
+  load_b(nch - 1);
   for (int it = 0; it < nch; ++it) {
     const int c = nch - 1 - it, st = it & 1;
-    const long long unit = (long long)(c0 + c) * H + h;
-    if (it + 1 < nch) {
-      issue_loads(c - 1, st ^ 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    // G' of this chunk: bf16 into shared memory (operand) and the workspace.
+    const long long unit = unit_of(c);
+    // G' slice of this chunk: bf16 into shared memory (operand) and the workspace
 #pragma unroll
-    for (int nt = 0; nt < 16; ++nt) {
-      const int i = 16 * warp + g, j = 8 * nt + 2 * t;
+    for (int nt = 0; nt < kGT; ++nt) {
+      const int i = gm0 + g, j = gn0 + 8 * nt + 2 * t;
       st_pair(Gs, kLd128, i, j, G[0][nt][0], G[0][nt][1]);
       st_pair(Gs, kLd128, i + 8, j, G[0][nt][2], G[0][nt][3]);
     }
-    __syncthreads();   // stage st landed for every thread's copies; Gs complete
+    cp_async_wait<1>();   // group A of this chunk (B may still be in flight)
+    __syncthreads();
     if (GDN_IN_BOUNDS(ctrl, unit, (long long)max_chunks * H)) {
-      uint4 *dst = reinterpret_cast<uint4 *>(gprime + unit * (kD * kD));
-      for (int e = tid; e < 128 * 16; e += kThreads) {
+      uint4 *dst = reinterpret_cast<uint4 *>(gprime + unit * (kD * kD) + size_t(i0) * kD);
+      for (int e = tid; e < kSlice * 16; e += kChainThreads) {
         const int r = e >> 4, cc = e & 15;
         dst[r * 16 + cc] = *reinterpret_cast<const uint4 *>(Gs + r * kLd128 + 8 * cc);
       }
     }
-    const uint32_t sa = stage_addr(st);
-    const float *gam = reinterpret_cast<const float *>(smem + kCh_STAGE + st * kStage + kSt_GAM);
-    bf16 *DO = reinterpret_cast<bf16 *>(smem + kCh_STAGE + st * kStage + kSt_DO);
+    const float *gam = reinterpret_cast<const float *>(smem + kCh_GAM + st * 512);
+    bf16 *DO = reinterpret_cast<bf16 *>(smem + kCh_DO + st * kTDoS);
     {
-      // dX = P^T dO + (D K) G^T: warp w -> tokens [16 (w % 4), +16), d_v [64 (w / 4), +64)
-      const int m0 = 16 * (warp & 3), n0 = 64 * (warp >> 2);
-      float acc[1][8][4];
+      // dX slice = P^T dO + (D K) G^T: warp w -> tokens [16 (w % 4), +16),
+      // local d_v [16 (w / 4), +16)
+      const int m0 = 16 * (warp & 3), n0 = 16 * (warp >> 2);
+      float acc[1][2][4];
       zero_acc(acc);
-      warp_mma<1, 8, true, true>(acc, sa + kSt_PM, kLd64, m0, sa + kSt_DO, kLd128, n0, 64, lane);
-      warp_mma<1, 8, true, false>(acc, sa + kSt_KT, kLd64, m0, sbase + kCh_G, kLd128, n0, 128,
-                                  lane);
+      warp_mma<1, 2, true, true, 64>(acc, sb + kCh_PM, kLd64, m0, sb + kCh_DO + st * kTDoS, kLdS, n0, lane);
+      warp_mma<1, 2, true, false, 128>(acc, sb + kCh_KT, kLd64, m0, sb + kCh_G, kLd128, n0, lane);
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
+      for (int nt = 0; nt < 2; ++nt) {
         const int r = m0 + g, cc = n0 + 8 * nt + 2 * t;
-        st_pair(DXs, kLd128, r, cc, acc[0][nt][0], acc[0][nt][1]);
-        st_pair(DXs, kLd128, r + 8, cc, acc[0][nt][2], acc[0][nt][3]);
+        st_pair(DXs, kLdS, r, cc, acc[0][nt][0], acc[0][nt][1]);
+        st_pair(DXs, kLdS, r + 8, cc, acc[0][nt][2], acc[0][nt][3]);
       }
     }
-    __syncthreads();   // dX complete; every read of the unscaled dO done
+    __syncthreads();   // dX complete; (D K)^T, P and the unscaled dO no longer read
+    load_a(c - 1, st ^ 1);
     // gamma dO in place (bf16, rounded once)
-    for (int e = tid; e < 64 * 64; e += kThreads) {
-      const int r = e >> 6, cc = 2 * (e & 63);
-      const float2 x = ld_pair(DO, kLd128, r, cc);
-      st_pair(DO, kLd128, r, cc, gam[r] * x.x, gam[r] * x.y);
+    for (int e = tid; e < 64 * (kSlice / 2); e += kChainThreads) {
+      const int r = e / (kSlice / 2), cc = 2 * (e - r * (kSlice / 2));
+      const float2 x = ld_pair(DO, kLdS, r, cc);
+      st_pair(DO, kLdS, r, cc, gam[r] * x.x, gam[r] * x.y);
     }
+    cp_async_wait<1>();   // group B of this chunk
     __syncthreads();
     {
-      // G <- gamma_last G - dX^T W + (gamma dO)^T Q  (rows 16 w.., all d_k)
+      // G <- gamma_last G - dX^T W + (gamma dO)^T Q
       const float gl = gam[kC - 1];
 #pragma unroll
-      for (int nt = 0; nt < 16; ++nt)
+      for (int nt = 0; nt < kGT; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) G[0][nt][e] *= gl;
-      warp_mma<1, 16, true, true>(G, sbase + kCh_DX, kLd128, 16 * warp, sa + kSt_WN, kLd128, 0,
-                                  64, lane);
-      warp_mma<1, 16, true, true>(G, sa + kSt_DO, kLd128, 16 * warp, sa + kSt_Q, kLd128, 0, 64,
-                                  lane);
+      warp_mma<1, kGT, true, true, 64>(G, sb + kCh_DX, kLdS, gm0, sb + kCh_WN, kLd128, gn0, lane);
+      warp_mma<1, kGT, true, true, 64>(G, sb + kCh_DO + st * kTDoS, kLdS, gm0, sb + kCh_Q, kLd128, gn0, lane);
     }
-    __syncthreads();   // Gs, dXs and stage st free for the next chunk
+    __syncthreads();   // G slice, dX, -W and Q free
+    load_b(c - 1);
   }
+  cp_async_wait<0>();
   if (!(ctrl[0] & kErrBadSeqlens) && GDN_IN_BOUNDS(ctrl, (long long)n * H + h, (long long)N * H)) {
     float *dst = ds0 + (size_t(n) * H + h) * kD * kD;
 #pragma unroll
-    for (int nt = 0; nt < 16; ++nt)
+    for (int nt = 0; nt < kGT; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int i = 16 * warp + g + 8 * (e >> 1), j = 8 * nt + 2 * t + (e & 1);
+        const int i = i0 + gm0 + g + 8 * (e >> 1), j = gn0 + 8 * nt + 2 * t + (e & 1);
         dst[j * kD + i] = G[0][nt][e];
       }
   }
@@ -319,9 +406,54 @@ constexpr uint32_t kU_W = kU_P + kT64x64;         // -W; then dX
 constexpr uint32_t kU_KT = kU_W + kT64x128;       // (D K)^T [d_k][tokens]; then dV
 constexpr uint32_t kU_X = kU_KT + kT128x64;       // X
 constexpr uint32_t kU_VEC = kU_X + kT64x128;      // Gamma, gamma, D, dGamma, dbeta, delta [64] each
-constexpr uint32_t kU_RED = kU_VEC + 6 * 64 * 4;  // block reduction scratch [8]
-constexpr uint32_t kUnitSmem = kU_RED + 64;
+constexpr uint32_t kU_RED = kU_VEC + 6 * 64 * 4;  // block reduction scratch [kWarps]
+constexpr uint32_t kUnitSmem = kU_RED + 4 * kWarps;
 static_assert(kT128x64 >= kT64x128 && kUnitSmem <= 232448, "unit kernel shared memory");
+
+// Calls f(mt, nt, hf, row, col) for every fragment pair (row, col..col+1)
+// of a warp's acc[MT][NT] tile with origin (m0, n0); the pair is
+// acc[mt][nt][2 hf], acc[mt][nt][2 hf + 1].
+template <int MT, int NT, typename F>
+__device__ __forceinline__ void each_pair(int m0, int n0, int lane, F &&f) {
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf)
+        f(mt, nt, hf, m0 + 16 * mt + (lane >> 2) + 8 * hf, n0 + 8 * nt + 2 * (lane & 3));
+}
+
+// Adds the per-row partial sums part[mt][hf] of a warp tile (rows m0 + 16 mt
+// + lane / 4 + 8 hf) over the four lanes of a row, then into dst[row].
+template <int MT>
+__device__ __forceinline__ void add_rows(float *dst, float (&part)[MT][2], int m0, int lane) {
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      float x = part[mt][hf];
+      x += __shfl_xor_sync(0xffffffffu, x, 1);
+      x += __shfl_xor_sync(0xffffffffu, x, 2);
+      if ((lane & 3) == 0) atomicAdd(dst + m0 + 16 * mt + (lane >> 2) + 8 * hf, x);
+    }
+}
+
+// Subtracts the per-column partial sums part[nt][2] (columns n0 + 8 nt + 2 t,
+// +1) over the eight lanes of a column, then from dst[col].
+template <int NT>
+__device__ __forceinline__ void sub_cols(float *dst, float (&part)[NT][2], int n0, int lane) {
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      float x = part[nt][b];
+      x += __shfl_xor_sync(0xffffffffu, x, 4);
+      x += __shfl_xor_sync(0xffffffffu, x, 8);
+      x += __shfl_xor_sync(0xffffffffu, x, 16);
+      if ((lane >> 2) == 0) atomicAdd(dst + n0 + 8 * nt + 2 * (lane & 3) + b, -x);
+    }
+}
 
 __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
     const bf16 *__restrict__ q, const bf16 *__restrict__ k, const bf16 *__restrict__ v,
@@ -335,7 +467,6 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
   (void)rows;
   extern __shared__ __align__(16) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int gq = lane >> 2, tq = lane & 3;
   const uint32_t sb = smem_u32(smem);
   bf16 *Qs = reinterpret_cast<bf16 *>(smem + kU_Q);
   bf16 *Ks = reinterpret_cast<bf16 *>(smem + kU_K);
@@ -352,9 +483,25 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
         *delta = Gam + 320;
   float *red = reinterpret_cast<float *>(smem + kU_RED);
   const int nunits = (ctrl[0] & kErrBadSeqlens) ? 0 : int(ctrl[1]) * H;
-  // Output tiles of 64 x 128: warp w -> rows [16 (w % 4), +16), columns
-  // [64 (w / 4), +64); of 64 x 64: rows [16 (w % 4), +16), columns [32 (w / 4), +32).
-  const int m0 = 16 * (warp & 3), n0 = 64 * (warp >> 2), p0 = 32 * (warp >> 2);
+  // Warp tiles: 64 x 128 outputs as 2 x 4 tiles of 32 x 32 (rows m0, columns
+  // n0); 64 x 64 outputs as 2 x 4 tiles of 32 x 16 (columns p0).
+  constexpr int kMT = 2, kNT = 4, kNP = 2;
+  const int m0 = 32 * (warp & 1), n0 = 32 * (warp >> 1), p0 = 16 * (warp >> 1);
+  using Acc = float[kMT][kNT][4];
+  using AccP = float[kMT][kNP][4];
+  // stores a 64 x 128 fp32 result tile (rows < len) to out [B*T][H][128]
+  auto store_out = [&](float *out, Acc &a, const ChunkInfo &ci, int h) {
+    each_pair<kMT, kNT>(m0, n0, lane, [&](int mt, int nt, int hf, int r, int c) {
+      const long long o = (((long long)ci.row0 + r) * H + h) * kD + c;
+      if (r < ci.len && GDN_IN_BOUNDS(ctrl, o + 1, rows * H * kD))
+        *reinterpret_cast<float2 *>(out + o) = make_float2(a[mt][nt][2 * hf], a[mt][nt][2 * hf + 1]);
+    });
+  };
+  auto store_tile = [&](bf16 *t, Acc &a) {
+    each_pair<kMT, kNT>(m0, n0, lane, [&](int mt, int nt, int hf, int r, int c) {
+      st_pair(t, kLd128, r, c, a[mt][nt][2 * hf], a[mt][nt][2 * hf + 1]);
+    });
+  };
   for (int unit = blockIdx.x; unit < nunits; unit += gridDim.x) {
     const int chunk = unit / H, h = unit - chunk * H;
     const ChunkInfo ci =
@@ -403,294 +550,158 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
     cp_async_wait<0>();
     __syncthreads();
     // <G', S> (for the last token's dGamma)
-    float gs_dot = 0.f;
-    for (int e = tid; e < 128 * 64; e += kThreads) {
-      const int r = e >> 6, c = 2 * (e & 63);
-      const float2 a = ld_pair(Gp, kLd128, r, c), b = ld_pair(Ss, kLd128, r, c);
-      gs_dot += a.x * b.x + a.y * b.y;
-    }
+    {
+      float gs_dot = 0.f;
+      for (int e = tid; e < 128 * 64; e += kThreads) {
+        const int r = e >> 6, c = 2 * (e & 63);
+        const float2 a = ld_pair(Gp, kLd128, r, c), b = ld_pair(Ss, kLd128, r, c);
+        gs_dot += a.x * b.x + a.y * b.y;
+      }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) gs_dot += __shfl_xor_sync(0xffffffffu, gs_dot, off);
-    if (lane == 0) red[warp] = gs_dot;
+      for (int off = 16; off > 0; off >>= 1) gs_dot += __shfl_xor_sync(0xffffffffu, gs_dot, off);
+      if (lane == 0) red[warp] = gs_dot;
+    }
 
-    // X = TB V + (-W) S^T ; kept in fp32 for delta
-    float xr[1][8][4];
+    // X = TB V + (-W) S^T; kept in fp32 for delta
+    Acc xr;
     zero_acc(xr);
-    warp_mma<1, 8, false, true>(xr, sb + kU_TB, kLd64, m0, sb + kU_V, kLd128, n0, 64, lane);
-    warp_mma<1, 8, false, false>(xr, sb + kU_W, kLd128, m0, sb + kU_S, kLd128, n0, 128, lane);
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      const int r = m0 + gq, c = n0 + 8 * nt + 2 * tq;
-      st_pair(Xs, kLd128, r, c, xr[0][nt][0], xr[0][nt][1]);
-      st_pair(Xs, kLd128, r + 8, c, xr[0][nt][2], xr[0][nt][3]);
-    }
+    warp_mma<kMT, kNT, false, true, 64>(xr, sb + kU_TB, kLd64, m0, sb + kU_V, kLd128, n0, lane);
+    warp_mma<kMT, kNT, false, false, 128>(xr, sb + kU_W, kLd128, m0, sb + kU_S, kLd128, n0, lane);
+    store_tile(Xs, xr);
     __syncthreads();   // X complete; -W no longer read
     // dX = P^T dO + (D K) G'^T;  delta_s = X_s . ((D K) G'^T)_s
-    float dx[1][8][4];
+    Acc dx;
     zero_acc(dx);
-    warp_mma<1, 8, true, false>(dx, sb + kU_KT, kLd64, m0, sb + kU_GP, kLd128, n0, 128, lane);
+    warp_mma<kMT, kNT, true, false, 128>(dx, sb + kU_KT, kLd64, m0, sb + kU_GP, kLd128, n0, lane);
     {
-      float d0 = 0.f, d1 = 0.f;
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        d0 += xr[0][nt][0] * dx[0][nt][0] + xr[0][nt][1] * dx[0][nt][1];
-        d1 += xr[0][nt][2] * dx[0][nt][2] + xr[0][nt][3] * dx[0][nt][3];
-      }
-      d0 += __shfl_xor_sync(0xffffffffu, d0, 1);
-      d0 += __shfl_xor_sync(0xffffffffu, d0, 2);
-      d1 += __shfl_xor_sync(0xffffffffu, d1, 1);
-      d1 += __shfl_xor_sync(0xffffffffu, d1, 2);
-      if (tq == 0) {
-        atomicAdd(delta + m0 + gq, d0);
-        atomicAdd(delta + m0 + gq + 8, d1);
-      }
+      float part[kMT][2] = {};
+      each_pair<kMT, kNT>(m0, n0, lane, [&](int mt, int nt, int hf, int, int) {
+        part[mt][hf] += xr[mt][nt][2 * hf] * dx[mt][nt][2 * hf] +
+                        xr[mt][nt][2 * hf + 1] * dx[mt][nt][2 * hf + 1];
+      });
+      add_rows<kMT>(delta, part, m0, lane);
     }
-    warp_mma<1, 8, true, true>(dx, sb + kU_P, kLd64, m0, sb + kU_DO, kLd128, n0, 64, lane);
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      const int r = m0 + gq, c = n0 + 8 * nt + 2 * tq;
-      st_pair(DXs, kLd128, r, c, dx[0][nt][0], dx[0][nt][1]);
-      st_pair(DXs, kLd128, r + 8, c, dx[0][nt][2], dx[0][nt][3]);
-    }
+    warp_mma<kMT, kNT, true, true, 64>(dx, sb + kU_P, kLd64, m0, sb + kU_DO, kLd128, n0, lane);
+    store_tile(DXs, dx);
     __syncthreads();   // dX complete; (D K)^T no longer read
     // dV = TB^T dX -> output and bf16 operand
     {
-      float acc[1][8][4];
+      Acc acc;
       zero_acc(acc);
-      warp_mma<1, 8, true, true>(acc, sb + kU_TB, kLd64, m0, sb + kU_W, kLd128, n0, 64, lane);
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        const int c = n0 + 8 * nt + 2 * tq;
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const int r = m0 + gq + 8 * hf;
-          st_pair(DVs, kLd128, r, c, acc[0][nt][2 * hf], acc[0][nt][2 * hf + 1]);
-          const long long o = (((long long)ci.row0 + r) * H + h) * kD + c;
-          if (r < len && GDN_IN_BOUNDS(ctrl, o + 1, rows * H * kD))
-            *reinterpret_cast<float2 *>(dv + o) = make_float2(acc[0][nt][2 * hf], acc[0][nt][2 * hf + 1]);
-        }
-      }
+      warp_mma<kMT, kNT, true, true, 64>(acc, sb + kU_TB, kLd64, m0, sb + kU_W, kLd128, n0, lane);
+      store_tile(DVs, acc);
+      store_out(dv, acc, ci, h);
     }
     __syncthreads();   // dV complete; TB no longer read
     // -L = -(K K^T) .* E, s < r (bf16, in place of TB)
     {
-      float acc[1][4][4];
+      AccP acc;
       zero_acc(acc);
-      warp_mma<1, 4, false, false>(acc, sb + kU_K, kLd128, m0, sb + kU_K, kLd128, p0, 128, lane);
-#pragma unroll
-      for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const int r = m0 + gq + 8 * hf, s = p0 + 8 * nt + 2 * tq;
-          const float e0 = s < r ? -ex2(Gam[r] - Gam[s]) : 0.f;
-          const float e1 = s + 1 < r ? -ex2(Gam[r] - Gam[s + 1]) : 0.f;
-          st_pair(Ls, kLd64, r, s, e0 * acc[0][nt][2 * hf], e1 * acc[0][nt][2 * hf + 1]);
-        }
+      warp_mma<kMT, kNP, false, false, 128>(acc, sb + kU_K, kLd128, m0, sb + kU_K, kLd128, p0, lane);
+      each_pair<kMT, kNP>(m0, p0, lane, [&](int mt, int nt, int hf, int r, int s) {
+        const float e0 = s < r ? -ex2(Gam[r] - Gam[s]) : 0.f;
+        const float e1 = s + 1 < r ? -ex2(Gam[r] - Gam[s + 1]) : 0.f;
+        st_pair(Ls, kLd64, r, s, e0 * acc[mt][nt][2 * hf], e1 * acc[mt][nt][2 * hf + 1]);
+      });
     }
     __syncthreads();
     // dY = dX - L^T dV (in dx);  e = V - gamma (K S^T) - L X;  dbeta = rowsum(dY .* e)
-    warp_mma<1, 8, true, true>(dx, sb + kU_TB, kLd64, m0, sb + kU_KT, kLd128, n0, 64, lane);
+    warp_mma<kMT, kNT, true, true, 64>(dx, sb + kU_TB, kLd64, m0, sb + kU_KT, kLd128, n0, lane);
     {
-      float ee[1][8][4];
+      Acc ee;
       zero_acc(ee);
-      warp_mma<1, 8, false, false>(ee, sb + kU_K, kLd128, m0, sb + kU_S, kLd128, n0, 128, lane);
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const int r = m0 + gq + 8 * hf, c = n0 + 8 * nt + 2 * tq;
-          const float2 vv = ld_pair(Vs, kLd128, r, c);
-          ee[0][nt][2 * hf] = vv.x - gam[r] * ee[0][nt][2 * hf];
-          ee[0][nt][2 * hf + 1] = vv.y - gam[r] * ee[0][nt][2 * hf + 1];
-        }
-      warp_mma<1, 8, false, true>(ee, sb + kU_TB, kLd64, m0, sb + kU_X, kLd128, n0, 64, lane);
-      float d0 = 0.f, d1 = 0.f;
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        d0 += dx[0][nt][0] * ee[0][nt][0] + dx[0][nt][1] * ee[0][nt][1];
-        d1 += dx[0][nt][2] * ee[0][nt][2] + dx[0][nt][3] * ee[0][nt][3];
-      }
-      d0 += __shfl_xor_sync(0xffffffffu, d0, 1);
-      d0 += __shfl_xor_sync(0xffffffffu, d0, 2);
-      d1 += __shfl_xor_sync(0xffffffffu, d1, 1);
-      d1 += __shfl_xor_sync(0xffffffffu, d1, 2);
-      if (tq == 0) {
-        atomicAdd(dBet + m0 + gq, d0);
-        atomicAdd(dBet + m0 + gq + 8, d1);
-      }
+      warp_mma<kMT, kNT, false, false, 128>(ee, sb + kU_K, kLd128, m0, sb + kU_S, kLd128, n0, lane);
+      each_pair<kMT, kNT>(m0, n0, lane, [&](int mt, int nt, int hf, int r, int c) {
+        const float2 vv = ld_pair(Vs, kLd128, r, c);
+        ee[mt][nt][2 * hf] = vv.x - gam[r] * ee[mt][nt][2 * hf];
+        ee[mt][nt][2 * hf + 1] = vv.y - gam[r] * ee[mt][nt][2 * hf + 1];
+      });
+      warp_mma<kMT, kNT, false, true, 64>(ee, sb + kU_TB, kLd64, m0, sb + kU_X, kLd128, n0, lane);
+      float part[kMT][2] = {};
+      each_pair<kMT, kNT>(m0, n0, lane, [&](int mt, int nt, int hf, int, int) {
+        part[mt][hf] += dx[mt][nt][2 * hf] * ee[mt][nt][2 * hf] +
+                        dx[mt][nt][2 * hf + 1] * ee[mt][nt][2 * hf + 1];
+      });
+      add_rows<kMT>(dBet, part, m0, lane);
     }
     __syncthreads();   // every read of -L as an operand done
     // dP = dO X^T -> dGamma (dP .* P), then dP .* E (s <= r) over P;
     // R' = dV X^T -> dGamma (-R' .* L), then R = -R' .* E (s < r) over -L
     {
-      float acc[1][4][4];
-      zero_acc(acc);
-      warp_mma<1, 4, false, false>(acc, sb + kU_DO, kLd128, m0, sb + kU_X, kLd128, p0, 128, lane);
-      float rs[2] = {0.f, 0.f};
-#pragma unroll
-      for (int nt = 0; nt < 4; ++nt) {
-        const int s = p0 + 8 * nt + 2 * tq;
-        float cs0 = 0.f, cs1 = 0.f;
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const int r = m0 + gq + 8 * hf;
-          const float2 pp = ld_pair(Ps, kLd64, r, s);
-          const float f0 = acc[0][nt][2 * hf] * pp.x, f1 = acc[0][nt][2 * hf + 1] * pp.y;
-          rs[hf] += f0 + f1;
-          cs0 += f0;
-          cs1 += f1;
-          const float e0 = s <= r ? ex2(Gam[r] - Gam[s]) : 0.f;
-          const float e1 = s + 1 <= r ? ex2(Gam[r] - Gam[s + 1]) : 0.f;
-          st_pair(Ps, kLd64, r, s, e0 * acc[0][nt][2 * hf], e1 * acc[0][nt][2 * hf + 1]);
-        }
-        // column sums over this warp's 16 rows: reduce over g (lanes with equal t)
-#pragma unroll
-        for (int off = 4; off < 32; off <<= 1) {
-          cs0 += __shfl_xor_sync(0xffffffffu, cs0, off);
-          cs1 += __shfl_xor_sync(0xffffffffu, cs1, off);
-        }
-        if (gq == 0) {
-          atomicAdd(dGam + s, -cs0);
-          atomicAdd(dGam + s + 1, -cs1);
-        }
-      }
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        rs[hf] += __shfl_xor_sync(0xffffffffu, rs[hf], 1);
-        rs[hf] += __shfl_xor_sync(0xffffffffu, rs[hf], 2);
-      }
-      if (tq == 0) {
-        atomicAdd(dGam + m0 + gq, rs[0]);
-        atomicAdd(dGam + m0 + gq + 8, rs[1]);
-      }
-    }
-    {
-      float acc[1][4][4];
-      zero_acc(acc);
-      warp_mma<1, 4, false, false>(acc, sb + kU_KT, kLd128, m0, sb + kU_X, kLd128, p0, 128, lane);
-      float rs[2] = {0.f, 0.f};
-#pragma unroll
-      for (int nt = 0; nt < 4; ++nt) {
-        const int s = p0 + 8 * nt + 2 * tq;
-        float cs0 = 0.f, cs1 = 0.f;
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const int r = m0 + gq + 8 * hf;
-          const float2 nl = ld_pair(Ls, kLd64, r, s);   // -L
-          const float f0 = acc[0][nt][2 * hf] * nl.x, f1 = acc[0][nt][2 * hf + 1] * nl.y;
-          rs[hf] += f0 + f1;
-          cs0 += f0;
-          cs1 += f1;
-          const float e0 = s < r ? -ex2(Gam[r] - Gam[s]) : 0.f;
-          const float e1 = s + 1 < r ? -ex2(Gam[r] - Gam[s + 1]) : 0.f;
-          st_pair(Ls, kLd64, r, s, e0 * acc[0][nt][2 * hf], e1 * acc[0][nt][2 * hf + 1]);
-        }
-#pragma unroll
-        for (int off = 4; off < 32; off <<= 1) {
-          cs0 += __shfl_xor_sync(0xffffffffu, cs0, off);
-          cs1 += __shfl_xor_sync(0xffffffffu, cs1, off);
-        }
-        if (gq == 0) {
-          atomicAdd(dGam + s, -cs0);
-          atomicAdd(dGam + s + 1, -cs1);
-        }
-      }
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        rs[hf] += __shfl_xor_sync(0xffffffffu, rs[hf], 1);
-        rs[hf] += __shfl_xor_sync(0xffffffffu, rs[hf], 2);
-      }
-      if (tq == 0) {
-        atomicAdd(dGam + m0 + gq, rs[0]);
-        atomicAdd(dGam + m0 + gq + 8, rs[1]);
-      }
+      AccP dp, rp;
+      zero_acc(dp);
+      zero_acc(rp);
+      warp_mma2<kMT, kNP, false, false, false, false, 128>(dp, sb + kU_DO, kLd128, sb + kU_X,
+                                                           kLd128, rp, sb + kU_KT, kLd128,
+                                                           sb + kU_X, kLd128, m0, p0, lane);
+      float rows_[kMT][2] = {}, cols_[kNP][2] = {};
+      each_pair<kMT, kNP>(m0, p0, lane, [&](int mt, int nt, int hf, int r, int s) {
+        const float2 pp = ld_pair(Ps, kLd64, r, s);
+        const float2 nl = ld_pair(Ls, kLd64, r, s);   // -L
+        const float* a = &dp[mt][nt][2 * hf];
+        const float* b = &rp[mt][nt][2 * hf];
+        const float f0 = a[0] * pp.x + b[0] * nl.x, f1 = a[1] * pp.y + b[1] * nl.y;
+        rows_[mt][hf] += f0 + f1;
+        cols_[nt][0] += f0;
+        cols_[nt][1] += f1;
+        const float e0 = s <= r ? ex2(Gam[r] - Gam[s]) : 0.f;
+        const float e1 = s + 1 <= r ? ex2(Gam[r] - Gam[s + 1]) : 0.f;
+        st_pair(Ps, kLd64, r, s, e0 * a[0], e1 * a[1]);
+        // R = -R' .* E, strictly below the diagonal
+        st_pair(Ls, kLd64, r, s, s < r ? -e0 * b[0] : 0.f, s + 1 < r ? -e1 * b[1] : 0.f);
+      });
+      add_rows<kMT>(dGam, rows_, m0, lane);
+      sub_cols<kNP>(dGam, cols_, p0, lane);
     }
     __syncthreads();   // dP .* E and R complete
     // dQ = gamma (dO S) + (dP .* E) K;  dGamma_r += gamma_r q_r . (dO S)_r
     {
-      float acc[1][8][4];
+      Acc acc;
       zero_acc(acc);
-      warp_mma<1, 8, false, true>(acc, sb + kU_DO, kLd128, m0, sb + kU_S, kLd128, n0, 128, lane);
-      float rs[2] = {0.f, 0.f};
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const int r = m0 + gq + 8 * hf, c = n0 + 8 * nt + 2 * tq;
-          const float2 qq = ld_pair(Qs, kLd128, r, c);
-          rs[hf] += qq.x * acc[0][nt][2 * hf] + qq.y * acc[0][nt][2 * hf + 1];
-          acc[0][nt][2 * hf] *= gam[r];
-          acc[0][nt][2 * hf + 1] *= gam[r];
-        }
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        rs[hf] += __shfl_xor_sync(0xffffffffu, rs[hf], 1);
-        rs[hf] += __shfl_xor_sync(0xffffffffu, rs[hf], 2);
-      }
-      if (tq == 0) {
-        atomicAdd(dGam + m0 + gq, gam[m0 + gq] * rs[0]);
-        atomicAdd(dGam + m0 + gq + 8, gam[m0 + gq + 8] * rs[1]);
-      }
-      warp_mma<1, 8, false, true>(acc, sb + kU_P, kLd64, m0, sb + kU_K, kLd128, n0, 64, lane);
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const int r = m0 + gq + 8 * hf, c = n0 + 8 * nt + 2 * tq;
-          const long long o = (((long long)ci.row0 + r) * H + h) * kD + c;
-          if (r < len && GDN_IN_BOUNDS(ctrl, o + 1, rows * H * kD))
-            *reinterpret_cast<float2 *>(dq + o) = make_float2(acc[0][nt][2 * hf], acc[0][nt][2 * hf + 1]);
-        }
+      warp_mma<kMT, kNT, false, true, 128>(acc, sb + kU_DO, kLd128, m0, sb + kU_S, kLd128, n0, lane);
+      float part[kMT][2] = {};
+      each_pair<kMT, kNT>(m0, n0, lane, [&](int mt, int nt, int hf, int r, int c) {
+        const float2 qq = ld_pair(Qs, kLd128, r, c);
+        part[mt][hf] += gam[r] * (qq.x * acc[mt][nt][2 * hf] + qq.y * acc[mt][nt][2 * hf + 1]);
+        acc[mt][nt][2 * hf] *= gam[r];
+        acc[mt][nt][2 * hf + 1] *= gam[r];
+      });
+      add_rows<kMT>(dGam, part, m0, lane);
+      warp_mma<kMT, kNT, false, true, 64>(acc, sb + kU_P, kLd64, m0, sb + kU_K, kLd128, n0, lane);
+      store_out(dq, acc, ci, h);
     }
     // dK = (dP .* E)^T Q + D (X G') - gamma (dV S) + R K + R^T K;
     // dGamma_r -= gamma_r k_r . (dV S)_r
     {
-      float acc[1][8][4], vs[1][8][4];
+      Acc acc, vs;
       zero_acc(acc);
       zero_acc(vs);
-      warp_mma<1, 8, false, true>(acc, sb + kU_X, kLd128, m0, sb + kU_GP, kLd128, n0, 128, lane);
-      warp_mma<1, 8, false, true>(vs, sb + kU_KT, kLd128, m0, sb + kU_S, kLd128, n0, 128, lane);
-      float rs[2] = {0.f, 0.f};
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const int r = m0 + gq + 8 * hf, c = n0 + 8 * nt + 2 * tq;
-          const float2 kk = ld_pair(Ks, kLd128, r, c);
-          rs[hf] += kk.x * vs[0][nt][2 * hf] + kk.y * vs[0][nt][2 * hf + 1];
-          acc[0][nt][2 * hf] = Dv[r] * acc[0][nt][2 * hf] - gam[r] * vs[0][nt][2 * hf];
-          acc[0][nt][2 * hf + 1] = Dv[r] * acc[0][nt][2 * hf + 1] - gam[r] * vs[0][nt][2 * hf + 1];
-        }
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        rs[hf] += __shfl_xor_sync(0xffffffffu, rs[hf], 1);
-        rs[hf] += __shfl_xor_sync(0xffffffffu, rs[hf], 2);
-      }
-      if (tq == 0) {
-        atomicAdd(dGam + m0 + gq, -gam[m0 + gq] * rs[0]);
-        atomicAdd(dGam + m0 + gq + 8, -gam[m0 + gq + 8] * rs[1]);
-      }
-      warp_mma<1, 8, true, true>(acc, sb + kU_P, kLd64, m0, sb + kU_Q, kLd128, n0, 64, lane);
-      warp_mma<1, 8, false, true>(acc, sb + kU_TB, kLd64, m0, sb + kU_K, kLd128, n0, 64, lane);
-      warp_mma<1, 8, true, true>(acc, sb + kU_TB, kLd64, m0, sb + kU_K, kLd128, n0, 64, lane);
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const int r = m0 + gq + 8 * hf, c = n0 + 8 * nt + 2 * tq;
-          const long long o = (((long long)ci.row0 + r) * H + h) * kD + c;
-          if (r < len && GDN_IN_BOUNDS(ctrl, o + 1, rows * H * kD))
-            *reinterpret_cast<float2 *>(dk + o) = make_float2(acc[0][nt][2 * hf], acc[0][nt][2 * hf + 1]);
-        }
+      warp_mma2<kMT, kNT, false, true, false, true, 128>(acc, sb + kU_X, kLd128, sb + kU_GP,
+                                                         kLd128, vs, sb + kU_KT, kLd128,
+                                                         sb + kU_S, kLd128, m0, n0, lane);
+      float part[kMT][2] = {};
+      each_pair<kMT, kNT>(m0, n0, lane, [&](int mt, int nt, int hf, int r, int c) {
+        const float2 kk = ld_pair(Ks, kLd128, r, c);
+        float *a = &acc[mt][nt][2 * hf];
+        const float *b = &vs[mt][nt][2 * hf];
+        part[mt][hf] -= gam[r] * (kk.x * b[0] + kk.y * b[1]);
+        a[0] = Dv[r] * a[0] - gam[r] * b[0];
+        a[1] = Dv[r] * a[1] - gam[r] * b[1];
+      });
+      add_rows<kMT>(dGam, part, m0, lane);
+      warp_mma<kMT, kNT, true, true, 64>(acc, sb + kU_P, kLd64, m0, sb + kU_Q, kLd128, n0, lane);
+      warp_mma<kMT, kNT, false, true, 64>(acc, sb + kU_TB, kLd64, m0, sb + kU_K, kLd128, n0, lane);
+      warp_mma<kMT, kNT, true, true, 64>(acc, sb + kU_TB, kLd64, m0, sb + kU_K, kLd128, n0, lane);
+      store_out(dk, acc, ci, h);
     }
     __syncthreads();   // dGamma, dbeta, delta and the <G', S> partials complete
     if (warp == 0) {
       // dGamma_s -= delta_s; the last token adds sum(delta) + gamma_last <G', S>;
-      // dg = reverse cumsum of dGamma over the valid tokens (log2(e) is
-      // folded out: Gam holds log2(e) Gamma but dGamma is d/dGamma).
+      // dg = reverse cumsum of dGamma over the valid tokens (Gam holds
+      // log2(e) Gamma, but dGamma is the derivative with respect to Gamma).
       float gsd = 0.f;
 #pragma unroll
-      for (int w = 0; w < 8; ++w) gsd += red[w];
+      for (int w = 0; w < kWarps; ++w) gsd += red[w];
       const float dl0 = delta[lane], dl1 = delta[lane + 32];
       float tot = dl0 + dl1;
 #pragma unroll
@@ -702,7 +713,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
       if (lane + 32 == last) x1 += extra;
       if (lane > last) x0 = 0.f;
       if (lane + 32 > last) x1 = 0.f;
-      // reverse inclusive scan over 64 values: x1 (tokens 32..63) then x0
+      // reverse inclusive scan over the 64 tokens: each half, then x0 += sum(x1)
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
         const float y0 = __shfl_down_sync(0xffffffffu, x0, off);
@@ -752,7 +763,7 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const flo
   e = cudaFuncSetAttribute(gdn_bwd_unit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kUnitSmem);
   if (e != cudaSuccess) return e;
-  gdn_bwd_chain_kernel<<<dim3(N, H), kThreads, kChainSmem, s>>>(
+  gdn_bwd_chain_kernel<<<dim3(N, H, kSlices), kChainThreads, kChainSmem, s>>>(
       static_cast<const bf16 *>(q), static_cast<const bf16 *>(d_o), d_sN, ds0,
       reinterpret_cast<const uint8_t *>(base + L.fwd.w),
       reinterpret_cast<const uint8_t *>(base + L.fwd.kt),

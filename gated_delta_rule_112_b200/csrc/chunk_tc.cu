@@ -1448,6 +1448,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
         for (int t = 0; t < 16; ++t) pk[q][t] = pack_bf16x2(S[32 * q + 2 * t], S[32 * q + 2 * t + 1]);
         tmem_st16(lane_base + kT_S + 32 * hh + 16 * q, pk[q]);
       }
+      tmem_st_wait();
+      tc_fence_before();
+      named_bar_arrive(kBarS, kChainHandoff);
+      // off the chain's path: the MMA warp already has the state
       if (s_chunks && cs < nch) {
         const long long u = (long long)(c0 + cs) * H + h;
         if (GDN_IN_BOUNDS(ctrl, u, (long long)max_chunks * H)) {
@@ -1459,9 +1463,6 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
               dst[4 * q + t / 4] = make_uint4(pk[q][t], pk[q][t + 1], pk[q][t + 2], pk[q][t + 3]);
         }
       }
-      tmem_st_wait();
-      tc_fence_before();
-      named_bar_arrive(kBarS, kChainHandoff);
     };
     store_state(0);
     for (int c = 0; c < nch; ++c) {
