@@ -80,7 +80,8 @@ KERNEL_SOURCES = {
     "chunk_fwd_step": ["chunk_map.cu", "chunk_tc.cu", "gdn_internal.cuh", "sm100_ptx.cuh"],
     "kda_chunk_fwd_step": ["chunk_map.cu", "chunk_tc.cu", "gdn_internal.cuh", "sm100_ptx.cuh"],
     "decode": ["decode.cu", "gdn_internal.cuh", "sm100_ptx.cuh"],
-    "bwd_step": ["backward.cu", "bwd_internal.cuh", "gdn_internal.cuh", "sm100_ptx.cuh"],
+    "bwd_step": ["chunk_bwd_tc.cu", "chunk_map.cu", "chunk_tc.cu", "bwd_internal.cuh",
+                 "gdn_internal.cuh", "sm100_ptx.cuh"],
 }
 
 
@@ -466,12 +467,15 @@ def main():
         # dg, dbeta out; the final-state gradient in and the initial-state gradient out
         bw_bytes = tokens * H * (4 * 128 * 2 + 2 * 4 + 3 * 128 * 4 + 2 * 4) + \
             (2 + (1 if s0 is not None else 0)) * nseq * H * 128 * 128 * 4
-        # every token's S_{t-1} written by the replay and read back by the reverse sweep
-        scratch = 2 * tokens * H * 128 * 128 * 4
+        # per (chunk, head): the forward's intermediates written and read back (48.5 KB
+        # each way), the entering state S_c and the state gradient dS_{c+1} (bf16 32 KB
+        # each, written once and read by the unit kernel)
+        units = -(-T // 64) * H * nseq if cu is None else (tokens // 64 + nseq) * H
+        scratch = units * (2 * 49664 + 2 * 2 * 32768)
         gbs_b = bw_bytes / (ms_b * 1e-3) / 1e9
         backward = {"workload": wl, "ms_per_step": ms_b, "steps": kb, "warmup": 3,
                     "value": replicas.job_rate(tokens, ms_b, world) / 1e6, "unit": UNIT,
-                    "gpu_launches": 2 * kb,
+                    "gpu_launches": 5 * kb,
                     "api": "gated_delta_rule_112_b200.chunk_bwd (C ABI gdn_chunk_bwd)",
                     "roofline": {"bound": "hbm", "achieved": gbs_b, "peak": pk["hbm"],
                                  "unit": "GB/s", "frac": gbs_b / pk["hbm"],
@@ -479,7 +483,8 @@ def main():
                                  "scratch_bytes": scratch,
                                  "traffic": recorded_traffic("bwd_step/" + wl),
                                  "scratch_frac": scratch / (ms_b * 1e-3) / 1e9 / pk["hbm"],
-                                 "kernel": "gdn_bwd_replay_kernel + gdn_bwd_kernel",
+                                 "kernel": "chunk_map + prep + scan (replay, chunk states) + "
+                                           "gdn_bwd_chain_kernel + gdn_bwd_unit_kernel",
                                  "peak_source": pk["source"]}}
         del d_o, dsN, bws
         ws = None
