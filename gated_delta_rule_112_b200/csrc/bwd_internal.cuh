@@ -24,9 +24,10 @@ inline BwdLayout bwd_layout(int B, int T, int H, int dk, int dv) {
 // Workspace of the chunkwise backward pass on the tensor cores (bf16,
 // d_k = d_v = 128, 64-token chunks): the forward pass's layout (one segment:
 // chunk table, prep tiles -W, (D K)^T, T diag(beta), P and the decay
-// factors), then per (chunk, head) unit the state entering the chunk and the
-// gradient with respect to the state leaving it, both bf16 [d_v][d_k]:
-// O(T / 64 d^2) in all.
+// factors), then per (chunk, head) unit the state entering the chunk (bf16,
+// in the state scan's store order: the 16-byte piece of columns 8 p .. 8 p + 7
+// of row i at piece index p * 128 + i) and the gradient with respect to the
+// state leaving it (bf16 [d_v][d_k]): O(T / 64 d^2) in all.
 struct BwdTcLayout {
   WsLayout fwd;
   size_t s_chunks, gprime, total;

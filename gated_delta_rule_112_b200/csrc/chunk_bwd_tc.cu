@@ -512,7 +512,14 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
     load_tokens(sb + kU_K, k + size_t(h) * kD, ci.row0, ustride, len, tid);
     load_tokens(sb + kU_V, v + size_t(h) * kD, ci.row0, ustride, len, tid);
     load_tokens(sb + kU_DO, d_o + size_t(h) * kD, ci.row0, ustride, len, tid);
-    load_dense<128>(sb + kU_S, s_chunks + (long long)unit * (kD * kD), 128, tid);
+    {
+      // S_c: piece p (columns 8 p .. 8 p + 7) of row i at piece index p * 128 + i
+      const bf16 *src = s_chunks + (long long)unit * (kD * kD);
+      for (int e = tid; e < 128 * 16; e += kThreads) {
+        const int p = e >> 7, i = e & 127;
+        cp_async16(sb + kU_S + uint32_t(i * kLd128 + 8 * p) * 2u, src + (p * 128 + i) * 8, 16u);
+      }
+    }
     load_dense<128>(sb + kU_GP, gprime + (long long)unit * (kD * kD), 128, tid);
     load_dense<64>(sb + kU_TB, reinterpret_cast<const bf16 *>(ws_tb) + (long long)unit * (kC * kC), 64, tid);
     load_dense<64>(sb + kU_P, reinterpret_cast<const bf16 *>(ws_pm) + (long long)unit * (kC * kC), 64, tid);

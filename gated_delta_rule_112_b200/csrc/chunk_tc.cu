@@ -772,14 +772,49 @@ __global__ void __launch_bounds__(kKdaPrepThreads, 2) gdn_kda_prep_kernel(
       }
     }
     __syncthreads();   // every thread is past the previous unit's reads of Gm, RR, LK, LQ
-    // g of the chunk (rows past the sequence end read as 0) and beta.
-    for (int e = tid; e < 64 * 32; e += kKdaPrepThreads) {
-      const int r = e >> 5, c4 = e & 31;
-      const long long idx = ((long long)(ci.row0 + r) * H + h) * 128 + 4 * c4;
-      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (r < L && GDN_IN_BOUNDS(ctrl, idx + 3, rows * H * 128))
-        x = *reinterpret_cast<const float4 *>(g + idx);
-      *reinterpret_cast<float4 *>(Gm + r * 128 + 4 * c4) = x;
+    // log2(e) Gamma: inclusive cumsum of g over the tokens (rows past the
+    // sequence end read as 0) as a blocked scan. Thread t owns channels
+    // 4 (t % 32) .. +3 of rows 8 (t / 32) .. +7: a scan over its 8 rows, the
+    // 8 blocks' totals through shared memory (the right-operand area, free
+    // here), then each block adds the totals of the blocks before it.
+    float4 *Tot = reinterpret_cast<float4 *>(sm + kK_RR);   // [8 blocks][32 channel groups]
+    {
+      const int c4 = tid & 31, rb = tid >> 5;
+      float4 run = make_float4(0.f, 0.f, 0.f, 0.f), part[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = 8 * rb + i;
+        const long long idx = ((long long)(ci.row0 + r) * H + h) * 128 + 4 * c4;
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r < L && GDN_IN_BOUNDS(ctrl, idx + 3, rows * H * 128))
+          x = *reinterpret_cast<const float4 *>(g + idx);
+        run.x = fmaf(x.x, kLog2e, run.x);
+        run.y = fmaf(x.y, kLog2e, run.y);
+        run.z = fmaf(x.z, kLog2e, run.z);
+        run.w = fmaf(x.w, kLog2e, run.w);
+        part[i] = run;
+      }
+      Tot[rb * 32 + c4] = run;
+      __syncthreads();
+      float4 off = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int b = 0; b < rb; ++b) {
+        const float4 t4 = Tot[b * 32 + c4];
+        off.x += t4.x;
+        off.y += t4.y;
+        off.z += t4.z;
+        off.w += t4.w;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        *reinterpret_cast<float4 *>(Gm + (8 * rb + i) * 128 + 4 * c4) =
+            make_float4(part[i].x + off.x, part[i].y + off.y, part[i].z + off.z,
+                        part[i].w + off.w);
+      if (rb == 7) {
+        El[4 * c4] = ex2_approx(part[7].x + off.x);
+        El[4 * c4 + 1] = ex2_approx(part[7].y + off.y);
+        El[4 * c4 + 2] = ex2_approx(part[7].z + off.z);
+        El[4 * c4 + 3] = ex2_approx(part[7].w + off.w);
+      }
     }
     if (tid < 64) {
       const long long idx = (long long)(ci.row0 + tid) * H + h;
@@ -793,17 +828,6 @@ __global__ void __launch_bounds__(kKdaPrepThreads, 2) gdn_kda_prep_kernel(
       const long long wi = (long long)(16 * R + rr) * 32 + 8 * S + 4 * half;
       if (GDN_IN_BOUNDS(ctrl, (long long)unit * 2048 + wi + 3, pm_words))
         *reinterpret_cast<uint4 *>(pm + wi) = make_uint4(0, 0, 0, 0);
-    }
-    __syncthreads();
-    // log2(e) Gamma: inclusive cumsum over the tokens, one thread per channel.
-    if (tid < 128) {
-      float acc = 0.f;
-#pragma unroll 8
-      for (int r = 0; r < 64; ++r) {
-        acc = fmaf(Gm[r * 128 + tid], kLog2e, acc);
-        Gm[r * 128 + tid] = acc;
-      }
-      El[tid] = ex2_approx(acc);
     }
     const bool loaded = mbar_wait(bar_load, it & 1, ctrl, &abort_flag);
     if (loaded && L < kC) {
@@ -1129,9 +1153,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
     const int32_t *__restrict__ seq_first, int split, float *__restrict__ sN_trans,
     int sN_group, long long rows, int max_chunks, int n_first, int n_s0, int n_sN, int kda,
     __nv_bfloat16 *__restrict__ s_chunks) {
-  // s_chunks (may be null): the state entering every chunk, bf16 [unit][d_v][d_k]
-  // (unit = chunk * H + head, formula orientation: row i = d_v), for the
-  // backward pass.
+  // s_chunks (may be null): the state entering every chunk in bf16, for the
+  // backward pass: per unit (chunk * H + head) 128 x 128 values of S
+  // (formula orientation, row i = d_v, column j = d_k), the 16-byte piece
+  // holding columns 8 p .. 8 p + 7 of row i at piece index p * 128 + i.
   // kda: the channel-wise gate. Q comes per unit from the prep (Q .* e^Gamma,
   // 2-D map tm_q over [units * 64][128]), the decay records are 256 wide and
   // S decays per d_k channel.
@@ -1451,16 +1476,20 @@ __global__ void __launch_bounds__(kScanThreads, 1) gdn_scan_kernel(
       tmem_st_wait();
       tc_fence_before();
       named_bar_arrive(kBarS, kChainHandoff);
-      // off the chain's path: the MMA warp already has the state
+      // off the chain's path: the MMA warp already has the state. Layout per
+      // unit: 16-byte piece p (= columns 8 p .. 8 p + 7) of row i at piece
+      // index p * 128 + i, so each store instruction of a warp writes 32
+      // consecutive pieces (512 contiguous bytes).
       if (s_chunks && cs < nch) {
         const long long u = (long long)(c0 + cs) * H + h;
         if (GDN_IN_BOUNDS(ctrl, u, (long long)max_chunks * H)) {
-          uint4 *dst = reinterpret_cast<uint4 *>(s_chunks + (u * kD + i) * kD + 64 * hh);
+          uint4 *dst = reinterpret_cast<uint4 *>(s_chunks + u * kD * kD) + i;
 #pragma unroll
           for (int q = 0; q < 2; ++q)
 #pragma unroll
             for (int t = 0; t < 16; t += 4)
-              dst[4 * q + t / 4] = make_uint4(pk[q][t], pk[q][t + 1], pk[q][t + 2], pk[q][t + 3]);
+              dst[(8 * hh + 4 * q + t / 4) * kD] =
+                  make_uint4(pk[q][t], pk[q][t + 1], pk[q][t + 2], pk[q][t + 3]);
         }
       }
     };
