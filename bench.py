@@ -60,6 +60,9 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-decode", action="store_true")
+    p.add_argument("--decode-n", type=int, default=0,
+                   help="sequences of the decode step (default: the workload's 256; a smaller "
+                        "count makes a small case of the same kernel for profiler captures)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--scaling", choices=["weak", "strong"], default="weak",
@@ -496,7 +499,8 @@ def main():
     decode = None
     if not args.no_decode:
         dwl = "kda_decode" if kda else "decode"
-        d = make_decode_inputs(dwl, seed=replicas.shard_seed(WORKLOADS[dwl].seed, rank))
+        d = make_decode_inputs(dwl, seed=replicas.shard_seed(WORKLOADS[dwl].seed, rank),
+                               N=args.decode_n or None)
         dstep = gdn.kda_decode_step if kda else gdn.decode_step
         N, Hd, S = d["N"], d["H"], d["steps"]
         dq, dk, dvv, dg, db = (d[x].to(dev) for x in ("q", "k", "v", "g", "beta"))
@@ -523,12 +527,12 @@ def main():
         bytes_step = (2 * N * Hd * 128 * 128 * 4 + 3 * N * Hd * 128 * 2 + N * Hd * 128 * 2
                       + N * Hd * 4 + N * Hd * (128 if kda else 1) * 4)
         gbs = bytes_step / (us * 1e-6) / 1e9
-        decode = {"workload": f"{dwl} N256 H32 d128 fp32 state, 64 steps", "us_per_step": us,
+        decode = {"workload": f"{dwl} N{N} H{Hd} d128 fp32 state, {S} steps", "us_per_step": us,
                   "value": world * gbs, "unit": "GB/s", "bytes_per_step": bytes_step,
                   "gpu_launches": reps * S,
                   "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"],
                                "unit": "GB/s", "frac": gbs / pk["hbm"],
-                               "traffic": recorded_traffic(f"decode/{dwl}_n256h32"),
+                               "traffic": recorded_traffic(f"decode/{dwl}_n{N}h{Hd}"),
                                "kernel": "gdn_decode_kernel", "peak_source": pk["source"]}}
         del dq, dk, dvv, dg, db, st, do
 
