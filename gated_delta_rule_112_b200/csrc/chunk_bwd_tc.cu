@@ -394,65 +394,156 @@ __global__ void __launch_bounds__(kChainThreads, 2) gdn_bwd_chain_kernel(
 }
 
 // ------------------------------------------------------------------ units
-constexpr uint32_t kU_Q = 0;
-constexpr uint32_t kU_K = kU_Q + kT64x128;
-constexpr uint32_t kU_V = kU_K + kT64x128;
-constexpr uint32_t kU_DO = kU_V + kT64x128;
-constexpr uint32_t kU_S = kU_DO + kT64x128;       // S_c [d_v][d_k]
-constexpr uint32_t kU_GP = kU_S + kT128x128;      // G' [d_v][d_k]
-constexpr uint32_t kU_TB = kU_GP + kT128x128;     // T diag(beta); then -L; then R
-constexpr uint32_t kU_P = kU_TB + kT64x64;        // P; then dP .* E
-constexpr uint32_t kU_W = kU_P + kT64x64;         // -W; then dX
-constexpr uint32_t kU_KT = kU_W + kT64x128;       // (D K)^T [d_k][tokens]; then dV
-constexpr uint32_t kU_X = kU_KT + kT128x64;       // X
-constexpr uint32_t kU_VEC = kU_X + kT64x128;      // Gamma, gamma, D, dGamma, dbeta, delta [64] each
-constexpr uint32_t kU_RED = kU_VEC + 6 * 64 * 4;  // block reduction scratch [kWarps]
-constexpr uint32_t kUnitSmem = kU_RED + 4 * kWarps;
-static_assert(kT128x64 >= kT64x128 && kUnitSmem <= 232448, "unit kernel shared memory");
+// Per (chunk, head) unit on tcgen05: every product is an M = 64 (tokens)
+// tcgen05.mma issued by one thread, operands read by the tensor core straight
+// from shared memory, fp32 accumulators in tensor memory (512 columns, one
+// CTA per SM). M = 64 accumulator row r sits in TMEM lane 32 (r / 16) + r % 16,
+// so warp w reads rows 16 (w % 4) .. +15 with tcgen05.ld.16x256b in the
+// mma-fragment layout (rows g, g + 8; columns 2 t, 2 t + 1). All tiles are bf16
+// in 128-byte-swizzled panels of 64 columns; a stored tile serves as a K-major
+// operand (rows = M or N) or as an MN-major one (rows = K) per product.
+// Six phases, each an MMA group, one commit and an epilogue by all 8 warps:
+//   1  X = TB V + (-W) S^T [X];  DKG = (D K) G'^T [D];  K K^T [KK]
+//      -> X bf16, delta = rowsum(X .* DKG), -L... L = K K^T .* E (s < r) bf16
+//   2  D += P^T dO (= dX);  K S^T [KS]          -> dX bf16
+//   3  dV = TB^T dX [X]                         -> dv, dV bf16
+//   4  D -= L^T dV (= dY);  L X [LX];  dO X^T [dP];  dV X^T [R']
+//      -> e = V - gamma KS - LX, dbeta = rowsum(dY .* e); dGamma from dP .* P
+//         and -R' .* L; dP .* E (s <= r) and R = -R' .* E (s < r) bf16
+//   5  dO S [A];  (dP .* E) K [B];  X G' [C];  dV S [E]
+//      -> dq = gamma A + B; dGamma terms; the first part of dk in registers
+//   6  (dP .* E)^T Q + R K + R^T K [A]          -> dk
+constexpr uint32_t kV_Q = 0;                  // [64][128]: two 8 KB panels
+constexpr uint32_t kV_K = kV_Q + 16384;
+constexpr uint32_t kV_V = kV_K + 16384;
+constexpr uint32_t kV_DO = kV_V + 16384;
+constexpr uint32_t kV_S = kV_DO + 16384;      // [128][128] (S_c, rows d_v): two 16 KB panels
+constexpr uint32_t kV_GP = kV_S + 32768;      // G' [d_v][d_k]
+constexpr uint32_t kV_TB = kV_GP + 32768;     // [64][64]: one 8 KB panel
+constexpr uint32_t kV_P = kV_TB + 8192;       // P; then dP .* E
+constexpr uint32_t kV_W = kV_P + 8192;        // -W [64][128]; then dX
+constexpr uint32_t kV_KT = kV_W + 16384;      // (D K)^T [128][64] (one 16 KB panel); then dV [64][128]
+constexpr uint32_t kV_X = kV_KT + 16384;      // X [64][128]
+constexpr uint32_t kV_L = kV_X + 16384;       // L [64][64]; then R
+constexpr uint32_t kV_VEC = kV_L + 8192;      // Gamma, gamma, D, dGamma, dbeta, delta [64] fp32
+constexpr uint32_t kV_RED = kV_VEC + 6 * 64 * 4;
+constexpr uint32_t kV_BAR = kV_RED + 4 * kWarps;   // mbarrier, TMEM slot, abort flag
+constexpr uint32_t kUnitSmem = kV_BAR + 32 + 1024;  // + 1024: the window is aligned up to 1 KB
+static_assert(kV_Q % 1024 == 0 && kV_S % 1024 == 0 && kV_TB % 1024 == 0 && kV_KT % 1024 == 0 &&
+                  kV_X % 1024 == 0 && kV_L % 1024 == 0 && kUnitSmem <= 232448,
+              "unit kernel shared memory");
+// tensor-memory columns of the accumulators
+constexpr uint32_t kC0 = 0, kC1 = 128, kC2 = 256, kC3 = 384;
 
-// Calls f(mt, nt, hf, row, col) for every fragment pair (row, col..col+1)
-// of a warp's acc[MT][NT] tile with origin (m0, n0); the pair is
-// acc[mt][nt][2 hf], acc[mt][nt][2 hf + 1].
-template <int MT, int NT, typename F>
+// Byte offset of element (r, c) of a [rows][*] bf16 tile stored as 64-column
+// panels with the 128-byte swizzle (8-row atoms; tile base 1024-aligned).
+__device__ __forceinline__ uint32_t swz(int rows, int r, int c) {
+  return uint32_t((c >> 6) * rows * 128 + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) +
+                  (c & 7) * 2);
+}
+
+// One operand of a product: tile base, its rows and whether it is read
+// MN-major (stored [K rows][M or N]) or K-major (stored [M or N rows][K]).
+struct Opnd {
+  uint32_t base;
+  int rows;
+  bool mn;
+};
+// Shared-memory descriptor of k-step kk (16 elements of K).
+__device__ __forceinline__ uint64_t opnd_desc(const Opnd &o, int kk) {
+  if (o.mn) return make_sdesc(o.base + uint32_t(kk) * 2048u, uint32_t(o.rows) * 128u, 1024);
+  return make_sdesc(o.base + uint32_t(kk >> 2) * uint32_t(o.rows) * 128u + uint32_t(kk & 3) * 32u,
+                    16, 1024);
+}
+// acc[tmem col] (+)= A B over K = 16 ksteps; M = 64; N = n.
+__device__ __forceinline__ void mma_product(uint32_t tmem, uint32_t col, const Opnd &a,
+                                            const Opnd &b, int n, int ksteps, bool accumulate,
+                                            bool negate = false) {
+  const uint32_t idesc = make_idesc_bf16(64, n, a.mn ? 1 : 0, b.mn ? 1 : 0, negate ? 1 : 0);
+  for (int kk = 0; kk < ksteps; ++kk)
+    tc_mma_bf16(tmem + col, opnd_desc(a, kk), opnd_desc(b, kk), idesc,
+                (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// 32 (x4: 16) columns of an M = 64 accumulator: r[4 j + 0..3] = rows
+// lane/4 and lane/4 + 8 of the warp's 16-row block, columns 8 j + 2 (lane % 4), +1.
+__device__ __forceinline__ void tmem_ld16x256_x4(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+// A warp's share of an M = 64 accumulator: rows 16 (w % 4) + g (+ 8), columns
+// col0 + 8 j + 2 t (+1) for j < NJ, as acc[j][0..3] (NJ = 8: 64 columns per
+// warp, N = 128 split over the two warps of each row block; NJ = 4: 32 of 64).
+template <int NJ>
+__device__ __forceinline__ void load_acc(float (&acc)[NJ][4], uint32_t taddr) {
+  if constexpr (NJ == 8) {
+    uint32_t r[32];
+    tmem_ld16x256_x8(taddr, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[j][e] = __uint_as_float(r[4 * j + e]);
+  } else {
+    uint32_t r[16];
+    tmem_ld16x256_x4(taddr, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[j][e] = __uint_as_float(r[4 * j + e]);
+  }
+}
+
+// Calls f(j, hf, row, col) for the fragment pairs (row, col..col+1) of a
+// warp's tile with origin (m0, n0); the pair is acc[j][2 hf], acc[j][2 hf + 1].
+template <int NJ, typename F>
 __device__ __forceinline__ void each_pair(int m0, int n0, int lane, F &&f) {
 #pragma unroll
-  for (int mt = 0; mt < MT; ++mt)
+  for (int j = 0; j < NJ; ++j)
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf)
-        f(mt, nt, hf, m0 + 16 * mt + (lane >> 2) + 8 * hf, n0 + 8 * nt + 2 * (lane & 3));
+    for (int hf = 0; hf < 2; ++hf)
+      f(j, hf, m0 + (lane >> 2) + 8 * hf, n0 + 8 * j + 2 * (lane & 3));
 }
 
-// Adds the per-row partial sums part[mt][hf] of a warp tile (rows m0 + 16 mt
-// + lane / 4 + 8 hf) over the four lanes of a row, then into dst[row].
-template <int MT>
-__device__ __forceinline__ void add_rows(float *dst, float (&part)[MT][2], int m0, int lane) {
+// Adds the per-row partial sums part[hf] (rows m0 + lane/4 + 8 hf) over the
+// four lanes of a row, then into dst[row].
+__device__ __forceinline__ void add_rows(float *dst, const float (&part)[2], int m0, int lane) {
 #pragma unroll
-  for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-      float x = part[mt][hf];
-      x += __shfl_xor_sync(0xffffffffu, x, 1);
-      x += __shfl_xor_sync(0xffffffffu, x, 2);
-      if ((lane & 3) == 0) atomicAdd(dst + m0 + 16 * mt + (lane >> 2) + 8 * hf, x);
-    }
+  for (int hf = 0; hf < 2; ++hf) {
+    float x = part[hf];
+    x += __shfl_xor_sync(0xffffffffu, x, 1);
+    x += __shfl_xor_sync(0xffffffffu, x, 2);
+    if ((lane & 3) == 0) atomicAdd(dst + m0 + (lane >> 2) + 8 * hf, x);
+  }
 }
-
-// Subtracts the per-column partial sums part[nt][2] (columns n0 + 8 nt + 2 t,
-// +1) over the eight lanes of a column, then from dst[col].
-template <int NT>
-__device__ __forceinline__ void sub_cols(float *dst, float (&part)[NT][2], int n0, int lane) {
+// Subtracts the per-column partial sums part[j][b] (columns n0 + 8 j + 2 t + b)
+// over the eight lanes of a column from dst[col].
+template <int NJ>
+__device__ __forceinline__ void sub_cols(float *dst, const float (&part)[NJ][2], int n0, int lane) {
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
+  for (int j = 0; j < NJ; ++j)
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
-      float x = part[nt][b];
+      float x = part[j][b];
       x += __shfl_xor_sync(0xffffffffu, x, 4);
       x += __shfl_xor_sync(0xffffffffu, x, 8);
       x += __shfl_xor_sync(0xffffffffu, x, 16);
-      if ((lane >> 2) == 0) atomicAdd(dst + n0 + 8 * nt + 2 * (lane & 3) + b, -x);
+      if ((lane >> 2) == 0) atomicAdd(dst + n0 + 8 * j + 2 * (lane & 3) + b, -x);
     }
+}
+
+__device__ __forceinline__ float2 swz_ld(const uint8_t *t, int rows, int r, int c) {
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(t + swz(rows, r, c)));
+}
+__device__ __forceinline__ void swz_st(uint8_t *t, int rows, int r, int c, float x, float y) {
+  *reinterpret_cast<uint32_t *>(t + swz(rows, r, c)) = pack_bf16x2(x, y);
 }
 
 __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
@@ -465,67 +556,108 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
     float *__restrict__ dbeta, int H, uint32_t *__restrict__ ctrl,
     const ChunkInfo *__restrict__ table, long long rows, int max_chunks) {
   (void)rows;
-  extern __shared__ __align__(16) uint8_t smem[];
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t sb = smem_u32(smem);
-  bf16 *Qs = reinterpret_cast<bf16 *>(smem + kU_Q);
-  bf16 *Ks = reinterpret_cast<bf16 *>(smem + kU_K);
-  bf16 *Vs = reinterpret_cast<bf16 *>(smem + kU_V);
-  bf16 *Ss = reinterpret_cast<bf16 *>(smem + kU_S);
-  bf16 *Gp = reinterpret_cast<bf16 *>(smem + kU_GP);
-  bf16 *Ls = reinterpret_cast<bf16 *>(smem + kU_TB);
-  bf16 *Ps = reinterpret_cast<bf16 *>(smem + kU_P);
-  bf16 *DXs = reinterpret_cast<bf16 *>(smem + kU_W);
-  bf16 *DVs = reinterpret_cast<bf16 *>(smem + kU_KT);
-  bf16 *Xs = reinterpret_cast<bf16 *>(smem + kU_X);
-  float *Gam = reinterpret_cast<float *>(smem + kU_VEC);   // log2(e) Gamma
+  const uint32_t sb = smem_u32(sm);
+  float *Gam = reinterpret_cast<float *>(sm + kV_VEC);   // log2(e) Gamma
   float *gam = Gam + 64, *Dv = Gam + 128, *dGam = Gam + 192, *dBet = Gam + 256,
         *delta = Gam + 320;
-  float *red = reinterpret_cast<float *>(smem + kU_RED);
+  float *red = reinterpret_cast<float *>(sm + kV_RED);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kV_BAR);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kV_BAR + 8);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kV_BAR + 12);
+  if (tid == 0) {
+    *abort_flag = 0;
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // epilogue ownership: rows [m0, m0 + 16) (TMEM lanes 32 (w % 4) ..), columns
+  // [n0, n0 + 64) of N = 128 accumulators, [p0, p0 + 32) of N = 64 ones
+  const int m0 = 16 * (warp & 3), n0 = 64 * (warp >> 2), p0 = 32 * (warp >> 2);
+  const uint32_t lanes = tmem + (uint32_t(32 * (warp & 3)) << 16);
+  // operands
+  const Opnd Qk{sb + kV_Q, 64, false}, Qm{sb + kV_Q, 64, true};
+  const Opnd Kk{sb + kV_K, 64, false}, Km{sb + kV_K, 64, true};
+  const Opnd Vm{sb + kV_V, 64, true};
+  const Opnd DOk{sb + kV_DO, 64, false}, DOm{sb + kV_DO, 64, true};
+  const Opnd Sk{sb + kV_S, 128, false}, Sm{sb + kV_S, 128, true};
+  const Opnd GPk{sb + kV_GP, 128, false}, GPm{sb + kV_GP, 128, true};
+  const Opnd TBk{sb + kV_TB, 64, false}, TBm{sb + kV_TB, 64, true};
+  const Opnd Pk{sb + kV_P, 64, false}, Pm{sb + kV_P, 64, true};
+  const Opnd Wk{sb + kV_W, 64, false}, DXm{sb + kV_W, 64, true};
+  const Opnd KTm{sb + kV_KT, 128, true}, DVk{sb + kV_KT, 64, false}, DVm{sb + kV_KT, 64, true};
+  const Opnd Xk{sb + kV_X, 64, false}, Xm{sb + kV_X, 64, true};
+  const Opnd Lk{sb + kV_L, 64, false}, Lm{sb + kV_L, 64, true};
+  uint32_t phase = 0;
+  // hand the shared-memory writes to the tensor core, then one thread issues
+  // the group and commits it; everyone waits for it
+  auto run = [&](auto &&issue) {
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      if (!*abort_flag) issue();
+      tc_commit(bar);
+    }
+    mbar_wait(bar, phase & 1, ctrl, abort_flag);
+    ++phase;
+    tc_fence_after();
+  };
   const int nunits = (ctrl[0] & kErrBadSeqlens) ? 0 : int(ctrl[1]) * H;
-  // Warp tiles: 64 x 128 outputs as 2 x 4 tiles of 32 x 32 (rows m0, columns
-  // n0); 64 x 64 outputs as 2 x 4 tiles of 32 x 16 (columns p0).
-  constexpr int kMT = 2, kNT = 4, kNP = 2;
-  const int m0 = 32 * (warp & 1), n0 = 32 * (warp >> 1), p0 = 16 * (warp >> 1);
-  using Acc = float[kMT][kNT][4];
-  using AccP = float[kMT][kNP][4];
-  // stores a 64 x 128 fp32 result tile (rows < len) to out [B*T][H][128]
-  auto store_out = [&](float *out, Acc &a, const ChunkInfo &ci, int h) {
-    each_pair<kMT, kNT>(m0, n0, lane, [&](int mt, int nt, int hf, int r, int c) {
-      const long long o = (((long long)ci.row0 + r) * H + h) * kD + c;
-      if (r < ci.len && GDN_IN_BOUNDS(ctrl, o + 1, rows * H * kD))
-        *reinterpret_cast<float2 *>(out + o) = make_float2(a[mt][nt][2 * hf], a[mt][nt][2 * hf + 1]);
-    });
-  };
-  auto store_tile = [&](bf16 *t, Acc &a) {
-    each_pair<kMT, kNT>(m0, n0, lane, [&](int mt, int nt, int hf, int r, int c) {
-      st_pair(t, kLd128, r, c, a[mt][nt][2 * hf], a[mt][nt][2 * hf + 1]);
-    });
-  };
   for (int unit = blockIdx.x; unit < nunits; unit += gridDim.x) {
     const int chunk = unit / H, h = unit - chunk * H;
     const ChunkInfo ci =
         GDN_IN_BOUNDS(ctrl, chunk, max_chunks) ? table[chunk] : ChunkInfo{0, 0, 0, 0};
     const int len = ci.len;
-    const long long ustride = (long long)H * kD;
-    load_tokens(sb + kU_Q, q + size_t(h) * kD, ci.row0, ustride, len, tid);
-    load_tokens(sb + kU_K, k + size_t(h) * kD, ci.row0, ustride, len, tid);
-    load_tokens(sb + kU_V, v + size_t(h) * kD, ci.row0, ustride, len, tid);
-    load_tokens(sb + kU_DO, d_o + size_t(h) * kD, ci.row0, ustride, len, tid);
+    // ---- loads (rows of q, k, v, dO past the sequence end read as zero)
     {
-      // S_c: piece p (columns 8 p .. 8 p + 7) of row i at piece index p * 128 + i
-      const bf16 *src = s_chunks + (long long)unit * (kD * kD);
+      const long long st = (long long)H * kD;
+      const bf16 *srcs[4] = {q, k, v, d_o};
+      const uint32_t dsts[4] = {kV_Q, kV_K, kV_V, kV_DO};
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        for (int e = tid; e < 64 * 16; e += kThreads) {
+          const int r = e >> 4, c16 = e & 15;
+          const bool ok = r < len;
+          const bf16 *src = ok ? srcs[m] + ((long long)ci.row0 + r) * st + size_t(h) * kD + 8 * c16
+                               : srcs[m];
+          cp_async16(sb + dsts[m] + swz(64, r, 8 * c16), src, ok ? 16u : 0u);
+        }
+      const bf16 *sc = s_chunks + (long long)unit * (kD * kD);
+      const bf16 *gp = gprime + (long long)unit * (kD * kD);
       for (int e = tid; e < 128 * 16; e += kThreads) {
-        const int p = e >> 7, i = e & 127;
-        cp_async16(sb + kU_S + uint32_t(i * kLd128 + 8 * p) * 2u, src + (p * 128 + i) * 8, 16u);
+        const int p = e >> 7, i = e & 127;     // S_c: piece p of row i at p * 128 + i
+        cp_async16(sb + kV_S + swz(128, i, 8 * p), sc + (p * 128 + i) * 8, 16u);
+        const int r = e >> 4, c16 = e & 15;     // G': row-major [d_v][d_k]
+        cp_async16(sb + kV_GP + swz(128, r, 8 * c16), gp + r * kD + 8 * c16, 16u);
       }
+      const bf16 *tb = reinterpret_cast<const bf16 *>(ws_tb) + (long long)unit * (kC * kC);
+      const bf16 *pm = reinterpret_cast<const bf16 *>(ws_pm) + (long long)unit * (kC * kC);
+      const bf16 *wn = reinterpret_cast<const bf16 *>(ws_w) + (long long)unit * (kC * kD);
+      const bf16 *kt = reinterpret_cast<const bf16 *>(ws_kt) + (long long)unit * (kD * kC);
+      for (int e = tid; e < 64 * 8; e += kThreads) {
+        const int r = e >> 3, c16 = e & 7;
+        cp_async16(sb + kV_TB + swz(64, r, 8 * c16), tb + r * kC + 8 * c16, 16u);
+        cp_async16(sb + kV_P + swz(64, r, 8 * c16), pm + r * kC + 8 * c16, 16u);
+      }
+      for (int e = tid; e < 64 * 16; e += kThreads) {
+        const int r = e >> 4, c16 = e & 15;
+        cp_async16(sb + kV_W + swz(64, r, 8 * c16), wn + r * kD + 8 * c16, 16u);
+        const int r2 = e >> 3, c2 = e & 7;      // (D K)^T [128][64]
+        cp_async16(sb + kV_KT + swz(128, r2, 8 * c2), kt + r2 * kC + 8 * c2, 16u);
+      }
+      cp_async_commit();
     }
-    load_dense<128>(sb + kU_GP, gprime + (long long)unit * (kD * kD), 128, tid);
-    load_dense<64>(sb + kU_TB, reinterpret_cast<const bf16 *>(ws_tb) + (long long)unit * (kC * kC), 64, tid);
-    load_dense<64>(sb + kU_P, reinterpret_cast<const bf16 *>(ws_pm) + (long long)unit * (kC * kC), 64, tid);
-    load_dense<128>(sb + kU_W, reinterpret_cast<const bf16 *>(ws_w) + (long long)unit * (kC * kD), 64, tid);
-    load_dense<64>(sb + kU_KT, reinterpret_cast<const bf16 *>(ws_kt) + (long long)unit * (kD * kC), 128, tid);
-    cp_async_commit();
     if (warp == 0) {
       // log2(e) Gamma by a warp scan over the 64 tokens (g = 0 past the end)
       float x0 = 0.f, x1 = 0.f;
@@ -555,152 +687,159 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
       delta[lane] = delta[lane + 32] = 0.f;
     }
     cp_async_wait<0>();
-    __syncthreads();
-    // <G', S> (for the last token's dGamma)
+    // ---- phase 1
+    run([&] {
+      mma_product(tmem, kC0, TBk, Vm, 128, 4, false);       // X = TB V
+      mma_product(tmem, kC0, Wk, Sk, 128, 8, true);         //   + (-W) S^T
+      mma_product(tmem, kC1, KTm, GPk, 128, 8, false);      // DKG = (D K) G'^T
+      mma_product(tmem, kC3, Kk, Kk, 64, 8, false);         // K K^T
+    });
     {
+      // <G', S> for the last token's dGamma
       float gs_dot = 0.f;
       for (int e = tid; e < 128 * 64; e += kThreads) {
         const int r = e >> 6, c = 2 * (e & 63);
-        const float2 a = ld_pair(Gp, kLd128, r, c), b = ld_pair(Ss, kLd128, r, c);
+        const float2 a = swz_ld(sm + kV_GP, 128, r, c), b = swz_ld(sm + kV_S, 128, r, c);
         gs_dot += a.x * b.x + a.y * b.y;
       }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) gs_dot += __shfl_xor_sync(0xffffffffu, gs_dot, off);
       if (lane == 0) red[warp] = gs_dot;
-    }
-
-    // X = TB V + (-W) S^T; kept in fp32 for delta
-    Acc xr;
-    zero_acc(xr);
-    warp_mma<kMT, kNT, false, true, 64>(xr, sb + kU_TB, kLd64, m0, sb + kU_V, kLd128, n0, lane);
-    warp_mma<kMT, kNT, false, false, 128>(xr, sb + kU_W, kLd128, m0, sb + kU_S, kLd128, n0, lane);
-    store_tile(Xs, xr);
-    __syncthreads();   // X complete; -W no longer read
-    // dX = P^T dO + (D K) G'^T;  delta_s = X_s . ((D K) G'^T)_s
-    Acc dx;
-    zero_acc(dx);
-    warp_mma<kMT, kNT, true, false, 128>(dx, sb + kU_KT, kLd64, m0, sb + kU_GP, kLd128, n0, lane);
-    {
-      float part[kMT][2] = {};
-      each_pair<kMT, kNT>(m0, n0, lane, [&](int mt, int nt, int hf, int, int) {
-        part[mt][hf] += xr[mt][nt][2 * hf] * dx[mt][nt][2 * hf] +
-                        xr[mt][nt][2 * hf + 1] * dx[mt][nt][2 * hf + 1];
+      float xr[8][4], dkg[8][4];
+      load_acc<8>(xr, lanes + kC0 + n0);
+      load_acc<8>(dkg, lanes + kC1 + n0);
+      float part[2] = {0.f, 0.f};
+      each_pair<8>(m0, n0, lane, [&](int j, int hf, int r, int c) {
+        swz_st(sm + kV_X, 64, r, c, xr[j][2 * hf], xr[j][2 * hf + 1]);
+        part[hf] += xr[j][2 * hf] * dkg[j][2 * hf] + xr[j][2 * hf + 1] * dkg[j][2 * hf + 1];
       });
-      add_rows<kMT>(delta, part, m0, lane);
-    }
-    warp_mma<kMT, kNT, true, true, 64>(dx, sb + kU_P, kLd64, m0, sb + kU_DO, kLd128, n0, lane);
-    store_tile(DXs, dx);
-    __syncthreads();   // dX complete; (D K)^T no longer read
-    // dV = TB^T dX -> output and bf16 operand
-    {
-      Acc acc;
-      zero_acc(acc);
-      warp_mma<kMT, kNT, true, true, 64>(acc, sb + kU_TB, kLd64, m0, sb + kU_W, kLd128, n0, lane);
-      store_tile(DVs, acc);
-      store_out(dv, acc, ci, h);
-    }
-    __syncthreads();   // dV complete; TB no longer read
-    // -L = -(K K^T) .* E, s < r (bf16, in place of TB)
-    {
-      AccP acc;
-      zero_acc(acc);
-      warp_mma<kMT, kNP, false, false, 128>(acc, sb + kU_K, kLd128, m0, sb + kU_K, kLd128, p0, lane);
-      each_pair<kMT, kNP>(m0, p0, lane, [&](int mt, int nt, int hf, int r, int s) {
-        const float e0 = s < r ? -ex2(Gam[r] - Gam[s]) : 0.f;
-        const float e1 = s + 1 < r ? -ex2(Gam[r] - Gam[s + 1]) : 0.f;
-        st_pair(Ls, kLd64, r, s, e0 * acc[mt][nt][2 * hf], e1 * acc[mt][nt][2 * hf + 1]);
+      add_rows(delta, part, m0, lane);
+      float kk[4][4];
+      load_acc<4>(kk, lanes + kC3 + p0);
+      each_pair<4>(m0, p0, lane, [&](int j, int hf, int r, int s) {
+        const float e0 = s < r ? ex2(Gam[r] - Gam[s]) : 0.f;
+        const float e1 = s + 1 < r ? ex2(Gam[r] - Gam[s + 1]) : 0.f;
+        swz_st(sm + kV_L, 64, r, s, e0 * kk[j][2 * hf], e1 * kk[j][2 * hf + 1]);
       });
     }
-    __syncthreads();
-    // dY = dX - L^T dV (in dx);  e = V - gamma (K S^T) - L X;  dbeta = rowsum(dY .* e)
-    warp_mma<kMT, kNT, true, true, 64>(dx, sb + kU_TB, kLd64, m0, sb + kU_KT, kLd128, n0, lane);
+    // ---- phase 2
+    run([&] {
+      mma_product(tmem, kC1, Pm, DOm, 128, 4, true);        // dX = DKG + P^T dO
+      mma_product(tmem, kC2, Kk, Sk, 128, 8, false);        // K S^T
+    });
     {
-      Acc ee;
-      zero_acc(ee);
-      warp_mma<kMT, kNT, false, false, 128>(ee, sb + kU_K, kLd128, m0, sb + kU_S, kLd128, n0, lane);
-      each_pair<kMT, kNT>(m0, n0, lane, [&](int mt, int nt, int hf, int r, int c) {
-        const float2 vv = ld_pair(Vs, kLd128, r, c);
-        ee[mt][nt][2 * hf] = vv.x - gam[r] * ee[mt][nt][2 * hf];
-        ee[mt][nt][2 * hf + 1] = vv.y - gam[r] * ee[mt][nt][2 * hf + 1];
+      float dx[8][4];
+      load_acc<8>(dx, lanes + kC1 + n0);
+      each_pair<8>(m0, n0, lane, [&](int j, int hf, int r, int c) {
+        swz_st(sm + kV_W, 64, r, c, dx[j][2 * hf], dx[j][2 * hf + 1]);
       });
-      warp_mma<kMT, kNT, false, true, 64>(ee, sb + kU_TB, kLd64, m0, sb + kU_X, kLd128, n0, lane);
-      float part[kMT][2] = {};
-      each_pair<kMT, kNT>(m0, n0, lane, [&](int mt, int nt, int hf, int, int) {
-        part[mt][hf] += dx[mt][nt][2 * hf] * ee[mt][nt][2 * hf] +
-                        dx[mt][nt][2 * hf + 1] * ee[mt][nt][2 * hf + 1];
-      });
-      add_rows<kMT>(dBet, part, m0, lane);
     }
-    __syncthreads();   // every read of -L as an operand done
-    // dP = dO X^T -> dGamma (dP .* P), then dP .* E (s <= r) over P;
-    // R' = dV X^T -> dGamma (-R' .* L), then R = -R' .* E (s < r) over -L
+    // ---- phase 3
+    run([&] { mma_product(tmem, kC0, TBm, DXm, 128, 4, false); });   // dV = TB^T dX
     {
-      AccP dp, rp;
-      zero_acc(dp);
-      zero_acc(rp);
-      warp_mma2<kMT, kNP, false, false, false, false, 128>(dp, sb + kU_DO, kLd128, sb + kU_X,
-                                                           kLd128, rp, sb + kU_KT, kLd128,
-                                                           sb + kU_X, kLd128, m0, p0, lane);
-      float rows_[kMT][2] = {}, cols_[kNP][2] = {};
-      each_pair<kMT, kNP>(m0, p0, lane, [&](int mt, int nt, int hf, int r, int s) {
-        const float2 pp = ld_pair(Ps, kLd64, r, s);
-        const float2 nl = ld_pair(Ls, kLd64, r, s);   // -L
-        const float* a = &dp[mt][nt][2 * hf];
-        const float* b = &rp[mt][nt][2 * hf];
-        const float f0 = a[0] * pp.x + b[0] * nl.x, f1 = a[1] * pp.y + b[1] * nl.y;
-        rows_[mt][hf] += f0 + f1;
-        cols_[nt][0] += f0;
-        cols_[nt][1] += f1;
+      float a[8][4];
+      load_acc<8>(a, lanes + kC0 + n0);
+      each_pair<8>(m0, n0, lane, [&](int j, int hf, int r, int c) {
+        swz_st(sm + kV_KT, 64, r, c, a[j][2 * hf], a[j][2 * hf + 1]);
+        const long long o = (((long long)ci.row0 + r) * H + h) * kD + c;
+        if (r < len && GDN_IN_BOUNDS(ctrl, o + 1, rows * H * kD))
+          *reinterpret_cast<float2 *>(dv + o) = make_float2(a[j][2 * hf], a[j][2 * hf + 1]);
+      });
+    }
+    // ---- phase 4
+    run([&] {
+      mma_product(tmem, kC1, Lm, DVm, 128, 4, true, true);  // dY = dX - L^T dV
+      mma_product(tmem, kC3, Lk, Xm, 128, 4, false);        // L X
+      mma_product(tmem, kC0, DOk, Xk, 64, 8, false);        // dP = dO X^T  (cols 0..63)
+      mma_product(tmem, kC0 + 64, DVk, Xk, 64, 8, false);   // R' = dV X^T (cols 64..127)
+    });
+    {
+      // e = V - gamma (K S^T) - L X;  dbeta = rowsum(dY .* e)
+      float dy[8][4], ks[8][4], lx[8][4];
+      load_acc<8>(dy, lanes + kC1 + n0);
+      load_acc<8>(ks, lanes + kC2 + n0);
+      load_acc<8>(lx, lanes + kC3 + n0);
+      float part[2] = {0.f, 0.f};
+      each_pair<8>(m0, n0, lane, [&](int j, int hf, int r, int c) {
+        const float2 vv = swz_ld(sm + kV_V, 64, r, c);
+        const float e0 = vv.x - gam[r] * ks[j][2 * hf] - lx[j][2 * hf];
+        const float e1 = vv.y - gam[r] * ks[j][2 * hf + 1] - lx[j][2 * hf + 1];
+        part[hf] += dy[j][2 * hf] * e0 + dy[j][2 * hf + 1] * e1;
+      });
+      add_rows(dBet, part, m0, lane);
+      // dP .* P and -R' .* L -> dGamma; dP .* E (s <= r) over P, R = -R' .* E (s < r) over L
+      float dp[4][4], rp[4][4];
+      load_acc<4>(dp, lanes + kC0 + p0);
+      load_acc<4>(rp, lanes + kC0 + 64 + p0);
+      float rows_[2] = {0.f, 0.f}, cols_[4][2] = {};
+      each_pair<4>(m0, p0, lane, [&](int j, int hf, int r, int s) {
+        const float2 pp = swz_ld(sm + kV_P, 64, r, s);
+        const float2 ll = swz_ld(sm + kV_L, 64, r, s);
+        const float *a = &dp[j][2 * hf];
+        const float *b = &rp[j][2 * hf];
+        const float f0 = a[0] * pp.x - b[0] * ll.x, f1 = a[1] * pp.y - b[1] * ll.y;
+        rows_[hf] += f0 + f1;
+        cols_[j][0] += f0;
+        cols_[j][1] += f1;
         const float e0 = s <= r ? ex2(Gam[r] - Gam[s]) : 0.f;
         const float e1 = s + 1 <= r ? ex2(Gam[r] - Gam[s + 1]) : 0.f;
-        st_pair(Ps, kLd64, r, s, e0 * a[0], e1 * a[1]);
-        // R = -R' .* E, strictly below the diagonal
-        st_pair(Ls, kLd64, r, s, s < r ? -e0 * b[0] : 0.f, s + 1 < r ? -e1 * b[1] : 0.f);
+        swz_st(sm + kV_P, 64, r, s, e0 * a[0], e1 * a[1]);
+        swz_st(sm + kV_L, 64, r, s, s < r ? -e0 * b[0] : 0.f, s + 1 < r ? -e1 * b[1] : 0.f);
       });
-      add_rows<kMT>(dGam, rows_, m0, lane);
-      sub_cols<kNP>(dGam, cols_, p0, lane);
+      add_rows(dGam, rows_, m0, lane);
+      sub_cols<4>(dGam, cols_, p0, lane);
     }
-    __syncthreads();   // dP .* E and R complete
-    // dQ = gamma (dO S) + (dP .* E) K;  dGamma_r += gamma_r q_r . (dO S)_r
+    // ---- phase 5
+    run([&] {
+      mma_product(tmem, kC0, DOk, Sm, 128, 8, false);       // dO S
+      mma_product(tmem, kC1, Pk, Km, 128, 4, false);        // (dP .* E) K
+      mma_product(tmem, kC2, Xk, GPm, 128, 8, false);       // X G'
+      mma_product(tmem, kC3, DVk, Sm, 128, 8, false);       // dV S
+    });
+    float dkp[8][4];   // D (X G') - gamma (dV S): the first part of dk
     {
-      Acc acc;
-      zero_acc(acc);
-      warp_mma<kMT, kNT, false, true, 128>(acc, sb + kU_DO, kLd128, m0, sb + kU_S, kLd128, n0, lane);
-      float part[kMT][2] = {};
-      each_pair<kMT, kNT>(m0, n0, lane, [&](int mt, int nt, int hf, int r, int c) {
-        const float2 qq = ld_pair(Qs, kLd128, r, c);
-        part[mt][hf] += gam[r] * (qq.x * acc[mt][nt][2 * hf] + qq.y * acc[mt][nt][2 * hf + 1]);
-        acc[mt][nt][2 * hf] *= gam[r];
-        acc[mt][nt][2 * hf + 1] *= gam[r];
+      float a[8][4], b[8][4];
+      load_acc<8>(a, lanes + kC0 + n0);
+      load_acc<8>(b, lanes + kC1 + n0);
+      float part[2] = {0.f, 0.f};
+      each_pair<8>(m0, n0, lane, [&](int j, int hf, int r, int c) {
+        const float2 qq = swz_ld(sm + kV_Q, 64, r, c);
+        part[hf] += gam[r] * (qq.x * a[j][2 * hf] + qq.y * a[j][2 * hf + 1]);
+        const long long o = (((long long)ci.row0 + r) * H + h) * kD + c;
+        if (r < len && GDN_IN_BOUNDS(ctrl, o + 1, rows * H * kD))
+          *reinterpret_cast<float2 *>(dq + o) =
+              make_float2(gam[r] * a[j][2 * hf] + b[j][2 * hf],
+                          gam[r] * a[j][2 * hf + 1] + b[j][2 * hf + 1]);
       });
-      add_rows<kMT>(dGam, part, m0, lane);
-      warp_mma<kMT, kNT, false, true, 64>(acc, sb + kU_P, kLd64, m0, sb + kU_K, kLd128, n0, lane);
-      store_out(dq, acc, ci, h);
+      add_rows(dGam, part, m0, lane);
+      load_acc<8>(a, lanes + kC2 + n0);
+      load_acc<8>(b, lanes + kC3 + n0);
+      float part2[2] = {0.f, 0.f};
+      each_pair<8>(m0, n0, lane, [&](int j, int hf, int r, int c) {
+        const float2 kk2 = swz_ld(sm + kV_K, 64, r, c);
+        part2[hf] -= gam[r] * (kk2.x * b[j][2 * hf] + kk2.y * b[j][2 * hf + 1]);
+        dkp[j][2 * hf] = Dv[r] * a[j][2 * hf] - gam[r] * b[j][2 * hf];
+        dkp[j][2 * hf + 1] = Dv[r] * a[j][2 * hf + 1] - gam[r] * b[j][2 * hf + 1];
+      });
+      add_rows(dGam, part2, m0, lane);
     }
-    // dK = (dP .* E)^T Q + D (X G') - gamma (dV S) + R K + R^T K;
-    // dGamma_r -= gamma_r k_r . (dV S)_r
+    // ---- phase 6
+    run([&] {
+      mma_product(tmem, kC0, Pm, Qm, 128, 4, false);        // (dP .* E)^T Q
+      mma_product(tmem, kC0, Lk, Km, 128, 4, true);         //   + R K
+      mma_product(tmem, kC0, Lm, Km, 128, 4, true);         //   + R^T K
+    });
     {
-      Acc acc, vs;
-      zero_acc(acc);
-      zero_acc(vs);
-      warp_mma2<kMT, kNT, false, true, false, true, 128>(acc, sb + kU_X, kLd128, sb + kU_GP,
-                                                         kLd128, vs, sb + kU_KT, kLd128,
-                                                         sb + kU_S, kLd128, m0, n0, lane);
-      float part[kMT][2] = {};
-      each_pair<kMT, kNT>(m0, n0, lane, [&](int mt, int nt, int hf, int r, int c) {
-        const float2 kk = ld_pair(Ks, kLd128, r, c);
-        float *a = &acc[mt][nt][2 * hf];
-        const float *b = &vs[mt][nt][2 * hf];
-        part[mt][hf] -= gam[r] * (kk.x * b[0] + kk.y * b[1]);
-        a[0] = Dv[r] * a[0] - gam[r] * b[0];
-        a[1] = Dv[r] * a[1] - gam[r] * b[1];
+      float a[8][4];
+      load_acc<8>(a, lanes + kC0 + n0);
+      each_pair<8>(m0, n0, lane, [&](int j, int hf, int r, int c) {
+        const long long o = (((long long)ci.row0 + r) * H + h) * kD + c;
+        if (r < len && GDN_IN_BOUNDS(ctrl, o + 1, rows * H * kD))
+          *reinterpret_cast<float2 *>(dk + o) =
+              make_float2(dkp[j][2 * hf] + a[j][2 * hf], dkp[j][2 * hf + 1] + a[j][2 * hf + 1]);
       });
-      add_rows<kMT>(dGam, part, m0, lane);
-      warp_mma<kMT, kNT, true, true, 64>(acc, sb + kU_P, kLd64, m0, sb + kU_Q, kLd128, n0, lane);
-      warp_mma<kMT, kNT, false, true, 64>(acc, sb + kU_TB, kLd64, m0, sb + kU_K, kLd128, n0, lane);
-      warp_mma<kMT, kNT, true, true, 64>(acc, sb + kU_TB, kLd64, m0, sb + kU_K, kLd128, n0, lane);
-      store_out(dk, acc, ci, h);
     }
+    tc_fence_before();
     __syncthreads();   // dGamma, dbeta, delta and the <G', S> partials complete
     if (warp == 0) {
       // dGamma_s -= delta_s; the last token adds sum(delta) + gamma_last <G', S>;
@@ -720,7 +859,6 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
       if (lane + 32 == last) x1 += extra;
       if (lane > last) x0 = 0.f;
       if (lane + 32 > last) x1 = 0.f;
-      // reverse inclusive scan over the 64 tokens: each half, then x0 += sum(x1)
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
         const float y0 = __shfl_down_sync(0xffffffffu, x0, off);
@@ -742,6 +880,12 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
       }
     }
     __syncthreads();   // shared memory free for the next unit
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
   }
 }
 
