@@ -427,7 +427,7 @@ constexpr uint32_t kV_X = kV_KT + 16384;      // X [64][128]
 constexpr uint32_t kV_L = kV_X + 16384;       // L [64][64]; then R
 constexpr uint32_t kV_VEC = kV_L + 8192;      // Gamma, gamma, D, dGamma, dbeta, delta [64] fp32
 constexpr uint32_t kV_RED = kV_VEC + 6 * 64 * 4;
-constexpr uint32_t kV_BAR = kV_RED + 4 * kWarps;   // mbarrier, TMEM slot, abort flag
+constexpr uint32_t kV_BAR = kV_RED + 4 * kWarps;   // 2 mbarriers, TMEM slot, abort flag
 constexpr uint32_t kUnitSmem = kV_BAR + 32 + 1024;  // + 1024: the window is aligned up to 1 KB
 static_assert(kV_Q % 1024 == 0 && kV_S % 1024 == 0 && kV_TB % 1024 == 0 && kV_KT % 1024 == 0 &&
                   kV_X % 1024 == 0 && kV_L % 1024 == 0 && kUnitSmem <= 232448,
@@ -475,6 +475,20 @@ __device__ __forceinline__ void tmem_ld16x256_x4(uint32_t taddr, uint32_t (&r)[1
         "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
         "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
+}
+
+// After tcgen05.wait::ld: ties later uses of the loaded registers to the wait.
+template <int N>
+__device__ __forceinline__ void reg_dep(uint32_t (&r)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+template <int NJ>
+__device__ __forceinline__ void to_acc(float (&acc)[NJ][4], const uint32_t (&r)[4 * NJ]) {
+#pragma unroll
+  for (int j = 0; j < NJ; ++j)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[j][e] = __uint_as_float(r[4 * j + e]);
 }
 
 // A warp's share of an M = 64 accumulator: rows 16 (w % 4) + g (+ 8), columns
@@ -564,12 +578,13 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
   float *gam = Gam + 64, *Dv = Gam + 128, *dGam = Gam + 192, *dBet = Gam + 256,
         *delta = Gam + 320;
   float *red = reinterpret_cast<float *>(sm + kV_RED);
-  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kV_BAR);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kV_BAR + 8);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kV_BAR + 12);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kV_BAR);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kV_BAR + 16);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kV_BAR + 20);
   if (tid == 0) {
     *abort_flag = 0;
-    mbar_init(bar, 1);
+    mbar_init(bars, 1);
+    mbar_init(bars + 1, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -597,67 +612,102 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
   const Opnd KTm{sb + kV_KT, 128, true}, DVk{sb + kV_KT, 64, false}, DVm{sb + kV_KT, 64, true};
   const Opnd Xk{sb + kV_X, 64, false}, Xm{sb + kV_X, 64, true};
   const Opnd Lk{sb + kV_L, 64, false}, Lm{sb + kV_L, 64, true};
-  uint32_t phase = 0;
-  // hand the shared-memory writes to the tensor core, then one thread issues
-  // the group and commits it; everyone waits for it
-  auto run = [&](auto &&issue) {
+  // Each phase is one or two MMA groups, committed to the two mbarriers in
+  // turn (at most one phase of a barrier is ever outstanding): `issue` hands
+  // the shared-memory writes to the tensor core and one thread issues the
+  // groups; `wait_group` waits for the oldest outstanding group.
+  uint32_t parity[2] = {0u, 0u};
+  int next_commit = 0, next_wait = 0;
+  auto issue = [&](auto &&a, auto &&b, bool two) {
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     if (tid == 0) {
       tc_fence_after();
-      if (!*abort_flag) issue();
-      tc_commit(bar);
+      if (!*abort_flag) a();
+      tc_commit(bars + (next_commit & 1));
+      if (two) {
+        if (!*abort_flag) b();
+        tc_commit(bars + ((next_commit + 1) & 1));
+      }
     }
-    mbar_wait(bar, phase & 1, ctrl, abort_flag);
-    ++phase;
+    next_commit += two ? 2 : 1;
+  };
+  auto wait_group = [&]() {
+    const int b = next_wait & 1;
+    mbar_wait(bars + b, parity[b], ctrl, abort_flag);
+    parity[b] ^= 1u;
+    ++next_wait;
     tc_fence_after();
   };
+  auto none = [] {};
   const int nunits = (ctrl[0] & kErrBadSeqlens) ? 0 : int(ctrl[1]) * H;
+  auto info = [&](int u) {
+    const int c = u / H;
+    return GDN_IN_BOUNDS(ctrl, c, max_chunks) ? table[c] : ChunkInfo{0, 0, 0, 0};
+  };
+  // token tile of head h (rows past len read as zero) into a [64][128] tile
+  auto load_tok = [&](uint32_t dst, const bf16 *src0, const ChunkInfo &c, int h) {
+    const long long st = (long long)H * kD;
+    for (int e = tid; e < 64 * 16; e += kThreads) {
+      const int r = e >> 4, c16 = e & 15;
+      const bool ok = r < c.len;
+      const bf16 *src = ok ? src0 + ((long long)c.row0 + r) * st + size_t(h) * kD + 8 * c16 : src0;
+      cp_async16(sb + dst + swz(64, r, 8 * c16), src, ok ? 16u : 0u);
+    }
+  };
+  auto load_a = [&](int u) {
+    const ChunkInfo c = info(u);
+    const int hu = u % H;
+    load_tok(kV_Q, q, c, hu);
+    load_tok(kV_K, k, c, hu);
+    const bf16 *pm = reinterpret_cast<const bf16 *>(ws_pm) + (long long)u * (kC * kC);
+    for (int e = tid; e < 64 * 8; e += kThreads) {
+      const int r = e >> 3, c16 = e & 7;
+      cp_async16(sb + kV_P + swz(64, r, 8 * c16), pm + r * kC + 8 * c16, 16u);
+    }
+    cp_async_commit();
+  };
+  auto load_b = [&](int u) {
+    const ChunkInfo c = info(u);
+    const int hu = u % H;
+    load_tok(kV_V, v, c, hu);
+    load_tok(kV_DO, d_o, c, hu);
+    const bf16 *sc = s_chunks + (long long)u * (kD * kD);
+    const bf16 *gp = gprime + (long long)u * (kD * kD);
+    for (int e = tid; e < 128 * 16; e += kThreads) {
+      const int p = e >> 7, i = e & 127;     // S_c: piece p of row i at p * 128 + i
+      cp_async16(sb + kV_S + swz(128, i, 8 * p), sc + (p * 128 + i) * 8, 16u);
+      const int r = e >> 4, c16 = e & 15;     // G': row-major [d_v][d_k]
+      cp_async16(sb + kV_GP + swz(128, r, 8 * c16), gp + r * kD + 8 * c16, 16u);
+    }
+    const bf16 *tb = reinterpret_cast<const bf16 *>(ws_tb) + (long long)u * (kC * kC);
+    const bf16 *wn = reinterpret_cast<const bf16 *>(ws_w) + (long long)u * (kC * kD);
+    const bf16 *kt = reinterpret_cast<const bf16 *>(ws_kt) + (long long)u * (kD * kC);
+    for (int e = tid; e < 64 * 8; e += kThreads) {
+      const int r = e >> 3, c16 = e & 7;
+      cp_async16(sb + kV_TB + swz(64, r, 8 * c16), tb + r * kC + 8 * c16, 16u);
+    }
+    for (int e = tid; e < 64 * 16; e += kThreads) {
+      const int r = e >> 4, c16 = e & 15;
+      cp_async16(sb + kV_W + swz(64, r, 8 * c16), wn + r * kD + 8 * c16, 16u);
+      const int r2 = e >> 3, c2 = e & 7;      // (D K)^T [128][64]
+      cp_async16(sb + kV_KT + swz(128, r2, 8 * c2), kt + r2 * kC + 8 * c2, 16u);
+    }
+    cp_async_commit();
+  };
+  bool first = true;
   for (int unit = blockIdx.x; unit < nunits; unit += gridDim.x) {
     const int chunk = unit / H, h = unit - chunk * H;
     const ChunkInfo ci =
         GDN_IN_BOUNDS(ctrl, chunk, max_chunks) ? table[chunk] : ChunkInfo{0, 0, 0, 0};
     const int len = ci.len;
-    // ---- loads (rows of q, k, v, dO past the sequence end read as zero)
-    {
-      const long long st = (long long)H * kD;
-      const bf16 *srcs[4] = {q, k, v, d_o};
-      const uint32_t dsts[4] = {kV_Q, kV_K, kV_V, kV_DO};
-#pragma unroll
-      for (int m = 0; m < 4; ++m)
-        for (int e = tid; e < 64 * 16; e += kThreads) {
-          const int r = e >> 4, c16 = e & 15;
-          const bool ok = r < len;
-          const bf16 *src = ok ? srcs[m] + ((long long)ci.row0 + r) * st + size_t(h) * kD + 8 * c16
-                               : srcs[m];
-          cp_async16(sb + dsts[m] + swz(64, r, 8 * c16), src, ok ? 16u : 0u);
-        }
-      const bf16 *sc = s_chunks + (long long)unit * (kD * kD);
-      const bf16 *gp = gprime + (long long)unit * (kD * kD);
-      for (int e = tid; e < 128 * 16; e += kThreads) {
-        const int p = e >> 7, i = e & 127;     // S_c: piece p of row i at p * 128 + i
-        cp_async16(sb + kV_S + swz(128, i, 8 * p), sc + (p * 128 + i) * 8, 16u);
-        const int r = e >> 4, c16 = e & 15;     // G': row-major [d_v][d_k]
-        cp_async16(sb + kV_GP + swz(128, r, 8 * c16), gp + r * kD + 8 * c16, 16u);
-      }
-      const bf16 *tb = reinterpret_cast<const bf16 *>(ws_tb) + (long long)unit * (kC * kC);
-      const bf16 *pm = reinterpret_cast<const bf16 *>(ws_pm) + (long long)unit * (kC * kC);
-      const bf16 *wn = reinterpret_cast<const bf16 *>(ws_w) + (long long)unit * (kC * kD);
-      const bf16 *kt = reinterpret_cast<const bf16 *>(ws_kt) + (long long)unit * (kD * kC);
-      for (int e = tid; e < 64 * 8; e += kThreads) {
-        const int r = e >> 3, c16 = e & 7;
-        cp_async16(sb + kV_TB + swz(64, r, 8 * c16), tb + r * kC + 8 * c16, 16u);
-        cp_async16(sb + kV_P + swz(64, r, 8 * c16), pm + r * kC + 8 * c16, 16u);
-      }
-      for (int e = tid; e < 64 * 16; e += kThreads) {
-        const int r = e >> 4, c16 = e & 15;
-        cp_async16(sb + kV_W + swz(64, r, 8 * c16), wn + r * kD + 8 * c16, 16u);
-        const int r2 = e >> 3, c2 = e & 7;      // (D K)^T [128][64]
-        cp_async16(sb + kV_KT + swz(128, r2, 8 * c2), kt + r2 * kC + 8 * c2, 16u);
-      }
-      cp_async_commit();
-    }
+    // ---- loads (rows of q, k, v, dO past the sequence end read as zero). Group
+    // B (S_c, G', dO, V, -W, (D K)^T, T diag(beta)) of this unit was issued
+    // during the previous one, as soon as its phase 5 had read them; group A
+    // (Q, K, P) here.
+    if (first) load_b(unit);
+    load_a(unit);
     if (warp == 0) {
       // log2(e) Gamma by a warp scan over the 64 tokens (g = 0 past the end)
       float x0 = 0.f, x1 = 0.f;
@@ -688,32 +738,50 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
     }
     cp_async_wait<0>();
     // ---- phase 1
-    run([&] {
+    issue([&] {
       mma_product(tmem, kC0, TBk, Vm, 128, 4, false);       // X = TB V
       mma_product(tmem, kC0, Wk, Sk, 128, 8, true);         //   + (-W) S^T
       mma_product(tmem, kC1, KTm, GPk, 128, 8, false);      // DKG = (D K) G'^T
+    }, [&] {
       mma_product(tmem, kC3, Kk, Kk, 64, 8, false);         // K K^T
-    });
+    }, true);
     {
       // <G', S> for the last token's dGamma
+      // (both tiles share one layout: a plain walk over their bytes)
       float gs_dot = 0.f;
-      for (int e = tid; e < 128 * 64; e += kThreads) {
-        const int r = e >> 6, c = 2 * (e & 63);
-        const float2 a = swz_ld(sm + kV_GP, 128, r, c), b = swz_ld(sm + kV_S, 128, r, c);
-        gs_dot += a.x * b.x + a.y * b.y;
+      for (int e = tid; e < 128 * 16; e += kThreads) {
+        const uint4 a = *reinterpret_cast<const uint4 *>(sm + kV_GP + 16 * e);
+        const uint4 b = *reinterpret_cast<const uint4 *>(sm + kV_S + 16 * e);
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          gs_dot = fmaf(__uint_as_float(aw[i] << 16), __uint_as_float(bw[i] << 16), gs_dot);
+          gs_dot = fmaf(__uint_as_float(aw[i] & 0xffff0000u), __uint_as_float(bw[i] & 0xffff0000u),
+                        gs_dot);
+        }
       }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) gs_dot += __shfl_xor_sync(0xffffffffu, gs_dot, off);
       if (lane == 0) red[warp] = gs_dot;
+      wait_group();
       float xr[8][4], dkg[8][4];
-      load_acc<8>(xr, lanes + kC0 + n0);
-      load_acc<8>(dkg, lanes + kC1 + n0);
+      {
+        uint32_t r1[32], r2[32];
+        tmem_ld16x256_x8(lanes + kC0 + n0, r1);
+        tmem_ld16x256_x8(lanes + kC1 + n0, r2);
+        tmem_ld_wait();
+        reg_dep(r1);
+        reg_dep(r2);
+        to_acc<8>(xr, r1);
+        to_acc<8>(dkg, r2);
+      }
       float part[2] = {0.f, 0.f};
       each_pair<8>(m0, n0, lane, [&](int j, int hf, int r, int c) {
         swz_st(sm + kV_X, 64, r, c, xr[j][2 * hf], xr[j][2 * hf + 1]);
         part[hf] += xr[j][2 * hf] * dkg[j][2 * hf] + xr[j][2 * hf + 1] * dkg[j][2 * hf + 1];
       });
       add_rows(delta, part, m0, lane);
+      wait_group();
       float kk[4][4];
       load_acc<4>(kk, lanes + kC3 + p0);
       each_pair<4>(m0, p0, lane, [&](int j, int hf, int r, int s) {
@@ -723,10 +791,12 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
       });
     }
     // ---- phase 2
-    run([&] {
+    issue([&] {
       mma_product(tmem, kC1, Pm, DOm, 128, 4, true);        // dX = DKG + P^T dO
-      mma_product(tmem, kC2, Kk, Sk, 128, 8, false);        // K S^T
-    });
+    }, [&] {
+      mma_product(tmem, kC2, Kk, Sk, 128, 8, false);        // K S^T (read in phase 4)
+    }, true);
+    wait_group();
     {
       float dx[8][4];
       load_acc<8>(dx, lanes + kC1 + n0);
@@ -735,7 +805,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
       });
     }
     // ---- phase 3
-    run([&] { mma_product(tmem, kC0, TBm, DXm, 128, 4, false); });   // dV = TB^T dX
+    issue([&] { mma_product(tmem, kC0, TBm, DXm, 128, 4, false); }, none, false);   // dV = TB^T dX
+    wait_group();   // K S^T
+    wait_group();   // dV
     {
       float a[8][4];
       load_acc<8>(a, lanes + kC0 + n0);
@@ -747,60 +819,94 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
       });
     }
     // ---- phase 4
-    run([&] {
-      mma_product(tmem, kC1, Lm, DVm, 128, 4, true, true);  // dY = dX - L^T dV
-      mma_product(tmem, kC3, Lk, Xm, 128, 4, false);        // L X
+    // L is read by the second group's products and rewritten (as R) after
+    // it: the first group's epilogue handles dP, then waits for the second
+    issue([&] {
       mma_product(tmem, kC0, DOk, Xk, 64, 8, false);        // dP = dO X^T  (cols 0..63)
       mma_product(tmem, kC0 + 64, DVk, Xk, 64, 8, false);   // R' = dV X^T (cols 64..127)
-    });
+    }, [&] {
+      mma_product(tmem, kC1, Lm, DVm, 128, 4, true, true);  // dY = dX - L^T dV
+      mma_product(tmem, kC3, Lk, Xm, 128, 4, false);        // L X
+    }, true);
+    wait_group();
     {
-      // e = V - gamma (K S^T) - L X;  dbeta = rowsum(dY .* e)
-      float dy[8][4], ks[8][4], lx[8][4];
-      load_acc<8>(dy, lanes + kC1 + n0);
-      load_acc<8>(ks, lanes + kC2 + n0);
-      load_acc<8>(lx, lanes + kC3 + n0);
-      float part[2] = {0.f, 0.f};
-      each_pair<8>(m0, n0, lane, [&](int j, int hf, int r, int c) {
-        const float2 vv = swz_ld(sm + kV_V, 64, r, c);
-        const float e0 = vv.x - gam[r] * ks[j][2 * hf] - lx[j][2 * hf];
-        const float e1 = vv.y - gam[r] * ks[j][2 * hf + 1] - lx[j][2 * hf + 1];
-        part[hf] += dy[j][2 * hf] * e0 + dy[j][2 * hf + 1] * e1;
-      });
-      add_rows(dBet, part, m0, lane);
-      // dP .* P and -R' .* L -> dGamma; dP .* E (s <= r) over P, R = -R' .* E (s < r) over L
       float dp[4][4], rp[4][4];
-      load_acc<4>(dp, lanes + kC0 + p0);
-      load_acc<4>(rp, lanes + kC0 + 64 + p0);
+      {
+        uint32_t r1[16], r2[16];
+        tmem_ld16x256_x4(lanes + kC0 + p0, r1);
+        tmem_ld16x256_x4(lanes + kC0 + 64 + p0, r2);
+        tmem_ld_wait();
+        reg_dep(r1);
+        reg_dep(r2);
+        to_acc<4>(dp, r1);
+        to_acc<4>(rp, r2);
+      }
+      // dP .* P -> dGamma and dP .* E (s <= r) over P, while the second group runs
       float rows_[2] = {0.f, 0.f}, cols_[4][2] = {};
       each_pair<4>(m0, p0, lane, [&](int j, int hf, int r, int s) {
         const float2 pp = swz_ld(sm + kV_P, 64, r, s);
-        const float2 ll = swz_ld(sm + kV_L, 64, r, s);
         const float *a = &dp[j][2 * hf];
-        const float *b = &rp[j][2 * hf];
-        const float f0 = a[0] * pp.x - b[0] * ll.x, f1 = a[1] * pp.y - b[1] * ll.y;
+        const float f0 = a[0] * pp.x, f1 = a[1] * pp.y;
         rows_[hf] += f0 + f1;
         cols_[j][0] += f0;
         cols_[j][1] += f1;
         const float e0 = s <= r ? ex2(Gam[r] - Gam[s]) : 0.f;
         const float e1 = s + 1 <= r ? ex2(Gam[r] - Gam[s + 1]) : 0.f;
         swz_st(sm + kV_P, 64, r, s, e0 * a[0], e1 * a[1]);
-        swz_st(sm + kV_L, 64, r, s, s < r ? -e0 * b[0] : 0.f, s + 1 < r ? -e1 * b[1] : 0.f);
+      });
+      wait_group();   // L is free once L^T dV and L X are done
+      // -R' .* L -> dGamma, and R = -R' .* E (s < r) over L
+      each_pair<4>(m0, p0, lane, [&](int j, int hf, int r, int s) {
+        const float2 ll = swz_ld(sm + kV_L, 64, r, s);
+        const float *b = &rp[j][2 * hf];
+        const float f0 = -b[0] * ll.x, f1 = -b[1] * ll.y;
+        rows_[hf] += f0 + f1;
+        cols_[j][0] += f0;
+        cols_[j][1] += f1;
+        const float e0 = s < r ? ex2(Gam[r] - Gam[s]) : 0.f;
+        const float e1 = s + 1 < r ? ex2(Gam[r] - Gam[s + 1]) : 0.f;
+        swz_st(sm + kV_L, 64, r, s, -e0 * b[0], -e1 * b[1]);
       });
       add_rows(dGam, rows_, m0, lane);
       sub_cols<4>(dGam, cols_, p0, lane);
+      // e = V - gamma (K S^T) - L X;  dbeta = rowsum(dY .* e)
+      {
+        float dy[8][4], ks[8][4], lx[8][4];
+        load_acc<8>(dy, lanes + kC1 + n0);
+        load_acc<8>(ks, lanes + kC2 + n0);
+        load_acc<8>(lx, lanes + kC3 + n0);
+        float part[2] = {0.f, 0.f};
+        each_pair<8>(m0, n0, lane, [&](int j, int hf, int r, int c) {
+          const float2 vv = swz_ld(sm + kV_V, 64, r, c);
+          const float e0 = vv.x - gam[r] * ks[j][2 * hf] - lx[j][2 * hf];
+          const float e1 = vv.y - gam[r] * ks[j][2 * hf + 1] - lx[j][2 * hf + 1];
+          part[hf] += dy[j][2 * hf] * e0 + dy[j][2 * hf + 1] * e1;
+        });
+        add_rows(dBet, part, m0, lane);
+      }
     }
     // ---- phase 5
-    run([&] {
+    issue([&] {
       mma_product(tmem, kC0, DOk, Sm, 128, 8, false);       // dO S
       mma_product(tmem, kC1, Pk, Km, 128, 4, false);        // (dP .* E) K
+    }, [&] {
       mma_product(tmem, kC2, Xk, GPm, 128, 8, false);       // X G'
       mma_product(tmem, kC3, DVk, Sm, 128, 8, false);       // dV S
-    });
+    }, true);
+    wait_group();
     float dkp[8][4];   // D (X G') - gamma (dV S): the first part of dk
     {
       float a[8][4], b[8][4];
-      load_acc<8>(a, lanes + kC0 + n0);
-      load_acc<8>(b, lanes + kC1 + n0);
+      {
+        uint32_t r1[32], r2[32];
+        tmem_ld16x256_x8(lanes + kC0 + n0, r1);
+        tmem_ld16x256_x8(lanes + kC1 + n0, r2);
+        tmem_ld_wait();
+        reg_dep(r1);
+        reg_dep(r2);
+        to_acc<8>(a, r1);
+        to_acc<8>(b, r2);
+      }
       float part[2] = {0.f, 0.f};
       each_pair<8>(m0, n0, lane, [&](int j, int hf, int r, int c) {
         const float2 qq = swz_ld(sm + kV_Q, 64, r, c);
@@ -812,8 +918,20 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
                           gam[r] * a[j][2 * hf + 1] + b[j][2 * hf + 1]);
       });
       add_rows(dGam, part, m0, lane);
-      load_acc<8>(a, lanes + kC2 + n0);
-      load_acc<8>(b, lanes + kC3 + n0);
+      wait_group();
+      // S_c, G', dO, V, -W, (D K)^T and T diag(beta) are read for the last
+      // time by phase 5: the next unit's copies land during the rest of this one
+      if (unit + int(gridDim.x) < nunits) load_b(unit + int(gridDim.x));
+      {
+        uint32_t r1[32], r2[32];
+        tmem_ld16x256_x8(lanes + kC2 + n0, r1);
+        tmem_ld16x256_x8(lanes + kC3 + n0, r2);
+        tmem_ld_wait();
+        reg_dep(r1);
+        reg_dep(r2);
+        to_acc<8>(a, r1);
+        to_acc<8>(b, r2);
+      }
       float part2[2] = {0.f, 0.f};
       each_pair<8>(m0, n0, lane, [&](int j, int hf, int r, int c) {
         const float2 kk2 = swz_ld(sm + kV_K, 64, r, c);
@@ -824,11 +942,12 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
       add_rows(dGam, part2, m0, lane);
     }
     // ---- phase 6
-    run([&] {
+    issue([&] {
       mma_product(tmem, kC0, Pm, Qm, 128, 4, false);        // (dP .* E)^T Q
       mma_product(tmem, kC0, Lk, Km, 128, 4, true);         //   + R K
       mma_product(tmem, kC0, Lm, Km, 128, 4, true);         //   + R^T K
-    });
+    }, none, false);
+    wait_group();
     {
       float a[8][4];
       load_acc<8>(a, lanes + kC0 + n0);
@@ -880,7 +999,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
       }
     }
     __syncthreads();   // shared memory free for the next unit
+    first = false;
   }
+  cp_async_wait<0>();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
