@@ -29,13 +29,13 @@
 // The kernels of one call:
 //   1. the forward's chunk map, prep and state scan, the scan also writing
 //      every chunk's entering state S_c (bf16) and no output;
-//   2. gdn_bwd_chain_kernel, one CTA per (sequence, head): the reverse chain
+//   2. gdn_bwd_chain_kernel, two CTAs per (sequence, head): the reverse chain
 //      dS_c = gamma_last dS_{c+1} - dX^T W + (gamma dO)^T Q over the chunks,
 //      writing each chunk's G' = dS_{c+1} (bf16) and d_initial_state;
 //   3. gdn_bwd_unit_kernel, persistent over (chunk, head) units: everything
 //      else above, from the chunk's tiles, S_c and G'.
-// Products run on the warp-level tensor-core path (mma.sync m16n8k16, bf16
-// operands, fp32 accumulation) from padded shared-memory tiles.
+// Every product of kernels 2 and 3 is a tcgen05.mma (bf16 operands from
+// 128-byte-swizzled shared tiles, fp32 accumulators in tensor memory).
 #include <cuda_bf16.h>
 
 #include "bwd_internal.cuh"
@@ -46,13 +46,6 @@ namespace {
 
 using bf16 = __nv_bfloat16;
 constexpr int kC = 64, kD = 128;
-// Row strides (bf16 elements) of the shared tiles: 272- and 144-byte rows put
-// the 8 rows an ldmatrix reads in 8 distinct 16-byte bank groups.
-constexpr int kLd128 = 136, kLd64 = 72;
-constexpr uint32_t kT64x128 = 64 * kLd128 * 2;    // [64][128] tile, 17,408 B
-constexpr uint32_t kT128x128 = 128 * kLd128 * 2;  // [128][128] tile, 34,816 B
-constexpr uint32_t kT64x64 = 64 * kLd64 * 2;      // [64][64] tile, 9,216 B
-constexpr uint32_t kT128x64 = 128 * kLd64 * 2;    // [128][64] tile, 18,432 B
 constexpr int kThreads = 256, kWarps = kThreads / 32;   // the unit kernel's block
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -69,328 +62,10 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
-      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// One warp: acc[MT][NT] (16 x 8 tiles, rows m0 + 16 mt, columns n0 + 8 nt)
-// += op(A) op(B) over k in [0, K) (fully unrolled). A is stored [m][k] (AT = false) or [k][m]
-// (AT = true) at shared address A with row stride lda elements; B is stored
-// [n][k] (BT = false) or [k][n] (BT = true). Fragment layout of acc[mt][nt]:
-// with g = lane / 4, t = lane % 4, elements (g, 2t), (g, 2t+1), (g+8, 2t),
-// (g+8, 2t+1) of the tile. NT is even (B is read two n-tiles at a time).
-template <int MT, int NT, bool AT, bool BT, int K>
-__device__ __forceinline__ void warp_mma(float (&acc)[MT][NT][4], uint32_t A, int lda, int m0,
-                                         uint32_t B, int ldb, int n0, int lane) {
-#pragma unroll
-  for (int k0 = 0; k0 < K; k0 += 16) {
-    uint32_t a[MT][4];
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-      if (!AT) {
-        const int r = m0 + 16 * mt + (lane & 15), c = k0 + 8 * (lane >> 4);
-        ldsm_x4(A + 2u * uint32_t(r * lda + c), a[mt]);
-      } else {
-        const int r = k0 + (lane & 7) + 8 * (lane >> 4), c = m0 + 16 * mt + 8 * ((lane >> 3) & 1);
-        ldsm_x4_trans(A + 2u * uint32_t(r * lda + c), a[mt]);
-      }
-    }
-#pragma unroll
-    for (int nt = 0; nt < NT; nt += 2) {
-      uint32_t b[4];
-      if (!BT) {
-        const int r = n0 + 8 * nt + 8 * (lane >> 4) + (lane & 7), c = k0 + 8 * ((lane >> 3) & 1);
-        ldsm_x4(B + 2u * uint32_t(r * ldb + c), b);
-      } else {
-        const int r = k0 + (lane & 7) + 8 * ((lane >> 3) & 1), c = n0 + 8 * nt + 8 * (lane >> 4);
-        ldsm_x4_trans(B + 2u * uint32_t(r * ldb + c), b);
-      }
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        mma16816(acc[mt][nt], a[mt], b[0], b[1]);
-        mma16816(acc[mt][nt + 1], a[mt], b[2], b[3]);
-      }
-    }
-  }
-}
-
-// Two independent products of the same shape and depth in one loop (twice
-// the independent accumulators per step): acc1 += op(A1) op(B1), acc2 +=
-// op(A2) op(B2), operands as for warp_mma.
-template <int MT, int NT, bool AT1, bool BT1, bool AT2, bool BT2, int K>
-__device__ __forceinline__ void warp_mma2(float (&acc1)[MT][NT][4], uint32_t A1, int lda1,
-                                          uint32_t B1, int ldb1, float (&acc2)[MT][NT][4],
-                                          uint32_t A2, int lda2, uint32_t B2, int ldb2, int m0,
-                                          int n0, int lane) {
-#pragma unroll
-  for (int k0 = 0; k0 < K; k0 += 16) {
-    uint32_t a1[MT][4], a2[MT][4];
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-      if (!AT1)
-        ldsm_x4(A1 + 2u * uint32_t((m0 + 16 * mt + (lane & 15)) * lda1 + k0 + 8 * (lane >> 4)), a1[mt]);
-      else
-        ldsm_x4_trans(A1 + 2u * uint32_t((k0 + (lane & 7) + 8 * (lane >> 4)) * lda1 + m0 + 16 * mt +
-                                         8 * ((lane >> 3) & 1)), a1[mt]);
-      if (!AT2)
-        ldsm_x4(A2 + 2u * uint32_t((m0 + 16 * mt + (lane & 15)) * lda2 + k0 + 8 * (lane >> 4)), a2[mt]);
-      else
-        ldsm_x4_trans(A2 + 2u * uint32_t((k0 + (lane & 7) + 8 * (lane >> 4)) * lda2 + m0 + 16 * mt +
-                                         8 * ((lane >> 3) & 1)), a2[mt]);
-    }
-#pragma unroll
-    for (int nt = 0; nt < NT; nt += 2) {
-      uint32_t b1[4], b2[4];
-      if (!BT1)
-        ldsm_x4(B1 + 2u * uint32_t((n0 + 8 * nt + 8 * (lane >> 4) + (lane & 7)) * ldb1 + k0 +
-                                   8 * ((lane >> 3) & 1)), b1);
-      else
-        ldsm_x4_trans(B1 + 2u * uint32_t((k0 + (lane & 7) + 8 * ((lane >> 3) & 1)) * ldb1 + n0 +
-                                         8 * nt + 8 * (lane >> 4)), b1);
-      if (!BT2)
-        ldsm_x4(B2 + 2u * uint32_t((n0 + 8 * nt + 8 * (lane >> 4) + (lane & 7)) * ldb2 + k0 +
-                                   8 * ((lane >> 3) & 1)), b2);
-      else
-        ldsm_x4_trans(B2 + 2u * uint32_t((k0 + (lane & 7) + 8 * ((lane >> 3) & 1)) * ldb2 + n0 +
-                                         8 * nt + 8 * (lane >> 4)), b2);
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        mma16816(acc1[mt][nt], a1[mt], b1[0], b1[1]);
-        mma16816(acc2[mt][nt], a2[mt], b2[0], b2[1]);
-        mma16816(acc1[mt][nt + 1], a1[mt], b1[2], b1[3]);
-        mma16816(acc2[mt][nt + 1], a2[mt], b2[2], b2[3]);
-      }
-    }
-  }
-}
-
-template <int MT, int NT>
-__device__ __forceinline__ void zero_acc(float (&acc)[MT][NT][4]) {
-#pragma unroll
-  for (int i = 0; i < MT; ++i)
-#pragma unroll
-    for (int j = 0; j < NT; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
-}
-
-// Fragment pair (row, 2 columns) of a [rows][ld] bf16 tile as two floats.
-__device__ __forceinline__ float2 ld_pair(const bf16 *t, int ld, int r, int c) {
-  const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162 *>(t + r * ld + c);
-  return __bfloat1622float2(v);
-}
-__device__ __forceinline__ void st_pair(bf16 *t, int ld, int r, int c, float x, float y) {
-  *reinterpret_cast<uint32_t *>(t + r * ld + c) = pack_bf16x2(x, y);
-}
-
-// Copies rows [0, 64) of a token tile (128 bf16 per row, row r at
-// base + (row0 + r) * stride elements) into a [64][kLd128] shared tile; rows
-// r >= len read as zero.
-__device__ __forceinline__ void load_tokens(uint32_t dst, const bf16 *base, long long row0,
-                                            long long stride, int len, int tid) {
-  for (int e = tid; e < 64 * 16; e += kThreads) {
-    const int r = e >> 4, c = e & 15;
-    const bool ok = r < len;
-    const bf16 *src = ok ? base + (row0 + r) * stride + 8 * c : base;
-    cp_async16(dst + uint32_t(r * kLd128 + 8 * c) * 2u, src, ok ? 16u : 0u);
-  }
-}
-// Copies a dense [rows][cols] bf16 tile (cols = 64 or 128) into a padded one.
-template <int COLS>
-__device__ __forceinline__ void load_dense(uint32_t dst, const bf16 *src, int rows, int tid) {
-  constexpr int kPer = COLS / 8, kLd = COLS == 128 ? kLd128 : kLd64;
-  for (int e = tid; e < rows * kPer; e += kThreads) {
-    const int r = e / kPer, c = e - r * kPer;
-    cp_async16(dst + uint32_t(r * kLd + 8 * c) * 2u, src + r * COLS + 8 * c, 16u);
-  }
-}
-
-// ------------------------------------------------------------------ chain
-// Row i of dS_c depends only on row i of dS_{c+1} (dX column i only on row i
-// of G'), so each (sequence, head) chain runs as kSlices CTAs of kSlice d_v
-// rows, two CTAs per SM. Shared memory: the G slice (bf16 [kSlice][d_k]), the
-// dX slice (bf16 [tokens][kSlice]), one chunk's (D K)^T, P, -W and Q, and two
-// stages of the dO slice and the decay factors. (D K)^T and P of the next
-// chunk load while the G update runs, -W and Q while the next dX runs.
-constexpr int kSlices = 4, kSlice = kD / kSlices, kLdS = kSlice + 8;
-constexpr int kChainThreads = 256, kChainWarps = kChainThreads / 32;
-constexpr uint32_t kTDoS = 64 * kLdS * 2;             // [64][kSlice] tile
-constexpr uint32_t kCh_G = 0;                          // [kSlice][kLd128]
-constexpr uint32_t kCh_DX = kCh_G + kSlice * kLd128 * 2;
-constexpr uint32_t kCh_KT = kCh_DX + kTDoS;            // (D K)^T [d_k][tokens]
-constexpr uint32_t kCh_PM = kCh_KT + kT128x64;         // P [r][s]
-constexpr uint32_t kCh_WN = kCh_PM + kT64x64;          // -W [tokens][d_k]
-constexpr uint32_t kCh_Q = kCh_WN + kT64x128;          // Q [tokens][d_k]
-constexpr uint32_t kCh_DO = kCh_Q + kT64x128;          // 2 x dO slice, then gamma dO
-constexpr uint32_t kCh_GAM = kCh_DO + 2 * kTDoS;       // 2 x (gamma [64], D [64])
-constexpr uint32_t kChainSmem = kCh_GAM + 2 * 128 * 4;
-static_assert(2 * (kChainSmem + 1024) <= 233472, "chain kernel: two CTAs per SM");
-
-__global__ void __launch_bounds__(kChainThreads, 2) gdn_bwd_chain_kernel(
-    const bf16 *__restrict__ q, const bf16 *__restrict__ d_o, const float *__restrict__ d_sN,
-    float *__restrict__ ds0, const uint8_t *__restrict__ ws_w, const uint8_t *__restrict__ ws_kt,
-    const uint8_t *__restrict__ ws_pm, const float *__restrict__ ws_gam,
-    bf16 *__restrict__ gprime, int H, uint32_t *__restrict__ ctrl,
-    const ChunkInfo *__restrict__ table, const int32_t *__restrict__ seq_first, int N,
-    long long rows, int max_chunks) {
-  (void)rows;
-  extern __shared__ __align__(16) uint8_t smem[];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, t = lane & 3;
-  const int n = blockIdx.x, h = blockIdx.y, i0 = kSlice * int(blockIdx.z);
-  const uint32_t sb = smem_u32(smem);
-  bf16 *Gs = reinterpret_cast<bf16 *>(smem + kCh_G);
-  bf16 *DXs = reinterpret_cast<bf16 *>(smem + kCh_DX);
-  int c0 = 0, nch = 0;
-  if (!(ctrl[0] & kErrBadSeqlens) && GDN_IN_BOUNDS(ctrl, n + 1, N + 1)) {
-    c0 = seq_first[n];
-    nch = seq_first[n + 1] - c0;
-  }
-  // G = dL/dS rows [i0, i0 + kSlice) (formula orientation [d_v i][d_k j]);
-  // warp w: local rows [gm0, gm0 + 16), columns [gn0, gn0 + 32).
-  constexpr int kGT = 4;
-  const int gm0 = 16 * (warp & 1), gn0 = 32 * (warp >> 1);
-  float G[1][kGT][4];
-  {
-    const float *src = d_sN ? d_sN + (size_t(n) * H + h) * kD * kD : nullptr;
-#pragma unroll
-    for (int nt = 0; nt < kGT; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = i0 + gm0 + g + 8 * (e >> 1), j = gn0 + 8 * nt + 2 * t + (e & 1);
-        G[0][nt][e] = src ? src[j * kD + i] : 0.f;   // stored [d_k][d_v]
-      }
-  }
-  auto unit_of = [&](int c) { return (long long)(c0 + c) * H + h; };
-  auto info_of = [&](int c) {
-    const long long chunk = c0 + c;
-    return GDN_IN_BOUNDS(ctrl, chunk, max_chunks) ? table[chunk] : ChunkInfo{0, 0, 0, 0};
-  };
-  // group A: (D K)^T, P, the dO slice and the decay factors of chunk c
-  auto load_a = [&](int c, int st) {
-    if (c >= 0) {
-      const long long unit = unit_of(c);
-      const ChunkInfo ci = info_of(c);
-      for (int e = tid; e < 128 * 8; e += kChainThreads) {
-        const int r = e >> 3, cc = e & 7;
-        cp_async16(sb + kCh_KT + uint32_t(r * kLd64 + 8 * cc) * 2u,
-                   reinterpret_cast<const bf16 *>(ws_kt) + unit * (kD * kC) + r * kC + 8 * cc, 16u);
-      }
-      for (int e = tid; e < 64 * 8; e += kChainThreads) {
-        const int r = e >> 3, cc = e & 7;
-        cp_async16(sb + kCh_PM + uint32_t(r * kLd64 + 8 * cc) * 2u,
-                   reinterpret_cast<const bf16 *>(ws_pm) + unit * (kC * kC) + r * kC + 8 * cc, 16u);
-      }
-      for (int e = tid; e < 64 * (kSlice / 8); e += kChainThreads) {
-        const int r = e / (kSlice / 8), cc = e - r * (kSlice / 8);
-        const bool ok = r < ci.len;
-        const bf16 *src = ok ? d_o + ((long long)ci.row0 + r) * H * kD + size_t(h) * kD + i0 + 8 * cc
-                             : d_o;
-        cp_async16(sb + kCh_DO + st * kTDoS + uint32_t(r * kLdS + 8 * cc) * 2u, src, ok ? 16u : 0u);
-      }
-      if (tid < 32)
-        cp_async16(sb + kCh_GAM + st * 512 + 16 * tid, ws_gam + unit * 128 + 4 * tid, 16u);
-    }
-    cp_async_commit();
-  };
-  // group B: -W and Q of chunk c
-  auto load_b = [&](int c) {
-    if (c >= 0) {
-      const long long unit = unit_of(c);
-      const ChunkInfo ci = info_of(c);
-      for (int e = tid; e < 64 * 16; e += kChainThreads) {
-        const int r = e >> 4, cc = e & 15;
-        cp_async16(sb + kCh_WN + uint32_t(r * kLd128 + 8 * cc) * 2u,
-                   reinterpret_cast<const bf16 *>(ws_w) + unit * (kC * kD) + r * kD + 8 * cc, 16u);
-        const bool ok = r < ci.len;
-        const bf16 *src = ok ? q + ((long long)ci.row0 + r) * H * kD + size_t(h) * kD + 8 * cc : q;
-        cp_async16(sb + kCh_Q + uint32_t(r * kLd128 + 8 * cc) * 2u, src, ok ? 16u : 0u);
-      }
-    }
-    cp_async_commit();
-  };
-  load_a(nch - 1, 0);
-  load_b(nch - 1);
-  for (int it = 0; it < nch; ++it) {
-    const int c = nch - 1 - it, st = it & 1;
-    const long long unit = unit_of(c);
-    // G' slice of this chunk: bf16 into shared memory (operand) and the workspace
-#pragma unroll
-    for (int nt = 0; nt < kGT; ++nt) {
-      const int i = gm0 + g, j = gn0 + 8 * nt + 2 * t;
-      st_pair(Gs, kLd128, i, j, G[0][nt][0], G[0][nt][1]);
-      st_pair(Gs, kLd128, i + 8, j, G[0][nt][2], G[0][nt][3]);
-    }
-    cp_async_wait<1>();   // group A of this chunk (B may still be in flight)
-    __syncthreads();
-    if (GDN_IN_BOUNDS(ctrl, unit, (long long)max_chunks * H)) {
-      uint4 *dst = reinterpret_cast<uint4 *>(gprime + unit * (kD * kD) + size_t(i0) * kD);
-      for (int e = tid; e < kSlice * 16; e += kChainThreads) {
-        const int r = e >> 4, cc = e & 15;
-        dst[r * 16 + cc] = *reinterpret_cast<const uint4 *>(Gs + r * kLd128 + 8 * cc);
-      }
-    }
-    const float *gam = reinterpret_cast<const float *>(smem + kCh_GAM + st * 512);
-    bf16 *DO = reinterpret_cast<bf16 *>(smem + kCh_DO + st * kTDoS);
-    {
-      // dX slice = P^T dO + (D K) G^T: warp w -> tokens [16 (w % 4), +16),
-      // local d_v [16 (w / 4), +16)
-      const int m0 = 16 * (warp & 3), n0 = 16 * (warp >> 2);
-      float acc[1][2][4];
-      zero_acc(acc);
-      warp_mma<1, 2, true, true, 64>(acc, sb + kCh_PM, kLd64, m0, sb + kCh_DO + st * kTDoS, kLdS, n0, lane);
-      warp_mma<1, 2, true, false, 128>(acc, sb + kCh_KT, kLd64, m0, sb + kCh_G, kLd128, n0, lane);
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const int r = m0 + g, cc = n0 + 8 * nt + 2 * t;
-        st_pair(DXs, kLdS, r, cc, acc[0][nt][0], acc[0][nt][1]);
-        st_pair(DXs, kLdS, r + 8, cc, acc[0][nt][2], acc[0][nt][3]);
-      }
-    }
-    __syncthreads();   // dX complete; (D K)^T, P and the unscaled dO no longer read
-    load_a(c - 1, st ^ 1);
-    // gamma dO in place (bf16, rounded once)
-    for (int e = tid; e < 64 * (kSlice / 2); e += kChainThreads) {
-      const int r = e / (kSlice / 2), cc = 2 * (e - r * (kSlice / 2));
-      const float2 x = ld_pair(DO, kLdS, r, cc);
-      st_pair(DO, kLdS, r, cc, gam[r] * x.x, gam[r] * x.y);
-    }
-    cp_async_wait<1>();   // group B of this chunk
-    __syncthreads();
-    {
-      // G <- gamma_last G - dX^T W + (gamma dO)^T Q
-      const float gl = gam[kC - 1];
-#pragma unroll
-      for (int nt = 0; nt < kGT; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) G[0][nt][e] *= gl;
-      warp_mma<1, kGT, true, true, 64>(G, sb + kCh_DX, kLdS, gm0, sb + kCh_WN, kLd128, gn0, lane);
-      warp_mma<1, kGT, true, true, 64>(G, sb + kCh_DO + st * kTDoS, kLdS, gm0, sb + kCh_Q, kLd128, gn0, lane);
-    }
-    __syncthreads();   // G slice, dX, -W and Q free
-    load_b(c - 1);
-  }
-  cp_async_wait<0>();
-  if (!(ctrl[0] & kErrBadSeqlens) && GDN_IN_BOUNDS(ctrl, (long long)n * H + h, (long long)N * H)) {
-    float *dst = ds0 + (size_t(n) * H + h) * kD * kD;
-#pragma unroll
-    for (int nt = 0; nt < kGT; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = i0 + gm0 + g + 8 * (e >> 1), j = gn0 + 8 * nt + 2 * t + (e & 1);
-        dst[j * kD + i] = G[0][nt][e];
-      }
-  }
 }
 
 // ------------------------------------------------------------------ units
@@ -600,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
   const int m0 = 16 * (warp & 3), n0 = 64 * (warp >> 2), p0 = 32 * (warp >> 2);
   const uint32_t lanes = tmem + (uint32_t(32 * (warp & 3)) << 16);
   // operands
-  const Opnd Qk{sb + kV_Q, 64, false}, Qm{sb + kV_Q, 64, true};
+  const Opnd Qm{sb + kV_Q, 64, true};
   const Opnd Kk{sb + kV_K, 64, false}, Km{sb + kV_K, 64, true};
   const Opnd Vm{sb + kV_V, 64, true};
   const Opnd DOk{sb + kV_DO, 64, false}, DOm{sb + kV_DO, 64, true};
@@ -1010,6 +685,238 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
   }
 }
 
+// ------------------------------------------------------------------ chain
+// The reverse chain over a sequence's chunks on tcgen05. Row i of dS_c depends
+// only on row i of dS_{c+1}, so each (sequence, head) runs as two CTAs of 64
+// d_v rows. The slice of G = dL/dS (64 d_v x 128 d_k, fp32) lives in tensor
+// memory as an M = 64 accumulator; per chunk c, with G = dS_{c+1}:
+//   E0  G -> bf16 (operand, and dS_{c+1} for the unit kernel); G *= gamma_last
+//       in tensor memory; Q *= gamma by rows in shared memory
+//   M1  dX = P^T dO + (D K) G^T                     [64 tokens x 64 d_v]
+//   E1  dX -> bf16
+//   M2  G += dX^T (-W) + dO^T (gamma Q)             [64 d_v x 128 d_k]
+// The next chunk's tiles load (cp.async, two stages) while this one runs.
+constexpr int kChainThreads = 256, kChainSlices = 2, kChainRows = kD / kChainSlices;
+constexpr uint32_t kH_G = 0;                  // G' bf16 [64 d_v][128 d_k]: two 8 KB panels
+constexpr uint32_t kH_DX = kH_G + 16384;      // dX bf16 [64 tokens][64 d_v]: one panel
+constexpr uint32_t kH_STAGE = kH_DX + 8192;
+constexpr uint32_t kHs_KT = 0;                // (D K)^T [128 d_k][64 tokens]: one 16 KB panel
+constexpr uint32_t kHs_P = kHs_KT + 16384;    // P [64][64]
+constexpr uint32_t kHs_DO = kHs_P + 8192;     // dO slice [64 tokens][64 d_v]
+constexpr uint32_t kHs_W = kHs_DO + 8192;     // -W [64][128]
+constexpr uint32_t kHs_Q = kHs_W + 16384;     // Q [64][128], then gamma Q
+constexpr uint32_t kHs_GAM = kHs_Q + 16384;   // gamma [64], D [64]
+constexpr uint32_t kHStage = kHs_GAM + 1024;  // (1 KB keeps the stages 1024-aligned)
+constexpr uint32_t kH_BAR = kH_STAGE + 2 * kHStage;
+constexpr uint32_t kChainSmem = kH_BAR + 32 + 1024;
+static_assert(kHStage % 1024 == 0 && kH_STAGE % 1024 == 0 && kChainSmem <= 232448,
+              "chain kernel shared memory");
+
+__device__ __forceinline__ void tmem_st16x256_x8(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x256b.x8.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__global__ void __launch_bounds__(kChainThreads, 1) gdn_bwd_chain_kernel(
+    const bf16 *__restrict__ q, const bf16 *__restrict__ d_o, const float *__restrict__ d_sN,
+    float *__restrict__ ds0, const uint8_t *__restrict__ ws_w, const uint8_t *__restrict__ ws_kt,
+    const uint8_t *__restrict__ ws_pm, const float *__restrict__ ws_gam,
+    bf16 *__restrict__ gprime, int H, uint32_t *__restrict__ ctrl,
+    const ChunkInfo *__restrict__ table, const int32_t *__restrict__ seq_first, int N,
+    long long rows, int max_chunks) {
+  (void)rows;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n = blockIdx.x, h = blockIdx.y, i0 = kChainRows * int(blockIdx.z);
+  const uint32_t sb = smem_u32(sm);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kH_BAR);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kH_BAR + 8);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kH_BAR + 12);
+  if (tid == 0) {
+    *abort_flag = 0;
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  constexpr uint32_t kCG = 0, kCX = 128;      // TMEM columns: G (128), dX (64)
+  const uint32_t lanes = tmem + (uint32_t(32 * (warp & 3)) << 16);
+  const int m0 = 16 * (warp & 3);             // rows of this warp (d_v for G, tokens for dX)
+  const int gn0 = 64 * (warp >> 2), xn0 = 32 * (warp >> 2);
+  int c0 = 0, nch = 0;
+  if (!(ctrl[0] & kErrBadSeqlens) && GDN_IN_BOUNDS(ctrl, n + 1, N + 1)) {
+    c0 = seq_first[n];
+    nch = seq_first[n + 1] - c0;
+  }
+  auto info_of = [&](int c) {
+    const long long chunk = c0 + c;
+    return GDN_IN_BOUNDS(ctrl, chunk, max_chunks) ? table[chunk] : ChunkInfo{0, 0, 0, 0};
+  };
+  auto load_stage = [&](int c, int st) {
+    if (c >= 0) {
+      const long long unit = (long long)(c0 + c) * H + h;
+      const ChunkInfo ci = info_of(c);
+      const uint32_t sa = sb + kH_STAGE + uint32_t(st) * kHStage;
+      const bf16 *kt = reinterpret_cast<const bf16 *>(ws_kt) + unit * (kD * kC);
+      const bf16 *pm = reinterpret_cast<const bf16 *>(ws_pm) + unit * (kC * kC);
+      const bf16 *wn = reinterpret_cast<const bf16 *>(ws_w) + unit * (kC * kD);
+      for (int e = tid; e < 128 * 8; e += kChainThreads) {
+        const int r = e >> 3, c8 = e & 7;
+        cp_async16(sa + kHs_KT + swz(128, r, 8 * c8), kt + r * kC + 8 * c8, 16u);
+      }
+      for (int e = tid; e < 64 * 8; e += kChainThreads) {
+        const int r = e >> 3, c8 = e & 7;
+        cp_async16(sa + kHs_P + swz(64, r, 8 * c8), pm + r * kC + 8 * c8, 16u);
+        const bool ok = r < ci.len;
+        const bf16 *src =
+            ok ? d_o + ((long long)ci.row0 + r) * H * kD + size_t(h) * kD + i0 + 8 * c8 : d_o;
+        cp_async16(sa + kHs_DO + swz(64, r, 8 * c8), src, ok ? 16u : 0u);
+      }
+      for (int e = tid; e < 64 * 16; e += kChainThreads) {
+        const int r = e >> 4, c16 = e & 15;
+        cp_async16(sa + kHs_W + swz(64, r, 8 * c16), wn + r * kD + 8 * c16, 16u);
+        const bool ok = r < ci.len;
+        const bf16 *src = ok ? q + ((long long)ci.row0 + r) * H * kD + size_t(h) * kD + 8 * c16 : q;
+        cp_async16(sa + kHs_Q + swz(64, r, 8 * c16), src, ok ? 16u : 0u);
+      }
+      if (tid < 32) cp_async16(sa + kHs_GAM + 16 * tid, ws_gam + unit * 128 + 4 * tid, 16u);
+    }
+    cp_async_commit();
+  };
+  // G slice = d_final_state rows [i0, i0 + 64) (stored [d_k][d_v]) into tensor memory
+  {
+    const float *src = d_sN ? d_sN + (size_t(n) * H + h) * kD * kD : nullptr;
+    uint32_t r[32];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = i0 + m0 + (lane >> 2) + 8 * (e >> 1);
+        const int jj = gn0 + 8 * j + 2 * (lane & 3) + (e & 1);
+        r[4 * j + e] = __float_as_uint(src ? src[jj * kD + i] : 0.f);
+      }
+    tmem_st16x256_x8(lanes + kCG + gn0, r);
+    tmem_st_wait();
+  }
+  uint32_t parity = 0;
+  auto mma_sync_wait = [&](auto &&issue) {
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      if (!*abort_flag) issue();
+      tc_commit(bar);
+    }
+    mbar_wait(bar, parity, ctrl, abort_flag);
+    parity ^= 1u;
+    tc_fence_after();
+  };
+  load_stage(nch - 1, 0);
+  for (int it = 0; it < nch; ++it) {
+    const int c = nch - 1 - it, st = it & 1;
+    const long long unit = (long long)(c0 + c) * H + h;
+    load_stage(c - 1, st ^ 1);     // the other stage was last read by chunk c + 1's products
+    cp_async_wait<1>();
+    __syncthreads();               // this stage landed for every thread's copies
+    uint8_t *stage = sm + kH_STAGE + st * kHStage;
+    const uint32_t sa = sb + kH_STAGE + uint32_t(st) * kHStage;
+    const float *gam = reinterpret_cast<const float *>(stage + kHs_GAM);
+    // E0: G' -> bf16; G *= gamma_last; Q *= gamma by rows
+    {
+      uint32_t r[32];
+      tmem_ld16x256_x8(lanes + kCG + gn0, r);
+      tmem_ld_wait();
+      reg_dep(r);
+      const float gl = gam[kC - 1];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int rr = m0 + (lane >> 2) + 8 * hf, cc = gn0 + 8 * j + 2 * (lane & 3);
+          const float x = __uint_as_float(r[4 * j + 2 * hf]), y = __uint_as_float(r[4 * j + 2 * hf + 1]);
+          swz_st(sm + kH_G, 64, rr, cc, x, y);
+          r[4 * j + 2 * hf] = __float_as_uint(gl * x);
+          r[4 * j + 2 * hf + 1] = __float_as_uint(gl * y);
+        }
+      tmem_st16x256_x8(lanes + kCG + gn0, r);
+      tmem_st_wait();
+      for (int e = tid; e < 64 * 64; e += kChainThreads) {
+        const int rr = e >> 6, cc = 2 * (e & 63);
+        const float2 x = swz_ld(stage + kHs_Q, 64, rr, cc);
+        swz_st(stage + kHs_Q, 64, rr, cc, gam[rr] * x.x, gam[rr] * x.y);
+      }
+    }
+    // M1: dX = P^T dO + (D K) G^T   (M = 64 tokens, N = 64 d_v)
+    mma_sync_wait([&] {
+      const Opnd Pm{sa + kHs_P, 64, true}, DOm{sa + kHs_DO, 64, true};
+      const Opnd KTm{sa + kHs_KT, 128, true}, Gk{sb + kH_G, 64, false};
+      mma_product(tmem, kCX, Pm, DOm, 64, 4, false);
+      mma_product(tmem, kCX, KTm, Gk, 64, 8, true);
+    });
+    // dS_{c+1} (bf16, row-major [d_v][d_k]) for the unit kernel, from the G tile
+    if (GDN_IN_BOUNDS(ctrl, unit, (long long)max_chunks * H)) {
+      uint4 *dst = reinterpret_cast<uint4 *>(gprime + unit * (kD * kD) + size_t(i0) * kD);
+      for (int e = tid; e < kChainRows * 16; e += kChainThreads) {
+        const int rr = e >> 4, c16 = e & 15;
+        dst[rr * 16 + c16] = *reinterpret_cast<const uint4 *>(sm + kH_G + swz(64, rr, 8 * c16));
+      }
+    }
+    // E1: dX -> bf16 [tokens][d_v]
+    {
+      float a[4][4];
+      load_acc<4>(a, lanes + kCX + xn0);
+      each_pair<4>(m0, xn0, lane, [&](int j, int hf, int rr, int cc) {
+        swz_st(sm + kH_DX, 64, rr, cc, a[j][2 * hf], a[j][2 * hf + 1]);
+      });
+    }
+    // M2: G += dX^T (-W) + dO^T (gamma Q)   (M = 64 d_v, N = 128 d_k)
+    mma_sync_wait([&] {
+      const Opnd DXm{sb + kH_DX, 64, true}, Wm{sa + kHs_W, 64, true};
+      const Opnd DOm{sa + kHs_DO, 64, true}, Qm{sa + kHs_Q, 64, true};
+      mma_product(tmem, kCG, DXm, Wm, 128, 4, true);
+      mma_product(tmem, kCG, DOm, Qm, 128, 4, true);
+    });
+  }
+  cp_async_wait<0>();
+  if (!(ctrl[0] & kErrBadSeqlens) && GDN_IN_BOUNDS(ctrl, (long long)n * H + h, (long long)N * H)) {
+    uint32_t r[32];
+    tmem_ld16x256_x8(lanes + kCG + gn0, r);
+    tmem_ld_wait();
+    reg_dep(r);
+    float *dst = ds0 + (size_t(n) * H + h) * kD * kD;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = i0 + m0 + (lane >> 2) + 8 * (e >> 1);
+        const int jj = gn0 + 8 * j + 2 * (lane & 3) + (e & 1);
+        dst[jj * kD + i] = __uint_as_float(r[4 * j + e]);
+      }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const float *g,
@@ -1035,7 +942,7 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const flo
   e = cudaFuncSetAttribute(gdn_bwd_unit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kUnitSmem);
   if (e != cudaSuccess) return e;
-  gdn_bwd_chain_kernel<<<dim3(N, H, kSlices), kChainThreads, kChainSmem, s>>>(
+  gdn_bwd_chain_kernel<<<dim3(N, H, kChainSlices), kChainThreads, kChainSmem, s>>>(
       static_cast<const bf16 *>(q), static_cast<const bf16 *>(d_o), d_sN, ds0,
       reinterpret_cast<const uint8_t *>(base + L.fwd.w),
       reinterpret_cast<const uint8_t *>(base + L.fwd.kt),
