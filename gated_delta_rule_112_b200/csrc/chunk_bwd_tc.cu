@@ -690,13 +690,19 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
 // only on row i of dS_{c+1}, so each (sequence, head) runs as two CTAs of 64
 // d_v rows. The slice of G = dL/dS (64 d_v x 128 d_k, fp32) lives in tensor
 // memory as an M = 64 accumulator; per chunk c, with G = dS_{c+1}:
-//   E0  G -> bf16 (operand, and dS_{c+1} for the unit kernel); G *= gamma_last
-//       in tensor memory; Q *= gamma by rows in shared memory
-//   M1  dX = P^T dO + (D K) G^T                     [64 tokens x 64 d_v]
+//   E0  G -> bf16 G' (operand, and dS_{c+1} for the unit kernel)
+//   M1  dX = P^T dO + (D K) G'^T                    [64 tokens x 64 d_v]
+//       then, behind it in the tensor pipe: G *= gamma_last (tcgen05.st) and
+//       G += dO^T (gamma Q)
 //   E1  dX -> bf16
-//   M2  G += dX^T (-W) + dO^T (gamma Q)             [64 d_v x 128 d_k]
-// The next chunk's tiles load (cp.async, two stages) while this one runs.
-constexpr int kChainThreads = 256, kChainSlices = 2, kChainRows = kD / kChainSlices;
+//   M2  G += dX^T (-W)                              [64 d_v x 128 d_k]
+// Only E0 -> M1 -> E1 -> M2 is sequential. Warp 8 is the issuer: one thread
+// loads the chunks' tiles by TMA (three stages, two chunks ahead, 128-byte
+// swizzle: the layouts the MMAs read) and issues every MMA, each group when the mbarrier of its
+// operands completes. Warps 0-7 run the epilogues (E0, E1, the gamma scaling
+// of Q and the bf16 copy of G' to global memory) and arrive on those barriers.
+constexpr int kChainEpi = 256, kChainThreads = kChainEpi + 32;
+constexpr int kChainSlices = 2, kChainRows = kD / kChainSlices;
 constexpr uint32_t kH_G = 0;                  // G' bf16 [64 d_v][128 d_k]: two 8 KB panels
 constexpr uint32_t kH_DX = kH_G + 16384;      // dX bf16 [64 tokens][64 d_v]: one panel
 constexpr uint32_t kH_STAGE = kH_DX + 8192;
@@ -707,8 +713,10 @@ constexpr uint32_t kHs_W = kHs_DO + 8192;     // -W [64][128]
 constexpr uint32_t kHs_Q = kHs_W + 16384;     // Q [64][128], then gamma Q
 constexpr uint32_t kHs_GAM = kHs_Q + 16384;   // gamma [64], D [64]
 constexpr uint32_t kHStage = kHs_GAM + 1024;  // (1 KB keeps the stages 1024-aligned)
-constexpr uint32_t kH_BAR = kH_STAGE + 2 * kHStage;
-constexpr uint32_t kChainSmem = kH_BAR + 32 + 1024;
+constexpr uint32_t kStageBytes = 16384 + 8192 + 8192 + 16384 + 16384 + 512;   // one stage's TMA bytes
+constexpr int kChainStages = 3;
+constexpr uint32_t kH_BAR = kH_STAGE + kChainStages * kHStage;   // 11 mbarriers, TMEM slot, abort flag
+constexpr uint32_t kChainSmem = kH_BAR + 128 + 1024;
 static_assert(kHStage % 1024 == 0 && kH_STAGE % 1024 == 0 && kChainSmem <= 232448,
               "chain kernel shared memory");
 
@@ -725,25 +733,45 @@ __device__ __forceinline__ void tmem_st16x256_x8(uint32_t taddr, const uint32_t 
       : "memory");
 }
 
+// Tensor maps: q and dO as [rows, H, 128] tokens (box 64 x 1 x 64); -W
+// [units * 64][128], (D K)^T [units * 128][64] and P [units * 64][64] (box
+// 64 x rows); the decay factors [units][128] fp32 (one row).
 __global__ void __launch_bounds__(kChainThreads, 1) gdn_bwd_chain_kernel(
-    const bf16 *__restrict__ q, const bf16 *__restrict__ d_o, const float *__restrict__ d_sN,
-    float *__restrict__ ds0, const uint8_t *__restrict__ ws_w, const uint8_t *__restrict__ ws_kt,
-    const uint8_t *__restrict__ ws_pm, const float *__restrict__ ws_gam,
-    bf16 *__restrict__ gprime, int H, uint32_t *__restrict__ ctrl,
-    const ChunkInfo *__restrict__ table, const int32_t *__restrict__ seq_first, int N,
-    long long rows, int max_chunks) {
-  (void)rows;
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+    const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_kt,
+    const __grid_constant__ CUtensorMap tm_pm, const __grid_constant__ CUtensorMap tm_gm,
+    const float *__restrict__ d_sN, float *__restrict__ ds0, bf16 *__restrict__ gprime, int H,
+    uint32_t *__restrict__ ctrl, const ChunkInfo *__restrict__ table,
+    const int32_t *__restrict__ seq_first, int N, int max_chunks) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n = blockIdx.x, h = blockIdx.y, i0 = kChainRows * int(blockIdx.z);
   const uint32_t sb = smem_u32(sm);
+  // mbarriers. One phase per chunk unless noted; "x8": one arrival per epilogue warp.
   uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kH_BAR);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kH_BAR + 8);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kH_BAR + 12);
+  uint64_t *full = bar;           // [3] stage's TMA bytes landed (one phase per use of the stage)
+  uint64_t *ready = bar + 3;      // [3] x8: stage's dO tail zeroed and Q scaled (per use)
+  uint64_t *gb_full = bar + 6;    // x8: G' (bf16) written
+  uint64_t *g_scaled = bar + 7;   // x8: G *= gamma_last stored to tensor memory
+  uint64_t *dx_full = bar + 8;    // commit: dX accumulated
+  uint64_t *dxs_full = bar + 9;   // x8: dX (bf16) written, dX columns read
+  uint64_t *g_full = bar + 10;    // commit: every product of the chunk done
+  uint64_t *drain = bar + 11;     // commit: the issuer's last MMAs done (teardown)
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kH_BAR + 96);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kH_BAR + 100);
   if (tid == 0) {
     *abort_flag = 0;
-    mbar_init(bar, 1);
+    for (int st = 0; st < kChainStages; ++st) {
+      mbar_init(full + st, 1);
+      mbar_init(ready + st, kChainEpi / 32);
+    }
+    mbar_init(gb_full, kChainEpi / 32);
+    mbar_init(g_scaled, kChainEpi / 32);
+    mbar_init(dx_full, 1);
+    mbar_init(dxs_full, kChainEpi / 32);
+    mbar_init(g_full, 1);
+    mbar_init(drain, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -755,9 +783,6 @@ __global__ void __launch_bounds__(kChainThreads, 1) gdn_bwd_chain_kernel(
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   constexpr uint32_t kCG = 0, kCX = 128;      // TMEM columns: G (128), dX (64)
-  const uint32_t lanes = tmem + (uint32_t(32 * (warp & 3)) << 16);
-  const int m0 = 16 * (warp & 3);             // rows of this warp (d_v for G, tokens for dX)
-  const int gn0 = 64 * (warp >> 2), xn0 = 32 * (warp >> 2);
   int c0 = 0, nch = 0;
   if (!(ctrl[0] & kErrBadSeqlens) && GDN_IN_BOUNDS(ctrl, n + 1, N + 1)) {
     c0 = seq_first[n];
@@ -767,147 +792,193 @@ __global__ void __launch_bounds__(kChainThreads, 1) gdn_bwd_chain_kernel(
     const long long chunk = c0 + c;
     return GDN_IN_BOUNDS(ctrl, chunk, max_chunks) ? table[chunk] : ChunkInfo{0, 0, 0, 0};
   };
-  auto load_stage = [&](int c, int st) {
-    if (c >= 0) {
-      const long long unit = (long long)(c0 + c) * H + h;
-      const ChunkInfo ci = info_of(c);
-      const uint32_t sa = sb + kH_STAGE + uint32_t(st) * kHStage;
-      const bf16 *kt = reinterpret_cast<const bf16 *>(ws_kt) + unit * (kD * kC);
-      const bf16 *pm = reinterpret_cast<const bf16 *>(ws_pm) + unit * (kC * kC);
-      const bf16 *wn = reinterpret_cast<const bf16 *>(ws_w) + unit * (kC * kD);
-      for (int e = tid; e < 128 * 8; e += kChainThreads) {
-        const int r = e >> 3, c8 = e & 7;
-        cp_async16(sa + kHs_KT + swz(128, r, 8 * c8), kt + r * kC + 8 * c8, 16u);
+  // Iteration k runs chunk nch - 1 - k from stage k % 3 (the stage's (k / 3)-th use).
+  if (warp == kChainEpi / 32) {
+    // ------------------------------------------------------------ issuer
+    if (lane == 0) {
+      int issued = 0;
+      auto load = [&](int k) {   // TMA of iteration k's tiles (coordinates past the tensors read as zero)
+        const int c = nch - 1 - k;
+        const int unit = (c0 + c) * H + h;
+        const ChunkInfo ci = info_of(c);
+        uint8_t *stage = sm + kH_STAGE + (k % kChainStages) * kHStage;
+        uint64_t *fb = full + k % kChainStages;
+        mbar_arrive_expect_tx(fb, kStageBytes);
+        tma_load_2d(stage + kHs_KT, &tm_kt, fb, 0, unit * kD);
+        tma_load_2d(stage + kHs_P, &tm_pm, fb, 0, unit * kC);
+        tma_load_3d(stage + kHs_DO, &tm_do, fb, i0, h, ci.row0);
+        tma_load_2d(stage + kHs_W, &tm_w, fb, 0, unit * kC);
+        tma_load_2d(stage + kHs_W + 8192, &tm_w, fb, 64, unit * kC);
+        tma_load_3d(stage + kHs_Q, &tm_q, fb, 0, h, ci.row0);
+        tma_load_3d(stage + kHs_Q + 8192, &tm_q, fb, 64, h, ci.row0);
+        tma_load_2d(stage + kHs_GAM, &tm_gm, fb, 0, unit);
+        issued = k + 1;
+      };
+      auto wait_on = [&](uint64_t *b, uint32_t ph) {
+        mbar_wait(b, ph, ctrl, abort_flag);
+        tc_fence_after();
+        return !*abort_flag;
+      };
+      for (int k = 0; k < kChainStages && k < nch; ++k) load(k);
+      for (int it = 0; it < nch; ++it) {
+        const int st = it % kChainStages;
+        const uint32_t ph = uint32_t(it) & 1u, sa = sb + kH_STAGE + uint32_t(st) * kHStage;
+        const Opnd Pm{sa + kHs_P, 64, true}, DOm{sa + kHs_DO, 64, true};
+        const Opnd KTm{sa + kHs_KT, 128, true}, Gk{sb + kH_G, 64, false};
+        const Opnd Wm{sa + kHs_W, 64, true}, Qm{sa + kHs_Q, 64, true};
+        const Opnd DXm{sb + kH_DX, 64, true};
+        // the previous chunk's stage is free once its products are done
+        if (it >= 1 && wait_on(g_full, ph ^ 1u) && it + 2 < nch) load(it + 2);
+        if (wait_on(ready + st, uint32_t(it / kChainStages) & 1u))
+          mma_product(tmem, kCX, Pm, DOm, 64, 4, false);       // dX = P^T dO
+        if (wait_on(gb_full, ph)) mma_product(tmem, kCX, KTm, Gk, 64, 8, true);   // + (D K) G'^T
+        tc_commit(dx_full);
+        if (wait_on(g_scaled, ph)) mma_product(tmem, kCG, DOm, Qm, 128, 4, true);   // G += dO^T (gamma Q)
+        if (wait_on(dxs_full, ph)) mma_product(tmem, kCG, DXm, Wm, 128, 4, true);   // G += dX^T (-W)
+        tc_commit(g_full);
       }
-      for (int e = tid; e < 64 * 8; e += kChainThreads) {
-        const int r = e >> 3, c8 = e & 7;
-        cp_async16(sa + kHs_P + swz(64, r, 8 * c8), pm + r * kC + 8 * c8, 16u);
-        const bool ok = r < ci.len;
-        const bf16 *src =
-            ok ? d_o + ((long long)ci.row0 + r) * H * kD + size_t(h) * kD + i0 + 8 * c8 : d_o;
-        cp_async16(sa + kHs_DO + swz(64, r, 8 * c8), src, ok ? 16u : 0u);
-      }
-      for (int e = tid; e < 64 * 16; e += kChainThreads) {
-        const int r = e >> 4, c16 = e & 15;
-        cp_async16(sa + kHs_W + swz(64, r, 8 * c16), wn + r * kD + 8 * c16, 16u);
-        const bool ok = r < ci.len;
-        const bf16 *src = ok ? q + ((long long)ci.row0 + r) * H * kD + size_t(h) * kD + 8 * c16 : q;
-        cp_async16(sa + kHs_Q + swz(64, r, 8 * c16), src, ok ? 16u : 0u);
-      }
-      if (tid < 32) cp_async16(sa + kHs_GAM + 16 * tid, ws_gam + unit * 128 + 4 * tid, 16u);
+      // teardown: every MMA complete and (after an abort) every copy landed
+      tc_commit(drain);
+      volatile int keep_waiting = 0;
+      mbar_wait(drain, 0, ctrl, &keep_waiting);
+      for (int k = issued - kChainStages < 0 ? 0 : issued - kChainStages; k < issued; ++k)
+        mbar_wait(full + k % kChainStages, uint32_t(k / kChainStages) & 1u, ctrl, &keep_waiting);
     }
-    cp_async_commit();
-  };
-  // G slice = d_final_state rows [i0, i0 + 64) (stored [d_k][d_v]) into tensor memory
-  {
-    const float *src = d_sN ? d_sN + (size_t(n) * H + h) * kD * kD : nullptr;
-    uint32_t r[32];
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = i0 + m0 + (lane >> 2) + 8 * (e >> 1);
-        const int jj = gn0 + 8 * j + 2 * (lane & 3) + (e & 1);
-        r[4 * j + e] = __float_as_uint(src ? src[jj * kD + i] : 0.f);
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const uint32_t lanes = tmem + (uint32_t(32 * (warp & 3)) << 16);
+    const int m0 = 16 * (warp & 3);           // rows of this warp (d_v for G, tokens for dX)
+    const int gn0 = 64 * (warp >> 2), xn0 = 32 * (warp >> 2);
+    auto arrive = [&](uint64_t *b) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b);
+    };
+    // Wait for iteration k's stage, zero the rows of dO past the chunk's end
+    // (they belong to the next sequence) and scale Q rows by gamma (rows past
+    // the end to zero).
+    auto land = [&](int k) {
+      const int st = k % kChainStages;
+      mbar_wait(full + st, uint32_t(k / kChainStages) & 1u, ctrl, abort_flag);
+      const int len = info_of(nch - 1 - k).len;
+      uint8_t *stage = sm + kH_STAGE + st * kHStage;
+      const float *gam = reinterpret_cast<const float *>(stage + kHs_GAM);
+      for (int e = tid; e < (kC - len) * 8; e += kChainEpi) {
+        const int rr = len + (e >> 3), c8 = 8 * (e & 7);
+        *reinterpret_cast<uint4 *>(stage + kHs_DO + swz(64, rr, c8)) = make_uint4(0, 0, 0, 0);
       }
-    tmem_st16x256_x8(lanes + kCG + gn0, r);
-    tmem_st_wait();
-  }
-  uint32_t parity = 0;
-  auto mma_sync_wait = [&](auto &&issue) {
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-      if (!*abort_flag) issue();
-      tc_commit(bar);
-    }
-    mbar_wait(bar, parity, ctrl, abort_flag);
-    parity ^= 1u;
-    tc_fence_after();
-  };
-  load_stage(nch - 1, 0);
-  for (int it = 0; it < nch; ++it) {
-    const int c = nch - 1 - it, st = it & 1;
-    const long long unit = (long long)(c0 + c) * H + h;
-    load_stage(c - 1, st ^ 1);     // the other stage was last read by chunk c + 1's products
-    cp_async_wait<1>();
-    __syncthreads();               // this stage landed for every thread's copies
-    uint8_t *stage = sm + kH_STAGE + st * kHStage;
-    const uint32_t sa = sb + kH_STAGE + uint32_t(st) * kHStage;
-    const float *gam = reinterpret_cast<const float *>(stage + kHs_GAM);
-    // E0: G' -> bf16; G *= gamma_last; Q *= gamma by rows
+      for (int e = tid; e < 64 * 16; e += kChainEpi) {
+        const int rr = e >> 4, c8 = 8 * (e & 15);
+        uint4 *p = reinterpret_cast<uint4 *>(stage + kHs_Q + swz(64, rr, c8));
+        uint4 x = make_uint4(0, 0, 0, 0);
+        if (rr < len) {
+          x = *p;
+          const float gr = gam[rr];
+          uint32_t *w = reinterpret_cast<uint32_t *>(&x);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(w + u));
+            w[u] = pack_bf16x2(gr * f.x, gr * f.y);
+          }
+        }
+        *p = x;
+      }
+      fence_proxy_async_smem();
+      arrive(ready + st);
+    };
+    // G slice = d_final_state rows [i0, i0 + 64) (stored [d_k][d_v]) into tensor memory
     {
+      const float *src = d_sN ? d_sN + (size_t(n) * H + h) * kD * kD : nullptr;
+      uint32_t r[32];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = i0 + m0 + (lane >> 2) + 8 * (e >> 1);
+          const int jj = gn0 + 8 * j + 2 * (lane & 3) + (e & 1);
+          r[4 * j + e] = __float_as_uint(src ? src[jj * kD + i] : 0.f);
+        }
+      tmem_st16x256_x8(lanes + kCG + gn0, r);
+      tmem_st_wait();
+    }
+    if (nch > 0) land(0);
+    for (int it = 0; it < nch; ++it) {
+      const int c = nch - 1 - it;
+      const uint32_t ph = uint32_t(it) & 1u;
+      const long long unit = (long long)(c0 + c) * H + h;
+      const float *gam =
+          reinterpret_cast<const float *>(sm + kH_STAGE + (it % kChainStages) * kHStage + kHs_GAM);
+      if (it >= 1) {
+        mbar_wait(g_full, ph ^ 1u, ctrl, abort_flag);
+        tc_fence_after();
+      }
+      // E0: G' -> bf16 (operand of the dX product)
       uint32_t r[32];
       tmem_ld16x256_x8(lanes + kCG + gn0, r);
       tmem_ld_wait();
       reg_dep(r);
-      const float gl = gam[kC - 1];
+      named_bar_sync(1, kChainEpi);   // the previous chunk's G' tile copied out by every warp
 #pragma unroll
       for (int j = 0; j < 8; ++j)
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const int rr = m0 + (lane >> 2) + 8 * hf, cc = gn0 + 8 * j + 2 * (lane & 3);
-          const float x = __uint_as_float(r[4 * j + 2 * hf]), y = __uint_as_float(r[4 * j + 2 * hf + 1]);
-          swz_st(sm + kH_G, 64, rr, cc, x, y);
-          r[4 * j + 2 * hf] = __float_as_uint(gl * x);
-          r[4 * j + 2 * hf + 1] = __float_as_uint(gl * y);
-        }
+        for (int hf = 0; hf < 2; ++hf)
+          swz_st(sm + kH_G, 64, m0 + (lane >> 2) + 8 * hf, gn0 + 8 * j + 2 * (lane & 3),
+                 __uint_as_float(r[4 * j + 2 * hf]), __uint_as_float(r[4 * j + 2 * hf + 1]));
+      fence_proxy_async_smem();
+      arrive(gb_full);
+      // G *= gamma_last in tensor memory (the chunk's products then accumulate on it)
+      const float gl = gam[kC - 1];
+#pragma unroll
+      for (int u = 0; u < 32; ++u) r[u] = __float_as_uint(gl * __uint_as_float(r[u]));
       tmem_st16x256_x8(lanes + kCG + gn0, r);
       tmem_st_wait();
-      for (int e = tid; e < 64 * 64; e += kChainThreads) {
-        const int rr = e >> 6, cc = 2 * (e & 63);
-        const float2 x = swz_ld(stage + kHs_Q, 64, rr, cc);
-        swz_st(stage + kHs_Q, 64, rr, cc, gam[rr] * x.x, gam[rr] * x.y);
+      tc_fence_before();
+      arrive(g_scaled);
+      // E1: dX -> bf16 [tokens][d_v]
+      mbar_wait(dx_full, ph, ctrl, abort_flag);
+      tc_fence_after();
+      {
+        float a[4][4];
+        load_acc<4>(a, lanes + kCX + xn0);
+        each_pair<4>(m0, xn0, lane, [&](int j, int hf, int rr, int cc) {
+          swz_st(sm + kH_DX, 64, rr, cc, a[j][2 * hf], a[j][2 * hf + 1]);
+        });
       }
-    }
-    // M1: dX = P^T dO + (D K) G^T   (M = 64 tokens, N = 64 d_v)
-    mma_sync_wait([&] {
-      const Opnd Pm{sa + kHs_P, 64, true}, DOm{sa + kHs_DO, 64, true};
-      const Opnd KTm{sa + kHs_KT, 128, true}, Gk{sb + kH_G, 64, false};
-      mma_product(tmem, kCX, Pm, DOm, 64, 4, false);
-      mma_product(tmem, kCX, KTm, Gk, 64, 8, true);
-    });
-    // dS_{c+1} (bf16, row-major [d_v][d_k]) for the unit kernel, from the G tile
-    if (GDN_IN_BOUNDS(ctrl, unit, (long long)max_chunks * H)) {
-      uint4 *dst = reinterpret_cast<uint4 *>(gprime + unit * (kD * kD) + size_t(i0) * kD);
-      for (int e = tid; e < kChainRows * 16; e += kChainThreads) {
-        const int rr = e >> 4, c16 = e & 15;
-        dst[rr * 16 + c16] = *reinterpret_cast<const uint4 *>(sm + kH_G + swz(64, rr, 8 * c16));
+      fence_proxy_async_smem();
+      tc_fence_before();
+      arrive(dxs_full);
+      // dS_{c+1} (bf16, row-major [d_v][d_k]) for the unit kernel, from the G'
+      // tile once every epilogue warp has written its part
+      named_bar_sync(1, kChainEpi);
+      if (GDN_IN_BOUNDS(ctrl, unit, (long long)max_chunks * H)) {
+        uint4 *dst = reinterpret_cast<uint4 *>(gprime + unit * (kD * kD) + size_t(i0) * kD);
+        for (int e = tid; e < kChainRows * 16; e += kChainEpi) {
+          const int rr = e >> 4, c16 = e & 15;
+          dst[rr * 16 + c16] = *reinterpret_cast<const uint4 *>(sm + kH_G + swz(64, rr, 8 * c16));
+        }
       }
+      if (it + 1 < nch) land(it + 1);
     }
-    // E1: dX -> bf16 [tokens][d_v]
-    {
-      float a[4][4];
-      load_acc<4>(a, lanes + kCX + xn0);
-      each_pair<4>(m0, xn0, lane, [&](int j, int hf, int rr, int cc) {
-        swz_st(sm + kH_DX, 64, rr, cc, a[j][2 * hf], a[j][2 * hf + 1]);
-      });
+    if (nch > 0) {
+      mbar_wait(g_full, uint32_t(nch - 1) & 1u, ctrl, abort_flag);
+      tc_fence_after();
     }
-    // M2: G += dX^T (-W) + dO^T (gamma Q)   (M = 64 d_v, N = 128 d_k)
-    mma_sync_wait([&] {
-      const Opnd DXm{sb + kH_DX, 64, true}, Wm{sa + kHs_W, 64, true};
-      const Opnd DOm{sa + kHs_DO, 64, true}, Qm{sa + kHs_Q, 64, true};
-      mma_product(tmem, kCG, DXm, Wm, 128, 4, true);
-      mma_product(tmem, kCG, DOm, Qm, 128, 4, true);
-    });
-  }
-  cp_async_wait<0>();
-  if (!(ctrl[0] & kErrBadSeqlens) && GDN_IN_BOUNDS(ctrl, (long long)n * H + h, (long long)N * H)) {
-    uint32_t r[32];
-    tmem_ld16x256_x8(lanes + kCG + gn0, r);
-    tmem_ld_wait();
-    reg_dep(r);
-    float *dst = ds0 + (size_t(n) * H + h) * kD * kD;
+    if (!(ctrl[0] & kErrBadSeqlens) &&
+        GDN_IN_BOUNDS(ctrl, (long long)n * H + h, (long long)N * H)) {
+      uint32_t r[32];
+      tmem_ld16x256_x8(lanes + kCG + gn0, r);
+      tmem_ld_wait();
+      reg_dep(r);
+      float *dst = ds0 + (size_t(n) * H + h) * kD * kD;
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+      for (int j = 0; j < 8; ++j)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = i0 + m0 + (lane >> 2) + 8 * (e >> 1);
-        const int jj = gn0 + 8 * j + 2 * (lane & 3) + (e & 1);
-        dst[jj * kD + i] = __uint_as_float(r[4 * j + e]);
-      }
+        for (int e = 0; e < 4; ++e) {
+          const int i = i0 + m0 + (lane >> 2) + 8 * (e >> 1);
+          const int jj = gn0 + 8 * j + 2 * (lane & 3) + (e & 1);
+          dst[jj * kD + i] = __uint_as_float(r[4 * j + e]);
+        }
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -942,13 +1013,27 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const flo
   e = cudaFuncSetAttribute(gdn_bwd_unit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kUnitSmem);
   if (e != cudaSuccess) return e;
-  gdn_bwd_chain_kernel<<<dim3(N, H, kChainSlices), kChainThreads, kChainSmem, s>>>(
-      static_cast<const bf16 *>(q), static_cast<const bf16 *>(d_o), d_sN, ds0,
-      reinterpret_cast<const uint8_t *>(base + L.fwd.w),
-      reinterpret_cast<const uint8_t *>(base + L.fwd.kt),
-      reinterpret_cast<const uint8_t *>(base + L.fwd.pm),
-      reinterpret_cast<const float *>(base + L.fwd.gam), gp, H, ctrl, table, seq_first, N, rows,
-      L.fwd.max_chunks);
+  if (T > 0 && L.fwd.max_chunks > 0) {
+    const long long units = (long long)L.fwd.max_chunks * H;
+    CUtensorMap mq, mdo, mw, mkt, mpm, mgm;
+    if (!map_tokens(&mq, q, rows, H) || !map_tokens(&mdo, d_o, rows, H) ||
+        !map_2d(&mw, base + L.fwd.w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, units * kC, kD, 64, kC,
+                CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map_2d(&mkt, base + L.fwd.kt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, units * kD, kC, 64,
+                kD, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map_2d(&mpm, base + L.fwd.pm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, units * kC, kC, 64,
+                kC, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map_2d(&mgm, base + L.fwd.gam, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, units, 128, 128, 1,
+                CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+    gdn_bwd_chain_kernel<<<dim3(N, H, kChainSlices), kChainThreads, kChainSmem, s>>>(
+        mq, mdo, mw, mkt, mpm, mgm, d_sN, ds0, gp, H, ctrl, table, seq_first, N,
+        L.fwd.max_chunks);
+  } else {
+    gdn_bwd_chain_kernel<<<dim3(N, H, kChainSlices), kChainThreads, kChainSmem, s>>>(
+        CUtensorMap{}, CUtensorMap{}, CUtensorMap{}, CUtensorMap{}, CUtensorMap{},
+        CUtensorMap{}, d_sN, ds0, gp, H, ctrl, table, seq_first, N, L.fwd.max_chunks);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int sms = device_sms();

@@ -1751,13 +1751,15 @@ __global__ void __launch_bounds__(256) gdn_segment_combine_kernel(
   }
 }
 
+}  // namespace
+
 // ------------------------------------------------------------------ host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-EncodeTiledFn get_encoder() {
+static EncodeTiledFn get_encoder() {
   static EncodeTiledFn fn = nullptr;
   if (!fn) {
     void *p = nullptr;
@@ -1797,8 +1799,6 @@ bool map_2d(CUtensorMap *m, const void *base, CUtensorMapDataType t, int esize, 
              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-
-}  // namespace
 
 cudaError_t launch_chunk_tc(const void *q, const void *k, const void *v, const float *g,
                             const float *beta, const float *s0, int B, int T, int H, int N,

@@ -2,6 +2,7 @@
 #pragma once
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -157,6 +158,14 @@ inline void prof_record(cudaEvent_t e, cudaStream_t s) {
 }
 
 // Kernel launchers (defined in the .cu files; return a cudaError_t).
+// Tensor maps (host side) for TMA loads, 128-byte swizzle where noted:
+// tokens [rows, H, 128] bf16 with a 64 x 1 x 64 box (swizzled), and a 2-D
+// [rows, inner] map with a (box_inner, box_rows) box. False when the driver's
+// encoder is unavailable or rejects the map.
+bool map_tokens(CUtensorMap *m, const void *base, long long rows, int H);
+bool map_2d(CUtensorMap *m, const void *base, CUtensorMapDataType t, int esize, long long rows,
+            int inner, int box_inner, int box_rows, CUtensorMapSwizzle sw);
+
 cudaError_t launch_chunk_map(const int32_t *cu_seqlens, int B, int T, int num_seqs, int chunk,
                              void *ws, const WsLayout &L, cudaStream_t s);
 // Streaming multiprocessors of the current device (0 if it cannot be read).
