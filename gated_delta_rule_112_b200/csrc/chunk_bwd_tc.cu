@@ -49,17 +49,14 @@ constexpr int kC = 64, kD = 128;
 constexpr int kThreads = 256, kWarps = kThreads / 32;   // the unit kernel's block
 constexpr float kLog2e = 1.4426950408889634f;
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-               "r"(src_bytes)
-               : "memory");
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -102,8 +99,8 @@ constexpr uint32_t kV_X = kV_KT + 16384;      // X [64][128]
 constexpr uint32_t kV_L = kV_X + 16384;       // L [64][64]; then R
 constexpr uint32_t kV_VEC = kV_L + 8192;      // Gamma, gamma, D, dGamma, dbeta, delta [64] fp32
 constexpr uint32_t kV_RED = kV_VEC + 6 * 64 * 4;
-constexpr uint32_t kV_BAR = kV_RED + 4 * kWarps;   // 2 mbarriers, TMEM slot, abort flag
-constexpr uint32_t kUnitSmem = kV_BAR + 32 + 1024;  // + 1024: the window is aligned up to 1 KB
+constexpr uint32_t kV_BAR = kV_RED + 4 * kWarps;   // 4 mbarriers, TMEM slot, abort flag
+constexpr uint32_t kUnitSmem = kV_BAR + 64 + 1024;  // + 1024: the window is aligned up to 1 KB
 static_assert(kV_Q % 1024 == 0 && kV_S % 1024 == 0 && kV_TB % 1024 == 0 && kV_KT % 1024 == 0 &&
                   kV_X % 1024 == 0 && kV_L % 1024 == 0 && kUnitSmem <= 232448,
               "unit kernel shared memory");
@@ -235,16 +232,22 @@ __device__ __forceinline__ void swz_st(uint8_t *t, int rows, int r, int c, float
   *reinterpret_cast<uint32_t *>(t + swz(rows, r, c)) = pack_bf16x2(x, y);
 }
 
+// Loads by TMA (one thread; coordinates past the tensors read as zero):
+// tokens q, k, v, dO [rows, H, 128] (box 64 x 1 x 64, two per tile); -W, T
+// diag(beta), P [units * 64][*] and (D K)^T [units * 128][64] (box 64 x rows);
+// G' [units * 128][128] (box 64 x 128). S_c, stored by the scan in 16-byte
+// pieces (piece p of row i at p * 128 + i), is gathered by cp.async from all
+// threads into the same swizzled row-major layout.
 __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
-    const bf16 *__restrict__ q, const bf16 *__restrict__ k, const bf16 *__restrict__ v,
-    const float *__restrict__ g, const bf16 *__restrict__ d_o,
-    const uint8_t *__restrict__ ws_w, const uint8_t *__restrict__ ws_kt,
-    const uint8_t *__restrict__ ws_tb, const uint8_t *__restrict__ ws_pm,
-    const bf16 *__restrict__ s_chunks, const bf16 *__restrict__ gprime, float *__restrict__ dq,
-    float *__restrict__ dk, float *__restrict__ dv, float *__restrict__ dg,
-    float *__restrict__ dbeta, int H, uint32_t *__restrict__ ctrl,
-    const ChunkInfo *__restrict__ table, long long rows, int max_chunks) {
-  (void)rows;
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+    const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_kt,
+    const __grid_constant__ CUtensorMap tm_tb, const __grid_constant__ CUtensorMap tm_pm,
+    const __grid_constant__ CUtensorMap tm_gp, const bf16 *__restrict__ s_chunks,
+    const float *__restrict__ g, float *__restrict__ dq, float *__restrict__ dk,
+    float *__restrict__ dv, float *__restrict__ dg, float *__restrict__ dbeta, int H,
+    uint32_t *__restrict__ ctrl, const ChunkInfo *__restrict__ table, long long rows,
+    int max_chunks) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -253,13 +256,14 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
   float *gam = Gam + 64, *Dv = Gam + 128, *dGam = Gam + 192, *dBet = Gam + 256,
         *delta = Gam + 320;
   float *red = reinterpret_cast<float *>(sm + kV_RED);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kV_BAR);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kV_BAR + 16);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kV_BAR + 20);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kV_BAR);   // MMA groups (2), loads A, B
+  uint64_t *ld_a = bars + 2, *ld_b = bars + 3;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kV_BAR + 32);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kV_BAR + 36);
   if (tid == 0) {
     *abort_flag = 0;
-    mbar_init(bars, 1);
-    mbar_init(bars + 1, 1);
+#pragma unroll
+    for (int b = 0; b < 4; ++b) mbar_init(bars + b, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -321,57 +325,47 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
     const int c = u / H;
     return GDN_IN_BOUNDS(ctrl, c, max_chunks) ? table[c] : ChunkInfo{0, 0, 0, 0};
   };
-  // token tile of head h (rows past len read as zero) into a [64][128] tile
-  auto load_tok = [&](uint32_t dst, const bf16 *src0, const ChunkInfo &c, int h) {
-    const long long st = (long long)H * kD;
-    for (int e = tid; e < 64 * 16; e += kThreads) {
-      const int r = e >> 4, c16 = e & 15;
-      const bool ok = r < c.len;
-      const bf16 *src = ok ? src0 + ((long long)c.row0 + r) * st + size_t(h) * kD + 8 * c16 : src0;
-      cp_async16(sb + dst + swz(64, r, 8 * c16), src, ok ? 16u : 0u);
+  // group A (Q, K, P) and group B (V, dO, G', T diag(beta), -W, (D K)^T) of
+  // unit u, issued by thread 0; each load completes one phase of its barrier.
+  // S_c of unit u: every thread's share, one cp.async group.
+  auto load_sc = [&](int u) {
+    const bf16 *sc = s_chunks + (long long)u * (kD * kD);
+    for (int e = tid; e < 128 * 16; e += kThreads) {
+      const int p = e >> 7, i = e & 127;
+      cp_async16(sb + kV_S + swz(128, i, 8 * p), sc + (p * 128 + i) * 8);
     }
+    cp_async_commit();
   };
+  int na = 0, nb = 0;
   auto load_a = [&](int u) {
     const ChunkInfo c = info(u);
     const int hu = u % H;
-    load_tok(kV_Q, q, c, hu);
-    load_tok(kV_K, k, c, hu);
-    const bf16 *pm = reinterpret_cast<const bf16 *>(ws_pm) + (long long)u * (kC * kC);
-    for (int e = tid; e < 64 * 8; e += kThreads) {
-      const int r = e >> 3, c16 = e & 7;
-      cp_async16(sb + kV_P + swz(64, r, 8 * c16), pm + r * kC + 8 * c16, 16u);
-    }
-    cp_async_commit();
+    mbar_arrive_expect_tx(ld_a, 2 * 16384 + 8192);
+    tma_load_3d(sm + kV_Q, &tm_q, ld_a, 0, hu, c.row0);
+    tma_load_3d(sm + kV_Q + 8192, &tm_q, ld_a, 64, hu, c.row0);
+    tma_load_3d(sm + kV_K, &tm_k, ld_a, 0, hu, c.row0);
+    tma_load_3d(sm + kV_K + 8192, &tm_k, ld_a, 64, hu, c.row0);
+    tma_load_2d(sm + kV_P, &tm_pm, ld_a, 0, u * kC);
+    ++na;
   };
   auto load_b = [&](int u) {
     const ChunkInfo c = info(u);
     const int hu = u % H;
-    load_tok(kV_V, v, c, hu);
-    load_tok(kV_DO, d_o, c, hu);
-    const bf16 *sc = s_chunks + (long long)u * (kD * kD);
-    const bf16 *gp = gprime + (long long)u * (kD * kD);
-    for (int e = tid; e < 128 * 16; e += kThreads) {
-      const int p = e >> 7, i = e & 127;     // S_c: piece p of row i at p * 128 + i
-      cp_async16(sb + kV_S + swz(128, i, 8 * p), sc + (p * 128 + i) * 8, 16u);
-      const int r = e >> 4, c16 = e & 15;     // G': row-major [d_v][d_k]
-      cp_async16(sb + kV_GP + swz(128, r, 8 * c16), gp + r * kD + 8 * c16, 16u);
-    }
-    const bf16 *tb = reinterpret_cast<const bf16 *>(ws_tb) + (long long)u * (kC * kC);
-    const bf16 *wn = reinterpret_cast<const bf16 *>(ws_w) + (long long)u * (kC * kD);
-    const bf16 *kt = reinterpret_cast<const bf16 *>(ws_kt) + (long long)u * (kD * kC);
-    for (int e = tid; e < 64 * 8; e += kThreads) {
-      const int r = e >> 3, c16 = e & 7;
-      cp_async16(sb + kV_TB + swz(64, r, 8 * c16), tb + r * kC + 8 * c16, 16u);
-    }
-    for (int e = tid; e < 64 * 16; e += kThreads) {
-      const int r = e >> 4, c16 = e & 15;
-      cp_async16(sb + kV_W + swz(64, r, 8 * c16), wn + r * kD + 8 * c16, 16u);
-      const int r2 = e >> 3, c2 = e & 7;      // (D K)^T [128][64]
-      cp_async16(sb + kV_KT + swz(128, r2, 8 * c2), kt + r2 * kC + 8 * c2, 16u);
-    }
-    cp_async_commit();
+    mbar_arrive_expect_tx(ld_b, 4 * 16384 + 32768 + 8192);
+    tma_load_3d(sm + kV_V, &tm_v, ld_b, 0, hu, c.row0);
+    tma_load_3d(sm + kV_V + 8192, &tm_v, ld_b, 64, hu, c.row0);
+    tma_load_3d(sm + kV_DO, &tm_do, ld_b, 0, hu, c.row0);
+    tma_load_3d(sm + kV_DO + 8192, &tm_do, ld_b, 64, hu, c.row0);
+    tma_load_2d(sm + kV_GP, &tm_gp, ld_b, 0, u * kD);
+    tma_load_2d(sm + kV_GP + 16384, &tm_gp, ld_b, 64, u * kD);
+    tma_load_2d(sm + kV_TB, &tm_tb, ld_b, 0, u * kC);
+    tma_load_2d(sm + kV_W, &tm_w, ld_b, 0, u * kC);
+    tma_load_2d(sm + kV_W + 8192, &tm_w, ld_b, 64, u * kC);
+    tma_load_2d(sm + kV_KT, &tm_kt, ld_b, 0, u * kD);
+    ++nb;
   };
   bool first = true;
+  int it_count = 0;
   for (int unit = blockIdx.x; unit < nunits; unit += gridDim.x) {
     const int chunk = unit / H, h = unit - chunk * H;
     const ChunkInfo ci =
@@ -381,8 +375,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
     // B (S_c, G', dO, V, -W, (D K)^T, T diag(beta)) of this unit was issued
     // during the previous one, as soon as its phase 5 had read them; group A
     // (Q, K, P) here.
-    if (first) load_b(unit);
-    load_a(unit);
+    if (first) load_sc(unit);
+    if (tid == 0) {
+      if (first) load_b(unit);
+      load_a(unit);
+    }
     if (warp == 0) {
       // log2(e) Gamma by a warp scan over the 64 tokens (g = 0 past the end)
       float x0 = 0.f, x1 = 0.f;
@@ -411,7 +408,23 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
       dBet[lane] = dBet[lane + 32] = 0.f;
       delta[lane] = delta[lane + 32] = 0.f;
     }
-    cp_async_wait<0>();
+    {
+      // this unit's tiles landed (group B was issued during the previous unit);
+      // rows of q, k, v, dO past the chunk's end (the next sequence's) to zero
+      const uint32_t ph = uint32_t(it_count) & 1u;
+      mbar_wait(ld_a, ph, ctrl, abort_flag);
+      mbar_wait(ld_b, ph, ctrl, abort_flag);
+      cp_async_wait_all();   // S_c (visible to all after the phase-1 barrier)
+      for (int e = tid; e < (kC - len) * 16; e += kThreads) {
+        const int r = len + (e >> 4), c8 = 8 * (e & 15);
+        const uint32_t o = swz(64, r, c8);
+        const uint4 z = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4 *>(sm + kV_Q + o) = z;
+        *reinterpret_cast<uint4 *>(sm + kV_K + o) = z;
+        *reinterpret_cast<uint4 *>(sm + kV_V + o) = z;
+        *reinterpret_cast<uint4 *>(sm + kV_DO + o) = z;
+      }
+    }
     // ---- phase 1
     issue([&] {
       mma_product(tmem, kC0, TBk, Vm, 128, 4, false);       // X = TB V
@@ -596,7 +609,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
       wait_group();
       // S_c, G', dO, V, -W, (D K)^T and T diag(beta) are read for the last
       // time by phase 5: the next unit's copies land during the rest of this one
-      if (unit + int(gridDim.x) < nunits) load_b(unit + int(gridDim.x));
+      if (unit + int(gridDim.x) < nunits) {
+        load_sc(unit + int(gridDim.x));
+        if (tid == 0) load_b(unit + int(gridDim.x));
+      }
       {
         uint32_t r1[32], r2[32];
         tmem_ld16x256_x8(lanes + kC2 + n0, r1);
@@ -673,10 +689,18 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
         }
       }
     }
+    fence_proxy_async_smem();   // generic writes to Q, K, P before their next TMA
     __syncthreads();   // shared memory free for the next unit
     first = false;
+    ++it_count;
   }
-  cp_async_wait<0>();
+  if (tid == 0) {
+    // after an abort: copies still in flight land before the CTA exits (bounded)
+    volatile int keep_waiting = 0;
+    if (na > 0) mbar_wait(ld_a, uint32_t(na - 1) & 1u, ctrl, &keep_waiting);
+    if (nb > 0) mbar_wait(ld_b, uint32_t(nb - 1) & 1u, ctrl, &keep_waiting);
+  }
+  cp_async_wait_all();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -1013,39 +1037,35 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const flo
   e = cudaFuncSetAttribute(gdn_bwd_unit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kUnitSmem);
   if (e != cudaSuccess) return e;
+  // tensor maps (all zero when there are no chunks: no kernel then loads)
+  CUtensorMap mq{}, mk{}, mv{}, mdo{}, mw{}, mkt{}, mtb{}, mpm{}, mgm{}, mgp{};
+  const long long units = (long long)L.fwd.max_chunks * H;
   if (T > 0 && L.fwd.max_chunks > 0) {
-    const long long units = (long long)L.fwd.max_chunks * H;
-    CUtensorMap mq, mdo, mw, mkt, mpm, mgm;
-    if (!map_tokens(&mq, q, rows, H) || !map_tokens(&mdo, d_o, rows, H) ||
+    if (!map_tokens(&mq, q, rows, H) || !map_tokens(&mk, k, rows, H) ||
+        !map_tokens(&mv, v, rows, H) || !map_tokens(&mdo, d_o, rows, H) ||
         !map_2d(&mw, base + L.fwd.w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, units * kC, kD, 64, kC,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
         !map_2d(&mkt, base + L.fwd.kt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, units * kD, kC, 64,
                 kD, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map_2d(&mtb, base + L.fwd.tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, units * kC, kC, 64,
+                kC, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !map_2d(&mpm, base + L.fwd.pm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, units * kC, kC, 64,
                 kC, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !map_2d(&mgm, base + L.fwd.gam, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, units, 128, 128, 1,
-                CU_TENSOR_MAP_SWIZZLE_NONE))
+                CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !map_2d(&mgp, gp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, units * kD, kD, 64, kD,
+                CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
-    gdn_bwd_chain_kernel<<<dim3(N, H, kChainSlices), kChainThreads, kChainSmem, s>>>(
-        mq, mdo, mw, mkt, mpm, mgm, d_sN, ds0, gp, H, ctrl, table, seq_first, N,
-        L.fwd.max_chunks);
-  } else {
-    gdn_bwd_chain_kernel<<<dim3(N, H, kChainSlices), kChainThreads, kChainSmem, s>>>(
-        CUtensorMap{}, CUtensorMap{}, CUtensorMap{}, CUtensorMap{}, CUtensorMap{},
-        CUtensorMap{}, d_sN, ds0, gp, H, ctrl, table, seq_first, N, L.fwd.max_chunks);
   }
+  gdn_bwd_chain_kernel<<<dim3(N, H, kChainSlices), kChainThreads, kChainSmem, s>>>(
+      mq, mdo, mw, mkt, mpm, mgm, d_sN, ds0, gp, H, ctrl, table, seq_first, N, L.fwd.max_chunks);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int sms = device_sms();
-  const long long units = (long long)L.fwd.max_chunks * H;
-  const int grid = int(std::min<long long>(units, sms > 0 ? sms : 148));
+  const int grid = int(std::min<long long>(units > 0 ? units : 1, sms > 0 ? sms : 148));
   gdn_bwd_unit_kernel<<<grid, kThreads, kUnitSmem, s>>>(
-      static_cast<const bf16 *>(q), static_cast<const bf16 *>(k), static_cast<const bf16 *>(v),
-      g, static_cast<const bf16 *>(d_o), reinterpret_cast<const uint8_t *>(base + L.fwd.w),
-      reinterpret_cast<const uint8_t *>(base + L.fwd.kt),
-      reinterpret_cast<const uint8_t *>(base + L.fwd.tb),
-      reinterpret_cast<const uint8_t *>(base + L.fwd.pm), sc, gp, dq, dkk, dvv, dg, dbeta, H,
-      ctrl, table, rows, L.fwd.max_chunks);
+      mq, mk, mv, mdo, mw, mkt, mtb, mpm, mgp, sc, g, dq, dkk, dvv, dg, dbeta, H, ctrl, table,
+      rows, L.fwd.max_chunks);
   (void)beta;
   return cudaGetLastError();
 }
