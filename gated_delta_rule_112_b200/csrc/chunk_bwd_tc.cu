@@ -46,7 +46,8 @@ namespace {
 
 using bf16 = __nv_bfloat16;
 constexpr int kC = 64, kD = 128;
-constexpr int kThreads = 256, kWarps = kThreads / 32;   // the unit kernel's block
+// the unit kernel's block: 8 epilogue warps and one issuer warp (TMA and MMAs)
+constexpr int kThreads = 256, kWarps = kThreads / 32, kUnitThreads = kThreads + 32;
 constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
@@ -238,7 +239,7 @@ __device__ __forceinline__ void swz_st(uint8_t *t, int rows, int r, int c, float
 // G' [units * 128][128] (box 64 x 128). S_c, stored by the scan in 16-byte
 // pieces (piece p of row i at p * 128 + i), is gathered by cp.async from all
 // threads into the same swizzled row-major layout.
-__global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
+__global__ void __launch_bounds__(kUnitThreads, 1) gdn_bwd_unit_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_kt,
@@ -251,6 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool epi = warp < kWarps, issuer = warp == kWarps && lane == 0;
   const uint32_t sb = smem_u32(sm);
   float *Gam = reinterpret_cast<float *>(sm + kV_VEC);   // log2(e) Gamma
   float *gam = Gam + 64, *Dv = Gam + 128, *dGam = Gam + 192, *dBet = Gam + 256,
@@ -301,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) {
+    if (issuer) {
       tc_fence_after();
       if (!*abort_flag) a();
       tc_commit(bars + (next_commit & 1));
@@ -312,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
     }
     next_commit += two ? 2 : 1;
   };
-  auto wait_group = [&]() {
+  auto wait_group = [&]() {   // epilogue warps: the oldest outstanding group
     const int b = next_wait & 1;
     mbar_wait(bars + b, parity[b], ctrl, abort_flag);
     parity[b] ^= 1u;
@@ -375,8 +377,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
     // B (S_c, G', dO, V, -W, (D K)^T, T diag(beta)) of this unit was issued
     // during the previous one, as soon as its phase 5 had read them; group A
     // (Q, K, P) here.
-    if (first) load_sc(unit);
-    if (tid == 0) {
+    if (first && epi) load_sc(unit);
+    if (issuer) {
       if (first) load_b(unit);
       load_a(unit);
     }
@@ -415,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
       mbar_wait(ld_a, ph, ctrl, abort_flag);
       mbar_wait(ld_b, ph, ctrl, abort_flag);
       cp_async_wait_all();   // S_c (visible to all after the phase-1 barrier)
-      for (int e = tid; e < (kC - len) * 16; e += kThreads) {
+      for (int e = tid; epi && e < (kC - len) * 16; e += kThreads) {
         const int r = len + (e >> 4), c8 = 8 * (e & 15);
         const uint32_t o = swz(64, r, c8);
         const uint4 z = make_uint4(0, 0, 0, 0);
@@ -433,7 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
     }, [&] {
       mma_product(tmem, kC3, Kk, Kk, 64, 8, false);         // K K^T
     }, true);
-    {
+    if (epi) {
       // <G', S> for the last token's dGamma
       // (both tiles share one layout: a plain walk over their bytes)
       float gs_dot = 0.f;
@@ -484,8 +486,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
     }, [&] {
       mma_product(tmem, kC2, Kk, Sk, 128, 8, false);        // K S^T (read in phase 4)
     }, true);
-    wait_group();
-    {
+    if (epi) {
+      wait_group();
       float dx[8][4];
       load_acc<8>(dx, lanes + kC1 + n0);
       each_pair<8>(m0, n0, lane, [&](int j, int hf, int r, int c) {
@@ -494,9 +496,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
     }
     // ---- phase 3
     issue([&] { mma_product(tmem, kC0, TBm, DXm, 128, 4, false); }, none, false);   // dV = TB^T dX
-    wait_group();   // K S^T
-    wait_group();   // dV
-    {
+    if (epi) {
+      wait_group();   // K S^T
+      wait_group();   // dV
       float a[8][4];
       load_acc<8>(a, lanes + kC0 + n0);
       each_pair<8>(m0, n0, lane, [&](int j, int hf, int r, int c) {
@@ -516,8 +518,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
       mma_product(tmem, kC1, Lm, DVm, 128, 4, true, true);  // dY = dX - L^T dV
       mma_product(tmem, kC3, Lk, Xm, 128, 4, false);        // L X
     }, true);
-    wait_group();
-    {
+    if (epi) {
+      wait_group();
       float dp[4][4], rp[4][4];
       {
         uint32_t r1[16], r2[16];
@@ -581,9 +583,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
       mma_product(tmem, kC2, Xk, GPm, 128, 8, false);       // X G'
       mma_product(tmem, kC3, DVk, Sm, 128, 8, false);       // dV S
     }, true);
-    wait_group();
     float dkp[8][4];   // D (X G') - gamma (dV S): the first part of dk
-    {
+    if (epi) {
+      wait_group();
       float a[8][4], b[8][4];
       {
         uint32_t r1[32], r2[32];
@@ -609,10 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
       wait_group();
       // S_c, G', dO, V, -W, (D K)^T and T diag(beta) are read for the last
       // time by phase 5: the next unit's copies land during the rest of this one
-      if (unit + int(gridDim.x) < nunits) {
-        load_sc(unit + int(gridDim.x));
-        if (tid == 0) load_b(unit + int(gridDim.x));
-      }
+      if (unit + int(gridDim.x) < nunits) load_sc(unit + int(gridDim.x));
       {
         uint32_t r1[32], r2[32];
         tmem_ld16x256_x8(lanes + kC2 + n0, r1);
@@ -632,14 +631,21 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
       });
       add_rows(dGam, part2, m0, lane);
     }
+    if (issuer && unit + int(gridDim.x) < nunits) {
+      // phase 5's second group (the last reader of the group-B tiles) done:
+      // the next unit's group B loads during the rest of this one
+      const int gidx = next_commit - 1;
+      mbar_wait(bars + (gidx & 1), uint32_t(gidx >> 1) & 1u, ctrl, abort_flag);
+      load_b(unit + int(gridDim.x));
+    }
     // ---- phase 6
     issue([&] {
       mma_product(tmem, kC0, Pm, Qm, 128, 4, false);        // (dP .* E)^T Q
       mma_product(tmem, kC0, Lk, Km, 128, 4, true);         //   + R K
       mma_product(tmem, kC0, Lm, Km, 128, 4, true);         //   + R^T K
     }, none, false);
-    wait_group();
-    {
+    if (epi) {
+      wait_group();
       float a[8][4];
       load_acc<8>(a, lanes + kC0 + n0);
       each_pair<8>(m0, n0, lane, [&](int j, int hf, int r, int c) {
@@ -694,7 +700,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_bwd_unit_kernel(
     first = false;
     ++it_count;
   }
-  if (tid == 0) {
+  if (issuer) {
     // after an abort: copies still in flight land before the CTA exits (bounded)
     volatile int keep_waiting = 0;
     if (na > 0) mbar_wait(ld_a, uint32_t(na - 1) & 1u, ctrl, &keep_waiting);
@@ -1063,7 +1069,7 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const flo
   if (e != cudaSuccess) return e;
   const int sms = device_sms();
   const int grid = int(std::min<long long>(units > 0 ? units : 1, sms > 0 ? sms : 148));
-  gdn_bwd_unit_kernel<<<grid, kThreads, kUnitSmem, s>>>(
+  gdn_bwd_unit_kernel<<<grid, kUnitThreads, kUnitSmem, s>>>(
       mq, mk, mv, mdo, mw, mkt, mtb, mpm, mgp, sc, g, dq, dkk, dvv, dg, dbeta, H, ctrl, table,
       rows, L.fwd.max_chunks);
   (void)beta;
