@@ -46,8 +46,10 @@ namespace {
 
 using bf16 = __nv_bfloat16;
 constexpr int kC = 64, kD = 128;
-// the unit kernel's block: 8 epilogue warps and one issuer warp (TMA and MMAs)
-constexpr int kThreads = 256, kWarps = kThreads / 32, kUnitThreads = kThreads + 32;
+// the unit kernel's block: 16 epilogue warps (four per TMEM lane quadrant,
+// each with a quarter of an accumulator's columns) and one issuer warp (TMA
+// and MMAs)
+constexpr int kThreads = 512, kWarps = kThreads / 32, kUnitThreads = kThreads + 32;
 constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
@@ -169,7 +171,15 @@ __device__ __forceinline__ void to_acc(float (&acc)[NJ][4], const uint32_t (&r)[
 // warp, N = 128 split over the two warps of each row block; NJ = 4: 32 of 64).
 template <int NJ>
 __device__ __forceinline__ void load_acc(float (&acc)[NJ][4], uint32_t taddr) {
-  if constexpr (NJ == 8) {
+  if constexpr (NJ == 2) {
+    uint32_t r[8];
+    tmem_ld16x256_x2(taddr, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[j][e] = __uint_as_float(r[4 * j + e]);
+  } else if constexpr (NJ == 8) {
     uint32_t r[32];
     tmem_ld16x256_x8(taddr, r);
     tmem_ld_wait();
@@ -277,8 +287,8 @@ __global__ void __launch_bounds__(kUnitThreads, 1) gdn_bwd_unit_kernel(
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // epilogue ownership: rows [m0, m0 + 16) (TMEM lanes 32 (w % 4) ..), columns
-  // [n0, n0 + 64) of N = 128 accumulators, [p0, p0 + 32) of N = 64 ones
-  const int m0 = 16 * (warp & 3), n0 = 64 * (warp >> 2), p0 = 32 * (warp >> 2);
+  // [n0, n0 + 32) of N = 128 accumulators, [p0, p0 + 16) of N = 64 ones
+  const int m0 = 16 * (warp & 3), n0 = 32 * (warp >> 2), p0 = 16 * (warp >> 2);
   const uint32_t lanes = tmem + (uint32_t(32 * (warp & 3)) << 16);
   // operands
   const Opnd Qm{sb + kV_Q, 64, true};
@@ -454,27 +464,27 @@ __global__ void __launch_bounds__(kUnitThreads, 1) gdn_bwd_unit_kernel(
       for (int off = 16; off > 0; off >>= 1) gs_dot += __shfl_xor_sync(0xffffffffu, gs_dot, off);
       if (lane == 0) red[warp] = gs_dot;
       wait_group();
-      float xr[8][4], dkg[8][4];
+      float xr[4][4], dkg[4][4];
       {
-        uint32_t r1[32], r2[32];
-        tmem_ld16x256_x8(lanes + kC0 + n0, r1);
-        tmem_ld16x256_x8(lanes + kC1 + n0, r2);
+        uint32_t r1[16], r2[16];
+        tmem_ld16x256_x4(lanes + kC0 + n0, r1);
+        tmem_ld16x256_x4(lanes + kC1 + n0, r2);
         tmem_ld_wait();
         reg_dep(r1);
         reg_dep(r2);
-        to_acc<8>(xr, r1);
-        to_acc<8>(dkg, r2);
+        to_acc<4>(xr, r1);
+        to_acc<4>(dkg, r2);
       }
       float part[2] = {0.f, 0.f};
-      each_pair<8>(m0, n0, lane, [&](int j, int hf, int r, int c) {
+      each_pair<4>(m0, n0, lane, [&](int j, int hf, int r, int c) {
         swz_st(sm + kV_X, 64, r, c, xr[j][2 * hf], xr[j][2 * hf + 1]);
         part[hf] += xr[j][2 * hf] * dkg[j][2 * hf] + xr[j][2 * hf + 1] * dkg[j][2 * hf + 1];
       });
       add_rows(delta, part, m0, lane);
       wait_group();
-      float kk[4][4];
-      load_acc<4>(kk, lanes + kC3 + p0);
-      each_pair<4>(m0, p0, lane, [&](int j, int hf, int r, int s) {
+      float kk[2][4];
+      load_acc<2>(kk, lanes + kC3 + p0);
+      each_pair<2>(m0, p0, lane, [&](int j, int hf, int r, int s) {
         const float e0 = s < r ? ex2(Gam[r] - Gam[s]) : 0.f;
         const float e1 = s + 1 < r ? ex2(Gam[r] - Gam[s + 1]) : 0.f;
         swz_st(sm + kV_L, 64, r, s, e0 * kk[j][2 * hf], e1 * kk[j][2 * hf + 1]);
@@ -488,9 +498,9 @@ __global__ void __launch_bounds__(kUnitThreads, 1) gdn_bwd_unit_kernel(
     }, true);
     if (epi) {
       wait_group();
-      float dx[8][4];
-      load_acc<8>(dx, lanes + kC1 + n0);
-      each_pair<8>(m0, n0, lane, [&](int j, int hf, int r, int c) {
+      float dx[4][4];
+      load_acc<4>(dx, lanes + kC1 + n0);
+      each_pair<4>(m0, n0, lane, [&](int j, int hf, int r, int c) {
         swz_st(sm + kV_W, 64, r, c, dx[j][2 * hf], dx[j][2 * hf + 1]);
       });
     }
@@ -499,9 +509,9 @@ __global__ void __launch_bounds__(kUnitThreads, 1) gdn_bwd_unit_kernel(
     if (epi) {
       wait_group();   // K S^T
       wait_group();   // dV
-      float a[8][4];
-      load_acc<8>(a, lanes + kC0 + n0);
-      each_pair<8>(m0, n0, lane, [&](int j, int hf, int r, int c) {
+      float a[4][4];
+      load_acc<4>(a, lanes + kC0 + n0);
+      each_pair<4>(m0, n0, lane, [&](int j, int hf, int r, int c) {
         swz_st(sm + kV_KT, 64, r, c, a[j][2 * hf], a[j][2 * hf + 1]);
         const long long o = (((long long)ci.row0 + r) * H + h) * kD + c;
         if (r < len && GDN_IN_BOUNDS(ctrl, o + 1, rows * H * kD))
@@ -520,20 +530,20 @@ __global__ void __launch_bounds__(kUnitThreads, 1) gdn_bwd_unit_kernel(
     }, true);
     if (epi) {
       wait_group();
-      float dp[4][4], rp[4][4];
+      float dp[2][4], rp[2][4];
       {
-        uint32_t r1[16], r2[16];
-        tmem_ld16x256_x4(lanes + kC0 + p0, r1);
-        tmem_ld16x256_x4(lanes + kC0 + 64 + p0, r2);
+        uint32_t r1[8], r2[8];
+        tmem_ld16x256_x2(lanes + kC0 + p0, r1);
+        tmem_ld16x256_x2(lanes + kC0 + 64 + p0, r2);
         tmem_ld_wait();
         reg_dep(r1);
         reg_dep(r2);
-        to_acc<4>(dp, r1);
-        to_acc<4>(rp, r2);
+        to_acc<2>(dp, r1);
+        to_acc<2>(rp, r2);
       }
       // dP .* P -> dGamma and dP .* E (s <= r) over P, while the second group runs
-      float rows_[2] = {0.f, 0.f}, cols_[4][2] = {};
-      each_pair<4>(m0, p0, lane, [&](int j, int hf, int r, int s) {
+      float rows_[2] = {0.f, 0.f}, cols_[2][2] = {};
+      each_pair<2>(m0, p0, lane, [&](int j, int hf, int r, int s) {
         const float2 pp = swz_ld(sm + kV_P, 64, r, s);
         const float *a = &dp[j][2 * hf];
         const float f0 = a[0] * pp.x, f1 = a[1] * pp.y;
@@ -546,7 +556,7 @@ __global__ void __launch_bounds__(kUnitThreads, 1) gdn_bwd_unit_kernel(
       });
       wait_group();   // L is free once L^T dV and L X are done
       // -R' .* L -> dGamma, and R = -R' .* E (s < r) over L
-      each_pair<4>(m0, p0, lane, [&](int j, int hf, int r, int s) {
+      each_pair<2>(m0, p0, lane, [&](int j, int hf, int r, int s) {
         const float2 ll = swz_ld(sm + kV_L, 64, r, s);
         const float *b = &rp[j][2 * hf];
         const float f0 = -b[0] * ll.x, f1 = -b[1] * ll.y;
@@ -558,15 +568,15 @@ __global__ void __launch_bounds__(kUnitThreads, 1) gdn_bwd_unit_kernel(
         swz_st(sm + kV_L, 64, r, s, -e0 * b[0], -e1 * b[1]);
       });
       add_rows(dGam, rows_, m0, lane);
-      sub_cols<4>(dGam, cols_, p0, lane);
+      sub_cols<2>(dGam, cols_, p0, lane);
       // e = V - gamma (K S^T) - L X;  dbeta = rowsum(dY .* e)
       {
-        float dy[8][4], ks[8][4], lx[8][4];
-        load_acc<8>(dy, lanes + kC1 + n0);
-        load_acc<8>(ks, lanes + kC2 + n0);
-        load_acc<8>(lx, lanes + kC3 + n0);
+        float dy[4][4], ks[4][4], lx[4][4];
+        load_acc<4>(dy, lanes + kC1 + n0);
+        load_acc<4>(ks, lanes + kC2 + n0);
+        load_acc<4>(lx, lanes + kC3 + n0);
         float part[2] = {0.f, 0.f};
-        each_pair<8>(m0, n0, lane, [&](int j, int hf, int r, int c) {
+        each_pair<4>(m0, n0, lane, [&](int j, int hf, int r, int c) {
           const float2 vv = swz_ld(sm + kV_V, 64, r, c);
           const float e0 = vv.x - gam[r] * ks[j][2 * hf] - lx[j][2 * hf];
           const float e1 = vv.y - gam[r] * ks[j][2 * hf + 1] - lx[j][2 * hf + 1];
@@ -583,22 +593,22 @@ __global__ void __launch_bounds__(kUnitThreads, 1) gdn_bwd_unit_kernel(
       mma_product(tmem, kC2, Xk, GPm, 128, 8, false);       // X G'
       mma_product(tmem, kC3, DVk, Sm, 128, 8, false);       // dV S
     }, true);
-    float dkp[8][4];   // D (X G') - gamma (dV S): the first part of dk
+    float dkp[4][4];   // D (X G') - gamma (dV S): the first part of dk
     if (epi) {
       wait_group();
-      float a[8][4], b[8][4];
+      float a[4][4], b[4][4];
       {
-        uint32_t r1[32], r2[32];
-        tmem_ld16x256_x8(lanes + kC0 + n0, r1);
-        tmem_ld16x256_x8(lanes + kC1 + n0, r2);
+        uint32_t r1[16], r2[16];
+        tmem_ld16x256_x4(lanes + kC0 + n0, r1);
+        tmem_ld16x256_x4(lanes + kC1 + n0, r2);
         tmem_ld_wait();
         reg_dep(r1);
         reg_dep(r2);
-        to_acc<8>(a, r1);
-        to_acc<8>(b, r2);
+        to_acc<4>(a, r1);
+        to_acc<4>(b, r2);
       }
       float part[2] = {0.f, 0.f};
-      each_pair<8>(m0, n0, lane, [&](int j, int hf, int r, int c) {
+      each_pair<4>(m0, n0, lane, [&](int j, int hf, int r, int c) {
         const float2 qq = swz_ld(sm + kV_Q, 64, r, c);
         part[hf] += gam[r] * (qq.x * a[j][2 * hf] + qq.y * a[j][2 * hf + 1]);
         const long long o = (((long long)ci.row0 + r) * H + h) * kD + c;
@@ -613,17 +623,17 @@ __global__ void __launch_bounds__(kUnitThreads, 1) gdn_bwd_unit_kernel(
       // time by phase 5: the next unit's copies land during the rest of this one
       if (unit + int(gridDim.x) < nunits) load_sc(unit + int(gridDim.x));
       {
-        uint32_t r1[32], r2[32];
-        tmem_ld16x256_x8(lanes + kC2 + n0, r1);
-        tmem_ld16x256_x8(lanes + kC3 + n0, r2);
+        uint32_t r1[16], r2[16];
+        tmem_ld16x256_x4(lanes + kC2 + n0, r1);
+        tmem_ld16x256_x4(lanes + kC3 + n0, r2);
         tmem_ld_wait();
         reg_dep(r1);
         reg_dep(r2);
-        to_acc<8>(a, r1);
-        to_acc<8>(b, r2);
+        to_acc<4>(a, r1);
+        to_acc<4>(b, r2);
       }
       float part2[2] = {0.f, 0.f};
-      each_pair<8>(m0, n0, lane, [&](int j, int hf, int r, int c) {
+      each_pair<4>(m0, n0, lane, [&](int j, int hf, int r, int c) {
         const float2 kk2 = swz_ld(sm + kV_K, 64, r, c);
         part2[hf] -= gam[r] * (kk2.x * b[j][2 * hf] + kk2.y * b[j][2 * hf + 1]);
         dkp[j][2 * hf] = Dv[r] * a[j][2 * hf] - gam[r] * b[j][2 * hf];
@@ -646,9 +656,9 @@ __global__ void __launch_bounds__(kUnitThreads, 1) gdn_bwd_unit_kernel(
     }, none, false);
     if (epi) {
       wait_group();
-      float a[8][4];
-      load_acc<8>(a, lanes + kC0 + n0);
-      each_pair<8>(m0, n0, lane, [&](int j, int hf, int r, int c) {
+      float a[4][4];
+      load_acc<4>(a, lanes + kC0 + n0);
+      each_pair<4>(m0, n0, lane, [&](int j, int hf, int r, int c) {
         const long long o = (((long long)ci.row0 + r) * H + h) * kD + c;
         if (r < len && GDN_IN_BOUNDS(ctrl, o + 1, rows * H * kD))
           *reinterpret_cast<float2 *>(dk + o) =
