@@ -70,16 +70,18 @@ __device__ __forceinline__ float ex2(float x) {
 
 // ------------------------------------------------------------------ units
 // Per (chunk, head) unit on tcgen05: every product is an M = 64 (tokens)
-// tcgen05.mma issued by one thread, operands read by the tensor core straight
-// from shared memory, fp32 accumulators in tensor memory (512 columns, one
-// CTA per SM). M = 64 accumulator row r sits in TMEM lane 32 (r / 16) + r % 16,
-// so warp w reads rows 16 (w % 4) .. +15 with tcgen05.ld.16x256b in the
-// mma-fragment layout (rows g, g + 8; columns 2 t, 2 t + 1). All tiles are bf16
-// in 128-byte-swizzled panels of 64 columns; a stored tile serves as a K-major
+// tcgen05.mma issued by one thread of the issuer warp, operands read by the
+// tensor core straight from shared memory, fp32 accumulators in tensor memory
+// (512 columns, one CTA per SM). M = 64 accumulator row r sits in TMEM lane
+// 32 (r / 16) + r % 16, so epilogue warp w reads rows 16 (w % 4) .. +15 with
+// tcgen05.ld.16x256b in the mma-fragment layout (rows g, g + 8; columns 2 t,
+// 2 t + 1), a quarter (w / 4) of the columns. All tiles are bf16 in
+// 128-byte-swizzled panels of 64 columns; a stored tile serves as a K-major
 // operand (rows = M or N) or as an MN-major one (rows = K) per product.
-// Six phases, each an MMA group, one commit and an epilogue by all 8 warps:
+// Six phases, each one or two MMA groups (a commit per group) and an epilogue
+// by the 16 epilogue warps:
 //   1  X = TB V + (-W) S^T [X];  DKG = (D K) G'^T [D];  K K^T [KK]
-//      -> X bf16, delta = rowsum(X .* DKG), -L... L = K K^T .* E (s < r) bf16
+//      -> X bf16, delta = rowsum(X .* DKG), L = K K^T .* E (s < r) bf16
 //   2  D += P^T dO (= dX);  K S^T [KS]          -> dX bf16
 //   3  dV = TB^T dX [X]                         -> dv, dV bf16
 //   4  D -= L^T dV (= dY);  L X [LX];  dO X^T [dP];  dV X^T [R']
