@@ -489,7 +489,47 @@ def main():
                                  "kernel": "chunk_map + prep + scan (replay, chunk states) + "
                                            "gdn_bwd_chain_kernel + gdn_bwd_unit_kernel",
                                  "peak_source": pk["source"]}}
-        del d_o, dsN, bws
+        # A training step: the forward keeping its intermediates and chunk states
+        # (gdn_chunk_fwd_save), then the backward from them (gdn_chunk_bwd_saved,
+        # no replay); and that backward alone, after one saving forward.
+        o_t = torch.empty_like(v)
+
+        def tstep():
+            gdn.chunk_fwd_save(q, k, v, g, beta, s0, cu, workspace=bws, out=o_t)
+            return gdn.chunk_bwd_saved(q, k, v, g, beta, d_o, bws, s0, cu, dsN)
+
+        def timed(fn):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            assert gdn.get_status(bws) == gdn.OK
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(kb)]
+            barrier()
+            torch.cuda.synchronize()
+            for i in range(kb):
+                flush.fill_(i & 0xFF)
+                ev[i][0].record(stream)
+                fn()
+                ev[i][1].record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            return max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / kb)
+
+        ms_t = timed(tstep)
+        gdn.chunk_fwd_save(q, k, v, g, beta, s0, cu, workspace=bws, out=o_t)
+        ms_bs = timed(lambda: gdn.chunk_bwd_saved(q, k, v, g, beta, d_o, bws, s0, cu, dsN))
+        backward["training_step"] = {
+            "ms_per_step": ms_t, "value": replicas.job_rate(tokens, ms_t, world) / 1e6,
+            "unit": UNIT, "gpu_launches": 5 * kb,
+            "api": "chunk_fwd_save + chunk_bwd_saved (C ABI gdn_chunk_fwd_save, "
+                   "gdn_chunk_bwd_saved)",
+            "backward_saved_ms": ms_bs,
+            "replaying_pair_ms": ms + ms_b,
+            "note": "forward with its intermediates and chunk states kept, then the backward "
+                    "from them (no replay); replaying_pair_ms = the forward step above plus "
+                    "the replaying backward"}
+        del d_o, dsN, bws, o_t
         ws = None
 
     del q, k, v, g, beta, o, ws

@@ -14,7 +14,8 @@ import os
 
 import torch
 
-__all__ = ["chunk_fwd", "decode_step", "workspace_size", "chunk_path", "get_status",
+__all__ = ["chunk_fwd", "chunk_bwd", "chunk_fwd_save", "chunk_bwd_saved", "decode_step",
+           "workspace_size", "chunk_path", "get_status",
            "lib", "GdnError", "BF16", "F32", "PATH_TCGEN05", "PATH_SIMT"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -82,6 +83,11 @@ def lib() -> ctypes.CDLL:
         L.gdn_chunk_bwd.argtypes = [vp, vp, vp, fp, fp, fp, ip, vp, fp, ci, ci, ci, ci, ci, ci,
                                     ci, fp, fp, fp, fp, fp, fp, vp, sz, vp]
         L.gdn_chunk_bwd.restype = ci
+        L.gdn_chunk_bwd_saved.argtypes = L.gdn_chunk_bwd.argtypes
+        L.gdn_chunk_bwd_saved.restype = ci
+        L.gdn_chunk_fwd_save.argtypes = [vp, vp, vp, fp, fp, fp, ip, ci, ci, ci, ci, ci, ci, ci,
+                                         vp, fp, vp, sz, vp]
+        L.gdn_chunk_fwd_save.restype = ci
         L.gdn_chunk_bwd_exact.argtypes = [vp, vp, vp, fp, fp, fp, ip, vp, fp, ci, ci, ci, ci, ci, ci,
                                     ci, fp, fp, fp, fp, fp, fp, vp, sz, vp]
         L.gdn_chunk_bwd_exact.restype = ci
@@ -200,7 +206,7 @@ def bwd_workspace_size(B, T, H, d_k, d_v, num_seqs=0, dtype=torch.bfloat16,
 
 
 def chunk_bwd(q, k, v, g, beta, d_o, initial_state=None, cu_seqlens=None, d_final_state=None,
-              workspace=None, stream=None, exact=False):
+              workspace=None, stream=None, exact=False, _saved=False):
     """Gradients of ``chunk_fwd`` (scalar gate) for the loss
     sum(d_o * o) + sum(d_final_state * final_state).
 
@@ -225,17 +231,61 @@ def chunk_bwd(q, k, v, g, beta, d_o, initial_state=None, cu_seqlens=None, d_fina
     need = bwd_workspace_size(B, T, H, dk, dv, num_seqs, q.dtype, exact)
     if need == 0:
         raise GdnError(ERR_INVALID_ARG, "gdn_chunk_bwd_workspace_size")
-    if workspace is None or workspace.numel() < need:
+    if _saved:
+        if workspace is None or workspace.numel() < need:
+            raise GdnError(ERR_WORKSPACE, "gdn_chunk_bwd_saved")
+    elif workspace is None or workspace.numel() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
-    fn = lib().gdn_chunk_bwd_exact if exact else lib().gdn_chunk_bwd
+    fn = (lib().gdn_chunk_bwd_saved if _saved else
+          lib().gdn_chunk_bwd_exact if exact else lib().gdn_chunk_bwd)
+    name = "gdn_chunk_bwd_saved" if _saved else "gdn_chunk_bwd_exact" if exact else "gdn_chunk_bwd"
     rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
             _ptr(cu_seqlens), _ptr(d_o), _ptr(d_final_state), B, T, H, dk, dv,
             num_seqs, _dtype_code(q.dtype), _ptr(out["dq"]), _ptr(out["dk"]),
             _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dbeta"]),
             _ptr(out["d_initial_state"]), _ptr(workspace), workspace.numel(),
             _stream_ptr(stream))
-    _check(rc, "gdn_chunk_bwd_exact" if exact else "gdn_chunk_bwd")
+    _check(rc, name)
     return out
+
+
+def chunk_fwd_save(q, k, v, g, beta, initial_state=None, cu_seqlens=None,
+                   output_final_state=True, workspace=None, out=None, stream=None):
+    """Forward pass of a training step (bf16, d_k = d_v = 128): ``chunk_fwd``
+    that also keeps in its workspace what ``chunk_bwd_saved`` needs (the chunk
+    map, the prep tiles and every chunk's entering state). Returns ``(o,
+    final_state or None, saved)``; hand ``saved`` unchanged to
+    ``chunk_bwd_saved`` with the same inputs."""
+    _require_cuda(q, k, v, g, beta, initial_state, cu_seqlens)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if tuple(g.shape) != (B, T, H):
+        raise ValueError(f"gdn_chunk_fwd_save: g has shape {tuple(g.shape)}")
+    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    N = num_seqs if cu_seqlens is not None else B
+    o = torch.empty(B, T, H, dv, dtype=q.dtype, device=q.device) if out is None else out
+    fs = (torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device)
+          if output_final_state else None)
+    need = bwd_workspace_size(B, T, H, dk, dv, num_seqs, q.dtype)
+    if need == 0:
+        raise GdnError(ERR_INVALID_ARG, "gdn_chunk_bwd_workspace_size")
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    rc = lib().gdn_chunk_fwd_save(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                  _ptr(initial_state), _ptr(cu_seqlens), B, T, H, dk, dv,
+                                  num_seqs, _dtype_code(q.dtype), _ptr(o), _ptr(fs),
+                                  _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    _check(rc, "gdn_chunk_fwd_save")
+    return o, fs, workspace
+
+
+def chunk_bwd_saved(q, k, v, g, beta, d_o, saved, initial_state=None, cu_seqlens=None,
+                    d_final_state=None, stream=None):
+    """``chunk_bwd`` from the workspace ``saved`` that ``chunk_fwd_save`` filled
+    for the same inputs: the forward replay is skipped. Returns the same dict
+    of fp32 gradients."""
+    return chunk_bwd(q, k, v, g, beta, d_o, initial_state, cu_seqlens, d_final_state,
+                     workspace=saved, stream=stream, _saved=True)
 
 
 def get_status(workspace=None, stream=None) -> int:

@@ -42,12 +42,16 @@ inline BwdTcLayout bwd_tc_layout(int B, int T, int H, int num_seqs) {
   return L;
 }
 
+// The chunkwise backward's kernels. replay = false: ws already holds the
+// chunk map, the prep tiles and the chunk states of a forward pass over the
+// same inputs (gdn_chunk_fwd_save), so only the reverse chain and the unit
+// kernel run.
 cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const float *g,
                           const float *beta, const float *s0, const int32_t *cu,
                           const void *d_o, const float *d_sN, int N, int B, int T, int H,
                           int num_seqs, float *dq, float *dkk, float *dvv, float *dg,
                           float *dbeta, float *ds0, void *ws, const BwdTcLayout &L,
-                          cudaStream_t s);
+                          cudaStream_t s, bool replay = true);
 
 cudaError_t launch_bwd(const void *q, const void *k, const void *v, const float *g,
                        const float *beta, const float *s0, const int32_t *cu, const void *d_o,

@@ -1037,14 +1037,17 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const flo
                           const void *d_o, const float *d_sN, int N, int B, int T, int H,
                           int num_seqs, float *dq, float *dkk, float *dvv, float *dg,
                           float *dbeta, float *ds0, void *ws, const BwdTcLayout &L,
-                          cudaStream_t s) {
+                          cudaStream_t s, bool replay) {
   char *base = static_cast<char *>(ws);
-  cudaError_t e = launch_chunk_map(cu, B, T, num_seqs, kC, ws, L.fwd, s);
-  if (e != cudaSuccess) return e;
   bf16 *sc = reinterpret_cast<bf16 *>(base + L.s_chunks);
   bf16 *gp = reinterpret_cast<bf16 *>(base + L.gprime);
-  e = launch_chunk_tc(q, k, v, g, beta, s0, B, T, H, N, nullptr, nullptr, ws, L.fwd, s, sc);
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
+  if (replay) {
+    e = launch_chunk_map(cu, B, T, num_seqs, kC, ws, L.fwd, s);
+    if (e != cudaSuccess) return e;
+    e = launch_chunk_tc(q, k, v, g, beta, s0, B, T, H, N, nullptr, nullptr, ws, L.fwd, s, sc);
+    if (e != cudaSuccess) return e;
+  }
   uint32_t *ctrl = reinterpret_cast<uint32_t *>(base);
   const ChunkInfo *table = reinterpret_cast<const ChunkInfo *>(base + L.fwd.chunk_table);
   const int32_t *seq_first = reinterpret_cast<const int32_t *>(base + L.fwd.seq_first);

@@ -194,7 +194,9 @@ size_t gdn_chunk_bwd_workspace_size(int B, int T, int H, int d_k, int d_v, int n
 
 namespace {
 
-int run_bwd(bool exact, const void *q, const void *k, const void *v, const float *g,
+// saved: the workspace holds a gdn_chunk_fwd_save pass over the same inputs
+// (tensor-core path only), so the forward replay is skipped.
+int run_bwd(bool exact, bool saved, const void *q, const void *k, const void *v, const float *g,
             const float *beta, const float *initial_state, const int32_t *cu_seqlens,
             const void *d_o, const float *d_final_state, int B, int T, int H, int d_k, int d_v,
             int num_seqs, int dtype, float *dq, float *dk, float *dv, float *dg, float *dbeta,
@@ -218,6 +220,7 @@ int run_bwd(bool exact, const void *q, const void *k, const void *v, const float
   const int N = cu_seqlens ? num_seqs : B;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
+  if (saved && !tc_path(d_k, d_v, 64, dtype)) return GDN_ERR_UNSUPPORTED;
   if (!exact && tc_path(d_k, d_v, 64, dtype)) {
     const BwdTcLayout L = bwd_tc_layout(B, T, H, cu_seqlens ? num_seqs : 0);
     if (workspace_bytes < L.total) return GDN_ERR_WORKSPACE;
@@ -231,7 +234,7 @@ int run_bwd(bool exact, const void *q, const void *k, const void *v, const float
     } else {
       e = launch_bwd_tc(q, k, v, g, beta, initial_state, cu_seqlens, d_o, d_final_state, N, B,
                         T, H, cu_seqlens ? num_seqs : 0, dq, dk, dv, dg, dbeta,
-                        d_initial_state, workspace, L, s);
+                        d_initial_state, workspace, L, s, !saved);
     }
   } else {
     const BwdLayout L = bwd_layout(B, T, H, d_k, d_v);
@@ -252,9 +255,45 @@ int gdn_chunk_bwd(const void *q, const void *k, const void *v, const float *g, c
                   int num_seqs, int dtype, float *dq, float *dk, float *dv, float *dg,
                   float *dbeta, float *d_initial_state, void *workspace,
                   size_t workspace_bytes, void *stream) {
-  return run_bwd(false, q, k, v, g, beta, initial_state, cu_seqlens, d_o, d_final_state, B, T, H,
-                 d_k, d_v, num_seqs, dtype, dq, dk, dv, dg, dbeta, d_initial_state, workspace,
-                 workspace_bytes, stream);
+  return run_bwd(false, false, q, k, v, g, beta, initial_state, cu_seqlens, d_o, d_final_state,
+                 B, T, H, d_k, d_v, num_seqs, dtype, dq, dk, dv, dg, dbeta, d_initial_state,
+                 workspace, workspace_bytes, stream);
+}
+
+int gdn_chunk_bwd_saved(const void *q, const void *k, const void *v, const float *g,
+                        const float *beta, const float *initial_state,
+                        const int32_t *cu_seqlens, const void *d_o, const float *d_final_state,
+                        int B, int T, int H, int d_k, int d_v, int num_seqs, int dtype,
+                        float *dq, float *dk, float *dv, float *dg, float *dbeta,
+                        float *d_initial_state, void *workspace, size_t workspace_bytes,
+                        void *stream) {
+  return run_bwd(false, true, q, k, v, g, beta, initial_state, cu_seqlens, d_o, d_final_state,
+                 B, T, H, d_k, d_v, num_seqs, dtype, dq, dk, dv, dg, dbeta, d_initial_state,
+                 workspace, workspace_bytes, stream);
+}
+
+int gdn_chunk_fwd_save(const void *q, const void *k, const void *v, const float *g,
+                       const float *beta, const float *initial_state, const int32_t *cu_seqlens,
+                       int B, int T, int H, int d_k, int d_v, int num_seqs, int dtype, void *o,
+                       float *final_state, void *workspace, size_t workspace_bytes,
+                       void *stream) {
+  int rc = check_chunk_args(q, k, v, g, beta, initial_state, cu_seqlens, B, T, H, d_k, d_v,
+                            num_seqs, 64, dtype, o, final_state, workspace);
+  if (rc != GDN_OK) return rc;
+  if (!tc_path(d_k, d_v, 64, dtype)) return GDN_ERR_UNSUPPORTED;
+  const int ns = cu_seqlens ? num_seqs : 0;
+  const BwdTcLayout L = bwd_tc_layout(B, T, H, ns);
+  if (workspace_bytes < L.total) return GDN_ERR_WORKSPACE;
+  const int N = cu_seqlens ? num_seqs : B;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_chunk_map(cu_seqlens, B, T, ns, 64, workspace, L.fwd, s);
+  if (e == cudaSuccess) {
+    __nv_bfloat16 *sc =
+        reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(workspace) + L.s_chunks);
+    e = launch_chunk_tc(q, k, v, g, beta, initial_state, B, T, H, N, o, final_state, workspace,
+                        L.fwd, s, sc);
+  }
+  return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 int gdn_chunk_bwd_exact(const void *q, const void *k, const void *v, const float *g,
@@ -264,9 +303,9 @@ int gdn_chunk_bwd_exact(const void *q, const void *k, const void *v, const float
                         float *dq, float *dk, float *dv, float *dg, float *dbeta,
                         float *d_initial_state, void *workspace, size_t workspace_bytes,
                         void *stream) {
-  return run_bwd(true, q, k, v, g, beta, initial_state, cu_seqlens, d_o, d_final_state, B, T, H,
-                 d_k, d_v, num_seqs, dtype, dq, dk, dv, dg, dbeta, d_initial_state, workspace,
-                 workspace_bytes, stream);
+  return run_bwd(true, false, q, k, v, g, beta, initial_state, cu_seqlens, d_o, d_final_state,
+                 B, T, H, d_k, d_v, num_seqs, dtype, dq, dk, dv, dg, dbeta, d_initial_state,
+                 workspace, workspace_bytes, stream);
 }
 
 int gdn_get_status(void *workspace, void *stream) {

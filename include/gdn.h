@@ -314,10 +314,11 @@ size_t gdn_chunk_bwd_exact_workspace_size(int B, int T, int H, int d_k, int d_v,
  * 8-byte aligned. bf16 with d_k = d_v = 128 runs the chunkwise backward on
  * the tensor cores (64-token chunks; the derivation is in the header of the
  * kernels' source): the forward pass again, its scan also keeping every
- * chunk's entering state S_c (bf16); a reverse scan over the chunks, one CTA
+ * chunk's entering state S_c (bf16); a reverse scan over the chunks, two CTAs
  * per (sequence, head), of dS_c = gamma_last dS_{c+1} - dX^T W +
  * (gamma dO)^T Q, keeping each chunk's dS_{c+1} (bf16); and one kernel over
- * all (chunk, head) units for dq, dk, dv, dg, dbeta. bf16 operands, fp32
+ * all (chunk, head) units for dq, dk, dv, dg, dbeta. gdn_chunk_fwd_save and
+ * gdn_chunk_bwd_saved split the same work for a training step (below). bf16 operands, fp32
  * accumulation: its parity bar is the bf16 tolerance. Every other size and
  * dtype runs gdn_chunk_bwd_exact. Bad cu_seqlens contents are reported by
  * gdn_get_status (GDN_ERR_INVALID_ARG); the affected sequences are not
@@ -329,6 +330,47 @@ int gdn_chunk_bwd(const void *q, const void *k, const void *v, const float *g, c
                   int num_seqs, int dtype, float *dq, float *dk, float *dv, float *dg,
                   float *dbeta, float *d_initial_state, void *workspace,
                   size_t workspace_bytes, void *stream);
+
+/*
+ * gdn_chunk_fwd_save -- the forward pass of a training step: gdn_chunk_fwd
+ * (same arguments and outputs, 64-token chunks) that also leaves in
+ * `workspace` what the chunkwise backward would otherwise recompute: the
+ * chunk map, the prep tiles (-W, (D K)^T, T diag(beta), P, the decay
+ * factors) and every chunk's entering state S_c (bf16). The pages present the
+ * chunkwise algorithm for training (phantomic12 page, mechanism paragraph);
+ * keeping the forward's intermediates for the backward is this library's
+ * reading of that use.
+ *   workspace          >= gdn_chunk_bwd_workspace_size() bytes for the same
+ *                      sizes, 256-byte aligned; owned by the caller and handed
+ *                      unchanged to gdn_chunk_bwd_saved.
+ * Tensor-core path only (bf16, d_k = d_v = 128): GDN_ERR_UNSUPPORTED
+ * otherwise. The state scan always runs as one pass per (sequence, head) here
+ * (gdn_chunk_fwd may split long sequences into segments), so o and
+ * final_state are those of that pass.
+ */
+int gdn_chunk_fwd_save(const void *q, const void *k, const void *v, const float *g,
+                       const float *beta, const float *initial_state, const int32_t *cu_seqlens,
+                       int B, int T, int H, int d_k, int d_v, int num_seqs, int dtype, void *o,
+                       float *final_state, void *workspace, size_t workspace_bytes,
+                       void *stream);
+
+/*
+ * gdn_chunk_bwd_saved -- gdn_chunk_bwd (same arguments and outputs) for a
+ * workspace that gdn_chunk_fwd_save filled from the same q, k, v, g, beta,
+ * initial_state, cu_seqlens and sizes on this stream: the forward replay is
+ * skipped and only the reverse chain and the per-unit kernel run. The
+ * workspace's saved part is read, not changed (the call may be repeated for
+ * another d_o). Tensor-core path only: GDN_ERR_UNSUPPORTED otherwise. The
+ * kernels trust the saved chunk table: a workspace that gdn_chunk_fwd_save
+ * did not fill for these inputs is undefined behaviour.
+ */
+int gdn_chunk_bwd_saved(const void *q, const void *k, const void *v, const float *g,
+                        const float *beta, const float *initial_state,
+                        const int32_t *cu_seqlens, const void *d_o, const float *d_final_state,
+                        int B, int T, int H, int d_k, int d_v, int num_seqs, int dtype,
+                        float *dq, float *dk, float *dv, float *dg, float *dbeta,
+                        float *d_initial_state, void *workspace, size_t workspace_bytes,
+                        void *stream);
 
 /*
  * gdn_chunk_bwd_exact -- the same gradients by the token-level recurrence in

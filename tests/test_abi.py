@@ -199,3 +199,34 @@ def test_bwd_host_checks(L):
     fwd = L.gdn_chunk_fwd_workspace_size(4, 4096, 16, 128, 128, 0, 64, gdn.BF16)
     assert tc >= fwd + 4096 * 2 * 128 * 128 * 2
     assert tc < fwd + 4096 * 2 * 128 * 128 * 2 + (1 << 20)
+
+
+def test_saved_pair_host_checks(L):
+    """gdn_chunk_fwd_save / gdn_chunk_bwd_saved: tensor-core path only, and the
+    backward's workspace size (checked before anything is launched)."""
+    vp = ctypes.c_void_p
+    p = vp(1 << 20)
+
+    def fwd(**kw):
+        a = dict(B=1, T=64, H=1, dk=128, dv=128, ns=0, dtype=gdn.BF16, o=p, ws=p, wsb=1 << 40)
+        a.update(kw)
+        return L.gdn_chunk_fwd_save(p, p, p, p, p, None, None, a["B"], a["T"], a["H"], a["dk"],
+                                    a["dv"], a["ns"], a["dtype"], a["o"], None, a["ws"],
+                                    a["wsb"], None)
+
+    def bwd(**kw):
+        a = dict(dk=128, dv=128, dtype=gdn.BF16, wsb=1 << 40)
+        a.update(kw)
+        return L.gdn_chunk_bwd_saved(p, p, p, p, p, None, None, p, None, 1, 64, 1, a["dk"],
+                                     a["dv"], 0, a["dtype"], p, p, p, p, p, p, p, a["wsb"], None)
+
+    assert fwd(dtype=gdn.F32) == gdn.ERR_UNSUPPORTED
+    assert fwd(dk=64) == gdn.ERR_UNSUPPORTED
+    assert fwd(o=None) == gdn.ERR_INVALID_ARG
+    assert fwd(ws=None) == gdn.ERR_WORKSPACE
+    need = L.gdn_chunk_bwd_workspace_size(1, 64, 1, 128, 128, 0, gdn.BF16)
+    assert need > L.gdn_chunk_fwd_workspace_size(1, 64, 1, 128, 128, 0, 64, gdn.BF16)
+    assert fwd(wsb=need - 1) == gdn.ERR_WORKSPACE
+    assert bwd(dtype=gdn.F32) == gdn.ERR_UNSUPPORTED
+    assert bwd(dk=64) == gdn.ERR_UNSUPPORTED
+    assert bwd(wsb=need - 1) == gdn.ERR_WORKSPACE

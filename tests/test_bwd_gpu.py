@@ -15,7 +15,7 @@ import torch
 
 import oracle
 from gated_delta_rule_112_b200.inputs import Workload, make_chunk_inputs
-from tests.parity import TOL_BF16, TOL_F32, assert_close, np64, to_dev
+from tests.parity import TOL_BF16, TOL_F32, assert_close, np64, oracle_chunk, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -181,3 +181,77 @@ def test_workload_bwd_b4h16t4096():
     inp = make_chunk_inputs("b4h16t4096")
     d_o, dsN = upstream(inp, seed=5)
     check(inp, d_o, dsN, tol=TOL_BF16)
+
+
+def check_saved(inp, d_o, dsN):
+    """A training step through chunk_fwd_save and chunk_bwd_saved: the forward
+    outputs and all six gradients against the oracle, the gradients also
+    against the replaying chunk_bwd (the saved intermediates and chunk states
+    are the ones the replay recomputes), and a second backward from the same
+    saved workspace unchanged."""
+    import gated_delta_rule_112_b200 as gdn
+    d = to_dev(inp)
+    fwd = (d["q"], d["k"], d["v"], d["g"], d["beta"])
+    dsn = None if dsN is None else dsN.cuda()
+    o, fs, saved = gdn.chunk_fwd_save(*fwd, d["initial_state"], d["cu_seqlens"])
+    torch.cuda.synchronize()
+    assert gdn.get_status() == gdn.OK
+    ref_o, ref_s = oracle_chunk(inp)
+    assert_close("o", np64(o), ref_o, TOL_BF16)
+    assert_close("final_state", np64(fs), ref_s, TOL_BF16)
+    got = gdn.chunk_bwd_saved(*fwd, d_o.cuda(), saved, d["initial_state"], d["cu_seqlens"], dsn)
+    again = gdn.chunk_bwd_saved(*fwd, d_o.cuda(), saved, d["initial_state"], d["cu_seqlens"],
+                                dsn)
+    replay = gdn.chunk_bwd(*fwd, d_o.cuda(), d["initial_state"], d["cu_seqlens"], dsn)
+    torch.cuda.synchronize()
+    assert gdn.get_status() == gdn.OK
+    s0, cu = inp["initial_state"], inp["cu_seqlens"]
+    ref = oracle.chunk_bwd(np64(inp["q"]), np64(inp["k"]), np64(inp["v"]), np64(inp["g"]),
+                           np64(inp["beta"]), np64(d_o), None if s0 is None else np64(s0),
+                           None if cu is None else cu.numpy(),
+                           None if dsN is None else np64(dsN))
+    for key in KEYS:
+        assert_close(key, np64(got[key]), ref[key], TOL_BF16)
+        if key in ("dg", "dbeta"):
+            # summed from per-warp partials by shared-memory atomics: equal
+            # across calls to rounding, not bit for bit
+            assert_close(key + " (repeat)", np64(again[key]), np64(got[key]), 1e-6)
+        else:
+            assert torch.equal(got[key], again[key]), key
+        # the same kernels on the same intermediates as the replay
+        assert_close(key + " (saved vs replay)", np64(got[key]), np64(replay[key]), 1e-5)
+    return got
+
+
+def test_bwd_saved_batch_heads():
+    inp = make_chunk_inputs(TC, B=3, H=5, T=257, random_state=True)
+    d_o, dsN = upstream(inp, seed=46)
+    check_saved(inp, d_o, dsN)
+
+
+def test_bwd_saved_varlen_with_empty_sequences():
+    inp = make_chunk_inputs(TC, H=2, lengths=[50, 0, 131, 1, 64], random_state=True)
+    d_o, dsN = upstream(inp, seed=47)
+    got = check_saved(inp, d_o, dsN)
+    np.testing.assert_array_equal(np64(got["d_initial_state"][1]), np64(dsN[1]))
+
+
+def test_bwd_saved_zero_tokens():
+    import gated_delta_rule_112_b200 as gdn
+    inp = make_chunk_inputs(TC, T=0, random_state=True)
+    d_o, dsN = upstream(inp, seed=48)
+    d = to_dev(inp)
+    fwd = (d["q"], d["k"], d["v"], d["g"], d["beta"])
+    o, fs, saved = gdn.chunk_fwd_save(*fwd, d["initial_state"])
+    got = gdn.chunk_bwd_saved(*fwd, d_o.cuda(), saved, d["initial_state"], None, dsN.cuda())
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(np64(fs), np64(inp["initial_state"]))
+    np.testing.assert_array_equal(np64(got["d_initial_state"]), np64(dsN))
+
+
+def test_bwd_saved_rejects_other_paths():
+    import gated_delta_rule_112_b200 as gdn
+    inp = make_chunk_inputs(SMALL, T=64)          # fp32: the token-level backward's domain
+    d = to_dev(inp)
+    with pytest.raises(gdn.GdnError):
+        gdn.chunk_fwd_save(d["q"], d["k"], d["v"], d["g"], d["beta"])
