@@ -740,10 +740,12 @@ __global__ void __launch_bounds__(kUnitThreads, 1) gdn_bwd_unit_kernel(
 //   M2  G += dX^T (-W)                              [64 d_v x 128 d_k]
 // Only E0 -> M1 -> E1 -> M2 is sequential. Warp 8 is the issuer: one thread
 // loads the chunks' tiles by TMA (three stages, two chunks ahead, 128-byte
-// swizzle: the layouts the MMAs read) and issues every MMA, each group when the mbarrier of its
-// operands completes. Warps 0-7 run the epilogues (E0, E1, the gamma scaling
-// of Q and the bf16 copy of G' to global memory) and arrive on those barriers.
-constexpr int kChainEpi = 256, kChainThreads = kChainEpi + 32;
+// swizzle: the layouts the MMAs read) and issues every MMA, each group when
+// the mbarrier of its operands completes. Warps 0-7 run the epilogues E0 and
+// E1 and the gamma_last scaling of G; warps 9-12 copy each G' tile to global
+// memory and prepare each landed stage (the dO tail zeroed, Q scaled by
+// gamma), all handing over on mbarriers.
+constexpr int kChainEpi = 256, kChainLoad = 128, kChainThreads = kChainEpi + 32 + kChainLoad;
 constexpr int kChainSlices = 2, kChainRows = kD / kChainSlices;
 constexpr uint32_t kH_G = 0;                  // G' bf16 [64 d_v][128 d_k]: two 8 KB panels
 constexpr uint32_t kH_DX = kH_G + 16384;      // dX bf16 [64 tokens][64 d_v]: one panel
@@ -757,7 +759,7 @@ constexpr uint32_t kHs_GAM = kHs_Q + 16384;   // gamma [64], D [64]
 constexpr uint32_t kHStage = kHs_GAM + 1024;  // (1 KB keeps the stages 1024-aligned)
 constexpr uint32_t kStageBytes = 16384 + 8192 + 8192 + 16384 + 16384 + 512;   // one stage's TMA bytes
 constexpr int kChainStages = 3;
-constexpr uint32_t kH_BAR = kH_STAGE + kChainStages * kHStage;   // 11 mbarriers, TMEM slot, abort flag
+constexpr uint32_t kH_BAR = kH_STAGE + kChainStages * kHStage;   // 13 mbarriers, TMEM slot, abort flag
 constexpr uint32_t kChainSmem = kH_BAR + 128 + 1024;
 static_assert(kHStage % 1024 == 0 && kH_STAGE % 1024 == 0 && kChainSmem <= 232448,
               "chain kernel shared memory");
@@ -793,21 +795,23 @@ __global__ void __launch_bounds__(kChainThreads, 1) gdn_bwd_chain_kernel(
   // mbarriers. One phase per chunk unless noted; "x8": one arrival per epilogue warp.
   uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kH_BAR);
   uint64_t *full = bar;           // [3] stage's TMA bytes landed (one phase per use of the stage)
-  uint64_t *ready = bar + 3;      // [3] x8: stage's dO tail zeroed and Q scaled (per use)
+  uint64_t *ready = bar + 3;      // [3] x4: stage's dO tail zeroed and Q scaled (per use)
   uint64_t *gb_full = bar + 6;    // x8: G' (bf16) written
   uint64_t *g_scaled = bar + 7;   // x8: G *= gamma_last stored to tensor memory
   uint64_t *dx_full = bar + 8;    // commit: dX accumulated
   uint64_t *dxs_full = bar + 9;   // x8: dX (bf16) written, dX columns read
   uint64_t *g_full = bar + 10;    // commit: every product of the chunk done
   uint64_t *drain = bar + 11;     // commit: the issuer's last MMAs done (teardown)
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kH_BAR + 96);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kH_BAR + 100);
+  uint64_t *gb_free = bar + 12;   // x4: G' copied to global memory (the tile may be rewritten)
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kH_BAR + 104);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kH_BAR + 108);
   if (tid == 0) {
     *abort_flag = 0;
     for (int st = 0; st < kChainStages; ++st) {
       mbar_init(full + st, 1);
-      mbar_init(ready + st, kChainEpi / 32);
+      mbar_init(ready + st, kChainLoad / 32);
     }
+    mbar_init(gb_free, kChainLoad / 32);
     mbar_init(gb_full, kChainEpi / 32);
     mbar_init(g_scaled, kChainEpi / 32);
     mbar_init(dx_full, 1);
@@ -887,11 +891,9 @@ __global__ void __launch_bounds__(kChainThreads, 1) gdn_bwd_chain_kernel(
         mbar_wait(full + k % kChainStages, uint32_t(k / kChainStages) & 1u, ctrl, &keep_waiting);
     }
     __syncwarp();
-  } else {
-    // ------------------------------------------------------------ epilogue
-    const uint32_t lanes = tmem + (uint32_t(32 * (warp & 3)) << 16);
-    const int m0 = 16 * (warp & 3);           // rows of this warp (d_v for G, tokens for dX)
-    const int gn0 = 64 * (warp >> 2), xn0 = 32 * (warp >> 2);
+  } else if (warp > kChainEpi / 32) {
+    // ------------------------------------------------------------ loader warps
+    const int lt = tid - (kChainEpi + 32);
     auto arrive = [&](uint64_t *b) {
       __syncwarp();
       if (lane == 0) mbar_arrive(b);
@@ -905,11 +907,11 @@ __global__ void __launch_bounds__(kChainThreads, 1) gdn_bwd_chain_kernel(
       const int len = info_of(nch - 1 - k).len;
       uint8_t *stage = sm + kH_STAGE + st * kHStage;
       const float *gam = reinterpret_cast<const float *>(stage + kHs_GAM);
-      for (int e = tid; e < (kC - len) * 8; e += kChainEpi) {
+      for (int e = lt; e < (kC - len) * 8; e += kChainLoad) {
         const int rr = len + (e >> 3), c8 = 8 * (e & 7);
         *reinterpret_cast<uint4 *>(stage + kHs_DO + swz(64, rr, c8)) = make_uint4(0, 0, 0, 0);
       }
-      for (int e = tid; e < 64 * 16; e += kChainEpi) {
+      for (int e = lt; e < 64 * 16; e += kChainLoad) {
         const int rr = e >> 4, c8 = 8 * (e & 15);
         uint4 *p = reinterpret_cast<uint4 *>(stage + kHs_Q + swz(64, rr, c8));
         uint4 x = make_uint4(0, 0, 0, 0);
@@ -928,6 +930,30 @@ __global__ void __launch_bounds__(kChainThreads, 1) gdn_bwd_chain_kernel(
       fence_proxy_async_smem();
       arrive(ready + st);
     };
+    if (nch > 0) land(0);
+    for (int it = 0; it < nch; ++it) {
+      const long long unit = (long long)(c0 + nch - 1 - it) * H + h;
+      // dS_{c+1} (bf16, row-major [d_v][d_k]) for the unit kernel, from the G' tile
+      mbar_wait(gb_full, uint32_t(it) & 1u, ctrl, abort_flag);
+      if (GDN_IN_BOUNDS(ctrl, unit, (long long)max_chunks * H)) {
+        uint4 *dst = reinterpret_cast<uint4 *>(gprime + unit * (kD * kD) + size_t(i0) * kD);
+        for (int e = lt; e < kChainRows * 16; e += kChainLoad) {
+          const int rr = e >> 4, c16 = e & 15;
+          dst[rr * 16 + c16] = *reinterpret_cast<const uint4 *>(sm + kH_G + swz(64, rr, 8 * c16));
+        }
+      }
+      arrive(gb_free);
+      if (it + 1 < nch) land(it + 1);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const uint32_t lanes = tmem + (uint32_t(32 * (warp & 3)) << 16);
+    const int m0 = 16 * (warp & 3);           // rows of this warp (d_v for G, tokens for dX)
+    const int gn0 = 64 * (warp >> 2), xn0 = 32 * (warp >> 2);
+    auto arrive = [&](uint64_t *b) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b);
+    };
     // G slice = d_final_state rows [i0, i0 + 64) (stored [d_k][d_v]) into tensor memory
     {
       const float *src = d_sN ? d_sN + (size_t(n) * H + h) * kD * kD : nullptr;
@@ -943,23 +969,22 @@ __global__ void __launch_bounds__(kChainThreads, 1) gdn_bwd_chain_kernel(
       tmem_st16x256_x8(lanes + kCG + gn0, r);
       tmem_st_wait();
     }
-    if (nch > 0) land(0);
     for (int it = 0; it < nch; ++it) {
-      const int c = nch - 1 - it;
       const uint32_t ph = uint32_t(it) & 1u;
-      const long long unit = (long long)(c0 + c) * H + h;
       const float *gam =
           reinterpret_cast<const float *>(sm + kH_STAGE + (it % kChainStages) * kHStage + kHs_GAM);
       if (it >= 1) {
         mbar_wait(g_full, ph ^ 1u, ctrl, abort_flag);
         tc_fence_after();
       }
+      // the stage landed (gamma_last is read below)
+      mbar_wait(ready + it % kChainStages, uint32_t(it / kChainStages) & 1u, ctrl, abort_flag);
       // E0: G' -> bf16 (operand of the dX product)
       uint32_t r[32];
       tmem_ld16x256_x8(lanes + kCG + gn0, r);
       tmem_ld_wait();
       reg_dep(r);
-      named_bar_sync(1, kChainEpi);   // the previous chunk's G' tile copied out by every warp
+      if (it >= 1) mbar_wait(gb_free, ph ^ 1u, ctrl, abort_flag);   // previous G' copied out
 #pragma unroll
       for (int j = 0; j < 8; ++j)
 #pragma unroll
@@ -989,17 +1014,6 @@ __global__ void __launch_bounds__(kChainThreads, 1) gdn_bwd_chain_kernel(
       fence_proxy_async_smem();
       tc_fence_before();
       arrive(dxs_full);
-      // dS_{c+1} (bf16, row-major [d_v][d_k]) for the unit kernel, from the G'
-      // tile once every epilogue warp has written its part
-      named_bar_sync(1, kChainEpi);
-      if (GDN_IN_BOUNDS(ctrl, unit, (long long)max_chunks * H)) {
-        uint4 *dst = reinterpret_cast<uint4 *>(gprime + unit * (kD * kD) + size_t(i0) * kD);
-        for (int e = tid; e < kChainRows * 16; e += kChainEpi) {
-          const int rr = e >> 4, c16 = e & 15;
-          dst[rr * 16 + c16] = *reinterpret_cast<const uint4 *>(sm + kH_G + swz(64, rr, 8 * c16));
-        }
-      }
-      if (it + 1 < nch) land(it + 1);
     }
     if (nch > 0) {
       mbar_wait(g_full, uint32_t(nch - 1) & 1u, ctrl, abort_flag);
