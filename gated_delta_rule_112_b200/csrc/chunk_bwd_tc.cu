@@ -52,14 +52,15 @@ constexpr int kC = 64, kD = 128;
 constexpr int kThreads = 512, kWarps = kThreads / 32, kUnitThreads = kThreads + 32;
 constexpr float kLog2e = 1.4426950408889634f;
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.wait_group 0;" ::: "memory");
+// One contiguous copy global -> shared (16-byte aligned, size a multiple of
+// 16) that completes `bytes` of the mbarrier's transaction count; no cluster
+// broadcast.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes,
+                                          uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -94,7 +95,7 @@ constexpr uint32_t kV_Q = 0;                  // [64][128]: two 8 KB panels
 constexpr uint32_t kV_K = kV_Q + 16384;
 constexpr uint32_t kV_V = kV_K + 16384;
 constexpr uint32_t kV_DO = kV_V + 16384;
-constexpr uint32_t kV_S = kV_DO + 16384;      // [128][128] (S_c, rows d_v): two 16 KB panels
+constexpr uint32_t kV_S = kV_DO + 16384;      // S_c [128 d_v][128 d_k] in the scan's piece order, unswizzled
 constexpr uint32_t kV_GP = kV_S + 32768;      // G' [d_v][d_k]
 constexpr uint32_t kV_TB = kV_GP + 32768;     // [64][64]: one 8 KB panel
 constexpr uint32_t kV_P = kV_TB + 8192;       // P; then dP .* E
@@ -121,13 +122,36 @@ __device__ __forceinline__ uint32_t swz(int rows, int r, int c) {
 
 // One operand of a product: tile base, its rows and whether it is read
 // MN-major (stored [K rows][M or N]) or K-major (stored [M or N rows][K]).
+// piece: a 128 x 128 tile stored unswizzled in 16-byte pieces, element (i, j)
+// at byte (j / 8) * 2048 + i * 16 + (j % 8) * 2 (the state scan's store order);
+// its rows i are then N (K-major) or K (MN-major).
 struct Opnd {
   uint32_t base;
   int rows;
   bool mn;
+  bool piece = false;
 };
+// Descriptor of an unswizzled operand (layout type 0): 8 x 16-byte core
+// matrices, lbo / sbo their strides along K / along M or N for K-major
+// operands and along K / along M or N, swapped, for MN-major ones.
+__device__ __forceinline__ uint64_t make_sdesc_plain(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= uint64_t((saddr >> 4) & 0x3FFFu);
+  d |= uint64_t((lbo >> 4) & 0x3FFFu) << 16;
+  d |= uint64_t((sbo >> 4) & 0x3FFFu) << 32;
+  d |= uint64_t(1) << 46;              // descriptor version (sm_100); layout 0: no swizzle
+  return d;
+}
 // Shared-memory descriptor of k-step kk (16 elements of K).
 __device__ __forceinline__ uint64_t opnd_desc(const Opnd &o, int kk) {
+  if (o.piece) {
+    // K-major (rows i = N, K = j): the two core matrices of a k-step are two
+    // pieces (2048 B apart), 8-row groups 128 B apart. MN-major (K = i, N = j):
+    // a k-step is 16 rows (256 B); 8-column groups (pieces) 2048 B apart,
+    // 8-row groups of K 128 B apart.
+    if (o.mn) return make_sdesc_plain(o.base + uint32_t(kk) * 256u, 128, 2048);
+    return make_sdesc_plain(o.base + uint32_t(kk) * 4096u, 2048, 128);
+  }
   if (o.mn) return make_sdesc(o.base + uint32_t(kk) * 2048u, uint32_t(o.rows) * 128u, 1024);
   return make_sdesc(o.base + uint32_t(kk >> 2) * uint32_t(o.rows) * 128u + uint32_t(kk & 3) * 32u,
                     16, 1024);
@@ -249,8 +273,8 @@ __device__ __forceinline__ void swz_st(uint8_t *t, int rows, int r, int c, float
 // tokens q, k, v, dO [rows, H, 128] (box 64 x 1 x 64, two per tile); -W, T
 // diag(beta), P [units * 64][*] and (D K)^T [units * 128][64] (box 64 x rows);
 // G' [units * 128][128] (box 64 x 128). S_c, stored by the scan in 16-byte
-// pieces (piece p of row i at p * 128 + i), is gathered by cp.async from all
-// threads into the same swizzled row-major layout.
+// pieces (piece p of row i at p * 128 + i), arrives by one 32 KB bulk copy in
+// that order and is read by the MMAs through unswizzled descriptors.
 __global__ void __launch_bounds__(kUnitThreads, 1) gdn_bwd_unit_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -297,7 +321,7 @@ __global__ void __launch_bounds__(kUnitThreads, 1) gdn_bwd_unit_kernel(
   const Opnd Kk{sb + kV_K, 64, false}, Km{sb + kV_K, 64, true};
   const Opnd Vm{sb + kV_V, 64, true};
   const Opnd DOk{sb + kV_DO, 64, false}, DOm{sb + kV_DO, 64, true};
-  const Opnd Sk{sb + kV_S, 128, false}, Sm{sb + kV_S, 128, true};
+  const Opnd Sk{sb + kV_S, 128, false, true}, Sm{sb + kV_S, 128, true, true};
   const Opnd GPk{sb + kV_GP, 128, false}, GPm{sb + kV_GP, 128, true};
   const Opnd TBk{sb + kV_TB, 64, false}, TBm{sb + kV_TB, 64, true};
   const Opnd Pk{sb + kV_P, 64, false}, Pm{sb + kV_P, 64, true};
@@ -339,17 +363,9 @@ __global__ void __launch_bounds__(kUnitThreads, 1) gdn_bwd_unit_kernel(
     const int c = u / H;
     return GDN_IN_BOUNDS(ctrl, c, max_chunks) ? table[c] : ChunkInfo{0, 0, 0, 0};
   };
-  // group A (Q, K, P) and group B (V, dO, G', T diag(beta), -W, (D K)^T) of
-  // unit u, issued by thread 0; each load completes one phase of its barrier.
-  // S_c of unit u: every thread's share, one cp.async group.
-  auto load_sc = [&](int u) {
-    const bf16 *sc = s_chunks + (long long)u * (kD * kD);
-    for (int e = tid; e < 128 * 16; e += kThreads) {
-      const int p = e >> 7, i = e & 127;
-      cp_async16(sb + kV_S + swz(128, i, 8 * p), sc + (p * 128 + i) * 8);
-    }
-    cp_async_commit();
-  };
+  // group A (Q, K, P) and group B (V, dO, S_c, G', T diag(beta), -W, (D K)^T)
+  // of unit u, issued by the issuer thread; each load completes one phase of
+  // its barrier.
   int na = 0, nb = 0;
   auto load_a = [&](int u) {
     const ChunkInfo c = info(u);
@@ -365,7 +381,8 @@ __global__ void __launch_bounds__(kUnitThreads, 1) gdn_bwd_unit_kernel(
   auto load_b = [&](int u) {
     const ChunkInfo c = info(u);
     const int hu = u % H;
-    mbar_arrive_expect_tx(ld_b, 4 * 16384 + 32768 + 8192);
+    mbar_arrive_expect_tx(ld_b, 4 * 16384 + 2 * 32768 + 8192);
+    bulk_load(sm + kV_S, s_chunks + (long long)u * (kD * kD), 32768, ld_b);
     tma_load_3d(sm + kV_V, &tm_v, ld_b, 0, hu, c.row0);
     tma_load_3d(sm + kV_V + 8192, &tm_v, ld_b, 64, hu, c.row0);
     tma_load_3d(sm + kV_DO, &tm_do, ld_b, 0, hu, c.row0);
@@ -389,7 +406,6 @@ __global__ void __launch_bounds__(kUnitThreads, 1) gdn_bwd_unit_kernel(
     // B (S_c, G', dO, V, -W, (D K)^T, T diag(beta)) of this unit was issued
     // during the previous one, as soon as its phase 5 had read them; group A
     // (Q, K, P) here.
-    if (first && epi) load_sc(unit);
     if (issuer) {
       if (first) load_b(unit);
       load_a(unit);
@@ -428,7 +444,6 @@ __global__ void __launch_bounds__(kUnitThreads, 1) gdn_bwd_unit_kernel(
       const uint32_t ph = uint32_t(it_count) & 1u;
       mbar_wait(ld_a, ph, ctrl, abort_flag);
       mbar_wait(ld_b, ph, ctrl, abort_flag);
-      cp_async_wait_all();   // S_c (visible to all after the phase-1 barrier)
       for (int e = tid; epi && e < (kC - len) * 16; e += kThreads) {
         const int r = len + (e >> 4), c8 = 8 * (e & 15);
         const uint32_t o = swz(64, r, c8);
@@ -448,11 +463,12 @@ __global__ void __launch_bounds__(kUnitThreads, 1) gdn_bwd_unit_kernel(
       mma_product(tmem, kC3, Kk, Kk, 64, 8, false);         // K K^T
     }, true);
     if (epi) {
-      // <G', S> for the last token's dGamma
-      // (both tiles share one layout: a plain walk over their bytes)
+      // <G', S> for the last token's dGamma: S_c's piece e = (p, i) holds
+      // row i, columns 8 p .. 8 p + 7, found in G' (swizzled rows) by swz
       float gs_dot = 0.f;
       for (int e = tid; e < 128 * 16; e += kThreads) {
-        const uint4 a = *reinterpret_cast<const uint4 *>(sm + kV_GP + 16 * e);
+        const int p = e >> 7, i = e & 127;
+        const uint4 a = *reinterpret_cast<const uint4 *>(sm + kV_GP + swz(128, i, 8 * p));
         const uint4 b = *reinterpret_cast<const uint4 *>(sm + kV_S + 16 * e);
         const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
@@ -621,9 +637,6 @@ __global__ void __launch_bounds__(kUnitThreads, 1) gdn_bwd_unit_kernel(
       });
       add_rows(dGam, part, m0, lane);
       wait_group();
-      // S_c, G', dO, V, -W, (D K)^T and T diag(beta) are read for the last
-      // time by phase 5: the next unit's copies land during the rest of this one
-      if (unit + int(gridDim.x) < nunits) load_sc(unit + int(gridDim.x));
       {
         uint32_t r1[16], r2[16];
         tmem_ld16x256_x4(lanes + kC2 + n0, r1);
@@ -718,7 +731,6 @@ __global__ void __launch_bounds__(kUnitThreads, 1) gdn_bwd_unit_kernel(
     if (na > 0) mbar_wait(ld_a, uint32_t(na - 1) & 1u, ctrl, &keep_waiting);
     if (nb > 0) mbar_wait(ld_b, uint32_t(nb - 1) & 1u, ctrl, &keep_waiting);
   }
-  cp_async_wait_all();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
