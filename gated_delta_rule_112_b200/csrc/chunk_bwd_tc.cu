@@ -402,12 +402,11 @@ __global__ void __launch_bounds__(kUnitThreads, 1) gdn_bwd_unit_kernel(
     const ChunkInfo ci =
         GDN_IN_BOUNDS(ctrl, chunk, max_chunks) ? table[chunk] : ChunkInfo{0, 0, 0, 0};
     const int len = ci.len;
-    // ---- loads (rows of q, k, v, dO past the sequence end read as zero). Group
-    // B (S_c, G', dO, V, -W, (D K)^T, T diag(beta)) of this unit was issued
-    // during the previous one, as soon as its phase 5 had read them; group A
-    // (Q, K, P) here.
-    if (issuer) {
-      if (first) load_b(unit);
+    // ---- loads. Both groups of this unit were issued during the previous
+    // one, each as soon as its last reader there was done (group B after phase
+    // 5's products, group A (Q, K, P) after phase 6's); the first unit's here.
+    if (issuer && first) {
+      load_b(unit);
       load_a(unit);
     }
     if (warp == 0) {
@@ -669,6 +668,13 @@ __global__ void __launch_bounds__(kUnitThreads, 1) gdn_bwd_unit_kernel(
       mma_product(tmem, kC0, Lk, Km, 128, 4, true);         //   + R K
       mma_product(tmem, kC0, Lm, Km, 128, 4, true);         //   + R^T K
     }, none, false);
+    if (issuer && unit + int(gridDim.x) < nunits) {
+      // phase 6's group (the last reader of Q, K and P; the epilogues read
+      // them before its issue) done: the next unit's group A loads now
+      const int gidx = next_commit - 1;
+      mbar_wait(bars + (gidx & 1), uint32_t(gidx >> 1) & 1u, ctrl, abort_flag);
+      load_a(unit + int(gridDim.x));
+    }
     if (epi) {
       wait_group();
       float a[4][4];
@@ -720,7 +726,6 @@ __global__ void __launch_bounds__(kUnitThreads, 1) gdn_bwd_unit_kernel(
         }
       }
     }
-    fence_proxy_async_smem();   // generic writes to Q, K, P before their next TMA
     __syncthreads();   // shared memory free for the next unit
     first = false;
     ++it_count;
