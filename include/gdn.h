@@ -360,7 +360,9 @@ int gdn_chunk_fwd_save(const void *q, const void *k, const void *v, const float 
  * initial_state, cu_seqlens and sizes on this stream: the forward replay is
  * skipped and only the reverse chain and the per-unit kernel run. The
  * workspace's saved part is read, not changed (the call may be repeated for
- * another d_o). Tensor-core path only: GDN_ERR_UNSUPPORTED otherwise. The
+ * another d_o); its scratch part takes each chunk's dS_{c+1}, so two calls
+ * on one workspace must not overlap on the GPU. Tensor-core path only:
+ * GDN_ERR_UNSUPPORTED otherwise. The
  * kernels trust the saved chunk table: a workspace that gdn_chunk_fwd_save
  * did not fill for these inputs is undefined behaviour.
  */
