@@ -71,7 +71,9 @@ def parse_args():
     p.add_argument("--no-extra-workloads", action="store_true",
                    help="skip the long64k and varlen64 sub-measurements")
     p.add_argument("--bwd", action="store_true",
-                   help="also time the backward pass (gdn_chunk_bwd) on the workload")
+                   help="time the backward pass (the default; kept for older command lines)")
+    p.add_argument("--no-bwd", action="store_true",
+                   help="skip the backward-pass and training-step sub-measurements")
     p.add_argument("--workload", default=WORKLOAD,
                    help="chunked-forward workload (inputs.WORKLOADS); the default is the "
                         "headline configuration, the others are for extra measurements")
@@ -437,7 +439,7 @@ def main():
 
     # --------------------------------------------------------------- backward pass
     backward = None
-    if args.bwd and not kda:
+    if not args.no_bwd and not kda:
         del ws
         torch.cuda.empty_cache()
         gen = torch.Generator("cpu").manual_seed(1000 + rank)
